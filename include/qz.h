@@ -1,0 +1,199 @@
+/*
+ * qz.h -- C ABI of the grouped block-scaled quantization library (libqz.so)
+ * for NVIDIA B200 (sm_100a).
+ *
+ * The library quantizes groups of bf16 matrices ("experts") to
+ *   MXFP8: e4m3 payload, one E8M0 scale byte per 32 consecutive row elements;
+ *   NVFP4: packed e2m1 payload, one E4M3 scale byte per 16 consecutive row
+ *          elements, plus an FP32 second-level amax per tensor or per row;
+ * and writes each expert's scale factors (SF) in the linear row-major layout
+ * or the swizzled 128x4 layout, each expert into its own independently padded
+ * region.  A fused residual-add + RMSNorm entry point writes the bf16 norm and
+ * its quantized form from one read.
+ *
+ * Conventions that hold for every entry point:
+ *  - Pointers whose name starts with d_, and every pointer inside a table, are
+ *    DEVICE pointers.  The caller owns every buffer; the library allocates
+ *    nothing and keeps no state besides a per-device cache of launch limits.
+ *  - `stream` is a cudaStream_t (NULL: the legacy default stream).  Every call
+ *    is asynchronous on that stream; inputs must be ready on it.  No call
+ *    synchronizes.
+ *  - Arguments the host can check are checked before anything is launched; on
+ *    error nothing is written and the status says why.  Table entries live in
+ *    device memory, so they are checked by the kernel: an invalid entry is
+ *    skipped (none of its bytes are written) and, when opts->d_err is given,
+ *    the reason bits below are OR-ed into *opts->d_err.
+ *  - Only the bytes named by the table (payload rows, the expert's own SF
+ *    region, its amax slot(s)) are written: re-quantizing one expert is a call
+ *    with a one-entry table and touches no other expert's storage.
+ *  - Element encodings: RNE with saturation (satfinite); the sign of a zero or
+ *    of a value that rounds to zero is kept; an all-zero block gets scale byte
+ *    0x00.  Non-finite inputs are outside the contract.
+ *
+ * Citations (web pages, by title and section):
+ *  [MX]   NVIDIA-NeMo/RL PR #3804 "perf(refit): batch MXFP8 expert
+ *         prequantization" -- Summary, Why, Self-review.
+ *  [FOLD] NVIDIA/Model-Optimizer PR #2750 "Fold fused experts' quantizers into
+ *         their weights shard-locally" -- weight_scale_2 review; zero-block notes.
+ *  [LSF]  NVIDIA/TensorRT-LLM PR #17452 "NVFP4 linear-SF AllReduce epilogue" --
+ *         commits 1-3.
+ *  [SPL]  NVIDIA/TransformerEngine PR #3800 (row-scaled NVFP4 split
+ *         quantization) -- Description, Changes.
+ *  [CAR]  NVIDIA/TensorRT-LLM PR #17453 "MXFP8 carrier and quantize folds" --
+ *         commits 2, 3, 5, 6.
+ */
+#ifndef QZ_H
+#define QZ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum qz_status {
+    QZ_OK = 0,
+    QZ_ERR_INVALID_ARG = 1, /* bad count, null pointer, unknown enum, bad size */
+    QZ_ERR_ALIGNMENT = 2,   /* a host-visible pointer or stride is misaligned */
+    QZ_ERR_UNSUPPORTED = 3, /* a shape/format/layout combination the kernels do not cover */
+    QZ_ERR_CUDA = 4         /* the CUDA runtime reported an error at launch */
+} qz_status;
+
+typedef enum qz_sf_layout {
+    QZ_SF_LINEAR = 0,        /* byte (row, k) at row * kv + k              ([LSF] commit 1) */
+    QZ_SF_SWIZZLED_128x4 = 1 /* 128-row x 4-column tiles of 512 bytes, row-block-major;
+                                inside a tile byte ((row%32)*4 + (row%128)/32)*4 + k%4;
+                                rows padded to 128 and k to 4 with 0x00 ([CAR] commits 3, 6;
+                                cuBLAS "1D Block Scaling Factors Layout") */
+} qz_sf_layout;
+
+typedef enum qz_format {
+    QZ_FMT_MXFP8 = 0,
+    QZ_FMT_NVFP4 = 1
+} qz_format;
+
+typedef enum qz_nvfp4_scale_mode {
+    QZ_NVFP4_PER_TENSOR_GIVEN = 0,   /* amax[0] is an input (e.g. a calibrated value) */
+    QZ_NVFP4_PER_TENSOR_COMPUTE = 1, /* amax[0] = max |x| over the expert, written by the call */
+    QZ_NVFP4_PER_ROW = 2             /* amax[r] = max |x| over row r, written by the call ([SPL]) */
+} qz_nvfp4_scale_mode;
+
+/* Reason bits OR-ed into *opts->d_err for table entries a kernel skipped. */
+#define QZ_DERR_SHAPE 0x1u     /* rows < 0, cols <= 0, cols not a multiple of the block, ld < cols */
+#define QZ_DERR_NULL 0x2u      /* x, q, sf (or amax for NVFP4) null on a non-empty entry */
+#define QZ_DERR_ALIGN 0x4u     /* x not 16-byte aligned or ld not a multiple of 8; q not
+                                  8-byte (MXFP8) / 4-byte (NVFP4) aligned; sf not 16-byte
+                                  aligned (swizzled); amax not 4-byte aligned */
+#define QZ_DERR_TOO_LARGE 0x8u /* the call's total tile or row count exceeds 2^31 - 1 */
+
+/* Largest table a grouped call accepts (the kernels keep the table's prefix
+ * sums in shared memory). */
+#define QZ_MAX_EXPERTS 4096
+
+/* Largest hidden size of qz_rmsnorm_quantize (one row is held in registers). */
+#define QZ_MAX_HIDDEN 16384
+
+/* One table entry per expert ([MX] Summary: many same-shape experts per call;
+ * [SPL] Description: one concatenated activation split unevenly by expert).
+ * The table itself and every pointer in it are device memory.  56 bytes. */
+typedef struct qz_expert {
+    const void *x; /* bf16 [rows, cols], row stride ld elements.  For a split
+                      activation: base + row_offset * ld. */
+    int64_t rows;  /* may be 0 (an empty split): nothing is read or written */
+    int64_t cols;  /* quantization axis; multiple of 32 (MXFP8) or 16 (NVFP4) */
+    int64_t ld;    /* row stride of x in elements, >= cols, multiple of 8 */
+    void *q;       /* payload, row-major and dense: MXFP8 e4m3 [rows, cols];
+                      NVFP4 e2m1 [rows, cols/2], element 2j in the low nibble
+                      of byte j and element 2j+1 in the high nibble */
+    uint8_t *sf;   /* this expert's SF region of qz_sf_bytes(rows, cols, fmt, layout) bytes */
+    float *amax;   /* NVFP4: per-tensor amax (one float: input in GIVEN mode,
+                      output in COMPUTE mode) or per-row amax [rows] (output);
+                      MXFP8: unused (may be NULL) */
+} qz_expert;
+
+/* One linear -> swizzled conversion ([MX] Summary: the receiver-side MXFP8
+ * layout conversion).  Device pointers. */
+typedef struct qz_sf_pair {
+    const uint8_t *src; /* linear SF [rows, kv], row-major, dense */
+    uint8_t *dst;       /* swizzled region of pad(rows,128) * pad(kv,4) bytes, 16-byte aligned */
+    int64_t rows;       /* >= 0 */
+    int64_t kv;         /* scale columns, >= 1 */
+} qz_sf_pair;
+
+/* Optional launch controls; pass NULL for the defaults. */
+typedef struct qz_launch_opts {
+    unsigned int *d_err; /* device word; kernels OR QZ_DERR_* bits into it (never clear it) */
+    int max_ctas;        /* 0: one wave of resident CTAs on every SM; > 0: cap on the grid.
+                            The results do not depend on it. */
+} qz_launch_opts;
+
+/* Bytes of one expert's SF region: rows * (cols/block) for the linear layout,
+ * pad(rows,128) * pad(cols/block,4) for the swizzled one, 0 when rows == 0.
+ * fmt selects the block (32 for MXFP8, 16 for NVFP4).  Returns 0 for
+ * arguments that describe no valid region (negative sizes, cols not a
+ * multiple of the block, unknown enums). */
+size_t qz_sf_bytes(int64_t rows, int64_t cols, int fmt, int layout);
+
+/* MXFP8 quantization of every expert in d_table, in one persistent launch
+ * ([MX] Summary, Why, Self-review; [CAR] commits 2, 3).  Per 32-element block
+ * B of a row: e = the smallest integer with max|B| <= 448 * 2^e, clamped below
+ * at -127 (zero blocks: -127); scale byte = e + 127; payload = e4m3(x * 2^-e).
+ * Errors: QZ_ERR_INVALID_ARG for n_experts < 0 or > QZ_MAX_EXPERTS, a NULL
+ * table with n_experts > 0, or an unknown layout; QZ_ERR_CUDA if the launch
+ * fails.  n_experts == 0 launches nothing and returns QZ_OK. */
+qz_status qz_quantize_grouped_mxfp8(const qz_expert *d_table, int n_experts, int layout,
+                                    void *stream, const qz_launch_opts *opts);
+
+/* NVFP4 quantization of every expert in d_table ([FOLD] weight_scale_2 review
+ * and zero-block notes; [SPL] Description, Changes; [LSF] commit 3).
+ * With A the tensor (or row) amax: g = RN32(A / 2688) is the FP32 decode
+ * scale, S = RN32(1 / g) (0 if g == 0) the encode scale; per 16-element block
+ * with amax b: scale s = e4m3(RN32(RN32(b / 6) * S)) (0 if b == 0); payload
+ * q = e2m1(RN32(x * r)), r = FTZ(RN32(S / s)) (0 if s == 0).
+ * PER_TENSOR_COMPUTE runs an amax pass before the quantize pass (three
+ * launches in stream order); PER_ROW reads each row once.
+ * Errors as for qz_quantize_grouped_mxfp8, plus QZ_ERR_INVALID_ARG for an
+ * unknown mode. */
+qz_status qz_quantize_grouped_nvfp4(const qz_expert *d_table, int n_experts, int mode, int layout,
+                                    void *stream, const qz_launch_opts *opts);
+
+/* Fused residual add + RMSNorm + quantize of T rows of H elements ([LSF]
+ * commits 2, 3; [CAR] commit 6):
+ *   h = bf16(x + residual)            -> d_residual_out (nullable)
+ *   y = bf16(h / sqrt(mean(h^2) + eps) * gamma)   -> d_norm_out
+ *   q, sf = quantize(y) exactly as the grouped entry points would quantize
+ *           d_norm_out (MXFP8, or NVFP4 with the per-tensor amax *d_global_amax)
+ * All of x, residual, norm_out, residual_out are bf16 [T, H] row-major, gamma
+ * bf16 [H].  The swizzled layout's padded rows (T .. pad(T,128)-1) are written
+ * as 0x00 by the kernel itself.
+ * Errors: QZ_ERR_INVALID_ARG for T < 0, H <= 0, H > QZ_MAX_HIDDEN, H not a
+ * multiple of the block (32 / 16), null required pointers, unknown fmt or
+ * layout, NVFP4 without d_global_amax; QZ_ERR_UNSUPPORTED for the swizzled
+ * layout with H/block not a multiple of 4 (the padded scale columns would be
+ * unreachable, [CAR] commit 6); QZ_ERR_ALIGNMENT for bf16 pointers not 16-byte
+ * aligned, q not 8-byte aligned, or sf not 16-byte aligned (swizzled) / 4-byte
+ * aligned (linear); QZ_ERR_CUDA on launch failure.  T == 0 launches nothing. */
+qz_status qz_rmsnorm_quantize(const void *d_x, const void *d_residual, const void *d_gamma, float eps,
+                              int64_t T, int64_t H, void *d_norm_out, void *d_residual_out,
+                              int fmt, void *d_q, uint8_t *d_sf, int layout,
+                              const float *d_global_amax, void *stream);
+
+/* Linear -> swizzled 128x4 conversion of n SF matrices in one launch, padding
+ * written as 0x00 ([MX] Summary; [CAR] commit 5: swizzled and linear agree).
+ * Errors: QZ_ERR_INVALID_ARG for n < 0, n > QZ_MAX_EXPERTS or a NULL table
+ * with n > 0; entries with rows < 0, kv < 1, null pointers or a misaligned
+ * dst are skipped and reported through opts->d_err. */
+qz_status qz_swizzle_scales(const qz_sf_pair *d_table, int n, void *stream, const qz_launch_opts *opts);
+
+/* A static, human-readable name for a status code. */
+const char *qz_status_string(qz_status status);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int qz_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QZ_H */

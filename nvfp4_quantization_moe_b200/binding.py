@@ -1,0 +1,261 @@
+"""ctypes binding of libqz.so -- argument marshalling only.
+
+Every byte of quantization work happens in the CUDA kernels behind the C ABI
+(include/qz.h).  This module packs expert tables into device memory, passes
+pointers, sizes and the current CUDA stream, and turns status codes into
+exceptions.  There is no fallback: if libqz.so is missing or a call fails, it
+raises.  PyTorch supplies device memory and streams.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+from dataclasses import dataclass
+from typing import Iterable, Optional, Sequence
+
+import numpy as np
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libqz.so")
+
+# enums of include/qz.h
+QZ_OK, QZ_ERR_INVALID_ARG, QZ_ERR_ALIGNMENT, QZ_ERR_UNSUPPORTED, QZ_ERR_CUDA = range(5)
+SF_LINEAR, SF_SWIZZLED = 0, 1
+FMT_MXFP8, FMT_NVFP4 = 0, 1
+NVFP4_PER_TENSOR_GIVEN, NVFP4_PER_TENSOR_COMPUTE, NVFP4_PER_ROW = 0, 1, 2
+DERR_SHAPE, DERR_NULL, DERR_ALIGN, DERR_TOO_LARGE = 0x1, 0x2, 0x4, 0x8
+MAX_EXPERTS = 4096
+MAX_HIDDEN = 16384
+
+EXPORTED = (
+    "qz_sf_bytes",
+    "qz_quantize_grouped_mxfp8",
+    "qz_quantize_grouped_nvfp4",
+    "qz_rmsnorm_quantize",
+    "qz_swizzle_scales",
+    "qz_status_string",
+    "qz_version",
+)
+
+
+class QzError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)}")
+
+
+class _Expert(ctypes.Structure):
+    _fields_ = [("x", ctypes.c_void_p), ("rows", ctypes.c_int64), ("cols", ctypes.c_int64),
+                ("ld", ctypes.c_int64), ("q", ctypes.c_void_p), ("sf", ctypes.c_void_p),
+                ("amax", ctypes.c_void_p)]
+
+
+class _SfPair(ctypes.Structure):
+    _fields_ = [("src", ctypes.c_void_p), ("dst", ctypes.c_void_p), ("rows", ctypes.c_int64),
+                ("kv", ctypes.c_int64)]
+
+
+class _Opts(ctypes.Structure):
+    _fields_ = [("d_err", ctypes.c_void_p), ("max_ctas", ctypes.c_int)]
+
+
+assert ctypes.sizeof(_Expert) == 56 and ctypes.sizeof(_SfPair) == 32
+
+_lock = threading.Lock()
+_lib = None
+
+
+def load(path: str = LIB_PATH):
+    """Load libqz.so (raises if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        if not os.path.exists(path):
+            raise RuntimeError(f"{path} is missing: build it with "
+                               "`python -m nvfp4_quantization_moe_b200.build` (nvcc, sm_100a)")
+        lib = ctypes.CDLL(path)
+        P, I, i64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64
+        lib.qz_sf_bytes.restype = ctypes.c_size_t
+        lib.qz_sf_bytes.argtypes = [i64, i64, I, I]
+        lib.qz_quantize_grouped_mxfp8.restype = I
+        lib.qz_quantize_grouped_mxfp8.argtypes = [P, I, I, P, P]
+        lib.qz_quantize_grouped_nvfp4.restype = I
+        lib.qz_quantize_grouped_nvfp4.argtypes = [P, I, I, I, P, P]
+        lib.qz_rmsnorm_quantize.restype = I
+        lib.qz_rmsnorm_quantize.argtypes = [P, P, P, ctypes.c_float, i64, i64, P, P, I, P, P, I, P, P]
+        lib.qz_swizzle_scales.restype = I
+        lib.qz_swizzle_scales.argtypes = [P, I, P, P]
+        lib.qz_status_string.restype = ctypes.c_char_p
+        lib.qz_status_string.argtypes = [I]
+        lib.qz_version.restype = I
+        lib.qz_version.argtypes = []
+        _lib = lib
+        return lib
+
+
+def status_string(status: int) -> str:
+    return load().qz_status_string(int(status)).decode()
+
+
+def _check(status: int, where: str):
+    if status != QZ_OK:
+        raise QzError(status, where)
+
+
+def _stream_ptr(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(int(stream.cuda_stream) if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _opts(err: Optional[torch.Tensor], max_ctas: int):
+    if err is None and not max_ctas:
+        return None
+    if err is not None:
+        assert err.dtype in (torch.int32, torch.uint32) and err.is_cuda and err.numel() >= 1
+    return ctypes.byref(_Opts(ctypes.c_void_p(err.data_ptr() if err is not None else 0), int(max_ctas)))
+
+
+def _ptr(t: Optional[torch.Tensor]) -> int:
+    return 0 if t is None else int(t.data_ptr())
+
+
+def sf_bytes(rows: int, cols: int, fmt: int, layout: int) -> int:
+    return int(load().qz_sf_bytes(int(rows), int(cols), int(fmt), int(layout)))
+
+
+# ---------------------------------------------------------------------------
+# device tables
+# ---------------------------------------------------------------------------
+
+@dataclass
+class Entry:
+    """One expert: a bf16 [rows, cols] view (row stride in elements may exceed
+    cols), its payload, SF region and (NVFP4) amax storage."""
+    x: torch.Tensor
+    q: torch.Tensor
+    sf: torch.Tensor
+    amax: Optional[torch.Tensor] = None
+
+
+class ExpertTable:
+    """A device-resident array of qz_expert entries.  Keeps references to the
+    tensors it points into, so they outlive the table."""
+
+    def __init__(self, entries: Sequence[Entry], device=None):
+        self.entries = list(entries)
+        n = len(self.entries)
+        arr = (_Expert * max(n, 1))()
+        for i, e in enumerate(self.entries):
+            x = e.x
+            assert x.dtype == torch.bfloat16 and x.dim() == 2
+            rows, cols = x.shape
+            ld = x.stride(0) if rows > 1 else max(cols, x.stride(0))
+            assert rows == 0 or x.stride(1) == 1, "rows must be contiguous"
+            arr[i] = _Expert(x.data_ptr() if rows else 0, rows, cols, ld, _ptr(e.q) if rows else 0,
+                             _ptr(e.sf) if rows else 0, _ptr(e.amax))
+        host = torch.frombuffer(bytearray(bytes(arr)), dtype=torch.uint8)
+        dev = device if device is not None else (self.entries[0].x.device if n else torch.device("cuda"))
+        self.dev = host.to(dev)
+        self.n = n
+
+    @property
+    def ptr(self) -> int:
+        return int(self.dev.data_ptr()) if self.n else 0
+
+    @classmethod
+    def from_raw(cls, raw: Iterable[tuple], device) -> "ExpertTable":
+        """Entries from raw (x_ptr, rows, cols, ld, q_ptr, sf_ptr, amax_ptr) tuples
+        (tests use this to build deliberately invalid entries)."""
+        self = cls.__new__(cls)
+        raw = list(raw)
+        arr = (_Expert * max(len(raw), 1))(*[_Expert(*r) for r in raw])
+        self.entries = []
+        self.n = len(raw)
+        self.dev = torch.frombuffer(bytearray(bytes(arr)), dtype=torch.uint8).to(device)
+        return self
+
+
+class SfPairTable:
+    def __init__(self, pairs: Sequence[tuple], device):
+        """pairs: (src linear uint8 tensor, dst swizzled uint8 tensor, rows, kv)."""
+        self.pairs = list(pairs)
+        arr = (_SfPair * max(len(self.pairs), 1))()
+        for i, (src, dst, rows, kv) in enumerate(self.pairs):
+            arr[i] = _SfPair(_ptr(src), _ptr(dst), int(rows), int(kv))
+        self.dev = torch.frombuffer(bytearray(bytes(arr)), dtype=torch.uint8).to(device)
+        self.n = len(self.pairs)
+
+
+# ---------------------------------------------------------------------------
+# entry points
+# ---------------------------------------------------------------------------
+
+def quantize_grouped_mxfp8(table: ExpertTable, layout: int, stream=None, err=None, max_ctas: int = 0):
+    _check(load().qz_quantize_grouped_mxfp8(ctypes.c_void_p(table.ptr), table.n, int(layout),
+                                            _stream_ptr(stream), _opts(err, max_ctas)),
+           "qz_quantize_grouped_mxfp8")
+
+
+def quantize_grouped_nvfp4(table: ExpertTable, mode: int, layout: int, stream=None, err=None, max_ctas: int = 0):
+    _check(load().qz_quantize_grouped_nvfp4(ctypes.c_void_p(table.ptr), table.n, int(mode), int(layout),
+                                            _stream_ptr(stream), _opts(err, max_ctas)),
+           "qz_quantize_grouped_nvfp4")
+
+
+def rmsnorm_quantize(x, residual, gamma, eps: float, norm_out, residual_out, fmt: int, q, sf, layout: int,
+                     global_amax=None, stream=None):
+    T, H = x.shape
+    _check(load().qz_rmsnorm_quantize(ctypes.c_void_p(_ptr(x)), ctypes.c_void_p(_ptr(residual)),
+                                      ctypes.c_void_p(_ptr(gamma)), ctypes.c_float(eps), int(T), int(H),
+                                      ctypes.c_void_p(_ptr(norm_out)), ctypes.c_void_p(_ptr(residual_out)),
+                                      int(fmt), ctypes.c_void_p(_ptr(q)), ctypes.c_void_p(_ptr(sf)), int(layout),
+                                      ctypes.c_void_p(_ptr(global_amax)), _stream_ptr(stream)),
+           "qz_rmsnorm_quantize")
+
+
+def swizzle_scales(table: SfPairTable, stream=None, err=None, max_ctas: int = 0):
+    _check(load().qz_swizzle_scales(ctypes.c_void_p(int(table.dev.data_ptr()) if table.n else 0), table.n,
+                                    _stream_ptr(stream), _opts(err, max_ctas)),
+           "qz_swizzle_scales")
+
+
+# ---------------------------------------------------------------------------
+# conveniences that allocate outputs with torch and call the entry points
+# ---------------------------------------------------------------------------
+
+def alloc_outputs(xs: Sequence[torch.Tensor], fmt: int, layout: int, mode: int = NVFP4_PER_ROW):
+    """Payload, SF and amax buffers for a list of bf16 [rows, cols] experts."""
+    entries = []
+    for x in xs:
+        rows, cols = x.shape
+        qcols = cols if fmt == FMT_MXFP8 else cols // 2
+        q = torch.empty((rows, qcols), dtype=torch.uint8, device=x.device)
+        sf = torch.empty(max(sf_bytes(rows, cols, fmt, layout), 16), dtype=torch.uint8, device=x.device)
+        amax = None
+        if fmt == FMT_NVFP4:
+            amax = torch.zeros(max(rows, 1) if mode == NVFP4_PER_ROW else 1, dtype=torch.float32, device=x.device)
+        entries.append(Entry(x, q, sf, amax))
+    return entries
+
+
+def quantize_experts(xs: Sequence[torch.Tensor], fmt: int, layout: int, mode: int = NVFP4_PER_ROW,
+                     amax_in: Optional[Sequence[float]] = None, stream=None):
+    """Quantize a list of bf16 experts in one launch; returns the entries with
+    q, sf (trimmed to the region size) and amax filled."""
+    entries = alloc_outputs(xs, fmt, layout, mode)
+    if fmt == FMT_NVFP4 and mode == NVFP4_PER_TENSOR_GIVEN:
+        for e, a in zip(entries, amax_in):
+            e.amax.fill_(float(a))
+    table = ExpertTable(entries)
+    if fmt == FMT_MXFP8:
+        quantize_grouped_mxfp8(table, layout, stream)
+    else:
+        quantize_grouped_nvfp4(table, mode, layout, stream)
+    for e in entries:
+        rows, cols = e.x.shape
+        e.sf = e.sf[: sf_bytes(rows, cols, fmt, layout)]
+    return entries

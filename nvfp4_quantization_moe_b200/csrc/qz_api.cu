@@ -1,0 +1,160 @@
+// qz_api.cu -- the extern "C" entry points declared in include/qz.h.
+//
+// Host side only: argument checks that need no device memory, grid sizing
+// (one wave of resident CTAs on every SM, cached per device), and the
+// launches.  Nothing here allocates, synchronizes or reads device memory.
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <mutex>
+
+#include "../../include/qz.h"
+
+namespace qz {
+cudaError_t launch_mxfp8(const qz_expert* table, int n, int layout, int grid, cudaStream_t s, unsigned* d_err);
+cudaError_t launch_nvfp4_tensor(const qz_expert* table, int n, int layout, bool compute_amax, int grid,
+                                cudaStream_t s, unsigned* d_err);
+cudaError_t launch_nvfp4_rows(const qz_expert* table, int n, int layout, int grid, cudaStream_t s, unsigned* d_err);
+cudaError_t launch_swizzle(const qz_sf_pair* table, int n, int grid, cudaStream_t s, unsigned* d_err);
+cudaError_t launch_rmsnorm_quant(const uint16_t* x, const uint16_t* r, const uint16_t* g, float eps, int64_t T,
+                                 int64_t H, uint16_t* y, uint16_t* h, int fmt, uint8_t* q, uint8_t* sf, int layout,
+                                 const float* amax, cudaStream_t s);
+int grouped_blocks_per_sm(int which, int n);
+int rows_blocks_per_sm(int n);
+}  // namespace qz
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr int kKinds = 5;  // mxfp8, nvfp4 tile, swizzle, amax, rows
+
+struct DeviceLimits {
+    int sms = 0;
+    int per_sm[kKinds] = {0, 0, 0, 0, 0};
+};
+
+std::mutex g_mu;
+DeviceLimits g_dev[kMaxDevices];
+
+// One wave of resident CTAs for kernel `kind` on the current device.  The
+// occupancy is taken once per device with the largest prefix table, so the
+// cached value never over-subscribes a smaller call.
+int wave_grid(int kind, const qz_launch_opts* opts) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
+    int grid;
+    {
+        std::lock_guard<std::mutex> lock(g_mu);
+        DeviceLimits& d = g_dev[dev];
+        if (d.sms == 0) {
+            int sms = 0;
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+            d.sms = sms > 0 ? sms : 1;
+        }
+        if (d.per_sm[kind] == 0)
+            d.per_sm[kind] = (kind == 4) ? qz::rows_blocks_per_sm(QZ_MAX_EXPERTS)
+                                         : qz::grouped_blocks_per_sm(kind, QZ_MAX_EXPERTS);
+        grid = d.sms * d.per_sm[kind];
+    }
+    if (opts && opts->max_ctas > 0 && opts->max_ctas < grid) grid = opts->max_ctas;
+    return grid;
+}
+
+bool aligned(const void* p, uintptr_t a) { return ((uintptr_t)p & (a - 1)) == 0; }
+
+unsigned* err_word(const qz_launch_opts* opts) { return opts ? opts->d_err : nullptr; }
+
+qz_status check_table(const void* table, int n) {
+    if (n < 0 || n > QZ_MAX_EXPERTS) return QZ_ERR_INVALID_ARG;
+    if (n > 0 && table == nullptr) return QZ_ERR_INVALID_ARG;
+    return QZ_OK;
+}
+
+bool valid_layout(int layout) { return layout == QZ_SF_LINEAR || layout == QZ_SF_SWIZZLED_128x4; }
+
+qz_status from_cuda(cudaError_t e) { return e == cudaSuccess ? QZ_OK : QZ_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+size_t qz_sf_bytes(int64_t rows, int64_t cols, int fmt, int layout) {
+    if (fmt != QZ_FMT_MXFP8 && fmt != QZ_FMT_NVFP4) return 0;
+    if (!valid_layout(layout)) return 0;
+    const int64_t block = fmt == QZ_FMT_MXFP8 ? 32 : 16;
+    if (rows <= 0 || cols <= 0 || cols % block != 0) return 0;
+    const int64_t kv = cols / block;
+    if (layout == QZ_SF_LINEAR) return (size_t)(rows * kv);
+    return (size_t)(((rows + 127) / 128) * 128 * ((kv + 3) / 4) * 4);
+}
+
+qz_status qz_quantize_grouped_mxfp8(const qz_expert* d_table, int n_experts, int layout, void* stream,
+                                    const qz_launch_opts* opts) {
+    qz_status st = check_table(d_table, n_experts);
+    if (st != QZ_OK) return st;
+    if (!valid_layout(layout)) return QZ_ERR_INVALID_ARG;
+    if (n_experts == 0) return QZ_OK;
+    return from_cuda(qz::launch_mxfp8(d_table, n_experts, layout, wave_grid(0, opts), (cudaStream_t)stream,
+                                      err_word(opts)));
+}
+
+qz_status qz_quantize_grouped_nvfp4(const qz_expert* d_table, int n_experts, int mode, int layout, void* stream,
+                                    const qz_launch_opts* opts) {
+    qz_status st = check_table(d_table, n_experts);
+    if (st != QZ_OK) return st;
+    if (!valid_layout(layout)) return QZ_ERR_INVALID_ARG;
+    if (mode != QZ_NVFP4_PER_TENSOR_GIVEN && mode != QZ_NVFP4_PER_TENSOR_COMPUTE && mode != QZ_NVFP4_PER_ROW)
+        return QZ_ERR_INVALID_ARG;
+    if (n_experts == 0) return QZ_OK;
+    cudaStream_t s = (cudaStream_t)stream;
+    if (mode == QZ_NVFP4_PER_ROW)
+        return from_cuda(qz::launch_nvfp4_rows(d_table, n_experts, layout, wave_grid(4, opts), s, err_word(opts)));
+    return from_cuda(qz::launch_nvfp4_tensor(d_table, n_experts, layout, mode == QZ_NVFP4_PER_TENSOR_COMPUTE,
+                                             wave_grid(1, opts), s, err_word(opts)));
+}
+
+qz_status qz_rmsnorm_quantize(const void* d_x, const void* d_residual, const void* d_gamma, float eps, int64_t T,
+                              int64_t H, void* d_norm_out, void* d_residual_out, int fmt, void* d_q, uint8_t* d_sf,
+                              int layout, const float* d_global_amax, void* stream) {
+    if (fmt != QZ_FMT_MXFP8 && fmt != QZ_FMT_NVFP4) return QZ_ERR_INVALID_ARG;
+    if (!valid_layout(layout)) return QZ_ERR_INVALID_ARG;
+    const int64_t block = fmt == QZ_FMT_MXFP8 ? 32 : 16;
+    if (T < 0 || H <= 0 || H > QZ_MAX_HIDDEN || H % block != 0) return QZ_ERR_INVALID_ARG;
+    if (T > 0x7FFFFF00LL) return QZ_ERR_INVALID_ARG;
+    if (layout == QZ_SF_SWIZZLED_128x4 && (H / block) % 4 != 0) return QZ_ERR_UNSUPPORTED;
+    if (T == 0) return QZ_OK;
+    if (!d_x || !d_residual || !d_gamma || !d_norm_out || !d_q || !d_sf) return QZ_ERR_INVALID_ARG;
+    if (fmt == QZ_FMT_NVFP4 && !d_global_amax) return QZ_ERR_INVALID_ARG;
+    if (!aligned(d_x, 16) || !aligned(d_residual, 16) || !aligned(d_gamma, 16) || !aligned(d_norm_out, 16) ||
+        (d_residual_out && !aligned(d_residual_out, 16)))
+        return QZ_ERR_ALIGNMENT;
+    if (!aligned(d_q, 8) || !aligned(d_sf, layout == QZ_SF_SWIZZLED_128x4 ? 16 : 4)) return QZ_ERR_ALIGNMENT;
+    if (d_global_amax && !aligned(d_global_amax, 4)) return QZ_ERR_ALIGNMENT;
+    return from_cuda(qz::launch_rmsnorm_quant(
+        static_cast<const uint16_t*>(d_x), static_cast<const uint16_t*>(d_residual),
+        static_cast<const uint16_t*>(d_gamma), eps, T, H, static_cast<uint16_t*>(d_norm_out),
+        static_cast<uint16_t*>(d_residual_out), fmt, static_cast<uint8_t*>(d_q), d_sf, layout, d_global_amax,
+        (cudaStream_t)stream));
+}
+
+qz_status qz_swizzle_scales(const qz_sf_pair* d_table, int n, void* stream, const qz_launch_opts* opts) {
+    qz_status st = check_table(d_table, n);
+    if (st != QZ_OK) return st;
+    if (n == 0) return QZ_OK;
+    return from_cuda(qz::launch_swizzle(d_table, n, wave_grid(2, opts), (cudaStream_t)stream, err_word(opts)));
+}
+
+const char* qz_status_string(qz_status status) {
+    switch (status) {
+        case QZ_OK: return "QZ_OK";
+        case QZ_ERR_INVALID_ARG: return "QZ_ERR_INVALID_ARG: invalid argument";
+        case QZ_ERR_ALIGNMENT: return "QZ_ERR_ALIGNMENT: misaligned pointer or stride";
+        case QZ_ERR_UNSUPPORTED: return "QZ_ERR_UNSUPPORTED: unsupported shape/format/layout combination";
+        case QZ_ERR_CUDA: return "QZ_ERR_CUDA: CUDA launch error";
+    }
+    return "unknown qz_status";
+}
+
+int qz_version(void) { return 100; }
+
+}  // extern "C"

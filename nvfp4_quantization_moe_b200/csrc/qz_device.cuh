@@ -1,0 +1,270 @@
+// qz_device.cuh -- device helpers of the grouped quantization kernels (sm_100a).
+//
+// Everything here is register/shared-memory arithmetic shared by the kernels
+// in this directory: 128-bit streaming loads, bf16 field access, the exact
+// E8M0 exponent, the NVFP4 two-level scale, hardware e4m3/e2m1 conversion,
+// the swizzled 128x4 offset and the expert-table walk.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/qz.h"
+
+namespace qz {
+
+constexpr int kThreads = 256;     // threads of every grouped CTA
+constexpr int kTileRows = 128;    // rows of a tile (one swizzled row block)
+constexpr int kTileCols = 128;    // bf16 columns of a tile: 16 chunks of 8 elements
+
+// ---------------------------------------------------------------------------
+// memory access
+// ---------------------------------------------------------------------------
+
+// 16-byte load that bypasses L1 allocation: every input byte is read once.
+__device__ __forceinline__ uint4 ld_stream(const void* p) {
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+
+__device__ __forceinline__ void st_v2(void* p, uint32_t a, uint32_t b) {
+    asm volatile("st.global.v2.u32 [%0], {%1,%2};" ::"l"(p), "r"(a), "r"(b) : "memory");
+}
+
+__device__ __forceinline__ void st_u32(void* p, uint32_t a) {
+    asm volatile("st.global.u32 [%0], %1;" ::"l"(p), "r"(a) : "memory");
+}
+
+__device__ __forceinline__ void st_v4(void* p, uint4 v) {
+    asm volatile("st.global.v4.u32 [%0], {%1,%2,%3,%4};" ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+                 : "memory");
+}
+
+// ---------------------------------------------------------------------------
+// bf16 fields
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// Largest |x| of the 8 bf16 in v, as bf16 magnitude bits.  For non-negative
+// IEEE values the integer order of the bit patterns is the numeric order.
+__device__ __forceinline__ uint32_t absmax_bits(uint4 v) {
+    uint32_t m = __vmaxu2(__vmaxu2(v.x & 0x7FFF7FFFu, v.y & 0x7FFF7FFFu),
+                          __vmaxu2(v.z & 0x7FFF7FFFu, v.w & 0x7FFF7FFFu));
+    return max(m & 0xFFFFu, m >> 16);
+}
+
+__device__ __forceinline__ float bits_to_float_bf16(uint32_t m16) { return __uint_as_float(m16 << 16); }
+
+// ---------------------------------------------------------------------------
+// MXFP8 scale
+// ---------------------------------------------------------------------------
+
+// E8M0 byte for a block whose largest magnitude has bf16 bits m16: the
+// smallest e with amax <= 448 * 2^e, as e + 127, clamped at 0.  With
+// amax = (1 + f/128) * 2^(E-127) and 448 = 1.75 * 2^8, e = E - 127 - 8 when
+// f <= 96 (significand <= 1.75) and one more otherwise.  Zero and subnormal
+// amax (< 2^-126 < 448 * 2^-128) clamp to byte 0.  Exact: no division.
+__device__ __forceinline__ uint32_t e8m0_byte(uint32_t m16) {
+    const int E = (int)(m16 >> 7);
+    if (E == 0) return 0u;
+    const int b = E - 8 + (((m16 & 0x7Fu) > 96u) ? 1 : 0);
+    return (uint32_t)max(b, 0);
+}
+
+// 2^-e for the scale byte (e = byte - 127): binary32 exponent field 254 - byte.
+// byte <= 247 for bf16 input, so the result is always a normal number and the
+// flush-to-zero rule never applies.
+__device__ __forceinline__ float e8m0_reciprocal(uint32_t byte) {
+    return __uint_as_float((254u - byte) << 23);
+}
+
+// ---------------------------------------------------------------------------
+// hardware conversions (PTX ISA: cvt with .satfinite; the first source
+// operand lands in the upper half of the packed result)
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ uint32_t cvt_e4m3x2(float lo, float hi) {
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// Eight e4m3 codes of x[i] * s, element 0 in the lowest byte.
+__device__ __forceinline__ uint2 e4m3x8_scaled(uint4 v, float s) {
+    const uint32_t a = cvt_e4m3x2(__fmul_rn(bf16_lo(v.x), s), __fmul_rn(bf16_hi(v.x), s));
+    const uint32_t b = cvt_e4m3x2(__fmul_rn(bf16_lo(v.y), s), __fmul_rn(bf16_hi(v.y), s));
+    const uint32_t c = cvt_e4m3x2(__fmul_rn(bf16_lo(v.z), s), __fmul_rn(bf16_hi(v.z), s));
+    const uint32_t d = cvt_e4m3x2(__fmul_rn(bf16_lo(v.w), s), __fmul_rn(bf16_hi(v.w), s));
+    return make_uint2(a | (b << 16), c | (d << 16));
+}
+
+// Eight e2m1 codes of x[i] * s, element 0 in the lowest nibble.
+__device__ __forceinline__ uint32_t e2m1x8_scaled(uint4 v, float s) {
+    uint32_t r;
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+        "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+        : "=r"(r)
+        : "f"(__fmul_rn(bf16_lo(v.x), s)), "f"(__fmul_rn(bf16_hi(v.x), s)),
+          "f"(__fmul_rn(bf16_lo(v.y), s)), "f"(__fmul_rn(bf16_hi(v.y), s)),
+          "f"(__fmul_rn(bf16_lo(v.z), s)), "f"(__fmul_rn(bf16_hi(v.z), s)),
+          "f"(__fmul_rn(bf16_lo(v.w), s)), "f"(__fmul_rn(bf16_hi(v.w), s)));
+    return r;
+}
+
+// e4m3 code (RNE, satfinite) of one non-negative float.
+__device__ __forceinline__ uint32_t e4m3_of(float v) { return cvt_e4m3x2(v, 0.0f) & 0xFFu; }
+
+// Value of a non-negative e4m3 code below 0x7F (bias 7, 3 mantissa bits).
+__device__ __forceinline__ float e4m3_value(uint32_t s) {
+    const uint32_t ef = s >> 3, m = s & 7u;
+    if (ef == 0) return (float)m * 0x1p-9f;
+    return __uint_as_float(((ef + 120u) << 23) | (m << 20));
+}
+
+// ---------------------------------------------------------------------------
+// NVFP4 two-level scale
+// ---------------------------------------------------------------------------
+
+// Encode scale from the tensor (or row) amax A: S = RN(1 / RN(A / 2688)),
+// zero when the decode scale is zero.
+__device__ __forceinline__ float nvfp4_encode_scale(float A) {
+    const float g = __fdiv_rn(A, 2688.0f);
+    return g == 0.0f ? 0.0f : __fdiv_rn(1.0f, g);
+}
+
+struct Nvfp4Block {
+    uint32_t scale;  // e4m3 code of the block scale
+    float rcp;       // multiplier applied to each element
+};
+
+// Block scale and element multiplier for a block of largest magnitude b.
+__device__ __forceinline__ Nvfp4Block nvfp4_block(float b, float S) {
+    Nvfp4Block r;
+    r.scale = (b == 0.0f) ? 0u : e4m3_of(__fmul_rn(__fdiv_rn(b, 6.0f), S));
+    r.rcp = 0.0f;
+    if (r.scale != 0u) {
+        float q = __fdiv_rn(S, e4m3_value(r.scale));
+        r.rcp = (q < 0x1p-126f) ? 0.0f : q;  // flush a subnormal reciprocal to zero
+    }
+    return r;
+}
+
+// ---------------------------------------------------------------------------
+// scale-factor layouts
+// ---------------------------------------------------------------------------
+
+__host__ __device__ __forceinline__ int64_t pad_to(int64_t a, int64_t b) { return (a + b - 1) / b * b; }
+
+// Byte of (row, k) inside a swizzled region with kv scale columns.
+__device__ __forceinline__ int64_t swz_offset(int64_t row, int64_t k, int64_t kv) {
+    const int64_t col_tiles = (kv + 3) >> 2;
+    const int64_t r = row & 127;
+    return (((row >> 7) * col_tiles + (k >> 2)) << 9) + ((((r & 31) << 2) + (r >> 5)) << 2) + (k & 3);
+}
+
+// Offset inside a 512-byte tile of (row in tile, k in tile).
+__device__ __forceinline__ int swz_in_tile(int r, int kc) { return ((((r & 31) << 2) + (r >> 5)) << 2) + kc; }
+
+// ---------------------------------------------------------------------------
+// expert table
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ bool aligned(const void* p, uintptr_t a) { return ((uintptr_t)p & (a - 1)) == 0; }
+
+// Check one table entry; returns the QZ_DERR_* bits that make it invalid.
+// fmt: QZ_FMT_MXFP8 / QZ_FMT_NVFP4; needs_amax: the NVFP4 modes.
+__device__ __forceinline__ unsigned entry_errors(const qz_expert& e, int fmt, int layout, bool needs_amax) {
+    const int64_t block = (fmt == QZ_FMT_MXFP8) ? 32 : 16;
+    unsigned bad = 0;
+    if (e.rows < 0 || e.cols <= 0 || (e.cols % block) != 0 || e.ld < e.cols) bad |= QZ_DERR_SHAPE;
+    if (e.rows > 0) {
+        if (!e.x || !e.q || !e.sf || (needs_amax && !e.amax)) bad |= QZ_DERR_NULL;
+        if (!aligned(e.x, 16) || (e.ld & 7) != 0) bad |= QZ_DERR_ALIGN;
+        if (!aligned(e.q, fmt == QZ_FMT_MXFP8 ? 8 : 4)) bad |= QZ_DERR_ALIGN;
+        if (layout == QZ_SF_SWIZZLED_128x4 && !aligned(e.sf, 16)) bad |= QZ_DERR_ALIGN;
+        if (needs_amax && !aligned(e.amax, 4)) bad |= QZ_DERR_ALIGN;
+    }
+    return bad;
+}
+
+__device__ __forceinline__ qz_expert load_entry(const qz_expert* t, int i) {
+    qz_expert e;
+    const int64_t* p = reinterpret_cast<const int64_t*>(t + i);
+    e.x = reinterpret_cast<const void*>(__ldg(p + 0));
+    e.rows = __ldg(p + 1);
+    e.cols = __ldg(p + 2);
+    e.ld = __ldg(p + 3);
+    e.q = reinterpret_cast<void*>(__ldg(p + 4));
+    e.sf = reinterpret_cast<uint8_t*>(__ldg(p + 5));
+    e.amax = reinterpret_cast<float*>(__ldg(p + 6));
+    return e;
+}
+
+// Exclusive prefix sum over i in [0, n) of count(i) into s_prefix[0..n] (ints);
+// every thread gets the total.  A total above INT32_MAX reports
+// QZ_DERR_TOO_LARGE and returns 0 (all CTAs agree).  Contains barriers: every
+// thread of the block must call it.
+template <typename Count>
+__device__ int block_prefix(int n, int* s_prefix, long long* s_scratch, Count count, unsigned* d_err) {
+    const int nt = blockDim.x;
+    const int per = (n + nt - 1) / nt;
+    const int beg = min(n, (int)threadIdx.x * per);
+    const int end = min(n, beg + per);
+    long long local = 0;
+    for (int i = beg; i < end; ++i) local += count(i);
+    // inclusive scan of `local` within the warp
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    long long incl = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        long long y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+        if (lane >= o) incl += y;
+    }
+    if (lane == 31) s_scratch[warp] = incl;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        long long run = 0;
+        for (int w = 0; w < nt / 32; ++w) {
+            long long t = s_scratch[w];
+            s_scratch[w] = run;
+            run += t;
+        }
+        s_scratch[32] = run;
+    }
+    __syncthreads();
+    long long total = s_scratch[32];
+    long long run = s_scratch[warp] + incl - local;
+    if (total <= 0x7FFFFFFFLL) {
+        for (int i = beg; i < end; ++i) {
+            s_prefix[i] = (int)run;
+            run += count(i);
+        }
+        if (threadIdx.x == 0) s_prefix[n] = (int)total;
+    } else if (threadIdx.x == 0 && blockIdx.x == 0 && d_err) {
+        atomicOr(d_err, QZ_DERR_TOO_LARGE);
+    }
+    __syncthreads();
+    return total <= 0x7FFFFFFFLL ? (int)total : 0;
+}
+
+// The expert owning unit u: the largest e with s_prefix[e] <= u (empty
+// experts share their successor's start and are skipped by the search).
+__device__ __forceinline__ int find_owner(const int* s_prefix, int n, int u) {
+    int lo = 0, hi = n - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (s_prefix[mid] <= u) lo = mid; else hi = mid - 1;
+    }
+    return lo;
+}
+
+}  // namespace qz

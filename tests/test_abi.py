@@ -1,0 +1,103 @@
+"""The C-ABI library builds, loads and exports every function include/qz.h
+declares; host-side argument checks answer without touching a GPU."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import nvfp4_quantization_moe_b200 as qz
+from nvfp4_quantization_moe_b200 import build as qzbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "qz.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(qz_[a-z0-9_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    qzbuild.build()
+    return qz.load()
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for n in ("qz_quantize_grouped_mxfp8", "qz_quantize_grouped_nvfp4", "qz_rmsnorm_quantize",
+              "qz_swizzle_scales", "qz_sf_bytes", "qz_status_string"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", qz.LIB_PATH], capture_output=True, text=True,
+                         check=True).stdout
+    exported = set(re.findall(r"\bT\s+(qz_[a-z0-9_]+)$", out, flags=re.M))
+    missing = [n for n in declared_functions() if n not in exported]
+    assert not missing, missing
+    for n in declared_functions():
+        assert hasattr(lib, n)
+    assert set(qz.EXPORTED) <= exported
+
+
+def test_sf_bytes_matches_oracle_regions(lib):
+    import oracle
+    for rows in (0, 1, 64, 127, 128, 129, 1536, 3000):
+        for cols in (16, 32, 48, 64, 256, 768, 2048, 4096, 7168):
+            for fmt, blk in ((qz.FMT_MXFP8, 32), (qz.FMT_NVFP4, 16)):
+                for layout in (qz.SF_LINEAR, qz.SF_SWIZZLED):
+                    got = qz.sf_bytes(rows, cols, fmt, layout)
+                    if cols % blk:
+                        assert got == 0
+                    else:
+                        assert got == oracle.sf_region_bytes(rows, cols // blk, layout)
+    assert qz.sf_bytes(4, 64, 7, 0) == 0 and qz.sf_bytes(4, 64, 0, 9) == 0 and qz.sf_bytes(-1, 64, 0, 0) == 0
+
+
+def test_host_errors_without_gpu(lib):
+    P = ctypes.c_void_p
+    assert lib.qz_quantize_grouped_mxfp8(None, -1, 0, None, None) == qz.QZ_ERR_INVALID_ARG
+    assert lib.qz_quantize_grouped_mxfp8(None, 3, 0, None, None) == qz.QZ_ERR_INVALID_ARG
+    assert lib.qz_quantize_grouped_mxfp8(P(0x1000), qz.MAX_EXPERTS + 1, 0, None, None) == qz.QZ_ERR_INVALID_ARG
+    assert lib.qz_quantize_grouped_mxfp8(P(0x1000), 2, 5, None, None) == qz.QZ_ERR_INVALID_ARG
+    assert lib.qz_quantize_grouped_mxfp8(None, 0, 0, None, None) == qz.QZ_OK
+    assert lib.qz_quantize_grouped_nvfp4(P(0x1000), 2, 7, 0, None, None) == qz.QZ_ERR_INVALID_ARG
+    assert lib.qz_quantize_grouped_nvfp4(None, 0, 2, 1, None, None) == qz.QZ_OK
+    assert lib.qz_swizzle_scales(None, 1, None, None) == qz.QZ_ERR_INVALID_ARG
+    assert lib.qz_swizzle_scales(None, 0, None, None) == qz.QZ_OK
+    a = P(0x10000)
+
+    def norm(T=4, H=7168, fmt=0, layout=1, x=a, r=a, g=a, y=a, h=None, q=a, sf=a, amax=None):
+        return lib.qz_rmsnorm_quantize(x, r, g, ctypes.c_float(1e-6), T, H, y, h, fmt, q, sf, layout, amax, None)
+
+    assert norm(T=-1) == qz.QZ_ERR_INVALID_ARG
+    assert norm(H=0) == qz.QZ_ERR_INVALID_ARG
+    assert norm(H=qz.MAX_HIDDEN + 128) == qz.QZ_ERR_INVALID_ARG
+    assert norm(H=7168 + 16) == qz.QZ_ERR_INVALID_ARG           # not a multiple of 32 (MXFP8)
+    assert norm(H=32 * 6) == qz.QZ_ERR_UNSUPPORTED               # swizzled with kv % 4 != 0
+    assert norm(fmt=1, layout=0) == qz.QZ_ERR_INVALID_ARG        # NVFP4 without the global amax
+    assert norm(x=None) == qz.QZ_ERR_INVALID_ARG
+    assert norm(x=P(0x10002)) == qz.QZ_ERR_ALIGNMENT
+    assert norm(sf=P(0x10004)) == qz.QZ_ERR_ALIGNMENT            # swizzled SF wants 16 bytes
+    assert norm(fmt=7) == qz.QZ_ERR_INVALID_ARG
+    assert norm(T=0) == qz.QZ_OK                                  # nothing to do, nothing launched
+
+
+def test_status_strings(lib):
+    for s in range(5):
+        assert qz.status_string(s).startswith("QZ_")
+    assert qz.status_string(99) == "unknown qz_status"
+
+
+def test_product_path_does_not_import_oracle():
+    """The binding and the CUDA sources never reach the oracle."""
+    pkg = os.path.join(ROOT, "nvfp4_quantization_moe_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                text = open(os.path.join(dirpath, f)).read()
+                assert "import oracle" not in text and "from oracle" not in text and "qz_oracle" not in text, f
