@@ -311,21 +311,43 @@ def e2e_refit(qz, device, steps, warmup, layers=48, per_call=16, pool=2):
 # extra workloads (one timed line each, not the headline)
 # ---------------------------------------------------------------------------
 
-def _time_call(fn, stream, reps=20, warm=5):
-    for _ in range(warm):
-        fn()
-    torch.cuda.synchronize()
-    evs = []
-    for _ in range(reps):
-        a = torch.cuda.Event(enable_timing=True)
-        b = torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        fn()
-        b.record(stream)
-        evs.append((a, b))
-    torch.cuda.synchronize()
-    ts = sorted(a.elapsed_time(b) for a, b in evs)
-    return ts[len(ts) // 2]
+def _time_graph(fn, reps=20, flush=None):
+    """Median-free device time of one call: `reps` calls (each after an L2
+    flush when given) captured in one CUDA graph, replayed and timed with CUDA
+    events; the flush time, measured the same way, is subtracted."""
+    def capture(body):
+        g = torch.cuda.CUDAGraph()
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            body()
+            torch.cuda.synchronize()
+            with torch.cuda.graph(g, stream=s):
+                for _ in range(reps):
+                    body()
+        torch.cuda.current_stream().wait_stream(s)
+        return g
+
+    def run(g):
+        g.replay()
+        torch.cuda.synchronize()
+        best = None
+        for _ in range(3):
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record()
+            g.replay()
+            b.record()
+            torch.cuda.synchronize()
+            t = a.elapsed_time(b) / reps
+            best = t if best is None else min(best, t)
+        return best
+
+    if flush is None:
+        return run(capture(fn))
+    both = run(capture(lambda: (flush(), fn())))
+    only = run(capture(flush))
+    return max(both - only, 1e-6)
 
 
 class L2Flush:
@@ -336,7 +358,7 @@ class L2Flush:
         self.buf.zero_()
 
 
-def extra_workloads(qz, device, stream, peak):
+def extra_workloads(qz, device, stream, peak, which=("split", "fused", "large")):
     out = []
     flush = L2Flush(device)
 
@@ -347,8 +369,17 @@ def extra_workloads(qz, device, stream, peak):
         d.update(kw)
         out.append(d)
 
-    # row-scaled NVFP4 split activation [16384, 4096], 64 experts
-    cfg = synth.SPLIT_ACT
+    if "split" in which:
+        _extra_split(qz, device, flush, rec)
+    if "fused" in which:
+        _extra_fused(qz, device, flush, out, peak)
+    if "large" in which:
+        _extra_large(qz, device, rec)
+    return out
+
+
+def _extra_split(qz, device, flush, rec):
+    """Row-scaled NVFP4 split activation [16384, 4096] over 64 experts."""
     x = synth.split_activation(device=device)
     counts = synth.dirichlet_splits()
     T, K = x.shape
@@ -365,17 +396,17 @@ def extra_workloads(qz, device, stream, peak):
     table = qz.ExpertTable(entries)
 
     def split_call():
-        flush()
-        qz.quantize_grouped_nvfp4(table, qz.NVFP4_PER_ROW, qz.SF_SWIZZLED, stream=stream)
+        qz.quantize_grouped_nvfp4(table, qz.NVFP4_PER_ROW, qz.SF_SWIZZLED)
 
-    ms_flush = _time_call(flush, stream)
-    ms = _time_call(split_call, stream) - ms_flush
+    ms = _time_graph(split_call, reps=10, flush=flush)
     nbytes = T * K * 2 + T * K // 2 + nsf_tot + T * 4
     rec("row-scaled NVFP4 split [16384,4096] over 64 Dirichlet(0.3) experts, swizzled", nbytes, ms, 1,
-        kernel="nvfp4_rows_kernel", l2="flushed before each call")
+        kernel="nvfp4_rows_kernel", l2="flushed before each call", timing="CUDA graph of 10 calls")
     del x, q, am, entries, table
 
-    # fused residual + RMSNorm + quantize, T sweep at H = 7168
+
+def _extra_fused(qz, device, flush, out, peak):
+    """Fused residual + RMSNorm + quantize, T sweep at H = 7168."""
     H = synth.FUSED_NORM["hidden"]
     for fmt, layout, fname in ((qz.FMT_MXFP8, qz.SF_SWIZZLED, "MXFP8 swizzled"), (qz.FMT_NVFP4, qz.SF_LINEAR, "NVFP4 linear")):
         sweep = []
@@ -388,21 +419,21 @@ def extra_workloads(qz, device, stream, peak):
             amax = torch.tensor([8.0], dtype=torch.float32, device=device) if fmt == qz.FMT_NVFP4 else None
 
             def call():
-                qz.rmsnorm_quantize(xs, rs, gs, 1e-6, y, h, fmt, qq, sff, layout, amax, stream=stream)
+                qz.rmsnorm_quantize(xs, rs, gs, 1e-6, y, h, fmt, qq, sff, layout, amax)
 
-            if Tn >= 1024:
-                ms = _time_call(lambda: (flush(), call()), stream) - ms_flush
-            else:
-                ms = _time_call(call, stream, reps=50)
+            ms = _time_graph(call, reps=10, flush=flush) if Tn >= 1024 else _time_graph(call, reps=50)
             qbytes = Tn * (H if fmt == qz.FMT_MXFP8 else H // 2)
             nbytes = Tn * H * 2 * 2 + 2 * H + Tn * H * 2 * 2 + qbytes + qz.sf_bytes(Tn, H, fmt, layout)
             sweep.append({"T": Tn, "us": round(ms * 1e3, 2), "GB/s": round(nbytes / (ms / 1e3) / GB, 1)})
         big = sweep[-1]
         out.append({"workload": f"fused residual+RMSNorm+{fname}, H=7168, T=1..4096 (residual_out written)",
                     "kernel": "rmsnorm_quant_kernel", "sweep": sweep,
+                    "timing": "CUDA graph of 50 calls (T < 1024) or 10 calls after an L2 flush each",
                     "frac_of_hbm_peak_T4096": round(big["GB/s"] / peak, 4)})
 
-    # one Qwen3-235B-A22B layer: 128 experts per projection per call
+
+def _extra_large(qz, device, rec):
+    """One Qwen3-235B-A22B layer: 128 experts per projection per call."""
     cfg = synth.QWEN3_235B
     for proj, shape in (("gate_up", cfg["gate_up"]), ("down", cfg["down"])):
         stack = synth.expert_stack(cfg["experts"], shape, cfg["std"], seed=cfg["seed"], device=device)
@@ -416,10 +447,10 @@ def extra_workloads(qz, device, stream, peak):
                     e.amax.fill_(0.1)
             tab = qz.ExpertTable(ents)
             if fmt == qz.FMT_MXFP8:
-                fn = lambda: qz.quantize_grouped_mxfp8(tab, qz.SF_SWIZZLED, stream=stream)  # noqa: E731
+                fn = lambda: qz.quantize_grouped_mxfp8(tab, qz.SF_SWIZZLED)  # noqa: E731
             else:
-                fn = lambda m=mode: qz.quantize_grouped_nvfp4(tab, m, qz.SF_SWIZZLED, stream=stream)  # noqa: E731
-            ms = _time_call(fn, stream, reps=10, warm=3)
+                fn = lambda m=mode: qz.quantize_grouped_nvfp4(tab, m, qz.SF_SWIZZLED)  # noqa: E731
+            ms = _time_graph(fn, reps=5)
             nsf = qz.sf_bytes(rows, cols, fmt, qz.SF_SWIZZLED)
             qb = rows * cols if fmt == qz.FMT_MXFP8 else rows * cols // 2
             nbytes = cfg["experts"] * (rows * cols * 2 + qb + nsf + (4 if fmt == qz.FMT_NVFP4 else 0))
@@ -428,7 +459,6 @@ def extra_workloads(qz, device, stream, peak):
             del ents, tab
         del stack
         torch.cuda.empty_cache()
-    return out
 
 
 # ---------------------------------------------------------------------------
@@ -449,7 +479,7 @@ def oracle_refit_sample(target_s: float = 12.0):
     oracle.quantize_grouped([gu, dn], oracle.MXFP8, oracle.SWIZZLED, threads=2)
     one = time.perf_counter() - t0                     # 2 experts on 2 threads
     pairs = max(1, int(target_s / max(one, 1e-3) * threads / 2))
-    pairs = min(pairs, 64)
+    pairs = min(pairs, 2048)
     experts = [gu, dn] * pairs
     t0 = time.perf_counter()
     oracle.quantize_grouped(experts, oracle.MXFP8, oracle.SWIZZLED, threads=threads)
@@ -491,13 +521,15 @@ def run_reference(args, rank, world):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--layers", type=int, default=48)
     ap.add_argument("--no-extra", action="store_true", help="skip the other workloads")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    ap.add_argument("--only", choices=["split", "fused", "large"], default=None,
+                    help="time only this secondary workload and print its record (profiling aid)")
     args = ap.parse_args()
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -519,6 +551,9 @@ def main():
         torch.distributed.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=device)
     stream = torch.cuda.current_stream()
     peak, peak_kind = hbm_peak()
+    if args.only:
+        print(json.dumps({"only": args.only, "extra": extra_workloads(qz, device, stream, peak, (args.only,))}))
+        return
 
     work = Refit30B(qz, device, layers=args.layers, seed_offset=rank)
     torch.cuda.synchronize()

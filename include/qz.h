@@ -86,6 +86,8 @@ typedef enum qz_nvfp4_scale_mode {
                                   8-byte (MXFP8) / 4-byte (NVFP4) aligned; sf not 16-byte
                                   aligned (swizzled); amax not 4-byte aligned */
 #define QZ_DERR_TOO_LARGE 0x8u /* the call's total tile or row count exceeds 2^31 - 1 */
+#define QZ_DERR_TIMEOUT 0x10u  /* a wait for an asynchronous copy exceeded its time limit; the
+                                  kernel stopped early (no such wait is expected to expire) */
 
 /* Largest table a grouped call accepts (the kernels keep the table's prefix
  * sums in shared memory). */

@@ -43,139 +43,135 @@ struct TableTiles {
 };
 
 // ---------------------------------------------------------------------------
-// MXFP8 tile
+// tile walk with a register prefetch ring
+//
+// Pass p (0..7) of warp w covers tile rows (p & 3) * 32 + 4w + 2 (p >> 2) +
+// lane / 16: the warp owns rows r with r % 32 in [4w, 4w + 4), i.e. exactly
+// four 16-byte chunks of every 512-byte swizzled scale tile, which it
+// assembles in its own 64 bytes of shared memory (no CTA barrier).  As soon
+// as pass p of the current tile is consumed, slot p is refilled with pass p
+// of the CTA's next tile, so about eight 16-byte loads per thread are always
+// in flight.
 // ---------------------------------------------------------------------------
-template <int LAYOUT>
-__device__ __forceinline__ void mxfp8_tile(const qz_expert& E, int64_t rt, int64_t ct, uint8_t* s_sf) {
-    const int t = threadIdx.x;
-    const int chunk = t & 15;
-    const int rsub = t >> 4;
-    const int64_t col = ct * kTileCols + chunk * 8;
-    const bool col_ok = col < E.cols;
-    const int64_t kv = E.cols >> 5;
-    const uint16_t* x = static_cast<const uint16_t*>(E.x);
-    uint8_t* q = static_cast<uint8_t*>(E.q);
 
-    uint4 v[8];
-#pragma unroll
-    for (int p = 0; p < 8; ++p) {
-        const int64_t row = rt * kTileRows + p * 16 + rsub;
-        v[p] = (row < E.rows && col_ok) ? ld_stream(x + row * E.ld + col) : make_uint4(0, 0, 0, 0);
-    }
-#pragma unroll
-    for (int p = 0; p < 8; ++p) {
-        const int r = p * 16 + rsub;
-        const int64_t row = rt * kTileRows + r;
-        const bool live = row < E.rows && col_ok;
-        uint32_t m = absmax_bits(v[p]);
-        m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
+struct TileRef {
+    const uint16_t* x;
+    int64_t rows, cols, ld;
+    uint8_t* q;
+    uint8_t* sf;
+    const float* amax;
+    int64_t rt, ct;
+    int expert;
+};
+
+__device__ __forceinline__ TileRef tile_ref(const qz_expert* table, const int* s_prefix, int n, int tile) {
+    const int e = find_owner(s_prefix, n, tile);
+    const qz_expert E = load_entry(table, e);
+    const int64_t local = tile - s_prefix[e];
+    const int64_t nct = (E.cols + kTileCols - 1) / kTileCols;
+    TileRef t;
+    t.x = static_cast<const uint16_t*>(E.x);
+    t.rows = E.rows;
+    t.cols = E.cols;
+    t.ld = E.ld;
+    t.q = static_cast<uint8_t*>(E.q);
+    t.sf = E.sf;
+    t.amax = E.amax;
+    t.rt = local / nct;
+    t.ct = local % nct;
+    t.expert = e;
+    return t;
+}
+
+__device__ __forceinline__ int tile_row(int p, int w, int lane) { return (p & 3) * 32 + 4 * w + 2 * (p >> 2) + (lane >> 4); }
+
+__device__ __forceinline__ uint4 tile_load(const TileRef& t, int p, int w, int lane) {
+    const int64_t row = t.rt * kTileRows + tile_row(p, w, lane);
+    const int64_t col = t.ct * kTileCols + (lane & 15) * 8;
+    return (row < t.rows && col < t.cols) ? ld_stream(t.x + row * t.ld + col) : make_uint4(0, 0, 0, 0);
+}
+
+// Quantize pass p of tile t (8 elements per thread in v).  MXFP8 blocks span
+// 4 lanes, NVFP4 blocks 2.  Swizzled scale bytes go to the warp's staging
+// area s (64 bytes per 4-column scale tile), linear ones straight to memory.
+template <int FMT, int LAYOUT>
+__device__ __forceinline__ void tile_pass(const TileRef& t, int p, int w, int lane, uint4 v, float S, uint8_t* s) {
+    const int chunk = lane & 15;
+    const int64_t row = t.rt * kTileRows + tile_row(p, w, lane);
+    const int64_t col = t.ct * kTileCols + chunk * 8;
+    const bool live = row < t.rows && col < t.cols;
+    const int stage = (2 * (p >> 2) + (lane >> 4)) * 16 + (p & 3) * 4;  // byte of this row in the warp's chunks
+    uint32_t m = absmax_bits(v);
+    m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
+    if (FMT == QZ_FMT_MXFP8) {
         m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
         const uint32_t byte = e8m0_byte(m);
-        const uint2 codes = e4m3x8_scaled(v[p], e8m0_reciprocal(byte));
-        if (live) st_v2(q + row * E.cols + col, codes.x, codes.y);
+        const uint2 codes = e4m3x8_scaled(v, e8m0_reciprocal(byte));
+        if (live) st_v2(t.q + row * t.cols + col, codes.x, codes.y);
         if ((chunk & 3) == 0) {
             const int kc = chunk >> 2;
-            if (LAYOUT == QZ_SF_SWIZZLED_128x4) {
-                s_sf[swz_in_tile(r, kc)] = live ? (uint8_t)byte : (uint8_t)0;
-            } else if (live) {
-                E.sf[row * kv + ct * 4 + kc] = (uint8_t)byte;
-            }
+            if (LAYOUT == QZ_SF_SWIZZLED_128x4) s[stage + kc] = live ? (uint8_t)byte : (uint8_t)0;
+            else if (live) t.sf[row * (t.cols >> 5) + t.ct * 4 + kc] = (uint8_t)byte;
         }
-    }
-    if (LAYOUT == QZ_SF_SWIZZLED_128x4) {
-        __syncthreads();
-        if (t < 32) {
-            const int64_t col_tiles = (kv + 3) >> 2;
-            uint8_t* dst = E.sf + ((rt * col_tiles + ct) << 9) + t * 16;
-            st_v4(dst, reinterpret_cast<const uint4*>(s_sf)[t]);
-        }
-    }
-}
-
-template <int LAYOUT>
-__global__ void __launch_bounds__(kThreads) mxfp8_grouped_kernel(const qz_expert* __restrict__ table, int n,
-                                                                 unsigned* d_err) {
-    extern __shared__ int s_prefix[];
-    __shared__ long long s_scan[33];
-    __shared__ __align__(16) uint8_t s_sf[2][512];
-    const int total = block_prefix(n, s_prefix, s_scan, TableTiles<QZ_FMT_MXFP8, LAYOUT, false>{table, d_err}, d_err);
-    int it = 0;
-    for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++it) {
-        const int e = find_owner(s_prefix, n, tile);
-        const qz_expert E = load_entry(table, e);
-        const int64_t local = tile - s_prefix[e];
-        const int64_t nct = (E.cols + kTileCols - 1) / kTileCols;
-        mxfp8_tile<LAYOUT>(E, local / nct, local % nct, s_sf[it & 1]);
-    }
-}
-
-// ---------------------------------------------------------------------------
-// NVFP4 tile, per-tensor second-level scale (amax[0] of the expert)
-// ---------------------------------------------------------------------------
-template <int LAYOUT>
-__device__ __forceinline__ void nvfp4_tile(const qz_expert& E, int64_t rt, int64_t ct, uint8_t* s_sf) {
-    const int t = threadIdx.x;
-    const int chunk = t & 15;
-    const int rsub = t >> 4;
-    const int64_t col = ct * kTileCols + chunk * 8;
-    const bool col_ok = col < E.cols;
-    const int64_t kv = E.cols >> 4;
-    const uint16_t* x = static_cast<const uint16_t*>(E.x);
-    uint8_t* q = static_cast<uint8_t*>(E.q);
-    const float S = nvfp4_encode_scale(*E.amax);
-
-    uint4 v[8];
-#pragma unroll
-    for (int p = 0; p < 8; ++p) {
-        const int64_t row = rt * kTileRows + p * 16 + rsub;
-        v[p] = (row < E.rows && col_ok) ? ld_stream(x + row * E.ld + col) : make_uint4(0, 0, 0, 0);
-    }
-#pragma unroll
-    for (int p = 0; p < 8; ++p) {
-        const int r = p * 16 + rsub;
-        const int64_t row = rt * kTileRows + r;
-        const bool live = row < E.rows && col_ok;
-        uint32_t m = absmax_bits(v[p]);
-        m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
+    } else {
         const Nvfp4Block blk = nvfp4_block(bits_to_float_bf16(m), S);
-        const uint32_t codes = e2m1x8_scaled(v[p], blk.rcp);
-        if (live) st_u32(q + row * (E.cols >> 1) + (col >> 1), codes);
+        const uint32_t codes = e2m1x8_scaled(v, blk.rcp);
+        if (live) st_u32(t.q + row * (t.cols >> 1) + (col >> 1), codes);
         if ((chunk & 1) == 0) {
             const int kk = chunk >> 1;  // 0..7: two 4-column scale tiles per tile
-            if (LAYOUT == QZ_SF_SWIZZLED_128x4) {
-                s_sf[((kk >> 2) << 9) + swz_in_tile(r, kk & 3)] = live ? (uint8_t)blk.scale : (uint8_t)0;
-            } else if (live) {
-                E.sf[row * kv + ct * 8 + kk] = (uint8_t)blk.scale;
-            }
-        }
-    }
-    if (LAYOUT == QZ_SF_SWIZZLED_128x4) {
-        __syncthreads();
-        if (t < 64) {
-            const int64_t col_tiles = (kv + 3) >> 2;
-            const int64_t ctile = ct * 2 + (t >> 5);
-            if (ctile < col_tiles) {
-                uint8_t* dst = E.sf + ((rt * col_tiles + ctile) << 9) + (t & 31) * 16;
-                st_v4(dst, reinterpret_cast<const uint4*>(s_sf)[t]);
-            }
+            if (LAYOUT == QZ_SF_SWIZZLED_128x4) s[(kk >> 2) * 64 + stage + (kk & 3)] = live ? (uint8_t)blk.scale : (uint8_t)0;
+            else if (live) t.sf[row * (t.cols >> 4) + t.ct * 8 + kk] = (uint8_t)blk.scale;
         }
     }
 }
 
-template <int LAYOUT>
-__global__ void __launch_bounds__(kThreads) nvfp4_tensor_grouped_kernel(const qz_expert* __restrict__ table, int n,
-                                                                        unsigned* d_err) {
+// Store the warp's staged chunks of the tile's swizzled scale tile(s).
+template <int FMT>
+__device__ __forceinline__ void tile_flush_sf(const TileRef& t, int w, int lane, const uint8_t* s) {
+    __syncwarp();
+    const int64_t kv = FMT == QZ_FMT_MXFP8 ? (t.cols >> 5) : (t.cols >> 4);
+    const int64_t col_tiles = (kv + 3) >> 2;
+    constexpr int kTilesPerTile = FMT == QZ_FMT_MXFP8 ? 1 : 2;
+    if (lane < 4 * kTilesPerTile) {
+        const int j = lane >> 2, c = lane & 3;
+        const int64_t ctile = t.ct * kTilesPerTile + j;
+        if (ctile < col_tiles)
+            st_v4(t.sf + ((t.rt * col_tiles + ctile) << 9) + (4 * w + c) * 16,
+                  *reinterpret_cast<const uint4*>(s + j * 64 + c * 16));
+    }
+    __syncwarp();
+}
+
+template <int FMT, int LAYOUT>
+__global__ void __launch_bounds__(kThreads, 3) grouped_tile_kernel(const qz_expert* __restrict__ table, int n,
+                                                                unsigned* d_err) {
     extern __shared__ int s_prefix[];
     __shared__ long long s_scan[33];
-    __shared__ __align__(16) uint8_t s_sf[2][1024];
-    const int total = block_prefix(n, s_prefix, s_scan, TableTiles<QZ_FMT_NVFP4, LAYOUT, true>{table, d_err}, d_err);
-    int it = 0;
-    for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++it) {
-        const int e = find_owner(s_prefix, n, tile);
-        const qz_expert E = load_entry(table, e);
-        const int64_t local = tile - s_prefix[e];
-        const int64_t nct = (E.cols + kTileCols - 1) / kTileCols;
-        nvfp4_tile<LAYOUT>(E, local / nct, local % nct, s_sf[it & 1]);
+    constexpr int kStage = FMT == QZ_FMT_MXFP8 ? 64 : 128;
+    __shared__ __align__(16) uint8_t s_sf[kThreads / 32][kStage];
+    constexpr bool kAmax = FMT == QZ_FMT_NVFP4;
+    const int total = block_prefix(n, s_prefix, s_scan, TableTiles<FMT, LAYOUT, kAmax>{table, d_err}, d_err);
+    const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    int tile = blockIdx.x;
+    if (tile >= total) return;
+    TileRef cur = tile_ref(table, s_prefix, n, tile);
+    uint4 v[8];
+#pragma unroll
+    for (int p = 0; p < 8; ++p) v[p] = tile_load(cur, p, w, lane);
+    for (;;) {
+        const int next = tile + gridDim.x;
+        const bool more = next < total;
+        const TileRef nxt = more ? tile_ref(table, s_prefix, n, next) : cur;
+        const float S = kAmax ? nvfp4_encode_scale(*cur.amax) : 0.0f;
+#pragma unroll
+        for (int p = 0; p < 8; ++p) {
+            tile_pass<FMT, LAYOUT>(cur, p, w, lane, v[p], S, s_sf[w]);
+            if (more) v[p] = tile_load(nxt, p, w, lane);
+        }
+        if (LAYOUT == QZ_SF_SWIZZLED_128x4) tile_flush_sf<FMT>(cur, w, lane, s_sf[w]);
+        if (!more) break;
+        cur = nxt;
+        tile = next;
     }
 }
 
@@ -191,47 +187,41 @@ __global__ void amax_clear_kernel(const qz_expert* __restrict__ table, int n, in
     }
 }
 
+// Same tile walk and prefetch ring as the quantize kernel; each warp keeps a
+// running maximum while its tiles stay in one expert and publishes it with
+// one atomic max (non-negative floats order like their bit patterns).
+template <int LAYOUT>
 __global__ void __launch_bounds__(kThreads) amax_grouped_kernel(const qz_expert* __restrict__ table, int n,
-                                                                int layout, unsigned* d_err) {
+                                                                unsigned* d_err) {
     extern __shared__ int s_prefix[];
     __shared__ long long s_scan[33];
-    __shared__ uint32_t s_max[kThreads / 32];
-    // the table check uses the caller's layout so that invalid entries are
-    // skipped identically by this pass and the quantize pass
-    int total;
-    if (layout == QZ_SF_SWIZZLED_128x4)
-        total = block_prefix(n, s_prefix, s_scan, TableTiles<QZ_FMT_NVFP4, QZ_SF_SWIZZLED_128x4, true>{table, d_err}, d_err);
-    else
-        total = block_prefix(n, s_prefix, s_scan, TableTiles<QZ_FMT_NVFP4, QZ_SF_LINEAR, true>{table, d_err}, d_err);
-    const int t = threadIdx.x, chunk = t & 15, rsub = t >> 4;
-    for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
-        const int e = find_owner(s_prefix, n, tile);
-        const qz_expert E = load_entry(table, e);
-        const int64_t local = tile - s_prefix[e];
-        const int64_t nct = (E.cols + kTileCols - 1) / kTileCols;
-        const int64_t rt = local / nct, ct = local % nct;
-        const int64_t col = ct * kTileCols + chunk * 8;
-        const uint16_t* x = static_cast<const uint16_t*>(E.x);
-        uint4 v[8];
+    const int total = block_prefix(n, s_prefix, s_scan, TableTiles<QZ_FMT_NVFP4, LAYOUT, true>{table, d_err}, d_err);
+    const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    int tile = blockIdx.x;
+    if (tile >= total) return;
+    TileRef cur = tile_ref(table, s_prefix, n, tile);
+    uint4 v[8];
+#pragma unroll
+    for (int p = 0; p < 8; ++p) v[p] = tile_load(cur, p, w, lane);
+    uint32_t run = 0;
+    for (;;) {
+        const int next = tile + gridDim.x;
+        const bool more = next < total;
+        const TileRef nxt = more ? tile_ref(table, s_prefix, n, next) : cur;
 #pragma unroll
         for (int p = 0; p < 8; ++p) {
-            const int64_t row = rt * kTileRows + p * 16 + rsub;
-            v[p] = (row < E.rows && col < E.cols) ? ld_stream(x + row * E.ld + col) : make_uint4(0, 0, 0, 0);
+            run = max(run, absmax_bits(v[p]));
+            if (more) v[p] = tile_load(nxt, p, w, lane);
         }
-        uint32_t m = 0;
+        if (!more || nxt.expert != cur.expert) {
 #pragma unroll
-        for (int p = 0; p < 8; ++p) m = max(m, absmax_bits(v[p]));
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
-        if ((t & 31) == 0) s_max[t >> 5] = m;
-        __syncthreads();
-        if (t == 0) {
-            uint32_t mm = 0;
-            for (int w = 0; w < kThreads / 32; ++w) mm = max(mm, s_max[w]);
-            // non-negative floats order like their bit patterns
-            atomicMax(reinterpret_cast<unsigned int*>(E.amax), mm << 16);
+            for (int o = 16; o > 0; o >>= 1) run = max(run, __shfl_xor_sync(0xFFFFFFFFu, run, o));
+            if (lane == 0) atomicMax(reinterpret_cast<unsigned int*>(const_cast<float*>(cur.amax)), run << 16);
+            run = 0;
         }
-        __syncthreads();
+        if (!more) break;
+        cur = nxt;
+        tile = next;
     }
 }
 
@@ -291,9 +281,9 @@ size_t prefix_smem(int n) { return (size_t)(n + 1) * sizeof(int); }
 
 cudaError_t launch_mxfp8(const qz_expert* table, int n, int layout, int grid, cudaStream_t s, unsigned* d_err) {
     if (layout == QZ_SF_SWIZZLED_128x4)
-        mxfp8_grouped_kernel<QZ_SF_SWIZZLED_128x4><<<grid, kThreads, prefix_smem(n), s>>>(table, n, d_err);
+        grouped_tile_kernel<QZ_FMT_MXFP8, QZ_SF_SWIZZLED_128x4><<<grid, kThreads, prefix_smem(n), s>>>(table, n, d_err);
     else
-        mxfp8_grouped_kernel<QZ_SF_LINEAR><<<grid, kThreads, prefix_smem(n), s>>>(table, n, d_err);
+        grouped_tile_kernel<QZ_FMT_MXFP8, QZ_SF_LINEAR><<<grid, kThreads, prefix_smem(n), s>>>(table, n, d_err);
     return cudaGetLastError();
 }
 
@@ -301,12 +291,15 @@ cudaError_t launch_nvfp4_tensor(const qz_expert* table, int n, int layout, bool 
                                 cudaStream_t s, unsigned* d_err) {
     if (compute_amax) {
         amax_clear_kernel<<<(n + kThreads - 1) / kThreads, kThreads, 0, s>>>(table, n, layout);
-        amax_grouped_kernel<<<grid, kThreads, prefix_smem(n), s>>>(table, n, layout, d_err);
+        if (layout == QZ_SF_SWIZZLED_128x4)
+            amax_grouped_kernel<QZ_SF_SWIZZLED_128x4><<<grid, kThreads, prefix_smem(n), s>>>(table, n, d_err);
+        else
+            amax_grouped_kernel<QZ_SF_LINEAR><<<grid, kThreads, prefix_smem(n), s>>>(table, n, d_err);
     }
     if (layout == QZ_SF_SWIZZLED_128x4)
-        nvfp4_tensor_grouped_kernel<QZ_SF_SWIZZLED_128x4><<<grid, kThreads, prefix_smem(n), s>>>(table, n, d_err);
+        grouped_tile_kernel<QZ_FMT_NVFP4, QZ_SF_SWIZZLED_128x4><<<grid, kThreads, prefix_smem(n), s>>>(table, n, d_err);
     else
-        nvfp4_tensor_grouped_kernel<QZ_SF_LINEAR><<<grid, kThreads, prefix_smem(n), s>>>(table, n, d_err);
+        grouped_tile_kernel<QZ_FMT_NVFP4, QZ_SF_LINEAR><<<grid, kThreads, prefix_smem(n), s>>>(table, n, d_err);
     return cudaGetLastError();
 }
 
@@ -320,10 +313,10 @@ int grouped_blocks_per_sm(int which, int n) {
     int b = 1;
     const size_t smem = prefix_smem(n);
     switch (which) {
-        case 0: cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, mxfp8_grouped_kernel<QZ_SF_SWIZZLED_128x4>, kThreads, smem); break;
-        case 1: cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, nvfp4_tensor_grouped_kernel<QZ_SF_SWIZZLED_128x4>, kThreads, smem); break;
+        case 0: cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, grouped_tile_kernel<QZ_FMT_MXFP8, QZ_SF_SWIZZLED_128x4>, kThreads, smem); break;
+        case 1: cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, grouped_tile_kernel<QZ_FMT_NVFP4, QZ_SF_SWIZZLED_128x4>, kThreads, smem); break;
         case 2: cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, swizzle_kernel, kThreads, smem); break;
-        default: cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, amax_grouped_kernel, kThreads, smem); break;
+        default: cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, amax_grouped_kernel<QZ_SF_SWIZZLED_128x4>, kThreads, smem); break;
     }
     return b > 0 ? b : 1;
 }

@@ -5,12 +5,14 @@
 // payload, row amax and scale factors land in per-expert storage whose
 // swizzled padding is independent per expert (uneven and empty splits).
 //
-// One warp per row.  A row of up to 4096 elements stays in registers (16
-// chunks of 8 bf16 per lane), so the row amax and the block scales come from a
-// single read of HBM; longer rows take a second pass over the row (served by
-// L2).  Lane l holds chunks l + 32i: the two chunks of a 16-element block sit
-// in lanes (2j, 2j+1) and the four blocks of one 4-byte scale group in eight
-// consecutive lanes, so a scale group leaves as one 32-bit store.
+// One warp per row.  Rows of up to 4096 elements are brought into shared
+// memory by one bulk (TMA) copy each: every warp keeps kRowDepth rows in
+// flight in its own ring of shared-memory slots, each slot with an mbarrier
+// that the copy completes, so HBM streams while the warp quantizes.  From the
+// slot a lane takes chunks l + 32i (8 bf16 each): the two chunks of a
+// 16-element block sit in lanes (2j, 2j+1) and the four blocks of one 4-byte
+// scale group in eight consecutive lanes, so a scale group leaves as one
+// 32-bit store.  Longer rows take a two-pass path straight from global memory.
 //
 // Units of work are "virtual rows": an expert owns rows (linear layout) or
 // pad(rows, 128) virtual rows (swizzled); a virtual row past the last live row
@@ -20,7 +22,12 @@
 
 namespace qz {
 
-constexpr int kRowChunks = 16;  // chunks of 8 elements per lane held in registers
+constexpr int kRowChunks = 16;                  // 16-byte chunks per lane for a 4096-element row
+constexpr int kRowSlot = 32 * kRowChunks * 16;  // bytes of one shared-memory row slot (8 KiB)
+constexpr int kRowDepth = 3;                    // rows in flight per warp
+constexpr int kRowWarps = kThreads / 32;
+constexpr int kRowBarBytes = 1024;              // mbarrier area at the start of shared memory
+constexpr size_t kRowRingBytes = (size_t)kRowWarps * kRowDepth * kRowSlot;
 
 template <int LAYOUT>
 struct RowUnits {
@@ -51,7 +58,7 @@ __device__ __forceinline__ void store_scale_group(const qz_expert& E, int64_t ro
     }
 }
 
-// Quantize the 16 chunks of pass i held in v (chunk index c = lane + 32 i + c0).
+// Quantize the 32 chunks c0 .. c0+31 of a row (this lane's chunk c = c0 + lane, in v).
 template <int LAYOUT>
 __device__ __forceinline__ void row_pass(const qz_expert& E, int64_t row, int64_t c, int64_t nch, int64_t kv,
                                          uint4 v, float S, int lane) {
@@ -64,73 +71,145 @@ __device__ __forceinline__ void row_pass(const qz_expert& E, int64_t row, int64_
     const uint32_t s1 = __shfl_down_sync(0xFFFFFFFFu, blk.scale, 2);
     const uint32_t s2 = __shfl_down_sync(0xFFFFFFFFu, blk.scale, 4);
     const uint32_t s3 = __shfl_down_sync(0xFFFFFFFFu, blk.scale, 6);
-    if ((lane & 7) == 0) {
-        const int64_t k0 = c >> 1;
-        store_scale_group<LAYOUT>(E, row, k0, kv, blk.scale | (s1 << 8) | (s2 << 16) | (s3 << 24));
+    if ((lane & 7) == 0) store_scale_group<LAYOUT>(E, row, c >> 1, kv, blk.scale | (s1 << 8) | (s2 << 16) | (s3 << 24));
+}
+
+// A row of at most 4096 elements whose chunks are in v (zeros past the row).
+template <int LAYOUT>
+__device__ __forceinline__ void row_from_regs(const qz_expert& E, int64_t row, const uint4 (&v)[kRowChunks], int lane) {
+    const int64_t nch = E.cols >> 3, kv = E.cols >> 4, nsc = 2 * pad_to(kv, 4);
+    uint32_t m = 0;
+#pragma unroll
+    for (int i = 0; i < kRowChunks; ++i) m = max(m, absmax_bits(v[i]));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+    const float A = bits_to_float_bf16(m);
+    if (lane == 0) E.amax[row] = A;
+    const float S = nvfp4_encode_scale(A);
+#pragma unroll
+    for (int i = 0; i < kRowChunks; ++i) {
+        const int64_t c0 = 32 * i;
+        if (c0 < nsc) row_pass<LAYOUT>(E, row, c0 + lane, nch, kv, v[i], S, lane);
     }
+}
+
+// A row of any length straight from global memory: amax pass, then a
+// quantize pass re-reading the row (served by L2).
+template <int LAYOUT>
+__device__ __forceinline__ void row_two_pass(const qz_expert& E, int64_t row, int lane) {
+    const int64_t nch = E.cols >> 3, kv = E.cols >> 4, nsc = 2 * pad_to(kv, 4);
+    const uint16_t* xr = static_cast<const uint16_t*>(E.x) + row * E.ld;
+    uint32_t m = 0;
+    for (int64_t c = lane; c < nch; c += 32) m = max(m, absmax_bits(ld_stream(xr + c * 8)));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+    const float A = bits_to_float_bf16(m);
+    if (lane == 0) E.amax[row] = A;
+    const float S = nvfp4_encode_scale(A);
+    for (int64_t c0 = 0; c0 < nsc; c0 += 32) {
+        const int64_t c = c0 + lane;
+        const uint4 v = (c < nch) ? ld_stream(xr + c * 8) : make_uint4(0, 0, 0, 0);
+        row_pass<LAYOUT>(E, row, c, nch, kv, v, S, lane);
+    }
+}
+
+// Zero scale bytes of a padded row of the swizzled region.
+__device__ __forceinline__ void row_zero_scales(const qz_expert& E, int64_t row, int lane) {
+    const int64_t kv = E.cols >> 4;
+    for (int64_t k0 = 4 * lane; k0 < pad_to(kv, 4); k0 += 128) st_u32(E.sf + swz_offset(row, k0, kv), 0u);
+}
+
+struct RowRef {
+    qz_expert E;
+    int64_t row;
+};
+
+__device__ __forceinline__ RowRef row_ref(const qz_expert* table, const int* s_prefix, int n, int u) {
+    const int e = find_owner(s_prefix, n, u);
+    RowRef r;
+    r.E = load_entry(table, e);
+    r.row = u - s_prefix[e];
+    return r;
 }
 
 template <int LAYOUT>
-__global__ void __launch_bounds__(kThreads) nvfp4_rows_kernel(const qz_expert* __restrict__ table, int n,
-                                                              unsigned* d_err) {
-    extern __shared__ int s_prefix[];
+__global__ void __launch_bounds__(kThreads, 1) nvfp4_rows_kernel(const qz_expert* __restrict__ table, int n,
+                                                                 unsigned* d_err) {
+    extern __shared__ __align__(128) uint8_t smem[];
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem);
+    uint8_t* ring = smem + kRowBarBytes;
+    int* s_prefix = reinterpret_cast<int*>(ring + kRowRingBytes);
     __shared__ long long s_scan[33];
-    const int total = block_prefix(n, s_prefix, s_scan, RowUnits<LAYOUT>{table, d_err}, d_err);
-    const int lane = threadIdx.x & 31;
-    const int warps = kThreads / 32;
-    for (int u = blockIdx.x * warps + (threadIdx.x >> 5); u < total; u += gridDim.x * warps) {
-        const int e = find_owner(s_prefix, n, u);
-        const qz_expert E = load_entry(table, e);
-        const int64_t row = u - s_prefix[e];
-        const int64_t nch = E.cols >> 3;   // 16-byte chunks in the row
-        const int64_t kv = E.cols >> 4;    // scale columns
-        const int64_t nsc = 2 * pad_to(kv, 4);  // chunks whose scale bytes exist (incl. padding)
-        if (row >= E.rows) {
-            // padded row of the swizzled region: zero scale bytes only
-            for (int64_t k0 = 4 * lane; k0 < pad_to(kv, 4); k0 += 128) st_u32(E.sf + swz_offset(row, k0, kv), 0u);
-            continue;
+    if (threadIdx.x < kRowWarps * kRowDepth) mbar_init(&bars[threadIdx.x], 1);
+    mbar_init_fence();
+    const int total = block_prefix(n, s_prefix, s_scan, RowUnits<LAYOUT>{table, d_err}, d_err);  // has barriers
+    const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int stride = gridDim.x * kRowWarps;
+    const int first = blockIdx.x * kRowWarps + w;
+    uint8_t* slots = ring + (size_t)w * kRowDepth * kRowSlot;
+    uint64_t* my_bars = bars + w * kRowDepth;
+    unsigned issued = 0, phase = 0;  // per-slot bits, identical in every lane
+
+    // start the copy of unit u into slot s when it is a live row that fits a slot
+    auto issue = [&](long long u, int s) {
+        issued &= ~(1u << s);
+        if (u >= total) return;
+        const RowRef r = row_ref(table, s_prefix, n, (int)u);
+        const uint32_t bytes = (uint32_t)(r.E.cols * 2);
+        if (r.row >= r.E.rows || bytes > (uint32_t)kRowSlot) return;
+        if (lane == 0) {
+            fence_proxy_async_smem();
+            mbar_arrive_expect_tx(&my_bars[s], bytes);
+            bulk_load(slots + s * kRowSlot, static_cast<const uint16_t*>(r.E.x) + r.row * r.E.ld, bytes, &my_bars[s]);
         }
-        const uint16_t* xr = static_cast<const uint16_t*>(E.x) + row * E.ld;
-        if (nsc <= 32 * kRowChunks) {
+        issued |= 1u << s;
+    };
+
+#pragma unroll
+    for (int s = 0; s < kRowDepth; ++s) issue((long long)first + (long long)s * stride, s);
+
+    for (int i = 0;; ++i) {
+        const long long u = (long long)first + (long long)i * stride;
+        if (u >= total) break;
+        const int s = i % kRowDepth;
+        const RowRef r = row_ref(table, s_prefix, n, (int)u);
+        if (r.row >= r.E.rows) {
+            row_zero_scales(r.E, r.row, lane);
+        } else if ((issued >> s) & 1u) {
+            if (!mbar_wait_bounded(&my_bars[s], (phase >> s) & 1u)) {
+                if (lane == 0 && d_err) atomicOr(d_err, QZ_DERR_TIMEOUT);
+                break;
+            }
+            phase ^= 1u << s;
+            const uint8_t* slot = slots + s * kRowSlot;
+            const int64_t nch = r.E.cols >> 3;
             uint4 v[kRowChunks];
 #pragma unroll
-            for (int i = 0; i < kRowChunks; ++i) {
-                const int64_t c = lane + 32 * i;
-                v[i] = (c < nch) ? ld_stream(xr + c * 8) : make_uint4(0, 0, 0, 0);
+            for (int k = 0; k < kRowChunks; ++k) {
+                const int64_t c = lane + 32 * k;
+                v[k] = (c < nch) ? lds128(slot + c * 16) : make_uint4(0, 0, 0, 0);
             }
-            uint32_t m = 0;
-#pragma unroll
-            for (int i = 0; i < kRowChunks; ++i) m = max(m, absmax_bits(v[i]));
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
-            const float A = bits_to_float_bf16(m);
-            if (lane == 0) E.amax[row] = A;
-            const float S = nvfp4_encode_scale(A);
-#pragma unroll
-            for (int i = 0; i < kRowChunks; ++i) {
-                const int64_t c0 = 32 * i;
-                if (c0 < nsc) row_pass<LAYOUT>(E, row, c0 + lane, nch, kv, v[i], S, lane);
-            }
+            row_from_regs<LAYOUT>(r.E, r.row, v, lane);
         } else {
-            // long row: amax pass, then a quantize pass re-reading the row
-            uint32_t m = 0;
-            for (int64_t c = lane; c < nch; c += 32) m = max(m, absmax_bits(ld_stream(xr + c * 8)));
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
-            const float A = bits_to_float_bf16(m);
-            if (lane == 0) E.amax[row] = A;
-            const float S = nvfp4_encode_scale(A);
-            for (int64_t c0 = 0; c0 < nsc; c0 += 32) {
-                const int64_t c = c0 + lane;
-                const uint4 v = (c < nch) ? ld_stream(xr + c * 8) : make_uint4(0, 0, 0, 0);
-                row_pass<LAYOUT>(E, row, c, nch, kv, v, S, lane);
-            }
+            row_two_pass<LAYOUT>(r.E, r.row, lane);
         }
+        __syncwarp();  // every lane is done with slot s before it is refilled
+        issue(u + (long long)kRowDepth * stride, s);
     }
+    // drain: copies still in flight (units past a timeout) complete before exit
+#pragma unroll
+    for (int s = 0; s < kRowDepth; ++s)
+        if ((issued >> s) & 1u) {
+            if (!mbar_wait_bounded(&my_bars[s], (phase >> s) & 1u) && lane == 0 && d_err) atomicOr(d_err, QZ_DERR_TIMEOUT);
+            phase ^= 1u << s;
+            issued &= ~(1u << s);
+        }
 }
 
+size_t rows_smem_bytes(int n) { return kRowBarBytes + kRowRingBytes + (size_t)(n + 1) * sizeof(int); }
+
 cudaError_t launch_nvfp4_rows(const qz_expert* table, int n, int layout, int grid, cudaStream_t s, unsigned* d_err) {
-    const size_t smem = (size_t)(n + 1) * sizeof(int);
+    const size_t smem = rows_smem_bytes(n);
     if (layout == QZ_SF_SWIZZLED_128x4)
         nvfp4_rows_kernel<QZ_SF_SWIZZLED_128x4><<<grid, kThreads, smem, s>>>(table, n, d_err);
     else
@@ -138,10 +217,14 @@ cudaError_t launch_nvfp4_rows(const qz_expert* table, int n, int layout, int gri
     return cudaGetLastError();
 }
 
+// Opt the row kernels into their shared-memory size; returns resident CTAs per SM.
 int rows_blocks_per_sm(int n) {
+    const size_t smem = rows_smem_bytes(QZ_MAX_EXPERTS);
+    cudaFuncSetAttribute(nvfp4_rows_kernel<QZ_SF_SWIZZLED_128x4>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaFuncSetAttribute(nvfp4_rows_kernel<QZ_SF_LINEAR>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     int b = 1;
     cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, nvfp4_rows_kernel<QZ_SF_SWIZZLED_128x4>, kThreads,
-                                                  (size_t)(n + 1) * sizeof(int));
+                                                  rows_smem_bytes(n));
     return b > 0 ? b : 1;
 }
 
