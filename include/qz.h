@@ -80,7 +80,8 @@ typedef enum qz_nvfp4_scale_mode {
 } qz_nvfp4_scale_mode;
 
 /* Reason bits OR-ed into *opts->d_err for table entries a kernel skipped. */
-#define QZ_DERR_SHAPE 0x1u     /* rows < 0, cols <= 0, cols not a multiple of the block, ld < cols */
+#define QZ_DERR_SHAPE 0x1u     /* rows < 0, cols <= 0, cols not a multiple of the block,
+                                  ld < cols or ld > QZ_MAX_LD */
 #define QZ_DERR_NULL 0x2u      /* x, q, sf (or amax for NVFP4) null on a non-empty entry */
 #define QZ_DERR_ALIGN 0x4u     /* x not 16-byte aligned or ld not a multiple of 8; q not
                                   8-byte (MXFP8) / 4-byte (NVFP4) aligned; sf not 16-byte
@@ -93,6 +94,10 @@ typedef enum qz_nvfp4_scale_mode {
  * sums in shared memory). */
 #define QZ_MAX_EXPERTS 4096
 
+/* Largest row stride (elements) of a table entry: offsets inside a 128-row
+ * tile are 32-bit. */
+#define QZ_MAX_LD (1LL << 24)
+
 /* Largest hidden size of qz_rmsnorm_quantize (one row is held in registers). */
 #define QZ_MAX_HIDDEN 16384
 
@@ -104,7 +109,7 @@ typedef struct qz_expert {
                       activation: base + row_offset * ld. */
     int64_t rows;  /* may be 0 (an empty split): nothing is read or written */
     int64_t cols;  /* quantization axis; multiple of 32 (MXFP8) or 16 (NVFP4) */
-    int64_t ld;    /* row stride of x in elements, >= cols, multiple of 8 */
+    int64_t ld;    /* row stride of x in elements, >= cols, <= QZ_MAX_LD, multiple of 8 */
     void *q;       /* payload, row-major and dense: MXFP8 e4m3 [rows, cols];
                       NVFP4 e2m1 [rows, cols/2], element 2j in the low nibble
                       of byte j and element 2j+1 in the high nibble */

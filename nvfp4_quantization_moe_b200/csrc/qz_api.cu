@@ -18,7 +18,7 @@ cudaError_t launch_nvfp4_rows(const qz_expert* table, int n, int layout, int gri
 cudaError_t launch_swizzle(const qz_sf_pair* table, int n, int grid, cudaStream_t s, unsigned* d_err);
 cudaError_t launch_rmsnorm_quant(const uint16_t* x, const uint16_t* r, const uint16_t* g, float eps, int64_t T,
                                  int64_t H, uint16_t* y, uint16_t* h, int fmt, uint8_t* q, uint8_t* sf, int layout,
-                                 const float* amax, cudaStream_t s);
+                                 const float* amax, cudaStream_t s, bool latency_mode);
 int grouped_blocks_per_sm(int which, int n);
 int rows_blocks_per_sm(int n);
 }  // namespace qz
@@ -58,6 +58,20 @@ int wave_grid(int kind, const qz_launch_opts* opts) {
     }
     if (opts && opts->max_ctas > 0 && opts->max_ctas < grid) grid = opts->max_ctas;
     return grid;
+}
+
+// SM count of the current device (cached).
+int device_sms() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
+    std::lock_guard<std::mutex> lock(g_mu);
+    DeviceLimits& d = g_dev[dev];
+    if (d.sms == 0) {
+        int sms = 0;
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        d.sms = sms > 0 ? sms : 1;
+    }
+    return d.sms;
 }
 
 bool aligned(const void* p, uintptr_t a) { return ((uintptr_t)p & (a - 1)) == 0; }
@@ -130,11 +144,12 @@ qz_status qz_rmsnorm_quantize(const void* d_x, const void* d_residual, const voi
         return QZ_ERR_ALIGNMENT;
     if (!aligned(d_q, 8) || !aligned(d_sf, layout == QZ_SF_SWIZZLED_128x4 ? 16 : 4)) return QZ_ERR_ALIGNMENT;
     if (d_global_amax && !aligned(d_global_amax, 4)) return QZ_ERR_ALIGNMENT;
+    const bool latency_mode = T <= 2 * (int64_t)device_sms();
     return from_cuda(qz::launch_rmsnorm_quant(
         static_cast<const uint16_t*>(d_x), static_cast<const uint16_t*>(d_residual),
         static_cast<const uint16_t*>(d_gamma), eps, T, H, static_cast<uint16_t*>(d_norm_out),
         static_cast<uint16_t*>(d_residual_out), fmt, static_cast<uint8_t*>(d_q), d_sf, layout, d_global_amax,
-        (cudaStream_t)stream));
+        (cudaStream_t)stream, latency_mode));
 }
 
 qz_status qz_swizzle_scales(const qz_sf_pair* d_table, int n, void* stream, const qz_launch_opts* opts) {

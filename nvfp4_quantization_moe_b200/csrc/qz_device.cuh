@@ -146,10 +146,25 @@ struct Nvfp4Block {
     float rcp;       // multiplier applied to each element
 };
 
+// RN(b / 6) for a bf16 magnitude b (8 significant bits), by the quotient
+// correction of Markstein (IBM J. Res. Dev. 34(1), 1990): q0 = RN(b * RN(1/6)),
+// r = b - 6 q0 exactly (one FMA), q = RN(q0 + r * RN(1/6)).  The correction
+// is exact unless b/6 lies within a tiny fraction of an ulp of a rounding
+// midpoint; b/6 with an 8-bit b is either exact or has the periodic binary
+// expansion ...0101..., a third of an ulp or more from any midpoint, so q is
+// the correctly rounded quotient for every bf16 b (checked exhaustively
+// against IEEE division in the test suite).
+__device__ __forceinline__ float div6_rn(float b) {
+    const float c = 1.0f / 6.0f;
+    const float q0 = __fmul_rn(b, c);
+    const float r = __fmaf_rn(-q0, 6.0f, b);
+    return __fmaf_rn(r, c, q0);
+}
+
 // Block scale and element multiplier for a block of largest magnitude b.
 __device__ __forceinline__ Nvfp4Block nvfp4_block(float b, float S) {
     Nvfp4Block r;
-    r.scale = (b == 0.0f) ? 0u : e4m3_of(__fmul_rn(__fdiv_rn(b, 6.0f), S));
+    r.scale = (b == 0.0f) ? 0u : e4m3_of(__fmul_rn(div6_rn(b), S));
     r.rcp = 0.0f;
     if (r.scale != 0u) {
         float q = __fdiv_rn(S, e4m3_value(r.scale));
@@ -185,7 +200,7 @@ __device__ __forceinline__ bool aligned(const void* p, uintptr_t a) { return ((u
 __device__ __forceinline__ unsigned entry_errors(const qz_expert& e, int fmt, int layout, bool needs_amax) {
     const int64_t block = (fmt == QZ_FMT_MXFP8) ? 32 : 16;
     unsigned bad = 0;
-    if (e.rows < 0 || e.cols <= 0 || (e.cols % block) != 0 || e.ld < e.cols) bad |= QZ_DERR_SHAPE;
+    if (e.rows < 0 || e.cols <= 0 || (e.cols % block) != 0 || e.ld < e.cols || e.ld > QZ_MAX_LD) bad |= QZ_DERR_SHAPE;
     if (e.rows > 0) {
         if (!e.x || !e.q || !e.sf || (needs_amax && !e.amax)) bad |= QZ_DERR_NULL;
         if (!aligned(e.x, 16) || (e.ld & 7) != 0) bad |= QZ_DERR_ALIGN;

@@ -54,52 +54,66 @@ struct TableTiles {
 // in flight.
 // ---------------------------------------------------------------------------
 
+// One thread's view of a tile: pointers to its first row (tile row r0 =
+// 4w + lane/16) at its chunk's column; pass p adds kPassRow[p] rows, so the
+// per-pass address and bounds arithmetic is 32-bit.
 struct TileRef {
-    const uint16_t* x;
-    int64_t rows, cols, ld;
-    uint8_t* q;
-    uint8_t* sf;
+    const uint16_t* xp;  // x of (rt*128 + r0, ct*128 + chunk*8)
+    uint8_t* qp;         // payload byte of the same element
+    uint8_t* sfp;        // linear SF byte of (rt*128 + r0, block of the chunk); swizzled: region base
     const float* amax;
-    int64_t rt, ct;
+    int ld;              // x row stride, elements
+    int qld;             // payload row bytes
+    int kv;              // scale columns
+    int rows_left;       // pass p is live iff kPassRow[p] < rows_left (and col_ok)
+    bool col_ok;
+    int rt, ct;
     int expert;
 };
 
-__device__ __forceinline__ TileRef tile_ref(const qz_expert* table, const int* s_prefix, int n, int tile) {
+__device__ __forceinline__ constexpr int pass_row(int p) { return (p & 3) * 32 + 2 * (p >> 2); }
+
+template <int FMT, int LAYOUT>
+__device__ __forceinline__ TileRef tile_ref(const qz_expert* table, const int* s_prefix, int n, int tile, int w,
+                                            int lane) {
     const int e = find_owner(s_prefix, n, tile);
     const qz_expert E = load_entry(table, e);
-    const int64_t local = tile - s_prefix[e];
-    const int64_t nct = (E.cols + kTileCols - 1) / kTileCols;
+    const int local = tile - s_prefix[e];
+    const int nct = (int)((E.cols + kTileCols - 1) / kTileCols);
     TileRef t;
-    t.x = static_cast<const uint16_t*>(E.x);
-    t.rows = E.rows;
-    t.cols = E.cols;
-    t.ld = E.ld;
-    t.q = static_cast<uint8_t*>(E.q);
-    t.sf = E.sf;
-    t.amax = E.amax;
     t.rt = local / nct;
-    t.ct = local % nct;
+    t.ct = local - t.rt * nct;
+    const int chunk = lane & 15;
+    const int r0 = 4 * w + (lane >> 4);
+    const int64_t row0 = (int64_t)t.rt * kTileRows + r0;
+    const int64_t col = (int64_t)t.ct * kTileCols + chunk * 8;
+    t.ld = (int)E.ld;
+    t.qld = (int)(FMT == QZ_FMT_MXFP8 ? E.cols : E.cols >> 1);
+    t.kv = (int)(FMT == QZ_FMT_MXFP8 ? E.cols >> 5 : E.cols >> 4);
+    t.xp = static_cast<const uint16_t*>(E.x) + row0 * E.ld + col;
+    t.qp = static_cast<uint8_t*>(E.q) + row0 * t.qld + (FMT == QZ_FMT_MXFP8 ? col : col >> 1);
+    t.sfp = LAYOUT == QZ_SF_SWIZZLED_128x4 ? E.sf : E.sf + row0 * t.kv + (FMT == QZ_FMT_MXFP8 ? col >> 5 : col >> 4);
+    t.amax = E.amax;
+    const int64_t left = E.rows - row0;
+    t.rows_left = left > kTileRows ? kTileRows : (int)left;
+    t.col_ok = col < E.cols;
     t.expert = e;
     return t;
 }
 
-__device__ __forceinline__ int tile_row(int p, int w, int lane) { return (p & 3) * 32 + 4 * w + 2 * (p >> 2) + (lane >> 4); }
-
-__device__ __forceinline__ uint4 tile_load(const TileRef& t, int p, int w, int lane) {
-    const int64_t row = t.rt * kTileRows + tile_row(p, w, lane);
-    const int64_t col = t.ct * kTileCols + (lane & 15) * 8;
-    return (row < t.rows && col < t.cols) ? ld_stream(t.x + row * t.ld + col) : make_uint4(0, 0, 0, 0);
+__device__ __forceinline__ uint4 tile_load(const TileRef& t, int p) {
+    const int pr = pass_row(p);
+    return (t.col_ok && pr < t.rows_left) ? ld_stream(t.xp + pr * t.ld) : make_uint4(0, 0, 0, 0);
 }
 
 // Quantize pass p of tile t (8 elements per thread in v).  MXFP8 blocks span
 // 4 lanes, NVFP4 blocks 2.  Swizzled scale bytes go to the warp's staging
 // area s (64 bytes per 4-column scale tile), linear ones straight to memory.
 template <int FMT, int LAYOUT>
-__device__ __forceinline__ void tile_pass(const TileRef& t, int p, int w, int lane, uint4 v, float S, uint8_t* s) {
+__device__ __forceinline__ void tile_pass(const TileRef& t, int p, int lane, uint4 v, float S, uint8_t* s) {
     const int chunk = lane & 15;
-    const int64_t row = t.rt * kTileRows + tile_row(p, w, lane);
-    const int64_t col = t.ct * kTileCols + chunk * 8;
-    const bool live = row < t.rows && col < t.cols;
+    const int pr = pass_row(p);
+    const bool live = t.col_ok && pr < t.rows_left;
     const int stage = (2 * (p >> 2) + (lane >> 4)) * 16 + (p & 3) * 4;  // byte of this row in the warp's chunks
     uint32_t m = absmax_bits(v);
     m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
@@ -107,20 +121,19 @@ __device__ __forceinline__ void tile_pass(const TileRef& t, int p, int w, int la
         m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
         const uint32_t byte = e8m0_byte(m);
         const uint2 codes = e4m3x8_scaled(v, e8m0_reciprocal(byte));
-        if (live) st_v2(t.q + row * t.cols + col, codes.x, codes.y);
+        if (live) st_v2(t.qp + pr * t.qld, codes.x, codes.y);
         if ((chunk & 3) == 0) {
-            const int kc = chunk >> 2;
-            if (LAYOUT == QZ_SF_SWIZZLED_128x4) s[stage + kc] = live ? (uint8_t)byte : (uint8_t)0;
-            else if (live) t.sf[row * (t.cols >> 5) + t.ct * 4 + kc] = (uint8_t)byte;
+            if (LAYOUT == QZ_SF_SWIZZLED_128x4) s[stage + (chunk >> 2)] = live ? (uint8_t)byte : (uint8_t)0;
+            else if (live) t.sfp[pr * t.kv] = (uint8_t)byte;
         }
     } else {
         const Nvfp4Block blk = nvfp4_block(bits_to_float_bf16(m), S);
         const uint32_t codes = e2m1x8_scaled(v, blk.rcp);
-        if (live) st_u32(t.q + row * (t.cols >> 1) + (col >> 1), codes);
+        if (live) st_u32(t.qp + pr * t.qld, codes);
         if ((chunk & 1) == 0) {
             const int kk = chunk >> 1;  // 0..7: two 4-column scale tiles per tile
             if (LAYOUT == QZ_SF_SWIZZLED_128x4) s[(kk >> 2) * 64 + stage + (kk & 3)] = live ? (uint8_t)blk.scale : (uint8_t)0;
-            else if (live) t.sf[row * (t.cols >> 4) + t.ct * 8 + kk] = (uint8_t)blk.scale;
+            else if (live) t.sfp[pr * t.kv] = (uint8_t)blk.scale;
         }
     }
 }
@@ -129,14 +142,13 @@ __device__ __forceinline__ void tile_pass(const TileRef& t, int p, int w, int la
 template <int FMT>
 __device__ __forceinline__ void tile_flush_sf(const TileRef& t, int w, int lane, const uint8_t* s) {
     __syncwarp();
-    const int64_t kv = FMT == QZ_FMT_MXFP8 ? (t.cols >> 5) : (t.cols >> 4);
-    const int64_t col_tiles = (kv + 3) >> 2;
+    const int col_tiles = (t.kv + 3) >> 2;
     constexpr int kTilesPerTile = FMT == QZ_FMT_MXFP8 ? 1 : 2;
     if (lane < 4 * kTilesPerTile) {
         const int j = lane >> 2, c = lane & 3;
-        const int64_t ctile = t.ct * kTilesPerTile + j;
+        const int ctile = t.ct * kTilesPerTile + j;
         if (ctile < col_tiles)
-            st_v4(t.sf + ((t.rt * col_tiles + ctile) << 9) + (4 * w + c) * 16,
+            st_v4(t.sfp + (((int64_t)t.rt * col_tiles + ctile) << 9) + (4 * w + c) * 16,
                   *reinterpret_cast<const uint4*>(s + j * 64 + c * 16));
     }
     __syncwarp();
@@ -154,19 +166,19 @@ __global__ void __launch_bounds__(kThreads, 3) grouped_tile_kernel(const qz_expe
     const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
     int tile = blockIdx.x;
     if (tile >= total) return;
-    TileRef cur = tile_ref(table, s_prefix, n, tile);
+    TileRef cur = tile_ref<FMT, LAYOUT>(table, s_prefix, n, tile, w, lane);
     uint4 v[8];
 #pragma unroll
-    for (int p = 0; p < 8; ++p) v[p] = tile_load(cur, p, w, lane);
+    for (int p = 0; p < 8; ++p) v[p] = tile_load(cur, p);
     for (;;) {
         const int next = tile + gridDim.x;
         const bool more = next < total;
-        const TileRef nxt = more ? tile_ref(table, s_prefix, n, next) : cur;
+        const TileRef nxt = more ? tile_ref<FMT, LAYOUT>(table, s_prefix, n, next, w, lane) : cur;
         const float S = kAmax ? nvfp4_encode_scale(*cur.amax) : 0.0f;
 #pragma unroll
         for (int p = 0; p < 8; ++p) {
-            tile_pass<FMT, LAYOUT>(cur, p, w, lane, v[p], S, s_sf[w]);
-            if (more) v[p] = tile_load(nxt, p, w, lane);
+            tile_pass<FMT, LAYOUT>(cur, p, lane, v[p], S, s_sf[w]);
+            if (more) v[p] = tile_load(nxt, p);
         }
         if (LAYOUT == QZ_SF_SWIZZLED_128x4) tile_flush_sf<FMT>(cur, w, lane, s_sf[w]);
         if (!more) break;
@@ -199,19 +211,19 @@ __global__ void __launch_bounds__(kThreads) amax_grouped_kernel(const qz_expert*
     const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
     int tile = blockIdx.x;
     if (tile >= total) return;
-    TileRef cur = tile_ref(table, s_prefix, n, tile);
+    TileRef cur = tile_ref<QZ_FMT_NVFP4, LAYOUT>(table, s_prefix, n, tile, w, lane);
     uint4 v[8];
 #pragma unroll
-    for (int p = 0; p < 8; ++p) v[p] = tile_load(cur, p, w, lane);
+    for (int p = 0; p < 8; ++p) v[p] = tile_load(cur, p);
     uint32_t run = 0;
     for (;;) {
         const int next = tile + gridDim.x;
         const bool more = next < total;
-        const TileRef nxt = more ? tile_ref(table, s_prefix, n, next) : cur;
+        const TileRef nxt = more ? tile_ref<QZ_FMT_NVFP4, LAYOUT>(table, s_prefix, n, next, w, lane) : cur;
 #pragma unroll
         for (int p = 0; p < 8; ++p) {
             run = max(run, absmax_bits(v[p]));
-            if (more) v[p] = tile_load(nxt, p, w, lane);
+            if (more) v[p] = tile_load(nxt, p);
         }
         if (!more || nxt.expert != cur.expert) {
 #pragma unroll

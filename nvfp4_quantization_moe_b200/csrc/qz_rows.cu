@@ -6,13 +6,15 @@
 // swizzled padding is independent per expert (uneven and empty splits).
 //
 // One warp per row.  Rows of up to 4096 elements are brought into shared
-// memory by one bulk (TMA) copy each: every warp keeps kRowDepth rows in
-// flight in its own ring of shared-memory slots, each slot with an mbarrier
-// that the copy completes, so HBM streams while the warp quantizes.  From the
-// slot a lane takes chunks l + 32i (8 bf16 each): the two chunks of a
-// 16-element block sit in lanes (2j, 2j+1) and the four blocks of one 4-byte
-// scale group in eight consecutive lanes, so a scale group leaves as one
-// 32-bit store.  Longer rows take a two-pass path straight from global memory.
+// memory by one bulk (TMA) copy each: each of the 12 warps of a CTA keeps
+// kRowDepth rows in flight in its own ring of shared-memory slots, each slot
+// with an mbarrier that the copy completes, so HBM streams while the warp
+// quantizes.  The warp reads the slot twice (row amax, then quantization), so
+// few registers are live and many warps fit on an SM.  A lane takes chunks
+// l + 32i (8 bf16 each): the two chunks of a 16-element block sit in lanes
+// (2j, 2j+1) and the four blocks of one 4-byte scale group in eight
+// consecutive lanes, so a scale group leaves as one 32-bit store.  Longer
+// rows take a two-pass path straight from global memory.
 //
 // Units of work are "virtual rows": an expert owns rows (linear layout) or
 // pad(rows, 128) virtual rows (swizzled); a virtual row past the last live row
@@ -24,8 +26,9 @@ namespace qz {
 
 constexpr int kRowChunks = 16;                  // 16-byte chunks per lane for a 4096-element row
 constexpr int kRowSlot = 32 * kRowChunks * 16;  // bytes of one shared-memory row slot (8 KiB)
-constexpr int kRowDepth = 3;                    // rows in flight per warp
-constexpr int kRowWarps = kThreads / 32;
+constexpr int kRowDepth = 2;                    // rows in flight per warp
+constexpr int kRowWarps = 12;                   // warps per CTA
+constexpr int kRowThreads = 32 * kRowWarps;
 constexpr int kRowBarBytes = 1024;              // mbarrier area at the start of shared memory
 constexpr size_t kRowRingBytes = (size_t)kRowWarps * kRowDepth * kRowSlot;
 
@@ -74,22 +77,25 @@ __device__ __forceinline__ void row_pass(const qz_expert& E, int64_t row, int64_
     if ((lane & 7) == 0) store_scale_group<LAYOUT>(E, row, c >> 1, kv, blk.scale | (s1 << 8) | (s2 << 16) | (s3 << 24));
 }
 
-// A row of at most 4096 elements whose chunks are in v (zeros past the row).
+// A row of at most 4096 elements staged in shared memory: amax pass, then a
+// quantize pass over the same slot.
 template <int LAYOUT>
-__device__ __forceinline__ void row_from_regs(const qz_expert& E, int64_t row, const uint4 (&v)[kRowChunks], int lane) {
-    const int64_t nch = E.cols >> 3, kv = E.cols >> 4, nsc = 2 * pad_to(kv, 4);
+__device__ __forceinline__ void row_from_slot(const qz_expert& E, int64_t row, const uint8_t* slot, int lane) {
+    const int64_t nch = E.cols >> 3, kv = E.cols >> 4;
+    const int nsc = 2 * (int)pad_to(kv, 4);
     uint32_t m = 0;
-#pragma unroll
-    for (int i = 0; i < kRowChunks; ++i) m = max(m, absmax_bits(v[i]));
+#pragma unroll 4
+    for (int c = lane; c < nch; c += 32) m = max(m, absmax_bits(lds128(slot + c * 16)));
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
     const float A = bits_to_float_bf16(m);
     if (lane == 0) E.amax[row] = A;
     const float S = nvfp4_encode_scale(A);
-#pragma unroll
-    for (int i = 0; i < kRowChunks; ++i) {
-        const int64_t c0 = 32 * i;
-        if (c0 < nsc) row_pass<LAYOUT>(E, row, c0 + lane, nch, kv, v[i], S, lane);
+#pragma unroll 2
+    for (int c0 = 0; c0 < nsc; c0 += 32) {
+        const int c = c0 + lane;
+        const uint4 v = (c < nch) ? lds128(slot + c * 16) : make_uint4(0, 0, 0, 0);
+        row_pass<LAYOUT>(E, row, c, nch, kv, v, S, lane);
     }
 }
 
@@ -133,7 +139,7 @@ __device__ __forceinline__ RowRef row_ref(const qz_expert* table, const int* s_p
 }
 
 template <int LAYOUT>
-__global__ void __launch_bounds__(kThreads, 1) nvfp4_rows_kernel(const qz_expert* __restrict__ table, int n,
+__global__ void __launch_bounds__(kRowThreads, 1) nvfp4_rows_kernel(const qz_expert* __restrict__ table, int n,
                                                                  unsigned* d_err) {
     extern __shared__ __align__(128) uint8_t smem[];
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem);
@@ -181,15 +187,7 @@ __global__ void __launch_bounds__(kThreads, 1) nvfp4_rows_kernel(const qz_expert
                 break;
             }
             phase ^= 1u << s;
-            const uint8_t* slot = slots + s * kRowSlot;
-            const int64_t nch = r.E.cols >> 3;
-            uint4 v[kRowChunks];
-#pragma unroll
-            for (int k = 0; k < kRowChunks; ++k) {
-                const int64_t c = lane + 32 * k;
-                v[k] = (c < nch) ? lds128(slot + c * 16) : make_uint4(0, 0, 0, 0);
-            }
-            row_from_regs<LAYOUT>(r.E, r.row, v, lane);
+            row_from_slot<LAYOUT>(r.E, r.row, slots + s * kRowSlot, lane);
         } else {
             row_two_pass<LAYOUT>(r.E, r.row, lane);
         }
@@ -211,9 +209,9 @@ size_t rows_smem_bytes(int n) { return kRowBarBytes + kRowRingBytes + (size_t)(n
 cudaError_t launch_nvfp4_rows(const qz_expert* table, int n, int layout, int grid, cudaStream_t s, unsigned* d_err) {
     const size_t smem = rows_smem_bytes(n);
     if (layout == QZ_SF_SWIZZLED_128x4)
-        nvfp4_rows_kernel<QZ_SF_SWIZZLED_128x4><<<grid, kThreads, smem, s>>>(table, n, d_err);
+        nvfp4_rows_kernel<QZ_SF_SWIZZLED_128x4><<<grid, kRowThreads, smem, s>>>(table, n, d_err);
     else
-        nvfp4_rows_kernel<QZ_SF_LINEAR><<<grid, kThreads, smem, s>>>(table, n, d_err);
+        nvfp4_rows_kernel<QZ_SF_LINEAR><<<grid, kRowThreads, smem, s>>>(table, n, d_err);
     return cudaGetLastError();
 }
 
@@ -223,7 +221,7 @@ int rows_blocks_per_sm(int n) {
     cudaFuncSetAttribute(nvfp4_rows_kernel<QZ_SF_SWIZZLED_128x4>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     cudaFuncSetAttribute(nvfp4_rows_kernel<QZ_SF_LINEAR>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     int b = 1;
-    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, nvfp4_rows_kernel<QZ_SF_SWIZZLED_128x4>, kThreads,
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, nvfp4_rows_kernel<QZ_SF_SWIZZLED_128x4>, kRowThreads,
                                                   rows_smem_bytes(n));
     return b > 0 ? b : 1;
 }
