@@ -141,11 +141,6 @@ __device__ __forceinline__ float nvfp4_encode_scale(float A) {
     return g == 0.0f ? 0.0f : __fdiv_rn(1.0f, g);
 }
 
-struct Nvfp4Block {
-    uint32_t scale;  // e4m3 code of the block scale
-    float rcp;       // multiplier applied to each element
-};
-
 // RN(b / 6) for a bf16 magnitude b (8 significant bits), by the quotient
 // correction of Markstein (IBM J. Res. Dev. 34(1), 1990): q0 = RN(b * RN(1/6)),
 // r = b - 6 q0 exactly (one FMA), q = RN(q0 + r * RN(1/6)).  The correction
@@ -161,13 +156,42 @@ __device__ __forceinline__ float div6_rn(float b) {
     return __fmaf_rn(r, c, q0);
 }
 
+struct Nvfp4Block {
+    uint32_t scale;  // e4m3 code of the block scale
+    float rcp;       // multiplier applied to each element
+};
+
+// RN(1/m) for m = 0..15 (entry 0 unused), filled once per CTA in shared memory.
+__device__ __forceinline__ void fill_inv_table(float* inv) {
+    if (threadIdx.x < 16) inv[threadIdx.x] = threadIdx.x ? __fdiv_rn(1.0f, (float)threadIdx.x) : 0.0f;
+}
+
+// RN(S / value(s)) for a non-zero e4m3 code s < 0x7F, value(s) = m * 2^k.
+// RN(S / m) by Markstein's quotient correction (q0 = RN(S * RN(1/m)),
+// r = S - m q0 exactly, q = RN(q0 + r * RN(1/m))), exact for every binary32 S
+// and m = 1..15 (checked exhaustively over all significands in the test
+// suite); the power of two is then applied exactly.  With bf16 data and a
+// finite encode scale the quotient is never below 2^-126, where the rounding
+// of the two-step form and of a direct division could differ.
+__device__ __forceinline__ float div_by_e4m3(float S, uint32_t s, const float* inv) {
+    const uint32_t ef = s >> 3, mt = s & 7u;
+    const uint32_t m = ef ? 8u + mt : mt;
+    const int k = ef ? (int)ef - 10 : -9;  // value(s) = m * 2^k
+    const float c = inv[m];
+    const float fm = (float)m;
+    const float q0 = __fmul_rn(S, c);
+    const float r = __fmaf_rn(-q0, fm, S);
+    const float q = __fmaf_rn(r, c, q0);
+    return __fmul_rn(q, __uint_as_float((uint32_t)(127 - k) << 23));
+}
+
 // Block scale and element multiplier for a block of largest magnitude b.
-__device__ __forceinline__ Nvfp4Block nvfp4_block(float b, float S) {
+__device__ __forceinline__ Nvfp4Block nvfp4_block(float b, float S, const float* inv) {
     Nvfp4Block r;
     r.scale = (b == 0.0f) ? 0u : e4m3_of(__fmul_rn(div6_rn(b), S));
     r.rcp = 0.0f;
     if (r.scale != 0u) {
-        float q = __fdiv_rn(S, e4m3_value(r.scale));
+        const float q = div_by_e4m3(S, r.scale, inv);
         r.rcp = (q < 0x1p-126f) ? 0.0f : q;  // flush a subnormal reciprocal to zero
     }
     return r;

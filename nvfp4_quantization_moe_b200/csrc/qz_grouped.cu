@@ -110,7 +110,8 @@ __device__ __forceinline__ uint4 tile_load(const TileRef& t, int p) {
 // 4 lanes, NVFP4 blocks 2.  Swizzled scale bytes go to the warp's staging
 // area s (64 bytes per 4-column scale tile), linear ones straight to memory.
 template <int FMT, int LAYOUT>
-__device__ __forceinline__ void tile_pass(const TileRef& t, int p, int lane, uint4 v, float S, uint8_t* s) {
+__device__ __forceinline__ void tile_pass(const TileRef& t, int p, int lane, uint4 v, float S, uint8_t* s,
+                                          const float* inv) {
     const int chunk = lane & 15;
     const int pr = pass_row(p);
     const bool live = t.col_ok && pr < t.rows_left;
@@ -127,7 +128,7 @@ __device__ __forceinline__ void tile_pass(const TileRef& t, int p, int lane, uin
             else if (live) t.sfp[pr * t.kv] = (uint8_t)byte;
         }
     } else {
-        const Nvfp4Block blk = nvfp4_block(bits_to_float_bf16(m), S);
+        const Nvfp4Block blk = nvfp4_block(bits_to_float_bf16(m), S, inv);
         const uint32_t codes = e2m1x8_scaled(v, blk.rcp);
         if (live) st_u32(t.qp + pr * t.qld, codes);
         if ((chunk & 1) == 0) {
@@ -161,7 +162,9 @@ __global__ void __launch_bounds__(kThreads, 3) grouped_tile_kernel(const qz_expe
     __shared__ long long s_scan[33];
     constexpr int kStage = FMT == QZ_FMT_MXFP8 ? 64 : 128;
     __shared__ __align__(16) uint8_t s_sf[kThreads / 32][kStage];
+    __shared__ float s_inv[16];
     constexpr bool kAmax = FMT == QZ_FMT_NVFP4;
+    if (kAmax) fill_inv_table(s_inv);  // published by the barriers in block_prefix
     const int total = block_prefix(n, s_prefix, s_scan, TableTiles<FMT, LAYOUT, kAmax>{table, d_err}, d_err);
     const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
     int tile = blockIdx.x;
@@ -177,7 +180,7 @@ __global__ void __launch_bounds__(kThreads, 3) grouped_tile_kernel(const qz_expe
         const float S = kAmax ? nvfp4_encode_scale(*cur.amax) : 0.0f;
 #pragma unroll
         for (int p = 0; p < 8; ++p) {
-            tile_pass<FMT, LAYOUT>(cur, p, lane, v[p], S, s_sf[w]);
+            tile_pass<FMT, LAYOUT>(cur, p, lane, v[p], S, s_sf[w], s_inv);
             if (more) v[p] = tile_load(nxt, p);
         }
         if (LAYOUT == QZ_SF_SWIZZLED_128x4) tile_flush_sf<FMT>(cur, w, lane, s_sf[w]);

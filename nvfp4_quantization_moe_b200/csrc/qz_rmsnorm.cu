@@ -139,6 +139,8 @@ __global__ void __launch_bounds__(norm_max_threads(CPT)) rmsnorm_quant_kernel(
 
     // CTA reduction of the sum of squares in binary64
     __shared__ double s_red[kNormMaxThreads / 32];
+    __shared__ float s_inv[16];
+    if (FMT == QZ_FMT_NVFP4) fill_inv_table(s_inv);  // published by the barrier below
     double ss = (double)sh + (double)sl;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xFFFFFFFFu, ss, o);
@@ -176,7 +178,7 @@ __global__ void __launch_bounds__(norm_max_threads(CPT)) rmsnorm_quant_kernel(
             const uint2 codes = e4m3x8_scaled(y, e8m0_reciprocal(scale));
             if (c < nch) st_v2(q + row * H + c * 8, codes.x, codes.y);
         } else {
-            const Nvfp4Block blk = nvfp4_block(bits_to_float_bf16(m), S);
+            const Nvfp4Block blk = nvfp4_block(bits_to_float_bf16(m), S, s_inv);
             scale = blk.scale;
             const uint32_t codes = e2m1x8_scaled(y, blk.rcp);
             if (c < nch) st_u32(q + row * (H >> 1) + c * 4, codes);

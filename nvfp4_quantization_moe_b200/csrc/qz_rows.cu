@@ -10,11 +10,11 @@
 // kRowDepth rows in flight in its own ring of shared-memory slots, each slot
 // with an mbarrier that the copy completes, so HBM streams while the warp
 // quantizes.  The warp reads the slot twice (row amax, then quantization), so
-// few registers are live and many warps fit on an SM.  A lane takes chunks
-// l + 32i (8 bf16 each): the two chunks of a 16-element block sit in lanes
-// (2j, 2j+1) and the four blocks of one 4-byte scale group in eight
-// consecutive lanes, so a scale group leaves as one 32-bit store.  Longer
-// rows take a two-pass path straight from global memory.
+// few registers are live and many warps fit on an SM.  In the quantize pass a
+// lane takes one 16-element block at a time, so each block scale is computed
+// once, and the scale bytes of four consecutive blocks (four consecutive
+// lanes) leave as one 32-bit store.  Longer rows take a two-pass path
+// straight from global memory.
 //
 // Units of work are "virtual rows": an expert owns rows (linear layout) or
 // pad(rows, 128) virtual rows (swizzled); a virtual row past the last live row
@@ -61,28 +61,38 @@ __device__ __forceinline__ void store_scale_group(const qz_expert& E, int64_t ro
     }
 }
 
-// Quantize the 32 chunks c0 .. c0+31 of a row (this lane's chunk c = c0 + lane, in v).
+// Quantize blocks b0 .. b0+31 of a row, lane l taking block b = b0 + l whose
+// two chunks are v0, v1 (zeros past the row).  The scale bytes of four
+// consecutive blocks (lanes 4g .. 4g+3) leave as one 32-bit store.
 template <int LAYOUT>
-__device__ __forceinline__ void row_pass(const qz_expert& E, int64_t row, int64_t c, int64_t nch, int64_t kv,
-                                         uint4 v, float S, int lane) {
-    uint32_t m = absmax_bits(v);
-    m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
-    const Nvfp4Block blk = nvfp4_block(bits_to_float_bf16(m), S);
-    const uint32_t codes = e2m1x8_scaled(v, blk.rcp);
-    if (c < nch) st_u32(static_cast<uint8_t*>(E.q) + row * (E.cols >> 1) + c * 4, codes);
-    // gather the scale bytes of blocks k0..k0+3 (lanes base, base+2, base+4, base+6)
-    const uint32_t s1 = __shfl_down_sync(0xFFFFFFFFu, blk.scale, 2);
-    const uint32_t s2 = __shfl_down_sync(0xFFFFFFFFu, blk.scale, 4);
-    const uint32_t s3 = __shfl_down_sync(0xFFFFFFFFu, blk.scale, 6);
-    if ((lane & 7) == 0) store_scale_group<LAYOUT>(E, row, c >> 1, kv, blk.scale | (s1 << 8) | (s2 << 16) | (s3 << 24));
+__device__ __forceinline__ void row_blocks(const qz_expert& E, int64_t row, uint8_t* qrow, bool q8, int64_t b,
+                                           int64_t kv, uint4 v0, uint4 v1, float S, const float* inv, int lane) {
+    const uint32_t m = max(absmax_bits(v0), absmax_bits(v1));
+    const Nvfp4Block blk = nvfp4_block(bits_to_float_bf16(m), S, inv);
+    const uint32_t c0 = e2m1x8_scaled(v0, blk.rcp);
+    const uint32_t c1 = e2m1x8_scaled(v1, blk.rcp);
+    if (b < kv) {
+        if (q8) {
+            st_v2(qrow + b * 8, c0, c1);
+        } else {
+            st_u32(qrow + b * 8, c0);
+            st_u32(qrow + b * 8 + 4, c1);
+        }
+    }
+    const uint32_t s1 = __shfl_down_sync(0xFFFFFFFFu, blk.scale, 1);
+    const uint32_t s2 = __shfl_down_sync(0xFFFFFFFFu, blk.scale, 2);
+    const uint32_t s3 = __shfl_down_sync(0xFFFFFFFFu, blk.scale, 3);
+    if ((lane & 3) == 0) store_scale_group<LAYOUT>(E, row, b, kv, blk.scale | (s1 << 8) | (s2 << 16) | (s3 << 24));
 }
 
-// A row of at most 4096 elements staged in shared memory: amax pass, then a
-// quantize pass over the same slot.
+// A row of at most 4096 elements staged in shared memory: an amax pass over
+// the slot (lane l reads chunks l + 32i, conflict-free), then the quantize
+// pass with one 16-element block per lane.
 template <int LAYOUT>
-__device__ __forceinline__ void row_from_slot(const qz_expert& E, int64_t row, const uint8_t* slot, int lane) {
-    const int64_t nch = E.cols >> 3, kv = E.cols >> 4;
-    const int nsc = 2 * (int)pad_to(kv, 4);
+__device__ __forceinline__ void row_from_slot(const qz_expert& E, int64_t row, const uint8_t* slot, const float* inv,
+                                              int lane) {
+    const int nch = (int)(E.cols >> 3), kv = (int)(E.cols >> 4);
+    const int nbp = (int)pad_to(kv, 4);  // blocks whose scale bytes exist (incl. padding)
     uint32_t m = 0;
 #pragma unroll 4
     for (int c = lane; c < nch; c += 32) m = max(m, absmax_bits(lds128(slot + c * 16)));
@@ -91,19 +101,25 @@ __device__ __forceinline__ void row_from_slot(const qz_expert& E, int64_t row, c
     const float A = bits_to_float_bf16(m);
     if (lane == 0) E.amax[row] = A;
     const float S = nvfp4_encode_scale(A);
+    uint8_t* qrow = static_cast<uint8_t*>(E.q) + row * (E.cols >> 1);
+    const bool q8 = (((uintptr_t)qrow) & 7) == 0;
 #pragma unroll 2
-    for (int c0 = 0; c0 < nsc; c0 += 32) {
-        const int c = c0 + lane;
-        const uint4 v = (c < nch) ? lds128(slot + c * 16) : make_uint4(0, 0, 0, 0);
-        row_pass<LAYOUT>(E, row, c, nch, kv, v, S, lane);
+    for (int b0 = 0; b0 < nbp; b0 += 32) {
+        const int b = b0 + lane;
+        uint4 v0 = make_uint4(0, 0, 0, 0), v1 = make_uint4(0, 0, 0, 0);
+        if (b < kv) {
+            v0 = lds128(slot + b * 32);
+            v1 = lds128(slot + b * 32 + 16);
+        }
+        row_blocks<LAYOUT>(E, row, qrow, q8, b, kv, v0, v1, S, inv, lane);
     }
 }
 
 // A row of any length straight from global memory: amax pass, then a
 // quantize pass re-reading the row (served by L2).
 template <int LAYOUT>
-__device__ __forceinline__ void row_two_pass(const qz_expert& E, int64_t row, int lane) {
-    const int64_t nch = E.cols >> 3, kv = E.cols >> 4, nsc = 2 * pad_to(kv, 4);
+__device__ __forceinline__ void row_two_pass(const qz_expert& E, int64_t row, const float* inv, int lane) {
+    const int64_t nch = E.cols >> 3, kv = E.cols >> 4, nbp = pad_to(kv, 4);
     const uint16_t* xr = static_cast<const uint16_t*>(E.x) + row * E.ld;
     uint32_t m = 0;
     for (int64_t c = lane; c < nch; c += 32) m = max(m, absmax_bits(ld_stream(xr + c * 8)));
@@ -112,10 +128,16 @@ __device__ __forceinline__ void row_two_pass(const qz_expert& E, int64_t row, in
     const float A = bits_to_float_bf16(m);
     if (lane == 0) E.amax[row] = A;
     const float S = nvfp4_encode_scale(A);
-    for (int64_t c0 = 0; c0 < nsc; c0 += 32) {
-        const int64_t c = c0 + lane;
-        const uint4 v = (c < nch) ? ld_stream(xr + c * 8) : make_uint4(0, 0, 0, 0);
-        row_pass<LAYOUT>(E, row, c, nch, kv, v, S, lane);
+    uint8_t* qrow = static_cast<uint8_t*>(E.q) + row * (E.cols >> 1);
+    const bool q8 = (((uintptr_t)qrow) & 7) == 0;
+    for (int64_t b0 = 0; b0 < nbp; b0 += 32) {
+        const int64_t b = b0 + lane;
+        uint4 v0 = make_uint4(0, 0, 0, 0), v1 = make_uint4(0, 0, 0, 0);
+        if (b < kv) {
+            v0 = ld_stream(xr + b * 16);
+            v1 = ld_stream(xr + b * 16 + 8);
+        }
+        row_blocks<LAYOUT>(E, row, qrow, q8, b, kv, v0, v1, S, inv, lane);
     }
 }
 
@@ -146,6 +168,8 @@ __global__ void __launch_bounds__(kRowThreads, 1) nvfp4_rows_kernel(const qz_exp
     uint8_t* ring = smem + kRowBarBytes;
     int* s_prefix = reinterpret_cast<int*>(ring + kRowRingBytes);
     __shared__ long long s_scan[33];
+    __shared__ float s_inv[16];
+    fill_inv_table(s_inv);
     if (threadIdx.x < kRowWarps * kRowDepth) mbar_init(&bars[threadIdx.x], 1);
     mbar_init_fence();
     const int total = block_prefix(n, s_prefix, s_scan, RowUnits<LAYOUT>{table, d_err}, d_err);  // has barriers
@@ -187,9 +211,9 @@ __global__ void __launch_bounds__(kRowThreads, 1) nvfp4_rows_kernel(const qz_exp
                 break;
             }
             phase ^= 1u << s;
-            row_from_slot<LAYOUT>(r.E, r.row, slots + s * kRowSlot, lane);
+            row_from_slot<LAYOUT>(r.E, r.row, slots + s * kRowSlot, s_inv, lane);
         } else {
-            row_two_pass<LAYOUT>(r.E, r.row, lane);
+            row_two_pass<LAYOUT>(r.E, r.row, s_inv, lane);
         }
         __syncwarp();  // every lane is done with slot s before it is refilled
         issue(u + (long long)kRowDepth * stride, s);
