@@ -205,3 +205,21 @@ def test_qwen3_235b_experts_sampled():
         amax = x.double()
         assert torch.all(amax <= 448.0 * torch.exp2(e))
         assert torch.all((amax > 224.0 * torch.exp2(e)) | (amax == 0))
+
+
+def _blocks_with_every_amax(block: int) -> torch.Tensor:
+    """One block per positive finite bf16 value v: [v, -0.7 v, 0.3 v, 0, ...]."""
+    bits = np.arange(1, 0x7F80, dtype=np.uint32)
+    bits = bits[: bits.size // 8 * 8]
+    v = torch.from_numpy((bits << 16).view(np.float32).copy())
+    x = torch.zeros(v.numel(), block, dtype=torch.float32)
+    x[:, 0] = v
+    x[:, 1] = -0.7 * v
+    x[:, 2] = 0.3 * v
+    return x.to(torch.bfloat16).reshape(-1, 8 * block)
+
+
+@pytest.mark.parametrize("layout", LAYOUTS)
+def test_every_bf16_value_as_block_amax(layout):
+    x = _blocks_with_every_amax(32).cuda()
+    check_against_oracle([x], layout, run_mxfp8([x], layout))

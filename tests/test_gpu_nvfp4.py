@@ -189,3 +189,32 @@ def test_qwen3_235b_sampled_both_projections():
         check([xs[i] for i in sample], qz.SF_SWIZZLED, qz.NVFP4_PER_TENSOR_COMPUTE, got)
         del stack, xs, entries
         torch.cuda.empty_cache()
+
+
+def _blocks_with_every_amax(block: int) -> torch.Tensor:
+    bits = np.arange(1, 0x7F80, dtype=np.uint32)
+    bits = bits[: bits.size // 8 * 8]
+    v = torch.from_numpy((bits << 16).view(np.float32).copy())
+    x = torch.zeros(v.numel(), block, dtype=torch.float32)
+    x[:, 0] = v
+    x[:, 1] = -0.7 * v
+    x[:, 2] = 0.3 * v
+    x[:, 3] = 0.55 * v
+    return x.to(torch.bfloat16)
+
+
+def test_every_bf16_value_as_block_amax_per_row():
+    """Rows of one block: the row amax, the block amax and hence S and the
+    block scale take every bf16 magnitude."""
+    x = _blocks_with_every_amax(16)
+    x = x[x.float().abs().amax(dim=1) >= 2.0 ** -100].cuda()   # the contract's smallest amax
+    check([x], qz.SF_SWIZZLED, qz.NVFP4_PER_ROW, run_nvfp4([x], qz.SF_SWIZZLED, qz.NVFP4_PER_ROW))
+
+
+@pytest.mark.parametrize("A", [2688.0, 1.0, 3.0e4])
+def test_every_bf16_value_as_block_amax_given_scale(A):
+    """One tensor of blocks with every bf16 magnitude under a fixed encode
+    scale: the block scales span every e4m3 code, zero included."""
+    x = _blocks_with_every_amax(16).reshape(-1, 128)
+    x = x[x.float().abs().amax(dim=1) <= A].cuda()    # the given amax bounds the tensor
+    check([x], qz.SF_LINEAR, qz.NVFP4_PER_TENSOR_GIVEN, run_nvfp4([x], qz.SF_LINEAR, qz.NVFP4_PER_TENSOR_GIVEN, [A]), [A])
