@@ -199,7 +199,16 @@ class Refit30B:
             for s in side:
                 s.wait_event(start)
             for i, (table, _) in enumerate(self.calls):
-                qz.quantize_grouped_mxfp8(table, qz.SF_SWIZZLED, stream=side[i % len(side)])
+                st = side[i % len(side)]
+                if events is not None:
+                    a = torch.cuda.Event(enable_timing=True)
+                    b = torch.cuda.Event(enable_timing=True)
+                    a.record(st)
+                    qz.quantize_grouped_mxfp8(table, qz.SF_SWIZZLED, stream=st)
+                    b.record(st)
+                    events.append((a, b))
+                else:
+                    qz.quantize_grouped_mxfp8(table, qz.SF_SWIZZLED, stream=st)
             for s in side:
                 done = torch.cuda.Event()
                 done.record(s)
@@ -218,8 +227,10 @@ class Refit30B:
 
 
 def time_steps(work, steps, warmup, stream, dist_ok, side=None):
-    """W untimed steps, then K timed steps bracketed by barrier + sync.  On a
-    single stream, per-launch CUDA events are taken inside the timed region."""
+    """W untimed steps, then K timed steps bracketed by barrier + sync, with
+    per-launch CUDA events (on each launch's own stream) inside the timed
+    region.  Returns the total ms, every launch's duration and the length of
+    the union of all launch intervals (overlapping launches counted once)."""
     for _ in range(warmup):
         work.step(stream, side=side)
     torch.cuda.synchronize()
@@ -231,7 +242,7 @@ def time_steps(work, steps, warmup, stream, dist_ok, side=None):
     launch_events = []
     start.record(stream)
     for _ in range(steps):
-        work.step(stream, None if side else launch_events, side=side)
+        work.step(stream, launch_events, side=side)
     end.record(stream)
     torch.cuda.synchronize()
     if dist_ok:
@@ -239,7 +250,18 @@ def time_steps(work, steps, warmup, stream, dist_ok, side=None):
     torch.cuda.synchronize()
     total_ms = start.elapsed_time(end)
     launch_ms = [a.elapsed_time(b) for a, b in launch_events]
-    return total_ms, launch_ms
+    spans = sorted((start.elapsed_time(a), start.elapsed_time(b)) for a, b in launch_events)
+    busy, cur_a, cur_b = 0.0, None, None
+    for a, b in spans:
+        if cur_b is None or a > cur_b:
+            if cur_b is not None:
+                busy += cur_b - cur_a
+            cur_a, cur_b = a, b
+        else:
+            cur_b = max(cur_b, b)
+    if cur_b is not None:
+        busy += cur_b - cur_a
+    return total_ms, launch_ms, busy
 
 
 def e2e_refit(qz, device, steps, warmup, layers=48, per_call=16, pool=2):
@@ -373,7 +395,7 @@ class L2Flush:
         self.buf.zero_()
 
 
-def extra_workloads(qz, device, stream, peak, which=("split", "fused", "large")):
+def extra_workloads(qz, device, stream, peak, which=("split", "fused", "nvfp4", "large"), tokens=None):
     out = []
     flush = L2Flush(device)
 
@@ -387,7 +409,9 @@ def extra_workloads(qz, device, stream, peak, which=("split", "fused", "large"))
     if "split" in which:
         _extra_split(qz, device, flush, rec)
     if "fused" in which:
-        _extra_fused(qz, device, flush, out, peak)
+        _extra_fused(qz, device, flush, out, peak, tokens)
+    if "nvfp4" in which:
+        _extra_nvfp4_30b(qz, device, rec)
     if "large" in which:
         _extra_large(qz, device, rec)
     return out
@@ -420,12 +444,12 @@ def _extra_split(qz, device, flush, rec):
     del x, q, am, entries, table
 
 
-def _extra_fused(qz, device, flush, out, peak):
+def _extra_fused(qz, device, flush, out, peak, tokens=None):
     """Fused residual + RMSNorm + quantize, T sweep at H = 7168."""
     H = synth.FUSED_NORM["hidden"]
     for fmt, layout, fname in ((qz.FMT_MXFP8, qz.SF_SWIZZLED, "MXFP8 swizzled"), (qz.FMT_NVFP4, qz.SF_LINEAR, "NVFP4 linear")):
         sweep = []
-        for Tn in synth.FUSED_NORM["tokens"]:
+        for Tn in (tokens or synth.FUSED_NORM["tokens"]):
             xs, rs, gs = synth.fused_norm_inputs(Tn, device=device)
             y = torch.empty_like(xs)
             h = torch.empty_like(xs)
@@ -441,10 +465,33 @@ def _extra_fused(qz, device, flush, out, peak):
             nbytes = Tn * H * 2 * 2 + 2 * H + Tn * H * 2 * 2 + qbytes + qz.sf_bytes(Tn, H, fmt, layout)
             sweep.append({"T": Tn, "us": round(ms * 1e3, 2), "GB/s": round(nbytes / (ms / 1e3) / GB, 1)})
         big = sweep[-1]
+        if big["T"] != 4096:
+            big = {"GB/s": 0.0}
         out.append({"workload": f"fused residual+RMSNorm+{fname}, H=7168, T=1..4096 (residual_out written)",
                     "kernel": "rmsnorm_quant_kernel", "sweep": sweep,
                     "timing": "CUDA graph of 50 calls (T < 1024) or 10 calls after an L2 flush each",
                     "frac_of_hbm_peak_T4096": round(big["GB/s"] / peak, 4)})
+
+
+def _extra_nvfp4_30b(qz, device, rec):
+    """One Qwen3-30B-A3B gate_up projection (128 experts of [1536, 2048]) to
+    NVFP4 with a per-expert FP32 scale, given and computed, in one call."""
+    cfg = synth.QWEN3_30B
+    rows, cols = cfg["gate_up"]
+    stack = synth.expert_stack(cfg["experts"], (rows, cols), cfg["std"], seed=cfg["seed"], device=device)
+    for mode, fname in ((qz.NVFP4_PER_TENSOR_GIVEN, "given amax"), (qz.NVFP4_PER_TENSOR_COMPUTE, "computed amax")):
+        ents = qz.alloc_outputs(list(stack.unbind(0)), qz.FMT_NVFP4, qz.SF_SWIZZLED, mode)
+        for e in ents:
+            e.amax.fill_(0.1)
+        tab = qz.ExpertTable(ents)
+        ms = _time_graph(lambda m=mode: qz.quantize_grouped_nvfp4(tab, m, qz.SF_SWIZZLED), reps=5)
+        nsf = qz.sf_bytes(rows, cols, qz.FMT_NVFP4, qz.SF_SWIZZLED)
+        nbytes = cfg["experts"] * (rows * cols * 2 + rows * cols // 2 + nsf + 4)
+        rec(f"Qwen3-30B-A3B gate_up [1536, 2048] x128 experts, NVFP4 {fname}, swizzled, one call", nbytes, ms,
+            1 if mode == qz.NVFP4_PER_TENSOR_GIVEN else 3)
+        del ents, tab
+    del stack
+    torch.cuda.empty_cache()
 
 
 def _extra_large(qz, device, rec):
@@ -544,8 +591,10 @@ def main():
     ap.add_argument("--no-extra", action="store_true", help="skip the other workloads")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
-    ap.add_argument("--only", choices=["split", "fused", "large"], default=None,
+    ap.add_argument("--only", choices=["split", "fused", "nvfp4", "large"], default=None,
                     help="time only this secondary workload and print its record (profiling aid)")
+    ap.add_argument("--tokens", type=str, default=None,
+                    help="comma-separated token counts for the fused sweep (default: 1..4096)")
     args = ap.parse_args()
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -568,16 +617,17 @@ def main():
     stream = torch.cuda.current_stream()
     peak, peak_kind = hbm_peak()
     if args.only:
-        print(json.dumps({"only": args.only, "extra": extra_workloads(qz, device, stream, peak, (args.only,))}))
+        toks = [int(t) for t in args.tokens.split(",")] if args.tokens else None
+        print(json.dumps({"only": args.only, "extra": extra_workloads(qz, device, stream, peak, (args.only,), toks)}))
         return
 
     work = Refit30B(qz, device, layers=args.layers, seed_offset=rank)
     side = [torch.cuda.Stream() for _ in range(args.streams)] if args.streams > 1 else None
     torch.cuda.synchronize()
     with ClockSampler(local) as clocks:
-        total_ms, _ = time_steps(work, args.steps, args.warmup, stream, dist_ok, side=side)
-        # single-stream pass with per-launch events: the kernel's own duration
-        single_ms, launch_ms = time_steps(work, args.steps, 1, stream, dist_ok)
+        total_ms, launch_ms, busy_ms = time_steps(work, args.steps, args.warmup, stream, dist_ok, side=side)
+        # the same steps with every call in order on one stream, for comparison
+        single_ms, single_launch_ms, _ = time_steps(work, args.steps, 1, stream, dist_ok)
     if dist_ok:
         t = torch.tensor([total_ms, single_ms], dtype=torch.float64, device=device)
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
@@ -586,18 +636,25 @@ def main():
     value = world * work.bytes * args.steps / (total_ms / 1e3) / GB
     single_value = world * work.bytes * args.steps / (single_ms / 1e3) / GB
 
-    # roofline of the dominant (only) kernel: algorithmic bytes per launch
-    # over its mean CUDA-event duration inside the timed region
+    # roofline of the dominant (only) kernel: its algorithmic bytes over the
+    # time its launches occupied the GPU, from per-launch CUDA events inside
+    # the timed region (overlapping launches on the two streams counted once)
     call_bytes = [b for _, b in work.calls] * args.steps
-    achieved = sum(call_bytes) / (sum(launch_ms) / 1e3) / GB
+    achieved = sum(call_bytes) / (busy_ms / 1e3) / GB
+    achieved_single = sum(call_bytes) / (sum(single_launch_ms) / 1e3) / GB
     traffic = ncu_traffic(work.kernel)
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                 "frac": round(achieved / peak, 4), "traffic": traffic,
                 "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
                 else "fallback 6650 GB/s", "kernel": work.kernel,
-                "timing": "per-launch CUDA events in a single-stream pass of the same K steps",
+                "timing": "per-launch CUDA events on each launch's stream; achieved = bytes / union of launch "
+                          "intervals",
                 "bytes_per_launch": int(np.mean([b for _, b in work.calls])),
-                "mean_launch_us": round(1e3 * float(np.mean(launch_ms)), 2)}
+                "launches": len(launch_ms),
+                "mean_launch_us": round(1e3 * float(np.mean(launch_ms)), 2),
+                "single_stream_achieved": round(achieved_single, 1),
+                "single_stream_frac": round(achieved_single / peak, 4),
+                "single_stream_mean_launch_us": round(1e3 * float(np.mean(single_launch_ms)), 2)}
 
     line = {"metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(ms_step, 3), "higher_is_better": True, "scaling": "weak",

@@ -31,6 +31,7 @@ constexpr int kRowWarps = 12;                   // warps per CTA
 constexpr int kRowThreads = 32 * kRowWarps;
 constexpr int kRowBarBytes = 1024;              // mbarrier area at the start of shared memory
 constexpr size_t kRowRingBytes = (size_t)kRowWarps * kRowDepth * kRowSlot;
+constexpr size_t kRowStashBytes = (size_t)kRowWarps * (kRowSlot / 32) * sizeof(uint16_t);  // block amax per warp
 
 template <int LAYOUT>
 struct RowUnits {
@@ -62,12 +63,13 @@ __device__ __forceinline__ void store_scale_group(const qz_expert& E, int64_t ro
 }
 
 // Quantize blocks b0 .. b0+31 of a row, lane l taking block b = b0 + l whose
-// two chunks are v0, v1 (zeros past the row).  The scale bytes of four
-// consecutive blocks (lanes 4g .. 4g+3) leave as one 32-bit store.
+// two chunks are v0, v1 (zeros past the row) and whose amax has bf16 bits m.
+// The scale bytes of four consecutive blocks (lanes 4g .. 4g+3) leave as one
+// 32-bit store.
 template <int LAYOUT>
 __device__ __forceinline__ void row_blocks(const qz_expert& E, int64_t row, uint8_t* qrow, bool q8, int64_t b,
-                                           int64_t kv, uint4 v0, uint4 v1, float S, const float* inv, int lane) {
-    const uint32_t m = max(absmax_bits(v0), absmax_bits(v1));
+                                           int64_t kv, uint4 v0, uint4 v1, uint32_t m, float S, const float* inv,
+                                           int lane) {
     const Nvfp4Block blk = nvfp4_block(bits_to_float_bf16(m), S, inv);
     const uint32_t c0 = e2m1x8_scaled(v0, blk.rcp);
     const uint32_t c1 = e2m1x8_scaled(v1, blk.rcp);
@@ -85,19 +87,27 @@ __device__ __forceinline__ void row_blocks(const qz_expert& E, int64_t row, uint
     if ((lane & 3) == 0) store_scale_group<LAYOUT>(E, row, b, kv, blk.scale | (s1 << 8) | (s2 << 16) | (s3 << 24));
 }
 
-// A row of at most 4096 elements staged in shared memory: an amax pass over
-// the slot (lane l reads chunks l + 32i, conflict-free), then the quantize
-// pass with one 16-element block per lane.
+// A row of at most 4096 elements staged in shared memory.  Amax pass: lane l
+// reads chunks l + 32i (conflict-free), pairs of lanes combine a block's two
+// chunks and the block amax goes to the warp's stash (bf16 bits per block).
+// Quantize pass: one 16-element block per lane, its amax from the stash.
 template <int LAYOUT>
-__device__ __forceinline__ void row_from_slot(const qz_expert& E, int64_t row, const uint8_t* slot, const float* inv,
-                                              int lane) {
+__device__ __forceinline__ void row_from_slot(const qz_expert& E, int64_t row, const uint8_t* slot, uint16_t* stash,
+                                              const float* inv, int lane) {
     const int nch = (int)(E.cols >> 3), kv = (int)(E.cols >> 4);
     const int nbp = (int)pad_to(kv, 4);  // blocks whose scale bytes exist (incl. padding)
     uint32_t m = 0;
 #pragma unroll 4
-    for (int c = lane; c < nch; c += 32) m = max(m, absmax_bits(lds128(slot + c * 16)));
+    for (int c0 = 0; c0 < nch; c0 += 32) {  // nch is even: a block's chunks are both live or both not
+        const int c = c0 + lane;
+        uint32_t cm = c < nch ? absmax_bits(lds128(slot + c * 16)) : 0u;
+        cm = max(cm, __shfl_xor_sync(0xFFFFFFFFu, cm, 1));
+        if ((lane & 1) == 0 && c < nch) stash[c >> 1] = (uint16_t)cm;
+        m = max(m, cm);
+    }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+    __syncwarp();
     const float A = bits_to_float_bf16(m);
     if (lane == 0) E.amax[row] = A;
     const float S = nvfp4_encode_scale(A);
@@ -107,11 +117,13 @@ __device__ __forceinline__ void row_from_slot(const qz_expert& E, int64_t row, c
     for (int b0 = 0; b0 < nbp; b0 += 32) {
         const int b = b0 + lane;
         uint4 v0 = make_uint4(0, 0, 0, 0), v1 = make_uint4(0, 0, 0, 0);
+        uint32_t bm = 0;
         if (b < kv) {
             v0 = lds128(slot + b * 32);
             v1 = lds128(slot + b * 32 + 16);
+            bm = stash[b];
         }
-        row_blocks<LAYOUT>(E, row, qrow, q8, b, kv, v0, v1, S, inv, lane);
+        row_blocks<LAYOUT>(E, row, qrow, q8, b, kv, v0, v1, bm, S, inv, lane);
     }
 }
 
@@ -137,7 +149,7 @@ __device__ __forceinline__ void row_two_pass(const qz_expert& E, int64_t row, co
             v0 = ld_stream(xr + b * 16);
             v1 = ld_stream(xr + b * 16 + 8);
         }
-        row_blocks<LAYOUT>(E, row, qrow, q8, b, kv, v0, v1, S, inv, lane);
+        row_blocks<LAYOUT>(E, row, qrow, q8, b, kv, v0, v1, max(absmax_bits(v0), absmax_bits(v1)), S, inv, lane);
     }
 }
 
@@ -166,7 +178,8 @@ __global__ void __launch_bounds__(kRowThreads, 1) nvfp4_rows_kernel(const qz_exp
     extern __shared__ __align__(128) uint8_t smem[];
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem);
     uint8_t* ring = smem + kRowBarBytes;
-    int* s_prefix = reinterpret_cast<int*>(ring + kRowRingBytes);
+    uint16_t* stash_all = reinterpret_cast<uint16_t*>(ring + kRowRingBytes);
+    int* s_prefix = reinterpret_cast<int*>(ring + kRowRingBytes + kRowStashBytes);
     __shared__ long long s_scan[33];
     __shared__ float s_inv[16];
     fill_inv_table(s_inv);
@@ -178,6 +191,7 @@ __global__ void __launch_bounds__(kRowThreads, 1) nvfp4_rows_kernel(const qz_exp
     const int first = blockIdx.x * kRowWarps + w;
     uint8_t* slots = ring + (size_t)w * kRowDepth * kRowSlot;
     uint64_t* my_bars = bars + w * kRowDepth;
+    uint16_t* stash = stash_all + w * (kRowSlot / 32);
     unsigned issued = 0, phase = 0;  // per-slot bits, identical in every lane
 
     // start the copy of unit u into slot s when it is a live row that fits a slot
@@ -211,7 +225,7 @@ __global__ void __launch_bounds__(kRowThreads, 1) nvfp4_rows_kernel(const qz_exp
                 break;
             }
             phase ^= 1u << s;
-            row_from_slot<LAYOUT>(r.E, r.row, slots + s * kRowSlot, s_inv, lane);
+            row_from_slot<LAYOUT>(r.E, r.row, slots + s * kRowSlot, stash, s_inv, lane);
         } else {
             row_two_pass<LAYOUT>(r.E, r.row, s_inv, lane);
         }
@@ -228,7 +242,9 @@ __global__ void __launch_bounds__(kRowThreads, 1) nvfp4_rows_kernel(const qz_exp
         }
 }
 
-size_t rows_smem_bytes(int n) { return kRowBarBytes + kRowRingBytes + (size_t)(n + 1) * sizeof(int); }
+size_t rows_smem_bytes(int n) {
+    return kRowBarBytes + kRowRingBytes + kRowStashBytes + (size_t)(n + 1) * sizeof(int);
+}
 
 cudaError_t launch_nvfp4_rows(const qz_expert* table, int n, int layout, int grid, cudaStream_t s, unsigned* d_err) {
     const size_t smem = rows_smem_bytes(n);
