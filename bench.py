@@ -150,6 +150,28 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------------------
+# multi-rank host logic (weak scaling, no collective on the data path)
+# ---------------------------------------------------------------------------
+
+def rank_seed_offset(rank: int) -> int:
+    """Each rank quantizes its own synthetic workload: the seeds shift by rank."""
+    return int(rank)
+
+
+def max_over_ranks(values, device):
+    """Element-wise maximum over all ranks (the slowest rank sets the time)."""
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    if torch.distributed.is_available() and torch.distributed.is_initialized():
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def aggregate_gbs(bytes_per_rank: int, world: int, steps: int, total_ms: float) -> float:
+    """Whole-job throughput: the bytes of all ranks over the max-over-ranks time."""
+    return world * bytes_per_rank * steps / (total_ms / 1e3) / GB
+
+
+# ---------------------------------------------------------------------------
 # workloads (the product path: every launch goes through the C ABI)
 # ---------------------------------------------------------------------------
 
@@ -168,7 +190,7 @@ class Refit30B:
         self._keep = []
         for layer in range(layers):
             for proj, shape in (("gate_up", cfg["gate_up"]), ("down", cfg["down"])):
-                seed = cfg["seed"] + layer + seed_offset * 1000 + (0 if proj == "gate_up" else 500)
+                seed = cfg["seed"] + layer + rank_seed_offset(seed_offset) * 1000 + (0 if proj == "gate_up" else 500)
                 stack = synth.expert_stack(cfg["experts"], shape, cfg["std"], seed=seed, device=device)
                 rows, cols = shape
                 nsf = qz.sf_bytes(rows, cols, qz.FMT_MXFP8, qz.SF_SWIZZLED)
@@ -226,11 +248,12 @@ class Refit30B:
                 qz.quantize_grouped_mxfp8(table, qz.SF_SWIZZLED, stream=stream)
 
 
-def time_steps(work, steps, warmup, stream, dist_ok, side=None):
-    """W untimed steps, then K timed steps bracketed by barrier + sync, with
-    per-launch CUDA events (on each launch's own stream) inside the timed
-    region.  Returns the total ms, every launch's duration and the length of
-    the union of all launch intervals (overlapping launches counted once)."""
+def time_steps(work, steps, warmup, stream, dist_ok, side=None, per_launch=True):
+    """W untimed steps, then K timed steps bracketed by barrier + sync.  With
+    per_launch, CUDA events bracket every launch on its own stream (timing
+    events between the launches of two streams cost their overlap, so the
+    headline pass goes without them).  Returns the total ms, every launch's
+    duration and the union of the launch intervals (overlaps counted once)."""
     for _ in range(warmup):
         work.step(stream, side=side)
     torch.cuda.synchronize()
@@ -242,7 +265,7 @@ def time_steps(work, steps, warmup, stream, dist_ok, side=None):
     launch_events = []
     start.record(stream)
     for _ in range(steps):
-        work.step(stream, launch_events, side=side)
+        work.step(stream, launch_events if per_launch else None, side=side)
     end.record(stream)
     torch.cuda.synchronize()
     if dist_ok:
@@ -625,33 +648,33 @@ def main():
     side = [torch.cuda.Stream() for _ in range(args.streams)] if args.streams > 1 else None
     torch.cuda.synchronize()
     with ClockSampler(local) as clocks:
-        total_ms, launch_ms, busy_ms = time_steps(work, args.steps, args.warmup, stream, dist_ok, side=side)
-        # the same steps with every call in order on one stream, for comparison
+        total_ms, _, _ = time_steps(work, args.steps, args.warmup, stream, dist_ok, side=side, per_launch=False)
+        # the same steps with every call in order on one stream and an event
+        # pair around each launch: the kernel's own launch durations
         single_ms, single_launch_ms, _ = time_steps(work, args.steps, 1, stream, dist_ok)
-    if dist_ok:
-        t = torch.tensor([total_ms, single_ms], dtype=torch.float64, device=device)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        total_ms, single_ms = float(t[0].item()), float(t[1].item())
+    total_ms, single_ms = max_over_ranks([total_ms, single_ms], device)
     ms_step = total_ms / args.steps
-    value = world * work.bytes * args.steps / (total_ms / 1e3) / GB
-    single_value = world * work.bytes * args.steps / (single_ms / 1e3) / GB
+    value = aggregate_gbs(work.bytes, world, args.steps, total_ms)
+    single_value = aggregate_gbs(work.bytes, world, args.steps, single_ms)
 
-    # roofline of the dominant (only) kernel: its algorithmic bytes over the
-    # time its launches occupied the GPU, from per-launch CUDA events inside
-    # the timed region (overlapping launches on the two streams counted once)
+    # roofline of the dominant (only) kernel.  The timed region holds nothing
+    # but its launches (two streams, back to back), so its algorithmic bytes
+    # over the region's CUDA-event time is its achieved bandwidth, i.e. bytes
+    # per launch over the effective launch duration (region time / launches).
+    # The single-stream pass gives each launch's own event-timed duration.
     call_bytes = [b for _, b in work.calls] * args.steps
-    achieved = sum(call_bytes) / (busy_ms / 1e3) / GB
+    achieved = sum(call_bytes) / (total_ms / 1e3) / GB
     achieved_single = sum(call_bytes) / (sum(single_launch_ms) / 1e3) / GB
     traffic = ncu_traffic(work.kernel)
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                 "frac": round(achieved / peak, 4), "traffic": traffic,
                 "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
                 else "fallback 6650 GB/s", "kernel": work.kernel,
-                "timing": "per-launch CUDA events on each launch's stream; achieved = bytes / union of launch "
-                          "intervals",
+                "timing": "CUDA events around the timed region, which holds only this kernel's launches "
+                          "(2 streams); effective launch duration = region time / launches",
                 "bytes_per_launch": int(np.mean([b for _, b in work.calls])),
-                "launches": len(launch_ms),
-                "mean_launch_us": round(1e3 * float(np.mean(launch_ms)), 2),
+                "launches": work.launches * args.steps,
+                "effective_launch_us": round(1e3 * total_ms / (work.launches * args.steps), 2),
                 "single_stream_achieved": round(achieved_single, 1),
                 "single_stream_frac": round(achieved_single / peak, 4),
                 "single_stream_mean_launch_us": round(1e3 * float(np.mean(single_launch_ms)), 2)}
