@@ -84,7 +84,7 @@ typedef enum qz_nvfp4_scale_mode {
                                   ld < cols or ld > QZ_MAX_LD */
 #define QZ_DERR_NULL 0x2u      /* x, q, sf (or amax for NVFP4) null on a non-empty entry */
 #define QZ_DERR_ALIGN 0x4u     /* x not 16-byte aligned or ld not a multiple of 8; q not
-                                  8-byte (MXFP8) / 4-byte (NVFP4) aligned; sf not 16-byte
+                                  16-byte (MXFP8) / 8-byte (NVFP4) aligned; sf not 16-byte
                                   aligned (swizzled); amax not 4-byte aligned */
 #define QZ_DERR_TOO_LARGE 0x8u /* the call's total tile or row count exceeds 2^31 - 1 */
 #define QZ_DERR_TIMEOUT 0x10u  /* a wait for an asynchronous copy exceeded its time limit; the
@@ -110,7 +110,8 @@ typedef struct qz_expert {
     int64_t rows;  /* may be 0 (an empty split): nothing is read or written */
     int64_t cols;  /* quantization axis; multiple of 32 (MXFP8) or 16 (NVFP4) */
     int64_t ld;    /* row stride of x in elements, >= cols, <= QZ_MAX_LD, multiple of 8 */
-    void *q;       /* payload, row-major and dense: MXFP8 e4m3 [rows, cols];
+    void *q;       /* payload, row-major and dense (16-byte aligned for MXFP8, 8-byte
+                      for NVFP4): MXFP8 e4m3 [rows, cols];
                       NVFP4 e2m1 [rows, cols/2], element 2j in the low nibble
                       of byte j and element 2j+1 in the high nibble */
     uint8_t *sf;   /* this expert's SF region of qz_sf_bytes(rows, cols, fmt, layout) bytes */

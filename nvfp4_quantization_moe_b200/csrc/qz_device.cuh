@@ -38,6 +38,24 @@ __device__ __forceinline__ void st_u32(void* p, uint32_t a) {
     asm volatile("st.global.u32 [%0], %1;" ::"l"(p), "r"(a) : "memory");
 }
 
+// 32-byte load (the address must be 32-byte aligned).
+__device__ __forceinline__ void ld_stream_32(const void* p, uint32_t (&w)[8]) {
+    asm volatile("ld.global.nc.L1::no_allocate.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3]), "=r"(w[4]), "=r"(w[5]), "=r"(w[6]), "=r"(w[7])
+                 : "l"(p));
+}
+
+// 32 bytes from a 16-byte aligned address as two 16-byte loads that allocate
+// in L1 (the second finds the sectors the first brought in).
+__device__ __forceinline__ void ld_pair_16(const void* p, uint32_t (&w)[8]) {
+    asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3])
+                 : "l"(p));
+    asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(w[4]), "=r"(w[5]), "=r"(w[6]), "=r"(w[7])
+                 : "l"(static_cast<const char*>(p) + 16));
+}
+
 __device__ __forceinline__ void st_v4(void* p, uint4 v) {
     asm volatile("st.global.v4.u32 [%0], {%1,%2,%3,%4};" ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
                  : "memory");
@@ -124,6 +142,27 @@ __device__ __forceinline__ uint32_t e2m1x8_scaled(uint4 v, float s) {
           "f"(__fmul_rn(bf16_lo(v.z), s)), "f"(__fmul_rn(bf16_hi(v.z), s)),
           "f"(__fmul_rn(bf16_lo(v.w), s)), "f"(__fmul_rn(bf16_hi(v.w), s)));
     return r;
+}
+
+// Four e4m3 codes of the bf16 pairs in words a, b times s (element 0 lowest).
+__device__ __forceinline__ uint32_t e4m3x4_words(uint32_t a, uint32_t b, float s) {
+    const uint32_t lo = cvt_e4m3x2(__fmul_rn(bf16_lo(a), s), __fmul_rn(bf16_hi(a), s));
+    const uint32_t hi = cvt_e4m3x2(__fmul_rn(bf16_lo(b), s), __fmul_rn(bf16_hi(b), s));
+    return lo | (hi << 16);
+}
+
+// Eight e2m1 codes of the bf16 pairs in words a..d times s (element 0 lowest).
+__device__ __forceinline__ uint32_t e2m1x8_words(uint32_t a, uint32_t b, uint32_t c, uint32_t d, float s) {
+    return e2m1x8_scaled(make_uint4(a, b, c, d), s);
+}
+
+// Largest |x| of the bf16 pairs in w[0..N), as bf16 magnitude bits.
+template <int N>
+__device__ __forceinline__ uint32_t absmax_words(const uint32_t* w) {
+    uint32_t m = w[0] & 0x7FFF7FFFu;
+#pragma unroll
+    for (int i = 1; i < N; ++i) m = max_u16x2(m, w[i] & 0x7FFF7FFFu);
+    return max(m & 0xFFFFu, m >> 16);
 }
 
 // e4m3 code (RNE, satfinite) of one non-negative float.
@@ -234,7 +273,7 @@ __device__ __forceinline__ unsigned entry_errors(const qz_expert& e, int fmt, in
     if (e.rows > 0) {
         if (!e.x || !e.q || !e.sf || (needs_amax && !e.amax)) bad |= QZ_DERR_NULL;
         if (!aligned(e.x, 16) || (e.ld & 7) != 0) bad |= QZ_DERR_ALIGN;
-        if (!aligned(e.q, fmt == QZ_FMT_MXFP8 ? 8 : 4)) bad |= QZ_DERR_ALIGN;
+        if (!aligned(e.q, fmt == QZ_FMT_MXFP8 ? 16 : 8)) bad |= QZ_DERR_ALIGN;
         if (layout == QZ_SF_SWIZZLED_128x4 && !aligned(e.sf, 16)) bad |= QZ_DERR_ALIGN;
         if (needs_amax && !aligned(e.amax, 4)) bad |= QZ_DERR_ALIGN;
     }

@@ -43,39 +43,59 @@ struct TableTiles {
 };
 
 // ---------------------------------------------------------------------------
-// tile walk with a register prefetch ring
+// tile walk: one lane per scale block, register prefetch ring
 //
-// Pass p (0..7) of warp w covers tile rows (p & 3) * 32 + 4w + 2 (p >> 2) +
-// lane / 16: the warp owns rows r with r % 32 in [4w, 4w + 4), i.e. exactly
-// four 16-byte chunks of every 512-byte swizzled scale tile, which it
-// assembles in its own 64 bytes of shared memory (no CTA barrier).  As soon
-// as pass p of the current tile is consumed, slot p is refilled with pass p
-// of the CTA's next tile, so about eight 16-byte loads per thread are always
-// in flight.
+// A tile is 128 rows x 128 bf16 columns.  Each lane owns one whole scale
+// block per pass (MXFP8: 32 elements, 64 bytes; NVFP4: 16 elements, 32 bytes),
+// so the block amax, the scale and its reciprocal are computed once per block
+// with no shuffles.  LPR lanes cover a row of the tile, a warp covers RPP rows
+// per pass, and pass p of warp w covers the rows r with r % 32 = 4w + (l & 3)
+// and r / 32 = l >> 2, l = p * RPP + lane / LPR: the warp owns exactly four
+// 16-byte chunks of every 512-byte swizzled scale tile and assembles them in
+// its own shared-memory staging area (no CTA barrier).  As soon as pass p of
+// the current tile is consumed, its registers are refilled with pass p of the
+// CTA's next tile, so about 32 bytes of loads per lane stay in flight.
 // ---------------------------------------------------------------------------
 
-// One thread's view of a tile: pointers to its first row (tile row r0 =
-// 4w + lane/16) at its chunk's column; pass p adds kPassRow[p] rows, so the
-// per-pass address and bounds arithmetic is 32-bit.
+template <int FMT>
+struct TileGeo {
+    static constexpr int kBlock = FMT == QZ_FMT_MXFP8 ? 32 : 16;  // elements per scale block
+    static constexpr int kLpr = kTileCols / kBlock;                // lanes per tile row: 4 / 8
+    static constexpr int kRpp = 32 / kLpr;                         // rows per warp pass: 8 / 4
+    static constexpr int kPasses = 16 / kRpp;                      // passes per tile: 2 / 4
+    static constexpr int kWords = kBlock / 2;                      // bf16x2 words per lane per pass
+    static constexpr int kSfTiles = kTileCols / (4 * kBlock);      // 4-column scale tiles per tile: 1 / 2
+};
+
+// One thread's view of a tile: pointers for pass 0; pass p adds p * kRpp * 8 rows.
 struct TileRef {
-    const uint16_t* xp;  // x of (rt*128 + r0, ct*128 + chunk*8)
+    const uint16_t* xp;  // x of (rt*128 + r(0), ct*128 + kb*block)
     uint8_t* qp;         // payload byte of the same element
-    uint8_t* sfp;        // linear SF byte of (rt*128 + r0, block of the chunk); swizzled: region base
+    uint8_t* sfp;        // linear SF byte of (row(0), block); swizzled: region base
     const float* amax;
     int ld;              // x row stride, elements
     int qld;             // payload row bytes
     int kv;              // scale columns
-    int rows_left;       // pass p is live iff kPassRow[p] < rows_left (and col_ok)
+    int rows_left;       // pass p is live iff p * kRpp * 8 < rows_left (and col_ok)
     bool col_ok;
+    bool a32;            // rows are 32-byte aligned: one 256-bit load per 16 elements
     int rt, ct;
     int expert;
 };
 
-__device__ __forceinline__ constexpr int pass_row(int p) { return (p & 3) * 32 + 2 * (p >> 2); }
+template <int FMT>
+__device__ __forceinline__ int local_row(int p, int lane) { return p * TileGeo<FMT>::kRpp + lane / TileGeo<FMT>::kLpr; }
+
+template <int FMT>
+__device__ __forceinline__ int tile_row(int p, int w, int lane) {
+    const int l = local_row<FMT>(p, lane);
+    return (l >> 2) * 32 + 4 * w + (l & 3);
+}
 
 template <int FMT, int LAYOUT>
 __device__ __forceinline__ TileRef tile_ref(const qz_expert* table, const int* s_prefix, int n, int tile, int w,
                                             int lane) {
+    using G = TileGeo<FMT>;
     const int e = find_owner(s_prefix, n, tile);
     const qz_expert E = load_entry(table, e);
     const int local = tile - s_prefix[e];
@@ -83,59 +103,89 @@ __device__ __forceinline__ TileRef tile_ref(const qz_expert* table, const int* s
     TileRef t;
     t.rt = local / nct;
     t.ct = local - t.rt * nct;
-    const int chunk = lane & 15;
-    const int r0 = 4 * w + (lane >> 4);
-    const int64_t row0 = (int64_t)t.rt * kTileRows + r0;
-    const int64_t col = (int64_t)t.ct * kTileCols + chunk * 8;
+    const int kb = lane % G::kLpr;
+    const int64_t row0 = (int64_t)t.rt * kTileRows + tile_row<FMT>(0, w, lane);
+    const int64_t col = (int64_t)t.ct * kTileCols + kb * G::kBlock;
     t.ld = (int)E.ld;
     t.qld = (int)(FMT == QZ_FMT_MXFP8 ? E.cols : E.cols >> 1);
-    t.kv = (int)(FMT == QZ_FMT_MXFP8 ? E.cols >> 5 : E.cols >> 4);
+    t.kv = (int)(E.cols / G::kBlock);
     t.xp = static_cast<const uint16_t*>(E.x) + row0 * E.ld + col;
     t.qp = static_cast<uint8_t*>(E.q) + row0 * t.qld + (FMT == QZ_FMT_MXFP8 ? col : col >> 1);
-    t.sfp = LAYOUT == QZ_SF_SWIZZLED_128x4 ? E.sf : E.sf + row0 * t.kv + (FMT == QZ_FMT_MXFP8 ? col >> 5 : col >> 4);
+    t.sfp = LAYOUT == QZ_SF_SWIZZLED_128x4 ? E.sf : E.sf + row0 * t.kv + col / G::kBlock;
     t.amax = E.amax;
     const int64_t left = E.rows - row0;
     t.rows_left = left > kTileRows ? kTileRows : (int)left;
     t.col_ok = col < E.cols;
+    t.a32 = ((reinterpret_cast<uintptr_t>(E.x) & 31) == 0) && ((E.ld & 15) == 0);
     t.expert = e;
     return t;
 }
 
-__device__ __forceinline__ uint4 tile_load(const TileRef& t, int p) {
-    const int pr = pass_row(p);
-    return (t.col_ok && pr < t.rows_left) ? ld_stream(t.xp + pr * t.ld) : make_uint4(0, 0, 0, 0);
+template <int FMT>
+__device__ __forceinline__ bool pass_live(const TileRef& t, int p) {
+    return t.col_ok && p * TileGeo<FMT>::kRpp * 8 < t.rows_left;
 }
 
-// Quantize pass p of tile t (8 elements per thread in v).  MXFP8 blocks span
-// 4 lanes, NVFP4 blocks 2.  Swizzled scale bytes go to the warp's staging
-// area s (64 bytes per 4-column scale tile), linear ones straight to memory.
+// The lane's block of pass p (zeros outside the matrix).
+template <int FMT>
+__device__ __forceinline__ void tile_load(const TileRef& t, int p, uint32_t* w) {
+    using G = TileGeo<FMT>;
+    uint32_t (&a)[8] = *reinterpret_cast<uint32_t(*)[8]>(w);
+    uint32_t (&b)[8] = *reinterpret_cast<uint32_t(*)[8]>(w + 8 * (G::kWords / 8 - 1));
+    if (pass_live<FMT>(t, p)) {
+        const uint16_t* src = t.xp + p * G::kRpp * 8 * t.ld;
+        if (t.a32) {
+            ld_stream_32(src, a);
+            if (G::kWords == 16) ld_stream_32(src + 16, b);
+        } else {
+            ld_pair_16(src, a);
+            if (G::kWords == 16) ld_pair_16(src + 16, b);
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < G::kWords; ++i) w[i] = 0u;
+    }
+}
+
+// Quantize the lane's block of pass p; swizzled scale bytes go to the warp's
+// staging area s (64 bytes per 4-column scale tile), linear ones to memory.
 template <int FMT, int LAYOUT>
-__device__ __forceinline__ void tile_pass(const TileRef& t, int p, int lane, uint4 v, float S, uint8_t* s,
+__device__ __forceinline__ void tile_pass(const TileRef& t, int p, int lane, const uint32_t* w, float S, uint8_t* s,
                                           const float* inv) {
-    const int chunk = lane & 15;
-    const int pr = pass_row(p);
-    const bool live = t.col_ok && pr < t.rows_left;
-    const int stage = (2 * (p >> 2) + (lane >> 4)) * 16 + (p & 3) * 4;  // byte of this row in the warp's chunks
-    uint32_t m = absmax_bits(v);
-    m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
+    using G = TileGeo<FMT>;
+    const bool live = pass_live<FMT>(t, p);
+    const int l = local_row<FMT>(p, lane);
+    const int kb = lane % G::kLpr;
+    const uint32_t m = absmax_words<G::kWords>(w);
+    uint32_t scale;
     if (FMT == QZ_FMT_MXFP8) {
-        m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
-        const uint32_t byte = e8m0_byte(m);
-        const uint2 codes = e4m3x8_scaled(v, e8m0_reciprocal(byte));
-        if (live) st_v2(t.qp + pr * t.qld, codes.x, codes.y);
-        if ((chunk & 3) == 0) {
-            if (LAYOUT == QZ_SF_SWIZZLED_128x4) s[stage + (chunk >> 2)] = live ? (uint8_t)byte : (uint8_t)0;
-            else if (live) t.sfp[pr * t.kv] = (uint8_t)byte;
+        scale = e8m0_byte(m);
+        const float r = e8m0_reciprocal(scale);
+        uint4 c0, c1;
+        c0.x = e4m3x4_words(w[0], w[1], r);
+        c0.y = e4m3x4_words(w[2], w[3], r);
+        c0.z = e4m3x4_words(w[4], w[5], r);
+        c0.w = e4m3x4_words(w[6], w[7], r);
+        c1.x = e4m3x4_words(w[8], w[9], r);
+        c1.y = e4m3x4_words(w[10], w[11], r);
+        c1.z = e4m3x4_words(w[12], w[13], r);
+        c1.w = e4m3x4_words(w[14], w[15], r);
+        if (live) {
+            uint8_t* dst = t.qp + p * G::kRpp * 8 * t.qld;
+            st_v4(dst, c0);
+            st_v4(dst + 16, c1);
         }
     } else {
         const Nvfp4Block blk = nvfp4_block(bits_to_float_bf16(m), S, inv);
-        const uint32_t codes = e2m1x8_scaled(v, blk.rcp);
-        if (live) st_u32(t.qp + pr * t.qld, codes);
-        if ((chunk & 1) == 0) {
-            const int kk = chunk >> 1;  // 0..7: two 4-column scale tiles per tile
-            if (LAYOUT == QZ_SF_SWIZZLED_128x4) s[(kk >> 2) * 64 + stage + (kk & 3)] = live ? (uint8_t)blk.scale : (uint8_t)0;
-            else if (live) t.sfp[pr * t.kv] = (uint8_t)blk.scale;
-        }
+        scale = blk.scale;
+        const uint32_t c0 = e2m1x8_words(w[0], w[1], w[2], w[3], blk.rcp);
+        const uint32_t c1 = e2m1x8_words(w[4], w[5], w[6], w[7], blk.rcp);
+        if (live) st_v2(t.qp + p * G::kRpp * 8 * t.qld, c0, c1);
+    }
+    if (LAYOUT == QZ_SF_SWIZZLED_128x4) {
+        s[(kb >> 2) * 64 + (l & 3) * 16 + (l >> 2) * 4 + (kb & 3)] = live ? (uint8_t)scale : (uint8_t)0;
+    } else if (live) {
+        t.sfp[p * G::kRpp * 8 * t.kv] = (uint8_t)scale;
     }
 }
 
@@ -144,10 +194,10 @@ template <int FMT>
 __device__ __forceinline__ void tile_flush_sf(const TileRef& t, int w, int lane, const uint8_t* s) {
     __syncwarp();
     const int col_tiles = (t.kv + 3) >> 2;
-    constexpr int kTilesPerTile = FMT == QZ_FMT_MXFP8 ? 1 : 2;
-    if (lane < 4 * kTilesPerTile) {
+    constexpr int kT = TileGeo<FMT>::kSfTiles;
+    if (lane < 4 * kT) {
         const int j = lane >> 2, c = lane & 3;
-        const int ctile = t.ct * kTilesPerTile + j;
+        const int ctile = t.ct * kT + j;
         if (ctile < col_tiles)
             st_v4(t.sfp + (((int64_t)t.rt * col_tiles + ctile) << 9) + (4 * w + c) * 16,
                   *reinterpret_cast<const uint4*>(s + j * 64 + c * 16));
@@ -157,11 +207,11 @@ __device__ __forceinline__ void tile_flush_sf(const TileRef& t, int w, int lane,
 
 template <int FMT, int LAYOUT>
 __global__ void __launch_bounds__(kThreads, 3) grouped_tile_kernel(const qz_expert* __restrict__ table, int n,
-                                                                unsigned* d_err) {
+                                                                   unsigned* d_err) {
+    using G = TileGeo<FMT>;
     extern __shared__ int s_prefix[];
     __shared__ long long s_scan[33];
-    constexpr int kStage = FMT == QZ_FMT_MXFP8 ? 64 : 128;
-    __shared__ __align__(16) uint8_t s_sf[kThreads / 32][kStage];
+    __shared__ __align__(16) uint8_t s_sf[kThreads / 32][64 * G::kSfTiles];
     __shared__ float s_inv[16];
     constexpr bool kAmax = FMT == QZ_FMT_NVFP4;
     if (kAmax) fill_inv_table(s_inv);  // published by the barriers in block_prefix
@@ -170,18 +220,18 @@ __global__ void __launch_bounds__(kThreads, 3) grouped_tile_kernel(const qz_expe
     int tile = blockIdx.x;
     if (tile >= total) return;
     TileRef cur = tile_ref<FMT, LAYOUT>(table, s_prefix, n, tile, w, lane);
-    uint4 v[8];
+    uint32_t v[G::kPasses][G::kWords];
 #pragma unroll
-    for (int p = 0; p < 8; ++p) v[p] = tile_load(cur, p);
+    for (int p = 0; p < G::kPasses; ++p) tile_load<FMT>(cur, p, v[p]);
     for (;;) {
         const int next = tile + gridDim.x;
         const bool more = next < total;
         const TileRef nxt = more ? tile_ref<FMT, LAYOUT>(table, s_prefix, n, next, w, lane) : cur;
         const float S = kAmax ? nvfp4_encode_scale(*cur.amax) : 0.0f;
 #pragma unroll
-        for (int p = 0; p < 8; ++p) {
+        for (int p = 0; p < G::kPasses; ++p) {
             tile_pass<FMT, LAYOUT>(cur, p, lane, v[p], S, s_sf[w], s_inv);
-            if (more) v[p] = tile_load(nxt, p);
+            if (more) tile_load<FMT>(nxt, p, v[p]);
         }
         if (LAYOUT == QZ_SF_SWIZZLED_128x4) tile_flush_sf<FMT>(cur, w, lane, s_sf[w]);
         if (!more) break;
@@ -206,8 +256,9 @@ __global__ void amax_clear_kernel(const qz_expert* __restrict__ table, int n, in
 // running maximum while its tiles stay in one expert and publishes it with
 // one atomic max (non-negative floats order like their bit patterns).
 template <int LAYOUT>
-__global__ void __launch_bounds__(kThreads) amax_grouped_kernel(const qz_expert* __restrict__ table, int n,
-                                                                unsigned* d_err) {
+__global__ void __launch_bounds__(kThreads, 3) amax_grouped_kernel(const qz_expert* __restrict__ table, int n,
+                                                                   unsigned* d_err) {
+    using G = TileGeo<QZ_FMT_NVFP4>;
     extern __shared__ int s_prefix[];
     __shared__ long long s_scan[33];
     const int total = block_prefix(n, s_prefix, s_scan, TableTiles<QZ_FMT_NVFP4, LAYOUT, true>{table, d_err}, d_err);
@@ -215,18 +266,18 @@ __global__ void __launch_bounds__(kThreads) amax_grouped_kernel(const qz_expert*
     int tile = blockIdx.x;
     if (tile >= total) return;
     TileRef cur = tile_ref<QZ_FMT_NVFP4, LAYOUT>(table, s_prefix, n, tile, w, lane);
-    uint4 v[8];
+    uint32_t v[G::kPasses][G::kWords];
 #pragma unroll
-    for (int p = 0; p < 8; ++p) v[p] = tile_load(cur, p);
+    for (int p = 0; p < G::kPasses; ++p) tile_load<QZ_FMT_NVFP4>(cur, p, v[p]);
     uint32_t run = 0;
     for (;;) {
         const int next = tile + gridDim.x;
         const bool more = next < total;
         const TileRef nxt = more ? tile_ref<QZ_FMT_NVFP4, LAYOUT>(table, s_prefix, n, next, w, lane) : cur;
 #pragma unroll
-        for (int p = 0; p < 8; ++p) {
-            run = max(run, absmax_bits(v[p]));
-            if (more) v[p] = tile_load(nxt, p);
+        for (int p = 0; p < G::kPasses; ++p) {
+            run = max(run, absmax_words<G::kWords>(v[p]));
+            if (more) tile_load<QZ_FMT_NVFP4>(nxt, p, v[p]);
         }
         if (!more || nxt.expert != cur.expert) {
 #pragma unroll

@@ -72,8 +72,11 @@ def test_random_bit_patterns_and_zero_blocks():
 
 
 def test_strided_rows():
+    """Row strides and offsets that keep rows 32-byte aligned (256-bit loads)
+    and ones that only keep them 16-byte aligned (paired 128-bit loads)."""
     base = synth.normal_bf16((300, 2048 + 64), seed=9).cuda()
-    xs = [base[:, :2048], base[:150, 64:64 + 1024]]
+    odd = synth.normal_bf16((140, 2048 + 8), seed=10).cuda()
+    xs = [base[:, :2048], base[:150, 64:64 + 1024], odd[:, :2048], odd[:, 8:8 + 1536]]
     got = run_mxfp8(xs, qz.SF_SWIZZLED)
     check_against_oracle([x.contiguous() for x in xs], qz.SF_SWIZZLED, got)
 

@@ -218,3 +218,14 @@ def test_every_bf16_value_as_block_amax_given_scale(A):
     x = _blocks_with_every_amax(16).reshape(-1, 128)
     x = x[x.float().abs().amax(dim=1) <= A].cuda()    # the given amax bounds the tensor
     check([x], qz.SF_LINEAR, qz.NVFP4_PER_TENSOR_GIVEN, run_nvfp4([x], qz.SF_LINEAR, qz.NVFP4_PER_TENSOR_GIVEN, [A]), [A])
+
+
+@pytest.mark.parametrize("mode", list(MODES))
+def test_strided_rows_all_modes(mode):
+    m = MODES[mode]
+    base = synth.normal_bf16((260, 1024 + 64), seed=21).cuda()
+    odd = synth.normal_bf16((133, 1024 + 8), seed=22).cuda()
+    xs = [base[:, :1024], odd[:, :1024], odd[:, 8:8 + 512]]
+    amax_in = [float(x.float().abs().max()) for x in xs] if m == qz.NVFP4_PER_TENSOR_GIVEN else None
+    got = run_nvfp4(xs, qz.SF_SWIZZLED, m, amax_in)
+    check([x.contiguous() for x in xs], qz.SF_SWIZZLED, m, got, amax_in)
