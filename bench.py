@@ -502,16 +502,19 @@ def _extra_nvfp4_30b(qz, device, rec):
     cfg = synth.QWEN3_30B
     rows, cols = cfg["gate_up"]
     stack = synth.expert_stack(cfg["experts"], (rows, cols), cfg["std"], seed=cfg["seed"], device=device)
-    for mode, fname in ((qz.NVFP4_PER_TENSOR_GIVEN, "given amax"), (qz.NVFP4_PER_TENSOR_COMPUTE, "computed amax")):
+    ws = qz.alloc_workspace(cfg["experts"], device)
+    for mode, fname, w in ((qz.NVFP4_PER_TENSOR_GIVEN, "given amax", None),
+                           (qz.NVFP4_PER_TENSOR_COMPUTE, "computed amax (one L2-chunked launch)", ws),
+                           (qz.NVFP4_PER_TENSOR_COMPUTE, "computed amax (amax pass + quantize pass)", None)):
         ents = qz.alloc_outputs(list(stack.unbind(0)), qz.FMT_NVFP4, qz.SF_SWIZZLED, mode)
         for e in ents:
             e.amax.fill_(0.1)
         tab = qz.ExpertTable(ents)
-        ms = _time_graph(lambda m=mode: qz.quantize_grouped_nvfp4(tab, m, qz.SF_SWIZZLED), reps=5)
+        ms = _time_graph(lambda m=mode, w=w: qz.quantize_grouped_nvfp4(tab, m, qz.SF_SWIZZLED, workspace=w), reps=5)
         nsf = qz.sf_bytes(rows, cols, qz.FMT_NVFP4, qz.SF_SWIZZLED)
         nbytes = cfg["experts"] * (rows * cols * 2 + rows * cols // 2 + nsf + 4)
         rec(f"Qwen3-30B-A3B gate_up [1536, 2048] x128 experts, NVFP4 {fname}, swizzled, one call", nbytes, ms,
-            1 if mode == qz.NVFP4_PER_TENSOR_GIVEN else 3)
+            1 if mode == qz.NVFP4_PER_TENSOR_GIVEN else (2 if w is not None else 3))
         del ents, tab
     del stack
     torch.cuda.empty_cache()
@@ -523,6 +526,7 @@ def _extra_large(qz, device, rec):
     for proj, shape in (("gate_up", cfg["gate_up"]), ("down", cfg["down"])):
         stack = synth.expert_stack(cfg["experts"], shape, cfg["std"], seed=cfg["seed"], device=device)
         rows, cols = shape
+        ws = qz.alloc_workspace(cfg["experts"], device)
         for fmt, mode, fname in ((qz.FMT_MXFP8, None, "MXFP8"), (qz.FMT_NVFP4, qz.NVFP4_PER_TENSOR_GIVEN, "NVFP4 given amax"),
                                  (qz.FMT_NVFP4, qz.NVFP4_PER_TENSOR_COMPUTE, "NVFP4 computed amax")):
             ents = qz.alloc_outputs(list(stack.unbind(0)), fmt, qz.SF_SWIZZLED,
@@ -534,13 +538,14 @@ def _extra_large(qz, device, rec):
             if fmt == qz.FMT_MXFP8:
                 fn = lambda: qz.quantize_grouped_mxfp8(tab, qz.SF_SWIZZLED)  # noqa: E731
             else:
-                fn = lambda m=mode: qz.quantize_grouped_nvfp4(tab, m, qz.SF_SWIZZLED)  # noqa: E731
+                fn = lambda m=mode: qz.quantize_grouped_nvfp4(  # noqa: E731
+                    tab, m, qz.SF_SWIZZLED, workspace=ws if m == qz.NVFP4_PER_TENSOR_COMPUTE else None)
             ms = _time_graph(fn, reps=5)
             nsf = qz.sf_bytes(rows, cols, fmt, qz.SF_SWIZZLED)
             qb = rows * cols if fmt == qz.FMT_MXFP8 else rows * cols // 2
             nbytes = cfg["experts"] * (rows * cols * 2 + qb + nsf + (4 if fmt == qz.FMT_NVFP4 else 0))
             rec(f"Qwen3-235B-A22B {proj} {list(shape)} x128 experts, {fname}, swizzled", nbytes, ms,
-                1 if mode != qz.NVFP4_PER_TENSOR_COMPUTE else 3)
+                1 if mode != qz.NVFP4_PER_TENSOR_COMPUTE else 2)
             del ents, tab
         del stack
         torch.cuda.empty_cache()

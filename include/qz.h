@@ -131,10 +131,21 @@ typedef struct qz_sf_pair {
 
 /* Optional launch controls; pass NULL for the defaults. */
 typedef struct qz_launch_opts {
-    unsigned int *d_err; /* device word; kernels OR QZ_DERR_* bits into it (never clear it) */
-    int max_ctas;        /* 0: one wave of resident CTAs on every SM; > 0: cap on the grid.
-                            The results do not depend on it. */
+    unsigned int *d_err;    /* device word; kernels OR QZ_DERR_* bits into it (never clear it) */
+    int max_ctas;           /* 0: one wave of resident CTAs on every SM; > 0: cap on the grid.
+                               The results do not depend on it. */
+    void *d_workspace;      /* optional device scratch for QZ_NVFP4_PER_TENSOR_COMPUTE: with
+                               at least qz_workspace_bytes(n_experts) bytes (4-byte aligned),
+                               the call runs one L2-chunked launch instead of an amax pass
+                               and a quantize pass over HBM.  The call zeroes it first (in
+                               stream order); calls sharing a workspace must not overlap. */
+    size_t workspace_bytes; /* size of d_workspace in bytes */
 } qz_launch_opts;
+
+/* Bytes of device scratch qz_quantize_grouped_nvfp4 uses for
+ * QZ_NVFP4_PER_TENSOR_COMPUTE when given a workspace; 0 for n_experts outside
+ * [1, QZ_MAX_EXPERTS]. */
+size_t qz_workspace_bytes(int n_experts);
 
 /* Bytes of one expert's SF region: rows * (cols/block) for the linear layout,
  * pad(rows,128) * pad(cols/block,4) for the swizzled one, 0 when rows == 0.
@@ -159,8 +170,14 @@ qz_status qz_quantize_grouped_mxfp8(const qz_expert *d_table, int n_experts, int
  * scale, S = RN32(1 / g) (0 if g == 0) the encode scale; per 16-element block
  * with amax b: scale s = e4m3(RN32(RN32(b / 6) * S)) (0 if b == 0); payload
  * q = e2m1(RN32(x * r)), r = FTZ(RN32(S / s)) (0 if s == 0).
- * PER_TENSOR_COMPUTE runs an amax pass before the quantize pass (three
- * launches in stream order); PER_ROW reads each row once.
+ * PER_TENSOR_COMPUTE without a workspace runs a clear, an amax pass and the
+ * quantize pass (three launches in stream order, the input read twice from
+ * HBM); with opts->d_workspace it runs one launch that takes each expert's
+ * amax chunk by chunk and quantizes the chunk while its input is still in L2
+ * (plus a memset of the workspace).  PER_ROW reads each row once.
+ * Errors as below, plus QZ_ERR_INVALID_ARG for a workspace smaller than
+ * qz_workspace_bytes(n_experts) and QZ_ERR_ALIGNMENT for one not 4-byte
+ * aligned.
  * Errors as for qz_quantize_grouped_mxfp8, plus QZ_ERR_INVALID_ARG for an
  * unknown mode. */
 qz_status qz_quantize_grouped_nvfp4(const qz_expert *d_table, int n_experts, int mode, int layout,

@@ -37,6 +37,7 @@ EXPORTED = (
     "qz_swizzle_scales",
     "qz_status_string",
     "qz_version",
+    "qz_workspace_bytes",
 )
 
 
@@ -58,7 +59,8 @@ class _SfPair(ctypes.Structure):
 
 
 class _Opts(ctypes.Structure):
-    _fields_ = [("d_err", ctypes.c_void_p), ("max_ctas", ctypes.c_int)]
+    _fields_ = [("d_err", ctypes.c_void_p), ("max_ctas", ctypes.c_int), ("d_workspace", ctypes.c_void_p),
+                ("workspace_bytes", ctypes.c_size_t)]
 
 
 assert ctypes.sizeof(_Expert) == 56 and ctypes.sizeof(_SfPair) == 32
@@ -92,6 +94,8 @@ def load(path: str = LIB_PATH):
         lib.qz_status_string.argtypes = [I]
         lib.qz_version.restype = I
         lib.qz_version.argtypes = []
+        lib.qz_workspace_bytes.restype = ctypes.c_size_t
+        lib.qz_workspace_bytes.argtypes = [I]
         _lib = lib
         return lib
 
@@ -111,12 +115,25 @@ def _stream_ptr(stream) -> ctypes.c_void_p:
     return ctypes.c_void_p(int(stream.cuda_stream) if hasattr(stream, "cuda_stream") else int(stream))
 
 
-def _opts(err: Optional[torch.Tensor], max_ctas: int):
-    if err is None and not max_ctas:
+def _opts(err: Optional[torch.Tensor], max_ctas: int, workspace: Optional[torch.Tensor] = None):
+    if err is None and not max_ctas and workspace is None:
         return None
     if err is not None:
         assert err.dtype in (torch.int32, torch.uint32) and err.is_cuda and err.numel() >= 1
-    return ctypes.byref(_Opts(ctypes.c_void_p(err.data_ptr() if err is not None else 0), int(max_ctas)))
+    ws_ptr = workspace.data_ptr() if workspace is not None else 0
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    return ctypes.byref(_Opts(ctypes.c_void_p(err.data_ptr() if err is not None else 0), int(max_ctas),
+                              ctypes.c_void_p(ws_ptr), ctypes.c_size_t(ws_bytes)))
+
+
+def workspace_bytes(n_experts: int) -> int:
+    """Device scratch for the single-launch computed-amax NVFP4 path."""
+    return int(load().qz_workspace_bytes(int(n_experts)))
+
+
+def alloc_workspace(n_experts: int, device=None) -> torch.Tensor:
+    return torch.empty(max(workspace_bytes(n_experts), 4), dtype=torch.uint8,
+                       device=device if device is not None else "cuda")
 
 
 def _ptr(t: Optional[torch.Tensor]) -> int:
@@ -200,9 +217,10 @@ def quantize_grouped_mxfp8(table: ExpertTable, layout: int, stream=None, err=Non
            "qz_quantize_grouped_mxfp8")
 
 
-def quantize_grouped_nvfp4(table: ExpertTable, mode: int, layout: int, stream=None, err=None, max_ctas: int = 0):
+def quantize_grouped_nvfp4(table: ExpertTable, mode: int, layout: int, stream=None, err=None, max_ctas: int = 0,
+                           workspace: Optional[torch.Tensor] = None):
     _check(load().qz_quantize_grouped_nvfp4(ctypes.c_void_p(table.ptr), table.n, int(mode), int(layout),
-                                            _stream_ptr(stream), _opts(err, max_ctas)),
+                                            _stream_ptr(stream), _opts(err, max_ctas, workspace)),
            "qz_quantize_grouped_nvfp4")
 
 
@@ -243,7 +261,7 @@ def alloc_outputs(xs: Sequence[torch.Tensor], fmt: int, layout: int, mode: int =
 
 
 def quantize_experts(xs: Sequence[torch.Tensor], fmt: int, layout: int, mode: int = NVFP4_PER_ROW,
-                     amax_in: Optional[Sequence[float]] = None, stream=None):
+                     amax_in: Optional[Sequence[float]] = None, stream=None, workspace: Optional[torch.Tensor] = None):
     """Quantize a list of bf16 experts in one launch; returns the entries with
     q, sf (trimmed to the region size) and amax filled."""
     entries = alloc_outputs(xs, fmt, layout, mode)
@@ -254,7 +272,7 @@ def quantize_experts(xs: Sequence[torch.Tensor], fmt: int, layout: int, mode: in
     if fmt == FMT_MXFP8:
         quantize_grouped_mxfp8(table, layout, stream)
     else:
-        quantize_grouped_nvfp4(table, mode, layout, stream)
+        quantize_grouped_nvfp4(table, mode, layout, stream, workspace=workspace)
     for e in entries:
         rows, cols = e.x.shape
         e.sf = e.sf[: sf_bytes(rows, cols, fmt, layout)]

@@ -20,17 +20,20 @@ cudaError_t launch_rmsnorm_quant(const uint16_t* x, const uint16_t* r, const uin
                                  int64_t H, uint16_t* y, uint16_t* h, int fmt, uint8_t* q, uint8_t* sf, int layout,
                                  const float* amax, cudaStream_t s, bool latency_mode);
 int grouped_blocks_per_sm(int which, int n);
+size_t workspace_bytes(int n);
+cudaError_t launch_nvfp4_compute_l2(const qz_expert* table, int n, int layout, int grid, unsigned* ws,
+                                    cudaStream_t s, unsigned* d_err);
 int rows_blocks_per_sm(int n);
 }  // namespace qz
 
 namespace {
 
 constexpr int kMaxDevices = 64;
-constexpr int kKinds = 5;  // mxfp8, nvfp4 tile, swizzle, amax, rows
+constexpr int kKinds = 6;  // mxfp8, nvfp4 tile, swizzle, amax, rows, computed-amax L2 path
 
 struct DeviceLimits {
     int sms = 0;
-    int per_sm[kKinds] = {0, 0, 0, 0, 0};
+    int per_sm[kKinds] = {0, 0, 0, 0, 0, 0};
 };
 
 std::mutex g_mu;
@@ -119,8 +122,15 @@ qz_status qz_quantize_grouped_nvfp4(const qz_expert* d_table, int n_experts, int
     if (!valid_layout(layout)) return QZ_ERR_INVALID_ARG;
     if (mode != QZ_NVFP4_PER_TENSOR_GIVEN && mode != QZ_NVFP4_PER_TENSOR_COMPUTE && mode != QZ_NVFP4_PER_ROW)
         return QZ_ERR_INVALID_ARG;
+    if (mode == QZ_NVFP4_PER_TENSOR_COMPUTE && opts && opts->d_workspace) {
+        if (n_experts > 0 && opts->workspace_bytes < qz::workspace_bytes(n_experts)) return QZ_ERR_INVALID_ARG;
+        if (!aligned(opts->d_workspace, 4)) return QZ_ERR_ALIGNMENT;
+    }
     if (n_experts == 0) return QZ_OK;
     cudaStream_t s = (cudaStream_t)stream;
+    if (mode == QZ_NVFP4_PER_TENSOR_COMPUTE && opts && opts->d_workspace)
+        return from_cuda(qz::launch_nvfp4_compute_l2(d_table, n_experts, layout, wave_grid(5, opts),
+                                                     static_cast<unsigned*>(opts->d_workspace), s, err_word(opts)));
     if (mode == QZ_NVFP4_PER_ROW)
         return from_cuda(qz::launch_nvfp4_rows(d_table, n_experts, layout, wave_grid(4, opts), s, err_word(opts)));
     return from_cuda(qz::launch_nvfp4_tensor(d_table, n_experts, layout, mode == QZ_NVFP4_PER_TENSOR_COMPUTE,
@@ -157,6 +167,11 @@ qz_status qz_swizzle_scales(const qz_sf_pair* d_table, int n, void* stream, cons
     if (st != QZ_OK) return st;
     if (n == 0) return QZ_OK;
     return from_cuda(qz::launch_swizzle(d_table, n, wave_grid(2, opts), (cudaStream_t)stream, err_word(opts)));
+}
+
+size_t qz_workspace_bytes(int n_experts) {
+    if (n_experts < 1 || n_experts > QZ_MAX_EXPERTS) return 0;
+    return qz::workspace_bytes(n_experts);
 }
 
 const char* qz_status_string(qz_status status) {

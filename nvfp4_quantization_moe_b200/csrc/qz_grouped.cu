@@ -292,6 +292,165 @@ __global__ void __launch_bounds__(kThreads, 3) amax_grouped_kernel(const qz_expe
 }
 
 // ---------------------------------------------------------------------------
+// NVFP4 with a computed per-tensor amax in one launch (L2-chunked)
+//
+// The experts are cut into chunks of consecutive experts holding about
+// kChunkTiles tiles (~32 MB of bf16).  Work items are tiles, fetched from an
+// atomic counter in the order  A(0) | A(1) Q(0) | A(2) Q(1) | ... | Q(last):
+// an A item folds its tile's amax into its expert's slot (atomic max) and
+// counts itself done for its chunk; a Q item quantizes a tile of the previous
+// chunk once that chunk's A items are all done, re-reading its input from L2
+// where the A pass left it.  Every item waits only on items fetched before
+// it, and an A item never waits, so all items finish whatever the number of
+// resident CTAs; the wait is still bounded (QZ_DERR_TIMEOUT).
+//
+// Workspace (caller's device memory, zeroed by the call):
+//   ws[0] next item, ws[8 + k] done A tiles of chunk k, then one amax word per
+//   expert (bf16 magnitude bits << 16).
+// ---------------------------------------------------------------------------
+
+constexpr int kChunkTiles = 1024;      // ~32 MB of bf16 input per chunk
+constexpr int kMaxChunks = 4096;
+constexpr int kWsHeader = 8;
+
+__host__ __device__ constexpr size_t workspace_words(int n) { return (size_t)kWsHeader + kMaxChunks + (size_t)n; }
+
+template <int LAYOUT>
+__global__ void __launch_bounds__(kThreads, 3) nvfp4_compute_l2_kernel(const qz_expert* __restrict__ table, int n,
+                                                                       unsigned* __restrict__ ws, unsigned* d_err) {
+    using G = TileGeo<QZ_FMT_NVFP4>;
+    extern __shared__ int s_dyn[];
+    int* s_prefix = s_dyn;              // n + 1: first tile of each expert
+    int* s_cf = s_dyn + (n + 1);        // nchunks + 1: first tile of each chunk
+    int* s_seg = s_cf + (kMaxChunks + 1);  // nchunks + 2: first item of each segment
+    __shared__ long long s_scan[33];
+    __shared__ __align__(16) uint8_t s_sf[kThreads / 32][64 * G::kSfTiles];
+    __shared__ float s_inv[16];
+    __shared__ int s_item[2];
+    __shared__ unsigned s_amax[2];
+    __shared__ uint32_t s_wmax[kThreads / 32];
+    fill_inv_table(s_inv);
+    const int total = block_prefix(n, s_prefix, s_scan, TableTiles<QZ_FMT_NVFP4, LAYOUT, true>{table, d_err}, d_err);
+    if (total == 0) return;
+    const int tpc = max(kChunkTiles, (total + kMaxChunks - 1) / kMaxChunks);  // tiles per chunk
+    const int nchunks = (total + tpc - 1) / tpc;
+    // chunk k starts at the first expert whose first tile is >= k * tpc
+    for (int k = threadIdx.x; k <= nchunks; k += blockDim.x) {
+        const int target = k * tpc;
+        int lo = 0, hi = n;  // first e in [0, n] with s_prefix[e] >= target (s_prefix[n] = total)
+        while (lo < hi) {
+            const int mid = (lo + hi) >> 1;
+            if (s_prefix[mid] >= target) hi = mid; else lo = mid + 1;
+        }
+        s_cf[k] = s_prefix[lo];
+    }
+    __syncthreads();
+    // segment s = A(s) then Q(s-1); it starts at item cf[s] + cf[s-1]
+    for (int k = threadIdx.x; k <= nchunks + 1; k += blockDim.x) {
+        const int a = k <= nchunks ? s_cf[k] : total;
+        const int b = k >= 1 ? s_cf[k - 1] : 0;
+        s_seg[k] = a + b;
+    }
+    unsigned* next_item = ws;
+    unsigned* done = ws + kWsHeader;
+    unsigned* amax_ws = ws + kWsHeader + kMaxChunks;
+    const int items = 2 * total;
+    const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) s_item[0] = (int)atomicAdd(next_item, 1u);
+    __syncthreads();
+
+    // decode item j: tile index, whether it is an A item, its chunk
+    auto decode = [&](int j, int& tile, bool& is_a, int& chunk) {
+        int lo = 0, hi = nchunks + 1;  // last s with s_seg[s] <= j
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (s_seg[mid] <= j) lo = mid; else hi = mid - 1;
+        }
+        const int off = j - s_seg[lo];
+        const int a_len = lo < nchunks ? s_cf[lo + 1] - s_cf[lo] : 0;
+        is_a = off < a_len;
+        chunk = is_a ? lo : lo - 1;
+        tile = is_a ? s_cf[lo] + off : s_cf[lo - 1] + (off - a_len);
+    };
+
+    int it = 0;
+    int j = s_item[0];
+    if (j >= items) return;
+    int tile, chunk;
+    bool is_a;
+    decode(j, tile, is_a, chunk);
+    TileRef cur = tile_ref<QZ_FMT_NVFP4, LAYOUT>(table, s_prefix, n, tile, w, lane);
+    uint32_t v[G::kPasses][G::kWords];
+#pragma unroll
+    for (int p = 0; p < G::kPasses; ++p) tile_load<QZ_FMT_NVFP4>(cur, p, v[p]);
+    bool ok = true;
+    for (;; ++it) {
+        // fetch the next item while this one's dependency resolves
+        unsigned nxt_raw = 0;
+        if (threadIdx.x == 0) {
+            nxt_raw = atomicAdd(next_item, 1u);
+            if (!is_a) {
+                // wait until every A item of this tile's chunk is done
+                const unsigned need = (unsigned)(s_cf[chunk + 1] - s_cf[chunk]);
+                const long long t0 = clock64();
+                while (ld_acquire_gpu(done + chunk) < need) {
+                    if (clock64() - t0 > (1LL << 31)) {
+                        if (d_err) atomicOr(d_err, QZ_DERR_TIMEOUT);
+                        ok = false;
+                        break;
+                    }
+                }
+                s_amax[it & 1] = ld_acquire_gpu(amax_ws + cur.expert);
+            }
+            s_item[(it + 1) & 1] = (int)nxt_raw;
+        }
+        __syncthreads();
+        const int jn = s_item[(it + 1) & 1];
+        const bool more = jn < items;
+        int tile_n = 0, chunk_n = 0;
+        bool is_a_n = false;
+        if (more) decode(jn, tile_n, is_a_n, chunk_n);
+        const TileRef nxt = more ? tile_ref<QZ_FMT_NVFP4, LAYOUT>(table, s_prefix, n, tile_n, w, lane) : cur;
+        if (is_a) {
+            uint32_t m = 0;
+#pragma unroll
+            for (int p = 0; p < G::kPasses; ++p) {
+                m = max(m, absmax_words<G::kWords>(v[p]));
+                if (more) tile_load<QZ_FMT_NVFP4>(nxt, p, v[p]);
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+            if (lane == 0) s_wmax[w] = m;
+            __syncthreads();
+            if (threadIdx.x == 0) {
+                uint32_t mm = 0;
+                for (int k = 0; k < kThreads / 32; ++k) mm = max(mm, s_wmax[k]);
+                atomicMax(amax_ws + cur.expert, mm << 16);
+                __threadfence();
+                atomicAdd(done + chunk, 1u);
+            }
+        } else {
+            const unsigned abits = s_amax[it & 1];
+            const float A = __uint_as_float(abits);
+            const float S = nvfp4_encode_scale(A);
+#pragma unroll
+            for (int p = 0; p < G::kPasses; ++p) {
+                tile_pass<QZ_FMT_NVFP4, LAYOUT>(cur, p, lane, v[p], S, s_sf[w], s_inv);
+                if (more) tile_load<QZ_FMT_NVFP4>(nxt, p, v[p]);
+            }
+            if (LAYOUT == QZ_SF_SWIZZLED_128x4) tile_flush_sf<QZ_FMT_NVFP4>(cur, w, lane, s_sf[w]);
+            if (threadIdx.x == 0) *const_cast<float*>(cur.amax) = A;
+        }
+        if (!more) break;
+        cur = nxt;
+        is_a = is_a_n;
+        chunk = chunk_n;
+        j = jn;
+    }
+    (void)ok;
+}
+
+// ---------------------------------------------------------------------------
 // standalone linear -> swizzled conversion
 // ---------------------------------------------------------------------------
 
@@ -369,6 +528,23 @@ cudaError_t launch_nvfp4_tensor(const qz_expert* table, int n, int layout, bool 
     return cudaGetLastError();
 }
 
+size_t workspace_bytes(int n) { return workspace_words(n) * sizeof(unsigned); }
+
+size_t compute_l2_smem(int n) { return (size_t)(n + 1 + kMaxChunks + 1 + kMaxChunks + 2) * sizeof(int); }
+
+// One launch of the L2-chunked computed-amax path on a zeroed workspace.
+cudaError_t launch_nvfp4_compute_l2(const qz_expert* table, int n, int layout, int grid, unsigned* ws,
+                                    cudaStream_t s, unsigned* d_err) {
+    cudaError_t e = cudaMemsetAsync(ws, 0, workspace_bytes(n), s);
+    if (e != cudaSuccess) return e;
+    const size_t smem = compute_l2_smem(n);
+    if (layout == QZ_SF_SWIZZLED_128x4)
+        nvfp4_compute_l2_kernel<QZ_SF_SWIZZLED_128x4><<<grid, kThreads, smem, s>>>(table, n, ws, d_err);
+    else
+        nvfp4_compute_l2_kernel<QZ_SF_LINEAR><<<grid, kThreads, smem, s>>>(table, n, ws, d_err);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_swizzle(const qz_sf_pair* table, int n, int grid, cudaStream_t s, unsigned* d_err) {
     swizzle_kernel<<<grid, kThreads, prefix_smem(n), s>>>(table, n, d_err);
     return cudaGetLastError();
@@ -382,7 +558,14 @@ int grouped_blocks_per_sm(int which, int n) {
         case 0: cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, grouped_tile_kernel<QZ_FMT_MXFP8, QZ_SF_SWIZZLED_128x4>, kThreads, smem); break;
         case 1: cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, grouped_tile_kernel<QZ_FMT_NVFP4, QZ_SF_SWIZZLED_128x4>, kThreads, smem); break;
         case 2: cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, swizzle_kernel, kThreads, smem); break;
-        default: cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, amax_grouped_kernel<QZ_SF_SWIZZLED_128x4>, kThreads, smem); break;
+        case 3: cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, amax_grouped_kernel<QZ_SF_SWIZZLED_128x4>, kThreads, smem); break;
+        default: {
+            const size_t big = compute_l2_smem(n);
+            cudaFuncSetAttribute(nvfp4_compute_l2_kernel<QZ_SF_SWIZZLED_128x4>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)big);
+            cudaFuncSetAttribute(nvfp4_compute_l2_kernel<QZ_SF_LINEAR>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)big);
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, nvfp4_compute_l2_kernel<QZ_SF_SWIZZLED_128x4>, kThreads, big);
+            break;
+        }
     }
     return b > 0 ? b : 1;
 }

@@ -68,6 +68,13 @@ def test_host_errors_without_gpu(lib):
     assert lib.qz_quantize_grouped_nvfp4(P(0x1000), 2, 7, 0, None, None) == qz.QZ_ERR_INVALID_ARG
     assert lib.qz_quantize_grouped_nvfp4(None, 0, 2, 1, None, None) == qz.QZ_OK
     assert lib.qz_swizzle_scales(None, 1, None, None) == qz.QZ_ERR_INVALID_ARG
+    # a workspace smaller than qz_workspace_bytes is refused before any launch
+    small = qz.binding._Opts(None, 0, P(0x10000), ctypes.c_size_t(16))
+    assert lib.qz_quantize_grouped_nvfp4(P(0x1000), 4, 1, 1, None, ctypes.byref(small)) == qz.QZ_ERR_INVALID_ARG
+    odd = qz.binding._Opts(None, 0, P(0x10002), ctypes.c_size_t(qz.workspace_bytes(4)))
+    assert lib.qz_quantize_grouped_nvfp4(P(0x1000), 4, 1, 1, None, ctypes.byref(odd)) == qz.QZ_ERR_ALIGNMENT
+    assert qz.workspace_bytes(0) == 0 and qz.workspace_bytes(qz.MAX_EXPERTS + 1) == 0
+    assert qz.workspace_bytes(128) >= 4 * (128 + 1)
     assert lib.qz_swizzle_scales(None, 0, None, None) == qz.QZ_OK
     a = P(0x10000)
 

@@ -229,3 +229,53 @@ def test_strided_rows_all_modes(mode):
     amax_in = [float(x.float().abs().max()) for x in xs] if m == qz.NVFP4_PER_TENSOR_GIVEN else None
     got = run_nvfp4(xs, qz.SF_SWIZZLED, m, amax_in)
     check([x.contiguous() for x in xs], qz.SF_SWIZZLED, m, got, amax_in)
+
+
+def run_compute_l2(xs, layout, **kw):
+    """Computed per-tensor amax through the single-launch L2-chunked path."""
+    entries, keep = guarded_entries(xs, qz.FMT_NVFP4, layout, qz.NVFP4_PER_TENSOR_COMPUTE)
+    ws = qz.alloc_workspace(len(xs))
+    ws.fill_(0xFF)                       # the call zeroes what it needs
+    qz.quantize_grouped_nvfp4(qz.ExpertTable(entries), qz.NVFP4_PER_TENSOR_COMPUTE, layout, workspace=ws, **kw)
+    torch.cuda.synchronize()
+    out = []
+    for (q, sf, a), x in zip(keep, xs):
+        assert q.guards_intact() and sf.guards_intact() and a.guards_intact()
+        rows = x.shape[0]
+        out.append((q.host().reshape(rows, -1) if rows else q.host(), sf.host(),
+                    a.view.view(torch.float32).cpu().numpy()))
+    return out
+
+
+@pytest.mark.parametrize("layout", LAYOUTS)
+def test_compute_l2_path_parity(layout):
+    xs = [synth.blockwise_scaled(s, 16, seed=400 + i, lo=-20, hi=8).cuda() for i, s in enumerate(SHAPES)]
+    xs.insert(2, torch.zeros((0, 64), dtype=torch.bfloat16, device="cuda"))      # an empty expert
+    check(xs, layout, qz.NVFP4_PER_TENSOR_COMPUTE, run_compute_l2(xs, layout))
+
+
+def test_compute_l2_many_chunks_and_grid_invariance():
+    """3072 tiles -> three ~1024-tile chunks; one CTA, a few, and a full wave
+    give the same bytes (a single CTA exercises every wait in order)."""
+    xs = [synth.normal_bf16((1024, 1024), std=0.02, seed=500 + i).cuda() for i in range(48)]
+    xs[7].zero_()
+    base = run_compute_l2(xs, qz.SF_SWIZZLED)
+    for ctas in (1, 37):
+        other = run_compute_l2(xs, qz.SF_SWIZZLED, max_ctas=ctas)
+        for a, b in zip(base, other):
+            assert all(np.array_equal(u, v) for u, v in zip(a, b))
+    sample = [0, 7, 23, 47]
+    check([xs[i] for i in sample], qz.SF_SWIZZLED, qz.NVFP4_PER_TENSOR_COMPUTE, [base[i] for i in sample])
+    # and the same as the three-launch path
+    three = run_nvfp4(xs, qz.SF_SWIZZLED, qz.NVFP4_PER_TENSOR_COMPUTE)
+    for a, b in zip(base, three):
+        assert all(np.array_equal(u, v) for u, v in zip(a, b))
+
+
+def test_compute_l2_workspace_too_small_is_rejected():
+    xs = [synth.normal_bf16((64, 64), seed=1).cuda()]
+    entries, keep = guarded_entries(xs, qz.FMT_NVFP4, qz.SF_SWIZZLED, qz.NVFP4_PER_TENSOR_COMPUTE)
+    ws = torch.zeros(qz.workspace_bytes(1) - 4, dtype=torch.uint8, device="cuda")
+    with pytest.raises(qz.QzError):
+        qz.quantize_grouped_nvfp4(qz.ExpertTable(entries), qz.NVFP4_PER_TENSOR_COMPUTE, qz.SF_SWIZZLED, workspace=ws)
+    assert torch.all(keep[0][0].raw == 0xA5)
