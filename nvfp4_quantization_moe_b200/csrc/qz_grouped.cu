@@ -295,39 +295,49 @@ __global__ void __launch_bounds__(kThreads, 3) amax_grouped_kernel(const qz_expe
 // NVFP4 with a computed per-tensor amax in one launch (L2-chunked)
 //
 // The experts are cut into chunks of consecutive experts holding about
-// kChunkTiles tiles (~32 MB of bf16).  Work items are tiles, fetched from an
-// atomic counter in the order  A(0) | A(1) Q(0) | A(2) Q(1) | ... | Q(last):
-// an A item folds its tile's amax into its expert's slot (atomic max) and
-// counts itself done for its chunk; a Q item quantizes a tile of the previous
-// chunk once that chunk's A items are all done, re-reading its input from L2
-// where the A pass left it.  Every item waits only on items fetched before
-// it, and an A item never waits, so all items finish whatever the number of
-// resident CTAs; the wait is still bounded (QZ_DERR_TIMEOUT).
+// kChunkTiles tiles (~16 MB of bf16).  Work items are runs of up to
+// kItemTiles tiles of one chunk, fetched from an atomic counter in the order
+// A(0) | A(1) Q(0) | A(2) Q(1) | ... | Q(last): an A item folds its tiles'
+// amax into their experts' slots (atomic max) and adds its tile count to its
+// chunk's done counter; a Q item quantizes tiles of the previous chunk once
+// that chunk's A tiles are all done, re-reading the input from L2 where the A
+// pass left it.  Every item waits only on items fetched before it and A items
+// never wait, so all items finish whatever the number of resident CTAs; the
+// wait is still bounded (QZ_DERR_TIMEOUT).  The item index is fetched two
+// items ahead so the atomic's latency stays off the critical path.
 //
 // Workspace (caller's device memory, zeroed by the call):
 //   ws[0] next item, ws[8 + k] done A tiles of chunk k, then one amax word per
 //   expert (bf16 magnitude bits << 16).
 // ---------------------------------------------------------------------------
 
-constexpr int kChunkTiles = 1024;      // ~32 MB of bf16 input per chunk
+constexpr int kChunkTiles = 512;       // ~16 MB of bf16 input per chunk
+constexpr int kItemTiles = 4;          // tiles per work item
 constexpr int kMaxChunks = 4096;
 constexpr int kWsHeader = 8;
 
 __host__ __device__ constexpr size_t workspace_words(int n) { return (size_t)kWsHeader + kMaxChunks + (size_t)n; }
+
+struct ItemRef {
+    int first_tile;  // first tile of the run
+    int ntiles;      // tiles in the run (1..kItemTiles)
+    int chunk;
+    bool is_a;
+};
 
 template <int LAYOUT>
 __global__ void __launch_bounds__(kThreads, 3) nvfp4_compute_l2_kernel(const qz_expert* __restrict__ table, int n,
                                                                        unsigned* __restrict__ ws, unsigned* d_err) {
     using G = TileGeo<QZ_FMT_NVFP4>;
     extern __shared__ int s_dyn[];
-    int* s_prefix = s_dyn;              // n + 1: first tile of each expert
-    int* s_cf = s_dyn + (n + 1);        // nchunks + 1: first tile of each chunk
+    int* s_prefix = s_dyn;                 // n + 1: first tile of each expert
+    int* s_cf = s_dyn + (n + 1);           // nchunks + 1: first tile of each chunk
     int* s_seg = s_cf + (kMaxChunks + 1);  // nchunks + 2: first item of each segment
     __shared__ long long s_scan[33];
     __shared__ __align__(16) uint8_t s_sf[kThreads / 32][64 * G::kSfTiles];
     __shared__ float s_inv[16];
-    __shared__ int s_item[2];
-    __shared__ unsigned s_amax[2];
+    __shared__ int s_item[4];
+    __shared__ unsigned s_ok[2];
     __shared__ uint32_t s_wmax[kThreads / 32];
     fill_inv_table(s_inv);
     const int total = block_prefix(n, s_prefix, s_scan, TableTiles<QZ_FMT_NVFP4, LAYOUT, true>{table, d_err}, d_err);
@@ -345,109 +355,119 @@ __global__ void __launch_bounds__(kThreads, 3) nvfp4_compute_l2_kernel(const qz_
         s_cf[k] = s_prefix[lo];
     }
     __syncthreads();
-    // segment s = A(s) then Q(s-1); it starts at item cf[s] + cf[s-1]
-    for (int k = threadIdx.x; k <= nchunks + 1; k += blockDim.x) {
-        const int a = k <= nchunks ? s_cf[k] : total;
-        const int b = k >= 1 ? s_cf[k - 1] : 0;
-        s_seg[k] = a + b;
+    // items of chunk k: ceil(T(k) / kItemTiles); segment s = A(s) then Q(s-1)
+    auto chunk_items = [&](int k) { return (s_cf[k + 1] - s_cf[k] + kItemTiles - 1) / kItemTiles; };
+    if (threadIdx.x == 0) {
+        int run = 0, prev = 0;
+        for (int k = 0; k <= nchunks; ++k) {
+            s_seg[k] = run;
+            const int a = k < nchunks ? chunk_items(k) : 0;
+            run += a + prev;
+            prev = a;
+        }
+        s_seg[nchunks + 1] = run;
     }
     unsigned* next_item = ws;
     unsigned* done = ws + kWsHeader;
     unsigned* amax_ws = ws + kWsHeader + kMaxChunks;
-    const int items = 2 * total;
-    const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    if (threadIdx.x == 0) s_item[0] = (int)atomicAdd(next_item, 1u);
+    if (threadIdx.x == 0) {
+        s_item[0] = (int)atomicAdd(next_item, 1u);
+        s_item[1] = (int)atomicAdd(next_item, 1u);
+    }
     __syncthreads();
+    const int items = s_seg[nchunks + 1];
+    const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-    // decode item j: tile index, whether it is an A item, its chunk
-    auto decode = [&](int j, int& tile, bool& is_a, int& chunk) {
-        int lo = 0, hi = nchunks + 1;  // last s with s_seg[s] <= j
+    auto decode = [&](int j) {
+        int lo = 0, hi = nchunks;  // last s with s_seg[s] <= j
         while (lo < hi) {
             const int mid = (lo + hi + 1) >> 1;
             if (s_seg[mid] <= j) lo = mid; else hi = mid - 1;
         }
         const int off = j - s_seg[lo];
-        const int a_len = lo < nchunks ? s_cf[lo + 1] - s_cf[lo] : 0;
-        is_a = off < a_len;
-        chunk = is_a ? lo : lo - 1;
-        tile = is_a ? s_cf[lo] + off : s_cf[lo - 1] + (off - a_len);
+        const int a_items = lo < nchunks ? chunk_items(lo) : 0;
+        ItemRef r;
+        r.is_a = off < a_items;
+        r.chunk = r.is_a ? lo : lo - 1;
+        const int idx = r.is_a ? off : off - a_items;
+        r.first_tile = s_cf[r.chunk] + idx * kItemTiles;
+        r.ntiles = min(kItemTiles, s_cf[r.chunk + 1] - r.first_tile);
+        return r;
     };
 
-    int it = 0;
     int j = s_item[0];
     if (j >= items) return;
-    int tile, chunk;
-    bool is_a;
-    decode(j, tile, is_a, chunk);
-    TileRef cur = tile_ref<QZ_FMT_NVFP4, LAYOUT>(table, s_prefix, n, tile, w, lane);
+    ItemRef item = decode(j);
+    TileRef cur = tile_ref<QZ_FMT_NVFP4, LAYOUT>(table, s_prefix, n, item.first_tile, w, lane);
     uint32_t v[G::kPasses][G::kWords];
 #pragma unroll
     for (int p = 0; p < G::kPasses; ++p) tile_load<QZ_FMT_NVFP4>(cur, p, v[p]);
-    bool ok = true;
-    for (;; ++it) {
-        // fetch the next item while this one's dependency resolves
-        unsigned nxt_raw = 0;
+    for (int it = 0;; ++it) {
+        // item it is in s_item[it & 3], item it+1 in s_item[(it+1) & 3]; fetch item it+2
+        unsigned fetched = 0;
         if (threadIdx.x == 0) {
-            nxt_raw = atomicAdd(next_item, 1u);
-            if (!is_a) {
-                // wait until every A item of this tile's chunk is done
-                const unsigned need = (unsigned)(s_cf[chunk + 1] - s_cf[chunk]);
+            fetched = atomicAdd(next_item, 1u);
+            unsigned ok = 1;
+            if (!item.is_a) {
+                // wait until every A tile of this item's chunk is done
+                const unsigned need = (unsigned)(s_cf[item.chunk + 1] - s_cf[item.chunk]);
                 const long long t0 = clock64();
-                while (ld_acquire_gpu(done + chunk) < need) {
+                while (ld_acquire_gpu(done + item.chunk) < need) {
                     if (clock64() - t0 > (1LL << 31)) {
                         if (d_err) atomicOr(d_err, QZ_DERR_TIMEOUT);
-                        ok = false;
+                        ok = 0;
                         break;
                     }
                 }
-                s_amax[it & 1] = ld_acquire_gpu(amax_ws + cur.expert);
             }
-            s_item[(it + 1) & 1] = (int)nxt_raw;
+            s_ok[it & 1] = ok;
+            s_item[(it + 2) & 3] = (int)fetched;
         }
         __syncthreads();
-        const int jn = s_item[(it + 1) & 1];
-        const bool more = jn < items;
-        int tile_n = 0, chunk_n = 0;
-        bool is_a_n = false;
-        if (more) decode(jn, tile_n, is_a_n, chunk_n);
-        const TileRef nxt = more ? tile_ref<QZ_FMT_NVFP4, LAYOUT>(table, s_prefix, n, tile_n, w, lane) : cur;
-        if (is_a) {
-            uint32_t m = 0;
+        const int jn = s_item[(it + 1) & 3];
+        const bool more_items = jn < items;
+        const ItemRef nitem = more_items ? decode(jn) : item;
+        uint32_t run = 0;  // A: running max of this warp over the item's tiles of one expert
+        for (int k = 0; k < item.ntiles; ++k) {
+            const bool last = k + 1 == item.ntiles;
+            const bool more = !last || more_items;
+            const int ntile = last ? nitem.first_tile : item.first_tile + k + 1;
+            const TileRef nxt = more ? tile_ref<QZ_FMT_NVFP4, LAYOUT>(table, s_prefix, n, ntile, w, lane) : cur;
+            if (item.is_a) {
 #pragma unroll
-            for (int p = 0; p < G::kPasses; ++p) {
-                m = max(m, absmax_words<G::kWords>(v[p]));
-                if (more) tile_load<QZ_FMT_NVFP4>(nxt, p, v[p]);
-            }
+                for (int p = 0; p < G::kPasses; ++p) {
+                    run = max(run, absmax_words<G::kWords>(v[p]));
+                    if (more) tile_load<QZ_FMT_NVFP4>(nxt, p, v[p]);
+                }
+                if (last || nxt.expert != cur.expert) {
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
-            if (lane == 0) s_wmax[w] = m;
-            __syncthreads();
-            if (threadIdx.x == 0) {
-                uint32_t mm = 0;
-                for (int k = 0; k < kThreads / 32; ++k) mm = max(mm, s_wmax[k]);
-                atomicMax(amax_ws + cur.expert, mm << 16);
-                __threadfence();
-                atomicAdd(done + chunk, 1u);
-            }
-        } else {
-            const unsigned abits = s_amax[it & 1];
-            const float A = __uint_as_float(abits);
-            const float S = nvfp4_encode_scale(A);
+                    for (int o = 16; o > 0; o >>= 1) run = max(run, __shfl_xor_sync(0xFFFFFFFFu, run, o));
+                    if (lane == 0) {
+                        atomicMax(amax_ws + cur.expert, run << 16);
+                        __threadfence();
+                    }
+                    run = 0;
+                }
+            } else {
+                const float A = __uint_as_float(ld_acquire_gpu(amax_ws + cur.expert));
+                const float S = nvfp4_encode_scale(A);
 #pragma unroll
-            for (int p = 0; p < G::kPasses; ++p) {
-                tile_pass<QZ_FMT_NVFP4, LAYOUT>(cur, p, lane, v[p], S, s_sf[w], s_inv);
-                if (more) tile_load<QZ_FMT_NVFP4>(nxt, p, v[p]);
+                for (int p = 0; p < G::kPasses; ++p) {
+                    tile_pass<QZ_FMT_NVFP4, LAYOUT>(cur, p, lane, v[p], S, s_sf[w], s_inv);
+                    if (more) tile_load<QZ_FMT_NVFP4>(nxt, p, v[p]);
+                }
+                if (LAYOUT == QZ_SF_SWIZZLED_128x4) tile_flush_sf<QZ_FMT_NVFP4>(cur, w, lane, s_sf[w]);
+                if (threadIdx.x == 0) *const_cast<float*>(cur.amax) = A;
             }
-            if (LAYOUT == QZ_SF_SWIZZLED_128x4) tile_flush_sf<QZ_FMT_NVFP4>(cur, w, lane, s_sf[w]);
-            if (threadIdx.x == 0) *const_cast<float*>(cur.amax) = A;
+            cur = nxt;
         }
-        if (!more) break;
-        cur = nxt;
-        is_a = is_a_n;
-        chunk = chunk_n;
-        j = jn;
+        if (item.is_a) {
+            __syncthreads();  // every warp's atomic max (fenced) precedes the count
+            if (threadIdx.x == 0) atomicAdd(done + item.chunk, (unsigned)item.ntiles);
+        }
+        if (!more_items) break;
+        item = nitem;
     }
-    (void)ok;
 }
 
 // ---------------------------------------------------------------------------
