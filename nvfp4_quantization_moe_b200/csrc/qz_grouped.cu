@@ -296,15 +296,18 @@ __global__ void __launch_bounds__(kThreads, 3) amax_grouped_kernel(const qz_expe
 //
 // The experts are cut into chunks of consecutive experts holding about
 // kChunkTiles tiles (~16 MB of bf16).  Work items are runs of up to
-// kItemTiles tiles of one chunk, fetched from an atomic counter in the order
-// A(0) | A(1) Q(0) | A(2) Q(1) | ... | Q(last): an A item folds its tiles'
-// amax into their experts' slots (atomic max) and adds its tile count to its
-// chunk's done counter; a Q item quantizes tiles of the previous chunk once
-// that chunk's A tiles are all done, re-reading the input from L2 where the A
-// pass left it.  Every item waits only on items fetched before it and A items
-// never wait, so all items finish whatever the number of resident CTAs; the
-// wait is still bounded (QZ_DERR_TIMEOUT).  The item index is fetched two
-// items ahead so the atomic's latency stays off the critical path.
+// kItemTiles tiles of one chunk, fetched from an atomic counter in segment
+// order: segment s holds A(s) then Q(s - kLag) (the last kLag segments hold
+// only Q items).  An A item folds its tiles' amax into their experts' slots
+// (atomic max) and adds its tile count to its chunk's done counter; a Q item
+// quantizes tiles of chunk s - kLag once that chunk's A tiles are all done,
+// re-reading the input from L2 where the A pass left it.  kLag chunks of A
+// items (more than the items in flight on the whole GPU) separate a chunk's
+// A and Q items, so Q items rarely wait, while the kLag + 1 live chunks stay
+// well inside L2.  Every item waits only on items fetched before it and A
+// items never wait, so all items finish whatever the number of resident CTAs;
+// the wait is still bounded (QZ_DERR_TIMEOUT).  A CTA consumes each fetched
+// item index one item later, so the atomic's latency is hidden.
 //
 // Workspace (caller's device memory, zeroed by the call):
 //   ws[0] next item, ws[8 + k] done A tiles of chunk k, then one amax word per
@@ -312,9 +315,11 @@ __global__ void __launch_bounds__(kThreads, 3) amax_grouped_kernel(const qz_expe
 // ---------------------------------------------------------------------------
 
 constexpr int kChunkTiles = 512;       // ~16 MB of bf16 input per chunk
-constexpr int kItemTiles = 4;          // tiles per work item
+constexpr int kItemTiles = 2;          // tiles per work item
+constexpr int kLag = 2;                // chunks between a chunk's A items and its Q items
 constexpr int kMaxChunks = 4096;
 constexpr int kWsHeader = 8;
+static_assert(kLag >= 1, "Q items of a chunk must follow all of its A items");
 
 __host__ __device__ constexpr size_t workspace_words(int n) { return (size_t)kWsHeader + kMaxChunks + (size_t)n; }
 
@@ -332,7 +337,7 @@ __global__ void __launch_bounds__(kThreads, 3) nvfp4_compute_l2_kernel(const qz_
     extern __shared__ int s_dyn[];
     int* s_prefix = s_dyn;                 // n + 1: first tile of each expert
     int* s_cf = s_dyn + (n + 1);           // nchunks + 1: first tile of each chunk
-    int* s_seg = s_cf + (kMaxChunks + 1);  // nchunks + 2: first item of each segment
+    int* s_seg = s_cf + (kMaxChunks + 1);  // nchunks + kLag + 1: first item of each segment
     __shared__ long long s_scan[33];
     __shared__ __align__(16) uint8_t s_sf[kThreads / 32][64 * G::kSfTiles];
     __shared__ float s_inv[16];
@@ -355,40 +360,42 @@ __global__ void __launch_bounds__(kThreads, 3) nvfp4_compute_l2_kernel(const qz_
         s_cf[k] = s_prefix[lo];
     }
     __syncthreads();
-    // items of chunk k: ceil(T(k) / kItemTiles); segment s = A(s) then Q(s-1)
-    auto chunk_items = [&](int k) { return (s_cf[k + 1] - s_cf[k] + kItemTiles - 1) / kItemTiles; };
+    // items of chunk k: ceil(T(k) / kItemTiles); segment s = A(s) then Q(s - kLag)
+    auto chunk_items = [&](int k) {
+        return (k >= 0 && k < nchunks) ? (s_cf[k + 1] - s_cf[k] + kItemTiles - 1) / kItemTiles : 0;
+    };
+    const int nseg = nchunks + kLag;
     if (threadIdx.x == 0) {
-        int run = 0, prev = 0;
-        for (int k = 0; k <= nchunks; ++k) {
+        int run = 0;
+        for (int k = 0; k < nseg; ++k) {
             s_seg[k] = run;
-            const int a = k < nchunks ? chunk_items(k) : 0;
-            run += a + prev;
-            prev = a;
+            run += chunk_items(k) + chunk_items(k - kLag);
         }
-        s_seg[nchunks + 1] = run;
+        s_seg[nseg] = run;
     }
     unsigned* next_item = ws;
     unsigned* done = ws + kWsHeader;
     unsigned* amax_ws = ws + kWsHeader + kMaxChunks;
+    unsigned pending = 0;  // thread 0: an item index fetched one iteration ahead
     if (threadIdx.x == 0) {
         s_item[0] = (int)atomicAdd(next_item, 1u);
-        s_item[1] = (int)atomicAdd(next_item, 1u);
+        pending = atomicAdd(next_item, 1u);
     }
     __syncthreads();
-    const int items = s_seg[nchunks + 1];
+    const int items = s_seg[nseg];
     const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     auto decode = [&](int j) {
-        int lo = 0, hi = nchunks;  // last s with s_seg[s] <= j
+        int lo = 0, hi = nseg - 1;  // last s with s_seg[s] <= j
         while (lo < hi) {
             const int mid = (lo + hi + 1) >> 1;
             if (s_seg[mid] <= j) lo = mid; else hi = mid - 1;
         }
         const int off = j - s_seg[lo];
-        const int a_items = lo < nchunks ? chunk_items(lo) : 0;
+        const int a_items = chunk_items(lo);
         ItemRef r;
         r.is_a = off < a_items;
-        r.chunk = r.is_a ? lo : lo - 1;
+        r.chunk = r.is_a ? lo : lo - kLag;
         const int idx = r.is_a ? off : off - a_items;
         r.first_tile = s_cf[r.chunk] + idx * kItemTiles;
         r.ntiles = min(kItemTiles, s_cf[r.chunk + 1] - r.first_tile);
@@ -403,10 +410,10 @@ __global__ void __launch_bounds__(kThreads, 3) nvfp4_compute_l2_kernel(const qz_
 #pragma unroll
     for (int p = 0; p < G::kPasses; ++p) tile_load<QZ_FMT_NVFP4>(cur, p, v[p]);
     for (int it = 0;; ++it) {
-        // item it is in s_item[it & 3], item it+1 in s_item[(it+1) & 3]; fetch item it+2
-        unsigned fetched = 0;
+        // publish the index fetched during the previous item, fetch another
         if (threadIdx.x == 0) {
-            fetched = atomicAdd(next_item, 1u);
+            s_item[(it + 1) & 3] = (int)pending;
+            pending = atomicAdd(next_item, 1u);
             unsigned ok = 1;
             if (!item.is_a) {
                 // wait until every A tile of this item's chunk is done
@@ -421,7 +428,6 @@ __global__ void __launch_bounds__(kThreads, 3) nvfp4_compute_l2_kernel(const qz_
                 }
             }
             s_ok[it & 1] = ok;
-            s_item[(it + 2) & 3] = (int)fetched;
         }
         __syncthreads();
         const int jn = s_item[(it + 1) & 3];
@@ -550,7 +556,7 @@ cudaError_t launch_nvfp4_tensor(const qz_expert* table, int n, int layout, bool 
 
 size_t workspace_bytes(int n) { return workspace_words(n) * sizeof(unsigned); }
 
-size_t compute_l2_smem(int n) { return (size_t)(n + 1 + kMaxChunks + 1 + kMaxChunks + 2) * sizeof(int); }
+size_t compute_l2_smem(int n) { return (size_t)(n + 1 + kMaxChunks + 1 + kMaxChunks + kLag + 1) * sizeof(int); }
 
 // One launch of the L2-chunked computed-amax path on a zeroed workspace.
 cudaError_t launch_nvfp4_compute_l2(const qz_expert* table, int n, int layout, int grid, unsigned* ws,
