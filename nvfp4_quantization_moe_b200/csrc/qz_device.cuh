@@ -38,23 +38,37 @@ __device__ __forceinline__ void st_u32(void* p, uint32_t a) {
     asm volatile("st.global.u32 [%0], %1;" ::"l"(p), "r"(a) : "memory");
 }
 
+// L2 eviction priority of a load: default, keep (the data is read again
+// soon), or drop first (last use).
+enum L2Hint { kL2Normal = 0, kL2Last = 1, kL2First = 2 };
+
+#define QZ_LD32(HINTQ)                                                                                         \
+    asm volatile("ld.global.nc.L1::no_allocate" HINTQ ".v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"               \
+                 : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3]), "=r"(w[4]), "=r"(w[5]), "=r"(w[6]), "=r"(w[7]) \
+                 : "l"(p))
+#define QZ_LD16(HINTQ, OFF, A, B, C, D)                                                                        \
+    asm volatile("ld.global.nc" HINTQ ".v4.u32 {%0,%1,%2,%3}, [%4];"                                          \
+                 : "=r"(w[A]), "=r"(w[B]), "=r"(w[C]), "=r"(w[D])                                               \
+                 : "l"(static_cast<const char*>(p) + (OFF)))
+
 // 32-byte load (the address must be 32-byte aligned).
+template <int HINT = kL2Normal>
 __device__ __forceinline__ void ld_stream_32(const void* p, uint32_t (&w)[8]) {
-    asm volatile("ld.global.nc.L1::no_allocate.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
-                 : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3]), "=r"(w[4]), "=r"(w[5]), "=r"(w[6]), "=r"(w[7])
-                 : "l"(p));
+    if (HINT == kL2Last) QZ_LD32(".L2::evict_last");
+    else if (HINT == kL2First) QZ_LD32(".L2::evict_first");
+    else QZ_LD32("");
 }
 
 // 32 bytes from a 16-byte aligned address as two 16-byte loads that allocate
-// in L1 (the second finds the sectors the first brought in).
+// in L1 (the second finds the sectors the first brought in).  The L2
+// eviction qualifiers exist only for 256-bit loads, so the hint is dropped.
+template <int HINT = kL2Normal>
 __device__ __forceinline__ void ld_pair_16(const void* p, uint32_t (&w)[8]) {
-    asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3])
-                 : "l"(p));
-    asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(w[4]), "=r"(w[5]), "=r"(w[6]), "=r"(w[7])
-                 : "l"(static_cast<const char*>(p) + 16));
+    QZ_LD16("", 0, 0, 1, 2, 3);
+    QZ_LD16("", 16, 4, 5, 6, 7);
 }
+#undef QZ_LD32
+#undef QZ_LD16
 
 __device__ __forceinline__ void st_v4(void* p, uint4 v) {
     asm volatile("st.global.v4.u32 [%0], {%1,%2,%3,%4};" ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)

@@ -127,7 +127,7 @@ __device__ __forceinline__ bool pass_live(const TileRef& t, int p) {
 }
 
 // The lane's block of pass p (zeros outside the matrix).
-template <int FMT>
+template <int FMT, int HINT = kL2Normal>
 __device__ __forceinline__ void tile_load(const TileRef& t, int p, uint32_t* w) {
     using G = TileGeo<FMT>;
     uint32_t (&a)[8] = *reinterpret_cast<uint32_t(*)[8]>(w);
@@ -135,11 +135,11 @@ __device__ __forceinline__ void tile_load(const TileRef& t, int p, uint32_t* w) 
     if (pass_live<FMT>(t, p)) {
         const uint16_t* src = t.xp + p * G::kRpp * 8 * t.ld;
         if (t.a32) {
-            ld_stream_32(src, a);
-            if (G::kWords == 16) ld_stream_32(src + 16, b);
+            ld_stream_32<HINT>(src, a);
+            if (G::kWords == 16) ld_stream_32<HINT>(src + 16, b);
         } else {
-            ld_pair_16(src, a);
-            if (G::kWords == 16) ld_pair_16(src + 16, b);
+            ld_pair_16<HINT>(src, a);
+            if (G::kWords == 16) ld_pair_16<HINT>(src + 16, b);
         }
     } else {
 #pragma unroll
@@ -402,13 +402,22 @@ __global__ void __launch_bounds__(kThreads, 3) nvfp4_compute_l2_kernel(const qz_
         return r;
     };
 
+    // A reads keep their lines in L2 for the Q re-read; Q reads release them
+    auto load_tile = [&](const TileRef& t, bool a_item, uint32_t (&v)[G::kPasses][G::kWords]) {
+        if (a_item) {
+#pragma unroll
+            for (int p = 0; p < G::kPasses; ++p) tile_load<QZ_FMT_NVFP4, kL2Last>(t, p, v[p]);
+        } else {
+#pragma unroll
+            for (int p = 0; p < G::kPasses; ++p) tile_load<QZ_FMT_NVFP4, kL2First>(t, p, v[p]);
+        }
+    };
     int j = s_item[0];
     if (j >= items) return;
     ItemRef item = decode(j);
     TileRef cur = tile_ref<QZ_FMT_NVFP4, LAYOUT>(table, s_prefix, n, item.first_tile, w, lane);
     uint32_t v[G::kPasses][G::kWords];
-#pragma unroll
-    for (int p = 0; p < G::kPasses; ++p) tile_load<QZ_FMT_NVFP4>(cur, p, v[p]);
+    load_tile(cur, item.is_a, v);
     for (int it = 0;; ++it) {
         // publish the index fetched during the previous item, fetch another
         if (threadIdx.x == 0) {
@@ -438,13 +447,12 @@ __global__ void __launch_bounds__(kThreads, 3) nvfp4_compute_l2_kernel(const qz_
             const bool last = k + 1 == item.ntiles;
             const bool more = !last || more_items;
             const int ntile = last ? nitem.first_tile : item.first_tile + k + 1;
+            const bool next_a = last ? nitem.is_a : item.is_a;
             const TileRef nxt = more ? tile_ref<QZ_FMT_NVFP4, LAYOUT>(table, s_prefix, n, ntile, w, lane) : cur;
             if (item.is_a) {
 #pragma unroll
-                for (int p = 0; p < G::kPasses; ++p) {
-                    run = max(run, absmax_words<G::kWords>(v[p]));
-                    if (more) tile_load<QZ_FMT_NVFP4>(nxt, p, v[p]);
-                }
+                for (int p = 0; p < G::kPasses; ++p) run = max(run, absmax_words<G::kWords>(v[p]));
+                if (more) load_tile(nxt, next_a, v);
                 if (last || nxt.expert != cur.expert) {
 #pragma unroll
                     for (int o = 16; o > 0; o >>= 1) run = max(run, __shfl_xor_sync(0xFFFFFFFFu, run, o));
@@ -460,7 +468,10 @@ __global__ void __launch_bounds__(kThreads, 3) nvfp4_compute_l2_kernel(const qz_
 #pragma unroll
                 for (int p = 0; p < G::kPasses; ++p) {
                     tile_pass<QZ_FMT_NVFP4, LAYOUT>(cur, p, lane, v[p], S, s_sf[w], s_inv);
-                    if (more) tile_load<QZ_FMT_NVFP4>(nxt, p, v[p]);
+                    if (more) {
+                        if (next_a) tile_load<QZ_FMT_NVFP4, kL2Last>(nxt, p, v[p]);
+                        else tile_load<QZ_FMT_NVFP4, kL2First>(nxt, p, v[p]);
+                    }
                 }
                 if (LAYOUT == QZ_SF_SWIZZLED_128x4) tile_flush_sf<QZ_FMT_NVFP4>(cur, w, lane, s_sf[w]);
                 if (threadIdx.x == 0) *const_cast<float*>(cur.amax) = A;
