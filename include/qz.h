@@ -211,6 +211,34 @@ qz_status qz_rmsnorm_quantize(const void *d_x, const void *d_residual, const voi
  * dst are skipped and reported through opts->d_err. */
 qz_status qz_swizzle_scales(const qz_sf_pair *d_table, int n, void *stream, const qz_launch_opts *opts);
 
+/* Largest table of qz_quantize_grouped_nvfp4_compute_noalloc. */
+#define QZ_STATIC_WS_MAX_EXPERTS 1024
+
+/* Allocation-free NVFP4 quantization with a computed per-tensor amax: the
+ * same single L2-chunked launch as qz_quantize_grouped_nvfp4 in
+ * QZ_NVFP4_PER_TENSOR_COMPUTE mode with opts->d_workspace, but its scratch
+ * (a work counter, per-chunk counters and per-expert amax words, about 21 KB)
+ * is a device array inside the library, so the caller passes only the table,
+ * inputs and outputs.  The source pages have no counterpart of this entry
+ * point; it exists for callers that cannot allocate device memory themselves,
+ * such as code embedded in a framework that owns every device allocation, or
+ * a latency-critical loop in which a cudaMalloc would synchronize the device.
+ *  - The array is allocated with the library image: every GPU on which the
+ *    library is loaded keeps it until the process exits.  The library calls
+ *    no cudaMalloc, cudaFree or other allocating routine here.
+ *  - The first call on a device looks up the array's device address (a
+ *    one-time set-up per device); make that first call before any stream
+ *    capture.
+ *  - Every call clears the scratch it needs (a memset in stream order) and
+ *    leaves its own contents behind; all calls share the one array, so calls
+ *    that may overlap on the GPU (other streams, other host threads) race and
+ *    must be serialized by the caller.
+ *  - n_experts above QZ_STATIC_WS_MAX_EXPERTS returns QZ_ERR_INVALID_ARG
+ *    before anything is launched; other errors as qz_quantize_grouped_nvfp4;
+ *    opts->d_workspace is ignored. */
+qz_status qz_quantize_grouped_nvfp4_compute_noalloc(const qz_expert *d_table, int n_experts, int layout,
+                                                    void *stream, const qz_launch_opts *opts);
+
 /* A static, human-readable name for a status code. */
 const char *qz_status_string(qz_status status);
 

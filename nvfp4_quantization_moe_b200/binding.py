@@ -38,7 +38,9 @@ EXPORTED = (
     "qz_status_string",
     "qz_version",
     "qz_workspace_bytes",
+    "qz_quantize_grouped_nvfp4_compute_noalloc",
 )
+STATIC_WS_MAX_EXPERTS = 1024
 
 
 class QzError(RuntimeError):
@@ -96,6 +98,8 @@ def load(path: str = LIB_PATH):
         lib.qz_version.argtypes = []
         lib.qz_workspace_bytes.restype = ctypes.c_size_t
         lib.qz_workspace_bytes.argtypes = [I]
+        lib.qz_quantize_grouped_nvfp4_compute_noalloc.restype = I
+        lib.qz_quantize_grouped_nvfp4_compute_noalloc.argtypes = [P, I, I, P, P]
         _lib = lib
         return lib
 
@@ -222,6 +226,14 @@ def quantize_grouped_nvfp4(table: ExpertTable, mode: int, layout: int, stream=No
     _check(load().qz_quantize_grouped_nvfp4(ctypes.c_void_p(table.ptr), table.n, int(mode), int(layout),
                                             _stream_ptr(stream), _opts(err, max_ctas, workspace)),
            "qz_quantize_grouped_nvfp4")
+
+
+def quantize_grouped_nvfp4_compute_noalloc(table: ExpertTable, layout: int, stream=None, err=None, max_ctas: int = 0):
+    """NVFP4 with computed per-tensor amax, scratch inside the library (no
+    device allocation by anyone; see qz_quantize_grouped_nvfp4_compute_noalloc)."""
+    _check(load().qz_quantize_grouped_nvfp4_compute_noalloc(ctypes.c_void_p(table.ptr), table.n, int(layout),
+                                                            _stream_ptr(stream), _opts(err, max_ctas)),
+           "qz_quantize_grouped_nvfp4_compute_noalloc")
 
 
 def rmsnorm_quantize(x, residual, gamma, eps: float, norm_out, residual_out, fmt: int, q, sf, layout: int,

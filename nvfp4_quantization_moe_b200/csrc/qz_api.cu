@@ -23,6 +23,8 @@ int grouped_blocks_per_sm(int which, int n);
 size_t workspace_bytes(int n);
 cudaError_t launch_nvfp4_compute_l2(const qz_expert* table, int n, int layout, int grid, unsigned* ws,
                                     cudaStream_t s, unsigned* d_err);
+cudaError_t launch_nvfp4_compute_l2_static(const qz_expert* table, int n, int layout, int grid, cudaStream_t s,
+                                           unsigned* d_err);
 int rows_blocks_per_sm(int n);
 }  // namespace qz
 
@@ -167,6 +169,16 @@ qz_status qz_swizzle_scales(const qz_sf_pair* d_table, int n, void* stream, cons
     if (st != QZ_OK) return st;
     if (n == 0) return QZ_OK;
     return from_cuda(qz::launch_swizzle(d_table, n, wave_grid(2, opts), (cudaStream_t)stream, err_word(opts)));
+}
+
+qz_status qz_quantize_grouped_nvfp4_compute_noalloc(const qz_expert* d_table, int n_experts, int layout,
+                                                    void* stream, const qz_launch_opts* opts) {
+    if (n_experts < 0 || n_experts > QZ_STATIC_WS_MAX_EXPERTS) return QZ_ERR_INVALID_ARG;
+    if (n_experts > 0 && d_table == nullptr) return QZ_ERR_INVALID_ARG;
+    if (!valid_layout(layout)) return QZ_ERR_INVALID_ARG;
+    if (n_experts == 0) return QZ_OK;
+    return from_cuda(qz::launch_nvfp4_compute_l2_static(d_table, n_experts, layout, wave_grid(5, opts),
+                                                        (cudaStream_t)stream, err_word(opts)));
 }
 
 size_t qz_workspace_bytes(int n_experts) {

@@ -19,9 +19,14 @@
 // rows zeroed by the kernel; commit 5: grid-shape invariance);
 // Model-Optimizer "Fold fused experts' quantizers into their weights
 // shard-locally" (per-expert FP32 second-level scale).
+#include <mutex>
+
 #include "qz_device.cuh"
 
 namespace qz {
+
+constexpr int kStaticWsMaxExperts = QZ_STATIC_WS_MAX_EXPERTS;  // table limit of the allocation-free entry point
+constexpr int kStaticWsMaxDevices = 64;
 
 // Tiles of one expert; 0 for an empty or invalid entry (invalid entries are
 // reported by block 0 only).
@@ -605,6 +610,48 @@ int grouped_blocks_per_sm(int which, int n) {
         }
     }
     return b > 0 ? b : 1;
+}
+
+}  // namespace qz
+
+// ---------------------------------------------------------------------------
+// Allocation-free variant of the L2-chunked computed-amax launch: its scratch
+// is this file-scope device array instead of a caller workspace.  Every GPU
+// that loads the library holds it until the process exits.
+// ---------------------------------------------------------------------------
+namespace qz {
+
+static __device__ __align__(256) unsigned g_static_ws[workspace_words(kStaticWsMaxExperts)];
+
+namespace {
+std::mutex g_static_mu;
+unsigned* g_static_ws_dev[kStaticWsMaxDevices] = {};
+}  // namespace
+
+// Device address of g_static_ws on the current device, looked up once per
+// device (the host-side name is only a stand-in for the device copy).
+cudaError_t static_workspace(unsigned** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kStaticWsMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_static_mu);
+    if (!g_static_ws_dev[dev]) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_static_ws);
+        if (e != cudaSuccess) return e;
+        g_static_ws_dev[dev] = static_cast<unsigned*>(p);
+    }
+    *out = g_static_ws_dev[dev];
+    return cudaSuccess;
+}
+
+cudaError_t launch_nvfp4_compute_l2_static(const qz_expert* table, int n, int layout, int grid, cudaStream_t s,
+                                           unsigned* d_err) {
+    unsigned* ws = nullptr;
+    cudaError_t e = static_workspace(&ws);
+    if (e != cudaSuccess) return e;
+    return launch_nvfp4_compute_l2(table, n, layout, grid, ws, s, d_err);
 }
 
 }  // namespace qz
