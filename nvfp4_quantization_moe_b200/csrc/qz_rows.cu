@@ -5,16 +5,16 @@
 // payload, row amax and scale factors land in per-expert storage whose
 // swizzled padding is independent per expert (uneven and empty splits).
 //
-// One warp per row.  Rows of up to 4096 elements are brought into shared
-// memory by one bulk (TMA) copy each: each of the 12 warps of a CTA keeps
-// kRowDepth rows in flight in its own ring of shared-memory slots, each slot
-// with an mbarrier that the copy completes, so HBM streams while the warp
-// quantizes.  The warp reads the slot twice (row amax, then quantization), so
-// few registers are live and many warps fit on an SM.  In the quantize pass a
-// lane takes one 16-element block at a time, so each block scale is computed
-// once, and the scale bytes of four consecutive blocks (four consecutive
-// lanes) leave as one 32-bit store.  Longer rows take a two-pass path
-// straight from global memory.
+// One persistent 128-thread CTA works on one row at a time.  Thread t owns
+// the 16-element blocks t and t + 128 of the row (a row of up to 4096
+// elements is two 32-byte loads per thread), held in registers: the row amax
+// is a warp reduction plus a four-word exchange in shared memory, and each
+// block's scale is computed once, by its owner.  While a row is quantized,
+// the CTA's next row is already being loaded into the same registers, block
+// by block as they are consumed.  The scale bytes of four consecutive blocks
+// (four consecutive threads) leave as one 32-bit store.  Rows longer than
+// 4096 elements take a two-pass path (amax pass, then a quantize pass
+// re-reading the row from L2).
 //
 // Units of work are "virtual rows": an expert owns rows (linear layout) or
 // pad(rows, 128) virtual rows (swizzled); a virtual row past the last live row
@@ -24,14 +24,9 @@
 
 namespace qz {
 
-constexpr int kRowChunks = 16;                  // 16-byte chunks per lane for a 4096-element row
-constexpr int kRowSlot = 32 * kRowChunks * 16;  // bytes of one shared-memory row slot (8 KiB)
-constexpr int kRowDepth = 2;                    // rows in flight per warp
-constexpr int kRowWarps = 12;                   // warps per CTA
-constexpr int kRowThreads = 32 * kRowWarps;
-constexpr int kRowBarBytes = 1024;              // mbarrier area at the start of shared memory
-constexpr size_t kRowRingBytes = (size_t)kRowWarps * kRowDepth * kRowSlot;
-constexpr size_t kRowStashBytes = (size_t)kRowWarps * (kRowSlot / 32) * sizeof(uint16_t);  // block amax per warp
+constexpr int kRowThreads = 128;
+constexpr int kRowBlocksPerThread = 2;                              // register-resident blocks per thread
+constexpr int kRowMaxResident = kRowThreads * kRowBlocksPerThread;  // blocks of a register-resident row
 
 template <int LAYOUT>
 struct RowUnits {
@@ -48,206 +43,187 @@ struct RowUnits {
 
 // Store the scale group starting at block k0 (k0 % 4 == 0), bytes in `word`.
 template <int LAYOUT>
-__device__ __forceinline__ void store_scale_group(const qz_expert& E, int64_t row, int64_t k0, int64_t kv,
-                                                  uint32_t word) {
+__device__ __forceinline__ void store_scale_group(uint8_t* sf, int64_t row, int64_t k0, int64_t kv, uint32_t word) {
     if (LAYOUT == QZ_SF_SWIZZLED_128x4) {
-        if (k0 < pad_to(kv, 4)) st_u32(E.sf + swz_offset(row, k0, kv), word);
+        if (k0 < pad_to(kv, 4)) st_u32(sf + swz_offset(row, k0, kv), word);
     } else {
         const int64_t base = row * kv + k0;
-        if (k0 + 4 <= kv && (base & 3) == 0 && (((uintptr_t)E.sf) & 3) == 0) {
-            st_u32(E.sf + base, word);
+        if (k0 + 4 <= kv && (base & 3) == 0 && (((uintptr_t)sf) & 3) == 0) {
+            st_u32(sf + base, word);
         } else {
-            for (int j = 0; j < 4 && k0 + j < kv; ++j) E.sf[base + j] = (uint8_t)(word >> (8 * j));
+            for (int j = 0; j < 4 && k0 + j < kv; ++j) sf[base + j] = (uint8_t)(word >> (8 * j));
         }
     }
 }
 
-// Quantize blocks b0 .. b0+31 of a row, lane l taking block b = b0 + l whose
-// two chunks are v0, v1 (zeros past the row) and whose amax has bf16 bits m.
-// The scale bytes of four consecutive blocks (lanes 4g .. 4g+3) leave as one
-// 32-bit store.
+// One thread's view of one virtual row.
+struct RowRef {
+    const uint16_t* x;  // row start
+    uint8_t* q;         // payload row start
+    uint8_t* sf;        // expert's SF region
+    float* amax;        // expert's row amax array
+    int64_t row;        // row inside the expert
+    int kv;             // blocks per row
+    bool live;          // row < rows (else a padded row of the swizzled region)
+    bool a32;           // 32-byte aligned rows
+};
+
+__device__ __forceinline__ RowRef row_ref(const qz_expert* table, const int* s_prefix, int n, int u) {
+    const int e = find_owner(s_prefix, n, u);
+    const qz_expert E = load_entry(table, e);
+    RowRef r;
+    r.row = u - s_prefix[e];
+    r.live = r.row < E.rows;
+    r.x = static_cast<const uint16_t*>(E.x) + r.row * E.ld;
+    r.q = static_cast<uint8_t*>(E.q) + r.row * (E.cols >> 1);
+    r.sf = E.sf;
+    r.amax = E.amax;
+    r.kv = (int)(E.cols >> 4);
+    r.a32 = ((reinterpret_cast<uintptr_t>(E.x) & 31) == 0) && ((E.ld & 15) == 0);
+    return r;
+}
+
+// Block b of the row (zeros past the row).
+__device__ __forceinline__ void row_block_load(const RowRef& r, int b, uint32_t (&w)[8]) {
+    if (b < r.kv) {
+        if (r.a32) ld_stream_32(r.x + b * 16, w);
+        else ld_pair_16(r.x + b * 16, w);
+    } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) w[i] = 0u;
+    }
+}
+
+// The thread's register-resident blocks (t + 128 i) of a live row with kv <= 256.
+__device__ __forceinline__ void row_load_resident(const RowRef& r, int i, uint32_t (&w)[8]) {
+    if (r.live && r.kv <= kRowMaxResident) {
+        row_block_load(r, (int)threadIdx.x + kRowThreads * i, w);
+    } else {
+#pragma unroll
+        for (int k = 0; k < 8; ++k) w[k] = 0u;
+    }
+}
+
+// Quantize block b (words w, amax bits m) with encode scale S; four
+// consecutive threads' scale bytes leave as one store (all threads call this).
 template <int LAYOUT>
-__device__ __forceinline__ void row_blocks(const qz_expert& E, int64_t row, uint8_t* qrow, bool q8, int64_t b,
-                                           int64_t kv, uint4 v0, uint4 v1, uint32_t m, float S, const float* inv,
-                                           int lane) {
+__device__ __forceinline__ void row_block_quant(const RowRef& r, int b, const uint32_t (&w)[8], uint32_t m, float S,
+                                                const float* inv, bool q8) {
     const Nvfp4Block blk = nvfp4_block(bits_to_float_bf16(m), S, inv);
-    const uint32_t c0 = e2m1x8_scaled(v0, blk.rcp);
-    const uint32_t c1 = e2m1x8_scaled(v1, blk.rcp);
-    if (b < kv) {
+    const uint32_t c0 = e2m1x8_words(w[0], w[1], w[2], w[3], blk.rcp);
+    const uint32_t c1 = e2m1x8_words(w[4], w[5], w[6], w[7], blk.rcp);
+    if (b < r.kv) {
         if (q8) {
-            st_v2(qrow + b * 8, c0, c1);
+            st_v2(r.q + b * 8, c0, c1);
         } else {
-            st_u32(qrow + b * 8, c0);
-            st_u32(qrow + b * 8 + 4, c1);
+            st_u32(r.q + b * 8, c0);
+            st_u32(r.q + b * 8 + 4, c1);
         }
     }
     const uint32_t s1 = __shfl_down_sync(0xFFFFFFFFu, blk.scale, 1);
     const uint32_t s2 = __shfl_down_sync(0xFFFFFFFFu, blk.scale, 2);
     const uint32_t s3 = __shfl_down_sync(0xFFFFFFFFu, blk.scale, 3);
-    if ((lane & 3) == 0) store_scale_group<LAYOUT>(E, row, b, kv, blk.scale | (s1 << 8) | (s2 << 16) | (s3 << 24));
+    if ((threadIdx.x & 3) == 0)
+        store_scale_group<LAYOUT>(r.sf, r.row, b, r.kv, blk.scale | (s1 << 8) | (s2 << 16) | (s3 << 24));
 }
 
-// A row of at most 4096 elements staged in shared memory.  Amax pass: lane l
-// reads chunks l + 32i (conflict-free), pairs of lanes combine a block's two
-// chunks and the block amax goes to the warp's stash (bf16 bits per block).
-// Quantize pass: one 16-element block per lane, its amax from the stash.
-template <int LAYOUT>
-__device__ __forceinline__ void row_from_slot(const qz_expert& E, int64_t row, const uint8_t* slot, uint16_t* stash,
-                                              const float* inv, int lane) {
-    const int nch = (int)(E.cols >> 3), kv = (int)(E.cols >> 4);
-    const int nbp = (int)pad_to(kv, 4);  // blocks whose scale bytes exist (incl. padding)
-    uint32_t m = 0;
-#pragma unroll 4
-    for (int c0 = 0; c0 < nch; c0 += 32) {  // nch is even: a block's chunks are both live or both not
-        const int c = c0 + lane;
-        uint32_t cm = c < nch ? absmax_bits(lds128(slot + c * 16)) : 0u;
-        cm = max(cm, __shfl_xor_sync(0xFFFFFFFFu, cm, 1));
-        if ((lane & 1) == 0 && c < nch) stash[c >> 1] = (uint16_t)cm;
-        m = max(m, cm);
-    }
+// CTA-wide maximum of m (bf16 magnitude bits): one shared word per warp,
+// alternating between two sets on successive calls (`parity`), so that each
+// call needs a single barrier: a set is rewritten only after the next call's
+// barrier, which every thread reaches after reading it.
+__device__ __forceinline__ uint32_t cta_max(uint32_t m, uint32_t (*s_max)[kRowThreads / 32], int parity) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
-    __syncwarp();
-    const float A = bits_to_float_bf16(m);
-    if (lane == 0) E.amax[row] = A;
-    const float S = nvfp4_encode_scale(A);
-    uint8_t* qrow = static_cast<uint8_t*>(E.q) + row * (E.cols >> 1);
-    const bool q8 = (((uintptr_t)qrow) & 7) == 0;
-#pragma unroll 2
-    for (int b0 = 0; b0 < nbp; b0 += 32) {
-        const int b = b0 + lane;
-        uint4 v0 = make_uint4(0, 0, 0, 0), v1 = make_uint4(0, 0, 0, 0);
-        uint32_t bm = 0;
-        if (b < kv) {
-            v0 = lds128(slot + b * 32);
-            v1 = lds128(slot + b * 32 + 16);
-            bm = stash[b];
-        }
-        row_blocks<LAYOUT>(E, row, qrow, q8, b, kv, v0, v1, bm, S, inv, lane);
-    }
-}
-
-// A row of any length straight from global memory: amax pass, then a
-// quantize pass re-reading the row (served by L2).
-template <int LAYOUT>
-__device__ __forceinline__ void row_two_pass(const qz_expert& E, int64_t row, const float* inv, int lane) {
-    const int64_t nch = E.cols >> 3, kv = E.cols >> 4, nbp = pad_to(kv, 4);
-    const uint16_t* xr = static_cast<const uint16_t*>(E.x) + row * E.ld;
-    uint32_t m = 0;
-    for (int64_t c = lane; c < nch; c += 32) m = max(m, absmax_bits(ld_stream(xr + c * 8)));
+    if ((threadIdx.x & 31) == 0) s_max[parity][threadIdx.x >> 5] = m;
+    __syncthreads();
+    uint32_t r = 0;
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
-    const float A = bits_to_float_bf16(m);
-    if (lane == 0) E.amax[row] = A;
-    const float S = nvfp4_encode_scale(A);
-    uint8_t* qrow = static_cast<uint8_t*>(E.q) + row * (E.cols >> 1);
-    const bool q8 = (((uintptr_t)qrow) & 7) == 0;
-    for (int64_t b0 = 0; b0 < nbp; b0 += 32) {
-        const int64_t b = b0 + lane;
-        uint4 v0 = make_uint4(0, 0, 0, 0), v1 = make_uint4(0, 0, 0, 0);
-        if (b < kv) {
-            v0 = ld_stream(xr + b * 16);
-            v1 = ld_stream(xr + b * 16 + 8);
-        }
-        row_blocks<LAYOUT>(E, row, qrow, q8, b, kv, v0, v1, max(absmax_bits(v0), absmax_bits(v1)), S, inv, lane);
-    }
-}
-
-// Zero scale bytes of a padded row of the swizzled region.
-__device__ __forceinline__ void row_zero_scales(const qz_expert& E, int64_t row, int lane) {
-    const int64_t kv = E.cols >> 4;
-    for (int64_t k0 = 4 * lane; k0 < pad_to(kv, 4); k0 += 128) st_u32(E.sf + swz_offset(row, k0, kv), 0u);
-}
-
-struct RowRef {
-    qz_expert E;
-    int64_t row;
-};
-
-__device__ __forceinline__ RowRef row_ref(const qz_expert* table, const int* s_prefix, int n, int u) {
-    const int e = find_owner(s_prefix, n, u);
-    RowRef r;
-    r.E = load_entry(table, e);
-    r.row = u - s_prefix[e];
+    for (int k = 0; k < kRowThreads / 32; ++k) r = max(r, s_max[parity][k]);
     return r;
 }
 
 template <int LAYOUT>
-__global__ void __launch_bounds__(kRowThreads, 1) nvfp4_rows_kernel(const qz_expert* __restrict__ table, int n,
+__global__ void __launch_bounds__(kRowThreads) nvfp4_rows_kernel(const qz_expert* __restrict__ table, int n,
                                                                  unsigned* d_err) {
-    extern __shared__ __align__(128) uint8_t smem[];
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem);
-    uint8_t* ring = smem + kRowBarBytes;
-    uint16_t* stash_all = reinterpret_cast<uint16_t*>(ring + kRowRingBytes);
-    int* s_prefix = reinterpret_cast<int*>(ring + kRowRingBytes + kRowStashBytes);
+    extern __shared__ int s_prefix[];
     __shared__ long long s_scan[33];
     __shared__ float s_inv[16];
+    __shared__ uint32_t s_max[2][kRowThreads / 32];
     fill_inv_table(s_inv);
-    if (threadIdx.x < kRowWarps * kRowDepth) mbar_init(&bars[threadIdx.x], 1);
-    mbar_init_fence();
     const int total = block_prefix(n, s_prefix, s_scan, RowUnits<LAYOUT>{table, d_err}, d_err);  // has barriers
-    const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int stride = gridDim.x * kRowWarps;
-    const int first = blockIdx.x * kRowWarps + w;
-    uint8_t* slots = ring + (size_t)w * kRowDepth * kRowSlot;
-    uint64_t* my_bars = bars + w * kRowDepth;
-    uint16_t* stash = stash_all + w * (kRowSlot / 32);
-    unsigned issued = 0, phase = 0;  // per-slot bits, identical in every lane
-
-    // start the copy of unit u into slot s when it is a live row that fits a slot
-    auto issue = [&](long long u, int s) {
-        issued &= ~(1u << s);
-        if (u >= total) return;
-        const RowRef r = row_ref(table, s_prefix, n, (int)u);
-        const uint32_t bytes = (uint32_t)(r.E.cols * 2);
-        if (r.row >= r.E.rows || bytes > (uint32_t)kRowSlot) return;
-        if (lane == 0) {
-            fence_proxy_async_smem();
-            mbar_arrive_expect_tx(&my_bars[s], bytes);
-            bulk_load(slots + s * kRowSlot, static_cast<const uint16_t*>(r.E.x) + r.row * r.E.ld, bytes, &my_bars[s]);
-        }
-        issued |= 1u << s;
-    };
-
+    const int t = threadIdx.x;
+    int u = blockIdx.x;
+    if (u >= total) return;
+    RowRef cur = row_ref(table, s_prefix, n, u);
+    uint32_t w[kRowBlocksPerThread][8];
 #pragma unroll
-    for (int s = 0; s < kRowDepth; ++s) issue((long long)first + (long long)s * stride, s);
-
-    for (int i = 0;; ++i) {
-        const long long u = (long long)first + (long long)i * stride;
-        if (u >= total) break;
-        const int s = i % kRowDepth;
-        const RowRef r = row_ref(table, s_prefix, n, (int)u);
-        if (r.row >= r.E.rows) {
-            row_zero_scales(r.E, r.row, lane);
-        } else if ((issued >> s) & 1u) {
-            if (!mbar_wait_bounded(&my_bars[s], (phase >> s) & 1u)) {
-                if (lane == 0 && d_err) atomicOr(d_err, QZ_DERR_TIMEOUT);
-                break;
+    for (int i = 0; i < kRowBlocksPerThread; ++i) row_load_resident(cur, i, w[i]);
+    int reductions = 0;  // CTA reductions so far: their shared words alternate
+    for (;;) {
+        const int un = u + gridDim.x;
+        const bool more = un < total;
+        const RowRef nxt = more ? row_ref(table, s_prefix, n, un) : cur;
+        if (!cur.live) {
+            // padded row of the swizzled region: zero scale bytes only
+            const int kvp = (int)pad_to(cur.kv, 4);
+            for (int k0 = 4 * t; k0 < kvp; k0 += 4 * kRowThreads) st_u32(cur.sf + swz_offset(cur.row, k0, cur.kv), 0u);
+            if (more) {
+#pragma unroll
+                for (int i = 0; i < kRowBlocksPerThread; ++i) row_load_resident(nxt, i, w[i]);
             }
-            phase ^= 1u << s;
-            row_from_slot<LAYOUT>(r.E, r.row, slots + s * kRowSlot, stash, s_inv, lane);
-        } else {
-            row_two_pass<LAYOUT>(r.E, r.row, s_inv, lane);
-        }
-        __syncwarp();  // every lane is done with slot s before it is refilled
-        issue(u + (long long)kRowDepth * stride, s);
-    }
-    // drain: copies still in flight (units past a timeout) complete before exit
+        } else if (cur.kv <= kRowMaxResident) {
+            uint32_t bm[kRowBlocksPerThread];
+            uint32_t m = 0;
 #pragma unroll
-    for (int s = 0; s < kRowDepth; ++s)
-        if ((issued >> s) & 1u) {
-            if (!mbar_wait_bounded(&my_bars[s], (phase >> s) & 1u) && lane == 0 && d_err) atomicOr(d_err, QZ_DERR_TIMEOUT);
-            phase ^= 1u << s;
-            issued &= ~(1u << s);
+            for (int i = 0; i < kRowBlocksPerThread; ++i) {
+                bm[i] = absmax_words<8>(w[i]);
+                m = max(m, bm[i]);
+            }
+            const uint32_t rowm = cta_max(m, s_max, (reductions++) & 1);
+            const float A = bits_to_float_bf16(rowm);
+            if (t == 0) cur.amax[cur.row] = A;
+            const float S = nvfp4_encode_scale(A);
+            const bool q8 = (((uintptr_t)cur.q) & 7) == 0;
+            const int nbp = (int)pad_to(cur.kv, 4);
+#pragma unroll
+            for (int i = 0; i < kRowBlocksPerThread; ++i) {
+                const int b0 = kRowThreads * i;
+                if (b0 < nbp) row_block_quant<LAYOUT>(cur, b0 + t, w[i], bm[i], S, s_inv, q8);  // uniform
+                // refill with the next row's block as soon as this one is consumed
+                if (more) row_load_resident(nxt, i, w[i]);
+            }
+        } else {
+            // long row: amax pass, then a quantize pass re-reading the row
+            uint32_t m = 0;
+            for (int b = t; b < cur.kv; b += kRowThreads) {
+                uint32_t v[8];
+                row_block_load(cur, b, v);
+                m = max(m, absmax_words<8>(v));
+            }
+            const uint32_t rowm = cta_max(m, s_max, (reductions++) & 1);
+            const float A = bits_to_float_bf16(rowm);
+            if (t == 0) cur.amax[cur.row] = A;
+            const float S = nvfp4_encode_scale(A);
+            const bool q8 = (((uintptr_t)cur.q) & 7) == 0;
+            const int nbp = (int)pad_to(cur.kv, 4);
+            for (int b0 = 0; b0 < nbp; b0 += kRowThreads) {
+                uint32_t v[8];
+                row_block_load(cur, b0 + t, v);
+                row_block_quant<LAYOUT>(cur, b0 + t, v, absmax_words<8>(v), S, s_inv, q8);
+            }
+            if (more) {
+#pragma unroll
+                for (int i = 0; i < kRowBlocksPerThread; ++i) row_load_resident(nxt, i, w[i]);
+            }
         }
-}
-
-size_t rows_smem_bytes(int n) {
-    return kRowBarBytes + kRowRingBytes + kRowStashBytes + (size_t)(n + 1) * sizeof(int);
+        if (!more) break;
+        cur = nxt;
+        u = un;
+    }
 }
 
 cudaError_t launch_nvfp4_rows(const qz_expert* table, int n, int layout, int grid, cudaStream_t s, unsigned* d_err) {
-    const size_t smem = rows_smem_bytes(n);
+    const size_t smem = (size_t)(n + 1) * sizeof(int);
     if (layout == QZ_SF_SWIZZLED_128x4)
         nvfp4_rows_kernel<QZ_SF_SWIZZLED_128x4><<<grid, kRowThreads, smem, s>>>(table, n, d_err);
     else
@@ -255,14 +231,11 @@ cudaError_t launch_nvfp4_rows(const qz_expert* table, int n, int layout, int gri
     return cudaGetLastError();
 }
 
-// Opt the row kernels into their shared-memory size; returns resident CTAs per SM.
+// Resident CTAs per SM (for a one-wave persistent grid).
 int rows_blocks_per_sm(int n) {
-    const size_t smem = rows_smem_bytes(QZ_MAX_EXPERTS);
-    cudaFuncSetAttribute(nvfp4_rows_kernel<QZ_SF_SWIZZLED_128x4>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    cudaFuncSetAttribute(nvfp4_rows_kernel<QZ_SF_LINEAR>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     int b = 1;
     cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, nvfp4_rows_kernel<QZ_SF_SWIZZLED_128x4>, kRowThreads,
-                                                  rows_smem_bytes(n));
+                                                  (size_t)(n + 1) * sizeof(int));
     return b > 0 ? b : 1;
 }
 
