@@ -113,12 +113,11 @@ __device__ __forceinline__ void store_scale_group(const RowRef& r, int k0, uint3
     }
 }
 
-// Quantize block b (words w, amax bits m) with encode scale S; four
-// consecutive lanes' scale bytes leave as one store (all lanes call this).
+// Quantize block b (words w) with its scale blk; four consecutive lanes'
+// scale bytes leave as one store (all lanes call this).
 template <int LAYOUT>
-__device__ __forceinline__ void row_block_quant(const RowRef& r, int b, const uint32_t (&w)[8], uint32_t m, float S,
-                                                const float* inv, int lane) {
-    const Nvfp4Block blk = nvfp4_block(bits_to_float_bf16(m), S, inv);
+__device__ __forceinline__ void row_block_store(const RowRef& r, int b, const uint32_t (&w)[8], Nvfp4Block blk,
+                                                int lane) {
     const uint32_t c0 = e2m1x8_words(w[0], w[1], w[2], w[3], blk.rcp);
     const uint32_t c1 = e2m1x8_words(w[4], w[5], w[6], w[7], blk.rcp);
     if (b < r.kv) {
@@ -133,6 +132,12 @@ __device__ __forceinline__ void row_block_quant(const RowRef& r, int b, const ui
     const uint32_t s2 = __shfl_down_sync(0xFFFFFFFFu, blk.scale, 2);
     const uint32_t s3 = __shfl_down_sync(0xFFFFFFFFu, blk.scale, 3);
     if ((lane & 3) == 0) store_scale_group<LAYOUT>(r, b, blk.scale | (s1 << 8) | (s2 << 16) | (s3 << 24));
+}
+
+template <int LAYOUT>
+__device__ __forceinline__ void row_block_quant(const RowRef& r, int b, const uint32_t (&w)[8], uint32_t m, float S,
+                                                const float* inv, int lane) {
+    row_block_store<LAYOUT>(r, b, w, nvfp4_block(bits_to_float_bf16(m), S, inv), lane);
 }
 
 __device__ __forceinline__ uint32_t warp_max(uint32_t m) {
@@ -181,9 +186,13 @@ __global__ void __launch_bounds__(kRowThreads) nvfp4_rows_kernel(const qz_expert
             if (lane == 0) *cur.amax = A;
             const float S = nvfp4_encode_scale(A);
             const int nbp = (cur.kv + 3) & ~3;
+            // all block scales first: eight independent chains for the scheduler
+            Nvfp4Block blk[kRowBlocksPerLane];
+#pragma unroll
+            for (int i = 0; i < kRowBlocksPerLane; ++i) blk[i] = nvfp4_block(bits_to_float_bf16(bm[i]), S, s_inv);
 #pragma unroll
             for (int i = 0; i < kRowBlocksPerLane; ++i) {
-                if (32 * i < nbp) row_block_quant<LAYOUT>(cur, lane + 32 * i, w[i], bm[i], S, s_inv, lane);  // uniform
+                if (32 * i < nbp) row_block_store<LAYOUT>(cur, lane + 32 * i, w[i], blk[i], lane);  // uniform
                 // refill with the next row's block as soon as this one is consumed
                 if (more) row_load_resident(nxt, i, lane, w[i]);
             }
