@@ -5,12 +5,11 @@
 // payload, row amax and scale factors land in per-expert storage whose
 // swizzled padding is independent per expert (uneven and empty splits).
 //
-// A pair of warps works on one row at a time (four pairs per CTA, a
-// persistent grid).  Lane l of half h owns the 16-element blocks
-// 128h + l + 32i of the row (a row of up to 4096 elements is four 32-byte
-// loads per lane), held in registers: the row amax is a warp reduction plus
-// an exchange between the two warps (a 64-thread named barrier), and each
-// block's scale is computed once, by its owner.  As soon as a block is quantized its registers
+// One warp works on one row at a time (four independent warps per CTA, a
+// persistent grid).  Lane l owns the 16-element blocks l + 32i of the row (a
+// row of up to 4096 elements is eight 32-byte loads per lane), held in
+// registers: the row amax is a warp reduction and each block's scale is
+// computed once, by its owner.  As soon as a block is quantized its registers
 // are refilled with the same block of the warp's next row, so the next row
 // streams in while this one is processed.  The scale bytes of four
 // consecutive blocks (four consecutive lanes) leave as one 32-bit store.
@@ -25,11 +24,10 @@
 
 namespace qz {
 
-constexpr int kRowThreads = 256;                          // four pairs of warps
-constexpr int kRowPairs = kRowThreads / 64;
-constexpr int kRowBlocksPerLane = 4;                      // register-resident blocks per lane
-constexpr int kRowHalfBlocks = 32 * kRowBlocksPerLane;    // blocks held by one warp of the pair
-constexpr int kRowMaxResident = 2 * kRowHalfBlocks;       // blocks of a register-resident row (4096 elements)
+constexpr int kRowThreads = 128;                          // four independent warps
+constexpr int kRowWarps = kRowThreads / 32;
+constexpr int kRowBlocksPerLane = 8;                      // register-resident blocks per lane
+constexpr int kRowMaxResident = 32 * kRowBlocksPerLane;   // blocks of a register-resident row (4096 elements)
 
 template <int LAYOUT>
 struct RowUnits {
@@ -90,11 +88,10 @@ __device__ __forceinline__ void row_block_load(const RowRef& r, int b, uint32_t 
     }
 }
 
-// The lane's register-resident block i (base + 32 i, base = 128 h + lane) of a
-// live row with kv <= 256.
-__device__ __forceinline__ void row_load_resident(const RowRef& r, int i, int base, uint32_t (&w)[8]) {
+// The lane's register-resident block i (lane + 32 i) of a live row with kv <= 256.
+__device__ __forceinline__ void row_load_resident(const RowRef& r, int i, int lane, uint32_t (&w)[8]) {
     if (r.live && r.kv <= kRowMaxResident) {
-        row_block_load(r, base + 32 * i, w);
+        row_block_load(r, lane + 32 * i, w);
     } else {
 #pragma unroll
         for (int k = 0; k < 8; ++k) w[k] = 0u;
@@ -149,39 +146,22 @@ __device__ __forceinline__ uint32_t warp_max(uint32_t m) {
     return m;
 }
 
-// Maximum over the pair of warps sharing a row: one shared word per warp,
-// alternating between two sets on successive calls (`parity`), published by
-// the pair's named barrier (ids 1..kRowPairs; 0 is the CTA barrier).  A set is
-// rewritten only after the pair's next barrier, which both warps reach after
-// reading it.
-__device__ __forceinline__ uint32_t pair_max(uint32_t m, uint32_t (*s_pair)[kRowPairs][2], int pair, int half,
-                                             int parity) {
-    m = warp_max(m);
-    if ((threadIdx.x & 31) == 0) s_pair[parity][pair][half] = m;
-    asm volatile("bar.sync %0, 64;" ::"r"(pair + 1) : "memory");
-    return max(s_pair[parity][pair][0], s_pair[parity][pair][1]);
-}
-
 template <int LAYOUT>
 __global__ void __launch_bounds__(kRowThreads) nvfp4_rows_kernel(const qz_expert* __restrict__ table, int n,
                                                                  unsigned* d_err) {
     extern __shared__ int s_prefix[];
     __shared__ long long s_scan[33];
     __shared__ float s_inv[16];
-    __shared__ uint32_t s_pair[2][kRowPairs][2];
     fill_inv_table(s_inv);
     const int total = block_prefix(n, s_prefix, s_scan, RowUnits<LAYOUT>{table, d_err}, d_err);  // has barriers
     const int lane = threadIdx.x & 31;
-    const int pair = threadIdx.x >> 6, half = (threadIdx.x >> 5) & 1;
-    const int base = kRowHalfBlocks * half + lane;  // this lane's first block of a row
-    const int stride = gridDim.x * kRowPairs;
-    int u = blockIdx.x * kRowPairs + pair;
-    if (u >= total) return;  // both warps of a pair leave together
+    const int stride = gridDim.x * kRowWarps;
+    int u = blockIdx.x * kRowWarps + (threadIdx.x >> 5);
+    if (u >= total) return;
     RowRef cur = row_ref<LAYOUT>(table, s_prefix, n, u);
     uint32_t w[kRowBlocksPerLane][8];
 #pragma unroll
-    for (int i = 0; i < kRowBlocksPerLane; ++i) row_load_resident(cur, i, base, w[i]);
-    int reductions = 0;  // pair reductions so far: their shared words alternate
+    for (int i = 0; i < kRowBlocksPerLane; ++i) row_load_resident(cur, i, lane, w[i]);
     for (;;) {
         const int un = u + stride;
         const bool more = un < total;
@@ -189,10 +169,10 @@ __global__ void __launch_bounds__(kRowThreads) nvfp4_rows_kernel(const qz_expert
         if (!cur.live) {
             // padded row of the swizzled region: zero scale bytes only
             const int kvp = (cur.kv + 3) & ~3;
-            for (int k0 = 4 * (lane + 32 * half); k0 < kvp; k0 += 256) st_u32(cur.sfrow + ((k0 >> 2) << 9), 0u);
+            for (int k0 = 4 * lane; k0 < kvp; k0 += 128) st_u32(cur.sfrow + ((k0 >> 2) << 9), 0u);
             if (more) {
 #pragma unroll
-                for (int i = 0; i < kRowBlocksPerLane; ++i) row_load_resident(nxt, i, base, w[i]);
+                for (int i = 0; i < kRowBlocksPerLane; ++i) row_load_resident(nxt, i, lane, w[i]);
             }
         } else if (cur.kv <= kRowMaxResident) {
             uint32_t bm[kRowBlocksPerLane];
@@ -202,41 +182,40 @@ __global__ void __launch_bounds__(kRowThreads) nvfp4_rows_kernel(const qz_expert
                 bm[i] = absmax_words<8>(w[i]);
                 m = max(m, bm[i]);
             }
-            const float A = bits_to_float_bf16(pair_max(m, s_pair, pair, half, (reductions++) & 1));
-            if (lane == 0 && half == 0) *cur.amax = A;
+            const float A = bits_to_float_bf16(warp_max(m));
+            if (lane == 0) *cur.amax = A;
             const float S = nvfp4_encode_scale(A);
             const int nbp = (cur.kv + 3) & ~3;
-            // all block scales first: independent chains for the scheduler
+            // all block scales first: eight independent chains for the scheduler
             Nvfp4Block blk[kRowBlocksPerLane];
 #pragma unroll
             for (int i = 0; i < kRowBlocksPerLane; ++i) blk[i] = nvfp4_block(bits_to_float_bf16(bm[i]), S, s_inv);
 #pragma unroll
             for (int i = 0; i < kRowBlocksPerLane; ++i) {
-                if (base - lane + 32 * i < nbp) row_block_store<LAYOUT>(cur, base + 32 * i, w[i], blk[i], lane);  // warp-uniform
+                if (32 * i < nbp) row_block_store<LAYOUT>(cur, lane + 32 * i, w[i], blk[i], lane);  // uniform
                 // refill with the next row's block as soon as this one is consumed
-                if (more) row_load_resident(nxt, i, base, w[i]);
+                if (more) row_load_resident(nxt, i, lane, w[i]);
             }
         } else {
             // long row: amax pass, then a quantize pass re-reading the row
-            // (half h takes block runs of 32 starting at 32 h, 64 apart)
             uint32_t m = 0;
-            for (int b = 32 * half + lane; b < cur.kv; b += 64) {
+            for (int b = lane; b < cur.kv; b += 32) {
                 uint32_t v[8];
                 row_block_load(cur, b, v);
                 m = max(m, absmax_words<8>(v));
             }
-            const float A = bits_to_float_bf16(pair_max(m, s_pair, pair, half, (reductions++) & 1));
-            if (lane == 0 && half == 0) *cur.amax = A;
+            const float A = bits_to_float_bf16(warp_max(m));
+            if (lane == 0) *cur.amax = A;
             const float S = nvfp4_encode_scale(A);
             const int nbp = (cur.kv + 3) & ~3;
-            for (int b0 = 32 * half; b0 < nbp; b0 += 64) {
+            for (int b0 = 0; b0 < nbp; b0 += 32) {
                 uint32_t v[8];
                 row_block_load(cur, b0 + lane, v);
                 row_block_quant<LAYOUT>(cur, b0 + lane, v, absmax_words<8>(v), S, s_inv, lane);
             }
             if (more) {
 #pragma unroll
-                for (int i = 0; i < kRowBlocksPerLane; ++i) row_load_resident(nxt, i, base, w[i]);
+                for (int i = 0; i < kRowBlocksPerLane; ++i) row_load_resident(nxt, i, lane, w[i]);
             }
         }
         if (!more) break;
