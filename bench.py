@@ -62,13 +62,24 @@ def hbm_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def kernel_sources_sha() -> str:
+# The source files each timed kernel is built from (its own file plus the
+# shared device helpers): a traffic figure stays valid while these are unchanged.
+KERNEL_SOURCES = {
+    "mxfp8_grouped_kernel": ("qz_grouped.cu", "qz_device.cuh"),
+    "nvfp4_tile_kernel": ("qz_grouped.cu", "qz_device.cuh"),
+    "nvfp4_compute_l2_kernel": ("qz_grouped.cu", "qz_device.cuh"),
+    "nvfp4_rows_kernel": ("qz_rows.cu", "qz_device.cuh"),
+    "rmsnorm_quant_kernel": ("qz_rmsnorm.cu", "qz_device.cuh"),
+}
+
+
+def kernel_sources_sha(kernel: str) -> str:
+    """sha256 (first 16 hex digits) over the named kernel's source files."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "nvfp4_quantization_moe_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
-        if f.endswith((".cu", ".cuh")):
-            with open(os.path.join(csrc, f), "rb") as fh:
-                h.update(f.encode() + fh.read())
+    for f in sorted(KERNEL_SOURCES[kernel]):
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(f.encode() + fh.read())
     return h.hexdigest()[:16]
 
 
@@ -78,7 +89,7 @@ def ncu_traffic(kernel: str):
     path = os.path.join(ROOT, "profiles", "ncu_traffic.md")
     if not os.path.exists(path):
         return None
-    sha = kernel_sources_sha()
+    sha = kernel_sources_sha(kernel)
     pat = re.compile(r"^traffic: kernel=(\S+) workload=(\S+) bytes_per_launch=(\d+) sources_sha=(\w+)")
     with open(path) as f:
         for line in f:
@@ -463,7 +474,8 @@ def _extra_split(qz, device, flush, rec):
     ms = _time_graph(split_call, reps=10, flush=flush)
     nbytes = T * K * 2 + T * K // 2 + nsf_tot + T * 4
     rec("row-scaled NVFP4 split [16384,4096] over 64 Dirichlet(0.3) experts, swizzled", nbytes, ms, 1,
-        kernel="nvfp4_rows_kernel", l2="flushed before each call", timing="CUDA graph of 10 calls")
+        kernel="nvfp4_rows_kernel", l2="flushed before each call", timing="CUDA graph of 10 calls",
+        traffic=ncu_traffic("nvfp4_rows_kernel"))
     del x, q, am, entries, table
 
 
@@ -493,7 +505,8 @@ def _extra_fused(qz, device, flush, out, peak, tokens=None):
         out.append({"workload": f"fused residual+RMSNorm+{fname}, H=7168, T=1..4096 (residual_out written)",
                     "kernel": "rmsnorm_quant_kernel", "sweep": sweep,
                     "timing": "CUDA graph of 50 calls (T < 1024) or 10 calls after an L2 flush each",
-                    "frac_of_hbm_peak_T4096": round(big["GB/s"] / peak, 4)})
+                    "frac_of_hbm_peak_T4096": round(big["GB/s"] / peak, 4),
+                    "traffic_T4096": ncu_traffic("rmsnorm_quant_kernel") if fmt == qz.FMT_MXFP8 else None})
 
 
 def _extra_nvfp4_30b(qz, device, rec):
