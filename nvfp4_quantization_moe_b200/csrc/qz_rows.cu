@@ -6,13 +6,21 @@
 // swizzled padding is independent per expert (uneven and empty splits).
 //
 // One warp works on one row at a time (four independent warps per CTA, a
-// persistent grid).  Lane l owns the 16-element blocks l + 32i of the row (a
-// row of up to 4096 elements is eight 32-byte loads per lane), held in
-// registers: the row amax is a warp reduction and each block's scale is
-// computed once, by its owner.  As soon as a block is quantized its registers
-// are refilled with the same block of the warp's next row, so the next row
-// streams in while this one is processed.  The scale bytes of four
-// consecutive blocks (four consecutive lanes) leave as one 32-bit store.
+// persistent grid); each warp takes a contiguous run of rows, so consecutive
+// rows mostly share an expert and its table entry.  Lane l owns the
+// 16-element blocks l + 32i of the row (a row of up to 4096 elements is eight
+// 32-byte loads per lane), held in registers: the row amax is a warp
+// reduction and each block's scale is computed once, by its owner.  As soon
+// as a block is quantized its registers are refilled with the same block of
+// the warp's next row, so the next row streams in while this one is
+// processed.
+//
+// Per row, the element multipliers RN(S / value(s)) of all 127 finite e4m3
+// scale codes s are tabulated once in the warp's shared memory (four exact
+// quotients per lane), so a block's multiplier is one table read.  Block
+// amaxes use the packed bf16 magnitude maximum; the block scales, the element
+// products and the e2m1 conversions run on packed f32 pairs.  The row's scale
+// bytes are gathered in shared memory and leave as 32-bit stores.
 // Rows longer than 4096 elements take a two-pass path (amax pass, then a
 // quantize pass re-reading the row from L2).
 //
@@ -28,6 +36,7 @@ constexpr int kRowThreads = 128;                          // four independent wa
 constexpr int kRowWarps = kRowThreads / 32;
 constexpr int kRowBlocksPerLane = 8;                      // register-resident blocks per lane
 constexpr int kRowMaxResident = 32 * kRowBlocksPerLane;   // blocks of a register-resident row (4096 elements)
+constexpr int kRcpCodes = 128;                            // e4m3 codes 0..127 (0x7F is never produced)
 
 template <int LAYOUT>
 struct RowUnits {
@@ -42,28 +51,124 @@ struct RowUnits {
     }
 };
 
+// ---------------------------------------------------------------------------
+// packed arithmetic (PTX ISA 8.6: f32x2 add/mul/fma on sm_100; bf16x2 max)
+// ---------------------------------------------------------------------------
+
+// Packed bf16 maximum of magnitudes: each half holds the larger |x| of the two
+// inputs' halves (its sign bit is the xor of theirs and is dropped later).
+__device__ __forceinline__ uint32_t max_abs_bf16x2(uint32_t a, uint32_t b) {
+    uint32_t r;
+    asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+
+// Largest |x| of the 16 bf16 in w, as bf16 magnitude bits.
+__device__ __forceinline__ uint32_t block_absmax(const uint32_t (&w)[8]) {
+    const uint32_t m = max_abs_bf16x2(max_abs_bf16x2(max_abs_bf16x2(w[0], w[1]), max_abs_bf16x2(w[2], w[3])),
+                                      max_abs_bf16x2(max_abs_bf16x2(w[4], w[5]), max_abs_bf16x2(w[6], w[7])));
+    const uint32_t a = m & 0x7FFF7FFFu;
+    return max(a & 0xFFFFu, a >> 16);
+}
+
+// Eight e2m1 codes of the bf16 pairs in a..d times s (element 0 lowest):
+// each pair is widened to two binary32 values, multiplied by s as one packed
+// RN product, and converted by cvt.rn.satfinite.e2m1x2 (first operand to the
+// upper nibble).
+__device__ __forceinline__ uint32_t e2m1x8_pairs(uint32_t a, uint32_t b, uint32_t c, uint32_t d, float s) {
+    uint32_t r;
+    asm("{\n\t"
+        ".reg .b32 l0, h0, l1, h1, l2, h2, l3, h3;\n\t"
+        ".reg .b64 p0, p1, p2, p3, ss;\n\t"
+        ".reg .b8 q0, q1, q2, q3;\n\t"
+        "mov.b64 ss, {%5, %5};\n\t"
+        "shl.b32 l0, %1, 16;\n\tand.b32 h0, %1, -65536;\n\tmov.b64 p0, {l0, h0};\n\t"
+        "shl.b32 l1, %2, 16;\n\tand.b32 h1, %2, -65536;\n\tmov.b64 p1, {l1, h1};\n\t"
+        "shl.b32 l2, %3, 16;\n\tand.b32 h2, %3, -65536;\n\tmov.b64 p2, {l2, h2};\n\t"
+        "shl.b32 l3, %4, 16;\n\tand.b32 h3, %4, -65536;\n\tmov.b64 p3, {l3, h3};\n\t"
+        "mul.rn.f32x2 p0, p0, ss;\n\tmul.rn.f32x2 p1, p1, ss;\n\t"
+        "mul.rn.f32x2 p2, p2, ss;\n\tmul.rn.f32x2 p3, p3, ss;\n\t"
+        "mov.b64 {l0, h0}, p0;\n\tmov.b64 {l1, h1}, p1;\n\tmov.b64 {l2, h2}, p2;\n\tmov.b64 {l3, h3}, p3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 q0, h0, l0;\n\tcvt.rn.satfinite.e2m1x2.f32 q1, h1, l1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 q2, h2, l2;\n\tcvt.rn.satfinite.e2m1x2.f32 q3, h3, l3;\n\t"
+        "mov.b32 %0, {q0, q1, q2, q3};\n\t"
+        "}"
+        : "=r"(r)
+        : "r"(a), "r"(b), "r"(c), "r"(d), "f"(s));
+    return r;
+}
+
+// e4m3 codes of RN(RN(b/6) * S) for two block amaxes b0, b1 (code of b0 in
+// bits 0-7, of b1 in bits 8-15), with RN(b/6) by the same quotient
+// correction as div6_rn (q0 = RN(b * RN(1/6)), r = b - 6 q0 exactly,
+// RN(q0 + r * RN(1/6))), on packed pairs.  b = 0 gives code 0.
+__device__ __forceinline__ uint32_t nvfp4_scale_pair(float b0, float b1, float S) {
+    uint16_t r;
+    asm("{\n\t"
+        ".reg .b64 b, c, m6, ss, q, t;\n\t"
+        ".reg .f32 lo, hi;\n\t"
+        "mov.b64 b, {%1, %2};\n\t"
+        "mov.b64 c, {%4, %4};\n\t"
+        "mov.b64 m6, {%5, %5};\n\t"
+        "mov.b64 ss, {%3, %3};\n\t"
+        "mul.rn.f32x2 q, b, c;\n\t"
+        "fma.rn.f32x2 t, q, m6, b;\n\t"
+        "fma.rn.f32x2 q, t, c, q;\n\t"
+        "mul.rn.f32x2 q, q, ss;\n\t"
+        "mov.b64 {lo, hi}, q;\n\t"
+        "cvt.rn.satfinite.e4m3x2.f32 %0, hi, lo;\n\t"
+        "}"
+        : "=h"(r)
+        : "f"(b0), "f"(b1), "f"(S), "f"(1.0f / 6.0f), "f"(-6.0f));
+    return r;
+}
+
+// ---------------------------------------------------------------------------
+// rows
+// ---------------------------------------------------------------------------
+
+// Where a warp reads one virtual row from (all a prefetch needs).
+struct RowSrc {
+    const uint16_t* x;  // row start
+    int kv;             // blocks per row
+    bool resident;      // live row with kv <= 256: read into registers
+    bool a32;           // 32-byte aligned rows
+};
+
 // One warp's view of one virtual row.
 struct RowRef {
-    const uint16_t* x;  // row start
+    RowSrc src;
     uint8_t* q;         // payload row start
     uint8_t* sfrow;     // swizzled: the row's byte of scale column 0; linear: the row's first SF byte
     float* amax;        // the row's amax slot
     int kv;             // blocks per row
     bool live;          // row < rows (else a padded row of the swizzled region)
-    bool a32;           // 32-byte aligned rows
     bool q8;            // payload row 8-byte aligned
 };
 
+// Row `row` of expert entry E, read side.
+__device__ __forceinline__ RowSrc row_src_of(const qz_expert& E, int64_t row) {
+    RowSrc r;
+    r.x = static_cast<const uint16_t*>(E.x) + row * E.ld;
+    r.kv = (int)(E.cols >> 4);
+    r.resident = row < E.rows && r.kv <= kRowMaxResident;
+    r.a32 = ((reinterpret_cast<uintptr_t>(E.x) & 31) == 0) && ((E.ld & 15) == 0);
+    return r;
+}
+
+__device__ __forceinline__ RowSrc row_src_at(const qz_expert* table, int e, int64_t row) {
+    return row_src_of(load_entry(table, e), row);
+}
+
+// Row `row` of expert e.
 template <int LAYOUT>
-__device__ __forceinline__ RowRef row_ref(const qz_expert* table, const int* s_prefix, int n, int u) {
-    const int e = find_owner(s_prefix, n, u);
+__device__ __forceinline__ RowRef row_ref_at(const qz_expert* table, int e, int64_t row) {
     const qz_expert E = load_entry(table, e);
     RowRef r;
-    const int64_t row = u - s_prefix[e];
+    r.src = row_src_of(E, row);
     r.live = row < E.rows;
-    r.x = static_cast<const uint16_t*>(E.x) + row * E.ld;
     r.q = static_cast<uint8_t*>(E.q) + row * (E.cols >> 1);
-    r.kv = (int)(E.cols >> 4);
+    r.kv = r.src.kv;
     if (LAYOUT == QZ_SF_SWIZZLED_128x4) {
         const int64_t col_tiles = (r.kv + 3) >> 2;
         const int rr = (int)(row & 127);
@@ -72,13 +177,12 @@ __device__ __forceinline__ RowRef row_ref(const qz_expert* table, const int* s_p
         r.sfrow = E.sf + row * r.kv;
     }
     r.amax = E.amax + row;
-    r.a32 = ((reinterpret_cast<uintptr_t>(E.x) & 31) == 0) && ((E.ld & 15) == 0);
     r.q8 = ((reinterpret_cast<uintptr_t>(r.q)) & 7) == 0;
     return r;
 }
 
 // Block b of the row (zeros past the row).
-__device__ __forceinline__ void row_block_load(const RowRef& r, int b, uint32_t (&w)[8]) {
+__device__ __forceinline__ void row_block_load(const RowSrc& r, int b, uint32_t (&w)[8]) {
     if (b < r.kv) {
         if (r.a32) ld_stream_32(r.x + b * 16, w);
         else ld_pair_16(r.x + b * 16, w);
@@ -89,8 +193,8 @@ __device__ __forceinline__ void row_block_load(const RowRef& r, int b, uint32_t 
 }
 
 // The lane's register-resident block i (lane + 32 i) of a live row with kv <= 256.
-__device__ __forceinline__ void row_load_resident(const RowRef& r, int i, int lane, uint32_t (&w)[8]) {
-    if (r.live && r.kv <= kRowMaxResident) {
+__device__ __forceinline__ void row_load_resident(const RowSrc& r, int i, int lane, uint32_t (&w)[8]) {
+    if (r.resident) {
         row_block_load(r, lane + 32 * i, w);
     } else {
 #pragma unroll
@@ -98,28 +202,8 @@ __device__ __forceinline__ void row_load_resident(const RowRef& r, int i, int la
     }
 }
 
-// Store the scale group of blocks k0..k0+3 (k0 % 4 == 0), bytes in `word`.
-template <int LAYOUT>
-__device__ __forceinline__ void store_scale_group(const RowRef& r, int k0, uint32_t word) {
-    if (LAYOUT == QZ_SF_SWIZZLED_128x4) {
-        if (k0 < ((r.kv + 3) & ~3)) st_u32(r.sfrow + ((k0 >> 2) << 9), word);
-    } else {
-        uint8_t* p = r.sfrow + k0;
-        if (k0 + 4 <= r.kv && (((uintptr_t)p) & 3) == 0) {
-            st_u32(p, word);
-        } else {
-            for (int j = 0; j < 4 && k0 + j < r.kv; ++j) p[j] = (uint8_t)(word >> (8 * j));
-        }
-    }
-}
-
-// Quantize block b (words w) with its scale blk; four consecutive lanes'
-// scale bytes leave as one store (all lanes call this).
-template <int LAYOUT>
-__device__ __forceinline__ void row_block_store(const RowRef& r, int b, const uint32_t (&w)[8], Nvfp4Block blk,
-                                                int lane) {
-    const uint32_t c0 = e2m1x8_words(w[0], w[1], w[2], w[3], blk.rcp);
-    const uint32_t c1 = e2m1x8_words(w[4], w[5], w[6], w[7], blk.rcp);
+// Payload bytes of block b (codes c0: elements 0-7, c1: 8-15).
+__device__ __forceinline__ void row_payload_store(const RowRef& r, int b, uint32_t c0, uint32_t c1) {
     if (b < r.kv) {
         if (r.q8) {
             st_v2(r.q + b * 8, c0, c1);
@@ -128,22 +212,86 @@ __device__ __forceinline__ void row_block_store(const RowRef& r, int b, const ui
             st_u32(r.q + b * 8 + 4, c1);
         }
     }
+}
+
+// The row's scale bytes, gathered in the warp's shared buffer `bytes`
+// (pad(kv, 4) of them; entries past kv are zero), to their layout.
+template <int LAYOUT>
+__device__ __forceinline__ void row_scales_store(const RowRef& r, const uint32_t* words, int lane) {
+    if (LAYOUT == QZ_SF_SWIZZLED_128x4) {
+        // word j holds scale columns 4j..4j+3: one 32-bit store per column tile
+        const int nw = (r.kv + 3) >> 2;
+        for (int j = lane; j < nw; j += 32) st_u32(r.sfrow + (j << 9), words[j]);
+    } else {
+        const uint8_t* bytes = reinterpret_cast<const uint8_t*>(words);
+        int k0 = 0;
+        if ((reinterpret_cast<uintptr_t>(r.sfrow) & 3) == 0) {
+            for (int j = lane; j < (r.kv >> 2); j += 32) st_u32(r.sfrow + 4 * j, words[j]);
+            k0 = r.kv & ~3;
+        }
+        for (int k = k0 + lane; k < r.kv; k += 32) r.sfrow[k] = bytes[k];
+    }
+}
+
+// Block b's quantization for the long-row path, scale bytes gathered from
+// four consecutive lanes by shuffles (all lanes call this).
+template <int LAYOUT>
+__device__ __forceinline__ void row_block_quant(const RowRef& r, int b, const uint32_t (&w)[8], float S,
+                                                const float* inv, int lane) {
+    const Nvfp4Block blk = nvfp4_block(bits_to_float_bf16(block_absmax(w)), S, inv);
+    row_payload_store(r, b, e2m1x8_pairs(w[0], w[1], w[2], w[3], blk.rcp), e2m1x8_pairs(w[4], w[5], w[6], w[7], blk.rcp));
     const uint32_t s1 = __shfl_down_sync(0xFFFFFFFFu, blk.scale, 1);
     const uint32_t s2 = __shfl_down_sync(0xFFFFFFFFu, blk.scale, 2);
     const uint32_t s3 = __shfl_down_sync(0xFFFFFFFFu, blk.scale, 3);
-    if ((lane & 3) == 0) store_scale_group<LAYOUT>(r, b, blk.scale | (s1 << 8) | (s2 << 16) | (s3 << 24));
+    if ((lane & 3) == 0) {
+        const uint32_t word = blk.scale | (s1 << 8) | (s2 << 16) | (s3 << 24);
+        if (LAYOUT == QZ_SF_SWIZZLED_128x4) {
+            if (b < ((r.kv + 3) & ~3)) st_u32(r.sfrow + ((b >> 2) << 9), word);
+        } else {
+            uint8_t* p = r.sfrow + b;
+            if (b + 4 <= r.kv && (((uintptr_t)p) & 3) == 0) {
+                st_u32(p, word);
+            } else {
+                for (int j = 0; j < 4 && b + j < r.kv; ++j) p[j] = (uint8_t)(word >> (8 * j));
+            }
+        }
+    }
 }
 
-template <int LAYOUT>
-__device__ __forceinline__ void row_block_quant(const RowRef& r, int b, const uint32_t (&w)[8], uint32_t m, float S,
-                                                const float* inv, int lane) {
-    row_block_store<LAYOUT>(r, b, w, nvfp4_block(bits_to_float_bf16(m), S, inv), lane);
+__device__ __forceinline__ uint32_t warp_max(uint32_t m) { return __reduce_max_sync(0xFFFFFFFFu, m); }
+
+// Encode scale S = RN(1 / RN(A / 2688)) of a row amax A (a bf16 value),
+// zero when the decode scale is zero.  RN(A / 2688) uses the quotient
+// correction of Markstein (IBM J. Res. Dev. 34(1), 1990): q0 = RN(A * RN(1/2688)),
+// r = A - 2688 q0 exactly (one FMA), RN(q0 + r * RN(1/2688)).  A has 8
+// significant bits and 2688 = 21 * 2^7, so A / 2688 is a multiple of an odd
+// fraction k/21 of an ulp away from the representable grid and never within
+// 1/42 ulp of a rounding midpoint: the correction returns the correctly
+// rounded quotient (checked against IEEE division for every bf16 A >= 2^-100
+// in the test suite).
+__device__ __forceinline__ float row_encode_scale(float A) {
+    const float c = 1.0f / 2688.0f;
+    const float q0 = __fmul_rn(A, c);
+    const float r = __fmaf_rn(-q0, 2688.0f, A);
+    const float g = __fmaf_rn(r, c, q0);
+    return g == 0.0f ? 0.0f : __frcp_rn(g);
 }
 
-__device__ __forceinline__ uint32_t warp_max(uint32_t m) {
+// The element multiplier of every e4m3 code for encode scale S: code 0 (a
+// zero block) gets 0, a subnormal quotient is flushed to zero.  Code 0x7F is
+// NaN in e4m3 and never produced by the saturating conversion; its entry is
+// unused.
+__device__ __forceinline__ void fill_rcp_table(float* tab, float S, const float* inv, int lane) {
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
-    return m;
+    for (int j = 0; j < kRcpCodes / 32; ++j) {
+        const uint32_t c = (uint32_t)(lane + 32 * j);
+        float q = 0.0f;
+        if (c != 0u) {
+            q = div_by_e4m3(S, c, inv);
+            if (q < 0x1p-126f) q = 0.0f;
+        }
+        tab[c] = q;
+    }
 }
 
 template <int LAYOUT>
@@ -152,24 +300,36 @@ __global__ void __launch_bounds__(kRowThreads) nvfp4_rows_kernel(const qz_expert
     extern __shared__ int s_prefix[];
     __shared__ long long s_scan[33];
     __shared__ float s_inv[16];
+    __shared__ float s_rcp[kRowWarps][kRcpCodes];
+    __shared__ uint32_t s_sfw[kRowWarps][kRowMaxResident / 4];
     fill_inv_table(s_inv);
     const int total = block_prefix(n, s_prefix, s_scan, RowUnits<LAYOUT>{table, d_err}, d_err);  // has barriers
-    const int lane = threadIdx.x & 31;
-    const int stride = gridDim.x * kRowWarps;
-    int u = blockIdx.x * kRowWarps + (threadIdx.x >> 5);
-    if (u >= total) return;
-    RowRef cur = row_ref<LAYOUT>(table, s_prefix, n, u);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    // the warp's contiguous run of virtual rows [u, u_end)
+    const long long W = (long long)gridDim.x * kRowWarps, g = (long long)blockIdx.x * kRowWarps + warp;
+    int u = (int)(g * total / W);
+    const int u_end = (int)((g + 1) * total / W);
+    if (u >= u_end) return;  // no CTA barrier follows
+    float* rcp_tab = s_rcp[warp];
+    uint32_t* sfw = s_sfw[warp];
+    uint8_t* sfb = reinterpret_cast<uint8_t*>(sfw);
+    int e = find_owner(s_prefix, n, u);
+    RowRef cur = row_ref_at<LAYOUT>(table, e, u - s_prefix[e]);
     uint32_t w[kRowBlocksPerLane][8];
 #pragma unroll
-    for (int i = 0; i < kRowBlocksPerLane; ++i) row_load_resident(cur, i, lane, w[i]);
+    for (int i = 0; i < kRowBlocksPerLane; ++i) row_load_resident(cur.src, i, lane, w[i]);
     for (;;) {
-        const int un = u + stride;
-        const bool more = un < total;
-        const RowRef nxt = more ? row_ref<LAYOUT>(table, s_prefix, n, un) : cur;
+        const int un = u + 1;
+        const bool more = un < u_end;
+        int en = e;
+        if (more) {
+            while (un >= s_prefix[en + 1]) ++en;  // s_prefix[n] == total > un
+        }
+        const RowSrc nxt = more ? row_src_at(table, en, un - s_prefix[en]) : cur.src;
         if (!cur.live) {
             // padded row of the swizzled region: zero scale bytes only
-            const int kvp = (cur.kv + 3) & ~3;
-            for (int k0 = 4 * lane; k0 < kvp; k0 += 128) st_u32(cur.sfrow + ((k0 >> 2) << 9), 0u);
+            const int nw = (cur.kv + 3) >> 2;
+            for (int j = lane; j < nw; j += 32) st_u32(cur.sfrow + (j << 9), 0u);
             if (more) {
 #pragma unroll
                 for (int i = 0; i < kRowBlocksPerLane; ++i) row_load_resident(nxt, i, lane, w[i]);
@@ -179,20 +339,36 @@ __global__ void __launch_bounds__(kRowThreads) nvfp4_rows_kernel(const qz_expert
             uint32_t m = 0;
 #pragma unroll
             for (int i = 0; i < kRowBlocksPerLane; ++i) {
-                bm[i] = absmax_words<8>(w[i]);
+                bm[i] = block_absmax(w[i]);
                 m = max(m, bm[i]);
             }
             const float A = bits_to_float_bf16(warp_max(m));
             if (lane == 0) *cur.amax = A;
-            const float S = nvfp4_encode_scale(A);
+            const float S = row_encode_scale(A);
             const int nbp = (cur.kv + 3) & ~3;
-            // all block scales first: eight independent chains for the scheduler
-            Nvfp4Block blk[kRowBlocksPerLane];
+            __syncwarp();  // the previous row's table and scale-byte reads are done
+            fill_rcp_table(rcp_tab, S, s_inv, lane);
+            uint32_t code[kRowBlocksPerLane];
 #pragma unroll
-            for (int i = 0; i < kRowBlocksPerLane; ++i) blk[i] = nvfp4_block(bits_to_float_bf16(bm[i]), S, s_inv);
+            for (int i = 0; i < kRowBlocksPerLane; i += 2) {
+                const uint32_t two =
+                    nvfp4_scale_pair(bits_to_float_bf16(bm[i]), bits_to_float_bf16(bm[i + 1]), S);
+                code[i] = two & 0xFFu;
+                code[i + 1] = two >> 8;
+            }
+#pragma unroll
+            for (int i = 0; i < kRowBlocksPerLane; ++i)
+                if (32 * i < nbp) sfb[lane + 32 * i] = (uint8_t)code[i];  // uniform
+            __syncwarp();  // table and scale bytes complete
+            row_scales_store<LAYOUT>(cur, sfw, lane);
 #pragma unroll
             for (int i = 0; i < kRowBlocksPerLane; ++i) {
-                if (32 * i < nbp) row_block_store<LAYOUT>(cur, lane + 32 * i, w[i], blk[i], lane);  // uniform
+                if (32 * i < nbp) {  // uniform
+                    const float rcp = rcp_tab[code[i]];
+                    const uint32_t c0 = e2m1x8_pairs(w[i][0], w[i][1], w[i][2], w[i][3], rcp);
+                    const uint32_t c1 = e2m1x8_pairs(w[i][4], w[i][5], w[i][6], w[i][7], rcp);
+                    row_payload_store(cur, lane + 32 * i, c0, c1);
+                }
                 // refill with the next row's block as soon as this one is consumed
                 if (more) row_load_resident(nxt, i, lane, w[i]);
             }
@@ -201,17 +377,17 @@ __global__ void __launch_bounds__(kRowThreads) nvfp4_rows_kernel(const qz_expert
             uint32_t m = 0;
             for (int b = lane; b < cur.kv; b += 32) {
                 uint32_t v[8];
-                row_block_load(cur, b, v);
-                m = max(m, absmax_words<8>(v));
+                row_block_load(cur.src, b, v);
+                m = max(m, block_absmax(v));
             }
             const float A = bits_to_float_bf16(warp_max(m));
             if (lane == 0) *cur.amax = A;
-            const float S = nvfp4_encode_scale(A);
+            const float S = row_encode_scale(A);
             const int nbp = (cur.kv + 3) & ~3;
             for (int b0 = 0; b0 < nbp; b0 += 32) {
                 uint32_t v[8];
-                row_block_load(cur, b0 + lane, v);
-                row_block_quant<LAYOUT>(cur, b0 + lane, v, absmax_words<8>(v), S, s_inv, lane);
+                row_block_load(cur.src, b0 + lane, v);
+                row_block_quant<LAYOUT>(cur, b0 + lane, v, S, s_inv, lane);
             }
             if (more) {
 #pragma unroll
@@ -219,8 +395,9 @@ __global__ void __launch_bounds__(kRowThreads) nvfp4_rows_kernel(const qz_expert
             }
         }
         if (!more) break;
-        cur = nxt;
         u = un;
+        e = en;
+        cur = row_ref_at<LAYOUT>(table, e, u - s_prefix[e]);
     }
 }
 
