@@ -82,18 +82,43 @@ __device__ __forceinline__ void st_v4(void* p, uint4 v) {
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
-// Largest |x| of the 8 bf16 in v, as bf16 magnitude bits.  For non-negative
-// IEEE values the integer order of the bit patterns is the numeric order.
-__device__ __forceinline__ uint32_t max_u16x2(uint32_t a, uint32_t b) {
+// Packed bf16 maximum of magnitudes (PTX max.xorsign.abs.bf16x2): each half
+// holds the larger |x| of the two inputs' halves; its sign bit is the xor of
+// theirs and is dropped by the callers.  Subnormal bf16 values are ordered
+// exactly (there is no flush for bf16).
+__device__ __forceinline__ uint32_t max_abs_bf16x2(uint32_t a, uint32_t b) {
     uint32_t r;
-    asm("max.u16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
     return r;
 }
 
+// bf16 magnitude bits of the larger half of a packed magnitude pair (for
+// non-negative IEEE values the integer order of the bit patterns is the
+// numeric order).
+__device__ __forceinline__ uint32_t larger_half(uint32_t m) {
+    const uint32_t a = m & 0x7FFF7FFFu;
+    return max(a & 0xFFFFu, a >> 16);
+}
+
+// Largest |x| of the bf16 pairs in w[0..N) (N a power of two), as bf16
+// magnitude bits: a tree of packed magnitude maxima.
+template <int N>
+__device__ __forceinline__ uint32_t absmax_words(const uint32_t* w) {
+    static_assert(N >= 1 && (N & (N - 1)) == 0, "N must be a power of two");
+    uint32_t m[N];
+#pragma unroll
+    for (int i = 0; i < N; ++i) m[i] = w[i];
+#pragma unroll
+    for (int s = 1; s < N; s <<= 1) {
+#pragma unroll
+        for (int i = 0; i + s < N; i += 2 * s) m[i] = max_abs_bf16x2(m[i], m[i + s]);
+    }
+    return larger_half(m[0]);
+}
+
+// Largest |x| of the 8 bf16 in v, as bf16 magnitude bits.
 __device__ __forceinline__ uint32_t absmax_bits(uint4 v) {
-    const uint32_t m = max_u16x2(max_u16x2(v.x & 0x7FFF7FFFu, v.y & 0x7FFF7FFFu),
-                                 max_u16x2(v.z & 0x7FFF7FFFu, v.w & 0x7FFF7FFFu));
-    return max(m & 0xFFFFu, m >> 16);
+    return larger_half(max_abs_bf16x2(max_abs_bf16x2(v.x, v.y), max_abs_bf16x2(v.z, v.w)));
 }
 
 __device__ __forceinline__ float bits_to_float_bf16(uint32_t m16) { return __uint_as_float(m16 << 16); }
@@ -132,52 +157,64 @@ __device__ __forceinline__ uint32_t cvt_e4m3x2(float lo, float hi) {
     return r;
 }
 
-// Eight e4m3 codes of x[i] * s, element 0 in the lowest byte.
-__device__ __forceinline__ uint2 e4m3x8_scaled(uint4 v, float s) {
-    const uint32_t a = cvt_e4m3x2(__fmul_rn(bf16_lo(v.x), s), __fmul_rn(bf16_hi(v.x), s));
-    const uint32_t b = cvt_e4m3x2(__fmul_rn(bf16_lo(v.y), s), __fmul_rn(bf16_hi(v.y), s));
-    const uint32_t c = cvt_e4m3x2(__fmul_rn(bf16_lo(v.z), s), __fmul_rn(bf16_hi(v.z), s));
-    const uint32_t d = cvt_e4m3x2(__fmul_rn(bf16_lo(v.w), s), __fmul_rn(bf16_hi(v.w), s));
-    return make_uint2(a | (b << 16), c | (d << 16));
-}
-
-// Eight e2m1 codes of x[i] * s, element 0 in the lowest nibble.
-__device__ __forceinline__ uint32_t e2m1x8_scaled(uint4 v, float s) {
-    uint32_t r;
-    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
-        "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
-        "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
-        "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
-        "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
-        "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
-        : "=r"(r)
-        : "f"(__fmul_rn(bf16_lo(v.x), s)), "f"(__fmul_rn(bf16_hi(v.x), s)),
-          "f"(__fmul_rn(bf16_lo(v.y), s)), "f"(__fmul_rn(bf16_hi(v.y), s)),
-          "f"(__fmul_rn(bf16_lo(v.z), s)), "f"(__fmul_rn(bf16_hi(v.z), s)),
-          "f"(__fmul_rn(bf16_lo(v.w), s)), "f"(__fmul_rn(bf16_hi(v.w), s)));
-    return r;
-}
+// The element products of the format conversions: each bf16 pair of a word
+// is widened to two binary32 values and multiplied by s as one packed
+// round-to-nearest product (PTX ISA 8.6 mul.rn.f32x2, sm_100), i.e. RN(x * s)
+// for each element, exactly as two scalar products.
 
 // Four e4m3 codes of the bf16 pairs in words a, b times s (element 0 lowest).
 __device__ __forceinline__ uint32_t e4m3x4_words(uint32_t a, uint32_t b, float s) {
-    const uint32_t lo = cvt_e4m3x2(__fmul_rn(bf16_lo(a), s), __fmul_rn(bf16_hi(a), s));
-    const uint32_t hi = cvt_e4m3x2(__fmul_rn(bf16_lo(b), s), __fmul_rn(bf16_hi(b), s));
-    return lo | (hi << 16);
+    uint32_t r;
+    asm("{\n\t"
+        ".reg .b32 l0, h0, l1, h1;\n\t"
+        ".reg .b64 p0, p1, ss;\n\t"
+        ".reg .b16 c0, c1;\n\t"
+        "mov.b64 ss, {%3, %3};\n\t"
+        "shl.b32 l0, %1, 16;\n\tand.b32 h0, %1, -65536;\n\tmov.b64 p0, {l0, h0};\n\t"
+        "shl.b32 l1, %2, 16;\n\tand.b32 h1, %2, -65536;\n\tmov.b64 p1, {l1, h1};\n\t"
+        "mul.rn.f32x2 p0, p0, ss;\n\tmul.rn.f32x2 p1, p1, ss;\n\t"
+        "mov.b64 {l0, h0}, p0;\n\tmov.b64 {l1, h1}, p1;\n\t"
+        "cvt.rn.satfinite.e4m3x2.f32 c0, h0, l0;\n\tcvt.rn.satfinite.e4m3x2.f32 c1, h1, l1;\n\t"
+        "mov.b32 %0, {c0, c1};\n\t"
+        "}"
+        : "=r"(r)
+        : "r"(a), "r"(b), "f"(s));
+    return r;
 }
 
-// Eight e2m1 codes of the bf16 pairs in words a..d times s (element 0 lowest).
+// Eight e4m3 codes of x[i] * s, element 0 in the lowest byte.
+__device__ __forceinline__ uint2 e4m3x8_scaled(uint4 v, float s) {
+    return make_uint2(e4m3x4_words(v.x, v.y, s), e4m3x4_words(v.z, v.w, s));
+}
+
+// Eight e2m1 codes of the bf16 pairs in words a..d times s (element 0 in the
+// lowest nibble; cvt.rn.satfinite.e2m1x2 puts its first operand in the upper
+// nibble).
 __device__ __forceinline__ uint32_t e2m1x8_words(uint32_t a, uint32_t b, uint32_t c, uint32_t d, float s) {
-    return e2m1x8_scaled(make_uint4(a, b, c, d), s);
+    uint32_t r;
+    asm("{\n\t"
+        ".reg .b32 l0, h0, l1, h1, l2, h2, l3, h3;\n\t"
+        ".reg .b64 p0, p1, p2, p3, ss;\n\t"
+        ".reg .b8 q0, q1, q2, q3;\n\t"
+        "mov.b64 ss, {%5, %5};\n\t"
+        "shl.b32 l0, %1, 16;\n\tand.b32 h0, %1, -65536;\n\tmov.b64 p0, {l0, h0};\n\t"
+        "shl.b32 l1, %2, 16;\n\tand.b32 h1, %2, -65536;\n\tmov.b64 p1, {l1, h1};\n\t"
+        "shl.b32 l2, %3, 16;\n\tand.b32 h2, %3, -65536;\n\tmov.b64 p2, {l2, h2};\n\t"
+        "shl.b32 l3, %4, 16;\n\tand.b32 h3, %4, -65536;\n\tmov.b64 p3, {l3, h3};\n\t"
+        "mul.rn.f32x2 p0, p0, ss;\n\tmul.rn.f32x2 p1, p1, ss;\n\t"
+        "mul.rn.f32x2 p2, p2, ss;\n\tmul.rn.f32x2 p3, p3, ss;\n\t"
+        "mov.b64 {l0, h0}, p0;\n\tmov.b64 {l1, h1}, p1;\n\tmov.b64 {l2, h2}, p2;\n\tmov.b64 {l3, h3}, p3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 q0, h0, l0;\n\tcvt.rn.satfinite.e2m1x2.f32 q1, h1, l1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 q2, h2, l2;\n\tcvt.rn.satfinite.e2m1x2.f32 q3, h3, l3;\n\t"
+        "mov.b32 %0, {q0, q1, q2, q3};\n\t"
+        "}"
+        : "=r"(r)
+        : "r"(a), "r"(b), "r"(c), "r"(d), "f"(s));
+    return r;
 }
 
-// Largest |x| of the bf16 pairs in w[0..N), as bf16 magnitude bits.
-template <int N>
-__device__ __forceinline__ uint32_t absmax_words(const uint32_t* w) {
-    uint32_t m = w[0] & 0x7FFF7FFFu;
-#pragma unroll
-    for (int i = 1; i < N; ++i) m = max_u16x2(m, w[i] & 0x7FFF7FFFu);
-    return max(m & 0xFFFFu, m >> 16);
-}
+// Eight e2m1 codes of x[i] * s, element 0 in the lowest nibble.
+__device__ __forceinline__ uint32_t e2m1x8_scaled(uint4 v, float s) { return e2m1x8_words(v.x, v.y, v.z, v.w, s); }
 
 // e4m3 code (RNE, satfinite) of one non-negative float.
 __device__ __forceinline__ uint32_t e4m3_of(float v) { return cvt_e4m3x2(v, 0.0f) & 0xFFu; }
@@ -253,6 +290,39 @@ __device__ __forceinline__ Nvfp4Block nvfp4_block(float b, float S, const float*
         const float q = div_by_e4m3(S, r.scale, inv);
         r.rcp = (q < 0x1p-126f) ? 0.0f : q;  // flush a subnormal reciprocal to zero
     }
+    return r;
+}
+
+// Element multiplier of e4m3 scale code s: 0 for s = 0, else
+// FTZ(RN(S / value(s))).
+__device__ __forceinline__ float nvfp4_rcp(float S, uint32_t s, const float* inv) {
+    if (s == 0u) return 0.0f;
+    const float q = div_by_e4m3(S, s, inv);
+    return (q < 0x1p-126f) ? 0.0f : q;
+}
+
+// e4m3 codes of RN(RN(b/6) * S) for two block amaxes b0, b1 (code of b0 in
+// bits 0-7, of b1 in bits 8-15): the block scales of nvfp4_block, two at a
+// time on packed f32 pairs, with RN(b/6) by the quotient correction of
+// div6_rn.  b = 0 gives code 0.
+__device__ __forceinline__ uint32_t nvfp4_scale_pair(float b0, float b1, float S) {
+    uint16_t r;
+    asm("{\n\t"
+        ".reg .b64 b, c, m6, ss, q, t;\n\t"
+        ".reg .f32 lo, hi;\n\t"
+        "mov.b64 b, {%1, %2};\n\t"
+        "mov.b64 c, {%4, %4};\n\t"
+        "mov.b64 m6, {%5, %5};\n\t"
+        "mov.b64 ss, {%3, %3};\n\t"
+        "mul.rn.f32x2 q, b, c;\n\t"
+        "fma.rn.f32x2 t, q, m6, b;\n\t"
+        "fma.rn.f32x2 q, t, c, q;\n\t"
+        "mul.rn.f32x2 q, q, ss;\n\t"
+        "mov.b64 {lo, hi}, q;\n\t"
+        "cvt.rn.satfinite.e4m3x2.f32 %0, hi, lo;\n\t"
+        "}"
+        : "=h"(r)
+        : "f"(b0), "f"(b1), "f"(S), "f"(1.0f / 6.0f), "f"(-6.0f));
     return r;
 }
 
@@ -426,6 +496,13 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
         if (clock64() - t0 > (1LL << 31)) return false;
     }
     return true;
+}
+
+// A strong (L2-coherent) load without ordering of its own.
+__device__ __forceinline__ unsigned ld_relaxed_gpu(const unsigned* p) {
+    unsigned v;
+    asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
 }
 
 __device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* p) {

@@ -152,46 +152,59 @@ __device__ __forceinline__ void tile_load(const TileRef& t, int p, uint32_t* w) 
     }
 }
 
-// Quantize the lane's block of pass p; swizzled scale bytes go to the warp's
+// Scale byte of the lane's block of pass p: swizzled bytes go to the warp's
 // staging area s (64 bytes per 4-column scale tile), linear ones to memory.
 template <int FMT, int LAYOUT>
-__device__ __forceinline__ void tile_pass(const TileRef& t, int p, int lane, const uint32_t* w, float S, uint8_t* s,
-                                          const float* inv) {
+__device__ __forceinline__ void tile_scale_store(const TileRef& t, int p, int lane, uint32_t scale, uint8_t* s) {
     using G = TileGeo<FMT>;
     const bool live = pass_live<FMT>(t, p);
     const int l = local_row<FMT>(p, lane);
     const int kb = lane % G::kLpr;
-    const uint32_t m = absmax_words<G::kWords>(w);
-    uint32_t scale;
-    if (FMT == QZ_FMT_MXFP8) {
-        scale = e8m0_byte(m);
-        const float r = e8m0_reciprocal(scale);
-        uint4 c0, c1;
-        c0.x = e4m3x4_words(w[0], w[1], r);
-        c0.y = e4m3x4_words(w[2], w[3], r);
-        c0.z = e4m3x4_words(w[4], w[5], r);
-        c0.w = e4m3x4_words(w[6], w[7], r);
-        c1.x = e4m3x4_words(w[8], w[9], r);
-        c1.y = e4m3x4_words(w[10], w[11], r);
-        c1.z = e4m3x4_words(w[12], w[13], r);
-        c1.w = e4m3x4_words(w[14], w[15], r);
-        if (live) {
-            uint8_t* dst = t.qp + p * G::kRpp * 8 * t.qld;
-            st_v4(dst, c0);
-            st_v4(dst + 16, c1);
-        }
-    } else {
-        const Nvfp4Block blk = nvfp4_block(bits_to_float_bf16(m), S, inv);
-        scale = blk.scale;
-        const uint32_t c0 = e2m1x8_words(w[0], w[1], w[2], w[3], blk.rcp);
-        const uint32_t c1 = e2m1x8_words(w[4], w[5], w[6], w[7], blk.rcp);
-        if (live) st_v2(t.qp + p * G::kRpp * 8 * t.qld, c0, c1);
-    }
     if (LAYOUT == QZ_SF_SWIZZLED_128x4) {
         s[(kb >> 2) * 64 + (l & 3) * 16 + (l >> 2) * 4 + (kb & 3)] = live ? (uint8_t)scale : (uint8_t)0;
     } else if (live) {
         t.sfp[p * G::kRpp * 8 * t.kv] = (uint8_t)scale;
     }
+}
+
+// MXFP8: quantize the lane's 32-element block of pass p.
+template <int LAYOUT>
+__device__ __forceinline__ void tile_pass_mx(const TileRef& t, int p, int lane, const uint32_t* w, uint8_t* s) {
+    using G = TileGeo<QZ_FMT_MXFP8>;
+    const uint32_t scale = e8m0_byte(absmax_words<G::kWords>(w));
+    const float r = e8m0_reciprocal(scale);
+    uint4 c0, c1;
+    c0.x = e4m3x4_words(w[0], w[1], r);
+    c0.y = e4m3x4_words(w[2], w[3], r);
+    c0.z = e4m3x4_words(w[4], w[5], r);
+    c0.w = e4m3x4_words(w[6], w[7], r);
+    c1.x = e4m3x4_words(w[8], w[9], r);
+    c1.y = e4m3x4_words(w[10], w[11], r);
+    c1.z = e4m3x4_words(w[12], w[13], r);
+    c1.w = e4m3x4_words(w[14], w[15], r);
+    if (pass_live<QZ_FMT_MXFP8>(t, p)) {
+        uint8_t* dst = t.qp + p * G::kRpp * 8 * t.qld;
+        st_v4(dst, c0);
+        st_v4(dst + 16, c1);
+    }
+    tile_scale_store<QZ_FMT_MXFP8, LAYOUT>(t, p, lane, scale, s);
+}
+
+// NVFP4: quantize the lane's 16-element block of pass p with scale code
+// `scale` and element multiplier rcp.
+template <int LAYOUT>
+__device__ __forceinline__ void tile_pass_nv(const TileRef& t, int p, int lane, const uint32_t* w, uint32_t scale,
+                                             float rcp, uint8_t* s) {
+    using G = TileGeo<QZ_FMT_NVFP4>;
+    const uint32_t c0 = e2m1x8_words(w[0], w[1], w[2], w[3], rcp);
+    const uint32_t c1 = e2m1x8_words(w[4], w[5], w[6], w[7], rcp);
+    if (pass_live<QZ_FMT_NVFP4>(t, p)) st_v2(t.qp + p * G::kRpp * 8 * t.qld, c0, c1);
+    tile_scale_store<QZ_FMT_NVFP4, LAYOUT>(t, p, lane, scale, s);
+}
+
+// NVFP4 block scale codes of passes p and p + 1 (one packed pair).
+__device__ __forceinline__ uint32_t tile_scales_nv(const uint32_t* w0, const uint32_t* w1, float S) {
+    return nvfp4_scale_pair(bits_to_float_bf16(absmax_words<8>(w0)), bits_to_float_bf16(absmax_words<8>(w1)), S);
 }
 
 // Store the warp's staged chunks of the tile's swizzled scale tile(s).
@@ -233,10 +246,22 @@ __global__ void __launch_bounds__(kThreads, 3) grouped_tile_kernel(const qz_expe
         const bool more = next < total;
         const TileRef nxt = more ? tile_ref<FMT, LAYOUT>(table, s_prefix, n, next, w, lane) : cur;
         const float S = kAmax ? nvfp4_encode_scale(*cur.amax) : 0.0f;
+        if (FMT == QZ_FMT_MXFP8) {
 #pragma unroll
-        for (int p = 0; p < G::kPasses; ++p) {
-            tile_pass<FMT, LAYOUT>(cur, p, lane, v[p], S, s_sf[w], s_inv);
-            if (more) tile_load<FMT>(nxt, p, v[p]);
+            for (int p = 0; p < G::kPasses; ++p) {
+                tile_pass_mx<LAYOUT>(cur, p, lane, v[p], s_sf[w]);
+                if (more) tile_load<FMT>(nxt, p, v[p]);
+            }
+        } else {
+#pragma unroll
+            for (int p = 0; p < G::kPasses; p += 2) {
+                const uint32_t sc = tile_scales_nv(v[p], v[p + 1], S);
+                const uint32_t sc0 = sc & 0xFFu, sc1 = sc >> 8;
+                tile_pass_nv<LAYOUT>(cur, p, lane, v[p], sc0, nvfp4_rcp(S, sc0, s_inv), s_sf[w]);
+                if (more) tile_load<FMT>(nxt, p, v[p]);
+                tile_pass_nv<LAYOUT>(cur, p + 1, lane, v[p + 1], sc1, nvfp4_rcp(S, sc1, s_inv), s_sf[w]);
+                if (more) tile_load<FMT>(nxt, p + 1, v[p + 1]);
+            }
         }
         if (LAYOUT == QZ_SF_SWIZZLED_128x4) tile_flush_sf<FMT>(cur, w, lane, s_sf[w]);
         if (!more) break;
@@ -348,7 +373,6 @@ __global__ void __launch_bounds__(kThreads, 3) nvfp4_compute_l2_kernel(const qz_
     __shared__ float s_inv[16];
     __shared__ int s_item[4];
     __shared__ unsigned s_ok[2];
-    __shared__ uint32_t s_wmax[kThreads / 32];
     fill_inv_table(s_inv);
     const int total = block_prefix(n, s_prefix, s_scan, TableTiles<QZ_FMT_NVFP4, LAYOUT, true>{table, d_err}, d_err);
     if (total == 0) return;
@@ -461,21 +485,24 @@ __global__ void __launch_bounds__(kThreads, 3) nvfp4_compute_l2_kernel(const qz_
                 if (last || nxt.expert != cur.expert) {
 #pragma unroll
                     for (int o = 16; o > 0; o >>= 1) run = max(run, __shfl_xor_sync(0xFFFFFFFFu, run, o));
-                    if (lane == 0) {
-                        atomicMax(amax_ws + cur.expert, run << 16);
-                        __threadfence();
-                    }
+                    if (lane == 0) atomicMax(amax_ws + cur.expert, run << 16);
                     run = 0;
                 }
             } else {
-                const float A = __uint_as_float(ld_acquire_gpu(amax_ws + cur.expert));
+                // ordered after thread 0's acquire of the chunk count by the barrier above
+                const float A = __uint_as_float(ld_relaxed_gpu(amax_ws + cur.expert));
                 const float S = nvfp4_encode_scale(A);
 #pragma unroll
-                for (int p = 0; p < G::kPasses; ++p) {
-                    tile_pass<QZ_FMT_NVFP4, LAYOUT>(cur, p, lane, v[p], S, s_sf[w], s_inv);
-                    if (more) {
-                        if (next_a) tile_load<QZ_FMT_NVFP4, kL2Last>(nxt, p, v[p]);
-                        else tile_load<QZ_FMT_NVFP4, kL2First>(nxt, p, v[p]);
+                for (int p = 0; p < G::kPasses; p += 2) {
+                    const uint32_t sc = tile_scales_nv(v[p], v[p + 1], S);
+#pragma unroll
+                    for (int q = 0; q < 2; ++q) {
+                        const uint32_t scq = (sc >> (8 * q)) & 0xFFu;
+                        tile_pass_nv<LAYOUT>(cur, p + q, lane, v[p + q], scq, nvfp4_rcp(S, scq, s_inv), s_sf[w]);
+                        if (more) {
+                            if (next_a) tile_load<QZ_FMT_NVFP4, kL2Last>(nxt, p + q, v[p + q]);
+                            else tile_load<QZ_FMT_NVFP4, kL2First>(nxt, p + q, v[p + q]);
+                        }
                     }
                 }
                 if (LAYOUT == QZ_SF_SWIZZLED_128x4) tile_flush_sf<QZ_FMT_NVFP4>(cur, w, lane, s_sf[w]);
@@ -484,8 +511,13 @@ __global__ void __launch_bounds__(kThreads, 3) nvfp4_compute_l2_kernel(const qz_
             cur = nxt;
         }
         if (item.is_a) {
-            __syncthreads();  // every warp's atomic max (fenced) precedes the count
-            if (threadIdx.x == 0) atomicAdd(done + item.chunk, (unsigned)item.ntiles);
+            // every warp's atomic max precedes the barrier; thread 0's fence
+            // then releases them all before the count (the grid-barrier idiom)
+            __syncthreads();
+            if (threadIdx.x == 0) {
+                __threadfence();
+                atomicAdd(done + item.chunk, (unsigned)item.ntiles);
+            }
         }
         if (!more_items) break;
         item = nitem;

@@ -18,8 +18,8 @@
 // Per row, the element multipliers RN(S / value(s)) of all 127 finite e4m3
 // scale codes s are tabulated once in the warp's shared memory (four exact
 // quotients per lane), so a block's multiplier is one table read.  Block
-// amaxes use the packed bf16 magnitude maximum; the block scales, the element
-// products and the e2m1 conversions run on packed f32 pairs.  The row's scale
+// amaxes use the packed bf16 magnitude maximum; the block scales and the
+// element products run on packed f32 pairs.  The row's scale
 // bytes are gathered in shared memory and leave as 32-bit stores.
 // Rows longer than 4096 elements take a two-pass path (amax pass, then a
 // quantize pass re-reading the row from L2).
@@ -50,78 +50,6 @@ struct RowUnits {
         return LAYOUT == QZ_SF_SWIZZLED_128x4 ? pad_to(e.rows, 128) : e.rows;
     }
 };
-
-// ---------------------------------------------------------------------------
-// packed arithmetic (PTX ISA 8.6: f32x2 add/mul/fma on sm_100; bf16x2 max)
-// ---------------------------------------------------------------------------
-
-// Packed bf16 maximum of magnitudes: each half holds the larger |x| of the two
-// inputs' halves (its sign bit is the xor of theirs and is dropped later).
-__device__ __forceinline__ uint32_t max_abs_bf16x2(uint32_t a, uint32_t b) {
-    uint32_t r;
-    asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
-    return r;
-}
-
-// Largest |x| of the 16 bf16 in w, as bf16 magnitude bits.
-__device__ __forceinline__ uint32_t block_absmax(const uint32_t (&w)[8]) {
-    const uint32_t m = max_abs_bf16x2(max_abs_bf16x2(max_abs_bf16x2(w[0], w[1]), max_abs_bf16x2(w[2], w[3])),
-                                      max_abs_bf16x2(max_abs_bf16x2(w[4], w[5]), max_abs_bf16x2(w[6], w[7])));
-    const uint32_t a = m & 0x7FFF7FFFu;
-    return max(a & 0xFFFFu, a >> 16);
-}
-
-// Eight e2m1 codes of the bf16 pairs in a..d times s (element 0 lowest):
-// each pair is widened to two binary32 values, multiplied by s as one packed
-// RN product, and converted by cvt.rn.satfinite.e2m1x2 (first operand to the
-// upper nibble).
-__device__ __forceinline__ uint32_t e2m1x8_pairs(uint32_t a, uint32_t b, uint32_t c, uint32_t d, float s) {
-    uint32_t r;
-    asm("{\n\t"
-        ".reg .b32 l0, h0, l1, h1, l2, h2, l3, h3;\n\t"
-        ".reg .b64 p0, p1, p2, p3, ss;\n\t"
-        ".reg .b8 q0, q1, q2, q3;\n\t"
-        "mov.b64 ss, {%5, %5};\n\t"
-        "shl.b32 l0, %1, 16;\n\tand.b32 h0, %1, -65536;\n\tmov.b64 p0, {l0, h0};\n\t"
-        "shl.b32 l1, %2, 16;\n\tand.b32 h1, %2, -65536;\n\tmov.b64 p1, {l1, h1};\n\t"
-        "shl.b32 l2, %3, 16;\n\tand.b32 h2, %3, -65536;\n\tmov.b64 p2, {l2, h2};\n\t"
-        "shl.b32 l3, %4, 16;\n\tand.b32 h3, %4, -65536;\n\tmov.b64 p3, {l3, h3};\n\t"
-        "mul.rn.f32x2 p0, p0, ss;\n\tmul.rn.f32x2 p1, p1, ss;\n\t"
-        "mul.rn.f32x2 p2, p2, ss;\n\tmul.rn.f32x2 p3, p3, ss;\n\t"
-        "mov.b64 {l0, h0}, p0;\n\tmov.b64 {l1, h1}, p1;\n\tmov.b64 {l2, h2}, p2;\n\tmov.b64 {l3, h3}, p3;\n\t"
-        "cvt.rn.satfinite.e2m1x2.f32 q0, h0, l0;\n\tcvt.rn.satfinite.e2m1x2.f32 q1, h1, l1;\n\t"
-        "cvt.rn.satfinite.e2m1x2.f32 q2, h2, l2;\n\tcvt.rn.satfinite.e2m1x2.f32 q3, h3, l3;\n\t"
-        "mov.b32 %0, {q0, q1, q2, q3};\n\t"
-        "}"
-        : "=r"(r)
-        : "r"(a), "r"(b), "r"(c), "r"(d), "f"(s));
-    return r;
-}
-
-// e4m3 codes of RN(RN(b/6) * S) for two block amaxes b0, b1 (code of b0 in
-// bits 0-7, of b1 in bits 8-15), with RN(b/6) by the same quotient
-// correction as div6_rn (q0 = RN(b * RN(1/6)), r = b - 6 q0 exactly,
-// RN(q0 + r * RN(1/6))), on packed pairs.  b = 0 gives code 0.
-__device__ __forceinline__ uint32_t nvfp4_scale_pair(float b0, float b1, float S) {
-    uint16_t r;
-    asm("{\n\t"
-        ".reg .b64 b, c, m6, ss, q, t;\n\t"
-        ".reg .f32 lo, hi;\n\t"
-        "mov.b64 b, {%1, %2};\n\t"
-        "mov.b64 c, {%4, %4};\n\t"
-        "mov.b64 m6, {%5, %5};\n\t"
-        "mov.b64 ss, {%3, %3};\n\t"
-        "mul.rn.f32x2 q, b, c;\n\t"
-        "fma.rn.f32x2 t, q, m6, b;\n\t"
-        "fma.rn.f32x2 q, t, c, q;\n\t"
-        "mul.rn.f32x2 q, q, ss;\n\t"
-        "mov.b64 {lo, hi}, q;\n\t"
-        "cvt.rn.satfinite.e4m3x2.f32 %0, hi, lo;\n\t"
-        "}"
-        : "=h"(r)
-        : "f"(b0), "f"(b1), "f"(S), "f"(1.0f / 6.0f), "f"(-6.0f));
-    return r;
-}
 
 // ---------------------------------------------------------------------------
 // rows
@@ -238,8 +166,8 @@ __device__ __forceinline__ void row_scales_store(const RowRef& r, const uint32_t
 template <int LAYOUT>
 __device__ __forceinline__ void row_block_quant(const RowRef& r, int b, const uint32_t (&w)[8], float S,
                                                 const float* inv, int lane) {
-    const Nvfp4Block blk = nvfp4_block(bits_to_float_bf16(block_absmax(w)), S, inv);
-    row_payload_store(r, b, e2m1x8_pairs(w[0], w[1], w[2], w[3], blk.rcp), e2m1x8_pairs(w[4], w[5], w[6], w[7], blk.rcp));
+    const Nvfp4Block blk = nvfp4_block(bits_to_float_bf16(absmax_words<8>(w)), S, inv);
+    row_payload_store(r, b, e2m1x8_words(w[0], w[1], w[2], w[3], blk.rcp), e2m1x8_words(w[4], w[5], w[6], w[7], blk.rcp));
     const uint32_t s1 = __shfl_down_sync(0xFFFFFFFFu, blk.scale, 1);
     const uint32_t s2 = __shfl_down_sync(0xFFFFFFFFu, blk.scale, 2);
     const uint32_t s3 = __shfl_down_sync(0xFFFFFFFFu, blk.scale, 3);
@@ -285,12 +213,7 @@ __device__ __forceinline__ void fill_rcp_table(float* tab, float S, const float*
 #pragma unroll
     for (int j = 0; j < kRcpCodes / 32; ++j) {
         const uint32_t c = (uint32_t)(lane + 32 * j);
-        float q = 0.0f;
-        if (c != 0u) {
-            q = div_by_e4m3(S, c, inv);
-            if (q < 0x1p-126f) q = 0.0f;
-        }
-        tab[c] = q;
+        tab[c] = nvfp4_rcp(S, c, inv);
     }
 }
 
@@ -339,7 +262,7 @@ __global__ void __launch_bounds__(kRowThreads) nvfp4_rows_kernel(const qz_expert
             uint32_t m = 0;
 #pragma unroll
             for (int i = 0; i < kRowBlocksPerLane; ++i) {
-                bm[i] = block_absmax(w[i]);
+                bm[i] = absmax_words<8>(w[i]);
                 m = max(m, bm[i]);
             }
             const float A = bits_to_float_bf16(warp_max(m));
@@ -365,8 +288,8 @@ __global__ void __launch_bounds__(kRowThreads) nvfp4_rows_kernel(const qz_expert
             for (int i = 0; i < kRowBlocksPerLane; ++i) {
                 if (32 * i < nbp) {  // uniform
                     const float rcp = rcp_tab[code[i]];
-                    const uint32_t c0 = e2m1x8_pairs(w[i][0], w[i][1], w[i][2], w[i][3], rcp);
-                    const uint32_t c1 = e2m1x8_pairs(w[i][4], w[i][5], w[i][6], w[i][7], rcp);
+                    const uint32_t c0 = e2m1x8_words(w[i][0], w[i][1], w[i][2], w[i][3], rcp);
+                    const uint32_t c1 = e2m1x8_words(w[i][4], w[i][5], w[i][6], w[i][7], rcp);
                     row_payload_store(cur, lane + 32 * i, c0, c1);
                 }
                 // refill with the next row's block as soon as this one is consumed
@@ -378,7 +301,7 @@ __global__ void __launch_bounds__(kRowThreads) nvfp4_rows_kernel(const qz_expert
             for (int b = lane; b < cur.kv; b += 32) {
                 uint32_t v[8];
                 row_block_load(cur.src, b, v);
-                m = max(m, block_absmax(v));
+                m = max(m, absmax_words<8>(v));
             }
             const float A = bits_to_float_bf16(warp_max(m));
             if (lane == 0) *cur.amax = A;
