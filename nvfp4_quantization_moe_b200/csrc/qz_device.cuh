@@ -301,6 +301,28 @@ __device__ __forceinline__ float nvfp4_rcp(float S, uint32_t s, const float* inv
     return (q < 0x1p-126f) ? 0.0f : q;
 }
 
+// Element multipliers for a whole warp from 16 exact quotients: lane m
+// (1..15) holds q_m = RN(S / m) (Markstein's correction, as in div_by_e4m3)
+// and lane 0 holds 0; the multiplier of code s = m * 2^k is then q_m * 2^-k
+// (exact scaling), read from lane m by a shuffle, and flushed to zero below
+// 2^-126 -- the same value as nvfp4_rcp(S, s, inv).  Every lane of the warp
+// must call both functions with the same S.
+__device__ __forceinline__ float rcp_lane_quotient(float S, const float* inv, int lane) {
+    if (lane < 1 || lane > 15) return 0.0f;
+    const float c = inv[lane];
+    const float q0 = __fmul_rn(S, c);
+    const float r = __fmaf_rn(-q0, (float)lane, S);
+    return __fmaf_rn(r, c, q0);
+}
+
+__device__ __forceinline__ float nvfp4_rcp_warp(float qm, uint32_t s) {
+    const uint32_t ef = s >> 3;
+    const uint32_t m = ef ? ((s & 7u) | 8u) : s;  // value(s) = m * 2^k, k = max(ef, 1) - 10
+    const float q = __shfl_sync(0xFFFFFFFFu, qm, (int)m);
+    const float r = __fmul_rn(q, __uint_as_float((137u - max(ef, 1u)) << 23));
+    return (r < 0x1p-126f) ? 0.0f : r;
+}
+
 // e4m3 codes of RN(RN(b/6) * S) for two block amaxes b0, b1 (code of b0 in
 // bits 0-7, of b1 in bits 8-15): the block scales of nvfp4_block, two at a
 // time on packed f32 pairs, with RN(b/6) by the quotient correction of
@@ -422,6 +444,16 @@ __device__ int block_prefix(int n, int* s_prefix, long long* s_scratch, Count co
     }
     __syncthreads();
     return total <= 0x7FFFFFFFLL ? (int)total : 0;
+}
+
+// floor(a / b) for 0 <= a, 1 <= b: for a < 2^22 a single-precision estimate (exact
+// in binary32: the truncated product of a and the rounded-toward-zero
+// reciprocal of b is floor(a / b) or one less) and one correction step.
+__device__ __forceinline__ int div_nonneg(int a, int b) {
+    if (a >= (1 << 22)) return a / b;
+    int q = __float2int_rz(__fmul_rz((float)a, __frcp_rz((float)b)));
+    if ((q + 1) * b <= a) ++q;
+    return q;
 }
 
 // The expert owning unit u: the largest e with s_prefix[e] <= u (empty

@@ -99,14 +99,20 @@ __device__ __forceinline__ int tile_row(int p, int w, int lane) {
 
 template <int FMT, int LAYOUT>
 __device__ __forceinline__ TileRef tile_ref(const qz_expert* table, const int* s_prefix, int n, int tile, int w,
-                                            int lane) {
+                                            int lane, int hint = -1) {
     using G = TileGeo<FMT>;
-    const int e = find_owner(s_prefix, n, tile);
+    int e = hint;
+    if (e < 0) {
+        e = find_owner(s_prefix, n, tile);
+    } else {
+        while (tile >= s_prefix[e + 1]) ++e;  // hint owns a tile <= this one; s_prefix[n] = total > tile
+    }
     const qz_expert E = load_entry(table, e);
     const int local = tile - s_prefix[e];
     const int nct = (int)((E.cols + kTileCols - 1) / kTileCols);
     TileRef t;
-    t.rt = local / nct;
+    // (the MXFP8 tiles measured faster with the plain division and search)
+    t.rt = FMT == QZ_FMT_NVFP4 ? div_nonneg(local, nct) : local / nct;
     t.ct = local - t.rt * nct;
     const int kb = lane % G::kLpr;
     const int64_t row0 = (int64_t)t.rt * kTileRows + tile_row<FMT>(0, w, lane);
@@ -244,7 +250,7 @@ __global__ void __launch_bounds__(kThreads, 3) grouped_tile_kernel(const qz_expe
     for (;;) {
         const int next = tile + gridDim.x;
         const bool more = next < total;
-        const TileRef nxt = more ? tile_ref<FMT, LAYOUT>(table, s_prefix, n, next, w, lane) : cur;
+        const TileRef nxt = more ? tile_ref<FMT, LAYOUT>(table, s_prefix, n, next, w, lane, FMT == QZ_FMT_NVFP4 ? cur.expert : -1) : cur;
         const float S = kAmax ? nvfp4_encode_scale(*cur.amax) : 0.0f;
         if (FMT == QZ_FMT_MXFP8) {
 #pragma unroll
@@ -253,13 +259,14 @@ __global__ void __launch_bounds__(kThreads, 3) grouped_tile_kernel(const qz_expe
                 if (more) tile_load<FMT>(nxt, p, v[p]);
             }
         } else {
+            const float qm = rcp_lane_quotient(S, s_inv, lane);
 #pragma unroll
             for (int p = 0; p < G::kPasses; p += 2) {
                 const uint32_t sc = tile_scales_nv(v[p], v[p + 1], S);
                 const uint32_t sc0 = sc & 0xFFu, sc1 = sc >> 8;
-                tile_pass_nv<LAYOUT>(cur, p, lane, v[p], sc0, nvfp4_rcp(S, sc0, s_inv), s_sf[w]);
+                tile_pass_nv<LAYOUT>(cur, p, lane, v[p], sc0, nvfp4_rcp_warp(qm, sc0), s_sf[w]);
                 if (more) tile_load<FMT>(nxt, p, v[p]);
-                tile_pass_nv<LAYOUT>(cur, p + 1, lane, v[p + 1], sc1, nvfp4_rcp(S, sc1, s_inv), s_sf[w]);
+                tile_pass_nv<LAYOUT>(cur, p + 1, lane, v[p + 1], sc1, nvfp4_rcp_warp(qm, sc1), s_sf[w]);
                 if (more) tile_load<FMT>(nxt, p + 1, v[p + 1]);
             }
         }
@@ -303,7 +310,7 @@ __global__ void __launch_bounds__(kThreads, 3) amax_grouped_kernel(const qz_expe
     for (;;) {
         const int next = tile + gridDim.x;
         const bool more = next < total;
-        const TileRef nxt = more ? tile_ref<QZ_FMT_NVFP4, LAYOUT>(table, s_prefix, n, next, w, lane) : cur;
+        const TileRef nxt = more ? tile_ref<QZ_FMT_NVFP4, LAYOUT>(table, s_prefix, n, next, w, lane, cur.expert) : cur;
 #pragma unroll
         for (int p = 0; p < G::kPasses; ++p) {
             run = max(run, absmax_words<G::kWords>(v[p]));
@@ -492,13 +499,14 @@ __global__ void __launch_bounds__(kThreads, 3) nvfp4_compute_l2_kernel(const qz_
                 // ordered after thread 0's acquire of the chunk count by the barrier above
                 const float A = __uint_as_float(ld_relaxed_gpu(amax_ws + cur.expert));
                 const float S = nvfp4_encode_scale(A);
+                const float qm = rcp_lane_quotient(S, s_inv, lane);
 #pragma unroll
                 for (int p = 0; p < G::kPasses; p += 2) {
                     const uint32_t sc = tile_scales_nv(v[p], v[p + 1], S);
 #pragma unroll
                     for (int q = 0; q < 2; ++q) {
                         const uint32_t scq = (sc >> (8 * q)) & 0xFFu;
-                        tile_pass_nv<LAYOUT>(cur, p + q, lane, v[p + q], scq, nvfp4_rcp(S, scq, s_inv), s_sf[w]);
+                        tile_pass_nv<LAYOUT>(cur, p + q, lane, v[p + q], scq, nvfp4_rcp_warp(qm, scq), s_sf[w]);
                         if (more) {
                             if (next_a) tile_load<QZ_FMT_NVFP4, kL2Last>(nxt, p + q, v[p + q]);
                             else tile_load<QZ_FMT_NVFP4, kL2First>(nxt, p + q, v[p + q]);
