@@ -66,6 +66,8 @@ def _declare(lib):
         "qzo_quantize_nvfp4": (None, [P, i64, i64, i64, P, P, c.c_int, c.c_int, P]),
         "qzo_residual_rmsnorm": (None, [P, P, P, c.c_float, i64, i64, P, P]),
         "qzo_rmsnorm_quantize": (None, [P, P, P, c.c_float, i64, i64, P, P, c.c_int, P, P, c.c_int, P]),
+        "qzo_dequantize_mxfp8": (None, [P, P, i64, i64, c.c_int, P, i64]),
+        "qzo_dequantize_nvfp4": (None, [P, P, P, c.c_int, i64, i64, c.c_int, P, i64]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -147,6 +149,34 @@ def quantize_nvfp4(x: np.ndarray, layout: int, mode: int, amax_in: float | None 
         lib.qzo_quantize_nvfp4(ctypes.c_void_p(x.__array_interface__["data"][0]), rows, cols, ld,
                                _ptr(q), _ptr(sf), layout, mode, _ptr(amax))
     return q, sf[:n_sf], (amax[:rows] if mode == NVFP4_PER_ROW else amax)
+
+
+def dequantize_mxfp8(q: np.ndarray, sf: np.ndarray, layout: int, lib=None) -> np.ndarray:
+    """bf16 bits [rows, cols] of an MXFP8 payload q [rows, cols] and its SF bytes (R11)."""
+    lib = lib or load()
+    rows, cols = q.shape
+    q = np.ascontiguousarray(q, dtype=np.uint8)
+    sf = np.ascontiguousarray(sf, dtype=np.uint8)
+    y = np.zeros((rows, cols), dtype=np.uint16)
+    if rows > 0:
+        lib.qzo_dequantize_mxfp8(_ptr(q), _ptr(sf), rows, cols, layout, _ptr(y), cols)
+    return y
+
+
+def dequantize_nvfp4(q: np.ndarray, sf: np.ndarray, amax: np.ndarray, per_row: bool, layout: int,
+                     lib=None) -> np.ndarray:
+    """bf16 bits [rows, cols] of a packed NVFP4 payload q [rows, cols/2], its SF
+    bytes and its amax (per tensor [1] or per row [rows]) (R11)."""
+    lib = lib or load()
+    rows, half = q.shape
+    cols = 2 * half
+    q = np.ascontiguousarray(q, dtype=np.uint8)
+    sf = np.ascontiguousarray(sf, dtype=np.uint8)
+    amax = np.ascontiguousarray(amax, dtype=np.float32)
+    y = np.zeros((rows, cols), dtype=np.uint16)
+    if rows > 0:
+        lib.qzo_dequantize_nvfp4(_ptr(q), _ptr(sf), _ptr(amax), 1 if per_row else 0, rows, cols, layout, _ptr(y), cols)
+    return y
 
 
 def swizzle(lin: np.ndarray, rows: int, kv: int, lib=None) -> np.ndarray:

@@ -41,6 +41,8 @@
  *     tiles row-block-major; padding bytes are 0x00.
  *  R7 Signed zero: the sign bit of the scaled element is kept.
  *  R8 RMSNorm over h = bf16(x + r); y = bf16(h * rstd * gamma).
+ *  R11 Dequantization: the exact product of code value, block scale value
+ *     (and the NVFP4 decode scale g), rounded once to bf16.
  */
 #include <math.h>
 #include <stdint.h>
@@ -410,4 +412,46 @@ void qzo_rmsnorm_quantize(const uint16_t *x, const uint16_t *res, const uint16_t
     qzo_residual_rmsnorm(x, res, gamma, eps, T, H, y, h);
     if (fmt == 0) qzo_quantize_mxfp8(y, T, H, H, q, sf, layout);
     else qzo_quantize_nvfp4(y, T, H, H, q, sf, layout, 0, amax);
+}
+
+/* ------------------------------------------------------------------------- */
+/* Dequantization: the decoded tensor of a quantized one ([SPL] Changes: the  */
+/* regression tests compare dequantized values; [CAR] commit 1: the dequant   */
+/* reference path works on the high-precision tensor).                        */
+/*   R11 an element's decoded value is the exact product of its code's value  */
+/*       and its block scale's value (and, for NVFP4, of the FP32 decode      */
+/*       scale g = RN32(A / 2688) of R2), rounded once to bf16 (RNE); the     */
+/*       product has at most 4 + 8 (MXFP8) or 2 + 4 + 24 (NVFP4) significant  */
+/*       bits, so binary64 holds it exactly.                                  */
+/*   y   : bf16 [rows, cols], row stride ldy                                  */
+/* ------------------------------------------------------------------------- */
+
+void qzo_dequantize_mxfp8(const uint8_t *q, const uint8_t *sf, int64_t rows, int64_t cols,
+                          int layout, uint16_t *y, int64_t ldy)
+{
+    int64_t kv = cols / 32;
+    for (int64_t r = 0; r < rows; r++)
+        for (int64_t c = 0; c < cols; c++) {
+            int byte = sf[sf_offset(layout, r, c / 32, kv)];
+            double v = qzo_e4m3_value(q[r * cols + c]) * ldexp(1.0, byte - 127);
+            y[r * ldy + c] = qzo_bf16_from_double(v);
+        }
+}
+
+/* amax: per-tensor amax[0] (per_row == 0) or per-row amax[r] (per_row != 0). */
+void qzo_dequantize_nvfp4(const uint8_t *q, const uint8_t *sf, const float *amax, int per_row,
+                          int64_t rows, int64_t cols, int layout, uint16_t *y, int64_t ldy)
+{
+    int64_t kv = cols / 16;
+    for (int64_t r = 0; r < rows; r++) {
+        float A = per_row ? amax[r] : amax[0];
+        float g = A / 2688.0f;                         /* R2: binary32 decode scale */
+        for (int64_t c = 0; c < cols; c++) {
+            uint8_t byte = q[r * (cols / 2) + c / 2];
+            uint8_t code = (c & 1) ? (uint8_t)(byte >> 4) : (uint8_t)(byte & 0xF);   /* R5 */
+            uint8_t s = sf[sf_offset(layout, r, c / 16, kv)];
+            double v = qzo_e2m1_value(code) * qzo_e4m3_value(s) * (double)g;
+            y[r * ldy + c] = qzo_bf16_from_double(v);
+        }
+    }
 }

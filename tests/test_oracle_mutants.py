@@ -19,7 +19,7 @@ import oracle
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 PIN_FILES = ["tests/test_oracle_formats.py", "tests/test_oracle_mxfp8.py", "tests/test_oracle_layout.py",
-             "tests/test_oracle_nvfp4.py", "tests/test_oracle_norm.py"]
+             "tests/test_oracle_nvfp4.py", "tests/test_oracle_norm.py", "tests/test_oracle_dequant.py"]
 
 MUTANTS = {
     "ties_away_from_even": ("return (fmod(f, 2.0) == 0.0) ? f : f + 1.0;", "return f + 1.0;"),
@@ -45,6 +45,15 @@ MUTANTS = {
     "rms_gamma_row_index": ("gamma[i]);", "gamma[t]);"),
     "rms_square_unrounded_sum": ("ss += hv * hv;", "ss += s * s;"),
     "mx_row_stride_ignored": ("const uint16_t *blk = x + r * ld + k * 32;", "const uint16_t *blk = x + r * cols + k * 32;"),
+    "dq_nibbles_swapped": ("uint8_t code = (c & 1) ? (uint8_t)(byte >> 4) : (uint8_t)(byte & 0xF);",
+                           "uint8_t code = (c & 1) ? (uint8_t)(byte & 0xF) : (uint8_t)(byte >> 4);"),
+    "dq_no_decode_scale": ("double v = qzo_e2m1_value(code) * qzo_e4m3_value(s) * (double)g;",
+                           "double v = qzo_e2m1_value(code) * qzo_e4m3_value(s);"),
+    "dq_binary32_product": ("double v = qzo_e2m1_value(code) * qzo_e4m3_value(s) * (double)g;",
+                            "double v = (double)(float)(qzo_e2m1_value(code) * qzo_e4m3_value(s) * (double)g);"),
+    "dq_mx_exponent_off_by_one": ("double v = qzo_e4m3_value(q[r * cols + c]) * ldexp(1.0, byte - 127);",
+                                  "double v = qzo_e4m3_value(q[r * cols + c]) * ldexp(1.0, byte - 126);"),
+    "dq_mx_linear_sf_index": ("int byte = sf[sf_offset(layout, r, c / 32, kv)];", "int byte = sf[r * kv + c / 32];"),
     "bf16_double_rounding": ("double n = round_half_even(a / step);\n    double r = n * step;",
                              "double n = round_half_even((double)(float)a / step);\n    double r = n * step;"),
 }
