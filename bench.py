@@ -70,6 +70,7 @@ KERNEL_SOURCES = {
     "nvfp4_compute_l2_kernel": ("qz_grouped.cu", "qz_device.cuh"),
     "nvfp4_rows_kernel": ("qz_rows.cu", "qz_device.cuh"),
     "rmsnorm_quant_kernel": ("qz_rmsnorm.cu", "qz_device.cuh"),
+    "dequant_kernel": ("qz_dequant.cu", "qz_device.cuh"),
 }
 
 
@@ -429,7 +430,7 @@ class L2Flush:
         self.buf.zero_()
 
 
-def extra_workloads(qz, device, stream, peak, which=("split", "fused", "nvfp4", "large"), tokens=None):
+def extra_workloads(qz, device, stream, peak, which=("split", "fused", "nvfp4", "large", "dequant"), tokens=None):
     out = []
     flush = L2Flush(device)
 
@@ -448,6 +449,8 @@ def extra_workloads(qz, device, stream, peak, which=("split", "fused", "nvfp4", 
         _extra_nvfp4_30b(qz, device, rec)
     if "large" in which:
         _extra_large(qz, device, rec)
+    if "dequant" in which:
+        _extra_dequant(qz, device, rec)
     return out
 
 
@@ -564,6 +567,33 @@ def _extra_large(qz, device, rec):
         torch.cuda.empty_cache()
 
 
+def _extra_dequant(qz, device, rec):
+    """Decode a Qwen3-30B-A3B gate_up projection (128 experts of [1536, 2048])
+    back to bf16 from MXFP8 and from NVFP4 (per-tensor scale), in one call."""
+    cfg = synth.QWEN3_30B
+    rows, cols = cfg["gate_up"]
+    stack = synth.expert_stack(cfg["experts"], (rows, cols), cfg["std"], seed=cfg["seed"], device=device)
+    for fmt, fname in ((qz.FMT_MXFP8, "MXFP8"), (qz.FMT_NVFP4, "NVFP4 (per-tensor amax)")):
+        mode = qz.NVFP4_PER_TENSOR_COMPUTE if fmt == qz.FMT_NVFP4 else qz.NVFP4_PER_ROW
+        ents = qz.alloc_outputs(list(stack.unbind(0)), fmt, qz.SF_SWIZZLED, mode)
+        tab = qz.ExpertTable(ents)
+        if fmt == qz.FMT_MXFP8:
+            qz.quantize_grouped_mxfp8(tab, qz.SF_SWIZZLED)
+        else:
+            qz.quantize_grouped_nvfp4(tab, mode, qz.SF_SWIZZLED)
+        ys = torch.empty_like(stack)
+        dtab = qz.DqTable([qz.DqEntry(e.q, e.sf, y, e.amax) for e, y in zip(ents, ys.unbind(0))])
+        ms = _time_graph(lambda f=fmt, t=dtab: qz.dequantize_grouped(t, f, False, qz.SF_SWIZZLED), reps=5)
+        nsf = qz.sf_bytes(rows, cols, fmt, qz.SF_SWIZZLED)
+        qb = rows * cols if fmt == qz.FMT_MXFP8 else rows * cols // 2
+        nbytes = cfg["experts"] * (qb + nsf + (4 if fmt == qz.FMT_NVFP4 else 0) + rows * cols * 2)
+        rec(f"dequantize Qwen3-30B-A3B gate_up [1536, 2048] x128 experts from {fname} to bf16, swizzled, one call",
+            nbytes, ms, 1, kernel="dequant_kernel")
+        del ents, tab, dtab, ys
+    del stack
+    torch.cuda.empty_cache()
+
+
 # ---------------------------------------------------------------------------
 # CPU oracle timing (the reference arm and the cpu_baseline key)
 # ---------------------------------------------------------------------------
@@ -632,7 +662,7 @@ def main():
     ap.add_argument("--no-extra", action="store_true", help="skip the other workloads")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
-    ap.add_argument("--only", choices=["split", "fused", "nvfp4", "large"], default=None,
+    ap.add_argument("--only", choices=["split", "fused", "nvfp4", "large", "dequant"], default=None,
                     help="time only this secondary workload and print its record (profiling aid)")
     ap.add_argument("--tokens", type=str, default=None,
                     help="comma-separated token counts for the fused sweep (default: 1..4096)")

@@ -129,6 +129,19 @@ typedef struct qz_sf_pair {
     int64_t kv;         /* scale columns, >= 1 */
 } qz_sf_pair;
 
+/* One expert's quantized tensor to decode (lives in DEVICE memory, 56 bytes). */
+typedef struct qz_dq_expert {
+    const void *q;      /* MXFP8: e4m3 [rows, cols], 16-byte aligned; NVFP4: packed e2m1
+                           [rows, cols/2] (low nibble first), 8-byte aligned; dense rows */
+    const uint8_t *sf;  /* this expert's SF region in the layout given to the call */
+    const float *amax;  /* NVFP4: amax[0] (per tensor) or amax[rows] (per row), 4-byte
+                           aligned; MXFP8: unused (may be NULL) */
+    int64_t rows;       /* >= 0 (0: empty, nothing is written) */
+    int64_t cols;       /* multiple of 32 (MXFP8) / 16 (NVFP4) */
+    void *y;            /* bf16 output [rows, cols], 16-byte aligned, row stride ldy */
+    int64_t ldy;        /* >= cols, multiple of 8, <= QZ_MAX_LD */
+} qz_dq_expert;
+
 /* Optional launch controls; pass NULL for the defaults. */
 typedef struct qz_launch_opts {
     unsigned int *d_err;    /* device word; kernels OR QZ_DERR_* bits into it (never clear it) */
@@ -210,6 +223,23 @@ qz_status qz_rmsnorm_quantize(const void *d_x, const void *d_residual, const voi
  * with n > 0; entries with rows < 0, kv < 1, null pointers or a misaligned
  * dst are skipped and reported through opts->d_err. */
 qz_status qz_swizzle_scales(const qz_sf_pair *d_table, int n, void *stream, const qz_launch_opts *opts);
+
+/* Decode grouped MXFP8 / NVFP4 tensors back to bf16: the inverse map of the
+ * quantizers, for reference paths and error checks (TransformerEngine PR #3800,
+ * Changes: regression tests on dequantized values; TensorRT-LLM "MXFP8 carrier
+ * and quantize folds", commit 1: the dequant reference path).  Element i of
+ * block k decodes to
+ *   MXFP8: value(q_i) * 2^(sf_k - 127)
+ *   NVFP4: value(q_i) * value(sf_k) * g,  g = RN32(A / 2688)
+ * (A = amax[0], or amax[row] when per_row != 0) computed exactly and rounded
+ * once to bf16, to nearest with ties to even.  fmt is QZ_FMT_MXFP8 or
+ * QZ_FMT_NVFP4, layout the SF layout of every entry.  One persistent launch,
+ * asynchronous on the stream, no allocation.
+ * Errors: QZ_ERR_INVALID_ARG for n < 0, n > QZ_MAX_EXPERTS, a NULL table with
+ * n > 0, an unknown fmt or layout; invalid entries are skipped and reported
+ * through opts->d_err (QZ_DERR_SHAPE / NULL / ALIGN with the alignments above). */
+qz_status qz_dequantize_grouped(const qz_dq_expert *d_table, int n_experts, int fmt, int per_row, int layout,
+                                void *stream, const qz_launch_opts *opts);
 
 /* Largest table of qz_quantize_grouped_nvfp4_compute_noalloc. */
 #define QZ_STATIC_WS_MAX_EXPERTS 1024

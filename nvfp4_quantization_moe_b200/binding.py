@@ -39,6 +39,7 @@ EXPORTED = (
     "qz_version",
     "qz_workspace_bytes",
     "qz_quantize_grouped_nvfp4_compute_noalloc",
+    "qz_dequantize_grouped",
 )
 STATIC_WS_MAX_EXPERTS = 1024
 
@@ -55,6 +56,12 @@ class _Expert(ctypes.Structure):
                 ("amax", ctypes.c_void_p)]
 
 
+class _DqExpert(ctypes.Structure):
+    _fields_ = [("q", ctypes.c_void_p), ("sf", ctypes.c_void_p), ("amax", ctypes.c_void_p),
+                ("rows", ctypes.c_int64), ("cols", ctypes.c_int64), ("y", ctypes.c_void_p),
+                ("ldy", ctypes.c_int64)]
+
+
 class _SfPair(ctypes.Structure):
     _fields_ = [("src", ctypes.c_void_p), ("dst", ctypes.c_void_p), ("rows", ctypes.c_int64),
                 ("kv", ctypes.c_int64)]
@@ -65,7 +72,7 @@ class _Opts(ctypes.Structure):
                 ("workspace_bytes", ctypes.c_size_t)]
 
 
-assert ctypes.sizeof(_Expert) == 56 and ctypes.sizeof(_SfPair) == 32
+assert ctypes.sizeof(_Expert) == 56 and ctypes.sizeof(_SfPair) == 32 and ctypes.sizeof(_DqExpert) == 56
 
 _lock = threading.Lock()
 _lib = None
@@ -100,6 +107,8 @@ def load(path: str = LIB_PATH):
         lib.qz_workspace_bytes.argtypes = [I]
         lib.qz_quantize_grouped_nvfp4_compute_noalloc.restype = I
         lib.qz_quantize_grouped_nvfp4_compute_noalloc.argtypes = [P, I, I, P, P]
+        lib.qz_dequantize_grouped.restype = I
+        lib.qz_dequantize_grouped.argtypes = [P, I, I, I, I, P, P]
         _lib = lib
         return lib
 
@@ -200,6 +209,53 @@ class ExpertTable:
         return self
 
 
+@dataclass
+class DqEntry:
+    """One quantized expert to decode: payload q ([rows, cols] e4m3 or
+    [rows, cols/2] packed e2m1), its SF region, its amax (NVFP4) and the bf16
+    output y [rows, cols] (row stride may exceed cols)."""
+    q: torch.Tensor
+    sf: torch.Tensor
+    y: torch.Tensor
+    amax: Optional[torch.Tensor] = None
+
+
+class DqTable:
+    """A device-resident array of qz_dq_expert entries (keeps its tensors alive)."""
+
+    def __init__(self, entries: Sequence[DqEntry], device=None):
+        self.entries = list(entries)
+        n = len(self.entries)
+        arr = (_DqExpert * max(n, 1))()
+        for i, e in enumerate(self.entries):
+            y = e.y
+            assert y.dtype == torch.bfloat16 and y.dim() == 2
+            rows, cols = y.shape
+            ldy = y.stride(0) if rows > 1 else max(cols, y.stride(0))
+            assert rows == 0 or y.stride(1) == 1, "rows must be contiguous"
+            arr[i] = _DqExpert(_ptr(e.q) if rows else 0, _ptr(e.sf) if rows else 0, _ptr(e.amax), rows, cols,
+                               y.data_ptr() if rows else 0, ldy)
+        host = torch.frombuffer(bytearray(bytes(arr)), dtype=torch.uint8)
+        dev = device if device is not None else (self.entries[0].y.device if n else torch.device("cuda"))
+        self.dev = host.to(dev)
+        self.n = n
+
+    @property
+    def ptr(self) -> int:
+        return int(self.dev.data_ptr()) if self.n else 0
+
+    @classmethod
+    def from_raw(cls, raw: Iterable[tuple], device) -> "DqTable":
+        """Entries from raw (q_ptr, sf_ptr, amax_ptr, rows, cols, y_ptr, ldy) tuples."""
+        self = cls.__new__(cls)
+        raw = list(raw)
+        arr = (_DqExpert * max(len(raw), 1))(*[_DqExpert(*r) for r in raw])
+        self.entries = []
+        self.n = len(raw)
+        self.dev = torch.frombuffer(bytearray(bytes(arr)), dtype=torch.uint8).to(device)
+        return self
+
+
 class SfPairTable:
     def __init__(self, pairs: Sequence[tuple], device):
         """pairs: (src linear uint8 tensor, dst swizzled uint8 tensor, rows, kv)."""
@@ -245,6 +301,13 @@ def rmsnorm_quantize(x, residual, gamma, eps: float, norm_out, residual_out, fmt
                                       int(fmt), ctypes.c_void_p(_ptr(q)), ctypes.c_void_p(_ptr(sf)), int(layout),
                                       ctypes.c_void_p(_ptr(global_amax)), _stream_ptr(stream)),
            "qz_rmsnorm_quantize")
+
+
+def dequantize_grouped(table: DqTable, fmt: int, per_row: bool, layout: int, stream=None, err=None,
+                       max_ctas: int = 0):
+    _check(load().qz_dequantize_grouped(ctypes.c_void_p(table.ptr), table.n, int(fmt), 1 if per_row else 0,
+                                        int(layout), _stream_ptr(stream), _opts(err, max_ctas)),
+           "qz_dequantize_grouped")
 
 
 def swizzle_scales(table: SfPairTable, stream=None, err=None, max_ctas: int = 0):

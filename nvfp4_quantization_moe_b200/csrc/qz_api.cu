@@ -26,16 +26,19 @@ cudaError_t launch_nvfp4_compute_l2(const qz_expert* table, int n, int layout, i
 cudaError_t launch_nvfp4_compute_l2_static(const qz_expert* table, int n, int layout, int grid, cudaStream_t s,
                                            unsigned* d_err);
 int rows_blocks_per_sm(int n);
+cudaError_t launch_dequant(const qz_dq_expert* table, int n, int fmt, bool per_row, int layout, int grid,
+                           cudaStream_t s, unsigned* d_err);
+int dequant_blocks_per_sm(int n);
 }  // namespace qz
 
 namespace {
 
 constexpr int kMaxDevices = 64;
-constexpr int kKinds = 6;  // mxfp8, nvfp4 tile, swizzle, amax, rows, computed-amax L2 path
+constexpr int kKinds = 7;  // mxfp8, nvfp4 tile, swizzle, amax, rows, computed-amax L2 path, dequantize
 
 struct DeviceLimits {
     int sms = 0;
-    int per_sm[kKinds] = {0, 0, 0, 0, 0, 0};
+    int per_sm[kKinds] = {0, 0, 0, 0, 0, 0, 0};
 };
 
 std::mutex g_mu;
@@ -57,8 +60,9 @@ int wave_grid(int kind, const qz_launch_opts* opts) {
             d.sms = sms > 0 ? sms : 1;
         }
         if (d.per_sm[kind] == 0)
-            d.per_sm[kind] = (kind == 4) ? qz::rows_blocks_per_sm(QZ_MAX_EXPERTS)
-                                         : qz::grouped_blocks_per_sm(kind, QZ_MAX_EXPERTS);
+            d.per_sm[kind] = (kind == 4)   ? qz::rows_blocks_per_sm(QZ_MAX_EXPERTS)
+                             : (kind == 6) ? qz::dequant_blocks_per_sm(QZ_MAX_EXPERTS)
+                                           : qz::grouped_blocks_per_sm(kind, QZ_MAX_EXPERTS);
         grid = d.sms * d.per_sm[kind];
     }
     if (opts && opts->max_ctas > 0 && opts->max_ctas < grid) grid = opts->max_ctas;
@@ -179,6 +183,17 @@ qz_status qz_quantize_grouped_nvfp4_compute_noalloc(const qz_expert* d_table, in
     if (n_experts == 0) return QZ_OK;
     return from_cuda(qz::launch_nvfp4_compute_l2_static(d_table, n_experts, layout, wave_grid(5, opts),
                                                         (cudaStream_t)stream, err_word(opts)));
+}
+
+qz_status qz_dequantize_grouped(const qz_dq_expert* d_table, int n_experts, int fmt, int per_row, int layout,
+                                void* stream, const qz_launch_opts* opts) {
+    qz_status st = check_table(d_table, n_experts);
+    if (st != QZ_OK) return st;
+    if (!valid_layout(layout)) return QZ_ERR_INVALID_ARG;
+    if (fmt != QZ_FMT_MXFP8 && fmt != QZ_FMT_NVFP4) return QZ_ERR_INVALID_ARG;
+    if (n_experts == 0) return QZ_OK;
+    return from_cuda(qz::launch_dequant(d_table, n_experts, fmt, per_row != 0, layout, wave_grid(6, opts),
+                                        (cudaStream_t)stream, err_word(opts)));
 }
 
 size_t qz_workspace_bytes(int n_experts) {

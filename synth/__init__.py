@@ -130,3 +130,27 @@ def blockwise_scaled(shape, block: int, seed: int = 0, lo: float = -40.0, hi: fl
 def bf16_bits(t: torch.Tensor) -> np.ndarray:
     """A CPU bf16 tensor as a numpy uint16 array (bit pattern, no copy of values)."""
     return t.contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def random_payload(rows: int, cols: int, fmt: int, seed: int = 0) -> np.ndarray:
+    """Random quantized payload bytes: e4m3 codes [rows, cols] without the two
+    NaN codes (fmt 0) or packed e2m1 pairs [rows, cols/2] (fmt 1)."""
+    rng = np.random.default_rng(seed)
+    if fmt == 0:
+        q = rng.integers(0, 256, size=(rows, cols), dtype=np.uint8)
+        q[(q & 0x7F) == 0x7F] = 0x00
+        return q
+    return rng.integers(0, 256, size=(rows, cols // 2), dtype=np.uint8)
+
+
+def random_scale_bytes(n: int, fmt: int, seed: int = 0) -> np.ndarray:
+    """Random scale bytes: E8M0 0..254 (fmt 0) or finite non-negative e4m3
+    codes 0..126 (fmt 1)."""
+    rng = np.random.default_rng(seed)
+    return rng.integers(0, 255 if fmt == 0 else 127, size=n, dtype=np.uint8)
+
+
+def random_amax(n: int, seed: int = 0, lo: float = -20.0, hi: float = 20.0) -> np.ndarray:
+    """Random positive binary32 amax values spread over 2^lo .. 2^hi."""
+    rng = np.random.default_rng(seed)
+    return (np.exp2(rng.uniform(lo, hi, size=n)) * rng.uniform(1.0, 2.0, size=n)).astype(np.float32)

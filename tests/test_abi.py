@@ -76,6 +76,11 @@ def test_host_errors_without_gpu(lib):
     assert qz.workspace_bytes(0) == 0 and qz.workspace_bytes(qz.MAX_EXPERTS + 1) == 0
     assert qz.workspace_bytes(128) >= 4 * (128 + 1)
     assert lib.qz_swizzle_scales(None, 0, None, None) == qz.QZ_OK
+    assert lib.qz_dequantize_grouped(None, -1, 0, 0, 0, None, None) == qz.QZ_ERR_INVALID_ARG
+    assert lib.qz_dequantize_grouped(None, 2, 0, 0, 0, None, None) == qz.QZ_ERR_INVALID_ARG
+    assert lib.qz_dequantize_grouped(P(0x1000), 2, 5, 0, 0, None, None) == qz.QZ_ERR_INVALID_ARG   # format
+    assert lib.qz_dequantize_grouped(P(0x1000), 2, 1, 0, 3, None, None) == qz.QZ_ERR_INVALID_ARG   # layout
+    assert lib.qz_dequantize_grouped(None, 0, 1, 1, 1, None, None) == qz.QZ_OK
     a = P(0x10000)
 
     def norm(T=4, H=7168, fmt=0, layout=1, x=a, r=a, g=a, y=a, h=None, q=a, sf=a, amax=None):
