@@ -10,9 +10,10 @@
 //
 // One persistent launch walks all experts' 128 x 128 tiles like the quantize
 // kernels: lane l of warp w owns one scale block per pass (MXFP8: 32
-// elements, NVFP4: 16) of rows w + 8 * (lane / LPR) + 32 p of the tile.  All
-// of a tile's payload loads are issued before any decoding; the bf16 output
-// leaves as 16-byte stores.
+// elements, NVFP4: 16) of rows w + 8 * (lane / LPR) + 64 p (MXFP8) or
+// + 32 p (NVFP4) of the tile.  The next tile's payload and scale loads are
+// issued before the current tile is decoded; the bf16 output leaves as
+// 32-byte stores (16-byte ones when the rows are only 16-byte aligned).
 #include <cuda_fp16.h>
 
 #include "qz_device.cuh"
@@ -73,6 +74,12 @@ struct DqTiles {
     }
 };
 
+__device__ __forceinline__ uint32_t __hmul2_rn_bits(uint32_t a, uint32_t b) {
+    uint32_t r;
+    asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+
 // bf16 bits of the exact value hi + lo (hi = RN32 of it, lo the exact
 // remainder), rounded to nearest even: rounding hi again is right unless hi
 // lies exactly halfway between two bf16 numbers, where lo decides.
@@ -85,22 +92,159 @@ __device__ __forceinline__ uint32_t bf16_of_exact(float hi, float lo) {
     return (u + 0x7FFFu + ((u >> 16) & 1u)) >> 16;
 }
 
-// Two e4m3 codes (low byte first) as two binary32 values, exactly.
-__device__ __forceinline__ float2 e4m3x2_to_f32x2(uint32_t pair) {
+// Two e4m3 codes (bits 0-15, low byte first) as an f16x2 pair, exactly.
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t pair) {
     uint32_t h;
     asm("{\n\t.reg .b16 c;\n\tcvt.u16.u32 c, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, c;\n\t}" : "=r"(h) : "r"(pair));
-    return __half22float2(*reinterpret_cast<const __half2*>(&h));
+    return h;
 }
 
-// Two e2m1 codes (low nibble first) as two binary32 values, exactly.
-__device__ __forceinline__ float2 e2m1x2_to_f32x2(uint32_t pair) {
+// Two e2m1 codes (bits 0-7, low nibble first) as an f16x2 pair, exactly.
+__device__ __forceinline__ uint32_t e2m1x2_to_f16x2(uint32_t pair) {
     uint32_t h;
     asm("{\n\t.reg .b8 c;\n\tcvt.u8.u32 c, %1;\n\tcvt.rn.f16x2.e2m1x2 %0, c;\n\t}" : "=r"(h) : "r"(pair));
-    return __half22float2(*reinterpret_cast<const __half2*>(&h));
+    return h;
 }
+
+// f16x2 pair times s in binary32 (exact for the products formed here): the
+// two binary32 results, low element first.
+__device__ __forceinline__ float2 f16x2_times(uint32_t h, float s) {
+    const float2 v = __half22float2(*reinterpret_cast<const __half2*>(&h));
+    float2 r;
+    asm("{\n\t.reg .b64 a, b;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %4};\n\t"
+        "mul.rn.f32x2 a, a, b;\n\tmov.b64 {%0, %1}, a;\n\t}"
+        : "=f"(r.x), "=f"(r.y)
+        : "f"(v.x), "f"(v.y), "f"(s));
+    return r;
+}
+
+// bf16x2 of two binary32 values (round to nearest even), low element first.
+__device__ __forceinline__ uint32_t bf16x2_rn(float lo, float hi) {
+    uint32_t r;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// Whether binary32 x lies exactly halfway between two bf16 numbers.
+__device__ __forceinline__ bool bf16_midpoint(float x) { return (__float_as_uint(x) & 0xFFFFu) == 0x8000u; }
 
 __device__ __forceinline__ int64_t dq_sf_index(int layout, int64_t row, int64_t k, int64_t kv) {
     return layout == QZ_SF_SWIZZLED_128x4 ? swz_offset(row, k, kv) : row * kv + k;
+}
+
+// One thread's view of one tile: its rows' payload words and scale bytes.
+template <int FMT>
+struct DqTile {
+    uint32_t qw[DqGeo<FMT>::kPasses][DqGeo<FMT>::kQWords];
+    uint32_t sc[DqGeo<FMT>::kPasses];
+};
+
+struct DqRef {
+    const uint8_t* q;   // payload byte of (row of pass 0, the lane's block)
+    uint16_t* y;        // output element of the same
+    const float* amax;  // amax[0], or the row amax of pass 0 (per row)
+    const uint8_t* sf;
+    int64_t row0, kv, k, qld, ldy, rows;
+    bool col_ok;
+    bool y32;           // output rows 32-byte aligned: 32-byte stores
+    int expert;
+};
+
+template <int FMT>
+__device__ __forceinline__ DqRef dq_ref(const qz_dq_expert* table, const int* s_prefix, int tile, int e, int w,
+                                        int lane, bool per_row) {
+    using G = DqGeo<FMT>;
+    while (tile >= s_prefix[e + 1]) ++e;  // tiles increase; s_prefix[n] == total > tile
+    const qz_dq_expert E = load_dq_entry(table, e);
+    const int local = tile - s_prefix[e];
+    const int nct = (int)((E.cols + kTileCols - 1) / kTileCols);
+    const int rt = local / nct, ct = local - rt * nct;
+    DqRef r;
+    r.expert = e;
+    r.kv = E.cols / G::kBlock;
+    r.k = (int64_t)ct * (kTileCols / G::kBlock) + lane % G::kLpr;
+    r.col_ok = r.k < r.kv;
+    r.qld = FMT == QZ_FMT_MXFP8 ? E.cols : E.cols >> 1;
+    r.ldy = E.ldy;
+    r.rows = E.rows;
+    r.row0 = (int64_t)rt * kTileRows + w + 8 * (lane / G::kLpr);
+    r.q = static_cast<const uint8_t*>(E.q) + r.row0 * r.qld + r.k * G::kQBytes;
+    r.y = static_cast<uint16_t*>(E.y) + r.row0 * E.ldy + r.k * G::kBlock;
+    r.amax = per_row ? E.amax + r.row0 : E.amax;
+    r.sf = E.sf;
+    r.y32 = ((reinterpret_cast<uintptr_t>(E.y) & 31) == 0) && ((E.ldy & 15) == 0);
+    return r;
+}
+
+template <int FMT>
+__device__ __forceinline__ bool dq_live(const DqRef& r, int p) {
+    return r.col_ok && r.row0 + p * DqGeo<FMT>::kRpp < r.rows;
+}
+
+template <int FMT, int LAYOUT>
+__device__ __forceinline__ void dq_load(const DqRef& r, DqTile<FMT>& t) {
+    using G = DqGeo<FMT>;
+#pragma unroll
+    for (int p = 0; p < G::kPasses; ++p) {
+        if (!dq_live<FMT>(r, p)) continue;
+        const uint8_t* src = r.q + (int64_t)p * G::kRpp * r.qld;
+        if (FMT == QZ_FMT_MXFP8) {
+            const uint4 a = ld_stream(src), b = ld_stream(src + 16);
+            t.qw[p][0] = a.x; t.qw[p][1] = a.y; t.qw[p][2] = a.z; t.qw[p][3] = a.w;
+            t.qw[p][4] = b.x; t.qw[p][5] = b.y; t.qw[p][6] = b.z; t.qw[p][7] = b.w;
+        } else {
+            const uint2 a = __ldg(reinterpret_cast<const uint2*>(src));
+            t.qw[p][0] = a.x;
+            t.qw[p][1] = a.y;
+        }
+        t.sc[p] = __ldg(r.sf + dq_sf_index(LAYOUT, r.row0 + p * G::kRpp, r.k, r.kv));
+    }
+}
+
+// MXFP8: 8 elements (two payload words) of one block, scale s = 2^(byte-127).
+__device__ __forceinline__ uint4 dq_mx8(uint32_t w0, uint32_t w1, float s) {
+    // exact products (at least 2^-136, above the binary32 subnormal step), so
+    // a single rounding to bf16 is the rounding of the exact value
+    uint4 o;
+    float2 v;
+    v = f16x2_times(e4m3x2_to_f16x2(w0 & 0xFFFFu), s); o.x = bf16x2_rn(v.x, v.y);
+    v = f16x2_times(e4m3x2_to_f16x2(w0 >> 16), s);     o.y = bf16x2_rn(v.x, v.y);
+    v = f16x2_times(e4m3x2_to_f16x2(w1 & 0xFFFFu), s); o.z = bf16x2_rn(v.x, v.y);
+    v = f16x2_times(e4m3x2_to_f16x2(w1 >> 16), s);     o.w = bf16x2_rn(v.x, v.y);
+    return o;
+}
+
+// NVFP4: 8 elements (one payload word) of one block: sv2 = value(s) as f16x2
+// (both halves), g the decode scale.  code value * value(s) is exact in f16
+// (at most 6 significant bits, at most 2688); RN32 of its product with g is
+// rounded to bf16, and the rare element whose RN32 product lies exactly
+// halfway between two bf16 numbers is rounded from the exact product.
+__device__ __forceinline__ uint4 dq_nv8(uint32_t word, uint32_t sv2, float g) {
+    uint4 o;
+    uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
+    bool tie = false;
+    float hv[8], pv[8];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const uint32_t ph = __hmul2_rn_bits(e2m1x2_to_f16x2((word >> (8 * j)) & 0xFFu), sv2);
+        const float2 p = __half22float2(*reinterpret_cast<const __half2*>(&ph));
+        const float2 h = f16x2_times(ph, g);
+        pv[2 * j] = p.x;
+        pv[2 * j + 1] = p.y;
+        hv[2 * j] = h.x;
+        hv[2 * j + 1] = h.y;
+        ow[j] = bf16x2_rn(h.x, h.y);
+        tie |= bf16_midpoint(h.x) | bf16_midpoint(h.y);
+    }
+    if (tie) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const float l0 = __fmaf_rn(pv[2 * j], g, -hv[2 * j]);
+            const float l1 = __fmaf_rn(pv[2 * j + 1], g, -hv[2 * j + 1]);
+            ow[j] = bf16_of_exact(hv[2 * j], l0) | (bf16_of_exact(hv[2 * j + 1], l1) << 16);
+        }
+    }
+    return o;
 }
 
 template <int FMT, int LAYOUT>
@@ -111,84 +255,55 @@ __global__ void __launch_bounds__(kDqThreads, 3) dequant_kernel(const qz_dq_expe
     __shared__ long long s_scan[33];
     const int total = block_prefix(n, s_prefix, s_scan, DqTiles<FMT, LAYOUT>{table, per_row, d_err}, d_err);
     const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int kb = lane % G::kLpr;
-    int e = 0;
-    for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
-        while (tile >= s_prefix[e + 1]) ++e;  // tiles increase; s_prefix[n] == total > tile
-        const qz_dq_expert E = load_dq_entry(table, e);
-        const int local = tile - s_prefix[e];
-        const int nct = (int)((E.cols + kTileCols - 1) / kTileCols);
-        const int rt = local / nct, ct = local - rt * nct;
-        const int64_t kv = E.cols / G::kBlock;
-        const int64_t k = (int64_t)ct * (kTileCols / G::kBlock) + kb;  // the lane's scale column
-        const bool col_ok = k < kv;
-        const int64_t qld = FMT == QZ_FMT_MXFP8 ? E.cols : E.cols >> 1;
-        // every pass's payload words and scale byte first
-        uint32_t qw[G::kPasses][G::kQWords];
-        uint32_t sc[G::kPasses];
-        int64_t rowp[G::kPasses];
-        bool live[G::kPasses];
+    int tile = blockIdx.x;
+    if (tile >= total) return;
+    DqRef cur = dq_ref<FMT>(table, s_prefix, tile, 0, w, lane, per_row);
+    DqTile<FMT> v;
+    dq_load<FMT, LAYOUT>(cur, v);
+    for (;;) {
+        const int next = tile + gridDim.x;
+        const bool more = next < total;
+        const DqRef nxt = more ? dq_ref<FMT>(table, s_prefix, next, cur.expert, w, lane, per_row) : cur;
+        const DqTile<FMT> t = v;
+        if (more) dq_load<FMT, LAYOUT>(nxt, v);  // the next tile's loads fly while this one decodes
+        float g = 0.0f;
+        if (FMT == QZ_FMT_NVFP4 && !per_row) g = __fdiv_rn(__ldg(cur.amax), 2688.0f);  // the FP32 decode scale
 #pragma unroll
         for (int p = 0; p < G::kPasses; ++p) {
-            const int64_t row = (int64_t)rt * kTileRows + p * G::kRpp + w + 8 * (lane / G::kLpr);
-            rowp[p] = row;
-            live[p] = col_ok && row < E.rows;
-            if (live[p]) {
-                const uint8_t* src = static_cast<const uint8_t*>(E.q) + row * qld + k * G::kQBytes;
-                if (FMT == QZ_FMT_MXFP8) {
-                    const uint4 a = ld_stream(src), b = ld_stream(src + 16);
-                    qw[p][0] = a.x; qw[p][1] = a.y; qw[p][2] = a.z; qw[p][3] = a.w;
-                    qw[p][4] = b.x; qw[p][5] = b.y; qw[p][6] = b.z; qw[p][7] = b.w;
-                } else {
-                    const uint2 a = __ldg(reinterpret_cast<const uint2*>(src));
-                    qw[p][0] = a.x;
-                    qw[p][1] = a.y;
-                }
-                sc[p] = __ldg(E.sf + dq_sf_index(LAYOUT, row, k, kv));
-            }
-        }
-#pragma unroll
-        for (int p = 0; p < G::kPasses; ++p) {
-            if (!live[p]) continue;
-            uint16_t* dst = static_cast<uint16_t*>(E.y) + rowp[p] * E.ldy + k * G::kBlock;
+            if (!dq_live<FMT>(cur, p)) continue;
+            uint16_t* dst = cur.y + (int64_t)p * G::kRpp * cur.ldy;
             if (FMT == QZ_FMT_MXFP8) {
                 // 2^(byte - 127); byte 0 is the subnormal 2^-127
-                const float s = sc[p] ? __uint_as_float(sc[p] << 23) : __uint_as_float(0x00400000u);
+                const float s = t.sc[p] ? __uint_as_float(t.sc[p] << 23) : __uint_as_float(0x00400000u);
 #pragma unroll
-                for (int h = 0; h < 4; ++h) {  // 8 elements per 16-byte store
-                    uint4 o;
-                    uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        const uint32_t word = qw[p][2 * h + (j >> 1)];
-                        const float2 v = e4m3x2_to_f32x2((j & 1) ? (word >> 16) : (word & 0xFFFFu));
-                        // exact products (at least 2^-136, above the binary32 subnormal step)
-                        const uint32_t lo = bf16_of_exact(__fmul_rn(v.x, s), 0.0f);
-                        const uint32_t hi = bf16_of_exact(__fmul_rn(v.y, s), 0.0f);
-                        ow[j] = lo | (hi << 16);
+                for (int h = 0; h < 4; h += 2) {
+                    const uint4 a = dq_mx8(t.qw[p][2 * h], t.qw[p][2 * h + 1], s);
+                    const uint4 b = dq_mx8(t.qw[p][2 * h + 2], t.qw[p][2 * h + 3], s);
+                    if (cur.y32) {
+                        st_v8(dst + 8 * h, a, b);
+                    } else {
+                        st_v4(dst + 8 * h, a);
+                        st_v4(dst + 8 * h + 8, b);
                     }
-                    st_v4(dst + 8 * h, o);
                 }
             } else {
-                const float A = __ldg(per_row ? E.amax + rowp[p] : E.amax);
-                const float g = __fdiv_rn(A, 2688.0f);  // the FP32 decode scale
-                const float sv = e4m3_value(sc[p]);
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    uint4 o;
-                    uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        const float2 c = e2m1x2_to_f32x2((qw[p][h] >> (8 * j)) & 0xFFu);
-                        const float p0 = __fmul_rn(c.x, sv), p1 = __fmul_rn(c.y, sv);  // exact: <= 6 bits
-                        const float h0 = __fmul_rn(p0, g), h1 = __fmul_rn(p1, g);
-                        const float l0 = __fmaf_rn(p0, g, -h0), l1 = __fmaf_rn(p1, g, -h1);
-                        ow[j] = bf16_of_exact(h0, l0) | (bf16_of_exact(h1, l1) << 16);
-                    }
-                    st_v4(dst + 8 * h, o);
+                if (per_row) g = __fdiv_rn(__ldg(cur.amax + (int64_t)p * G::kRpp), 2688.0f);
+                const __half sh = __float2half_rn(e4m3_value(t.sc[p]));  // exact: e4m3 values are f16 values
+                const __half2 sv = __halves2half2(sh, sh);
+                const uint32_t sv2 = *reinterpret_cast<const uint32_t*>(&sv);
+                const uint4 a = dq_nv8(t.qw[p][0], sv2, g);
+                const uint4 b = dq_nv8(t.qw[p][1], sv2, g);
+                if (cur.y32) {
+                    st_v8(dst, a, b);
+                } else {
+                    st_v4(dst, a);
+                    st_v4(dst + 8, b);
                 }
             }
         }
+        if (!more) break;
+        tile = next;
+        cur = nxt;
     }
 }
 

@@ -70,6 +70,13 @@ __device__ __forceinline__ void ld_pair_16(const void* p, uint32_t (&w)[8]) {
 #undef QZ_LD32
 #undef QZ_LD16
 
+// 32-byte store (the address must be 32-byte aligned).
+__device__ __forceinline__ void st_v8(void* p, uint4 a, uint4 b) {
+    asm volatile("st.global.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(p), "r"(a.x), "r"(a.y), "r"(a.z),
+                 "r"(a.w), "r"(b.x), "r"(b.y), "r"(b.z), "r"(b.w)
+                 : "memory");
+}
+
 __device__ __forceinline__ void st_v4(void* p, uint4 v) {
     asm volatile("st.global.v4.u32 [%0], {%1,%2,%3,%4};" ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
                  : "memory");

@@ -84,6 +84,7 @@ struct TileRef {
     int rows_left;       // pass p is live iff p * kRpp * 8 < rows_left (and col_ok)
     bool col_ok;
     bool a32;            // rows are 32-byte aligned: one 256-bit load per 16 elements
+    bool q32;            // payload rows 32-byte aligned (MXFP8): one 256-bit store per block
     int rt, ct;
     int expert;
 };
@@ -128,6 +129,7 @@ __device__ __forceinline__ TileRef tile_ref(const qz_expert* table, const int* s
     t.rows_left = left > kTileRows ? kTileRows : (int)left;
     t.col_ok = col < E.cols;
     t.a32 = ((reinterpret_cast<uintptr_t>(E.x) & 31) == 0) && ((E.ld & 15) == 0);
+    t.q32 = (reinterpret_cast<uintptr_t>(E.q) & 31) == 0;  // MXFP8 rows are cols bytes, a multiple of 32
     t.expert = e;
     return t;
 }
@@ -190,8 +192,12 @@ __device__ __forceinline__ void tile_pass_mx(const TileRef& t, int p, int lane, 
     c1.w = e4m3x4_words(w[14], w[15], r);
     if (pass_live<QZ_FMT_MXFP8>(t, p)) {
         uint8_t* dst = t.qp + p * G::kRpp * 8 * t.qld;
-        st_v4(dst, c0);
-        st_v4(dst + 16, c1);
+        if (t.q32) {
+            st_v8(dst, c0, c1);  // four lanes fill 128 contiguous bytes in one store
+        } else {
+            st_v4(dst, c0);
+            st_v4(dst + 16, c1);
+        }
     }
     tile_scale_store<QZ_FMT_MXFP8, LAYOUT>(t, p, lane, scale, s);
 }
