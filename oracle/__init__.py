@@ -68,6 +68,7 @@ def _declare(lib):
         "qzo_rmsnorm_quantize": (None, [P, P, P, c.c_float, i64, i64, P, P, c.c_int, P, P, c.c_int, P]),
         "qzo_dequantize_mxfp8": (None, [P, P, i64, i64, c.c_int, P, i64]),
         "qzo_dequantize_nvfp4": (None, [P, P, P, c.c_int, i64, i64, c.c_int, P, i64]),
+        "qzo_attention_merge": (None, [P, P, i64, i64, i64, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -176,6 +177,19 @@ def dequantize_nvfp4(q: np.ndarray, sf: np.ndarray, amax: np.ndarray, per_row: b
     y = np.zeros((rows, cols), dtype=np.uint16)
     if rows > 0:
         lib.qzo_dequantize_nvfp4(_ptr(q), _ptr(sf), _ptr(amax), 1 if per_row else 0, rows, cols, layout, _ptr(y), cols)
+    return y
+
+
+def attention_merge(O: np.ndarray, lse: np.ndarray, lib=None) -> np.ndarray:
+    """bf16 bits [T, H] of the merged attention output of partial outputs
+    O [S, T, H] (float32) with log-sum-exps lse [S, T] (float32) (R12)."""
+    lib = lib or load()
+    S, T, H = O.shape
+    O = np.ascontiguousarray(O, dtype=np.float32)
+    lse = np.ascontiguousarray(lse, dtype=np.float32)
+    y = np.zeros((T, H), dtype=np.uint16)
+    if T > 0:
+        lib.qzo_attention_merge(_ptr(O), _ptr(lse), S, T, H, _ptr(y))
     return y
 
 

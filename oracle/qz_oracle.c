@@ -43,6 +43,8 @@
  *  R8 RMSNorm over h = bf16(x + r); y = bf16(h * rstd * gamma).
  *  R11 Dequantization: the exact product of code value, block scale value
  *     (and the NVFP4 decode scale g), rounded once to bf16.
+ *  R12 Attention decode merge: partial outputs weighted by exp(lse - max lse),
+ *     normalised, rounded to bf16 (binary64 inside), then MXFP8 as usual.
  */
 #include <math.h>
 #include <stdint.h>
@@ -452,6 +454,35 @@ void qzo_dequantize_nvfp4(const uint8_t *q, const uint8_t *sf, const float *amax
             uint8_t s = sf[sf_offset(layout, r, c / 16, kv)];
             double v = qzo_e2m1_value(code) * qzo_e4m3_value(s) * (double)g;
             y[r * ldy + c] = qzo_bf16_from_double(v);
+        }
+    }
+}
+
+/* ------------------------------------------------------------------------- */
+/* Attention decode merge with its MXFP8 form ([CAR] commit 3: the merge      */
+/* kernel that finishes flash-decoding writes the attention output and its    */
+/* MXFP8 form, and the SF rows swizzling invents past the last live row).     */
+/*   R12 S partial outputs O[s, t, :] (binary32) with log-sum-exps lse[s, t]  */
+/*       (natural log, binary32) merge as                                     */
+/*         y[t, i] = bf16( sum_s w_s O[s, t, i] / sum_s w_s ),                */
+/*         w_s = exp(lse[s, t] - max_s lse[s, t])        (binary64 throughout) */
+/*       and y is then quantized to MXFP8 as qzo_quantize_mxfp8 does.         */
+/*   O: [S, T, H] contiguous; lse: [S, T]; y: [T, H] bf16                     */
+/* ------------------------------------------------------------------------- */
+
+void qzo_attention_merge(const float *O, const float *lse, int64_t S, int64_t T, int64_t H, uint16_t *y)
+{
+    for (int64_t t = 0; t < T; t++) {
+        double m = -INFINITY;
+        for (int64_t s = 0; s < S; s++)
+            if ((double)lse[s * T + t] > m) m = (double)lse[s * T + t];
+        double wsum = 0.0;
+        for (int64_t s = 0; s < S; s++) wsum += exp((double)lse[s * T + t] - m);
+        for (int64_t i = 0; i < H; i++) {
+            double acc = 0.0;
+            for (int64_t s = 0; s < S; s++)
+                acc += exp((double)lse[s * T + t] - m) * (double)O[(s * T + t) * H + i];
+            y[t * H + i] = qzo_bf16_from_double(acc / wsum);
         }
     }
 }

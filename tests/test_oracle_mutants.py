@@ -19,7 +19,8 @@ import oracle
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 PIN_FILES = ["tests/test_oracle_formats.py", "tests/test_oracle_mxfp8.py", "tests/test_oracle_layout.py",
-             "tests/test_oracle_nvfp4.py", "tests/test_oracle_norm.py", "tests/test_oracle_dequant.py"]
+             "tests/test_oracle_nvfp4.py", "tests/test_oracle_norm.py", "tests/test_oracle_dequant.py",
+             "tests/test_oracle_merge.py"]
 
 MUTANTS = {
     "ties_away_from_even": ("return (fmod(f, 2.0) == 0.0) ? f : f + 1.0;", "return f + 1.0;"),
@@ -54,6 +55,10 @@ MUTANTS = {
     "dq_mx_exponent_off_by_one": ("double v = qzo_e4m3_value(q[r * cols + c]) * ldexp(1.0, byte - 127);",
                                   "double v = qzo_e4m3_value(q[r * cols + c]) * ldexp(1.0, byte - 126);"),
     "dq_mx_linear_sf_index": ("int byte = sf[sf_offset(layout, r, c / 32, kv)];", "int byte = sf[r * kv + c / 32];"),
+    "merge_no_normalisation": ("y[t * H + i] = qzo_bf16_from_double(acc / wsum);",
+                               "y[t * H + i] = qzo_bf16_from_double(acc);"),
+    "merge_no_max_shift": ("wsum += exp((double)lse[s * T + t] - m);", "wsum += exp((double)lse[s * T + t]);"),
+    "merge_split_token_index": ("(double)O[(s * T + t) * H + i];", "(double)O[(t * S + s) * H + i];"),
     "bf16_double_rounding": ("double n = round_half_even(a / step);\n    double r = n * step;",
                              "double n = round_half_even((double)(float)a / step);\n    double r = n * step;"),
 }
