@@ -71,6 +71,7 @@ KERNEL_SOURCES = {
     "nvfp4_rows_kernel": ("qz_rows.cu", "qz_device.cuh"),
     "rmsnorm_quant_kernel": ("qz_rmsnorm.cu", "qz_device.cuh"),
     "dequant_kernel": ("qz_dequant.cu", "qz_device.cuh"),
+    "attention_merge_kernel": ("qz_merge.cu", "qz_device.cuh"),
 }
 
 
@@ -430,7 +431,8 @@ class L2Flush:
         self.buf.zero_()
 
 
-def extra_workloads(qz, device, stream, peak, which=("split", "fused", "nvfp4", "large", "dequant"), tokens=None):
+def extra_workloads(qz, device, stream, peak, which=("split", "fused", "nvfp4", "large", "dequant", "merge"),
+                    tokens=None):
     out = []
     flush = L2Flush(device)
 
@@ -451,6 +453,8 @@ def extra_workloads(qz, device, stream, peak, which=("split", "fused", "nvfp4", 
         _extra_large(qz, device, rec)
     if "dequant" in which:
         _extra_dequant(qz, device, rec)
+    if "merge" in which:
+        _extra_merge(qz, device, flush, out, peak, tokens)
     return out
 
 
@@ -594,6 +598,42 @@ def _extra_dequant(qz, device, rec):
     torch.cuda.empty_cache()
 
 
+def _extra_merge(qz, device, flush, out, peak, tokens=None):
+    """Attention decode merge of 8 splits at H = 7168 writing bf16 and MXFP8
+    (swizzled) in one kernel, against the same merge writing bf16 followed by
+    a standalone MXFP8 quantize of its output; T swept 1..4096."""
+    S, H = 8, 7168
+    sweep = []
+    for Tn in (tokens or (1, 16, 64, 512, 4096)):
+        O, lse = synth.merge_partials(S, Tn, H, seed=Tn)
+        Od, ld = torch.from_numpy(O).to(device), torch.from_numpy(lse).to(device)
+        y = torch.empty((Tn, H), dtype=torch.bfloat16, device=device)
+        q = torch.empty((Tn, H), dtype=torch.uint8, device=device)
+        sf = torch.empty(max(qz.sf_bytes(Tn, H, qz.FMT_MXFP8, qz.SF_SWIZZLED), 16), dtype=torch.uint8, device=device)
+        tab = qz.ExpertTable([qz.Entry(y, q, sf)])
+
+        def fused():
+            qz.attention_merge_quantize(Od, ld, y, q, sf, qz.SF_SWIZZLED)
+
+        def unfused():
+            qz.attention_merge_quantize(Od, ld, y, None, None, qz.SF_SWIZZLED)
+            qz.quantize_grouped_mxfp8(tab, qz.SF_SWIZZLED)
+
+        fl = flush if Tn >= 512 else None
+        ms_f = _time_graph(fused, reps=10 if fl else 50, flush=fl)
+        ms_u = _time_graph(unfused, reps=10 if fl else 50, flush=fl)
+        nbytes = S * Tn * H * 4 + S * Tn * 4 + Tn * H * 2 + Tn * H + qz.sf_bytes(Tn, H, qz.FMT_MXFP8, qz.SF_SWIZZLED)
+        sweep.append({"T": Tn, "fused_us": round(ms_f * 1e3, 2), "unfused_us": round(ms_u * 1e3, 2),
+                      "fused_GB/s": round(nbytes / (ms_f / 1e3) / GB, 1)})
+        del Od, ld, y, q, sf, tab
+    big = sweep[-1]
+    out.append({"workload": "attention decode merge, 8 splits, H=7168, bf16 + MXFP8 swizzled in one kernel "
+                            "vs merge then standalone quantize, T=1..4096",
+                "kernel": "attention_merge_kernel", "sweep": sweep,
+                "timing": "CUDA graph of 50 calls (T < 512) or 10 calls after an L2 flush each",
+                "frac_of_hbm_peak_fused_T4096": round(big["fused_GB/s"] / peak, 4) if big["T"] == 4096 else None})
+
+
 # ---------------------------------------------------------------------------
 # CPU oracle timing (the reference arm and the cpu_baseline key)
 # ---------------------------------------------------------------------------
@@ -662,7 +702,7 @@ def main():
     ap.add_argument("--no-extra", action="store_true", help="skip the other workloads")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
-    ap.add_argument("--only", choices=["split", "fused", "nvfp4", "large", "dequant"], default=None,
+    ap.add_argument("--only", choices=["split", "fused", "nvfp4", "large", "dequant", "merge"], default=None,
                     help="time only this secondary workload and print its record (profiling aid)")
     ap.add_argument("--tokens", type=str, default=None,
                     help="comma-separated token counts for the fused sweep (default: 1..4096)")

@@ -241,6 +241,31 @@ qz_status qz_swizzle_scales(const qz_sf_pair *d_table, int n, void *stream, cons
 qz_status qz_dequantize_grouped(const qz_dq_expert *d_table, int n_experts, int fmt, int per_row, int layout,
                                 void *stream, const qz_launch_opts *opts);
 
+/* Attention decode merge that also writes its MXFP8 form (TensorRT-LLM "MXFP8
+ * carrier and quantize folds", commit 3: the kernel finishing flash-decoding
+ * writes the attention output and its MXFP8 form, and zeroes the SF rows the
+ * swizzled layout invents past the last live row, so no memset is needed).
+ * A producer kernel built on include/qz_quant.cuh.
+ *   d_partial: float [S, T, H], the S partial outputs of each token
+ *   d_lse:     float [S, T], their natural-log sum-exps
+ *   d_out:     bf16 [T, H], y[t] = sum_s w_s O[s, t] / sum_s w_s,
+ *              w_s = exp(lse[s, t] - max_s lse[s, t]), rounded to nearest even
+ *   d_q, d_sf: e4m3 [T, H] and the SF region (qz_sf_bytes(T, H, QZ_FMT_MXFP8,
+ *              layout) bytes) of y quantized exactly as qz_quantize_grouped_mxfp8
+ *              would; d_q == NULL skips the MXFP8 form (d_sf is then ignored)
+ * The merge accumulates in binary64 and rounds once to bf16.
+ * 1 <= S <= QZ_MAX_SPLITS, T >= 0, H a multiple of 32 up to QZ_MAX_HIDDEN.
+ * One launch, asynchronous on the stream, no allocation.
+ * Errors (before any launch): QZ_ERR_INVALID_ARG for a bad S, T < 0, a bad H,
+ * an unknown layout or a NULL pointer that is needed; QZ_ERR_ALIGNMENT for
+ * d_partial / d_out not 16-byte aligned, d_q not 8-byte aligned or a
+ * swizzled d_sf not 16-byte aligned; QZ_ERR_UNSUPPORTED for a swizzled
+ * layout with H / 32 not a multiple of 4 (the kernel writes no padded
+ * scale columns). */
+#define QZ_MAX_SPLITS 4096
+qz_status qz_attention_merge_quantize(const float *d_partial, const float *d_lse, int S, int64_t T, int64_t H,
+                                      void *d_out, void *d_q, uint8_t *d_sf, int layout, void *stream);
+
 /* Largest table of qz_quantize_grouped_nvfp4_compute_noalloc. */
 #define QZ_STATIC_WS_MAX_EXPERTS 1024
 

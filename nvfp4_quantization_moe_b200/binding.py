@@ -40,6 +40,7 @@ EXPORTED = (
     "qz_workspace_bytes",
     "qz_quantize_grouped_nvfp4_compute_noalloc",
     "qz_dequantize_grouped",
+    "qz_attention_merge_quantize",
 )
 STATIC_WS_MAX_EXPERTS = 1024
 
@@ -109,6 +110,8 @@ def load(path: str = LIB_PATH):
         lib.qz_quantize_grouped_nvfp4_compute_noalloc.argtypes = [P, I, I, P, P]
         lib.qz_dequantize_grouped.restype = I
         lib.qz_dequantize_grouped.argtypes = [P, I, I, I, I, P, P]
+        lib.qz_attention_merge_quantize.restype = I
+        lib.qz_attention_merge_quantize.argtypes = [P, P, I, i64, i64, P, P, P, I, P]
         _lib = lib
         return lib
 
@@ -308,6 +311,16 @@ def dequantize_grouped(table: DqTable, fmt: int, per_row: bool, layout: int, str
     _check(load().qz_dequantize_grouped(ctypes.c_void_p(table.ptr), table.n, int(fmt), 1 if per_row else 0,
                                         int(layout), _stream_ptr(stream), _opts(err, max_ctas)),
            "qz_dequantize_grouped")
+
+
+def attention_merge_quantize(partial, lse, out, q=None, sf=None, layout: int = SF_SWIZZLED, stream=None):
+    """Merge float partial outputs [S, T, H] by their log-sum-exps [S, T] into
+    bf16 out [T, H] and (q given) its MXFP8 form q [T, H] + SF region sf."""
+    S, T, H = partial.shape
+    _check(load().qz_attention_merge_quantize(ctypes.c_void_p(_ptr(partial)), ctypes.c_void_p(_ptr(lse)), int(S),
+                                              int(T), int(H), ctypes.c_void_p(_ptr(out)), ctypes.c_void_p(_ptr(q)),
+                                              ctypes.c_void_p(_ptr(sf)), int(layout), _stream_ptr(stream)),
+           "qz_attention_merge_quantize")
 
 
 def swizzle_scales(table: SfPairTable, stream=None, err=None, max_ctas: int = 0):

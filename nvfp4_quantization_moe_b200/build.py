@@ -32,7 +32,8 @@ def sources():
 
 
 def _inputs():
-    return sources() + glob.glob(os.path.join(CSRC, "*.cuh")) + [os.path.join(INCLUDE, "qz.h")]
+    return sources() + glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(INCLUDE, "*.h")) + \
+        glob.glob(os.path.join(INCLUDE, "*.cuh"))
 
 
 def stale() -> bool:

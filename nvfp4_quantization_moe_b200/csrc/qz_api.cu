@@ -29,6 +29,8 @@ int rows_blocks_per_sm(int n);
 cudaError_t launch_dequant(const qz_dq_expert* table, int n, int fmt, bool per_row, int layout, int grid,
                            cudaStream_t s, unsigned* d_err);
 int dequant_blocks_per_sm(int n);
+cudaError_t launch_attention_merge(const float* O, const float* lse, int S, int64_t T, int64_t H, uint16_t* y,
+                                   uint8_t* q, uint8_t* sf, int layout, cudaStream_t s);
 }  // namespace qz
 
 namespace {
@@ -194,6 +196,20 @@ qz_status qz_dequantize_grouped(const qz_dq_expert* d_table, int n_experts, int 
     if (n_experts == 0) return QZ_OK;
     return from_cuda(qz::launch_dequant(d_table, n_experts, fmt, per_row != 0, layout, wave_grid(6, opts),
                                         (cudaStream_t)stream, err_word(opts)));
+}
+
+qz_status qz_attention_merge_quantize(const float* d_partial, const float* d_lse, int S, int64_t T, int64_t H,
+                                      void* d_out, void* d_q, uint8_t* d_sf, int layout, void* stream) {
+    if (S < 1 || S > QZ_MAX_SPLITS || T < 0 || T > 0x7FFFFFFFLL) return QZ_ERR_INVALID_ARG;
+    if (H <= 0 || H % 32 != 0 || H > QZ_MAX_HIDDEN) return QZ_ERR_INVALID_ARG;
+    if (!valid_layout(layout)) return QZ_ERR_INVALID_ARG;
+    if (d_q && layout == QZ_SF_SWIZZLED_128x4 && (H / 32) % 4 != 0) return QZ_ERR_UNSUPPORTED;
+    if (T == 0) return QZ_OK;
+    if (!d_partial || !d_lse || !d_out || (d_q && !d_sf)) return QZ_ERR_INVALID_ARG;
+    if (!aligned(d_partial, 16) || !aligned(d_out, 16)) return QZ_ERR_ALIGNMENT;
+    if (d_q && (!aligned(d_q, 8) || (layout == QZ_SF_SWIZZLED_128x4 && !aligned(d_sf, 16)))) return QZ_ERR_ALIGNMENT;
+    return from_cuda(qz::launch_attention_merge(d_partial, d_lse, S, T, H, static_cast<uint16_t*>(d_out),
+                                                static_cast<uint8_t*>(d_q), d_sf, layout, (cudaStream_t)stream));
 }
 
 size_t qz_workspace_bytes(int n_experts) {

@@ -154,3 +154,13 @@ def random_amax(n: int, seed: int = 0, lo: float = -20.0, hi: float = 20.0) -> n
     """Random positive binary32 amax values spread over 2^lo .. 2^hi."""
     rng = np.random.default_rng(seed)
     return (np.exp2(rng.uniform(lo, hi, size=n)) * rng.uniform(1.0, 2.0, size=n)).astype(np.float32)
+
+
+def merge_partials(splits: int, tokens: int, hidden: int, seed: int = 0):
+    """Flash-decoding partial outputs float32 [S, T, H] (N(0,1) times a per
+    split-and-token factor 2^U(-4,4)) and their log-sum-exps float32 [S, T]
+    (U(-6, 6))."""
+    rng = np.random.default_rng(seed)
+    O = rng.standard_normal((splits, tokens, hidden)) * np.exp2(rng.uniform(-4, 4, (splits, tokens, 1)))
+    lse = rng.uniform(-6, 6, (splits, tokens))
+    return O.astype(np.float32), lse.astype(np.float32)

@@ -81,6 +81,22 @@ def test_host_errors_without_gpu(lib):
     assert lib.qz_dequantize_grouped(P(0x1000), 2, 5, 0, 0, None, None) == qz.QZ_ERR_INVALID_ARG   # format
     assert lib.qz_dequantize_grouped(P(0x1000), 2, 1, 0, 3, None, None) == qz.QZ_ERR_INVALID_ARG   # layout
     assert lib.qz_dequantize_grouped(None, 0, 1, 1, 1, None, None) == qz.QZ_OK
+    a16 = P(0x10000)
+
+    def merge(S=4, T=3, H=1024, O=a16, lse=a16, y=a16, q=a16, sf=a16, layout=1):
+        return lib.qz_attention_merge_quantize(O, lse, S, T, H, y, q, sf, layout, None)
+
+    assert merge(S=0) == qz.QZ_ERR_INVALID_ARG
+    assert merge(S=4097) == qz.QZ_ERR_INVALID_ARG
+    assert merge(T=-1) == qz.QZ_ERR_INVALID_ARG
+    assert merge(H=1000) == qz.QZ_ERR_INVALID_ARG                 # not a multiple of 32
+    assert merge(H=96) == qz.QZ_ERR_UNSUPPORTED                   # swizzled with H / 32 = 3
+    assert merge(layout=2) == qz.QZ_ERR_INVALID_ARG
+    assert merge(O=None) == qz.QZ_ERR_INVALID_ARG
+    assert merge(sf=None) == qz.QZ_ERR_INVALID_ARG                # quantized form without SF storage
+    assert merge(y=P(0x10008)) == qz.QZ_ERR_ALIGNMENT
+    assert merge(sf=P(0x10004)) == qz.QZ_ERR_ALIGNMENT            # swizzled SF wants 16 bytes
+    assert merge(T=0) == qz.QZ_OK
     a = P(0x10000)
 
     def norm(T=4, H=7168, fmt=0, layout=1, x=a, r=a, g=a, y=a, h=None, q=a, sf=a, amax=None):
