@@ -193,6 +193,18 @@ def attention_merge(O: np.ndarray, lse: np.ndarray, lib=None) -> np.ndarray:
     return y
 
 
+def quantize_colwise(x: np.ndarray, fmt: int, layout: int, mode: int = NVFP4_PER_TENSOR_GIVEN,
+                     amax_in: float | None = None, lib=None):
+    """Column-wise quantization of x [rows, cols]: blocks run down the columns,
+    i.e. the row-wise quantization of the transpose x^T [cols, rows]
+    (payload [cols, rows] or [cols, rows/2], SF of a [cols, rows] matrix).
+    Returns (q, sf) for MXFP8, (q, sf, amax) for NVFP4."""
+    xt = np.ascontiguousarray(np.asarray(x, dtype=np.uint16).T)
+    if fmt == MXFP8:
+        return quantize_mxfp8(xt, layout, lib)
+    return quantize_nvfp4(xt, layout, mode, amax_in, lib)
+
+
 def swizzle(lin: np.ndarray, rows: int, kv: int, lib=None) -> np.ndarray:
     lib = lib or load()
     lin = np.ascontiguousarray(lin, dtype=np.uint8)
