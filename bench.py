@@ -72,6 +72,7 @@ KERNEL_SOURCES = {
     "rmsnorm_quant_kernel": ("qz_rmsnorm.cu", "qz_device.cuh"),
     "dequant_kernel": ("qz_dequant.cu", "qz_device.cuh"),
     "attention_merge_kernel": ("qz_merge.cu", "qz_device.cuh"),
+    "colwise_kernel": ("qz_colwise.cu", "qz_device.cuh"),
 }
 
 
@@ -431,7 +432,7 @@ class L2Flush:
         self.buf.zero_()
 
 
-def extra_workloads(qz, device, stream, peak, which=("split", "fused", "nvfp4", "large", "dequant", "merge"),
+def extra_workloads(qz, device, stream, peak, which=("split", "fused", "nvfp4", "large", "dequant", "merge", "colwise"),
                     tokens=None):
     out = []
     flush = L2Flush(device)
@@ -455,6 +456,8 @@ def extra_workloads(qz, device, stream, peak, which=("split", "fused", "nvfp4", 
         _extra_dequant(qz, device, rec)
     if "merge" in which:
         _extra_merge(qz, device, flush, out, peak, tokens)
+    if "colwise" in which:
+        _extra_colwise(qz, device, rec)
     return out
 
 
@@ -598,6 +601,33 @@ def _extra_dequant(qz, device, rec):
     torch.cuda.empty_cache()
 
 
+def _extra_colwise(qz, device, rec):
+    """Column-wise (transposed) quantization of a Qwen3-30B-A3B gate_up
+    projection (128 experts of [1536, 2048]) to MXFP8 and to NVFP4 (given
+    per-tensor amax), swizzled, in one call."""
+    cfg = synth.QWEN3_30B
+    rows, cols = cfg["gate_up"]
+    n = cfg["experts"]
+    stack = synth.expert_stack(n, (rows, cols), cfg["std"], seed=cfg["seed"], device=device)
+    for fmt, fname in ((qz.FMT_MXFP8, "MXFP8"), (qz.FMT_NVFP4, "NVFP4 (given amax)")):
+        qb = rows * cols if fmt == qz.FMT_MXFP8 else rows * cols // 2
+        nsf = qz.sf_bytes(cols, rows, fmt, qz.SF_SWIZZLED)
+        ents = []
+        for x in stack.unbind(0):
+            q = torch.empty(qb, dtype=torch.uint8, device=device)
+            sf = torch.empty(nsf, dtype=torch.uint8, device=device)
+            a = torch.full((1,), 0.1, dtype=torch.float32, device=device) if fmt == qz.FMT_NVFP4 else None
+            ents.append(qz.Entry(x, q, sf, a))
+        tab = qz.ExpertTable(ents)
+        ms = _time_graph(lambda f=fmt, t=tab: qz.quantize_grouped_colwise(t, f, qz.SF_SWIZZLED), reps=5)
+        nbytes = n * (rows * cols * 2 + qb + nsf + (4 if fmt == qz.FMT_NVFP4 else 0))
+        rec(f"column-wise quantize Qwen3-30B-A3B gate_up [1536, 2048] x128 experts to {fname}, swizzled, one call",
+            nbytes, ms, 1, kernel="colwise_kernel")
+        del ents, tab
+    del stack
+    torch.cuda.empty_cache()
+
+
 def _extra_merge(qz, device, flush, out, peak, tokens=None):
     """Attention decode merge of 8 splits at H = 7168 writing bf16 and MXFP8
     (swizzled) in one kernel, against the same merge writing bf16 followed by
@@ -702,7 +732,7 @@ def main():
     ap.add_argument("--no-extra", action="store_true", help="skip the other workloads")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
-    ap.add_argument("--only", choices=["split", "fused", "nvfp4", "large", "dequant", "merge"], default=None,
+    ap.add_argument("--only", choices=["split", "fused", "nvfp4", "large", "dequant", "merge", "colwise"], default=None,
                     help="time only this secondary workload and print its record (profiling aid)")
     ap.add_argument("--tokens", type=str, default=None,
                     help="comma-separated token counts for the fused sweep (default: 1..4096)")

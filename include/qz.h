@@ -241,6 +241,24 @@ qz_status qz_swizzle_scales(const qz_sf_pair *d_table, int n, void *stream, cons
 qz_status qz_dequantize_grouped(const qz_dq_expert *d_table, int n_experts, int fmt, int per_row, int layout,
                                 void *stream, const qz_launch_opts *opts);
 
+/* Column-wise (transposed) grouped quantization: the blocks run down the
+ * columns of each expert's x [rows, cols], i.e. x^T is quantized row-wise
+ * (TransformerEngine PR #3800, Changes: its fast path is "rowwise-only"; the
+ * column-wise form is the weight-gradient GEMM's operand).  Per expert:
+ *   q:  MXFP8 e4m3 [cols, rows] (16-byte aligned), NVFP4 packed e2m1
+ *       [cols, rows/2] (8-byte aligned), dense rows
+ *   sf: the SF region of a [cols, rows] matrix, qz_sf_bytes(cols, rows, fmt,
+ *       layout) bytes, padding written as 0x00
+ *   amax: NVFP4 only, the tensor amax, given (the row-wise
+ *       QZ_NVFP4_PER_TENSOR_COMPUTE call of the same tensor writes it)
+ * rows must be a multiple of 32 (MXFP8) / 16 (NVFP4); cols any positive
+ * number; x as for the row-wise calls.  Results equal the row-wise call on
+ * the transposed tensor byte for byte.  One persistent launch, no allocation.
+ * Errors: as qz_quantize_grouped_mxfp8, plus QZ_ERR_INVALID_ARG for an
+ * unknown fmt; invalid entries are skipped and reported through opts->d_err. */
+qz_status qz_quantize_grouped_colwise(const qz_expert *d_table, int n_experts, int fmt, int layout, void *stream,
+                                      const qz_launch_opts *opts);
+
 /* Attention decode merge that also writes its MXFP8 form (TensorRT-LLM "MXFP8
  * carrier and quantize folds", commit 3: the kernel finishing flash-decoding
  * writes the attention output and its MXFP8 form, and zeroes the SF rows the

@@ -11,7 +11,7 @@ from .binding import (  # noqa: F401
     DERR_ALIGN, DERR_NULL, DERR_SHAPE, DERR_TOO_LARGE, EXPORTED, FMT_MXFP8, FMT_NVFP4, LIB_PATH, MAX_EXPERTS,
     MAX_HIDDEN, NVFP4_PER_ROW, NVFP4_PER_TENSOR_COMPUTE, NVFP4_PER_TENSOR_GIVEN, QZ_ERR_ALIGNMENT, QZ_ERR_CUDA,
     QZ_ERR_INVALID_ARG, QZ_ERR_UNSUPPORTED, QZ_OK, SF_LINEAR, SF_SWIZZLED, DqEntry, DqTable, Entry, ExpertTable,
-    QzError, SfPairTable, alloc_outputs, attention_merge_quantize, dequantize_grouped, alloc_workspace, load, quantize_experts, quantize_grouped_mxfp8,
+    QzError, SfPairTable, alloc_outputs, attention_merge_quantize, dequantize_grouped, quantize_grouped_colwise, alloc_workspace, load, quantize_experts, quantize_grouped_mxfp8,
     quantize_grouped_nvfp4, quantize_grouped_nvfp4_compute_noalloc, rmsnorm_quantize, sf_bytes, status_string, swizzle_scales, workspace_bytes,
 )
 

@@ -41,6 +41,7 @@ EXPORTED = (
     "qz_quantize_grouped_nvfp4_compute_noalloc",
     "qz_dequantize_grouped",
     "qz_attention_merge_quantize",
+    "qz_quantize_grouped_colwise",
 )
 STATIC_WS_MAX_EXPERTS = 1024
 
@@ -110,6 +111,8 @@ def load(path: str = LIB_PATH):
         lib.qz_quantize_grouped_nvfp4_compute_noalloc.argtypes = [P, I, I, P, P]
         lib.qz_dequantize_grouped.restype = I
         lib.qz_dequantize_grouped.argtypes = [P, I, I, I, I, P, P]
+        lib.qz_quantize_grouped_colwise.restype = I
+        lib.qz_quantize_grouped_colwise.argtypes = [P, I, I, I, P, P]
         lib.qz_attention_merge_quantize.restype = I
         lib.qz_attention_merge_quantize.argtypes = [P, P, I, i64, i64, P, P, P, I, P]
         _lib = lib
@@ -311,6 +314,14 @@ def dequantize_grouped(table: DqTable, fmt: int, per_row: bool, layout: int, str
     _check(load().qz_dequantize_grouped(ctypes.c_void_p(table.ptr), table.n, int(fmt), 1 if per_row else 0,
                                         int(layout), _stream_ptr(stream), _opts(err, max_ctas)),
            "qz_dequantize_grouped")
+
+
+def quantize_grouped_colwise(table: ExpertTable, fmt: int, layout: int, stream=None, err=None, max_ctas: int = 0):
+    """Column-wise quantization: each entry's q / sf receive x^T quantized
+    row-wise (q [cols, rows] or [cols, rows/2]); NVFP4 uses the given amax."""
+    _check(load().qz_quantize_grouped_colwise(ctypes.c_void_p(table.ptr), table.n, int(fmt), int(layout),
+                                              _stream_ptr(stream), _opts(err, max_ctas)),
+           "qz_quantize_grouped_colwise")
 
 
 def attention_merge_quantize(partial, lse, out, q=None, sf=None, layout: int = SF_SWIZZLED, stream=None):

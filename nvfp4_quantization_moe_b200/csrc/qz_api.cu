@@ -29,6 +29,9 @@ int rows_blocks_per_sm(int n);
 cudaError_t launch_dequant(const qz_dq_expert* table, int n, int fmt, bool per_row, int layout, int grid,
                            cudaStream_t s, unsigned* d_err);
 int dequant_blocks_per_sm(int n);
+cudaError_t launch_colwise(const qz_expert* table, int n, int fmt, int layout, int grid, cudaStream_t s,
+                           unsigned* d_err);
+int colwise_blocks_per_sm(int n);
 cudaError_t launch_attention_merge(const float* O, const float* lse, int S, int64_t T, int64_t H, uint16_t* y,
                                    uint8_t* q, uint8_t* sf, int layout, cudaStream_t s);
 }  // namespace qz
@@ -36,11 +39,11 @@ cudaError_t launch_attention_merge(const float* O, const float* lse, int S, int6
 namespace {
 
 constexpr int kMaxDevices = 64;
-constexpr int kKinds = 7;  // mxfp8, nvfp4 tile, swizzle, amax, rows, computed-amax L2 path, dequantize
+constexpr int kKinds = 8;  // mxfp8, nvfp4 tile, swizzle, amax, rows, computed-amax L2 path, dequantize, colwise
 
 struct DeviceLimits {
     int sms = 0;
-    int per_sm[kKinds] = {0, 0, 0, 0, 0, 0, 0};
+    int per_sm[kKinds] = {0, 0, 0, 0, 0, 0, 0, 0};
 };
 
 std::mutex g_mu;
@@ -64,6 +67,7 @@ int wave_grid(int kind, const qz_launch_opts* opts) {
         if (d.per_sm[kind] == 0)
             d.per_sm[kind] = (kind == 4)   ? qz::rows_blocks_per_sm(QZ_MAX_EXPERTS)
                              : (kind == 6) ? qz::dequant_blocks_per_sm(QZ_MAX_EXPERTS)
+                             : (kind == 7) ? qz::colwise_blocks_per_sm(QZ_MAX_EXPERTS)
                                            : qz::grouped_blocks_per_sm(kind, QZ_MAX_EXPERTS);
         grid = d.sms * d.per_sm[kind];
     }
@@ -196,6 +200,17 @@ qz_status qz_dequantize_grouped(const qz_dq_expert* d_table, int n_experts, int 
     if (n_experts == 0) return QZ_OK;
     return from_cuda(qz::launch_dequant(d_table, n_experts, fmt, per_row != 0, layout, wave_grid(6, opts),
                                         (cudaStream_t)stream, err_word(opts)));
+}
+
+qz_status qz_quantize_grouped_colwise(const qz_expert* d_table, int n_experts, int fmt, int layout, void* stream,
+                                      const qz_launch_opts* opts) {
+    qz_status st = check_table(d_table, n_experts);
+    if (st != QZ_OK) return st;
+    if (!valid_layout(layout)) return QZ_ERR_INVALID_ARG;
+    if (fmt != QZ_FMT_MXFP8 && fmt != QZ_FMT_NVFP4) return QZ_ERR_INVALID_ARG;
+    if (n_experts == 0) return QZ_OK;
+    return from_cuda(qz::launch_colwise(d_table, n_experts, fmt, layout, wave_grid(7, opts), (cudaStream_t)stream,
+                                        err_word(opts)));
 }
 
 qz_status qz_attention_merge_quantize(const float* d_partial, const float* d_lse, int S, int64_t T, int64_t H,

@@ -81,6 +81,10 @@ def test_host_errors_without_gpu(lib):
     assert lib.qz_dequantize_grouped(P(0x1000), 2, 5, 0, 0, None, None) == qz.QZ_ERR_INVALID_ARG   # format
     assert lib.qz_dequantize_grouped(P(0x1000), 2, 1, 0, 3, None, None) == qz.QZ_ERR_INVALID_ARG   # layout
     assert lib.qz_dequantize_grouped(None, 0, 1, 1, 1, None, None) == qz.QZ_OK
+    assert lib.qz_quantize_grouped_colwise(None, 1, 0, 0, None, None) == qz.QZ_ERR_INVALID_ARG
+    assert lib.qz_quantize_grouped_colwise(P(0x1000), 1, 3, 0, None, None) == qz.QZ_ERR_INVALID_ARG
+    assert lib.qz_quantize_grouped_colwise(P(0x1000), 1, 0, 4, None, None) == qz.QZ_ERR_INVALID_ARG
+    assert lib.qz_quantize_grouped_colwise(None, 0, 1, 1, None, None) == qz.QZ_OK
     a16 = P(0x10000)
 
     def merge(S=4, T=3, H=1024, O=a16, lse=a16, y=a16, q=a16, sf=a16, layout=1):
