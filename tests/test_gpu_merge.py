@@ -1,7 +1,9 @@
 """GPU checks of the attention decode merge with its MXFP8 form
 (qz_attention_merge_quantize) and of the public device functions of
 include/qz_quant.cuh.  The merged bf16 output is within one bf16 ulp of the
-oracle's binary64 merge (the GPU uses binary32 and its own exp); its MXFP8
+oracle's binary64 merge (both accumulate in binary64, but the device exp and
+the host exp may differ in their last bits, which can move a result that lies
+next to a bf16 rounding boundary); its MXFP8
 payload and scales equal the oracle quantizer applied to the GPU's own bf16
 output, byte for byte, padded scale rows included.  The device functions are
 compiled here into a small test kernel and must match the oracle quantizers."""
