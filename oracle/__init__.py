@@ -29,6 +29,8 @@ _lock = threading.Lock()
 _lib = None
 
 MXFP8, NVFP4 = 0, 1
+FP8_BLOCK128 = 2            # e4m3 payload with FP32 scales of 128 x 128 blocks (split only)
+AMAX_NONE, AMAX_PER_TENSOR, AMAX_PER_ROW = 0, 1, 2
 LINEAR, SWIZZLED = 0, 1
 NVFP4_PER_TENSOR_GIVEN, NVFP4_PER_TENSOR_COMPUTE, NVFP4_PER_ROW = 0, 1, 2
 
@@ -69,6 +71,8 @@ def _declare(lib):
         "qzo_dequantize_mxfp8": (None, [P, P, i64, i64, c.c_int, P, i64]),
         "qzo_dequantize_nvfp4": (None, [P, P, P, c.c_int, i64, i64, c.c_int, P, i64]),
         "qzo_attention_merge": (None, [P, P, i64, i64, i64, P]),
+        "qzo_split_fused": (c.c_int, [c.c_int, P, P, P, c.c_int, i64, i64, i64, c.c_int, c.c_int,
+                                      P, P, P, P, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -191,6 +195,51 @@ def attention_merge(O: np.ndarray, lse: np.ndarray, lib=None) -> np.ndarray:
     if T > 0:
         lib.qzo_attention_merge(_ptr(O), _ptr(lse), S, T, H, _ptr(y))
     return y
+
+
+class CutRefused(ValueError):
+    """A gate|up cut that would divide a scale block (R14)."""
+
+
+def split_region_bytes(fmt: int, rows: int, cols: int, layout: int, lib=None) -> int:
+    """Scale bytes of one part of ``rows`` weight rows after the split."""
+    lib = lib or load()
+    if fmt == FP8_BLOCK128:
+        return -(-rows // 128) * -(-cols // 128) * 4 if rows > 0 else 0
+    return int(lib.qzo_sf_region_bytes(rows, cols // (32 if fmt == MXFP8 else 16), layout))
+
+
+def split_fused(fmt: int, q: np.ndarray, sf: np.ndarray, amax, amax_kind: int, cols: int, cut: int,
+                src_layout: int, dst_layout: int, lib=None):
+    """Cut a folded fused expert (payload q [rows, row_bytes], scales sf in
+    src_layout, amax per amax_kind) at weight row ``cut`` (R14).  Returns
+    [(q_p, sf_p, amax_p)] for part 0 (rows [0, cut)) and part 1 (rows
+    [cut, rows)); raises CutRefused when the cut divides a scale block."""
+    lib = lib or load()
+    q = np.ascontiguousarray(q, dtype=np.uint8)
+    rows = q.shape[0]
+    sf = np.ascontiguousarray(sf, dtype=np.uint8).reshape(-1)
+    row_bytes = cols // 2 if fmt == NVFP4 else cols
+    counts = (cut, rows - cut)
+    outs = []
+    for n in counts:
+        qp = np.full((max(n, 0), row_bytes), 0xA5, dtype=np.uint8)
+        sp = _dirty(split_region_bytes(fmt, max(n, 0), cols, dst_layout, lib))
+        ap = np.full(max(1 if amax_kind == AMAX_PER_TENSOR else max(n, 0), 1), np.nan, dtype=np.float32)
+        outs.append((qp, sp, ap))
+    a = np.ascontiguousarray(np.zeros(1, np.float32) if amax is None else amax, dtype=np.float32)
+    rc = lib.qzo_split_fused(fmt, _ptr(q) if q.size else None, _ptr(sf), _ptr(a), amax_kind, rows, cols, cut,
+                             src_layout, dst_layout,
+                             _ptr(outs[0][0]), _ptr(outs[0][1]), _ptr(outs[0][2]),
+                             _ptr(outs[1][0]), _ptr(outs[1][1]), _ptr(outs[1][2]))
+    if rc != 0:
+        raise CutRefused(f"cut {cut} of {rows} rows divides a scale block")
+    res = []
+    for (qp, sp, ap), n in zip(outs, counts):
+        nb = split_region_bytes(fmt, n, cols, dst_layout, lib)
+        na = 1 if amax_kind == AMAX_PER_TENSOR else (n if amax_kind == AMAX_PER_ROW else 0)
+        res.append((qp, sp[:nb], ap[:na]))
+    return res
 
 
 def quantize_colwise(x: np.ndarray, fmt: int, layout: int, mode: int = NVFP4_PER_TENSOR_GIVEN,

@@ -45,6 +45,9 @@
  *     (and the NVFP4 decode scale g), rounded once to bf16.
  *  R12 Attention decode merge: partial outputs weighted by exp(lse - max lse),
  *     normalised, rounded to bf16 (binary64 inside), then MXFP8 as usual.
+ *  R14 Fused gate|up split: rows [0, cut) and [cut, rows), scales cut with
+ *     their rows and laid out anew per part; a scale block that covers rows
+ *     on both sides of the cut is refused.
  */
 #include <math.h>
 #include <stdint.h>
@@ -485,4 +488,62 @@ void qzo_attention_merge(const float *O, const float *lse, int64_t S, int64_t T,
             y[t * H + i] = qzo_bf16_from_double(acc / wsum);
         }
     }
+}
+
+/* ------------------------------------------------------------------------- */
+/* Gate|up split of a folded fused expert ([FOLD] keep-fused fold: the fused  */
+/* (2I, H) expert is quantized as one tensor, gate and up sharing one         */
+/* per-tensor amax and so one weight_scale_2; the split then cuts the folded  */
+/* payload and its scales by weight rows into gate and up, each with its own  */
+/* storage, and refuses a scale block that the cut would divide).             */
+/*   R14 part 0 = weight rows [0, cut), part 1 = rows [cut, rows).            */
+/*       fmt 0 MXFP8 / 1 NVFP4: one scale row per weight row, so every cut    */
+/*       is exact; each part's SF region is laid out anew in dst_layout with  */
+/*       its own padding (0x00), whatever src_layout was.                     */
+/*       fmt 2 FP8 with FP32 scales of 128 x 128 blocks (linear only, scale   */
+/*       matrix [ceil(rows/128), ceil(cols/128)]): a scale row covers 128     */
+/*       weight rows, so a cut inside a block (cut % 128 != 0, cut < rows) is */
+/*       refused.                                                             */
+/*       amax_kind 0: none; 1: one per-tensor amax, given to both parts; 2:  */
+/*       one amax per row, cut with the rows.                                 */
+/*   Returns 0, or -1 for a refused cut (nothing is written then).            */
+/* ------------------------------------------------------------------------- */
+
+int qzo_split_fused(int fmt, const uint8_t *q, const uint8_t *sf, const float *amax, int amax_kind,
+                    int64_t rows, int64_t cols, int64_t cut, int src_layout, int dst_layout,
+                    uint8_t *q0, uint8_t *sf0, float *amax0, uint8_t *q1, uint8_t *sf1, float *amax1)
+{
+    int64_t row_block = (fmt == 2) ? 128 : 1;       /* weight rows per scale row */
+    if (cut < 0 || cut > rows) return -1;
+    if (cut % row_block != 0 && cut < rows) return -1;
+
+    int64_t row_bytes = (fmt == 1) ? cols / 2 : cols;
+    int64_t first[2] = {0, cut};
+    int64_t count[2] = {cut, rows - cut};
+    uint8_t *qo[2] = {q0, q1};
+    uint8_t *so[2] = {sf0, sf1};
+    float *ao[2] = {amax0, amax1};
+
+    for (int p = 0; p < 2; p++) {
+        for (int64_t i = 0; i < count[p] * row_bytes; i++) qo[p][i] = q[first[p] * row_bytes + i];
+
+        if (fmt == 2) {
+            /* FP32 block scales, row-major: scale rows [first/128, first/128 + ceil(count/128)) */
+            int64_t scols = (cols + 127) / 128;
+            int64_t srow0 = first[p] / 128;
+            int64_t srows = (count[p] + 127) / 128;
+            for (int64_t i = 0; i < srows * scols * 4; i++) so[p][i] = sf[srow0 * scols * 4 + i];
+        } else {
+            int64_t kv = cols / (fmt == 0 ? 32 : 16);
+            sf_clear(so[p], count[p], kv, dst_layout);
+            for (int64_t r = 0; r < count[p]; r++)
+                for (int64_t k = 0; k < kv; k++)
+                    so[p][sf_offset(dst_layout, r, k, kv)] = sf[sf_offset(src_layout, first[p] + r, k, kv)];
+        }
+
+        if (amax_kind == 1) ao[p][0] = amax[0];
+        if (amax_kind == 2)
+            for (int64_t r = 0; r < count[p]; r++) ao[p][r] = amax[first[p] + r];
+    }
+    return 0;
 }

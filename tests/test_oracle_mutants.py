@@ -20,7 +20,7 @@ import oracle
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 PIN_FILES = ["tests/test_oracle_formats.py", "tests/test_oracle_mxfp8.py", "tests/test_oracle_layout.py",
              "tests/test_oracle_nvfp4.py", "tests/test_oracle_norm.py", "tests/test_oracle_dequant.py",
-             "tests/test_oracle_merge.py"]
+             "tests/test_oracle_merge.py", "tests/test_oracle_split.py"]
 
 MUTANTS = {
     "ties_away_from_even": ("return (fmod(f, 2.0) == 0.0) ? f : f + 1.0;", "return f + 1.0;"),
@@ -59,6 +59,16 @@ MUTANTS = {
                                "y[t * H + i] = qzo_bf16_from_double(acc);"),
     "merge_no_max_shift": ("wsum += exp((double)lse[s * T + t] - m);", "wsum += exp((double)lse[s * T + t]);"),
     "merge_split_token_index": ("(double)O[(s * T + t) * H + i];", "(double)O[(t * S + s) * H + i];"),
+    "split_no_block_check": ("    if (cut % row_block != 0 && cut < rows) return -1;\n", ""),
+    "split_proportional_rule": ("    if (cut % row_block != 0 && cut < rows) return -1;\n",
+                                "    if (rows > 0 && (((rows + row_block - 1) / row_block) * cut) % rows != 0) return -1;\n"),
+    "split_second_part_offset": ("int64_t first[2] = {0, cut};", "int64_t first[2] = {0, cut - 1};"),
+    "split_padding_not_cleared": ("            sf_clear(so[p], count[p], kv, dst_layout);\n", ""),
+    "split_source_layout_ignored": ("= sf[sf_offset(src_layout, first[p] + r, k, kv)];",
+                                    "= sf[sf_offset(dst_layout, first[p] + r, k, kv)];"),
+    "split_amax_not_shared": ("if (amax_kind == 1) ao[p][0] = amax[0];",
+                              "if (amax_kind == 1 && p == 0) ao[p][0] = amax[0];"),
+    "split_block_scale_rows_floor": ("int64_t srows = (count[p] + 127) / 128;", "int64_t srows = count[p] / 128;"),
     "bf16_double_rounding": ("double n = round_half_even(a / step);\n    double r = n * step;",
                              "double n = round_half_even((double)(float)a / step);\n    double r = n * step;"),
 }
