@@ -73,6 +73,7 @@ KERNEL_SOURCES = {
     "dequant_kernel": ("qz_dequant.cu", "qz_device.cuh"),
     "attention_merge_kernel": ("qz_merge.cu", "qz_device.cuh"),
     "colwise_kernel": ("qz_colwise.cu", "qz_device.cuh"),
+    "split_fused_kernel": ("qz_split.cu", "qz_device.cuh"),
 }
 
 
@@ -432,8 +433,8 @@ class L2Flush:
         self.buf.zero_()
 
 
-def extra_workloads(qz, device, stream, peak, which=("split", "fused", "nvfp4", "large", "dequant", "merge", "colwise"),
-                    tokens=None):
+def extra_workloads(qz, device, stream, peak,
+                    which=("split", "fused", "nvfp4", "large", "dequant", "merge", "colwise", "gateup"), tokens=None):
     out = []
     flush = L2Flush(device)
 
@@ -458,6 +459,8 @@ def extra_workloads(qz, device, stream, peak, which=("split", "fused", "nvfp4", 
         _extra_merge(qz, device, flush, out, peak, tokens)
     if "colwise" in which:
         _extra_colwise(qz, device, rec)
+    if "gateup" in which:
+        _extra_gate_up_split(qz, device, rec)
     return out
 
 
@@ -601,6 +604,50 @@ def _extra_dequant(qz, device, rec):
     torch.cuda.empty_cache()
 
 
+def _extra_gate_up_split(qz, device, rec):
+    """Gate|up split of a folded Qwen3-30B-A3B gate_up projection (128 fused
+    experts of [1536, 2048], NVFP4 with a per-tensor amax, swizzled) at row
+    768; and the one-pass fold (gate and up quantized straight into their own
+    storage, sharing the expert's amax) against fold-then-split."""
+    cfg = synth.QWEN3_30B
+    rows, cols = cfg["gate_up"]
+    E, cut = cfg["experts"], rows // 2
+    swz, nv = qz.SF_SWIZZLED, qz.FMT_NVFP4
+    stack = synth.expert_stack(E, (rows, cols), cfg["std"], seed=cfg["seed"], device=device)
+    nsf, npart = qz.sf_bytes(rows, cols, nv, swz), qz.sf_bytes(cut, cols, nv, swz)
+    q = torch.empty((E, rows, cols // 2), dtype=torch.uint8, device=device)
+    sf = torch.empty((E, nsf), dtype=torch.uint8, device=device)
+    A = torch.empty((E, 1), dtype=torch.float32, device=device)
+    fold = qz.ExpertTable([qz.Entry(stack[e], q[e], sf[e], A[e]) for e in range(E)])
+    qz.quantize_grouped_nvfp4(fold, qz.NVFP4_PER_TENSOR_COMPUTE, swz)
+    qo = torch.empty((E, 2, cut, cols // 2), dtype=torch.uint8, device=device)
+    so = torch.empty((E, 2, npart), dtype=torch.uint8, device=device)
+    ao = torch.empty((E, 2, 1), dtype=torch.float32, device=device)
+    split = qz.SplitTable([qz.SplitEntry(q=q[e], sf=sf[e], rows=rows, cols=cols, cut=cut, sf_out=(so[e, 0], so[e, 1]),
+                                         q_out=(qo[e, 0], qo[e, 1]), amax=A[e], amax_out=(ao[e, 0], ao[e, 1]))
+                           for e in range(E)])
+
+    def split_call():
+        qz.split_fused_experts(split, nv, qz.AMAX_PER_TENSOR, swz, swz)
+
+    ms = _time_graph(split_call, reps=5)
+    nbytes = E * (2 * rows * (cols // 2) + nsf + 2 * npart + 3 * 4)
+    rec("gate|up split of a folded Qwen3-30B-A3B gate_up projection, 128 fused experts [1536, 2048] NVFP4 swizzled, "
+        "cut at row 768, one call", nbytes, ms, 1, kernel="split_fused_kernel", l2="inputs larger than L2",
+        traffic=ncu_traffic("split_fused_kernel"))
+    parts = qz.ExpertTable([qz.Entry(stack[e, p * cut:(p + 1) * cut], qo[e, p], so[e, p], A[e])
+                            for e in range(E) for p in range(2)])
+    ms_one = _time_graph(lambda: qz.quantize_grouped_nvfp4(parts, qz.NVFP4_PER_TENSOR_GIVEN, swz), reps=5)
+    ms_two = _time_graph(lambda: (qz.quantize_grouped_nvfp4(fold, qz.NVFP4_PER_TENSOR_GIVEN, swz), split_call()),
+                         reps=5)
+    qbytes = E * (rows * cols * 2 + rows * (cols // 2) + 2 * npart + 4)
+    rec("one-pass fold: Qwen3-30B-A3B gate_up [1536, 2048] x128 fused experts quantized to NVFP4 (given shared amax) "
+        "straight into separate gate and up storage", qbytes, ms_one, 1, kernel="nvfp4_tile_kernel",
+        fold_then_split_us=round(ms_two * 1e3, 2))
+    del stack, q, sf, qo, so, fold, split, parts
+    torch.cuda.empty_cache()
+
+
 def _extra_colwise(qz, device, rec):
     """Column-wise (transposed) quantization of a Qwen3-30B-A3B gate_up
     projection (128 experts of [1536, 2048]) to MXFP8 and to NVFP4 (given
@@ -732,7 +779,8 @@ def main():
     ap.add_argument("--no-extra", action="store_true", help="skip the other workloads")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
-    ap.add_argument("--only", choices=["split", "fused", "nvfp4", "large", "dequant", "merge", "colwise"], default=None,
+    ap.add_argument("--only", choices=["split", "fused", "nvfp4", "large", "dequant", "merge", "colwise", "gateup"],
+                    default=None,
                     help="time only this secondary workload and print its record (profiling aid)")
     ap.add_argument("--tokens", type=str, default=None,
                     help="comma-separated token counts for the fused sweep (default: 1..4096)")

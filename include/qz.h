@@ -70,8 +70,19 @@ typedef enum qz_sf_layout {
 
 typedef enum qz_format {
     QZ_FMT_MXFP8 = 0,
-    QZ_FMT_NVFP4 = 1
+    QZ_FMT_NVFP4 = 1,
+    QZ_FMT_FP8_BLOCK128 = 2 /* e4m3 payload with FP32 scales of 128 x 128 blocks, row-major
+                               [ceil(rows/128), ceil(cols/128)], linear only ([FOLD]: FP8 2-D
+                               blockwise experts).  Accepted by qz_sf_bytes and
+                               qz_split_fused_experts only; nothing here quantizes to it. */
 } qz_format;
+
+/* What a tensor's FP32 amax slot holds (qz_split_fused_experts). */
+typedef enum qz_amax_kind {
+    QZ_AMAX_NONE = 0,       /* no amax (MXFP8, FP8_BLOCK128) */
+    QZ_AMAX_PER_TENSOR = 1, /* one float per tensor (NVFP4 per-tensor scale) */
+    QZ_AMAX_PER_ROW = 2     /* one float per row (row-scaled NVFP4) */
+} qz_amax_kind;
 
 typedef enum qz_nvfp4_scale_mode {
     QZ_NVFP4_PER_TENSOR_GIVEN = 0,   /* amax[0] is an input (e.g. a calibrated value) */
@@ -89,6 +100,8 @@ typedef enum qz_nvfp4_scale_mode {
 #define QZ_DERR_TOO_LARGE 0x8u /* the call's total tile or row count exceeds 2^31 - 1 */
 #define QZ_DERR_TIMEOUT 0x10u  /* a wait for an asynchronous copy exceeded its time limit; the
                                   kernel stopped early (no such wait is expected to expire) */
+#define QZ_DERR_CUT 0x20u      /* qz_split_fused_experts: the cut falls inside a scale block
+                                  (FP8_BLOCK128: cut not a multiple of 128 and not the end) */
 
 /* Largest table a grouped call accepts (the kernels keep the table's prefix
  * sums in shared memory). */
@@ -142,6 +155,30 @@ typedef struct qz_dq_expert {
     int64_t ldy;        /* >= cols, multiple of 8, <= QZ_MAX_LD */
 } qz_dq_expert;
 
+/* One folded fused expert to cut in two (qz_split_fused_experts): part 0 is
+ * weight rows [0, cut) (the gate), part 1 rows [cut, rows) (the up
+ * projection).  Device memory, 96 bytes. */
+typedef struct qz_fused_split {
+    const void *q;       /* folded payload [rows, row_bytes], dense; row_bytes = cols (MXFP8,
+                            FP8_BLOCK128) or cols / 2 (NVFP4) */
+    const uint8_t *sf;   /* folded scales: the SF region of a [rows, cols] tensor in the call's
+                            src_layout (16-byte aligned when swizzled); FP8_BLOCK128: FP32
+                            [ceil(rows/128), ceil(cols/128)] row-major, 4-byte aligned */
+    const float *amax;   /* QZ_AMAX_PER_TENSOR: amax[0]; QZ_AMAX_PER_ROW: amax[rows]; 4-byte
+                            aligned; otherwise unused */
+    int64_t rows;        /* fused rows (gate + up), >= 0 */
+    int64_t cols;        /* multiple of 32 (MXFP8) / 16 (NVFP4), >= 1 (FP8_BLOCK128); <= QZ_MAX_LD */
+    int64_t cut;         /* first row of part 1, 0 <= cut <= rows */
+    void *q_out[2];      /* payload of each part [n_p, row_bytes], dense, any alignment (wider
+                            copies when 32/16/8-byte aligned); NULL: that part's payload is not
+                            copied (a caller keeping views into q) */
+    uint8_t *sf_out[2];  /* scales of each part: qz_sf_bytes(n_p, cols, fmt, dst_layout) bytes,
+                            padding written 0x00; 16-byte aligned when swizzled, 4-byte for
+                            FP8_BLOCK128 */
+    float *amax_out[2];  /* QZ_AMAX_PER_TENSOR: one float each, both receive amax[0];
+                            QZ_AMAX_PER_ROW: n_p floats each, the rows' amaxes */
+} qz_fused_split;
+
 /* Optional launch controls; pass NULL for the defaults. */
 typedef struct qz_launch_opts {
     unsigned int *d_err;    /* device word; kernels OR QZ_DERR_* bits into it (never clear it) */
@@ -162,7 +199,8 @@ size_t qz_workspace_bytes(int n_experts);
 
 /* Bytes of one expert's SF region: rows * (cols/block) for the linear layout,
  * pad(rows,128) * pad(cols/block,4) for the swizzled one, 0 when rows == 0.
- * fmt selects the block (32 for MXFP8, 16 for NVFP4).  Returns 0 for
+ * fmt selects the block (32 for MXFP8, 16 for NVFP4); QZ_FMT_FP8_BLOCK128
+ * (linear only) gives 4 * ceil(rows/128) * ceil(cols/128).  Returns 0 for
  * arguments that describe no valid region (negative sizes, cols not a
  * multiple of the block, unknown enums). */
 size_t qz_sf_bytes(int64_t rows, int64_t cols, int fmt, int layout);
@@ -283,6 +321,35 @@ qz_status qz_quantize_grouped_colwise(const qz_expert *d_table, int n_experts, i
 #define QZ_MAX_SPLITS 4096
 qz_status qz_attention_merge_quantize(const float *d_partial, const float *d_lse, int S, int64_t T, int64_t H,
                                       void *d_out, void *d_q, uint8_t *d_sf, int layout, void *stream);
+
+/* Gate|up split of folded fused experts (Model-Optimizer "Fold fused experts'
+ * quantizers into their weights shard-locally": a fused expert's (2I, H)
+ * weight is quantized as one tensor, gate and up sharing its per-tensor amax
+ * and so one weight_scale_2; the split then cuts the folded payload and its
+ * stacked scales by rows into gate and up, each in storage of its own, cuts a
+ * scale in proportion to the rows it covers and refuses a block scale that
+ * the cut would divide).  Per entry and part p (rows [first_p, first_p + n_p)):
+ *   payload: rows copied to q_out[p] (skipped when q_out[p] is NULL);
+ *   MXFP8 / NVFP4 scales: one scale row per weight row, so every cut is
+ *     exact; the part's SF region is written in dst_layout with its own
+ *     padding (0x00) from the source region in src_layout -- a swizzled
+ *     source cut inside a 128-row tile is re-laid, not refused;
+ *   FP8_BLOCK128 scales: whole scale rows copied; a cut that is not a
+ *     multiple of 128 and not the end divides a block: the entry is refused
+ *     (skipped, QZ_DERR_CUT);
+ *   amax: QZ_AMAX_PER_TENSOR gives amax[0] to both parts (one
+ *     weight_scale_2), QZ_AMAX_PER_ROW cuts it with the rows.
+ * Results equal quantizing each part's rows on their own (with the shared
+ * amax for a per-tensor scale).  One persistent launch, no allocation.
+ * Errors (before any launch): QZ_ERR_INVALID_ARG for n < 0 or > QZ_MAX_EXPERTS,
+ * a NULL table with n > 0, an unknown fmt, amax_kind or layout, an amax kind
+ * the format does not have (MXFP8 and FP8_BLOCK128 take QZ_AMAX_NONE only);
+ * QZ_ERR_UNSUPPORTED for FP8_BLOCK128 with a swizzled layout.  Invalid
+ * entries are skipped and reported through opts->d_err (QZ_DERR_SHAPE for
+ * bad sizes or a cut outside [0, rows], QZ_DERR_NULL, QZ_DERR_ALIGN,
+ * QZ_DERR_CUT). */
+qz_status qz_split_fused_experts(const qz_fused_split *d_table, int n, int fmt, int amax_kind, int src_layout,
+                                 int dst_layout, void *stream, const qz_launch_opts *opts);
 
 /* Largest table of qz_quantize_grouped_nvfp4_compute_noalloc. */
 #define QZ_STATIC_WS_MAX_EXPERTS 1024

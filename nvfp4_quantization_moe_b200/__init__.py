@@ -7,12 +7,14 @@ There is no CPU or library fallback: every call raises if the library is
 missing or reports an error.
 """
 from .binding import (  # noqa: F401
-    STATIC_WS_MAX_EXPERTS,
-    DERR_ALIGN, DERR_NULL, DERR_SHAPE, DERR_TOO_LARGE, EXPORTED, FMT_MXFP8, FMT_NVFP4, LIB_PATH, MAX_EXPERTS,
-    MAX_HIDDEN, NVFP4_PER_ROW, NVFP4_PER_TENSOR_COMPUTE, NVFP4_PER_TENSOR_GIVEN, QZ_ERR_ALIGNMENT, QZ_ERR_CUDA,
-    QZ_ERR_INVALID_ARG, QZ_ERR_UNSUPPORTED, QZ_OK, SF_LINEAR, SF_SWIZZLED, DqEntry, DqTable, Entry, ExpertTable,
-    QzError, SfPairTable, alloc_outputs, attention_merge_quantize, dequantize_grouped, quantize_grouped_colwise, alloc_workspace, load, quantize_experts, quantize_grouped_mxfp8,
-    quantize_grouped_nvfp4, quantize_grouped_nvfp4_compute_noalloc, rmsnorm_quantize, sf_bytes, status_string, swizzle_scales, workspace_bytes,
+    AMAX_NONE, AMAX_PER_ROW, AMAX_PER_TENSOR, DERR_ALIGN, DERR_CUT, DERR_NULL, DERR_SHAPE, DERR_TOO_LARGE, EXPORTED,
+    FMT_FP8_BLOCK128, FMT_MXFP8, FMT_NVFP4, LIB_PATH, MAX_EXPERTS, MAX_HIDDEN, NVFP4_PER_ROW,
+    NVFP4_PER_TENSOR_COMPUTE, NVFP4_PER_TENSOR_GIVEN, QZ_ERR_ALIGNMENT, QZ_ERR_CUDA, QZ_ERR_INVALID_ARG,
+    QZ_ERR_UNSUPPORTED, QZ_OK, SF_LINEAR, SF_SWIZZLED, STATIC_WS_MAX_EXPERTS, DqEntry, DqTable, Entry, ExpertTable,
+    QzError, SfPairTable, SplitEntry, SplitTable, alloc_outputs, alloc_workspace, attention_merge_quantize,
+    dequantize_grouped, load, quantize_experts, quantize_grouped_colwise, quantize_grouped_mxfp8,
+    quantize_grouped_nvfp4, quantize_grouped_nvfp4_compute_noalloc, rmsnorm_quantize, sf_bytes,
+    split_fused_experts, status_string, swizzle_scales, workspace_bytes,
 )
 
 __version__ = "0.1.0"

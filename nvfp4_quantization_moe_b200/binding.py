@@ -23,9 +23,11 @@ LIB_PATH = os.path.join(_HERE, "libqz.so")
 # enums of include/qz.h
 QZ_OK, QZ_ERR_INVALID_ARG, QZ_ERR_ALIGNMENT, QZ_ERR_UNSUPPORTED, QZ_ERR_CUDA = range(5)
 SF_LINEAR, SF_SWIZZLED = 0, 1
-FMT_MXFP8, FMT_NVFP4 = 0, 1
+FMT_MXFP8, FMT_NVFP4, FMT_FP8_BLOCK128 = 0, 1, 2
 NVFP4_PER_TENSOR_GIVEN, NVFP4_PER_TENSOR_COMPUTE, NVFP4_PER_ROW = 0, 1, 2
+AMAX_NONE, AMAX_PER_TENSOR, AMAX_PER_ROW = 0, 1, 2
 DERR_SHAPE, DERR_NULL, DERR_ALIGN, DERR_TOO_LARGE = 0x1, 0x2, 0x4, 0x8
+DERR_CUT = 0x20
 MAX_EXPERTS = 4096
 MAX_HIDDEN = 16384
 
@@ -42,6 +44,7 @@ EXPORTED = (
     "qz_dequantize_grouped",
     "qz_attention_merge_quantize",
     "qz_quantize_grouped_colwise",
+    "qz_split_fused_experts",
 )
 STATIC_WS_MAX_EXPERTS = 1024
 
@@ -69,12 +72,19 @@ class _SfPair(ctypes.Structure):
                 ("kv", ctypes.c_int64)]
 
 
+class _FusedSplit(ctypes.Structure):
+    _fields_ = [("q", ctypes.c_void_p), ("sf", ctypes.c_void_p), ("amax", ctypes.c_void_p),
+                ("rows", ctypes.c_int64), ("cols", ctypes.c_int64), ("cut", ctypes.c_int64),
+                ("q_out", ctypes.c_void_p * 2), ("sf_out", ctypes.c_void_p * 2), ("amax_out", ctypes.c_void_p * 2)]
+
+
 class _Opts(ctypes.Structure):
     _fields_ = [("d_err", ctypes.c_void_p), ("max_ctas", ctypes.c_int), ("d_workspace", ctypes.c_void_p),
                 ("workspace_bytes", ctypes.c_size_t)]
 
 
 assert ctypes.sizeof(_Expert) == 56 and ctypes.sizeof(_SfPair) == 32 and ctypes.sizeof(_DqExpert) == 56
+assert ctypes.sizeof(_FusedSplit) == 96
 
 _lock = threading.Lock()
 _lib = None
@@ -115,6 +125,8 @@ def load(path: str = LIB_PATH):
         lib.qz_quantize_grouped_colwise.argtypes = [P, I, I, I, P, P]
         lib.qz_attention_merge_quantize.restype = I
         lib.qz_attention_merge_quantize.argtypes = [P, P, I, i64, i64, P, P, P, I, P]
+        lib.qz_split_fused_experts.restype = I
+        lib.qz_split_fused_experts.argtypes = [P, I, I, I, I, I, P, P]
         _lib = lib
         return lib
 
@@ -262,6 +274,57 @@ class DqTable:
         return self
 
 
+@dataclass
+class SplitEntry:
+    """One folded fused expert to cut at row ``cut``: its payload q (rows
+    [rows, row_bytes]), scales sf, amax, and each part's outputs.  q_out[p] may
+    be None (that part's payload is not copied)."""
+    q: torch.Tensor
+    sf: torch.Tensor
+    rows: int
+    cols: int
+    cut: int
+    sf_out: tuple
+    q_out: tuple = (None, None)
+    amax: Optional[torch.Tensor] = None
+    amax_out: tuple = (None, None)
+
+
+class SplitTable:
+    """A device-resident array of qz_fused_split entries (keeps its tensors alive)."""
+
+    def __init__(self, entries: Sequence[SplitEntry], device=None):
+        self.entries = list(entries)
+        n = len(self.entries)
+        arr = (_FusedSplit * max(n, 1))()
+        P2 = ctypes.c_void_p * 2
+        for i, e in enumerate(self.entries):
+            arr[i] = _FusedSplit(_ptr(e.q), _ptr(e.sf), _ptr(e.amax), int(e.rows), int(e.cols), int(e.cut),
+                                 P2(*[_ptr(t) for t in e.q_out]), P2(*[_ptr(t) for t in e.sf_out]),
+                                 P2(*[_ptr(t) for t in e.amax_out]))
+        host = torch.frombuffer(bytearray(bytes(arr)), dtype=torch.uint8)
+        dev = device if device is not None else (self.entries[0].q.device if n else torch.device("cuda"))
+        self.dev = host.to(dev)
+        self.n = n
+
+    @property
+    def ptr(self) -> int:
+        return int(self.dev.data_ptr()) if self.n else 0
+
+    @classmethod
+    def from_raw(cls, raw: Iterable[tuple], device) -> "SplitTable":
+        """Entries from raw (q, sf, amax, rows, cols, cut, (q0, q1), (sf0, sf1), (a0, a1)) tuples of
+        integers (tests use this to build deliberately invalid entries)."""
+        self = cls.__new__(cls)
+        raw = list(raw)
+        P2 = ctypes.c_void_p * 2
+        arr = (_FusedSplit * max(len(raw), 1))(*[_FusedSplit(*r[:6], P2(*r[6]), P2(*r[7]), P2(*r[8])) for r in raw])
+        self.entries = []
+        self.n = len(raw)
+        self.dev = torch.frombuffer(bytearray(bytes(arr)), dtype=torch.uint8).to(device)
+        return self
+
+
 class SfPairTable:
     def __init__(self, pairs: Sequence[tuple], device):
         """pairs: (src linear uint8 tensor, dst swizzled uint8 tensor, rows, kv)."""
@@ -332,6 +395,15 @@ def attention_merge_quantize(partial, lse, out, q=None, sf=None, layout: int = S
                                               int(T), int(H), ctypes.c_void_p(_ptr(out)), ctypes.c_void_p(_ptr(q)),
                                               ctypes.c_void_p(_ptr(sf)), int(layout), _stream_ptr(stream)),
            "qz_attention_merge_quantize")
+
+
+def split_fused_experts(table: SplitTable, fmt: int, amax_kind: int, src_layout: int, dst_layout: int, stream=None,
+                        err=None, max_ctas: int = 0):
+    """Cut folded fused experts into gate (rows [0, cut)) and up (rows [cut, rows)):
+    payload rows, scales re-laid per part in dst_layout, amax shared or cut."""
+    _check(load().qz_split_fused_experts(ctypes.c_void_p(table.ptr), table.n, int(fmt), int(amax_kind),
+                                         int(src_layout), int(dst_layout), _stream_ptr(stream), _opts(err, max_ctas)),
+           "qz_split_fused_experts")
 
 
 def swizzle_scales(table: SfPairTable, stream=None, err=None, max_ctas: int = 0):

@@ -32,6 +32,9 @@ int dequant_blocks_per_sm(int n);
 cudaError_t launch_colwise(const qz_expert* table, int n, int fmt, int layout, int grid, cudaStream_t s,
                            unsigned* d_err);
 int colwise_blocks_per_sm(int n);
+cudaError_t launch_split_fused(const qz_fused_split* table, int n, int fmt, int amax_kind, int src_layout,
+                               int dst_layout, int grid, cudaStream_t s, unsigned* d_err);
+int split_blocks_per_sm(int n);
 cudaError_t launch_attention_merge(const float* O, const float* lse, int S, int64_t T, int64_t H, uint16_t* y,
                                    uint8_t* q, uint8_t* sf, int layout, cudaStream_t s);
 }  // namespace qz
@@ -39,11 +42,12 @@ cudaError_t launch_attention_merge(const float* O, const float* lse, int S, int6
 namespace {
 
 constexpr int kMaxDevices = 64;
-constexpr int kKinds = 8;  // mxfp8, nvfp4 tile, swizzle, amax, rows, computed-amax L2 path, dequantize, colwise
+constexpr int kKinds = 9;  // mxfp8, nvfp4 tile, swizzle, amax, rows, computed-amax L2 path, dequantize, colwise,
+                           // fused split
 
 struct DeviceLimits {
     int sms = 0;
-    int per_sm[kKinds] = {0, 0, 0, 0, 0, 0, 0, 0};
+    int per_sm[kKinds] = {0, 0, 0, 0, 0, 0, 0, 0, 0};
 };
 
 std::mutex g_mu;
@@ -68,6 +72,7 @@ int wave_grid(int kind, const qz_launch_opts* opts) {
             d.per_sm[kind] = (kind == 4)   ? qz::rows_blocks_per_sm(QZ_MAX_EXPERTS)
                              : (kind == 6) ? qz::dequant_blocks_per_sm(QZ_MAX_EXPERTS)
                              : (kind == 7) ? qz::colwise_blocks_per_sm(QZ_MAX_EXPERTS)
+                             : (kind == 8) ? qz::split_blocks_per_sm(QZ_MAX_EXPERTS)
                                            : qz::grouped_blocks_per_sm(kind, QZ_MAX_EXPERTS);
         grid = d.sms * d.per_sm[kind];
     }
@@ -108,6 +113,10 @@ qz_status from_cuda(cudaError_t e) { return e == cudaSuccess ? QZ_OK : QZ_ERR_CU
 extern "C" {
 
 size_t qz_sf_bytes(int64_t rows, int64_t cols, int fmt, int layout) {
+    if (fmt == QZ_FMT_FP8_BLOCK128) {
+        if (layout != QZ_SF_LINEAR || rows <= 0 || cols <= 0) return 0;
+        return (size_t)(4 * ((rows + 127) / 128) * ((cols + 127) / 128));
+    }
     if (fmt != QZ_FMT_MXFP8 && fmt != QZ_FMT_NVFP4) return 0;
     if (!valid_layout(layout)) return 0;
     const int64_t block = fmt == QZ_FMT_MXFP8 ? 32 : 16;
@@ -225,6 +234,22 @@ qz_status qz_attention_merge_quantize(const float* d_partial, const float* d_lse
     if (d_q && (!aligned(d_q, 8) || (layout == QZ_SF_SWIZZLED_128x4 && !aligned(d_sf, 16)))) return QZ_ERR_ALIGNMENT;
     return from_cuda(qz::launch_attention_merge(d_partial, d_lse, S, T, H, static_cast<uint16_t*>(d_out),
                                                 static_cast<uint8_t*>(d_q), d_sf, layout, (cudaStream_t)stream));
+}
+
+qz_status qz_split_fused_experts(const qz_fused_split* d_table, int n, int fmt, int amax_kind, int src_layout,
+                                 int dst_layout, void* stream, const qz_launch_opts* opts) {
+    qz_status st = check_table(d_table, n);
+    if (st != QZ_OK) return st;
+    if (fmt != QZ_FMT_MXFP8 && fmt != QZ_FMT_NVFP4 && fmt != QZ_FMT_FP8_BLOCK128) return QZ_ERR_INVALID_ARG;
+    if (amax_kind != QZ_AMAX_NONE && amax_kind != QZ_AMAX_PER_TENSOR && amax_kind != QZ_AMAX_PER_ROW)
+        return QZ_ERR_INVALID_ARG;
+    if (fmt != QZ_FMT_NVFP4 && amax_kind != QZ_AMAX_NONE) return QZ_ERR_INVALID_ARG;
+    if (!valid_layout(src_layout) || !valid_layout(dst_layout)) return QZ_ERR_INVALID_ARG;
+    if (fmt == QZ_FMT_FP8_BLOCK128 && (src_layout != QZ_SF_LINEAR || dst_layout != QZ_SF_LINEAR))
+        return QZ_ERR_UNSUPPORTED;
+    if (n == 0) return QZ_OK;
+    return from_cuda(qz::launch_split_fused(d_table, n, fmt, amax_kind, src_layout, dst_layout, wave_grid(8, opts),
+                                            (cudaStream_t)stream, err_word(opts)));
 }
 
 size_t qz_workspace_bytes(int n_experts) {

@@ -85,6 +85,21 @@ def test_host_errors_without_gpu(lib):
     assert lib.qz_quantize_grouped_colwise(P(0x1000), 1, 3, 0, None, None) == qz.QZ_ERR_INVALID_ARG
     assert lib.qz_quantize_grouped_colwise(P(0x1000), 1, 0, 4, None, None) == qz.QZ_ERR_INVALID_ARG
     assert lib.qz_quantize_grouped_colwise(None, 0, 1, 1, None, None) == qz.QZ_OK
+
+    def split(n=2, fmt=1, amax=1, src=1, dst=1, table=P(0x1000)):
+        return lib.qz_split_fused_experts(table, n, fmt, amax, src, dst, None, None)
+
+    assert split(n=-1) == qz.QZ_ERR_INVALID_ARG
+    assert split(table=None) == qz.QZ_ERR_INVALID_ARG
+    assert split(fmt=3) == qz.QZ_ERR_INVALID_ARG
+    assert split(amax=3) == qz.QZ_ERR_INVALID_ARG
+    assert split(fmt=0, amax=1) == qz.QZ_ERR_INVALID_ARG            # MXFP8 has no amax
+    assert split(fmt=2, amax=2) == qz.QZ_ERR_INVALID_ARG            # nor FP8 with 128 x 128 block scales
+    assert split(src=2) == qz.QZ_ERR_INVALID_ARG
+    assert split(fmt=2, amax=0, src=0, dst=1) == qz.QZ_ERR_UNSUPPORTED   # FP32 block scales are linear only
+    assert split(n=0, table=None) == qz.QZ_OK
+    assert qz.sf_bytes(300, 200, qz.FMT_FP8_BLOCK128, qz.SF_LINEAR) == 4 * 3 * 2
+    assert qz.sf_bytes(300, 200, qz.FMT_FP8_BLOCK128, qz.SF_SWIZZLED) == 0
     a16 = P(0x10000)
 
     def merge(S=4, T=3, H=1024, O=a16, lse=a16, y=a16, q=a16, sf=a16, layout=1):
