@@ -226,6 +226,14 @@ qz_status qz_quantize_grouped_mxfp8(const qz_expert *d_table, int n_experts, int
  * HBM); with opts->d_workspace it runs one launch that takes each expert's
  * amax chunk by chunk and quantizes the chunk while its input is still in L2
  * (plus a memset of the workspace).  PER_ROW reads each row once.
+ * Entries may share one amax slot, so that the gate and up halves of a fused
+ * expert ([FOLD]: one amax over the fused (2I, H) slice, one weight_scale_2)
+ * are quantized straight into their own storage in one call: in GIVEN mode
+ * the shared value is read by both, and in COMPUTE mode without a workspace
+ * every entry sharing the slot feeds the same maximum before any of them is
+ * quantized.  The single-launch COMPUTE path (with opts->d_workspace, and
+ * qz_quantize_grouped_nvfp4_compute_noalloc) keeps one amax per entry: there
+ * entries must not share a slot.
  * Errors as below, plus QZ_ERR_INVALID_ARG for a workspace smaller than
  * qz_workspace_bytes(n_experts) and QZ_ERR_ALIGNMENT for one not 4-byte
  * aligned.
