@@ -8,16 +8,17 @@
 // factors those of a [cols, rows] matrix in the linear or swizzled 128x4
 // layout, padding written as 0x00 by the kernel.
 //
-// One persistent launch walks all experts' 128 x 128 tiles.  A CTA loads a
-// tile with coalesced 16-byte loads (the next tile's loads fly while the
-// current one is quantized), pairs the elements of two consecutive rows into
-// one 32-bit word per column and writes the tile transposed into
-// shared memory (XOR-swizzled so that both the scattered writes and the
-// 16-byte row reads stay nearly conflict-free); then each thread quantizes
-// 64 consecutive elements of one transposed row with the library's block
-// quantizers (include/qz_quant.cuh) and writes them to the transposed
-// payload.  NVFP4 takes the tensor amax as given (the row-wise computed-amax
-// call of the same tensor produces it).
+// One persistent launch walks all experts' 128 x 128 tiles.  Each CTA keeps
+// three tiles in flight: asynchronous 16-byte copies (cp.async, zero-filled
+// past the matrix) bring a tile row-major into one of three shared-memory
+// stages while the tile before it is quantized, so the loads never wait on
+// the arithmetic and one CTA barrier per tile suffices.  A thread reads one
+// 32-bit word per row -- two neighbouring columns -- for 32 rows, pairs
+// consecutive rows of each column into bf16x2 words, quantizes the two
+// 32-element column segments with the library's block quantizers
+// (include/qz_quant.cuh) and writes them to the transposed payload.  NVFP4
+// takes the tensor amax as given (the row-wise computed-amax call of the
+// same tensor produces it).
 #include "../../include/qz_quant.cuh"
 
 namespace qz {
@@ -58,20 +59,7 @@ struct ColTiles {
     }
 };
 
-// Word index of (tile column cl, row pair rp) in the transposed shared tile:
-// 64 words (128 rows) per column, row pairs XOR-swizzled by
-// ((cl ^ cl / 8) mod 8) in bits 2-4.  The load phase writes 16 columns
-// 8 apart at a time and the quantize phase reads 8 consecutive columns at a
-// time; both see 8 different swizzles, so writes are at most 2-way and the
-// 16-byte reads conflict-free.  Bits 0-1 are untouched: 4 consecutive row
-// pairs from a multiple of 4 stay one aligned 16-byte chunk.
-__device__ __forceinline__ int col_word(int cl, int rp) { return cl * 64 + (rp ^ (((cl ^ (cl >> 3)) & 7) << 2)); }
-
-// One thread's share of a tile: 16 bf16 pairs (rows r0, r0 + 1 of 8 columns, 4 row pairs).
-struct ColLoad {
-    uint4 a[4], b[4];
-};
-
+// The tile a CTA works on: tile `tile` of the call, found from expert `e` on.
 struct ColRef {
     const uint16_t* x;
     int64_t R, C, ld;
@@ -95,114 +83,125 @@ __device__ __forceinline__ ColRef col_ref(const qz_expert* table, const int* s_p
     return r;
 }
 
-// Thread t's loads of a tile: 8 columns (chunk t % 16) of row pairs t / 16 + 16 k.
-__device__ __forceinline__ void col_load(const ColRef& r, int t, ColLoad& v) {
-    const int cc = t & 15;
-    const int64_t c = (int64_t)r.ct * kTileCols + 8 * cc;
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-        const int rp = (t >> 4) + 16 * k;
-        const int64_t r0 = (int64_t)r.rt * kTileRows + 2 * rp;
-        v.a[k] = make_uint4(0, 0, 0, 0);
-        v.b[k] = make_uint4(0, 0, 0, 0);
-        if (c < r.C) {
-            if (c + 8 <= r.C) {
-                if (r0 < r.R) v.a[k] = ld_stream(r.x + r0 * r.ld + c);
-                if (r0 + 1 < r.R) v.b[k] = ld_stream(r.x + (r0 + 1) * r.ld + c);
-            } else {  // a partial chunk at the end of a row, element by element
-                uint16_t* ah = reinterpret_cast<uint16_t*>(&v.a[k]);
-                uint16_t* bh = reinterpret_cast<uint16_t*>(&v.b[k]);
-                for (int j = 0; j < 8 && c + j < r.C; ++j) {
-                    if (r0 < r.R) ah[j] = r.x[r0 * r.ld + c + j];
-                    if (r0 + 1 < r.R) bh[j] = r.x[(r0 + 1) * r.ld + c + j];
-                }
-            }
-        }
-    }
+// ---------------------------------------------------------------------------
+// asynchronous global -> shared copies (cp.async, 16 bytes, zero-filled past
+// src_bytes); each thread waits for its own groups, a CTA barrier publishes
+// them to the other threads
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src, int src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
-// Write thread t's share into the transposed shared tile (one word per column and row pair).
-__device__ __forceinline__ void col_store_smem(uint32_t* s_t, int t, const ColLoad& v) {
+constexpr int kColStages = 3;                                     // tiles in flight per CTA
+constexpr int kColStageBytes = kTileRows * kTileCols * 2;         // one bf16 tile, row-major (32 KB)
+
+// Issue thread t's copies of a tile into a stage: chunk t % 16 (8 columns)
+// of rows t / 16 + 16 k.  Rows past the matrix and columns past its last one
+// are zero-filled without reading.
+__device__ __forceinline__ void col_issue(const ColRef& r, uint32_t stage, int t) {
     const int cc = t & 15;
+    const int64_t c = (int64_t)r.ct * kTileCols + 8 * cc;
+    const int64_t cols_left = r.C - c;
+    const int cbytes = cols_left >= 8 ? 16 : (cols_left > 0 ? (int)cols_left * 2 : 0);
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-        const int rp = (t >> 4) + 16 * k;
-        const uint32_t aw[4] = {v.a[k].x, v.a[k].y, v.a[k].z, v.a[k].w};
-        const uint32_t bw[4] = {v.b[k].x, v.b[k].y, v.b[k].z, v.b[k].w};
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const int cl = 8 * cc + 2 * j;
-            s_t[col_word(cl, rp)] = __byte_perm(aw[j], bw[j], 0x5410);      // (row r0, row r0 + 1) of column cl
-            s_t[col_word(cl + 1, rp)] = __byte_perm(aw[j], bw[j], 0x7632);  // the same of column cl + 1
-        }
+    for (int k = 0; k < 8; ++k) {
+        const int row = (t >> 4) + 16 * k;
+        const int64_t rg = (int64_t)r.rt * kTileRows + row;
+        const bool in = rg < r.R && cbytes > 0;
+        const void* src = in ? static_cast<const void*>(r.x + rg * r.ld + c) : static_cast<const void*>(r.x);
+        cp_async_16(stage + (uint32_t)(row * (kTileCols * 2) + 16 * cc), src, in ? cbytes : 0);
     }
 }
 
 template <int FMT, int LAYOUT>
-__global__ void __launch_bounds__(kColThreads, 3) colwise_kernel(const qz_expert* __restrict__ table, int n,
+__global__ void __launch_bounds__(kColThreads, 2) colwise_kernel(const qz_expert* __restrict__ table, int n,
                                                                  unsigned* d_err) {
     constexpr int kBlock = FMT == QZ_FMT_MXFP8 ? 32 : 16;
-    extern __shared__ int s_prefix[];
+    extern __shared__ __align__(16) int s_prefix[];  // [n + 1] prefix, then the stages (16-byte aligned)
     __shared__ long long s_scan[33];
-    __shared__ __align__(16) uint32_t s_t[kTileCols * 64];  // the tile transposed: [column][row pair]
     __shared__ float s_inv[16];
     if (FMT == QZ_FMT_NVFP4) fill_inv_table(s_inv);  // published by the barriers in block_prefix
     const int total = block_prefix(n, s_prefix, s_scan, ColTiles<FMT, LAYOUT>{table, d_err}, d_err);
     const int t = threadIdx.x;
-    int tile = blockIdx.x;
-    if (tile >= total) return;
-    ColRef cur = col_ref(table, s_prefix, tile, 0);
-    ColLoad v;
-    col_load(cur, t, v);
-    for (;;) {
-        col_store_smem(s_t, t, v);
-        __syncthreads();
-        const int next = tile + gridDim.x;
-        const bool more = next < total;
-        const ColRef nxt = more ? col_ref(table, s_prefix, next, cur.expert) : cur;
-        if (more) col_load(nxt, t, v);  // the next tile's loads fly while this one is quantized
+    if ((int)blockIdx.x >= total) return;
+    const uint32_t stages = (uint32_t)__cvta_generic_to_shared(s_prefix + ((n + 4) & ~3));
+    const uint32_t* s_words = reinterpret_cast<const uint32_t*>(s_prefix + ((n + 4) & ~3));
+
+    // prologue: the first kColStages - 1 tiles of this CTA in flight
+    int e_issue = 0, e_cur = 0;  // expert hints of the issuing and the consuming walk
+#pragma unroll
+    for (int s = 0; s < kColStages - 1; ++s) {
+        const int tile = blockIdx.x + s * gridDim.x;
+        if (tile < total) {
+            const ColRef r = col_ref(table, s_prefix, tile, e_issue);
+            e_issue = r.expert;
+            col_issue(r, stages + s * kColStageBytes, t);
+        }
+        cp_async_commit();
+    }
+    const int w = t >> 5, lane = t & 31;
+    const int ch = w & 1, rs = w >> 1;  // this warp's column half and 32-row segment of a tile
+    for (int k = 0;; ++k) {
+        const int tile = blockIdx.x + k * gridDim.x;
+        if (tile >= total) break;
+        const int cur_s = k % kColStages;
+        cp_async_wait<kColStages - 2>();  // this thread's copies of tile k have landed
+        __syncthreads();                  // ... and everyone's; tile k - 1's stage is free again
+        {
+            const int ahead = tile + (kColStages - 1) * gridDim.x;
+            const int s = (k + kColStages - 1) % kColStages;
+            if (ahead < total) {
+                const ColRef r = col_ref(table, s_prefix, ahead, e_issue);
+                e_issue = r.expert;
+                col_issue(r, stages + s * kColStageBytes, t);
+            }
+            cp_async_commit();
+        }
+        const ColRef cur = col_ref(table, s_prefix, tile, e_cur);
+        e_cur = cur.expert;
         const qz_expert E = load_entry(table, cur.expert);
         const int64_t R = cur.R, C = cur.C;
-        // ---- quantize: thread t takes rows 64 h .. 64 h + 63 of tile column t % 128
-        const int cl = t & 127, h = t >> 7;
-        const int64_t cg = (int64_t)cur.ct * kTileCols + cl;  // x column = transposed row
-        const int64_t cpad = LAYOUT == QZ_SF_SWIZZLED_128x4 ? ((C + 127) & ~(int64_t)127) : C;
-        const int64_t kvT = R / kBlock;                       // scale columns of the transposed matrix
-        const int64_t kvs = LAYOUT == QZ_SF_SWIZZLED_128x4 ? ((kvT + 3) & ~(int64_t)3) : kvT;
-        const int64_t e0 = (int64_t)cur.rt * kTileRows + 64 * h;  // first transposed column (x row) of the segment
-        // NVFP4: lanes 1..15 hold RN(S / m) for the tile's expert (every lane takes part in the shuffles)
-        const float qm = FMT == QZ_FMT_NVFP4 ? rcp_lane_quotient(nvfp4_encode_scale(__ldg(E.amax)), s_inv, t & 31) : 0.0f;
-        // every thread decodes its segment (columns past the matrix hold zeros), so
-        // that the NVFP4 shuffles see the whole warp; only the stores are guarded
-        const bool inreg = cg < cpad;  // a row of the transposed SF region
-        const bool live = cg < C;      // a row of the transposed payload
-        uint32_t w[32];
+        // ---- thread (warp w, lane l) quantizes tile columns 64 ch + 2 l and + 1,
+        //      rows 32 rs .. 32 rs + 31 of each: one word per row holds both columns
+        const uint32_t* tw = s_words + cur_s * (kColStageBytes / 4) + (32 * rs) * (kTileCols / 2) + 32 * ch + lane;
+        uint32_t xa[16], xb[16];  // column pairs (row 2i low, row 2i + 1 high) of the two columns
 #pragma unroll
-        for (int m = 0; m < 8; ++m) {
-            const uint4 u = *reinterpret_cast<const uint4*>(&s_t[col_word(cl, 32 * h + 4 * m)]);
-            w[4 * m] = u.x;
-            w[4 * m + 1] = u.y;
-            w[4 * m + 2] = u.z;
-            w[4 * m + 3] = u.w;
+        for (int i = 0; i < 16; ++i) {
+            const uint32_t r0 = tw[(2 * i) * (kTileCols / 2)], r1 = tw[(2 * i + 1) * (kTileCols / 2)];
+            xa[i] = __byte_perm(r0, r1, 0x5410);
+            xb[i] = __byte_perm(r0, r1, 0x7632);
         }
-        constexpr int kBlocks = 64 / kBlock;
-        uint32_t scales[kBlocks];
+        const int64_t cg = (int64_t)cur.ct * kTileCols + 64 * ch + 2 * lane;  // x column = transposed row
+        const int64_t e0 = (int64_t)cur.rt * kTileRows + 32 * rs;             // first x row of the segment
+        const int64_t cpad = LAYOUT == QZ_SF_SWIZZLED_128x4 ? ((C + 127) & ~(int64_t)127) : C;
+        const int64_t kvT = R / kBlock;  // scale columns of the transposed matrix
+        const int64_t kvs = LAYOUT == QZ_SF_SWIZZLED_128x4 ? ((kvT + 3) & ~(int64_t)3) : kvT;
+        const int64_t k0 = e0 / kBlock;  // the segment's first scale column
+        constexpr int kSeg = 32 / kBlock;  // scale blocks per column segment: 1 / 2
+        uint32_t sc[2][kSeg];
         if (FMT == QZ_FMT_MXFP8) {
-            uint8_t* qrow = static_cast<uint8_t*>(E.q) + cg * R + e0;
-            const bool q32 = ((reinterpret_cast<uintptr_t>(E.q) & 31) == 0);
+            uint32_t qa[8], qb[8];
+            sc[0][0] = qzq::mxfp8_block(xa, qa);
+            sc[1][0] = qzq::mxfp8_block(xb, qb);
+            if (e0 < R) {
+                const bool q32 = ((reinterpret_cast<uintptr_t>(E.q) & 31) == 0);
 #pragma unroll
-            for (int i = 0; i < kBlocks; ++i) {
-                uint32_t x[16], q[8];
-#pragma unroll
-                for (int j = 0; j < 16; ++j) x[j] = w[16 * i + j];
-                scales[i] = qzq::mxfp8_block(x, q);
-                if (live && e0 + 32 * i < R) {
-                    const uint4 lo = make_uint4(q[0], q[1], q[2], q[3]), hi = make_uint4(q[4], q[5], q[6], q[7]);
+                for (int j = 0; j < 2; ++j) {
+                    if (cg + j >= C) continue;
+                    const uint32_t* qq = j ? qb : qa;
+                    uint8_t* dst = static_cast<uint8_t*>(E.q) + (cg + j) * R + e0;
+                    const uint4 lo = make_uint4(qq[0], qq[1], qq[2], qq[3]), hi = make_uint4(qq[4], qq[5], qq[6], qq[7]);
                     if (q32) {
-                        st_v8(qrow + 32 * i, lo, hi);
+                        st_v8(dst, lo, hi);
                     } else {
-                        st_v4(qrow + 32 * i, lo);
-                        st_v4(qrow + 32 * i + 16, hi);
+                        st_v4(dst, lo);
+                        st_v4(dst + 16, hi);
                     }
                 }
             }
@@ -210,64 +209,51 @@ __global__ void __launch_bounds__(kColThreads, 3) colwise_kernel(const qz_expert
             // the tile kernels' NVFP4 arithmetic (same bytes as qzq::nvfp4_block): block
             // scales two at a time, element multipliers from 16 per-tile quotients
             const float S = nvfp4_encode_scale(__ldg(E.amax));
-            uint8_t* qrow = static_cast<uint8_t*>(E.q) + cg * (R >> 1) + (e0 >> 1);
+            const float qm = rcp_lane_quotient(S, s_inv, lane);  // every lane: the shuffles below need all
+            uint32_t c[2][4];
 #pragma unroll
-            for (int i = 0; i < kBlocks; i += 2) {
-                const uint32_t two = tile_scales_nv_words(w + 8 * i, w + 8 * i + 8, S);
-                scales[i] = two & 0xFFu;
-                scales[i + 1] = two >> 8;
+            for (int j = 0; j < 2; ++j) {
+                const uint32_t* xx = j ? xb : xa;
+                const uint32_t two = tile_scales_nv_words(xx, xx + 8, S);
+                sc[j][0] = two & 0xFFu;
+                sc[j][1] = two >> 8;
+#pragma unroll
+                for (int b = 0; b < 2; ++b) {
+                    const float rcp = nvfp4_rcp_warp(qm, sc[j][b]);
+                    c[j][2 * b] = e2m1x8_words(xx[8 * b], xx[8 * b + 1], xx[8 * b + 2], xx[8 * b + 3], rcp);
+                    c[j][2 * b + 1] = e2m1x8_words(xx[8 * b + 4], xx[8 * b + 5], xx[8 * b + 6], xx[8 * b + 7], rcp);
+                }
             }
-            uint32_t c[2 * kBlocks];
 #pragma unroll
-            for (int i = 0; i < kBlocks; ++i) {
-                const float rcp = nvfp4_rcp_warp(qm, scales[i]);  // all lanes
-                c[2 * i] = e2m1x8_words(w[8 * i], w[8 * i + 1], w[8 * i + 2], w[8 * i + 3], rcp);
-                c[2 * i + 1] = e2m1x8_words(w[8 * i + 4], w[8 * i + 5], w[8 * i + 6], w[8 * i + 7], rcp);
-            }
-            // the segment's 32 payload bytes: one 32-byte store when the row is 32-byte aligned
-            const uintptr_t qa = reinterpret_cast<uintptr_t>(qrow);
-            if (live && e0 + 64 <= R && (qa & 31) == 0) {
-                st_v8(qrow, make_uint4(c[0], c[1], c[2], c[3]), make_uint4(c[4], c[5], c[6], c[7]));
-            } else if (live && e0 + 64 <= R && (qa & 15) == 0) {
-                st_v4(qrow, make_uint4(c[0], c[1], c[2], c[3]));
-                st_v4(qrow + 16, make_uint4(c[4], c[5], c[6], c[7]));
-            } else if (live) {
-#pragma unroll
-                for (int i = 0; i < kBlocks; ++i)
-                    if (e0 + 16 * i < R) st_v2(qrow + 8 * i, c[2 * i], c[2 * i + 1]);
-            }
-        }
-        // scale bytes; blocks past the last row hold zeros and get scale 0,
-        // padded transposed rows (C <= cg < cpad) write 0x00
-        if (inreg) {
-            // the segment's kBlocks scale bytes are consecutive in both layouts (k0 % kBlocks == 0,
-            // and a swizzled row holds 4 consecutive columns per 4-byte group): one store when aligned
-            const int64_t k0 = e0 / kBlock;
-            uint32_t word = 0;
-#pragma unroll
-            for (int i = 0; i < kBlocks; ++i) word |= (live ? scales[i] : 0u) << (8 * i);
-            uint8_t* p = E.sf + qzq::sf_offset(cg, k0, kvT, LAYOUT);
-            if (k0 + kBlocks <= kvs && (reinterpret_cast<uintptr_t>(p) & (kBlocks - 1)) == 0) {
-                if (kBlocks == 4) *reinterpret_cast<uint32_t*>(p) = word;
-                else *reinterpret_cast<uint16_t*>(p) = (uint16_t)word;
-            } else {
-#pragma unroll
-                for (int i = 0; i < kBlocks; ++i) {
-                    const int64_t k = k0 + i;
-                    if (k < kvs) E.sf[qzq::sf_offset(cg, k, kvT, LAYOUT)] = (uint8_t)(word >> (8 * i));
+            for (int j = 0; j < 2; ++j) {
+                if (cg + j >= C || e0 >= R) continue;
+                uint8_t* dst = static_cast<uint8_t*>(E.q) + (cg + j) * (R >> 1) + (e0 >> 1);
+                if (e0 + 32 <= R && (reinterpret_cast<uintptr_t>(dst) & 15) == 0) {
+                    st_v4(dst, make_uint4(c[j][0], c[j][1], c[j][2], c[j][3]));
+                } else {
+                    st_v2(dst, c[j][0], c[j][1]);
+                    if (e0 + 32 <= R) st_v2(dst + 8, c[j][2], c[j][3]);
                 }
             }
         }
-        __syncthreads();  // the shared tile is rewritten with the next tile
-        if (!more) break;
-        tile = next;
-        cur = nxt;
+        // scale bytes: kSeg consecutive ones per column (blocks past the last row
+        // hold zeros and get scale 0; padded transposed rows C <= cg < cpad get 0x00)
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            const int64_t row = cg + j;
+            if (row >= cpad) continue;
+            const bool live = row < C;
+#pragma unroll
+            for (int b = 0; b < kSeg; ++b)
+                if (k0 + b < kvs) E.sf[qzq::sf_offset(row, k0 + b, kvT, LAYOUT)] = live ? (uint8_t)sc[j][b] : (uint8_t)0;
+        }
     }
+    cp_async_wait<0>();  // nothing is left in flight at exit
 }
 
 cudaError_t launch_colwise(const qz_expert* table, int n, int fmt, int layout, int grid, cudaStream_t s,
                            unsigned* d_err) {
-    const size_t smem = (size_t)(n + 1) * sizeof(int);
+    const size_t smem = (size_t)((n + 4) & ~3) * sizeof(int) + (size_t)kColStages * kColStageBytes;
     if (fmt == QZ_FMT_MXFP8) {
         if (layout == QZ_SF_SWIZZLED_128x4)
             colwise_kernel<QZ_FMT_MXFP8, QZ_SF_SWIZZLED_128x4><<<grid, kColThreads, smem, s>>>(table, n, d_err);
@@ -282,19 +268,19 @@ cudaError_t launch_colwise(const qz_expert* table, int n, int fmt, int layout, i
     return cudaGetLastError();
 }
 
-// Resident CTAs per SM (for a one-wave persistent grid).  The 32 KB shared
-// tile plus the largest prefix table exceed 48 KB, so every instantiation is
-// allowed more dynamic shared memory on the current device first (this runs
-// once per device before its first launch).
+// Resident CTAs per SM (for a one-wave persistent grid).  The stages plus the
+// largest prefix table exceed 48 KB, so every instantiation is allowed more
+// dynamic shared memory on the current device first (this runs once per
+// device before its first launch).
 int colwise_blocks_per_sm(int n) {
-    const int bytes = (int)((size_t)(QZ_MAX_EXPERTS + 1) * sizeof(int));
+    const int bytes = (int)((size_t)((QZ_MAX_EXPERTS + 4) & ~3) * sizeof(int) + (size_t)kColStages * kColStageBytes);
     cudaFuncSetAttribute(colwise_kernel<QZ_FMT_MXFP8, QZ_SF_SWIZZLED_128x4>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
     cudaFuncSetAttribute(colwise_kernel<QZ_FMT_MXFP8, QZ_SF_LINEAR>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
     cudaFuncSetAttribute(colwise_kernel<QZ_FMT_NVFP4, QZ_SF_SWIZZLED_128x4>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
     cudaFuncSetAttribute(colwise_kernel<QZ_FMT_NVFP4, QZ_SF_LINEAR>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
     int b = 1;
-    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, colwise_kernel<QZ_FMT_MXFP8, QZ_SF_SWIZZLED_128x4>,
-                                                  kColThreads, (size_t)(n + 1) * sizeof(int));
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, colwise_kernel<QZ_FMT_MXFP8, QZ_SF_SWIZZLED_128x4>, kColThreads,
+                                                  (size_t)((n + 4) & ~3) * sizeof(int) + (size_t)kColStages * kColStageBytes);
     return b > 0 ? b : 1;
 }
 
