@@ -8,11 +8,13 @@
 // factors those of a [cols, rows] matrix in the linear or swizzled 128x4
 // layout, padding written as 0x00 by the kernel.
 //
-// One persistent launch walks all experts' 128 x 128 tiles.  Each CTA keeps
-// three tiles in flight: asynchronous 16-byte copies (cp.async, zero-filled
-// past the matrix) bring a tile row-major into one of three shared-memory
-// stages while the tile before it is quantized, so the loads never wait on
-// the arithmetic and one CTA barrier per tile suffices.  A thread reads one
+// One persistent launch walks all experts' 128 x 128 tiles, each CTA a
+// contiguous run of them (so its expert -- the entry and the NVFP4 scale --
+// changes rarely).  Each CTA keeps three tiles in flight: asynchronous
+// 16-byte copies (cp.async, zero-filled past the matrix) bring a tile
+// row-major into one of three shared-memory stages while the tile before it
+// is quantized, so the loads never wait on the arithmetic and one CTA
+// barrier per tile suffices.  A thread reads one
 // 32-bit word per row -- two neighbouring columns -- for 32 rows, pairs
 // consecutive rows of each column into bf16x2 words, quantizes the two
 // 32-element column segments with the library's block quantizers
@@ -59,11 +61,16 @@ struct ColTiles {
     }
 };
 
-// The tile a CTA works on: tile `tile` of the call, found from expert `e` on.
+// A walk over consecutive tiles of the call: the tile's expert (its entry)
+// and its row / column tile.  Moving to the next tile reloads the entry only
+// when the expert changes.
 struct ColRef {
     const uint16_t* x;
     int64_t R, C, ld;
-    int rt, ct;
+    uint8_t* q;
+    uint8_t* sf;
+    const float* amax;
+    int rt, ct, nct;
     int expert;
 };
 
@@ -71,16 +78,31 @@ __device__ __forceinline__ ColRef col_ref(const qz_expert* table, const int* s_p
     while (tile >= s_prefix[e + 1]) ++e;  // tiles increase; s_prefix[n] == total > tile
     const qz_expert E = load_entry(table, e);
     const int local = tile - s_prefix[e];
-    const int nct = (int)((E.cols + kTileCols - 1) / kTileCols);
     ColRef r;
-    r.rt = local / nct;
-    r.ct = local - r.rt * nct;
+    r.nct = (int)((E.cols + kTileCols - 1) / kTileCols);
+    r.rt = local / r.nct;
+    r.ct = local - r.rt * r.nct;
     r.x = static_cast<const uint16_t*>(E.x);
     r.R = E.rows;
     r.C = E.cols;
     r.ld = E.ld;
+    r.q = static_cast<uint8_t*>(E.q);
+    r.sf = E.sf;
+    r.amax = E.amax;
     r.expert = e;
     return r;
+}
+
+// r describes tile - 1; make it describe tile.
+__device__ __forceinline__ void col_next(ColRef& r, const qz_expert* table, const int* s_prefix, int tile) {
+    if (tile < s_prefix[r.expert + 1]) {
+        if (++r.ct == r.nct) {
+            r.ct = 0;
+            ++r.rt;
+        }
+    } else {
+        r = col_ref(table, s_prefix, tile, r.expert + 1);
+    }
 }
 
 // ---------------------------------------------------------------------------
@@ -129,43 +151,50 @@ __global__ void __launch_bounds__(kColThreads, 2) colwise_kernel(const qz_expert
     if (FMT == QZ_FMT_NVFP4) fill_inv_table(s_inv);  // published by the barriers in block_prefix
     const int total = block_prefix(n, s_prefix, s_scan, ColTiles<FMT, LAYOUT>{table, d_err}, d_err);
     const int t = threadIdx.x;
-    if ((int)blockIdx.x >= total) return;
     const uint32_t stages = (uint32_t)__cvta_generic_to_shared(s_prefix + ((n + 4) & ~3));
     const uint32_t* s_words = reinterpret_cast<const uint32_t*>(s_prefix + ((n + 4) & ~3));
 
-    // prologue: the first kColStages - 1 tiles of this CTA in flight
-    int e_issue = 0, e_cur = 0;  // expert hints of the issuing and the consuming walk
+    // this CTA's tiles: a contiguous run [beg, end) of the call's tiles, so the
+    // expert (entry, NVFP4 scale) changes at most a few times per CTA
+    const int beg = (int)((int64_t)total * blockIdx.x / gridDim.x);
+    const int end = (int)((int64_t)total * (blockIdx.x + 1) / gridDim.x);
+    if (beg >= end) return;
+    ColRef iss = col_ref(table, s_prefix, beg, find_owner(s_prefix, n, beg));  // the walk issuing copies
+    ColRef cur = iss;                                                         // the walk quantizing
+    // prologue: the first kColStages - 1 tiles in flight
 #pragma unroll
     for (int s = 0; s < kColStages - 1; ++s) {
-        const int tile = blockIdx.x + s * gridDim.x;
-        if (tile < total) {
-            const ColRef r = col_ref(table, s_prefix, tile, e_issue);
-            e_issue = r.expert;
-            col_issue(r, stages + s * kColStageBytes, t);
+        if (beg + s < end) {
+            if (s > 0) col_next(iss, table, s_prefix, beg + s);
+            col_issue(iss, stages + s * kColStageBytes, t);
         }
         cp_async_commit();
     }
     const int w = t >> 5, lane = t & 31;
     const int ch = w & 1, rs = w >> 1;  // this warp's column half and 32-row segment of a tile
+    // NVFP4: the expert's encode scale, and lanes 1..15 holding RN(S / m)
+    int scale_expert = -1;
+    float S = 0.0f, qm = 0.0f;
     for (int k = 0;; ++k) {
-        const int tile = blockIdx.x + k * gridDim.x;
-        if (tile >= total) break;
+        const int tile = beg + k;
+        if (tile >= end) break;
         const int cur_s = k % kColStages;
         cp_async_wait<kColStages - 2>();  // this thread's copies of tile k have landed
         __syncthreads();                  // ... and everyone's; tile k - 1's stage is free again
         {
-            const int ahead = tile + (kColStages - 1) * gridDim.x;
-            const int s = (k + kColStages - 1) % kColStages;
-            if (ahead < total) {
-                const ColRef r = col_ref(table, s_prefix, ahead, e_issue);
-                e_issue = r.expert;
-                col_issue(r, stages + s * kColStageBytes, t);
+            const int ahead = tile + kColStages - 1;
+            if (ahead < end) {
+                col_next(iss, table, s_prefix, ahead);
+                col_issue(iss, stages + ((k + kColStages - 1) % kColStages) * kColStageBytes, t);
             }
             cp_async_commit();
         }
-        const ColRef cur = col_ref(table, s_prefix, tile, e_cur);
-        e_cur = cur.expert;
-        const qz_expert E = load_entry(table, cur.expert);
+        if (k > 0) col_next(cur, table, s_prefix, tile);
+        if (FMT == QZ_FMT_NVFP4 && cur.expert != scale_expert) {
+            scale_expert = cur.expert;
+            S = nvfp4_encode_scale(__ldg(cur.amax));
+            qm = rcp_lane_quotient(S, s_inv, lane);  // every lane: the shuffles below need all
+        }
         const int64_t R = cur.R, C = cur.C;
         // ---- thread (warp w, lane l) quantizes tile columns 64 ch + 2 l and + 1,
         //      rows 32 rs .. 32 rs + 31 of each: one word per row holds both columns
@@ -190,12 +219,12 @@ __global__ void __launch_bounds__(kColThreads, 2) colwise_kernel(const qz_expert
             sc[0][0] = qzq::mxfp8_block(xa, qa);
             sc[1][0] = qzq::mxfp8_block(xb, qb);
             if (e0 < R) {
-                const bool q32 = ((reinterpret_cast<uintptr_t>(E.q) & 31) == 0);
+                const bool q32 = ((reinterpret_cast<uintptr_t>(cur.q) & 31) == 0);
 #pragma unroll
                 for (int j = 0; j < 2; ++j) {
                     if (cg + j >= C) continue;
                     const uint32_t* qq = j ? qb : qa;
-                    uint8_t* dst = static_cast<uint8_t*>(E.q) + (cg + j) * R + e0;
+                    uint8_t* dst = cur.q + (cg + j) * R + e0;
                     const uint4 lo = make_uint4(qq[0], qq[1], qq[2], qq[3]), hi = make_uint4(qq[4], qq[5], qq[6], qq[7]);
                     if (q32) {
                         st_v8(dst, lo, hi);
@@ -208,8 +237,6 @@ __global__ void __launch_bounds__(kColThreads, 2) colwise_kernel(const qz_expert
         } else {
             // the tile kernels' NVFP4 arithmetic (same bytes as qzq::nvfp4_block): block
             // scales two at a time, element multipliers from 16 per-tile quotients
-            const float S = nvfp4_encode_scale(__ldg(E.amax));
-            const float qm = rcp_lane_quotient(S, s_inv, lane);  // every lane: the shuffles below need all
             uint32_t c[2][4];
 #pragma unroll
             for (int j = 0; j < 2; ++j) {
@@ -227,7 +254,7 @@ __global__ void __launch_bounds__(kColThreads, 2) colwise_kernel(const qz_expert
 #pragma unroll
             for (int j = 0; j < 2; ++j) {
                 if (cg + j >= C || e0 >= R) continue;
-                uint8_t* dst = static_cast<uint8_t*>(E.q) + (cg + j) * (R >> 1) + (e0 >> 1);
+                uint8_t* dst = cur.q + (cg + j) * (R >> 1) + (e0 >> 1);
                 if (e0 + 32 <= R && (reinterpret_cast<uintptr_t>(dst) & 15) == 0) {
                     st_v4(dst, make_uint4(c[j][0], c[j][1], c[j][2], c[j][3]));
                 } else {
@@ -245,7 +272,7 @@ __global__ void __launch_bounds__(kColThreads, 2) colwise_kernel(const qz_expert
             const bool live = row < C;
 #pragma unroll
             for (int b = 0; b < kSeg; ++b)
-                if (k0 + b < kvs) E.sf[qzq::sf_offset(row, k0 + b, kvT, LAYOUT)] = live ? (uint8_t)sc[j][b] : (uint8_t)0;
+                if (k0 + b < kvs) cur.sf[qzq::sf_offset(row, k0 + b, kvT, LAYOUT)] = live ? (uint8_t)sc[j][b] : (uint8_t)0;
         }
     }
     cp_async_wait<0>();  // nothing is left in flight at exit
