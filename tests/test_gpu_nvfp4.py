@@ -171,6 +171,20 @@ def test_grid_invariance_compute_mode():
             assert all(np.array_equal(u, v) for u, v in zip(a, b))
 
 
+@pytest.mark.parametrize("layout", LAYOUTS)
+def test_per_row_grid_sizes_and_a_large_table(layout):
+    """Per-row mode on rows staged through shared memory: a single CTA (the
+    stage ring wraps many times), a few CTAs, the default grid, and a table
+    of 1100 small experts (a prefix table past the small-table launch kind),
+    each against the oracle."""
+    shapes = [(1, 16), (37, 2064), (129, 4096), (64, 2048), (3, 6000), (200, 96), (0, 64)]
+    xs = [synth.blockwise_scaled(s, 16, seed=400 + i, lo=-12, hi=12).cuda() for i, s in enumerate(shapes)]
+    for ctas in (1, 3, 0):
+        check(xs, layout, qz.NVFP4_PER_ROW, run_nvfp4(xs, layout, qz.NVFP4_PER_ROW, max_ctas=ctas))
+    many = [synth.blockwise_scaled((1 + i % 3, 48), 16, seed=900 + i, lo=-8, hi=8).cuda() for i in range(1100)]
+    check(many, layout, qz.NVFP4_PER_ROW, run_nvfp4(many, layout, qz.NVFP4_PER_ROW))
+
+
 def test_qwen3_235b_sampled_both_projections():
     cfg = synth.QWEN3_235B
     for shape, seed in ((cfg["gate_up"], cfg["seed"]), (cfg["down"], cfg["seed"] + 1000)):
