@@ -465,59 +465,83 @@ def extra_workloads(qz, device, stream, peak,
 
 
 def _extra_split(qz, device, flush, rec):
-    """Row-scaled NVFP4 split activation [16384, 4096] over 64 experts."""
-    x = synth.split_activation(device=device)
+    """Row-scaled NVFP4 split activation [16384, 4096] over 64 experts.  Two
+    copies of the input and of every output are quantized alternately, so
+    consecutive calls share no bytes (2 x 173 MB moved, more than L2 holds)
+    and no flush buffer leaves dirty lines for the timed calls to write back."""
+    x0 = synth.split_activation(device=device)
     counts = synth.dirichlet_splits()
-    T, K = x.shape
-    q = torch.empty((T, K // 2), dtype=torch.uint8, device=device)
-    am = torch.empty(T, dtype=torch.float32, device=device)
-    entries, off, nsf_tot = [], 0, 0
-    for c in counts:
-        c = int(c)
-        n = qz.sf_bytes(c, K, qz.FMT_NVFP4, qz.SF_SWIZZLED)
-        sf = torch.empty(max(n, 16), dtype=torch.uint8, device=device)
-        entries.append(qz.Entry(x[off:off + c], q[off:off + c], sf, am[off:off + c]))
-        nsf_tot += n
-        off += c
-    table = qz.ExpertTable(entries)
+    T, K = x0.shape
+    tables, nsf_tot = [], 0
+    for copy in range(2):
+        x = x0 if copy == 0 else x0.clone()
+        q = torch.empty((T, K // 2), dtype=torch.uint8, device=device)
+        am = torch.empty(T, dtype=torch.float32, device=device)
+        entries, off, nsf_tot = [], 0, 0
+        for c in counts:
+            c = int(c)
+            n = qz.sf_bytes(c, K, qz.FMT_NVFP4, qz.SF_SWIZZLED)
+            sf = torch.empty(max(n, 16), dtype=torch.uint8, device=device)
+            entries.append(qz.Entry(x[off:off + c], q[off:off + c], sf, am[off:off + c]))
+            nsf_tot += n
+            off += c
+        tables.append(qz.ExpertTable(entries))
+    turn = [0]
 
     def split_call():
-        qz.quantize_grouped_nvfp4(table, qz.NVFP4_PER_ROW, qz.SF_SWIZZLED)
+        qz.quantize_grouped_nvfp4(tables[turn[0] % 2], qz.NVFP4_PER_ROW, qz.SF_SWIZZLED)
+        turn[0] += 1
 
-    ms = _time_graph(split_call, reps=10, flush=flush)
+    ms = _time_graph(split_call, reps=10)
     nbytes = T * K * 2 + T * K // 2 + nsf_tot + T * 4
     rec("row-scaled NVFP4 split [16384,4096] over 64 Dirichlet(0.3) experts, swizzled", nbytes, ms, 1,
-        kernel="nvfp4_rows_kernel", l2="flushed before each call", timing="CUDA graph of 10 calls",
-        traffic=ncu_traffic("nvfp4_rows_kernel"))
-    del x, q, am, entries, table
+        kernel="nvfp4_rows_kernel",
+        l2="inputs larger than L2: two copies of input and outputs alternated (no flush)",
+        timing="CUDA graph of 10 calls", traffic=ncu_traffic("nvfp4_rows_kernel"))
+    del x0, tables
 
 
 def _extra_fused(qz, device, flush, out, peak, tokens=None):
-    """Fused residual + RMSNorm + quantize, T sweep at H = 7168."""
+    """Fused residual + RMSNorm + quantize, T sweep at H = 7168.  From
+    T = 1024 on, enough copies of inputs and outputs are used round-robin that
+    a call's bytes were last touched more than twice the L2 size ago (no
+    flush, so no dirty flush lines are written back inside the timed calls);
+    below, calls repeat on the same buffers (latency mode, data in L2 as it
+    would be right after its producer)."""
     H = synth.FUSED_NORM["hidden"]
+    L2 = 126 * 2 ** 20
     for fmt, layout, fname in ((qz.FMT_MXFP8, qz.SF_SWIZZLED, "MXFP8 swizzled"), (qz.FMT_NVFP4, qz.SF_LINEAR, "NVFP4 linear")):
         sweep = []
         for Tn in (tokens or synth.FUSED_NORM["tokens"]):
-            xs, rs, gs = synth.fused_norm_inputs(Tn, device=device)
-            y = torch.empty_like(xs)
-            h = torch.empty_like(xs)
-            qq = torch.empty((Tn, H if fmt == qz.FMT_MXFP8 else H // 2), dtype=torch.uint8, device=device)
-            sff = torch.empty(max(qz.sf_bytes(Tn, H, fmt, layout), 16), dtype=torch.uint8, device=device)
-            amax = torch.tensor([8.0], dtype=torch.float32, device=device) if fmt == qz.FMT_NVFP4 else None
-
-            def call():
-                qz.rmsnorm_quantize(xs, rs, gs, 1e-6, y, h, fmt, qq, sff, layout, amax)
-
-            ms = _time_graph(call, reps=10, flush=flush) if Tn >= 1024 else _time_graph(call, reps=50)
             qbytes = Tn * (H if fmt == qz.FMT_MXFP8 else H // 2)
             nbytes = Tn * H * 2 * 2 + 2 * H + Tn * H * 2 * 2 + qbytes + qz.sf_bytes(Tn, H, fmt, layout)
-            sweep.append({"T": Tn, "us": round(ms * 1e3, 2), "GB/s": round(nbytes / (ms / 1e3) / GB, 1)})
+            copies = 1 if Tn < 1024 else -(-2 * L2 // nbytes) + 1
+            sets = []
+            xs, rs, gs = synth.fused_norm_inputs(Tn, device=device)
+            for c in range(copies):
+                sets.append((xs if c == 0 else xs.clone(), rs if c == 0 else rs.clone(), torch.empty_like(xs),
+                             torch.empty_like(xs),
+                             torch.empty((Tn, H if fmt == qz.FMT_MXFP8 else H // 2), dtype=torch.uint8, device=device),
+                             torch.empty(max(qz.sf_bytes(Tn, H, fmt, layout), 16), dtype=torch.uint8, device=device)))
+            amax = torch.tensor([8.0], dtype=torch.float32, device=device) if fmt == qz.FMT_NVFP4 else None
+            turn = [0]
+
+            def call():
+                x_, r_, y_, h_, q_, sf_ = sets[turn[0] % copies]
+                turn[0] += 1
+                qz.rmsnorm_quantize(x_, r_, gs, 1e-6, y_, h_, fmt, q_, sf_, layout, amax)
+
+            ms = _time_graph(call, reps=10 * copies) if Tn >= 1024 else _time_graph(call, reps=50)
+            sweep.append({"T": Tn, "us": round(ms * 1e3, 2), "GB/s": round(nbytes / (ms / 1e3) / GB, 1),
+                          "copies": copies})
+            del sets
         big = sweep[-1]
         if big["T"] != 4096:
             big = {"GB/s": 0.0}
         out.append({"workload": f"fused residual+RMSNorm+{fname}, H=7168, T=1..4096 (residual_out written)",
                     "kernel": "rmsnorm_quant_kernel", "sweep": sweep,
-                    "timing": "CUDA graph of 50 calls (T < 1024) or 10 calls after an L2 flush each",
+                    "timing": "CUDA graph of 50 calls on the same buffers (T < 1024) or of 10 rounds over "
+                              "`copies` buffer sets (T >= 1024, inputs larger than L2, no flush)",
                     "frac_of_hbm_peak_T4096": round(big["GB/s"] / peak, 4),
                     "traffic_T4096": ncu_traffic("rmsnorm_quant_kernel") if fmt == qz.FMT_MXFP8 else None})
 
@@ -696,9 +720,10 @@ def _extra_merge(qz, device, flush, out, peak, tokens=None):
             qz.attention_merge_quantize(Od, ld, y, None, None, qz.SF_SWIZZLED)
             qz.quantize_grouped_mxfp8(tab, qz.SF_SWIZZLED)
 
-        fl = flush if Tn >= 512 else None
-        ms_f = _time_graph(fused, reps=10 if fl else 50, flush=fl)
-        ms_u = _time_graph(unfused, reps=10 if fl else 50, flush=fl)
+        fl = flush if 512 <= Tn < 2048 else None  # from T = 2048 on the partials alone exceed L2
+        reps = 10 if Tn >= 512 else 50
+        ms_f = _time_graph(fused, reps=reps, flush=fl)
+        ms_u = _time_graph(unfused, reps=reps, flush=fl)
         nbytes = S * Tn * H * 4 + S * Tn * 4 + Tn * H * 2 + Tn * H + qz.sf_bytes(Tn, H, qz.FMT_MXFP8, qz.SF_SWIZZLED)
         sweep.append({"T": Tn, "fused_us": round(ms_f * 1e3, 2), "unfused_us": round(ms_u * 1e3, 2),
                       "fused_GB/s": round(nbytes / (ms_f / 1e3) / GB, 1)})
@@ -707,7 +732,8 @@ def _extra_merge(qz, device, flush, out, peak, tokens=None):
     out.append({"workload": "attention decode merge, 8 splits, H=7168, bf16 + MXFP8 swizzled in one kernel "
                             "vs merge then standalone quantize, T=1..4096",
                 "kernel": "attention_merge_kernel", "sweep": sweep,
-                "timing": "CUDA graph of 50 calls (T < 512) or 10 calls after an L2 flush each",
+                "timing": "CUDA graph of 50 calls (T < 512), of 10 calls after an L2 flush each (T = 512), "
+                          "or of 10 calls on partials larger than L2 (T >= 2048, no flush)",
                 "frac_of_hbm_peak_fused_T4096": round(big["fused_GB/s"] / peak, 4) if big["T"] == 4096 else None})
 
 
