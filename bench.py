@@ -72,7 +72,7 @@ KERNEL_SOURCES = {
     "rmsnorm_quant_kernel": ("qz_rmsnorm.cu", "qz_device.cuh"),
     "dequant_kernel": ("qz_dequant.cu", "qz_device.cuh"),
     "attention_merge_kernel": ("qz_merge.cu", "qz_device.cuh"),
-    "colwise_kernel": ("qz_colwise.cu", "qz_device.cuh"),
+    "colwise_kernel": ("qz_colwise.cu", "qz_device.cuh", "qz_async.cuh"),
     "split_fused_kernel": ("qz_split.cu", "qz_device.cuh"),
 }
 

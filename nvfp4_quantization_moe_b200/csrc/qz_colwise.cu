@@ -22,6 +22,7 @@
 // takes the tensor amax as given (the row-wise computed-amax call of the
 // same tensor produces it).
 #include "../../include/qz_quant.cuh"
+#include "qz_async.cuh"
 
 namespace qz {
 
