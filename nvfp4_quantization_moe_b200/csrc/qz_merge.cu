@@ -38,15 +38,39 @@ __global__ void __launch_bounds__(kMergeThreads) attention_merge_kernel(const fl
     __syncthreads();
     double wsum = 0.0;
     double acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-    for (int s = 0; s < S; ++s) {
+    // splits four at a time: their loads are all in flight before the first is summed
+    constexpr int kU = 4;
+    const float4* src = reinterpret_cast<const float4*>(O + (int64_t)t * H + c0);
+    const int64_t split_stride = T * H / 4;  // float4s between consecutive splits
+    int s = 0;
+    for (; s + kU <= S; s += kU) {
+        float4 a[kU], b[kU];
+        if (live) {
+#pragma unroll
+            for (int u = 0; u < kU; ++u) {
+                a[u] = __ldg(src + (s + u) * split_stride);
+                b[u] = __ldg(src + (s + u) * split_stride + 1);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+            const double wgt = s_w[s + u];
+            wsum = wsum + wgt;
+            if (live) {
+                const float v[8] = {a[u].x, a[u].y, a[u].z, a[u].w, b[u].x, b[u].y, b[u].z, b[u].w};
+#pragma unroll
+                for (int i = 0; i < 8; ++i) acc[i] = acc[i] + wgt * (double)v[i];  // product, then sum (no FMA)
+            }
+        }
+    }
+    for (; s < S; ++s) {
         const double wgt = s_w[s];
         wsum = wsum + wgt;
         if (live) {
-            const float4* src = reinterpret_cast<const float4*>(O + ((int64_t)s * T + t) * H + c0);
-            const float4 a = __ldg(src), b = __ldg(src + 1);
+            const float4 a = __ldg(src + s * split_stride), b = __ldg(src + s * split_stride + 1);
             const float v[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
 #pragma unroll
-            for (int i = 0; i < 8; ++i) acc[i] = acc[i] + wgt * (double)v[i];  // product, then sum (no FMA)
+            for (int i = 0; i < 8; ++i) acc[i] = acc[i] + wgt * (double)v[i];
         }
     }
     // one rounding to bf16 of the binary64 quotient
