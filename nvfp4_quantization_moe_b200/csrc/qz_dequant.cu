@@ -125,9 +125,6 @@ __device__ __forceinline__ uint32_t bf16x2_rn(float lo, float hi) {
     return r;
 }
 
-// Whether binary32 x lies exactly halfway between two bf16 numbers.
-__device__ __forceinline__ bool bf16_midpoint(float x) { return (__float_as_uint(x) & 0xFFFFu) == 0x8000u; }
-
 __device__ __forceinline__ int64_t dq_sf_index(int layout, int64_t row, int64_t k, int64_t kv) {
     return layout == QZ_SF_SWIZZLED_128x4 ? swz_offset(row, k, kv) : row * kv + k;
 }
@@ -222,8 +219,10 @@ __device__ __forceinline__ uint4 dq_mx8(uint32_t w0, uint32_t w1, float s) {
 __device__ __forceinline__ uint4 dq_nv8(uint32_t word, uint32_t sv2, float g) {
     uint4 o;
     uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
-    bool tie = false;
     float hv[8], pv[8];
+    // the low 16 bits of every RN32 product, xor 0x8000: a zero half marks a
+    // bf16 midpoint; their running minimum (per 16-bit half) finds any
+    uint32_t mid = 0xFFFFFFFFu;
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
         const uint32_t ph = __hmul2_rn_bits(e2m1x2_to_f16x2((word >> (8 * j)) & 0xFFu), sv2);
@@ -234,8 +233,9 @@ __device__ __forceinline__ uint4 dq_nv8(uint32_t word, uint32_t sv2, float g) {
         hv[2 * j] = h.x;
         hv[2 * j + 1] = h.y;
         ow[j] = bf16x2_rn(h.x, h.y);
-        tie |= bf16_midpoint(h.x) | bf16_midpoint(h.y);
+        mid = __vminu2(mid, __byte_perm(__float_as_uint(h.x), __float_as_uint(h.y), 0x5410) ^ 0x80008000u);
     }
+    const bool tie = (mid & 0xFFFFu) == 0u || (mid >> 16) == 0u;
     if (tie) {
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
