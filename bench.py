@@ -434,7 +434,8 @@ class L2Flush:
 
 
 def extra_workloads(qz, device, stream, peak,
-                    which=("split", "fused", "nvfp4", "large", "dequant", "merge", "colwise", "gateup"), tokens=None):
+                    which=("tiny", "split", "fused", "nvfp4", "large", "dequant", "merge", "colwise", "gateup"),
+                    tokens=None):
     out = []
     flush = L2Flush(device)
 
@@ -445,6 +446,8 @@ def extra_workloads(qz, device, stream, peak,
         d.update(kw)
         out.append(d)
 
+    if "tiny" in which:
+        _extra_tiny(qz, device, rec)
     if "split" in which:
         _extra_split(qz, device, flush, rec)
     if "fused" in which:
@@ -462,6 +465,34 @@ def extra_workloads(qz, device, stream, peak,
     if "gateup" in which:
         _extra_gate_up_split(qz, device, rec)
     return out
+
+
+def _extra_tiny(qz, device, rec):
+    """The tiny MXFP8 group (4 experts [64, 256], linear scales): a
+    launch-latency case.  Reports the median and the 10th / 90th percentile of
+    single calls, each timed with CUDA events on its own."""
+    xs = [x.to(device) for x in synth.tiny_group()]
+    ents = qz.alloc_outputs(xs, qz.FMT_MXFP8, qz.SF_LINEAR, qz.NVFP4_PER_ROW)
+    tab = qz.ExpertTable(ents)
+    for _ in range(20):
+        qz.quantize_grouped_mxfp8(tab, qz.SF_LINEAR)
+    torch.cuda.synchronize()
+    times = []
+    for _ in range(200):
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record()
+        qz.quantize_grouped_mxfp8(tab, qz.SF_LINEAR)
+        b.record()
+        b.synchronize()
+        times.append(a.elapsed_time(b))
+    times.sort()
+    med = times[len(times) // 2]
+    rows, cols = xs[0].shape
+    nbytes = len(xs) * (rows * cols * 3 + rows * cols // 32)
+    rec("tiny MXFP8 group: 4 experts [64, 256], linear scales", nbytes, med, 1, kernel="mxfp8_grouped_kernel",
+        timing="median of 200 single calls (CUDA events around each)",
+        p10_us=round(times[len(times) // 10] * 1e3, 2), p90_us=round(times[9 * len(times) // 10] * 1e3, 2))
 
 
 def _extra_split(qz, device, flush, rec):
@@ -805,12 +836,19 @@ def main():
     ap.add_argument("--no-extra", action="store_true", help="skip the other workloads")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
-    ap.add_argument("--only", choices=["split", "fused", "nvfp4", "large", "dequant", "merge", "colwise", "gateup"],
+    ap.add_argument("--config", type=int, choices=[1, 2, 3, 4, 5], default=None,
+                    help="one of the five workloads: 1 tiny MXFP8 group (latency), 2 the Qwen3-30B-A3B refit step "
+                         "(the default run), 3 the row-scaled NVFP4 split activation, 4 the fused residual + "
+                         "RMSNorm sweep, 5 the Qwen3-235B-A22B layer")
+    ap.add_argument("--only", choices=["tiny", "split", "fused", "nvfp4", "large", "dequant", "merge", "colwise",
+                                       "gateup"],
                     default=None,
                     help="time only this secondary workload and print its record (profiling aid)")
     ap.add_argument("--tokens", type=str, default=None,
                     help="comma-separated token counts for the fused sweep (default: 1..4096)")
     args = ap.parse_args()
+    if args.config is not None and args.config != 2:
+        args.only = {1: "tiny", 3: "split", 4: "fused", 5: "large"}[args.config]
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
