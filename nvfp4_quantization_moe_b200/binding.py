@@ -80,7 +80,7 @@ class _FusedSplit(ctypes.Structure):
 
 class _Opts(ctypes.Structure):
     _fields_ = [("d_err", ctypes.c_void_p), ("max_ctas", ctypes.c_int), ("d_workspace", ctypes.c_void_p),
-                ("workspace_bytes", ctypes.c_size_t)]
+                ("workspace_bytes", ctypes.c_size_t), ("elems_hint", ctypes.c_int64)]
 
 
 assert ctypes.sizeof(_Expert) == 56 and ctypes.sizeof(_SfPair) == 32 and ctypes.sizeof(_DqExpert) == 56
@@ -146,15 +146,15 @@ def _stream_ptr(stream) -> ctypes.c_void_p:
     return ctypes.c_void_p(int(stream.cuda_stream) if hasattr(stream, "cuda_stream") else int(stream))
 
 
-def _opts(err: Optional[torch.Tensor], max_ctas: int, workspace: Optional[torch.Tensor] = None):
-    if err is None and not max_ctas and workspace is None:
+def _opts(err: Optional[torch.Tensor], max_ctas: int, workspace: Optional[torch.Tensor] = None, elems_hint: int = 0):
+    if err is None and not max_ctas and workspace is None and not elems_hint:
         return None
     if err is not None:
         assert err.dtype in (torch.int32, torch.uint32) and err.is_cuda and err.numel() >= 1
     ws_ptr = workspace.data_ptr() if workspace is not None else 0
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     return ctypes.byref(_Opts(ctypes.c_void_p(err.data_ptr() if err is not None else 0), int(max_ctas),
-                              ctypes.c_void_p(ws_ptr), ctypes.c_size_t(ws_bytes)))
+                              ctypes.c_void_p(ws_ptr), ctypes.c_size_t(ws_bytes), ctypes.c_int64(int(elems_hint))))
 
 
 def workspace_bytes(n_experts: int) -> int:
@@ -209,6 +209,7 @@ class ExpertTable:
         dev = device if device is not None else (self.entries[0].x.device if n else torch.device("cuda"))
         self.dev = host.to(dev)
         self.n = n
+        self.elems = sum(int(e.x.shape[0]) * int(e.x.shape[1]) for e in self.entries)
 
     @property
     def ptr(self) -> int:
@@ -223,6 +224,7 @@ class ExpertTable:
         arr = (_Expert * max(len(raw), 1))(*[_Expert(*r) for r in raw])
         self.entries = []
         self.n = len(raw)
+        self.elems = 0
         self.dev = torch.frombuffer(bytearray(bytes(arr)), dtype=torch.uint8).to(device)
         return self
 
@@ -341,8 +343,10 @@ class SfPairTable:
 # ---------------------------------------------------------------------------
 
 def quantize_grouped_mxfp8(table: ExpertTable, layout: int, stream=None, err=None, max_ctas: int = 0):
+    """MXFP8 over the table; the table's element count goes along as the grid-size hint."""
     _check(load().qz_quantize_grouped_mxfp8(ctypes.c_void_p(table.ptr), table.n, int(layout),
-                                            _stream_ptr(stream), _opts(err, max_ctas)),
+                                            _stream_ptr(stream),
+                                            _opts(err, max_ctas, elems_hint=getattr(table, "elems", 0))),
            "qz_quantize_grouped_mxfp8")
 
 

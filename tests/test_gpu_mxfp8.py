@@ -3,6 +3,8 @@ payload and scale bytes, both layouts, ragged tiles, strided rows, batch-size
 and grid-shape invariance, per-expert independence (canaries), empty and
 invalid table entries, stream order and CUDA-graph replay, and the
 Qwen3-30B-A3B / Qwen3-235B-A22B expert shapes at full size (sampled experts)."""
+import ctypes
+
 import numpy as np
 import pytest
 import torch
@@ -95,6 +97,26 @@ def test_batch_size_and_grid_invariance():
         for (a, b), (c, d) in zip(whole, other):
             assert np.array_equal(a, c) and np.array_equal(b, d)
     check_against_oracle(xs, qz.SF_SWIZZLED, whole)
+
+
+@pytest.mark.parametrize("hint", [1, 1 << 26, 1 << 40])
+def test_grid_sized_by_the_element_hint(hint):
+    """The element-count hint only sizes the grid (one wave up to 16 waves of
+    short CTAs, most of them idle on a small table): the bytes stay the
+    oracle's."""
+    xs = [synth.blockwise_scaled(s, 32, seed=60 + i, lo=-10, hi=10).cuda()
+          for i, s in enumerate([(130, 256), (1, 64), (300, 96), (0, 32), (64, 512)])]
+    entries, keep = guarded_entries(xs, qz.FMT_MXFP8, qz.SF_SWIZZLED)
+    table = qz.ExpertTable(entries)
+    opts = qz.binding._opts(None, 0, elems_hint=hint)
+    st = qz.load().qz_quantize_grouped_mxfp8(ctypes.c_void_p(table.ptr), table.n, qz.SF_SWIZZLED,
+                                             qz.binding._stream_ptr(None), opts)
+    assert st == qz.QZ_OK
+    torch.cuda.synchronize()
+    for q, sf, _ in keep:
+        assert q.guards_intact() and sf.guards_intact()
+    got = [(q.host().reshape(x.shape[0], -1) if x.shape[0] else q.host(), sf.host()) for (q, sf, _), x in zip(keep, xs)]
+    check_against_oracle(xs, qz.SF_SWIZZLED, got)
 
 
 def test_requantize_one_expert_touches_nothing_else():
