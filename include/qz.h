@@ -190,11 +190,11 @@ typedef struct qz_launch_opts {
                                and a quantize pass over HBM.  The call zeroes it first (in
                                stream order); calls sharing a workspace must not overlap. */
     size_t workspace_bytes; /* size of d_workspace in bytes */
-    int64_t elems_hint;     /* qz_quantize_grouped_mxfp8: the call's elements (sum of rows * cols over
-                               the table), 0 if unknown.  With it, the grid is sized to the work: about
-                               one CTA per ten 128 x 128 tiles, in whole waves (1 to 16), which streams
-                               large calls faster than one persistent wave; without it, one wave.  Any
-                               value gives the same results. */
+    int64_t elems_hint;     /* qz_quantize_grouped_mxfp8 and the MXFP8 qz_dequantize_grouped: the call's
+                               elements (sum of rows * cols over the table), 0 if unknown.  With it, the
+                               grid is sized to the work: about one CTA per ten 128 x 128 tiles, in whole
+                               waves (1 to 16), which streams large calls faster than one persistent
+                               wave; without it, one wave.  Any value gives the same results. */
 } qz_launch_opts;
 
 /* Bytes of device scratch qz_quantize_grouped_nvfp4 uses for

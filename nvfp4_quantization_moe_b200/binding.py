@@ -259,6 +259,7 @@ class DqTable:
         dev = device if device is not None else (self.entries[0].y.device if n else torch.device("cuda"))
         self.dev = host.to(dev)
         self.n = n
+        self.elems = sum(int(e.y.shape[0]) * int(e.y.shape[1]) for e in self.entries)
 
     @property
     def ptr(self) -> int:
@@ -272,6 +273,7 @@ class DqTable:
         arr = (_DqExpert * max(len(raw), 1))(*[_DqExpert(*r) for r in raw])
         self.entries = []
         self.n = len(raw)
+        self.elems = 0
         self.dev = torch.frombuffer(bytearray(bytes(arr)), dtype=torch.uint8).to(device)
         return self
 
@@ -379,7 +381,8 @@ def rmsnorm_quantize(x, residual, gamma, eps: float, norm_out, residual_out, fmt
 def dequantize_grouped(table: DqTable, fmt: int, per_row: bool, layout: int, stream=None, err=None,
                        max_ctas: int = 0):
     _check(load().qz_dequantize_grouped(ctypes.c_void_p(table.ptr), table.n, int(fmt), 1 if per_row else 0,
-                                        int(layout), _stream_ptr(stream), _opts(err, max_ctas)),
+                                        int(layout), _stream_ptr(stream),
+                                        _opts(err, max_ctas, elems_hint=getattr(table, "elems", 0))),
            "qz_dequantize_grouped")
 
 

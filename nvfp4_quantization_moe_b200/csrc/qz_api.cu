@@ -108,16 +108,17 @@ bool valid_layout(int layout) { return layout == QZ_SF_LINEAR || layout == QZ_SF
 
 qz_status from_cuda(cudaError_t e) { return e == cudaSuccess ? QZ_OK : QZ_ERR_CUDA; }
 
-// Grid of the MXFP8 tile kernel: with an element count, about one CTA per
-// kTilesPerCta tiles in whole waves (at most kMaxWaves), since the hardware's
-// placement of many short CTAs streams a large call faster than one
-// persistent wave (measured: 5.4 -> 6.6 TB/s on 128 experts of 3072 x 4096);
-// a cap in opts->max_ctas still applies.
+// Grid of the MXFP8 tile kernels (quantize, dequantize): with an element
+// count, about one CTA per kTilesPerCta tiles in whole waves (at most
+// kMaxWaves), since the hardware's placement of many short CTAs streams a
+// large call faster than one persistent wave (measured: 5.4 -> 6.6 TB/s on
+// 128 experts of 3072 x 4096); a cap in opts->max_ctas still applies.  The
+// NVFP4 kernels measured slower that way and keep one wave.
 constexpr int64_t kTilesPerCta = 10;
 constexpr int64_t kMaxWaves = 16;
 
-int mxfp8_grid(const qz_launch_opts* opts) {
-    const int wave = wave_grid(0, nullptr);
+int sized_grid(int kind, const qz_launch_opts* opts) {
+    const int wave = wave_grid(kind, nullptr);
     int grid = wave;
     if (opts && opts->elems_hint > 0) {
         const int64_t tiles = (opts->elems_hint + 16383) / 16384;
@@ -153,7 +154,7 @@ qz_status qz_quantize_grouped_mxfp8(const qz_expert* d_table, int n_experts, int
     if (st != QZ_OK) return st;
     if (!valid_layout(layout)) return QZ_ERR_INVALID_ARG;
     if (n_experts == 0) return QZ_OK;
-    return from_cuda(qz::launch_mxfp8(d_table, n_experts, layout, mxfp8_grid(opts), (cudaStream_t)stream,
+    return from_cuda(qz::launch_mxfp8(d_table, n_experts, layout, sized_grid(0, opts), (cudaStream_t)stream,
                                       err_word(opts)));
 }
 
@@ -228,7 +229,8 @@ qz_status qz_dequantize_grouped(const qz_dq_expert* d_table, int n_experts, int 
     if (!valid_layout(layout)) return QZ_ERR_INVALID_ARG;
     if (fmt != QZ_FMT_MXFP8 && fmt != QZ_FMT_NVFP4) return QZ_ERR_INVALID_ARG;
     if (n_experts == 0) return QZ_OK;
-    return from_cuda(qz::launch_dequant(d_table, n_experts, fmt, per_row != 0, layout, wave_grid(6, opts),
+    return from_cuda(qz::launch_dequant(d_table, n_experts, fmt, per_row != 0, layout,
+                                        fmt == QZ_FMT_MXFP8 ? sized_grid(6, opts) : wave_grid(6, opts),
                                         (cudaStream_t)stream, err_word(opts)));
 }
 
