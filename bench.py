@@ -435,7 +435,7 @@ class L2Flush:
 
 def extra_workloads(qz, device, stream, peak,
                     which=("tiny", "split", "fused", "nvfp4", "large", "dequant", "merge", "colwise", "gateup"),
-                    tokens=None):
+                    tokens=None, experts=None):
     out = []
     flush = L2Flush(device)
 
@@ -455,7 +455,7 @@ def extra_workloads(qz, device, stream, peak,
     if "nvfp4" in which:
         _extra_nvfp4_30b(qz, device, rec)
     if "large" in which:
-        _extra_large(qz, device, rec)
+        _extra_large(qz, device, rec, experts)
     if "dequant" in which:
         _extra_dequant(qz, device, rec)
     if "merge" in which:
@@ -601,9 +601,12 @@ def _extra_nvfp4_30b(qz, device, rec):
     torch.cuda.empty_cache()
 
 
-def _extra_large(qz, device, rec):
-    """One Qwen3-235B-A22B layer: 128 experts per projection per call."""
-    cfg = synth.QWEN3_235B
+def _extra_large(qz, device, rec, experts=None):
+    """One Qwen3-235B-A22B layer: 128 experts per projection per call (or the
+    first `experts` of them, for a profiler capture)."""
+    cfg = dict(synth.QWEN3_235B)
+    if experts:
+        cfg["experts"] = experts
     for proj, shape in (("gate_up", cfg["gate_up"]), ("down", cfg["down"])):
         stack = synth.expert_stack(cfg["experts"], shape, cfg["std"], seed=cfg["seed"], device=device)
         rows, cols = shape
@@ -625,7 +628,7 @@ def _extra_large(qz, device, rec):
             nsf = qz.sf_bytes(rows, cols, fmt, qz.SF_SWIZZLED)
             qb = rows * cols if fmt == qz.FMT_MXFP8 else rows * cols // 2
             nbytes = cfg["experts"] * (rows * cols * 2 + qb + nsf + (4 if fmt == qz.FMT_NVFP4 else 0))
-            rec(f"Qwen3-235B-A22B {proj} {list(shape)} x128 experts, {fname}, swizzled", nbytes, ms,
+            rec(f"Qwen3-235B-A22B {proj} {list(shape)} x{cfg['experts']} experts, {fname}, swizzled", nbytes, ms,
                 1 if mode != qz.NVFP4_PER_TENSOR_COMPUTE else 2)
             del ents, tab
         del stack
@@ -844,6 +847,8 @@ def main():
                                        "gateup"],
                     default=None,
                     help="time only this secondary workload and print its record (profiling aid)")
+    ap.add_argument("--experts", type=int, default=None,
+                    help="experts per call of the Qwen3-235B-A22B workload (default 128; fewer for a profiler capture)")
     ap.add_argument("--tokens", type=str, default=None,
                     help="comma-separated token counts for the fused sweep (default: 1..4096)")
     args = ap.parse_args()
@@ -871,7 +876,8 @@ def main():
     peak, peak_kind = hbm_peak()
     if args.only:
         toks = [int(t) for t in args.tokens.split(",")] if args.tokens else None
-        print(json.dumps({"only": args.only, "extra": extra_workloads(qz, device, stream, peak, (args.only,), toks)}))
+        print(json.dumps({"only": args.only,
+                          "extra": extra_workloads(qz, device, stream, peak, (args.only,), toks, args.experts)}))
         return
 
     work = Refit30B(qz, device, layers=args.layers, seed_offset=rank)
