@@ -488,12 +488,15 @@ def _extra_tiny(qz, device, rec):
         b.record()
     torch.cuda.synchronize()
     times = sorted(a.elapsed_time(b) for a, b in ev)
-    med = times[len(times) // 2]
+    ms = _time_graph(lambda: qz.quantize_grouped_mxfp8(tab, qz.SF_LINEAR), reps=50)
     rows, cols = xs[0].shape
     nbytes = len(xs) * (rows * cols * 3 + rows * cols // 32)
-    rec("tiny MXFP8 group: 4 experts [64, 256], linear scales", nbytes, med, 1, kernel="mxfp8_grouped_kernel",
-        timing="median of 200 single calls (CUDA events around each, all queued behind a spinning kernel)",
-        p10_us=round(times[len(times) // 10] * 1e3, 2), p90_us=round(times[9 * len(times) // 10] * 1e3, 2))
+    rec("tiny MXFP8 group: 4 experts [64, 256], linear scales", nbytes, ms, 1, kernel="mxfp8_grouped_kernel",
+        timing="per call of a CUDA graph of 50 calls; single_call_* from 200 calls each bracketed by CUDA events "
+               "(event pair included), all queued behind a spinning kernel",
+        single_call_median_us=round(times[len(times) // 2] * 1e3, 2),
+        single_call_p10_us=round(times[len(times) // 10] * 1e3, 2),
+        single_call_p90_us=round(times[9 * len(times) // 10] * 1e3, 2))
 
 
 def _extra_split(qz, device, flush, rec):

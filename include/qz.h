@@ -194,7 +194,8 @@ typedef struct qz_launch_opts {
                                elements (sum of rows * cols over the table), 0 if unknown.  With it, the
                                grid is sized to the work: about one CTA per ten 128 x 128 tiles, in whole
                                waves (1 to 16), which streams large calls faster than one persistent
-                               wave; without it, one wave.  Any value gives the same results. */
+                               wave, and one CTA per tile below one wave; without it, one wave.  Any
+                               value gives the same results. */
 } qz_launch_opts;
 
 /* Bytes of device scratch qz_quantize_grouped_nvfp4 uses for

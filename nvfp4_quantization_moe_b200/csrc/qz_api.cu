@@ -112,7 +112,8 @@ qz_status from_cuda(cudaError_t e) { return e == cudaSuccess ? QZ_OK : QZ_ERR_CU
 // count, about one CTA per kTilesPerCta tiles in whole waves (at most
 // kMaxWaves), since the hardware's placement of many short CTAs streams a
 // large call faster than one persistent wave (measured: 5.4 -> 6.6 TB/s on
-// 128 experts of 3072 x 4096); a cap in opts->max_ctas still applies.  The
+// 128 experts of 3072 x 4096), and a call of fewer tiles than one wave
+// launches one CTA per tile; a cap in opts->max_ctas still applies.  The
 // NVFP4 kernels measured slower that way and keep one wave.
 constexpr int64_t kTilesPerCta = 10;
 constexpr int64_t kMaxWaves = 16;
@@ -125,6 +126,7 @@ int sized_grid(int kind, const qz_launch_opts* opts) {
         int64_t waves = (tiles + kTilesPerCta * wave / 2) / (kTilesPerCta * wave);  // rounded
         waves = waves < 1 ? 1 : (waves > kMaxWaves ? kMaxWaves : waves);
         grid = (int)(wave * waves);
+        if (tiles < grid) grid = (int)tiles;  // a small call launches no idle CTAs
     }
     if (opts && opts->max_ctas > 0 && opts->max_ctas < grid) grid = opts->max_ctas;
     return grid;
