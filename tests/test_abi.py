@@ -6,6 +6,7 @@ import re
 import subprocess
 
 import pytest
+import torch
 
 import nvfp4_quantization_moe_b200 as qz
 from nvfp4_quantization_moe_b200 import build as qzbuild
@@ -148,3 +149,21 @@ def test_product_path_does_not_import_oracle():
             if f.endswith((".py", ".cu", ".cuh", ".h")):
                 text = open(os.path.join(dirpath, f)).read()
                 assert "import oracle" not in text and "from oracle" not in text and "qz_oracle" not in text, f
+
+
+def test_element_hint_reaches_the_launch_options():
+    """The binding passes a table's element count as qz_launch_opts.elems_hint
+    (the MXFP8 kernels size their grid from it); tables built from raw entries
+    carry no hint."""
+    xs = [torch.zeros((r, c), dtype=torch.bfloat16) for r, c in ((3, 64), (0, 32), (130, 256))]
+    entries = [qz.Entry(x, torch.zeros(max(x.numel(), 1), dtype=torch.uint8), torch.zeros(16, dtype=torch.uint8))
+               for x in xs]
+    table = qz.ExpertTable(entries, device=torch.device("cpu"))
+    assert table.elems == 3 * 64 + 130 * 256
+    opts = qz.binding._opts(None, 0, elems_hint=table.elems)
+    assert opts._obj.elems_hint == table.elems and opts._obj.max_ctas == 0
+    assert qz.binding._opts(None, 0) is None
+    raw = qz.ExpertTable.from_raw([(0, 0, 64, 64, 0, 0, 0)], torch.device("cpu"))
+    assert raw.elems == 0
+    assert ctypes.sizeof(qz.binding._Opts) == 40
+
