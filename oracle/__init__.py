@@ -68,6 +68,7 @@ def _declare(lib):
         "qzo_quantize_nvfp4": (None, [P, i64, i64, i64, P, P, c.c_int, c.c_int, P]),
         "qzo_residual_rmsnorm": (None, [P, P, P, c.c_float, i64, i64, P, P]),
         "qzo_rmsnorm_quantize": (None, [P, P, P, c.c_float, i64, i64, P, P, c.c_int, P, P, c.c_int, P]),
+        "qzo_rank_sum": (None, [P, c.c_int, i64, P]),
         "qzo_dequantize_mxfp8": (None, [P, P, i64, i64, c.c_int, P, i64]),
         "qzo_dequantize_nvfp4": (None, [P, P, P, c.c_int, i64, i64, c.c_int, P, i64]),
         "qzo_attention_merge": (None, [P, P, i64, i64, i64, P]),
@@ -302,6 +303,24 @@ def rmsnorm_quantize(x, r, gamma, eps, fmt, layout, amax_in=None, lib=None):
     lib.qzo_rmsnorm_quantize(_ptr(x), _ptr(r), _ptr(gamma), ctypes.c_float(eps), T, H,
                              _ptr(y), _ptr(h), fmt, _ptr(q), _ptr(sf), layout, _ptr(amax))
     return y, h, q, sf[:n_sf]
+
+
+def rank_sum(xs, lib=None) -> np.ndarray:
+    """The AllReduce of same-shape uint16 (bf16 bits) rank inputs (R15)."""
+    lib = lib or load()
+    xs = [np.ascontiguousarray(x) for x in xs]
+    assert xs and all(x.dtype == np.uint16 and x.shape == xs[0].shape for x in xs)
+    out = np.zeros(xs[0].shape, dtype=np.uint16)
+    table = (ctypes.c_void_p * len(xs))(*[x.ctypes.data for x in xs])
+    lib.qzo_rank_sum(table, len(xs), out.size, _ptr(out))
+    return out
+
+
+def allreduce_rmsnorm_quantize(xs, r, gamma, eps, fmt, layout, amax_in=None, lib=None):
+    """The fused epilogue on the AllReduce of the rank inputs ``xs``:
+    ``rmsnorm_quantize`` applied to ``rank_sum(xs)``.  Returns (y, h, q, sf)."""
+    lib = lib or load()
+    return rmsnorm_quantize(rank_sum(xs, lib), r, gamma, eps, fmt, layout, amax_in, lib)
 
 
 def quantize_grouped(experts, fmt: int, layout: int, mode: int = NVFP4_PER_ROW,

@@ -48,6 +48,8 @@
  *  R14 Fused gate|up split: rows [0, cut) and [cut, rows), scales cut with
  *     their rows and laid out anew per part; a scale block that covers rows
  *     on both sides of the cut is refused.
+ *  R15 AllReduce ahead of the epilogue: the reduced element is the bf16
+ *     rounding of a binary32 sum taken in rank order, identical on every rank.
  */
 #include <math.h>
 #include <stdint.h>
@@ -417,6 +419,23 @@ void qzo_rmsnorm_quantize(const uint16_t *x, const uint16_t *res, const uint16_t
     qzo_residual_rmsnorm(x, res, gamma, eps, T, H, y, h);
     if (fmt == 0) qzo_quantize_mxfp8(y, T, H, H, q, sf, layout);
     else qzo_quantize_nvfp4(y, T, H, H, q, sf, layout, 0, amax);
+}
+
+/* ------------------------------------------------------------------------- */
+/* The AllReduce that opens the epilogue ([LSF] commit 2 and [CAR] commit 6:  */
+/* the tensor-parallel AllReduce hands the epilogue its input x).             */
+/*   R15 out[i] = bf16(acc), acc = x_0[i], then acc = RN32(acc + x_r[i]) for  */
+/*       r = 1 .. n-1 (binary32, rank order), so that every rank reduces to   */
+/*       the same bits; the epilogue above then runs on out as its x.         */
+/*   xs : n pointers to bf16 arrays of count elements                         */
+/* ------------------------------------------------------------------------- */
+void qzo_rank_sum(const uint16_t *const *xs, int n, int64_t count, uint16_t *out)
+{
+    for (int64_t i = 0; i < count; i++) {
+        float acc = qzo_bf16_value(xs[0][i]);
+        for (int r = 1; r < n; r++) acc = acc + qzo_bf16_value(xs[r][i]);
+        out[i] = qzo_bf16_from_double((double)acc);
+    }
 }
 
 /* ------------------------------------------------------------------------- */

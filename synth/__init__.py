@@ -16,6 +16,8 @@ shapes and a plausible value distribution):
 * row-scaled NVFP4 split: [16384, 4096] N(0,1) with 1% outliers x20; rows
   split over 64 experts by multinomial(Dirichlet(0.3))
 * fused residual + RMSNorm: x, r [T, 7168] N(0,1), gamma U(0.5, 1.5), eps 1e-6
+* AllReduce epilogue: the fused workload's x as the sum of n rank partials,
+  each N(0, 1/n) [T, 7168] (a row-parallel projection's partial outputs)
 * Qwen3-235B-A22B prequant: 128 experts/layer, gate_up [3072, 4096] and down
   [4096, 1536], N(0, 0.02), 94 layers, seed 5 + layer
 """
@@ -96,6 +98,18 @@ def fused_norm_inputs(tokens: int, hidden=FUSED_NORM["hidden"], seed=FUSED_NORM[
     r = torch.randn(tokens, hidden, generator=g, device=device, dtype=torch.float32).to(torch.bfloat16)
     gamma = (torch.rand(hidden, generator=g, device=device, dtype=torch.float32) + 0.5).to(torch.bfloat16)
     return x, r, gamma
+
+
+def rank_partials(ranks: int, tokens: int, hidden=FUSED_NORM["hidden"], seed=FUSED_NORM["seed"], device="cpu"):
+    """``ranks`` partial inputs ~ N(0, 1/ranks) [tokens, hidden] of a tensor-parallel
+    AllReduce (their sum is distributed like the fused workload's x), plus the
+    residual ~ N(0,1) and gamma ~ U(0.5, 1.5); all bf16."""
+    g = _gen(seed + 1000 * ranks, device)
+    xs = [(torch.randn(tokens, hidden, generator=g, device=device, dtype=torch.float32) / ranks ** 0.5)
+          .to(torch.bfloat16) for _ in range(ranks)]
+    r = torch.randn(tokens, hidden, generator=g, device=device, dtype=torch.float32).to(torch.bfloat16)
+    gamma = (torch.rand(hidden, generator=g, device=device, dtype=torch.float32) + 0.5).to(torch.bfloat16)
+    return xs, r, gamma
 
 
 def random_finite_bf16(shape, seed: int = 0, device="cpu") -> torch.Tensor:

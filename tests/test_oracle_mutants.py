@@ -20,7 +20,7 @@ import oracle
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 PIN_FILES = ["tests/test_oracle_formats.py", "tests/test_oracle_mxfp8.py", "tests/test_oracle_layout.py",
              "tests/test_oracle_nvfp4.py", "tests/test_oracle_norm.py", "tests/test_oracle_dequant.py",
-             "tests/test_oracle_merge.py", "tests/test_oracle_split.py"]
+             "tests/test_oracle_merge.py", "tests/test_oracle_split.py", "tests/test_oracle_allreduce.py"]
 
 MUTANTS = {
     "ties_away_from_even": ("return (fmod(f, 2.0) == 0.0) ? f : f + 1.0;", "return f + 1.0;"),
@@ -69,6 +69,12 @@ MUTANTS = {
     "split_amax_not_shared": ("if (amax_kind == 1) ao[p][0] = amax[0];",
                               "if (amax_kind == 1 && p == 0) ao[p][0] = amax[0];"),
     "split_block_scale_rows_floor": ("int64_t srows = (count[p] + 127) / 128;", "int64_t srows = count[p] / 128;"),
+    "rank_sum_binary64": ("float acc = qzo_bf16_value(xs[0][i]);", "double acc = qzo_bf16_value(xs[0][i]);"),
+    "rank_sum_drops_last_rank": ("for (int r = 1; r < n; r++) acc", "for (int r = 1; r < n - 1; r++) acc"),
+    "rank_sum_reverse_order": ("float acc = qzo_bf16_value(xs[0][i]);\n        for (int r = 1; r < n; r++) acc",
+                               "float acc = qzo_bf16_value(xs[n - 1][i]);\n        for (int r = n - 2; r >= 0; r--) acc"),
+    "rank_sum_first_rank_only": ("out[i] = qzo_bf16_from_double((double)acc);",
+                                 "out[i] = xs[0][i];"),
     "bf16_double_rounding": ("double n = round_half_even(a / step);\n    double r = n * step;",
                              "double n = round_half_even((double)(float)a / step);\n    double r = n * step;"),
 }
