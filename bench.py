@@ -14,8 +14,11 @@ kernel (bytes per launch over its CUDA-event duration, against the measured
 HBM copy bandwidth), an end-to-end figure through the same C ABI with the
 inputs coming from pinned host memory, the CPU oracle timed on a bounded
 sample, SM clocks sampled during the timed region, and (``extra``) the other
-workloads: the row-scaled NVFP4 split activation, the fused residual +
-RMSNorm + quantize sweep and a Qwen3-235B-A22B layer in MXFP8 and NVFP4.
+workloads: the tiny MXFP8 group, the row-scaled NVFP4 split activation, the
+fused residual + RMSNorm + quantize sweep and its AllReduce form over 8 rank
+buffers, the Qwen3-30B-A3B gate_up layer in NVFP4, a Qwen3-235B-A22B layer in
+MXFP8 and NVFP4, dequantization, column-wise quantization, the attention
+decode merge and the gate|up split.
 
 With torchrun (N > 1) every rank quantizes its own full workload on its own
 GPU (weak scaling, no collective on the data path); the time is the maximum
@@ -70,6 +73,7 @@ KERNEL_SOURCES = {
     "nvfp4_compute_l2_kernel": ("qz_grouped.cu", "qz_device.cuh"),
     "nvfp4_rows_kernel": ("qz_rows.cu", "qz_device.cuh"),
     "rmsnorm_quant_kernel": ("qz_rmsnorm.cu", "qz_device.cuh"),
+    "rmsnorm_quant_kernel_multi": ("qz_rmsnorm.cu", "qz_device.cuh"),   # the AllReduce instantiation
     "dequant_kernel": ("qz_dequant.cu", "qz_device.cuh"),
     "attention_merge_kernel": ("qz_merge.cu", "qz_device.cuh"),
     "colwise_kernel": ("qz_colwise.cu", "qz_device.cuh", "qz_async.cuh"),
@@ -434,7 +438,8 @@ class L2Flush:
 
 
 def extra_workloads(qz, device, stream, peak,
-                    which=("tiny", "split", "fused", "nvfp4", "large", "dequant", "merge", "colwise", "gateup"),
+                    which=("tiny", "split", "fused", "nvfp4", "large", "dequant", "merge", "colwise", "gateup",
+                           "allreduce"),
                     tokens=None, experts=None):
     out = []
     flush = L2Flush(device)
@@ -464,6 +469,8 @@ def extra_workloads(qz, device, stream, peak,
         _extra_colwise(qz, device, rec)
     if "gateup" in which:
         _extra_gate_up_split(qz, device, rec)
+    if "allreduce" in which:
+        _extra_allreduce(qz, device, out, peak, tokens)
     return out
 
 
@@ -775,6 +782,51 @@ def _extra_merge(qz, device, flush, out, peak, tokens=None):
                 "frac_of_hbm_peak_fused_T4096": round(big["fused_GB/s"] / peak, 4) if big["T"] == 4096 else None})
 
 
+def _extra_allreduce(qz, device, out, peak, tokens=None, ranks=8):
+    """AllReduce epilogue, one-shot form: the sum of 8 rank inputs + residual
+    add + RMSNorm + MXFP8 (swizzled), H = 7168, T swept 1..4096.  With one GPU
+    the 8 rank inputs are 8 buffers in this GPU's HBM, read through the same
+    plain pointers a peer mapping would give: the HBM-side cost of the kernel.
+    From T = 1024 on, buffer sets are used round-robin so that a call's bytes
+    were last touched more than twice the L2 size ago; below, calls repeat on
+    the same buffers."""
+    H = synth.FUSED_NORM["hidden"]
+    L2 = 126 * 2 ** 20
+    fmt, layout = qz.FMT_MXFP8, qz.SF_SWIZZLED
+    sweep = []
+    for Tn in (tokens or (1, 16, 64, 512, 4096)):
+        nbytes = (ranks + 1) * Tn * H * 2 + 2 * H + Tn * H * (2 + 2 + 1) + qz.sf_bytes(Tn, H, fmt, layout)
+        copies = 1 if Tn < 1024 else -(-2 * L2 // nbytes) + 1
+        xs, r, g = synth.rank_partials(ranks, Tn, device=device)
+        sets = []
+        for c in range(copies):
+            sets.append(([x if c == 0 else x.clone() for x in xs], r if c == 0 else r.clone(),
+                         [(torch.empty_like(r), torch.empty_like(r),
+                           torch.empty((Tn, H), dtype=torch.uint8, device=device),
+                           torch.empty(max(qz.sf_bytes(Tn, H, fmt, layout), 16), dtype=torch.uint8,
+                                       device=device))]))
+        turn = [0]
+
+        def call():
+            xs_, r_, d_ = sets[turn[0] % copies]
+            turn[0] += 1
+            qz.allreduce_rmsnorm_quantize(xs_, r_, g, 1e-6, d_, fmt, layout, Tn, H)
+
+        ms = _time_graph(call, reps=10 * copies) if Tn >= 1024 else _time_graph(call, reps=50)
+        sweep.append({"T": Tn, "us": round(ms * 1e3, 2), "GB/s": round(nbytes / (ms / 1e3) / GB, 1),
+                      "bytes_per_call": int(nbytes), "copies": copies})
+        del sets, xs, r, g
+    big = sweep[-1]
+    out.append({"workload": f"AllReduce epilogue (one-shot): sum of {ranks} rank inputs + residual + RMSNorm + "
+                            "MXFP8 swizzled, H=7168, T=1..4096 (residual_out written); the rank inputs are "
+                            "buffers on this one GPU",
+                "kernel": "rmsnorm_quant_kernel_multi", "sweep": sweep,
+                "timing": "CUDA graph of 50 calls on the same buffers (T < 1024) or of 10 rounds over "
+                          "`copies` buffer sets (T >= 1024, inputs larger than L2, no flush)",
+                "frac_of_hbm_peak_T4096": round(big["GB/s"] / peak, 4) if big["T"] == 4096 else None,
+                "traffic_T4096": ncu_traffic("rmsnorm_quant_kernel_multi")})
+
+
 # ---------------------------------------------------------------------------
 # CPU oracle timing (the reference arm and the cpu_baseline key)
 # ---------------------------------------------------------------------------
@@ -848,13 +900,13 @@ def main():
                          "(the default run), 3 the row-scaled NVFP4 split activation, 4 the fused residual + "
                          "RMSNorm sweep, 5 the Qwen3-235B-A22B layer")
     ap.add_argument("--only", choices=["tiny", "split", "fused", "nvfp4", "large", "dequant", "merge", "colwise",
-                                       "gateup"],
+                                       "gateup", "allreduce"],
                     default=None,
                     help="time only this secondary workload and print its record (profiling aid)")
     ap.add_argument("--experts", type=int, default=None,
                     help="experts per call of the Qwen3-235B-A22B workload (default 128; fewer for a profiler capture)")
     ap.add_argument("--tokens", type=str, default=None,
-                    help="comma-separated token counts for the fused sweep (default: 1..4096)")
+                    help="comma-separated token counts for the fused, merge and AllReduce sweeps")
     args = ap.parse_args()
     if args.config is not None and args.config != 2:
         args.only = {1: "tiny", 3: "split", 4: "fused", 5: "large"}[args.config]

@@ -269,6 +269,54 @@ qz_status qz_rmsnorm_quantize(const void *d_x, const void *d_residual, const voi
                               int fmt, void *d_q, uint8_t *d_sf, int layout,
                               const float *d_global_amax, void *stream);
 
+/* Largest number of rank inputs, and of destinations, of
+ * qz_allreduce_rmsnorm_quantize (one tensor-parallel group of an NVLink node). */
+#define QZ_MAX_RANKS 8
+
+/* One destination of the AllReduce epilogue's outputs.  Device pointers: this
+ * GPU's memory or a peer GPU's buffer mapped into this process. */
+typedef struct qz_norm_dest {
+    void *norm_out;     /* bf16 [T, H], 16-byte aligned */
+    void *residual_out; /* bf16 [T, H], 16-byte aligned, or NULL (not written) */
+    void *q;            /* e4m3 [T, H] (MXFP8) or packed e2m1 [T, H/2] (NVFP4), 8-byte aligned */
+    uint8_t *sf;        /* SF region of T rows: qz_sf_bytes(T, H, fmt, layout) bytes, aligned as in
+                           qz_rmsnorm_quantize */
+} qz_norm_dest;
+
+/* The fused epilogue behind a tensor-parallel AllReduce ([LSF] commits 2, 3 and
+ * [CAR] commit 6: the AllReduce that ends an attention or MoE block already
+ * holds the sum the norm reads, and emits the quantized norm from the same
+ * pass).  For the rows [row_begin, row_end):
+ *   x = bf16(sum over ranks of rank_x[r]), summed in binary32 in rank order
+ *       0 .. n_ranks-1 (rank 0 exact, one rounding per further rank) and
+ *       rounded once to bf16 (nearest-even), so every rank obtains the same bits
+ *   then exactly qz_rmsnorm_quantize on x: h = bf16(x + residual), y, q, sf,
+ * and every output row is written to each of the n_dests destinations.  One
+ * call with rows [0, T) and this GPU's buffers as its single destination is the
+ * one-shot form; a call per rank on its own slice with every rank's buffers as
+ * destinations is the reduce-scatter + all-gather form.  The slice with
+ * row_end == T also zeroes the swizzled layout's invented rows T .. pad(T,128)-1
+ * of every destination.
+ *   rank_x : HOST array of n_ranks device pointers, each to bf16 [T, H]
+ *            (16-byte aligned; this GPU's memory or a peer mapping)
+ *   dests  : HOST array of n_dests destinations
+ * Both host arrays are read during the call only.  The kernel reads the ranks'
+ * inputs with plain loads and writes the destinations with plain stores; it
+ * never waits on another GPU.  The caller orders the exchange: every rank's
+ * input is complete, and every destination free to be written, before this
+ * call starts on the stream (a cross-rank barrier), and no rank overwrites its
+ * input or reads a peer-written destination until every rank's call has
+ * finished (a second barrier).
+ * Errors: as qz_rmsnorm_quantize, plus QZ_ERR_INVALID_ARG for n_ranks or
+ * n_dests outside 1 .. QZ_MAX_RANKS, NULL arrays or entries, and a row range
+ * outside 0 <= row_begin <= row_end <= T; QZ_ERR_ALIGNMENT for any misaligned
+ * entry.  An empty range launches nothing unless it must zero invented rows. */
+qz_status qz_allreduce_rmsnorm_quantize(const void *const *rank_x, int n_ranks, const void *d_residual,
+                                        const void *d_gamma, float eps, int64_t T, int64_t H,
+                                        int64_t row_begin, int64_t row_end,
+                                        const qz_norm_dest *dests, int n_dests, int fmt, int layout,
+                                        const float *d_global_amax, void *stream);
+
 /* Linear -> swizzled 128x4 conversion of n SF matrices in one launch, padding
  * written as 0x00 ([MX] Summary; [CAR] commit 5: swizzled and linear agree).
  * Errors: QZ_ERR_INVALID_ARG for n < 0, n > QZ_MAX_EXPERTS or a NULL table

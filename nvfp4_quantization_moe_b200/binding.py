@@ -30,6 +30,7 @@ DERR_SHAPE, DERR_NULL, DERR_ALIGN, DERR_TOO_LARGE = 0x1, 0x2, 0x4, 0x8
 DERR_CUT = 0x20
 MAX_EXPERTS = 4096
 MAX_HIDDEN = 16384
+MAX_RANKS = 8
 
 EXPORTED = (
     "qz_sf_bytes",
@@ -45,6 +46,7 @@ EXPORTED = (
     "qz_attention_merge_quantize",
     "qz_quantize_grouped_colwise",
     "qz_split_fused_experts",
+    "qz_allreduce_rmsnorm_quantize",
 )
 STATIC_WS_MAX_EXPERTS = 1024
 
@@ -127,6 +129,9 @@ def load(path: str = LIB_PATH):
         lib.qz_attention_merge_quantize.argtypes = [P, P, I, i64, i64, P, P, P, I, P]
         lib.qz_split_fused_experts.restype = I
         lib.qz_split_fused_experts.argtypes = [P, I, I, I, I, I, P, P]
+        lib.qz_allreduce_rmsnorm_quantize.restype = I
+        lib.qz_allreduce_rmsnorm_quantize.argtypes = [P, I, P, P, ctypes.c_float, i64, i64, i64, i64, P, I, I, I,
+                                                      P, P]
         _lib = lib
         return lib
 
@@ -376,6 +381,36 @@ def rmsnorm_quantize(x, residual, gamma, eps: float, norm_out, residual_out, fmt
                                       int(fmt), ctypes.c_void_p(_ptr(q)), ctypes.c_void_p(_ptr(sf)), int(layout),
                                       ctypes.c_void_p(_ptr(global_amax)), _stream_ptr(stream)),
            "qz_rmsnorm_quantize")
+
+
+class NormDest(ctypes.Structure):
+    """One destination of the AllReduce epilogue (struct qz_norm_dest)."""
+    _fields_ = [("norm_out", ctypes.c_void_p), ("residual_out", ctypes.c_void_p), ("q", ctypes.c_void_p),
+                ("sf", ctypes.c_void_p)]
+
+
+def _addr(t) -> int:
+    """A tensor's device address, or an address given as an int (a peer mapping)."""
+    return int(t) if isinstance(t, int) else _ptr(t)
+
+
+def allreduce_rmsnorm_quantize(rank_x, residual, gamma, eps: float, dests, fmt: int, layout: int, T: int, H: int,
+                               rows=None, global_amax=None, stream=None):
+    """AllReduce of the rank inputs + residual add + RMSNorm + quantize
+    (qz_allreduce_rmsnorm_quantize).  ``rank_x``: bf16 [T, H] tensors or device
+    addresses (peer mappings), summed in this order; ``dests``: tuples
+    (norm_out, residual_out or None, q, sf) of tensors or addresses, each
+    written with the rows ``rows`` = (row_begin, row_end), default all T.
+    Every pointer argument takes a tensor, an int address or None."""
+    row_begin, row_end = (0, T) if rows is None else rows
+    xs = (ctypes.c_void_p * len(rank_x))(*[_addr(x) for x in rank_x])
+    ds = (NormDest * len(dests))(*[NormDest(*[_addr(p) for p in d]) for d in dests])
+    _check(load().qz_allreduce_rmsnorm_quantize(
+        ctypes.cast(xs, ctypes.c_void_p), len(rank_x), ctypes.c_void_p(_addr(residual)),
+        ctypes.c_void_p(_addr(gamma)), ctypes.c_float(eps), int(T), int(H), int(row_begin), int(row_end),
+        ctypes.cast(ds, ctypes.c_void_p), len(dests), int(fmt), int(layout), ctypes.c_void_p(_addr(global_amax)),
+        _stream_ptr(stream)),
+        "qz_allreduce_rmsnorm_quantize")
 
 
 def dequantize_grouped(table: DqTable, fmt: int, per_row: bool, layout: int, stream=None, err=None,

@@ -19,6 +19,10 @@ cudaError_t launch_swizzle(const qz_sf_pair* table, int n, int grid, cudaStream_
 cudaError_t launch_rmsnorm_quant(const uint16_t* x, const uint16_t* r, const uint16_t* g, float eps, int64_t T,
                                  int64_t H, uint16_t* y, uint16_t* h, int fmt, uint8_t* q, uint8_t* sf, int layout,
                                  const float* amax, cudaStream_t s, bool latency_mode);
+cudaError_t launch_allreduce_norm_quant(const uint16_t* const* xs, int n_x, const uint16_t* r, const uint16_t* g,
+                                        float eps, int64_t T, int64_t H, int64_t row_begin, int64_t row_end,
+                                        const qz_norm_dest* dsts, int n_dst, int fmt, int layout, const float* amax,
+                                        cudaStream_t s, bool latency_mode);
 int grouped_blocks_per_sm(int which, int n);
 size_t workspace_bytes(int n);
 cudaError_t launch_nvfp4_compute_l2(const qz_expert* table, int n, int layout, int grid, unsigned* ws,
@@ -205,6 +209,42 @@ qz_status qz_rmsnorm_quantize(const void* d_x, const void* d_residual, const voi
         static_cast<const uint16_t*>(d_gamma), eps, T, H, static_cast<uint16_t*>(d_norm_out),
         static_cast<uint16_t*>(d_residual_out), fmt, static_cast<uint8_t*>(d_q), d_sf, layout, d_global_amax,
         (cudaStream_t)stream, latency_mode));
+}
+
+qz_status qz_allreduce_rmsnorm_quantize(const void* const* rank_x, int n_ranks, const void* d_residual,
+                                        const void* d_gamma, float eps, int64_t T, int64_t H, int64_t row_begin,
+                                        int64_t row_end, const qz_norm_dest* dests, int n_dests, int fmt,
+                                        int layout, const float* d_global_amax, void* stream) {
+    if (fmt != QZ_FMT_MXFP8 && fmt != QZ_FMT_NVFP4) return QZ_ERR_INVALID_ARG;
+    if (!valid_layout(layout)) return QZ_ERR_INVALID_ARG;
+    if (n_ranks < 1 || n_ranks > QZ_MAX_RANKS || n_dests < 1 || n_dests > QZ_MAX_RANKS) return QZ_ERR_INVALID_ARG;
+    if (!rank_x || !dests) return QZ_ERR_INVALID_ARG;
+    const int64_t block = fmt == QZ_FMT_MXFP8 ? 32 : 16;
+    if (T < 0 || H <= 0 || H > QZ_MAX_HIDDEN || H % block != 0) return QZ_ERR_INVALID_ARG;
+    if (T > 0x7FFFFF00LL) return QZ_ERR_INVALID_ARG;
+    if (row_begin < 0 || row_begin > row_end || row_end > T) return QZ_ERR_INVALID_ARG;
+    if (layout == QZ_SF_SWIZZLED_128x4 && (H / block) % 4 != 0) return QZ_ERR_UNSUPPORTED;
+    if (T == 0) return QZ_OK;
+    if (!d_residual || !d_gamma || (fmt == QZ_FMT_NVFP4 && !d_global_amax)) return QZ_ERR_INVALID_ARG;
+    for (int i = 0; i < n_ranks; ++i)
+        if (!rank_x[i]) return QZ_ERR_INVALID_ARG;
+    for (int d = 0; d < n_dests; ++d)
+        if (!dests[d].norm_out || !dests[d].q || !dests[d].sf) return QZ_ERR_INVALID_ARG;
+    if (!aligned(d_residual, 16) || !aligned(d_gamma, 16)) return QZ_ERR_ALIGNMENT;
+    if (d_global_amax && !aligned(d_global_amax, 4)) return QZ_ERR_ALIGNMENT;
+    for (int i = 0; i < n_ranks; ++i)
+        if (!aligned(rank_x[i], 16)) return QZ_ERR_ALIGNMENT;
+    for (int d = 0; d < n_dests; ++d) {
+        const qz_norm_dest& o = dests[d];
+        if (!aligned(o.norm_out, 16) || (o.residual_out && !aligned(o.residual_out, 16)) || !aligned(o.q, 8) ||
+            !aligned(o.sf, layout == QZ_SF_SWIZZLED_128x4 ? 16 : 4))
+            return QZ_ERR_ALIGNMENT;
+    }
+    const bool latency_mode = row_end - row_begin <= 2 * (int64_t)device_sms();
+    return from_cuda(qz::launch_allreduce_norm_quant(
+        reinterpret_cast<const uint16_t* const*>(rank_x), n_ranks, static_cast<const uint16_t*>(d_residual),
+        static_cast<const uint16_t*>(d_gamma), eps, T, H, row_begin, row_end, dests, n_dests, fmt, layout,
+        d_global_amax, (cudaStream_t)stream, latency_mode));
 }
 
 qz_status qz_swizzle_scales(const qz_sf_pair* d_table, int n, void* stream, const qz_launch_opts* opts) {

@@ -22,11 +22,39 @@
 //            store y, then quantize y exactly like the grouped kernels.
 // A block of 32 (MXFP8) or 16 (NVFP4) elements is 4 or 2 consecutive chunks,
 // which sit in consecutive threads, so block amax is a butterfly shuffle.
+//
+// The same kernel, instantiated with MULTI, opens with the tensor-parallel
+// AllReduce that feeds the epilogue (the "AllReduce epilogue" of both pages):
+// x is the sum of up to eight rank inputs, read through plain pointers that
+// may be peer mappings of other GPUs' buffers, accumulated in binary32 in rank
+// order and rounded once to bf16, so every rank reduces to the same bits.  It
+// takes a row range (one rank's slice, or all rows) and writes every output to
+// up to eight destinations (the ranks' own buffers, for the all-gather half).
 #include "qz_device.cuh"
 
 namespace qz {
 
 constexpr int kNormMaxThreads = 1024;
+constexpr int kMaxRanks = QZ_MAX_RANKS;
+
+struct NormDst {
+    uint16_t* y;   // norm_out, bf16 [T, H]
+    uint16_t* h;   // residual_out, bf16 [T, H], nullable
+    uint8_t* q;    // payload of T rows
+    uint8_t* sf;   // SF region of T rows
+};
+
+struct NormArgs {
+    const uint16_t* x[kMaxRanks];  // rank inputs, bf16 [T, H] each
+    NormDst dst[kMaxRanks];
+    const uint16_t* res;           // residual bf16 [T, H]
+    const uint16_t* gamma;         // bf16 [H]
+    const float* global_amax;      // NVFP4 per-tensor amax
+    int64_t T, H;
+    int64_t row0;                  // first row of this launch (CTA b runs row row0 + b)
+    float eps;
+    int n_x, n_dst;
+};
 
 // bf16 (nearest-even) of hi + e, where |e| <= half an ulp of hi: the rounding
 // of hi decides unless hi sits exactly on a bf16 midpoint, where e breaks the tie.
@@ -90,35 +118,93 @@ __device__ __forceinline__ void two_sum_add(float& sh, float& sl, float t) {
 // Thread limit of an instance with CPT chunks per thread (register budget).
 __host__ __device__ constexpr int norm_max_threads(int cpt) { return cpt <= 2 ? 1024 : (cpt == 4 ? 512 : 256); }
 
-template <int FMT, int LAYOUT, int CPT>
-__global__ void __launch_bounds__(norm_max_threads(CPT)) rmsnorm_quant_kernel(
-    const uint16_t* __restrict__ x, const uint16_t* __restrict__ res, const uint16_t* __restrict__ gamma, float eps,
-    int64_t T, int64_t H, uint16_t* __restrict__ norm_out, uint16_t* __restrict__ res_out, uint8_t* __restrict__ q,
-    uint8_t* __restrict__ sf, const float* __restrict__ global_amax) {
+// bf16x2 words of the rank sum of chunks t + nt*i of one row: binary32
+// accumulation in rank order (rank 0 exactly, then one rounding per rank), one
+// bf16 rounding at the end.  Ranks are loaded two at a time so that two
+// chunks' loads per rank pair are in flight before either is added.
+template <int CPT>
+__device__ __forceinline__ void rank_sum_row(const NormArgs& a, int64_t row, int nch, int t, int nt,
+                                             uint4 (&h)[CPT]) {
+    float acc[CPT][8];
+    uint4 v[CPT], w[CPT];
+#pragma unroll
+    for (int i = 0; i < CPT; ++i) {
+        const int c = i * nt + t;
+        v[i] = c < nch ? ld_stream(a.x[0] + row * a.H + c * 8) : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int i = 0; i < CPT; ++i) {
+        const uint32_t* vw = reinterpret_cast<const uint32_t*>(&v[i]);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            acc[i][2 * j] = bf16_lo(vw[j]);
+            acc[i][2 * j + 1] = bf16_hi(vw[j]);
+        }
+    }
+    for (int r = 1; r < a.n_x; r += 2) {
+        const bool two = r + 1 < a.n_x;
+#pragma unroll
+        for (int i = 0; i < CPT; ++i) {
+            const int c = i * nt + t;
+            v[i] = c < nch ? ld_stream(a.x[r] + row * a.H + c * 8) : make_uint4(0, 0, 0, 0);
+            w[i] = (two && c < nch) ? ld_stream(a.x[r + 1] + row * a.H + c * 8) : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int i = 0; i < CPT; ++i) {
+            const uint32_t* vw = reinterpret_cast<const uint32_t*>(&v[i]);
+            const uint32_t* ww = reinterpret_cast<const uint32_t*>(&w[i]);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                acc[i][2 * j] = __fadd_rn(acc[i][2 * j], bf16_lo(vw[j]));
+                acc[i][2 * j + 1] = __fadd_rn(acc[i][2 * j + 1], bf16_hi(vw[j]));
+            }
+            if (two) {
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    acc[i][2 * j] = __fadd_rn(acc[i][2 * j], bf16_lo(ww[j]));
+                    acc[i][2 * j + 1] = __fadd_rn(acc[i][2 * j + 1], bf16_hi(ww[j]));
+                }
+            }
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < CPT; ++i) {
+        uint32_t* hw = reinterpret_cast<uint32_t*>(&h[i]);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) hw[j] = cvt_bf16x2(acc[i][2 * j], acc[i][2 * j + 1]);
+    }
+}
+
+// MULTI == false: one input, one destination, row0 == 0 (qz_rmsnorm_quantize).
+template <int FMT, int LAYOUT, int CPT, bool MULTI>
+__global__ void __launch_bounds__(norm_max_threads(CPT)) rmsnorm_quant_kernel(const __grid_constant__ NormArgs a) {
     constexpr int BLOCK = (FMT == QZ_FMT_MXFP8) ? 32 : 16;
     constexpr int CPB = BLOCK / 8;  // chunks per scale block
     const int t = threadIdx.x, lane = t & 31, nt = blockDim.x;
-    const int64_t row = blockIdx.x;
+    const int64_t T = a.T, H = a.H;
+    const int64_t row = (MULTI ? a.row0 : 0) + blockIdx.x;
     const int nch = (int)(H >> 3);
     const int kv = (int)(H / BLOCK);
+    const int n_dst = MULTI ? a.n_dst : 1;
 
     if (row >= T) {
         // an invented row of the swizzled layout: zero scale bytes (kv % 4 == 0)
-        for (int k0 = 4 * t; k0 < kv; k0 += 4 * nt) st_u32(sf + swz_offset(row, k0, kv), 0u);
+        for (int d = 0; d < n_dst; ++d)
+            for (int k0 = 4 * t; k0 < kv; k0 += 4 * nt) st_u32(a.dst[d].sf + swz_offset(row, k0, kv), 0u);
         return;
     }
 
-    const uint16_t* xr = x + row * H;
-    const uint16_t* rr = res + row * H;
+    const uint16_t* rr = a.res + row * H;
     uint4 h[CPT], rv[CPT], gv[CPT];
 #pragma unroll
     for (int i = 0; i < CPT; ++i) {
         const int c = i * nt + t;
         const bool ok = c < nch;
-        h[i] = ok ? ld_stream(xr + c * 8) : make_uint4(0, 0, 0, 0);
+        if (!MULTI) h[i] = ok ? ld_stream(a.x[0] + row * H + c * 8) : make_uint4(0, 0, 0, 0);
         rv[i] = ok ? ld_stream(rr + c * 8) : make_uint4(0, 0, 0, 0);
-        gv[i] = ok ? __ldg(reinterpret_cast<const uint4*>(gamma + c * 8)) : make_uint4(0, 0, 0, 0);
+        gv[i] = ok ? __ldg(reinterpret_cast<const uint4*>(a.gamma + c * 8)) : make_uint4(0, 0, 0, 0);
     }
+    if (MULTI) rank_sum_row<CPT>(a, row, nch, t, nt, h);
     float sh = 0.0f, sl = 0.0f;
 #pragma unroll
     for (int i = 0; i < CPT; ++i) {
@@ -129,12 +215,14 @@ __global__ void __launch_bounds__(norm_max_threads(CPT)) rmsnorm_quant_kernel(
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
             hw[j] = add_bf16x2(hw[j], rw[j]);
-            const float a = bf16_lo(hw[j]), b = bf16_hi(hw[j]);
-            cs = __fmaf_rn(a, a, cs);  // a * a is exact; one rounding per add
-            cs = __fmaf_rn(b, b, cs);
+            const float a0 = bf16_lo(hw[j]), b0 = bf16_hi(hw[j]);
+            cs = __fmaf_rn(a0, a0, cs);  // a0 * a0 is exact; one rounding per add
+            cs = __fmaf_rn(b0, b0, cs);
         }
         two_sum_add(sh, sl, cs);
-        if (res_out && c < nch) st_v4(res_out + row * H + c * 8, h[i]);
+        if (c < nch)
+            for (int d = 0; d < n_dst; ++d)
+                if (a.dst[d].h) st_v4(a.dst[d].h + row * H + c * 8, h[i]);
     }
 
     // CTA reduction of the sum of squares in binary64
@@ -148,12 +236,12 @@ __global__ void __launch_bounds__(norm_max_threads(CPT)) rmsnorm_quant_kernel(
     __syncthreads();
     double tot = 0.0;
     for (int w = 0; w < (nt >> 5); ++w) tot += s_red[w];
-    const double rstd = 1.0 / sqrt(tot / (double)H + (double)eps);
+    const double rstd = 1.0 / sqrt(tot / (double)H + (double)a.eps);
     const float rh = (float)rstd;
     const float rl = (float)(rstd - (double)rh);
 
     float S = 0.0f;
-    if (FMT == QZ_FMT_NVFP4) S = nvfp4_encode_scale(__ldg(global_amax));
+    if (FMT == QZ_FMT_NVFP4) S = nvfp4_encode_scale(__ldg(a.global_amax));
 
 #pragma unroll
     for (int i = 0; i < CPT; ++i) {
@@ -166,7 +254,8 @@ __global__ void __launch_bounds__(norm_max_threads(CPT)) rmsnorm_quant_kernel(
 #pragma unroll
         for (int j = 0; j < 4; ++j)
             yw[j] = y_pair(__fmul_rn(bf16_lo(hw[j]), bf16_lo(gw[j])), __fmul_rn(bf16_hi(hw[j]), bf16_hi(gw[j])), rh, rl);
-        if (c < nch) st_v4(norm_out + row * H + c * 8, y);
+        if (c < nch)
+            for (int d = 0; d < n_dst; ++d) st_v4(a.dst[d].y + row * H + c * 8, y);
 
         // quantize y
         uint32_t m = absmax_bits(y);
@@ -176,12 +265,14 @@ __global__ void __launch_bounds__(norm_max_threads(CPT)) rmsnorm_quant_kernel(
             m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
             scale = e8m0_byte(m);
             const uint2 codes = e4m3x8_scaled(y, e8m0_reciprocal(scale));
-            if (c < nch) st_v2(q + row * H + c * 8, codes.x, codes.y);
+            if (c < nch)
+                for (int d = 0; d < n_dst; ++d) st_v2(a.dst[d].q + row * H + c * 8, codes.x, codes.y);
         } else {
             const Nvfp4Block blk = nvfp4_block(bits_to_float_bf16(m), S, s_inv);
             scale = blk.scale;
             const uint32_t codes = e2m1x8_scaled(y, blk.rcp);
-            if (c < nch) st_u32(q + row * (H >> 1) + c * 4, codes);
+            if (c < nch)
+                for (int d = 0; d < n_dst; ++d) st_u32(a.dst[d].q + row * (H >> 1) + c * 4, codes);
         }
         // scale bytes of 4 consecutive blocks: threads base, base+CPB, base+2CPB, base+3CPB
         const uint32_t s1 = __shfl_down_sync(0xFFFFFFFFu, scale, CPB);
@@ -190,49 +281,95 @@ __global__ void __launch_bounds__(norm_max_threads(CPT)) rmsnorm_quant_kernel(
         if ((lane & (4 * CPB - 1)) == 0 && c < nch) {
             const int k0 = c / CPB;
             const uint32_t word = scale | (s1 << 8) | (s2 << 16) | (s3 << 24);
-            if (LAYOUT == QZ_SF_SWIZZLED_128x4) {
-                st_u32(sf + swz_offset(row, k0, kv), word);
-            } else {
-                const int64_t base = row * kv + k0;
-                if (k0 + 4 <= kv && (base & 3) == 0) st_u32(sf + base, word);
-                else for (int j = 0; j < 4 && k0 + j < kv; ++j) sf[base + j] = (uint8_t)(word >> (8 * j));
+            for (int d = 0; d < n_dst; ++d) {
+                uint8_t* sf = a.dst[d].sf;
+                if (LAYOUT == QZ_SF_SWIZZLED_128x4) {
+                    st_u32(sf + swz_offset(row, k0, kv), word);
+                } else {
+                    const int64_t base = row * kv + k0;
+                    if (k0 + 4 <= kv && (base & 3) == 0) st_u32(sf + base, word);
+                    else for (int j = 0; j < 4 && k0 + j < kv; ++j) sf[base + j] = (uint8_t)(word >> (8 * j));
+                }
             }
         }
     }
 }
 
-template <int FMT, int LAYOUT>
-static cudaError_t launch_norm_fmt(const uint16_t* x, const uint16_t* r, const uint16_t* g, float eps, int64_t T,
-                                   int64_t H, uint16_t* y, uint16_t* h, uint8_t* q, uint8_t* sf, const float* amax,
-                                   cudaStream_t s, bool latency_mode) {
-    const int64_t grid = (LAYOUT == QZ_SF_SWIZZLED_128x4) ? pad_to(T, 128) : T;
-    const int nch = (int)(H / 8);
+template <int FMT, int LAYOUT, bool MULTI>
+static cudaError_t launch_norm_fmt(const NormArgs& a, int64_t ctas, cudaStream_t s, bool latency_mode) {
+    const int nch = (int)(a.H / 8);
     // latency mode: as few chunks per thread as 1024 threads allow;
     // throughput mode: four chunks per thread (fewer, narrower CTAs per row)
     int cpt = latency_mode ? 1 : 4;
     while ((nch + cpt - 1) / cpt > norm_max_threads(cpt)) cpt *= 2;
     const int threads = (int)pad_to((nch + cpt - 1) / cpt, 32);
     switch (cpt) {
-        case 1: rmsnorm_quant_kernel<FMT, LAYOUT, 1><<<(unsigned)grid, threads, 0, s>>>(x, r, g, eps, T, H, y, h, q, sf, amax); break;
-        case 2: rmsnorm_quant_kernel<FMT, LAYOUT, 2><<<(unsigned)grid, threads, 0, s>>>(x, r, g, eps, T, H, y, h, q, sf, amax); break;
-        case 4: rmsnorm_quant_kernel<FMT, LAYOUT, 4><<<(unsigned)grid, threads, 0, s>>>(x, r, g, eps, T, H, y, h, q, sf, amax); break;
-        default: rmsnorm_quant_kernel<FMT, LAYOUT, 8><<<(unsigned)grid, threads, 0, s>>>(x, r, g, eps, T, H, y, h, q, sf, amax); break;
+        case 1: rmsnorm_quant_kernel<FMT, LAYOUT, 1, MULTI><<<(unsigned)ctas, threads, 0, s>>>(a); break;
+        case 2: rmsnorm_quant_kernel<FMT, LAYOUT, 2, MULTI><<<(unsigned)ctas, threads, 0, s>>>(a); break;
+        case 4: rmsnorm_quant_kernel<FMT, LAYOUT, 4, MULTI><<<(unsigned)ctas, threads, 0, s>>>(a); break;
+        default: rmsnorm_quant_kernel<FMT, LAYOUT, 8, MULTI><<<(unsigned)ctas, threads, 0, s>>>(a); break;
     }
     return cudaGetLastError();
+}
+
+template <bool MULTI>
+static cudaError_t launch_norm(const NormArgs& a, int fmt, int layout, int64_t ctas, cudaStream_t s,
+                               bool latency_mode) {
+    if (fmt == QZ_FMT_MXFP8) {
+        return layout == QZ_SF_SWIZZLED_128x4
+                   ? launch_norm_fmt<QZ_FMT_MXFP8, QZ_SF_SWIZZLED_128x4, MULTI>(a, ctas, s, latency_mode)
+                   : launch_norm_fmt<QZ_FMT_MXFP8, QZ_SF_LINEAR, MULTI>(a, ctas, s, latency_mode);
+    }
+    return layout == QZ_SF_SWIZZLED_128x4
+               ? launch_norm_fmt<QZ_FMT_NVFP4, QZ_SF_SWIZZLED_128x4, MULTI>(a, ctas, s, latency_mode)
+               : launch_norm_fmt<QZ_FMT_NVFP4, QZ_SF_LINEAR, MULTI>(a, ctas, s, latency_mode);
 }
 
 // latency_mode: few rows (at most about two per SM), so each row gets a wide CTA.
 cudaError_t launch_rmsnorm_quant(const uint16_t* x, const uint16_t* r, const uint16_t* g, float eps, int64_t T,
                                  int64_t H, uint16_t* y, uint16_t* h, int fmt, uint8_t* q, uint8_t* sf, int layout,
                                  const float* amax, cudaStream_t s, bool latency_mode) {
-    if (fmt == QZ_FMT_MXFP8) {
-        return layout == QZ_SF_SWIZZLED_128x4
-                   ? launch_norm_fmt<QZ_FMT_MXFP8, QZ_SF_SWIZZLED_128x4>(x, r, g, eps, T, H, y, h, q, sf, amax, s, latency_mode)
-                   : launch_norm_fmt<QZ_FMT_MXFP8, QZ_SF_LINEAR>(x, r, g, eps, T, H, y, h, q, sf, amax, s, latency_mode);
-    }
-    return layout == QZ_SF_SWIZZLED_128x4
-               ? launch_norm_fmt<QZ_FMT_NVFP4, QZ_SF_SWIZZLED_128x4>(x, r, g, eps, T, H, y, h, q, sf, amax, s, latency_mode)
-               : launch_norm_fmt<QZ_FMT_NVFP4, QZ_SF_LINEAR>(x, r, g, eps, T, H, y, h, q, sf, amax, s, latency_mode);
+    NormArgs a = {};
+    a.x[0] = x;
+    a.dst[0] = NormDst{y, h, q, sf};
+    a.res = r;
+    a.gamma = g;
+    a.global_amax = amax;
+    a.T = T;
+    a.H = H;
+    a.row0 = 0;
+    a.eps = eps;
+    a.n_x = 1;
+    a.n_dst = 1;
+    const int64_t ctas = (layout == QZ_SF_SWIZZLED_128x4) ? pad_to(T, 128) : T;
+    return launch_norm<false>(a, fmt, layout, ctas, s, latency_mode);
+}
+
+// Rows [row_begin, row_end) of the AllReduce epilogue; the slice that ends at
+// T also zeroes the swizzled layout's invented rows of every destination.
+cudaError_t launch_allreduce_norm_quant(const uint16_t* const* xs, int n_x, const uint16_t* r, const uint16_t* g,
+                                        float eps, int64_t T, int64_t H, int64_t row_begin, int64_t row_end,
+                                        const qz_norm_dest* dsts, int n_dst, int fmt, int layout, const float* amax,
+                                        cudaStream_t s, bool latency_mode) {
+    if (n_x < 1 || n_x > kMaxRanks || n_dst < 1 || n_dst > kMaxRanks) return cudaErrorInvalidValue;
+    NormArgs a = {};
+    for (int i = 0; i < n_x; ++i) a.x[i] = xs[i];
+    for (int d = 0; d < n_dst; ++d)
+        a.dst[d] = NormDst{static_cast<uint16_t*>(dsts[d].norm_out), static_cast<uint16_t*>(dsts[d].residual_out),
+                           static_cast<uint8_t*>(dsts[d].q), dsts[d].sf};
+    a.res = r;
+    a.gamma = g;
+    a.global_amax = amax;
+    a.T = T;
+    a.H = H;
+    a.row0 = row_begin;
+    a.eps = eps;
+    a.n_x = n_x;
+    a.n_dst = n_dst;
+    const int64_t last = (row_end == T && layout == QZ_SF_SWIZZLED_128x4) ? pad_to(T, 128) : row_end;
+    const int64_t ctas = last - row_begin;
+    if (ctas <= 0) return cudaSuccess;
+    return launch_norm<true>(a, fmt, layout, ctas, s, latency_mode);
 }
 
 }  // namespace qz

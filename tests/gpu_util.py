@@ -22,6 +22,14 @@ def host_bits(t: torch.Tensor) -> np.ndarray:
     return synth.bf16_bits(t.detach().to("cpu"))
 
 
+def bf16_ulp_diff(a: np.ndarray, b: np.ndarray) -> np.ndarray:
+    """|a - b| in units of bf16 ulps via the ordered integer map of the bits."""
+    def key(u):
+        u = u.astype(np.int32)
+        return np.where(u & 0x8000, -(u & 0x7FFF), u & 0x7FFF)
+    return np.abs(key(a) - key(b))
+
+
 def mismatch(a: np.ndarray, b: np.ndarray, what: str, limit: int = 8) -> str:
     a = np.asarray(a).reshape(-1)
     b = np.asarray(b).reshape(-1)

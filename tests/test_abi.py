@@ -135,6 +135,46 @@ def test_host_errors_without_gpu(lib):
     assert norm(T=0) == qz.QZ_OK                                  # nothing to do, nothing launched
 
 
+def test_allreduce_epilogue_host_checks(lib):
+    """Every argument error of qz_allreduce_rmsnorm_quantize is returned before
+    any launch (the checks read only the host arrays of addresses)."""
+    P = ctypes.c_void_p
+    a = 0x10000
+
+    def ar(n=2, nd=1, T=4, H=7168, rows=(0, 4), fmt=0, layout=1, xs=None, ds=None, r=a, g=a, amax=None,
+           null_arrays=False):
+        xs = [a] * n if xs is None else xs
+        ds = [(a, None, a, a)] * nd if ds is None else ds
+        xa = (P * max(len(xs), 1))(*xs)
+        da = (qz.NormDest * max(len(ds), 1))(*[qz.NormDest(*d) for d in ds])
+        return lib.qz_allreduce_rmsnorm_quantize(
+            None if null_arrays else ctypes.cast(xa, P), n, P(r), P(g), ctypes.c_float(1e-6), T, H, rows[0], rows[1],
+            None if null_arrays else ctypes.cast(da, P), nd, fmt, layout, P(amax) if amax else None, None)
+
+    assert ar(n=0) == qz.QZ_ERR_INVALID_ARG
+    assert ar(n=qz.MAX_RANKS + 1) == qz.QZ_ERR_INVALID_ARG
+    assert ar(nd=0) == qz.QZ_ERR_INVALID_ARG
+    assert ar(nd=qz.MAX_RANKS + 1) == qz.QZ_ERR_INVALID_ARG
+    assert ar(null_arrays=True) == qz.QZ_ERR_INVALID_ARG
+    assert ar(rows=(-1, 4)) == qz.QZ_ERR_INVALID_ARG
+    assert ar(rows=(3, 2)) == qz.QZ_ERR_INVALID_ARG
+    assert ar(rows=(0, 5)) == qz.QZ_ERR_INVALID_ARG               # past T
+    assert ar(H=7168 + 16) == qz.QZ_ERR_INVALID_ARG               # not a multiple of 32 (MXFP8)
+    assert ar(H=qz.MAX_HIDDEN + 128) == qz.QZ_ERR_INVALID_ARG
+    assert ar(H=32 * 6) == qz.QZ_ERR_UNSUPPORTED                   # swizzled with kv % 4 != 0
+    assert ar(fmt=1, layout=0) == qz.QZ_ERR_INVALID_ARG            # NVFP4 without the global amax
+    assert ar(fmt=3) == qz.QZ_ERR_INVALID_ARG
+    assert ar(layout=2) == qz.QZ_ERR_INVALID_ARG
+    assert ar(xs=[a, None]) == qz.QZ_ERR_INVALID_ARG               # a NULL rank input
+    assert ar(ds=[(a, None, None, a)]) == qz.QZ_ERR_INVALID_ARG    # a destination without payload storage
+    assert ar(r=None) == qz.QZ_ERR_INVALID_ARG
+    assert ar(xs=[a, a + 8]) == qz.QZ_ERR_ALIGNMENT                # rank inputs want 16 bytes
+    assert ar(nd=2, ds=[(a, None, a, a), (a, a + 2, a, a)]) == qz.QZ_ERR_ALIGNMENT   # residual_out of dest 1
+    assert ar(ds=[(a, None, a, a + 4)]) == qz.QZ_ERR_ALIGNMENT     # swizzled SF wants 16 bytes
+    assert ar(ds=[(a, None, a + 4, a)]) == qz.QZ_ERR_ALIGNMENT     # payload wants 8 bytes
+    assert ar(T=0, rows=(0, 0)) == qz.QZ_OK                        # nothing to do, nothing launched
+
+
 def test_status_strings(lib):
     for s in range(5):
         assert qz.status_string(s).startswith("QZ_")

@@ -16,19 +16,11 @@ import torch
 
 import oracle
 import synth
-from gpu_util import Guarded, assert_bytes_equal, host_bits
+from gpu_util import Guarded, assert_bytes_equal, bf16_ulp_diff, host_bits
 
 pytestmark = pytest.mark.gpu
 
 qz = pytest.importorskip("nvfp4_quantization_moe_b200")
-
-
-def bf16_ulp_diff(a: np.ndarray, b: np.ndarray) -> np.ndarray:
-    """|a - b| in units of bf16 ulps via the ordered integer map of the bits."""
-    def key(u):
-        u = u.astype(np.int32)
-        return np.where(u & 0x8000, -(u & 0x7FFF), u & 0x7FFF)
-    return np.abs(key(a) - key(b))
 
 
 def run_fused(x, r, g, eps, fmt, layout, amax=None, with_residual=True):
