@@ -30,6 +30,10 @@
 // order and rounded once to bf16, so every rank reduces to the same bits.  It
 // takes a row range (one rank's slice, or all rows) and writes every output to
 // up to eight destinations (the ranks' own buffers, for the all-gather half).
+// A row's rank inputs are read one after another, so each CTA first asks L2
+// for the whole row of every rank after the first (one bulk prefetch per
+// rank), and throughput mode runs two chunks per thread (two CTAs of 448
+// threads per SM at H = 7168) to keep more of those reads in flight.
 #include "qz_device.cuh"
 
 namespace qz {
@@ -175,6 +179,12 @@ __device__ __forceinline__ void rank_sum_row(const NormArgs& a, int64_t row, int
     }
 }
 
+// Bring `bytes` (a multiple of 16, 16-byte aligned) at p into L2; no registers
+// wait on it.
+__device__ __forceinline__ void prefetch_l2_bulk(const void* p, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
 // MULTI == false: one input, one destination, row0 == 0 (qz_rmsnorm_quantize).
 template <int FMT, int LAYOUT, int CPT, bool MULTI>
 __global__ void __launch_bounds__(norm_max_threads(CPT)) rmsnorm_quant_kernel(const __grid_constant__ NormArgs a) {
@@ -194,6 +204,8 @@ __global__ void __launch_bounds__(norm_max_threads(CPT)) rmsnorm_quant_kernel(co
         return;
     }
 
+    // thread k < n_x - 1 prefetches this row of rank k + 1 (H * 2 bytes, 16-byte aligned)
+    if (MULTI && t + 1 < a.n_x) prefetch_l2_bulk(a.x[t + 1] + row * H, (uint32_t)(H * 2));
     const uint16_t* rr = a.res + row * H;
     uint4 h[CPT], rv[CPT], gv[CPT];
 #pragma unroll
@@ -299,8 +311,10 @@ template <int FMT, int LAYOUT, bool MULTI>
 static cudaError_t launch_norm_fmt(const NormArgs& a, int64_t ctas, cudaStream_t s, bool latency_mode) {
     const int nch = (int)(a.H / 8);
     // latency mode: as few chunks per thread as 1024 threads allow;
-    // throughput mode: four chunks per thread (fewer, narrower CTAs per row)
-    int cpt = latency_mode ? 1 : 4;
+    // throughput mode: four chunks per thread (fewer, narrower CTAs per row),
+    // two with the rank sum (its accumulators cost registers, and more
+    // resident threads keep more rank reads in flight)
+    int cpt = latency_mode ? 1 : (MULTI ? 2 : 4);
     while ((nch + cpt - 1) / cpt > norm_max_threads(cpt)) cpt *= 2;
     const int threads = (int)pad_to((nch + cpt - 1) / cpt, 32);
     switch (cpt) {
