@@ -124,49 +124,50 @@ __host__ __device__ constexpr int norm_max_threads(int cpt) { return cpt <= 2 ? 
 
 // bf16x2 words of the rank sum of chunks t + nt*i of one row: binary32
 // accumulation in rank order (rank 0 exactly, then one rounding per rank), one
-// bf16 rounding at the end.  Ranks are loaded two at a time so that two
-// chunks' loads per rank pair are in flight before either is added.
+// bf16 rounding at the end.  Ranks after the first are loaded G at a time (all
+// of them with one chunk per thread, two at a time otherwise), so that G
+// chunks' loads per thread are in flight before the first of them is added.
 template <int CPT>
 __device__ __forceinline__ void rank_sum_row(const NormArgs& a, int64_t row, int nch, int t, int nt,
                                              uint4 (&h)[CPT]) {
+    constexpr int G = CPT == 1 ? kMaxRanks - 1 : 2;
     float acc[CPT][8];
-    uint4 v[CPT], w[CPT];
+    uint4 v[G][CPT];
 #pragma unroll
     for (int i = 0; i < CPT; ++i) {
         const int c = i * nt + t;
-        v[i] = c < nch ? ld_stream(a.x[0] + row * a.H + c * 8) : make_uint4(0, 0, 0, 0);
+        v[0][i] = c < nch ? ld_stream(a.x[0] + row * a.H + c * 8) : make_uint4(0, 0, 0, 0);
     }
 #pragma unroll
     for (int i = 0; i < CPT; ++i) {
-        const uint32_t* vw = reinterpret_cast<const uint32_t*>(&v[i]);
+        const uint32_t* vw = reinterpret_cast<const uint32_t*>(&v[0][i]);
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
             acc[i][2 * j] = bf16_lo(vw[j]);
             acc[i][2 * j + 1] = bf16_hi(vw[j]);
         }
     }
-    for (int r = 1; r < a.n_x; r += 2) {
-        const bool two = r + 1 < a.n_x;
+    for (int r = 1; r < a.n_x; r += G) {
 #pragma unroll
-        for (int i = 0; i < CPT; ++i) {
-            const int c = i * nt + t;
-            v[i] = c < nch ? ld_stream(a.x[r] + row * a.H + c * 8) : make_uint4(0, 0, 0, 0);
-            w[i] = (two && c < nch) ? ld_stream(a.x[r + 1] + row * a.H + c * 8) : make_uint4(0, 0, 0, 0);
+        for (int k = 0; k < G; ++k) {
+            const bool live = r + k < a.n_x;
+            const uint16_t* xk = a.x[live ? r + k : 0] + row * a.H;
+#pragma unroll
+            for (int i = 0; i < CPT; ++i) {
+                const int c = i * nt + t;
+                v[k][i] = (live && c < nch) ? ld_stream(xk + c * 8) : make_uint4(0, 0, 0, 0);
+            }
         }
 #pragma unroll
-        for (int i = 0; i < CPT; ++i) {
-            const uint32_t* vw = reinterpret_cast<const uint32_t*>(&v[i]);
-            const uint32_t* ww = reinterpret_cast<const uint32_t*>(&w[i]);
+        for (int k = 0; k < G; ++k) {
+            if (r + k >= a.n_x) break;
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                acc[i][2 * j] = __fadd_rn(acc[i][2 * j], bf16_lo(vw[j]));
-                acc[i][2 * j + 1] = __fadd_rn(acc[i][2 * j + 1], bf16_hi(vw[j]));
-            }
-            if (two) {
+            for (int i = 0; i < CPT; ++i) {
+                const uint32_t* vw = reinterpret_cast<const uint32_t*>(&v[k][i]);
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
-                    acc[i][2 * j] = __fadd_rn(acc[i][2 * j], bf16_lo(ww[j]));
-                    acc[i][2 * j + 1] = __fadd_rn(acc[i][2 * j + 1], bf16_hi(ww[j]));
+                    acc[i][2 * j] = __fadd_rn(acc[i][2 * j], bf16_lo(vw[j]));
+                    acc[i][2 * j + 1] = __fadd_rn(acc[i][2 * j + 1], bf16_hi(vw[j]));
                 }
             }
         }
