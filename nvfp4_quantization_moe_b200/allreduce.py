@@ -13,10 +13,12 @@ another GPU.  This module owns what surrounds it:
 * ``AllReduceEpilogue``: one call = a barrier (every rank's input written,
   every destination free), the launch with the group's addresses in rank
   order, and a second barrier (no rank overwrites its input, or reads a
-  destination that peers write, before all have finished);
-* ``from_symmetric_memory``: the group's buffers from torch symmetric memory
-  and an NCCL all-reduce of one integer as the stream-ordered barrier, whose
-  waits are bounded by the process group's timeout on the host.
+  destination that peers write, before all have finished).
+
+The addresses come from whatever maps the ranks' allocations into each
+process (CUDA IPC handles, or a symmetric-memory allocator's per-rank buffer
+pointers), and the barrier can be an NCCL all-reduce of one integer on the
+launching stream, whose waits the process group's timeout bounds on the host.
 
 The one-shot form computes all T rows on every rank into its own buffers;
 the slice form computes ``rank_rows(T, world, rank)`` and writes them to every
@@ -25,8 +27,6 @@ rank's buffers (reduce-scatter and all-gather in one kernel).
 from __future__ import annotations
 
 from typing import Callable, List, Optional, Sequence, Tuple
-
-import torch
 
 from . import binding
 
@@ -111,36 +111,3 @@ class AllReduceEpilogue:
         self.launch(xs, residual, gamma, eps, dests, L.fmt, L.sf_layout, T, L.H, rows=rows,
                     global_amax=global_amax, stream=stream)
         self.barrier()
-
-
-def from_symmetric_memory(group, max_T: int, H: int, fmt: int, sf_layout: int, slice_form: bool = True,
-                          device=None):
-    """The epilogue of ``group`` (one node, NCCL) over torch symmetric memory.
-
-    Returns (epilogue, views): ``views`` are this rank's own buffers as tensors
-    (``x`` [max_T, H] bf16 to write the rank's partial sum into, ``y``, ``h``,
-    ``q``, ``sf``).  Every rank calls this collectively with the same
-    arguments."""
-    import torch.distributed as dist
-    import torch.distributed._symmetric_memory as symm_mem
-
-    device = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
-    L = SymmetricLayout(max_T, H, fmt, sf_layout)
-    buf = symm_mem.empty(L.total, dtype=torch.uint8, device=device)
-    hdl = symm_mem.rendezvous(buf, group)
-    token = torch.zeros(1, dtype=torch.int32, device=device)
-
-    def barrier():
-        dist.all_reduce(token, group=group)
-
-    ep = AllReduceEpilogue(hdl.rank, hdl.world_size, list(hdl.buffer_ptrs), L, barrier, slice_form)
-    ep._keep = (buf, hdl, token)
-    bf = max_T * H * 2
-
-    def bf16(off):
-        return buf[off:off + bf].view(torch.bfloat16).view(max_T, H)
-
-    qcols = H if fmt == binding.FMT_MXFP8 else H // 2
-    views = {"x": bf16(L.x), "y": bf16(L.y), "h": bf16(L.h), "q": buf[L.q:L.q + max_T * qcols].view(max_T, qcols),
-             "sf": buf[L.sf:L.total]}
-    return ep, views
