@@ -44,7 +44,7 @@ def _worker(rank, world, port, out):
 def test_two_gloo_ranks_max_time_and_distinct_inputs():
     world = 2
     port = _free_port()
-    manager = mp.Manager()
+    manager = mp.get_context("spawn").Manager()
     out = manager.dict()
     mp.start_processes(_worker, args=(world, port, out), nprocs=world, join=True, start_method="spawn")
     g0, g1 = out[0], out[1]

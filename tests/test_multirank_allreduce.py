@@ -82,7 +82,7 @@ def _worker(rank, world, port, out):
 def test_two_gloo_ranks_call_sequence():
     world = 2
     port = _free_port()
-    manager = mp.Manager()
+    manager = mp.get_context("spawn").Manager()
     out = manager.dict()
     mp.start_processes(_worker, args=(world, port, out), nprocs=world, join=True, start_method="spawn")
     rows_seen = []
