@@ -207,3 +207,29 @@ def test_element_hint_reaches_the_launch_options():
     assert raw.elems == 0
     assert ctypes.sizeof(qz.binding._Opts) == 40
 
+
+
+def test_binding_structs_match_the_header(tmp_path):
+    """Every struct the binding mirrors with ctypes has the header's size and
+    field offsets (a probe compiled by gcc against include/qz.h prints them)."""
+    b = qz.binding
+    mirrors = {"qz_expert": b._Expert, "qz_dq_expert": b._DqExpert, "qz_sf_pair": b._SfPair,
+               "qz_fused_split": b._FusedSplit, "qz_launch_opts": b._Opts, "qz_norm_dest": b.NormDest}
+    lines = ["#include <stdio.h>", "#include <stddef.h>", '#include "qz.h"', "int main(void) {"]
+    for cname, cls in mirrors.items():
+        lines.append(f'  printf("{cname} size %zu\\n", sizeof({cname}));')
+        for fname, _ in cls._fields_:
+            lines.append(f'  printf("{cname} {fname} %zu\\n", offsetof({cname}, {fname}));')
+    lines += ["  return 0;", "}"]
+    src = tmp_path / "probe.c"
+    src.write_text("\n".join(lines) + "\n")
+    exe = tmp_path / "probe"
+    subprocess.run(["gcc", "-std=c11", "-I", os.path.join(ROOT, "include"), "-o", str(exe), str(src)], check=True)
+    got = {}
+    for line in subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.splitlines():
+        cname, field, value = line.split()
+        got[(cname, field)] = int(value)
+    for cname, cls in mirrors.items():
+        assert got[(cname, "size")] == ctypes.sizeof(cls), cname
+        for fname, _ in cls._fields_:
+            assert got[(cname, fname)] == getattr(cls, fname).offset, f"{cname}.{fname}"
