@@ -9,7 +9,8 @@
  * and writes each expert's scale factors (SF) in the linear row-major layout
  * or the swizzled 128x4 layout, each expert into its own independently padded
  * region.  A fused residual-add + RMSNorm entry point writes the bf16 norm and
- * its quantized form from one read.
+ * its quantized form from one read; its AllReduce form first sums up to eight
+ * tensor-parallel ranks' inputs, read through (peer-mapped) device pointers.
  *
  * Conventions that hold for every entry point:
  *  - Pointers whose name starts with d_, and every pointer inside a table, are
