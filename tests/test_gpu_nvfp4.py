@@ -293,3 +293,29 @@ def test_compute_l2_workspace_too_small_is_rejected():
     with pytest.raises(qz.QzError):
         qz.quantize_grouped_nvfp4(qz.ExpertTable(entries), qz.NVFP4_PER_TENSOR_COMPUTE, qz.SF_SWIZZLED, workspace=ws)
     assert torch.all(keep[0][0].raw == 0xA5)
+
+
+def _order_cases():
+    from golden_io import rows
+    return rows("nvfp4_rounding_order.txt")
+
+
+@pytest.mark.parametrize("path", ["compute", "compute_l2", "row", "given"])
+def test_rounding_order_golden_on_gpu(path):
+    """The hand-worked cases that fix the order of the binary32 roundings of
+    the two-level scale (encode scale, block scale, element multiplier) give
+    the golden bytes on every NVFP4 path of the kernels."""
+    for case in _order_cases():
+        elems = np.zeros((1, 32), dtype=np.uint16)
+        elems[0, 0], elems[0, 16], elems[0, 17] = (int(v, 16) for v in case[1:4])
+        x = torch.from_numpy(elems.view(np.int16).copy()).view(torch.bfloat16).cuda()
+        for layout in LAYOUTS:
+            mode = {"compute": qz.NVFP4_PER_TENSOR_COMPUTE, "compute_l2": qz.NVFP4_PER_TENSOR_COMPUTE,
+                    "row": qz.NVFP4_PER_ROW, "given": qz.NVFP4_PER_TENSOR_GIVEN}[path]
+            amax_in = [float.fromhex(case[4])] if path == "given" else None
+            ws = qz.alloc_workspace(1, "cuda") if path == "compute_l2" else None
+            (gq, gsf, ga), = run_nvfp4([x], layout, mode, amax_in, workspace=ws)
+            lin = gsf if layout == qz.SF_LINEAR else oracle.unswizzle(gsf, 1, 2)
+            assert float(ga[0]).hex() == case[4], case[0]
+            assert list(lin[:2]) == [int(case[5], 16), int(case[6], 16)], (case[0], path, layout)
+            assert gq[0].tobytes().hex().upper() == case[7], (case[0], path, layout)

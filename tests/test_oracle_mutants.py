@@ -33,6 +33,12 @@ MUTANTS = {
     "nvfp4_no_zero_guard": ("if ((s & 0x7F) != 0) {", "if (1) {"),
     "nvfp4_scale_448": ("float g = A / 2688.0f;", "float g = A / 448.0f;"),
     "nvfp4_block_no_div6": ("float v = (b / 6.0f) * S;", "float v = b * S;"),
+    "nvfp4_scale_direct": ("    float g = A / 2688.0f;            /* stored decode scale, 2688 = 448 * 6 */\n"
+                           "    if (g == 0.0f) return 0.0f;\n    return 1.0f / g;",
+                           "    float g = A / 2688.0f;            /* stored decode scale, 2688 = 448 * 6 */\n"
+                           "    if (g == 0.0f) return 0.0f;\n    return 2688.0f / A;"),
+    "nvfp4_block_fused_product": ("float v = (b / 6.0f) * S;", "float v = (b * S) / 6.0f;"),
+    "nvfp4_rcp_as_product": ("rcp = S / (float)qzo_e4m3_value(s);", "rcp = S * (1.0f / (float)qzo_e4m3_value(s));"),
     "nibbles_swapped": ("(uint8_t)(qzo_e2m1_encode(y0) | (qzo_e2m1_encode(y1) << 4))",
                         "(uint8_t)((qzo_e2m1_encode(y0) << 4) | qzo_e2m1_encode(y1))"),
     "swizzle_plain_rowmajor": ("int64_t inner = ((r % 32) * 4 + (r / 32)) * 4 + (k % 4);",

@@ -147,3 +147,114 @@ def test_nvfp4_packing_low_nibble_first(olib):
     # A = 2688 -> g = 1, S = 1; block amax 6 -> v = 1 -> scale 1.0 (0x38)
     assert sf[0] == 0x38
     assert q[0, 0] == (0x7 | (0x2 << 4)) and q[0, 1] == (0xC | (0x1 << 4))
+
+
+# ---------------------------------------------------------------------------
+# rounding order of the two-level scale (readings R2, R3, R4), hand-worked
+# cases in tests/golden/nvfp4_rounding_order.txt
+# ---------------------------------------------------------------------------
+
+from fractions import Fraction  # noqa: E402
+import struct  # noqa: E402
+
+
+def _bf16(bits):
+    return Fraction(struct.unpack("<f", struct.pack("<I", int(bits) << 16))[0])
+
+
+def _rn32(q):
+    """Exact rational -> nearest binary32 (ties to even), as a rational."""
+    if q == 0:
+        return Fraction(0)
+    sign = -1 if q < 0 else 1
+    a = abs(q)
+    e = a.numerator.bit_length() - a.denominator.bit_length()
+    while Fraction(2) ** e > a:
+        e -= 1
+    while Fraction(2) ** (e + 1) <= a:
+        e += 1
+    ulp = Fraction(2) ** (max(e, -126) - 23)
+    n = a / ulp
+    fl = n.numerator // n.denominator
+    rem = n - fl
+    if rem > Fraction(1, 2) or (rem == Fraction(1, 2) and fl % 2 == 1):
+        fl += 1
+    return sign * fl * ulp
+
+
+def _nearest(table, v):
+    """Index of the nearest table value to v >= 0, ties to the even index
+    (the even code; values beyond the last entry saturate to it)."""
+    v = min(v, table[-1])
+    best = None
+    for i, t in enumerate(table):
+        d = abs(t - v)
+        if best is None or d < best[0] or (d == best[0] and i % 2 == 0):
+            best = (d, i)
+    return best[1]
+
+
+_E4M3 = [Fraction(c & 7, 8) * Fraction(2) ** -6 if c >> 3 == 0 else (1 + Fraction(c & 7, 8)) * Fraction(2) ** ((c >> 3) - 7)
+         for c in range(0x7F)]
+_E2M1 = [Fraction(v) for v in ("0", "1/2", "1", "3/2", "2", "3", "4", "6")]
+
+
+def _e2m1(v):
+    return (8 if v < 0 else 0) | _nearest(_E2M1, abs(v))
+
+
+def _worked_row(elems, encode, block, rcp):
+    """The row's scale bytes and payload by the given orders of rounding."""
+    xs = [_bf16(b) for b in elems]
+    A = max(abs(v) for v in xs)
+    S = encode(A)
+    sf, codes = [], []
+    for k in range(len(xs) // 16):
+        blk = xs[16 * k:16 * k + 16]
+        b = max(abs(v) for v in blk)
+        s = _nearest(_E4M3, block(b, S)) if b else 0
+        r = rcp(S, _E4M3[s]) if s else Fraction(0)
+        sf.append(s)
+        codes += [_e2m1(_rn32(v * r)) for v in blk]
+    return A, sf, bytes(codes[2 * j] | (codes[2 * j + 1] << 4) for j in range(len(codes) // 2))
+
+
+_READING = dict(encode=lambda A: _rn32(1 / _rn32(A / 2688)),                 # R2
+                block=lambda b, S: _rn32(_rn32(b / 6) * S),                   # R3
+                rcp=lambda S, m: _rn32(S / m))                                # R4
+_OTHER = {"encode_order": dict(_READING, encode=lambda A: _rn32(Fraction(2688) / A)),
+          "block_order": dict(_READING, block=lambda b, S: _rn32(_rn32(b * S) / 6)),
+          "rcp_order": dict(_READING, rcp=lambda S, m: _rn32(S * _rn32(1 / m)))}
+_ORDER_CASES = rows("nvfp4_rounding_order.txt")
+
+
+def _order_row(case):
+    name, e0, e16, e17 = case[:4]
+    elems = [0] * 32
+    elems[0], elems[16], elems[17] = int(e0, 16), int(e16, 16), int(e17, 16)
+    return name, elems
+
+
+@pytest.mark.parametrize("case", _ORDER_CASES, ids=[c[0] for c in _ORDER_CASES])
+def test_rounding_order_golden_is_worked_right(case):
+    """The golden's bytes follow from readings R2-R4 in exact arithmetic, and
+    the alternative order the case was built for gives other bytes."""
+    name, elems = _order_row(case)
+    A, sf, q = _worked_row(elems, **_READING)
+    assert float(A).hex() == case[4]
+    assert sf == [int(case[5], 16), int(case[6], 16)]
+    assert q.hex().upper() == case[7]
+    _, sf_alt, q_alt = _worked_row(elems, **_OTHER[name])
+    assert (sf_alt, q_alt) != (sf, q)
+
+
+@pytest.mark.parametrize("mode", [oracle.NVFP4_PER_TENSOR_COMPUTE, oracle.NVFP4_PER_ROW])
+@pytest.mark.parametrize("case", _ORDER_CASES, ids=[c[0] for c in _ORDER_CASES])
+def test_rounding_order_golden(case, mode):
+    """The oracle takes its binary32 roundings in the order of R2-R4."""
+    _, elems = _order_row(case)
+    xb = np.array([elems], dtype=np.uint16)
+    q, sf, amax = oracle.quantize_nvfp4(xb, oracle.LINEAR, mode)
+    assert float(amax[0]).hex() == case[4]
+    assert list(sf) == [int(case[5], 16), int(case[6], 16)]
+    assert q[0].tobytes().hex().upper() == case[7]
