@@ -15,7 +15,9 @@
  * Conventions that hold for every entry point:
  *  - Pointers whose name starts with d_, and every pointer inside a table, are
  *    DEVICE pointers.  The caller owns every buffer; the library allocates
- *    nothing and keeps no state besides a per-device cache of launch limits.
+ *    nothing.  Its only state is a per-device cache of launch limits and the
+ *    static device scratch of qz_quantize_grouped_nvfp4_compute_noalloc (with
+ *    that array's device address, looked up once per device).
  *  - `stream` is a cudaStream_t (NULL: the legacy default stream).  Every call
  *    is asynchronous on that stream; inputs must be ready on it.  No call
  *    synchronizes.
@@ -99,8 +101,10 @@ typedef enum qz_nvfp4_scale_mode {
                                   16-byte (MXFP8) / 8-byte (NVFP4) aligned; sf not 16-byte
                                   aligned (swizzled); amax not 4-byte aligned */
 #define QZ_DERR_TOO_LARGE 0x8u /* the call's total tile or row count exceeds 2^31 - 1 */
-#define QZ_DERR_TIMEOUT 0x10u  /* a wait for an asynchronous copy exceeded its time limit; the
-                                  kernel stopped early (no such wait is expected to expire) */
+#define QZ_DERR_TIMEOUT 0x10u  /* a bounded wait of the single-launch computed-amax path (a CTA
+                                  waiting until every amax tile of a chunk has been counted)
+                                  exceeded its limit; the waiting CTA stopped early and some
+                                  outputs are unwritten (no such wait is expected to expire) */
 #define QZ_DERR_CUT 0x20u      /* qz_split_fused_experts: the cut falls inside a scale block
                                   (FP8_BLOCK128: cut not a multiple of 128 and not the end) */
 
@@ -435,7 +439,11 @@ qz_status qz_split_fused_experts(const qz_fused_split *d_table, int n, int fmt, 
  *  - Every call clears the scratch it needs (a memset in stream order) and
  *    leaves its own contents behind; all calls share the one array, so calls
  *    that may overlap on the GPU (other streams, other host threads) race and
- *    must be serialized by the caller.
+ *    must be serialized by the caller.  A race shows up as QZ_DERR_TIMEOUT in
+ *    *opts->d_err or as wrong amax, scale or payload bytes.
+ *  - The looked-up address is kept for the life of the process: after
+ *    cudaDeviceReset on a device, this entry point must not be called again
+ *    on that device (the array may have moved with the reloaded library image).
  *  - n_experts above QZ_STATIC_WS_MAX_EXPERTS returns QZ_ERR_INVALID_ARG
  *    before anything is launched; other errors as qz_quantize_grouped_nvfp4;
  *    opts->d_workspace is ignored. */

@@ -220,6 +220,10 @@ def test_binding_structs_match_the_header(tmp_path):
         lines.append(f'  printf("{cname} size %zu\\n", sizeof({cname}));')
         for fname, _ in cls._fields_:
             lines.append(f'  printf("{cname} {fname} %zu\\n", offsetof({cname}, {fname}));')
+    limits = {"QZ_MAX_EXPERTS": b.MAX_EXPERTS, "QZ_MAX_HIDDEN": b.MAX_HIDDEN, "QZ_MAX_RANKS": b.MAX_RANKS,
+              "QZ_STATIC_WS_MAX_EXPERTS": b.STATIC_WS_MAX_EXPERTS}
+    for name in limits:
+        lines.append(f'  printf("define {name} %lld\\n", (long long)({name}));')
     lines += ["  return 0;", "}"]
     src = tmp_path / "probe.c"
     src.write_text("\n".join(lines) + "\n")
@@ -229,6 +233,8 @@ def test_binding_structs_match_the_header(tmp_path):
     for line in subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.splitlines():
         cname, field, value = line.split()
         got[(cname, field)] = int(value)
+    for name, value in limits.items():
+        assert got[("define", name)] == value, f"binding constant of {name}"
     for cname, cls in mirrors.items():
         assert got[(cname, "size")] == ctypes.sizeof(cls), cname
         for fname, _ in cls._fields_:

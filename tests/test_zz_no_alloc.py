@@ -59,10 +59,30 @@ def test_noalloc_matches_existing_entry_point_twice(layout):
     _quantize_pair(ys, layout)
 
 
+@pytest.mark.gpu
+def test_noalloc_at_its_table_limit():
+    """Exactly the largest table the static scratch holds (tiny experts, so
+    the per-expert amax words at the top of the array are written), then a
+    smaller call: the clear at the start of each call must reset the words
+    the first call left behind."""
+    n = qz.STATIC_WS_MAX_EXPERTS
+    xs = [synth.blockwise_scaled((1 + i % 3, 32), 16, seed=2000 + i, lo=-10, hi=10).cuda() for i in range(n)]
+    xs[n - 1] = xs[n - 1] * 64          # the last expert's amax word holds the largest value
+    _quantize_pair(xs, qz.SF_SWIZZLED)
+    ys = [synth.blockwise_scaled((2, 32), 16, seed=3000 + i, lo=-30, hi=-20).cuda() for i in range(n // 2)]
+    _quantize_pair(ys, qz.SF_SWIZZLED)
+
+
 def test_noalloc_rejects_oversized_table():
-    """More experts than the static scratch holds: refused before any launch."""
+    """More experts than the static scratch holds: refused before any launch;
+    exactly the limit passes the host checks (with no GPU the call then fails
+    at the CUDA runtime, not on its arguments)."""
     lib = qz.load()
     st = lib.qz_quantize_grouped_nvfp4_compute_noalloc(ctypes.c_void_p(0x1000), qz.STATIC_WS_MAX_EXPERTS + 1,
                                                         qz.SF_SWIZZLED, None, None)
     assert st == qz.QZ_ERR_INVALID_ARG
     assert lib.qz_quantize_grouped_nvfp4_compute_noalloc(None, 0, qz.SF_SWIZZLED, None, None) == qz.QZ_OK
+    if not torch.cuda.is_available():
+        st = lib.qz_quantize_grouped_nvfp4_compute_noalloc(ctypes.c_void_p(0x1000), qz.STATIC_WS_MAX_EXPERTS,
+                                                            qz.SF_SWIZZLED, None, None)
+        assert st == qz.QZ_ERR_CUDA
