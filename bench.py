@@ -1,24 +1,34 @@
 """Benchmark of the grouped block-scaled quantization path on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--config 1..5]
 
-One step is the Qwen3-30B-A3B MXFP8 refit prequantization: 48 layers x 128
-experts (gate_up [1536, 2048] and down [2048, 768] bf16, N(0, 0.02)), swizzled
-128x4 E8M0 scales, 16 experts per call (8 calls per projection per layer,
-768 launches per step).  All 48 layers' inputs and outputs stay resident in
-HBM (88 GB per step, far above the 126 MB L2, so no call finds its input in
-cache).  The metric is (input + output bytes) / time in GB/s.
+One step (the default, config 5) is the Qwen3-235B-A22B expert
+prequantization sweep: 94 layers, each layer's 128 gate_up [3072, 4096] and
+128 down [4096, 1536] bf16 experts (N(0, 0.02), 4.83 GB) regenerated in place
+from seed 5 + layer before the layer is timed, then quantized per projection
+in one call each to
+  - MXFP8 (E8M0 scales, swizzled 128x4),
+  - NVFP4 with the per-tensor FP32 scale computed by the call (one
+    cooperative launch: bulk copies feed the amax side, the quantize side
+    re-reads from L2), and
+  - NVFP4 again with that amax given (a requantization with a known scale),
+six calls per layer, every call bracketed by CUDA events on the stream it
+runs on.  Inputs are far larger than L2 (3.2 GB per call).  The metric is
+(input + output bytes) / time in GB/s; the step time is the sum of the event
+times of its 564 calls (the regeneration between layers is not timed).
 
-Besides the headline line the JSON carries the roofline of the dominant
-kernel (bytes per launch over its CUDA-event duration, against the measured
-HBM copy bandwidth), an end-to-end figure through the same C ABI with the
-inputs coming from pinned host memory, the CPU oracle timed on a bounded
-sample, SM clocks sampled during the timed region, and (``extra``) the other
-workloads: the tiny MXFP8 group, the row-scaled NVFP4 split activation, the
-fused residual + RMSNorm + quantize sweep and its AllReduce form over 8 rank
-buffers, the Qwen3-30B-A3B gate_up layer in NVFP4, a Qwen3-235B-A22B layer in
-MXFP8 and NVFP4, dequantization, column-wise quantization, the attention
-decode merge and the gate|up split.
+The JSON line carries the roofline of every kernel of the step (algorithmic
+bytes per launch over its event time, against the measured HBM copy
+bandwidth; the dominant one as ``roofline``), an end-to-end figure through
+the same C ABI with every layer's weights coming from pinned host memory and
+the quantized bytes going back, the CPU oracle timed on a bounded sample on
+one host thread and on all of them, SM clocks sampled during the timed
+region, the Qwen3-30B-A3B MXFP8 refit step (config 2) as ``refit_30b``, and
+(``extra``) the other workloads: the tiny MXFP8 group, the row-scaled NVFP4
+split activation, the fused residual + RMSNorm + quantize sweep and its
+AllReduce form over 8 rank buffers, the Qwen3-30B-A3B gate_up layer in NVFP4,
+dequantization, column-wise quantization, the attention decode merge and the
+gate|up split.
 
 With torchrun (N > 1) every rank quantizes its own full workload on its own
 GPU (weak scaling, no collective on the data path); the time is the maximum
@@ -70,7 +80,7 @@ def hbm_peak():
 KERNEL_SOURCES = {
     "mxfp8_grouped_kernel": ("qz_grouped.cu", "qz_device.cuh"),
     "nvfp4_tile_kernel": ("qz_grouped.cu", "qz_device.cuh"),
-    "nvfp4_compute_l2_kernel": ("qz_grouped.cu", "qz_device.cuh"),
+    "nvfp4_compute_pipe_kernel": ("qz_grouped.cu", "qz_device.cuh"),
     "nvfp4_rows_kernel": ("qz_rows.cu", "qz_device.cuh"),
     "rmsnorm_quant_kernel": ("qz_rmsnorm.cu", "qz_device.cuh"),
     "rmsnorm_quant_kernel_multi": ("qz_rmsnorm.cu", "qz_device.cuh"),   # the AllReduce instantiation
@@ -229,10 +239,13 @@ class Refit30B:
     def launches(self):
         return len(self.calls)
 
-    def step(self, stream, events=None, side=None):
+    def step(self, stream, events=None, side=None, independent=False):
         """One pass over all calls.  With `side` streams, calls go round-robin
         to them (independent calls may overlap) and `stream` joins them at the
-        end; per-launch events are only taken on a single stream."""
+        end; per-launch events are only taken on a single stream.  With
+        `independent` every call is declared independent (QZ_OPT_INDEPENDENT):
+        on one stream, each call's tiles may start on the SMs the previous
+        call's tail frees."""
         qz = self.qz
         if side:
             start = torch.cuda.Event()
@@ -264,17 +277,17 @@ class Refit30B:
                 b.record(stream)
                 events.append((a, b))
             else:
-                qz.quantize_grouped_mxfp8(table, qz.SF_SWIZZLED, stream=stream)
+                qz.quantize_grouped_mxfp8(table, qz.SF_SWIZZLED, stream=stream, independent=independent)
 
 
-def time_steps(work, steps, warmup, stream, dist_ok, side=None, per_launch=True):
+def time_steps(work, steps, warmup, stream, dist_ok, side=None, per_launch=True, independent=False):
     """W untimed steps, then K timed steps bracketed by barrier + sync.  With
     per_launch, CUDA events bracket every launch on its own stream (timing
     events between the launches of two streams cost their overlap, so the
     headline pass goes without them).  Returns the total ms, every launch's
     duration and the union of the launch intervals (overlaps counted once)."""
     for _ in range(warmup):
-        work.step(stream, side=side)
+        work.step(stream, side=side, independent=independent)
     torch.cuda.synchronize()
     if dist_ok:
         torch.distributed.barrier()
@@ -284,7 +297,7 @@ def time_steps(work, steps, warmup, stream, dist_ok, side=None, per_launch=True)
     launch_events = []
     start.record(stream)
     for _ in range(steps):
-        work.step(stream, launch_events if per_launch else None, side=side)
+        work.step(stream, launch_events if per_launch else None, side=side, independent=independent)
     end.record(stream)
     torch.cuda.synchronize()
     if dist_ok:
@@ -384,6 +397,223 @@ def e2e_refit(qz, device, steps, warmup, layers=48, per_call=16, pool=2):
             "ms_per_step": round(ms / steps, 3), "wall_s": round(wall, 3),
             "note": f"host weights from {pool} pinned layer buffers cycled over {layers} layers; "
                     "H2D, kernels and D2H pipelined on three streams"}
+
+
+# ---------------------------------------------------------------------------
+# the headline: Qwen3-235B-A22B prequantization sweep, every layer regenerated
+# ---------------------------------------------------------------------------
+
+PROJS = ("gate_up", "down")
+SWEEP_MODES = ("mxfp8", "nvfp4_compute", "nvfp4_given")
+SWEEP_KERNELS = {"mxfp8": "mxfp8_grouped_kernel", "nvfp4_compute": "nvfp4_compute_pipe_kernel",
+                 "nvfp4_given": "nvfp4_tile_kernel"}
+
+
+class Prequant235B:
+    """Per layer: regenerate the layer's experts in place (untimed), then six
+    calls -- MXFP8, NVFP4 with the per-tensor amax computed, NVFP4 with that
+    amax given -- for gate_up and for down, 128 experts per call."""
+
+    def __init__(self, qz, device, layers=94, rank=0, compute_workspace=True):
+        cfg = synth.QWEN3_235B
+        self.qz, self.cfg, self.layers, self.rank = qz, cfg, layers, rank
+        E = cfg["experts"]
+        self.x, self.calls, self.keep = {}, [], []
+        self.ws = qz.alloc_workspace(E, device) if compute_workspace else None
+        self.compute_launches = 1 if compute_workspace else 3
+        self.kernels = dict(SWEEP_KERNELS)
+        if not compute_workspace:
+            self.kernels["nvfp4_compute"] = "amax_grouped_kernel+nvfp4_tile_kernel"
+        self.host_out = {}   # for e2e: what a layer's outputs are (device tensors)
+        for proj in PROJS:
+            rows, cols = cfg[proj]
+            x = torch.empty((E, rows, cols), dtype=torch.bfloat16, device=device)
+            self.x[proj] = x
+            nmx = qz.sf_bytes(rows, cols, qz.FMT_MXFP8, qz.SF_SWIZZLED)
+            nnv = qz.sf_bytes(rows, cols, qz.FMT_NVFP4, qz.SF_SWIZZLED)
+            mq = torch.empty((E, rows, cols), dtype=torch.uint8, device=device)
+            msf = torch.empty((E, nmx), dtype=torch.uint8, device=device)
+            nq = torch.empty((E, rows, cols // 2), dtype=torch.uint8, device=device)
+            nsf = torch.empty((E, nnv), dtype=torch.uint8, device=device)
+            amax = torch.zeros((E, 1), dtype=torch.float32, device=device)
+            self.keep.append((mq, msf, nq, nsf, amax))
+            self.host_out[proj] = (mq, msf, nq, nsf, amax)
+            mtab = qz.ExpertTable([qz.Entry(x[e], mq[e], msf[e]) for e in range(E)])
+            ntab = qz.ExpertTable([qz.Entry(x[e], nq[e], nsf[e], amax[e]) for e in range(E)])
+            bin_ = E * rows * cols * 2
+            self.calls.append(("mxfp8", proj, mtab, bin_ + E * (rows * cols + nmx)))
+            self.calls.append(("nvfp4_compute", proj, ntab, bin_ + E * (rows * cols // 2 + nnv + 4)))
+            self.calls.append(("nvfp4_given", proj, ntab, bin_ + E * (rows * cols // 2 + nnv + 4)))
+        order = {m: i for i, m in enumerate(SWEEP_MODES)}
+        self.calls.sort(key=lambda c: (order[c[0]], PROJS.index(c[1])))
+        self.bytes_per_layer = sum(c[3] for c in self.calls)
+        self.bytes = self.bytes_per_layer * layers
+        self.launches_per_layer = sum(self.compute_launches if c[0] == "nvfp4_compute" else 1 for c in self.calls)
+
+    def regenerate(self, layer):
+        for proj in PROJS:
+            synth.moe_layer(self.cfg, layer, proj, rank=self.rank, out=self.x[proj])
+
+    def call(self, mode, table, stream):
+        qz = self.qz
+        if mode == "mxfp8":
+            qz.quantize_grouped_mxfp8(table, qz.SF_SWIZZLED, stream=stream)
+        elif mode == "nvfp4_compute":
+            qz.quantize_grouped_nvfp4(table, qz.NVFP4_PER_TENSOR_COMPUTE, qz.SF_SWIZZLED, stream=stream,
+                                      workspace=self.ws)
+        else:
+            qz.quantize_grouped_nvfp4(table, qz.NVFP4_PER_TENSOR_GIVEN, qz.SF_SWIZZLED, stream=stream)
+
+    def layer_calls(self, stream, events=None):
+        for mode, proj, table, nbytes in self.calls:
+            if events is not None:
+                a = torch.cuda.Event(enable_timing=True)
+                b = torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                self.call(mode, table, stream)
+                b.record(stream)
+                events.append((mode, proj, nbytes, a, b))
+            else:
+                self.call(mode, table, stream)
+
+    def step(self, stream, events=None):
+        for layer in range(self.layers):
+            with torch.cuda.stream(stream):
+                self.regenerate(layer)
+            self.layer_calls(stream, events)
+
+
+def time_sweep(work, steps, warmup, stream, dist_ok):
+    """W untimed steps, then K steps bracketed by barrier + synchronize; every
+    call of the K steps is bracketed by CUDA events on its stream.  Returns the
+    per-mode totals (ms, bytes, calls), the summed call time and the device
+    time of the whole sweep including the untimed regeneration."""
+    for _ in range(warmup):
+        work.step(stream)
+    torch.cuda.synchronize()
+    if dist_ok:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    events = []
+    s0 = torch.cuda.Event(enable_timing=True)
+    s1 = torch.cuda.Event(enable_timing=True)
+    s0.record(stream)
+    for _ in range(steps):
+        work.step(stream, events)
+    s1.record(stream)
+    torch.cuda.synchronize()
+    if dist_ok:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    per = {m: {"ms": 0.0, "bytes": 0, "calls": 0, "by_proj": {p: [0.0, 0, 0] for p in PROJS}} for m in SWEEP_MODES}
+    for mode, proj, nbytes, a, b in events:
+        ms = a.elapsed_time(b)
+        d = per[mode]
+        d["ms"] += ms
+        d["bytes"] += nbytes
+        d["calls"] += 1
+        bp = d["by_proj"][proj]
+        bp[0] += ms
+        bp[1] += nbytes
+        bp[2] += 1
+    total_ms = sum(d["ms"] for d in per.values())
+    return per, total_ms, s0.elapsed_time(s1)
+
+
+def sweep_roofline(per, peak, peak_kind, launches, kernels):
+    """Roofline of every kernel of the sweep: algorithmic bytes per launch over
+    the launch's CUDA-event time (a call is one launch of the kernel, plus a
+    workspace memset for the computed-amax call)."""
+    out = {}
+    for mode, d in per.items():
+        achieved = d["bytes"] / (d["ms"] / 1e3) / GB
+        k = kernels[mode]
+        out[mode] = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4), "traffic": ncu_traffic(k) if k in KERNEL_SOURCES else None,
+                     "kernel": k,
+                     "launches_per_call": launches.get(mode, 1),
+                     "bytes_per_launch": int(d["bytes"] / max(1, d["calls"])),
+                     "mean_launch_us": round(1e3 * d["ms"] / max(1, d["calls"]), 1),
+                     "by_proj": {p: {"GB/s": round(v[1] / (v[0] / 1e3) / GB, 1),
+                                     "frac": round(v[1] / (v[0] / 1e3) / GB / peak, 4),
+                                     "us": round(1e3 * v[0] / max(1, v[2]), 1)}
+                                 for p, v in d["by_proj"].items() if v[2]}}
+    dom = max(per, key=lambda m: per[m]["ms"])
+    roof = dict(out[dom])
+    roof["peak_source"] = "measured (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured" else "fallback 6650 GB/s"
+    roof["timing"] = "CUDA events around every call on its stream, summed over the timed steps"
+    roof["dominant"] = dom
+    roof["by_mode"] = out
+    return roof
+
+
+def e2e_prequant(qz, device, steps, warmup, layers=4, pool=2, compute_workspace=True):
+    """The sweep end to end through the C ABI: every layer's bf16 experts come
+    host -> device from pinned memory, the six calls run, and every quantized
+    byte (both MXFP8 and NVFP4 payloads, scales and amax) goes device -> host.
+    Copies and calls are pipelined over three streams with double-buffered
+    device layers."""
+    cfg = synth.QWEN3_235B
+    E = cfg["experts"]
+    host_in = [{p: synth.moe_layer(cfg, 7000 + i, p, device=device).cpu().pin_memory() for p in PROJS}
+               for i in range(pool)]
+    works = [Prequant235B(qz, device, layers=1, compute_workspace=compute_workspace) for _ in range(2)]
+    host_out = {p: [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in works[0].host_out[p]] for p in PROJS}
+    h2d, comp, d2h = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+    done_d2h = [None, None]
+    h2d_bytes = sum(E * r * c * 2 for r, c in (cfg[p] for p in PROJS))
+    d2h_bytes = sum(t.numel() * t.element_size() for p in PROJS for t in works[0].host_out[p])
+
+    def one_step():
+        for layer in range(layers):
+            b = layer & 1
+            w = works[b]
+            src = host_in[layer % pool]
+            with torch.cuda.stream(h2d):
+                if done_d2h[b] is not None:
+                    h2d.wait_event(done_d2h[b])
+                for p in PROJS:
+                    w.x[p].copy_(src[p], non_blocking=True)
+                ev_in = torch.cuda.Event()
+                ev_in.record(h2d)
+            comp.wait_event(ev_in)
+            w.layer_calls(comp)
+            ev_c = torch.cuda.Event()
+            ev_c.record(comp)
+            with torch.cuda.stream(d2h):
+                d2h.wait_event(ev_c)
+                for p in PROJS:
+                    for hd, dv in zip(host_out[p], w.host_out[p]):
+                        hd.copy_(dv, non_blocking=True)
+                ev_o = torch.cuda.Event()
+                ev_o.record(d2h)
+                done_d2h[b] = ev_o
+
+    for _ in range(warmup):
+        one_step()
+    torch.cuda.synchronize()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    t0 = time.perf_counter()
+    start.record(h2d)
+    for _ in range(steps):
+        one_step()
+    cur = torch.cuda.current_stream()
+    for st in (d2h, comp, h2d):
+        cur.wait_stream(st)
+    end.record(cur)
+    torch.cuda.synchronize()
+    ms = start.elapsed_time(end)
+    wall = time.perf_counter() - t0
+    per_step = layers * works[0].bytes_per_layer
+    res = {"value": round(steps * per_step / (ms / 1e3) / GB, 2), "unit": "GB/s",
+           "h2d_bytes_per_step": layers * h2d_bytes, "d2h_bytes_per_step": layers * d2h_bytes,
+           "ms_per_step": round(ms / steps, 3), "wall_s": round(wall, 3), "layers_per_step": layers,
+           "note": f"weights of {pool} pinned host layers cycled over {layers} layers per step; H2D, the six "
+                   "calls and D2H of all outputs pipelined on three streams"}
+    del works, host_in, host_out
+    torch.cuda.empty_cache()
+    return res
 
 
 # ---------------------------------------------------------------------------
@@ -831,85 +1061,153 @@ def _extra_allreduce(qz, device, out, peak, tokens=None, ranks=8):
 # CPU oracle timing (the reference arm and the cpu_baseline key)
 # ---------------------------------------------------------------------------
 
-def oracle_refit_sample(target_s: float = 12.0):
-    """Time the CPU oracle on a bounded sample of the refit workload (whole
-    gate_up and down experts), on all host cores.  Returns (GB/s, cores,
-    sample description, seconds)."""
+def oracle_prequant_sample(threads: int, target_s: float = 10.0, min_pairs: int = 1, pairs: int = 0):
+    """Time the CPU oracle on a bounded sample of the headline workload: whole
+    Qwen3-235B-A22B experts (one gate_up [3072, 4096] and one down
+    [4096, 1536]) each quantized to MXFP8, to NVFP4 with the amax computed and
+    to NVFP4 with it given -- the six calls of a layer, per expert pair --
+    repeated over ``threads`` host threads for about ``target_s`` seconds.
+    ``pairs`` > 0 skips the sizing run.  Returns (GB/s, threads, sample
+    description, seconds, pairs)."""
     import oracle
-    cfg = synth.QWEN3_30B
-    threads = oracle.host_threads()
-    gu = synth.bf16_bits(synth.expert_stack(1, cfg["gate_up"], cfg["std"], seed=cfg["seed"])[0])
-    dn = synth.bf16_bits(synth.expert_stack(1, cfg["down"], cfg["std"], seed=cfg["seed"] + 500)[0])
-    per_pair = gu.size * 3 + gu.shape[0] * gu.shape[1] // 32 + dn.size * 3 + dn.shape[0] * dn.shape[1] // 32
+    from concurrent.futures import ThreadPoolExecutor
+    cfg = synth.QWEN3_235B
+    xs = {p: synth.bf16_bits(synth.moe_layer(dict(cfg, experts=1), 0, p, device="cpu")[0]) for p in PROJS}
+    per_pair = 0
+    for p in PROJS:
+        r, c = cfg[p]
+        per_pair += r * c * 2 + r * c + (r * c // 32)                      # MXFP8 (no padding at these shapes)
+        per_pair += 2 * (r * c * 2 + r * c // 2 + (r * c // 16) + 4)      # NVFP4 computed, NVFP4 given
+
+    def pair(_):
+        for p in PROJS:
+            x = xs[p]
+            oracle.quantize_mxfp8(x, oracle.SWIZZLED)
+            _, _, a = oracle.quantize_nvfp4(x, oracle.SWIZZLED, oracle.NVFP4_PER_TENSOR_COMPUTE)
+            oracle.quantize_nvfp4(x, oracle.SWIZZLED, oracle.NVFP4_PER_TENSOR_GIVEN, float(a[0]))
+
+    if pairs <= 0:
+        t0 = time.perf_counter()
+        pair(0)
+        one = time.perf_counter() - t0
+        pairs = max(min_pairs, threads, int(round(target_s / max(one, 1e-3) * threads)))
     t0 = time.perf_counter()
-    oracle.quantize_grouped([gu, dn], oracle.MXFP8, oracle.SWIZZLED, threads=2)
-    one = time.perf_counter() - t0                     # 2 experts on 2 threads
-    pairs = max(1, int(target_s / max(one, 1e-3) * threads / 2))
-    pairs = min(pairs, 2048)
-    experts = [gu, dn] * pairs
-    t0 = time.perf_counter()
-    oracle.quantize_grouped(experts, oracle.MXFP8, oracle.SWIZZLED, threads=threads)
+    if threads <= 1:
+        for i in range(pairs):
+            pair(i)
+    else:
+        with ThreadPoolExecutor(max_workers=threads) as ex:
+            list(ex.map(pair, range(pairs)))
     dt = time.perf_counter() - t0
     nbytes = pairs * per_pair
-    return nbytes / dt / GB, threads, f"{pairs} gate_up + {pairs} down experts of one Qwen3-30B-A3B layer " \
-                                      f"(MXFP8, swizzled), {nbytes / GB:.3f} GB", dt
+    desc = (f"{pairs} x (gate_up [3072,4096] + down [4096,1536]) Qwen3-235B-A22B experts, each to MXFP8, NVFP4 "
+            f"computed amax and NVFP4 given amax (swizzled), {nbytes / GB:.2f} GB, {threads} thread(s)")
+    return nbytes / dt / GB, threads, desc, dt, pairs
 
 
 def run_reference(args, rank, world):
+    """The reference arm: the CPU oracle as it stands on the host cores, on
+    the headline's workload (a bounded sample per step), rank 0 only."""
     if rank != 0:
         return
-    vals = []
-    t_total = 0.0
-    desc = cores = None
+    import oracle
+    threads = oracle.host_threads()
+    vals, t_total, desc = [], 0.0, None
+    npairs = 0
     for i in range(args.warmup + args.steps):
-        v, cores, desc, dt = oracle_refit_sample(target_s=max(2.0, 40.0 / max(1, args.steps + args.warmup)))
+        # the first step sizes the sample, the others repeat it
+        v, _, desc, dt, npairs = oracle_prequant_sample(
+            threads, target_s=max(1.0, 60.0 / max(1, args.steps + args.warmup)), pairs=npairs)
         if i >= args.warmup:
             vals.append(v)
             t_total += dt
     value = statistics.median(vals)
     line = {"metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": args.gpus, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(1e3 * t_total / max(1, args.steps), 1),
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16->mxfp8 (f32/f64 host)",
-            "data": "synthetic", "impl": "reference",
-            "config": {"workload": "Qwen3-30B-A3B MXFP8 refit prequant (48 layers x 128 experts, gate_up "
-                                   "[1536,2048] + down [2048,768], 16 experts/call, swizzled 128x4)",
-                       "sample": desc},
-            "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16->mxfp8/nvfp4 (f32 host)", "data": "synthetic", "impl": "reference",
+            "config": {"workload": HEADLINE_WORKLOAD, "sample": desc},
+            "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
                              "sample": desc},
             "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
+
+
+HEADLINE_WORKLOAD = "Qwen3-235B-A22B prequant: 94 layers x 2 projections x 128 experts, MXFP8 + NVFP4 (computed, given)"
 
 
 # ---------------------------------------------------------------------------
 # main
 # ---------------------------------------------------------------------------
 
+def refit_30b(qz, device, args, rank, dist_ok, peak):
+    """The Qwen3-30B-A3B MXFP8 refit step (config 2): 48 layers resident,
+    16 experts per call, calls round-robin on two streams; the same steps in
+    order on one stream give each launch's own event time."""
+    work = Refit30B(qz, device, layers=args.layers, seed_offset=rank)
+    side = [torch.cuda.Stream() for _ in range(args.streams)] if args.streams > 1 else None
+    stream = torch.cuda.current_stream()
+    torch.cuda.synchronize()
+    total_ms, _, _ = time_steps(work, args.steps, args.warmup, stream, dist_ok, side=side, per_launch=False)
+    single_ms, single_launch_ms, _ = time_steps(work, args.steps, 1, stream, dist_ok)
+    indep_ms, _, _ = time_steps(work, args.steps, 1, stream, dist_ok, per_launch=False, independent=True)
+    total_ms, single_ms, indep_ms = max_over_ranks([total_ms, single_ms, indep_ms], device)
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    value = aggregate_gbs(work.bytes, world, args.steps, total_ms)
+    call_bytes = [b for _, b in work.calls] * args.steps
+    achieved = sum(call_bytes) / (total_ms / 1e3) / GB
+    achieved_single = sum(call_bytes) / (sum(single_launch_ms) / 1e3) / GB
+    out = {"value": round(value, 1), "unit": "GB/s", "ms_per_step": round(total_ms / args.steps, 3),
+           "frac": round(achieved / peak, 4), "kernel": work.kernel,
+           "workload": f"Qwen3-30B-A3B MXFP8 refit: {args.layers} layers x 128 experts, 16 experts/call, swizzled",
+           "bytes_per_step_per_gpu": work.bytes, "launches_per_step": work.launches,
+           "issue": f"calls round-robin on {args.streams} streams" if side else "calls in order on one stream",
+           "bytes_per_launch": int(np.mean([b for _, b in work.calls])),
+           "effective_launch_us": round(1e3 * total_ms / (work.launches * args.steps), 2),
+           "traffic": ncu_traffic(work.kernel),
+           "single_stream": {"value": round(aggregate_gbs(work.bytes, world, args.steps, single_ms), 1),
+                             "frac": round(achieved_single / peak, 4),
+                             "mean_launch_us": round(1e3 * float(np.mean(single_launch_ms)), 2)},
+           "single_stream_independent": {
+               "value": round(aggregate_gbs(work.bytes, world, args.steps, indep_ms), 1),
+               "frac": round(sum(call_bytes) / (indep_ms / 1e3) / GB / peak, 4),
+               "how": "calls in order on one stream, each declared QZ_OPT_INDEPENDENT (programmatic dependent "
+                      "launch overlaps each call's tail with the next call's tiles); region timed"}}
+    del work
+    torch.cuda.empty_cache()
+    return out
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=5)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--layers", type=int, default=48)
-    ap.add_argument("--streams", type=int, default=2, help="streams the independent calls are spread over")
+    ap.add_argument("--layers", type=int, default=None,
+                    help="layers per step (default: 94 for the Qwen3-235B-A22B sweep, 48 for the 30B refit)")
+    ap.add_argument("--streams", type=int, default=2, help="streams the independent 30B refit calls are spread over")
+    ap.add_argument("--compute-path", choices=["single", "three"], default="three",
+                    help="NVFP4 computed amax: one cooperative launch with a workspace, or clear + amax + quantize")
     ap.add_argument("--no-extra", action="store_true", help="skip the other workloads")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    ap.add_argument("--no-refit", action="store_true", help="skip the Qwen3-30B-A3B refit step")
     ap.add_argument("--config", type=int, choices=[1, 2, 3, 4, 5], default=None,
-                    help="one of the five workloads: 1 tiny MXFP8 group (latency), 2 the Qwen3-30B-A3B refit step "
-                         "(the default run), 3 the row-scaled NVFP4 split activation, 4 the fused residual + "
-                         "RMSNorm sweep, 5 the Qwen3-235B-A22B layer")
+                    help="one of the five workloads: 1 tiny MXFP8 group (latency), 2 the Qwen3-30B-A3B refit step, "
+                         "3 the row-scaled NVFP4 split activation, 4 the fused residual + RMSNorm sweep, 5 the "
+                         "Qwen3-235B-A22B sweep (the default run)")
     ap.add_argument("--only", choices=["tiny", "split", "fused", "nvfp4", "large", "dequant", "merge", "colwise",
                                        "gateup", "allreduce"],
                     default=None,
                     help="time only this secondary workload and print its record (profiling aid)")
     ap.add_argument("--experts", type=int, default=None,
-                    help="experts per call of the Qwen3-235B-A22B workload (default 128; fewer for a profiler capture)")
+                    help="experts per call of the Qwen3-235B-A22B extra workload (fewer for a profiler capture)")
     ap.add_argument("--tokens", type=str, default=None,
                     help="comma-separated token counts for the fused, merge and AllReduce sweeps")
     args = ap.parse_args()
-    if args.config is not None and args.config != 2:
-        args.only = {1: "tiny", 3: "split", 4: "fused", 5: "large"}[args.config]
+    if args.config in (1, 3, 4):
+        args.only = {1: "tiny", 3: "split", 4: "fused"}[args.config]
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -936,68 +1234,79 @@ def main():
                           "extra": extra_workloads(qz, device, stream, peak, (args.only,), toks, args.experts)}))
         return
 
-    work = Refit30B(qz, device, layers=args.layers, seed_offset=rank)
-    side = [torch.cuda.Stream() for _ in range(args.streams)] if args.streams > 1 else None
+    if args.config == 2:
+        # the 30B refit step as the headline
+        args.layers = args.layers or 48
+        with ClockSampler(local) as clocks:
+            r = refit_30b(qz, device, args, rank, dist_ok, peak)
+        line = {"metric": METRIC, "value": r["value"], "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": r["ms_per_step"], "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "bf16->mxfp8 (e4m3 + e8m0)", "data": "synthetic",
+                "config": {"workload": r["workload"], "l2": "inputs larger than L2",
+                           "parallelism": f"{world} independent replicas (weak scaling, no collective)"},
+                "roofline": {"bound": "hbm", "achieved": round(r["frac"] * peak, 1), "peak": peak, "unit": "GB/s",
+                             "frac": r["frac"], "traffic": r["traffic"], "kernel": r["kernel"],
+                             "single_stream_frac": r["single_stream"]["frac"]},
+                "clocks": clocks.summary(), "gpu_launches": r["launches_per_step"] * (args.steps + 1),
+                "refit_30b": r}
+        if dist_ok:
+            torch.distributed.barrier()
+            torch.distributed.destroy_process_group()
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+        return
+
+    # ---- default: the Qwen3-235B-A22B sweep (config 5) ----
+    refit = None
+    if args.config is None and not args.no_refit:
+        refit_args = argparse.Namespace(**vars(args))
+        refit_args.layers = 48
+        refit_args.steps, refit_args.warmup = min(args.steps, 10), min(args.warmup, 3)
+        refit = refit_30b(qz, device, refit_args, rank, dist_ok, peak)
+    layers = args.layers or synth.QWEN3_235B["layers"]
+    work = Prequant235B(qz, device, layers=layers, rank=rank, compute_workspace=args.compute_path == "single")
     torch.cuda.synchronize()
     with ClockSampler(local) as clocks:
-        total_ms, _, _ = time_steps(work, args.steps, args.warmup, stream, dist_ok, side=side, per_launch=False)
-        # the same steps with every call in order on one stream and an event
-        # pair around each launch: the kernel's own launch durations
-        single_ms, single_launch_ms, _ = time_steps(work, args.steps, 1, stream, dist_ok)
-    total_ms, single_ms = max_over_ranks([total_ms, single_ms], device)
-    ms_step = total_ms / args.steps
+        per, total_ms, sweep_ms = time_sweep(work, args.steps, args.warmup, stream, dist_ok)
+    total_ms, sweep_ms = max_over_ranks([total_ms, sweep_ms], device)
     value = aggregate_gbs(work.bytes, world, args.steps, total_ms)
-    single_value = aggregate_gbs(work.bytes, world, args.steps, single_ms)
-
-    # roofline of the dominant (only) kernel.  The timed region holds nothing
-    # but its launches (two streams, back to back), so its algorithmic bytes
-    # over the region's CUDA-event time is its achieved bandwidth, i.e. bytes
-    # per launch over the effective launch duration (region time / launches).
-    # The single-stream pass gives each launch's own event-timed duration.
-    call_bytes = [b for _, b in work.calls] * args.steps
-    achieved = sum(call_bytes) / (total_ms / 1e3) / GB
-    achieved_single = sum(call_bytes) / (sum(single_launch_ms) / 1e3) / GB
-    traffic = ncu_traffic(work.kernel)
-    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                "frac": round(achieved / peak, 4), "traffic": traffic,
-                "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
-                else "fallback 6650 GB/s", "kernel": work.kernel,
-                "timing": "CUDA events around the timed region, which holds only this kernel's launches "
-                          "(2 streams); effective launch duration = region time / launches",
-                "bytes_per_launch": int(np.mean([b for _, b in work.calls])),
-                "launches": work.launches * args.steps,
-                "effective_launch_us": round(1e3 * total_ms / (work.launches * args.steps), 2),
-                "single_stream_achieved": round(achieved_single, 1),
-                "single_stream_frac": round(achieved_single / peak, 4),
-                "single_stream_mean_launch_us": round(1e3 * float(np.mean(single_launch_ms)), 2)}
-
+    roof = sweep_roofline(per, peak, peak_kind, {"nvfp4_compute": work.compute_launches}, work.kernels)
+    launches = work.launches_per_layer * layers * args.steps
     line = {"metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": round(ms_step, 3), "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16->mxfp8 (e4m3 + e8m0)", "data": "synthetic",
+            "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16->mxfp8/nvfp4 (e4m3+e8m0, e2m1+e4m3+f32)",
+            "data": "synthetic",
             "frac_of_hbm_peak": round(value / world / peak, 4),
-            "config": {"workload": f"Qwen3-30B-A3B MXFP8 refit prequant: {args.layers} layers x 128 experts, "
-                                   "gate_up [1536,2048] + down [2048,768] bf16 N(0,0.02), 16 experts/call, "
-                                   "swizzled 128x4 E8M0 scales",
-                       "bytes_per_step_per_gpu": work.bytes, "launches_per_step": work.launches,
-                       "l2": "inputs larger than L2 (each step streams all layers resident in HBM)",
-                       "streams": args.streams,
-                       "issue": f"calls round-robin on {args.streams} streams (calls are independent)"
-                       if args.streams > 1 else "calls in order on one stream",
+            "config": {"workload": HEADLINE_WORKLOAD,
+                       "experts": "gate_up [3072,4096] + down [4096,1536] bf16 N(0,0.02), seed 5+layer",
+                       "calls": "6 per layer: MXFP8, NVFP4 amax computed, NVFP4 amax given; 128 experts each",
+                       "layers_per_step": layers, "bytes_per_step_per_gpu": work.bytes,
+                       "l2": "inputs larger than L2 (3.2 / 1.6 GB per call)",
+                       "timing": "sum of per-call CUDA events; layer regeneration untimed",
+                       "compute_path": "one cooperative launch" if args.compute_path == "single" else "three launches",
                        "parallelism": f"{world} independent replicas (weak scaling, no collective)"},
-            "single_stream": {"value": round(single_value, 1), "ms_per_step": round(single_ms / args.steps, 3)},
-            "roofline": roofline, "clocks": clocks.summary(),
-            "gpu_launches": work.launches * args.steps}
+            "roofline": roof, "clocks": clocks.summary(), "gpu_launches": launches,
+            "sweep_device_ms_per_step": round(sweep_ms / args.steps, 1)}
+    if refit is not None:
+        line["refit_30b"] = refit
     del work
     torch.cuda.empty_cache()
 
     if rank == 0 and not args.no_e2e:
-        line["e2e"] = e2e_refit(qz, device, steps=max(1, min(args.steps, 2)), warmup=1, layers=args.layers)
-    if rank == 0 and not args.no_extra:
-        line["extra"] = extra_workloads(qz, device, stream, peak)
+        line["e2e"] = e2e_prequant(qz, device, steps=2, warmup=1, compute_workspace=args.compute_path == "single")
+    if rank == 0 and not args.no_extra and args.config is None:
+        line["extra"] = extra_workloads(qz, device, stream, peak,
+                                        which=("tiny", "split", "fused", "nvfp4", "dequant", "merge", "colwise",
+                                               "gateup", "allreduce"))
     if rank == 0 and not args.no_cpu:
-        v, cores, desc, dt = oracle_refit_sample()
-        line["cpu_baseline"] = {"value": round(v, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
-                                "sample": desc, "seconds": round(dt, 2)}
+        import oracle
+        threads = oracle.host_threads()
+        v1, _, d1, t1, _ = oracle_prequant_sample(1, target_s=8.0)
+        vn, cores, dn, tn, _ = oracle_prequant_sample(threads, target_s=10.0)
+        line["cpu_baseline"] = {"value": round(vn, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+                                "sample": dn, "seconds": round(tn, 2),
+                                "single_thread": {"value": round(v1, 4), "unit": "GB/s", "cores": 1, "sample": d1,
+                                                  "seconds": round(t1, 2)}}
     if dist_ok:
         torch.distributed.barrier()
         torch.distributed.destroy_process_group()

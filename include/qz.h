@@ -101,9 +101,10 @@ typedef enum qz_nvfp4_scale_mode {
                                   16-byte (MXFP8) / 8-byte (NVFP4) aligned; sf not 16-byte
                                   aligned (swizzled); amax not 4-byte aligned */
 #define QZ_DERR_TOO_LARGE 0x8u /* the call's total tile or row count exceeds 2^31 - 1 */
-#define QZ_DERR_TIMEOUT 0x10u  /* a bounded wait of the single-launch computed-amax path (a CTA
-                                  waiting until every amax tile of a chunk has been counted)
-                                  exceeded its limit; the waiting CTA stopped early and some
+#define QZ_DERR_TIMEOUT 0x10u  /* a bounded wait of the single-launch computed-amax path (quantize
+                                  warps waiting until every amax warp is done with a chunk, or
+                                  amax warps waiting for their CTA's quantize warps) exceeded
+                                  qz_launch_opts.wait_limit_ns; the launch stopped early and some
                                   outputs are unwritten (no such wait is expected to expire) */
 #define QZ_DERR_CUT 0x20u      /* qz_split_fused_experts: the cut falls inside a scale block
                                   (FP8_BLOCK128: cut not a multiple of 128 and not the end) */
@@ -201,7 +202,33 @@ typedef struct qz_launch_opts {
                                waves (1 to 16), which streams large calls faster than one persistent
                                wave, and one CTA per tile below one wave; without it, one wave.  Any
                                value gives the same results. */
+    int64_t wait_limit_ns;  /* single-launch computed-amax path (a workspace, or the allocation-free entry
+                               point): the limit of each of its bounded waits, in nanoseconds of the
+                               GPU's global timer; 0 = the default of 20 ms.  A wait that runs out
+                               sets QZ_DERR_TIMEOUT and ends the launch early. */
+    unsigned int test_flags; /* 0 in normal use.  QZ_TEST_WITHHOLD_ARRIVALS makes the single-launch
+                               computed-amax path skip the counts that release its quantize warps, so
+                               every wait runs out: a test of the timeout path that needs no fault. */
+    unsigned int launch_flags; /* QZ_OPT_INDEPENDENT: see below; 0 otherwise. */
 } qz_launch_opts;
+
+/* qz_launch_opts.test_flags bits. */
+#define QZ_TEST_WITHHOLD_ARRIVALS 0x1u
+
+/* qz_launch_opts.launch_flags bits.
+ * The MXFP8 and NVFP4 tile kernels (qz_quantize_grouped_mxfp8; NVFP4 in the
+ * GIVEN and PER_TENSOR_COMPUTE-without-workspace modes) are launched with
+ * programmatic stream serialization: each lets the next such launch on the
+ * stream begin while its own last CTAs still run.  By default a launch then
+ * waits, before it reads anything, until the launch before it has completed
+ * and its writes are visible, so stream order holds as for any launch.
+ * QZ_OPT_INDEPENDENT declares that this call's table and inputs are written,
+ * and its outputs read or written, by no kernel that may still be running on
+ * the stream -- e.g. a series of calls on disjoint experts whose weights were
+ * written earlier -- and skips that wait: the call's tiles start as soon as
+ * the previous call's CTAs free their SMs, which recovers, on one stream, the
+ * ramp and tail of each short call.  A wrong declaration is a data race. */
+#define QZ_OPT_INDEPENDENT 0x1u
 
 /* Bytes of device scratch qz_quantize_grouped_nvfp4 uses for
  * QZ_NVFP4_PER_TENSOR_COMPUTE when given a workspace; 0 for n_experts outside
@@ -234,9 +261,11 @@ qz_status qz_quantize_grouped_mxfp8(const qz_expert *d_table, int n_experts, int
  * q = e2m1(RN32(x * r)), r = FTZ(RN32(S / s)) (0 if s == 0).
  * PER_TENSOR_COMPUTE without a workspace runs a clear, an amax pass and the
  * quantize pass (three launches in stream order, the input read twice from
- * HBM); with opts->d_workspace it runs one launch that takes each expert's
- * amax chunk by chunk and quantizes the chunk while its input is still in L2
- * (plus a memset of the workspace).  PER_ROW reads each row once.
+ * HBM); with opts->d_workspace it runs one cooperative launch (plus a memset
+ * of the workspace) in which amax warps read each chunk of whole experts from
+ * HBM one chunk ahead of quantize warps, which re-read it from L2 once every
+ * amax warp of the grid is done with it (bounded waits: wait_limit_ns).
+ * PER_ROW reads each row once.
  * Entries may share one amax slot, so that the gate and up halves of a fused
  * expert ([FOLD]: one amax over the fused (2I, H) slice, one weight_scale_2)
  * are quantized straight into their own storage in one call: in GIVEN mode

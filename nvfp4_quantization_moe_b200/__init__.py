@@ -7,7 +7,8 @@ There is no CPU or library fallback: every call raises if the library is
 missing or reports an error.
 """
 from .binding import (  # noqa: F401
-    AMAX_NONE, AMAX_PER_ROW, AMAX_PER_TENSOR, DERR_ALIGN, DERR_CUT, DERR_NULL, DERR_SHAPE, DERR_TOO_LARGE, EXPORTED,
+    AMAX_NONE, AMAX_PER_ROW, AMAX_PER_TENSOR, DERR_ALIGN, DERR_CUT, DERR_NULL, DERR_SHAPE, DERR_TIMEOUT,
+    DERR_TOO_LARGE, EXPORTED, OPT_INDEPENDENT, TEST_WITHHOLD_ARRIVALS,
     FMT_FP8_BLOCK128, FMT_MXFP8, FMT_NVFP4, LIB_PATH, MAX_EXPERTS, MAX_HIDDEN, MAX_RANKS, NVFP4_PER_ROW,
     NVFP4_PER_TENSOR_COMPUTE, NVFP4_PER_TENSOR_GIVEN, QZ_ERR_ALIGNMENT, QZ_ERR_CUDA, QZ_ERR_INVALID_ARG,
     QZ_ERR_UNSUPPORTED, QZ_OK, SF_LINEAR, SF_SWIZZLED, STATIC_WS_MAX_EXPERTS, DqEntry, DqTable, Entry, ExpertTable,

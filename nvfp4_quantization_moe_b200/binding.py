@@ -27,7 +27,9 @@ FMT_MXFP8, FMT_NVFP4, FMT_FP8_BLOCK128 = 0, 1, 2
 NVFP4_PER_TENSOR_GIVEN, NVFP4_PER_TENSOR_COMPUTE, NVFP4_PER_ROW = 0, 1, 2
 AMAX_NONE, AMAX_PER_TENSOR, AMAX_PER_ROW = 0, 1, 2
 DERR_SHAPE, DERR_NULL, DERR_ALIGN, DERR_TOO_LARGE = 0x1, 0x2, 0x4, 0x8
-DERR_CUT = 0x20
+DERR_TIMEOUT, DERR_CUT = 0x10, 0x20
+TEST_WITHHOLD_ARRIVALS = 0x1
+OPT_INDEPENDENT = 0x1
 MAX_EXPERTS = 4096
 MAX_HIDDEN = 16384
 MAX_RANKS = 8
@@ -82,7 +84,8 @@ class _FusedSplit(ctypes.Structure):
 
 class _Opts(ctypes.Structure):
     _fields_ = [("d_err", ctypes.c_void_p), ("max_ctas", ctypes.c_int), ("d_workspace", ctypes.c_void_p),
-                ("workspace_bytes", ctypes.c_size_t), ("elems_hint", ctypes.c_int64)]
+                ("workspace_bytes", ctypes.c_size_t), ("elems_hint", ctypes.c_int64),
+                ("wait_limit_ns", ctypes.c_int64), ("test_flags", ctypes.c_uint), ("launch_flags", ctypes.c_uint)]
 
 
 assert ctypes.sizeof(_Expert) == 56 and ctypes.sizeof(_SfPair) == 32 and ctypes.sizeof(_DqExpert) == 56
@@ -151,15 +154,19 @@ def _stream_ptr(stream) -> ctypes.c_void_p:
     return ctypes.c_void_p(int(stream.cuda_stream) if hasattr(stream, "cuda_stream") else int(stream))
 
 
-def _opts(err: Optional[torch.Tensor], max_ctas: int, workspace: Optional[torch.Tensor] = None, elems_hint: int = 0):
-    if err is None and not max_ctas and workspace is None and not elems_hint:
+def _opts(err: Optional[torch.Tensor], max_ctas: int, workspace: Optional[torch.Tensor] = None, elems_hint: int = 0,
+          wait_limit_ns: int = 0, test_flags: int = 0, launch_flags: int = 0):
+    if (err is None and not max_ctas and workspace is None and not elems_hint and not wait_limit_ns and not test_flags
+            and not launch_flags):
         return None
     if err is not None:
         assert err.dtype in (torch.int32, torch.uint32) and err.is_cuda and err.numel() >= 1
     ws_ptr = workspace.data_ptr() if workspace is not None else 0
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     return ctypes.byref(_Opts(ctypes.c_void_p(err.data_ptr() if err is not None else 0), int(max_ctas),
-                              ctypes.c_void_p(ws_ptr), ctypes.c_size_t(ws_bytes), ctypes.c_int64(int(elems_hint))))
+                              ctypes.c_void_p(ws_ptr), ctypes.c_size_t(ws_bytes), ctypes.c_int64(int(elems_hint)),
+                              ctypes.c_int64(int(wait_limit_ns)), ctypes.c_uint(int(test_flags)),
+                              ctypes.c_uint(int(launch_flags))))
 
 
 def workspace_bytes(n_experts: int) -> int:
@@ -349,26 +356,36 @@ class SfPairTable:
 # entry points
 # ---------------------------------------------------------------------------
 
-def quantize_grouped_mxfp8(table: ExpertTable, layout: int, stream=None, err=None, max_ctas: int = 0):
-    """MXFP8 over the table; the table's element count goes along as the grid-size hint."""
+def quantize_grouped_mxfp8(table: ExpertTable, layout: int, stream=None, err=None, max_ctas: int = 0,
+                           independent: bool = False):
+    """MXFP8 over the table; the table's element count goes along as the
+    grid-size hint.  ``independent`` sets QZ_OPT_INDEPENDENT (the call touches
+    nothing that work still running on the stream touches)."""
     _check(load().qz_quantize_grouped_mxfp8(ctypes.c_void_p(table.ptr), table.n, int(layout),
                                             _stream_ptr(stream),
-                                            _opts(err, max_ctas, elems_hint=getattr(table, "elems", 0))),
+                                            _opts(err, max_ctas, elems_hint=getattr(table, "elems", 0),
+                                                  launch_flags=OPT_INDEPENDENT if independent else 0)),
            "qz_quantize_grouped_mxfp8")
 
 
 def quantize_grouped_nvfp4(table: ExpertTable, mode: int, layout: int, stream=None, err=None, max_ctas: int = 0,
-                           workspace: Optional[torch.Tensor] = None):
+                           workspace: Optional[torch.Tensor] = None, wait_limit_ns: int = 0, test_flags: int = 0,
+                           independent: bool = False):
     _check(load().qz_quantize_grouped_nvfp4(ctypes.c_void_p(table.ptr), table.n, int(mode), int(layout),
-                                            _stream_ptr(stream), _opts(err, max_ctas, workspace)),
+                                            _stream_ptr(stream),
+                                            _opts(err, max_ctas, workspace, wait_limit_ns=wait_limit_ns,
+                                                  test_flags=test_flags,
+                                                  launch_flags=OPT_INDEPENDENT if independent else 0)),
            "qz_quantize_grouped_nvfp4")
 
 
-def quantize_grouped_nvfp4_compute_noalloc(table: ExpertTable, layout: int, stream=None, err=None, max_ctas: int = 0):
+def quantize_grouped_nvfp4_compute_noalloc(table: ExpertTable, layout: int, stream=None, err=None, max_ctas: int = 0,
+                                           wait_limit_ns: int = 0):
     """NVFP4 with computed per-tensor amax, scratch inside the library (no
     device allocation by anyone; see qz_quantize_grouped_nvfp4_compute_noalloc)."""
     _check(load().qz_quantize_grouped_nvfp4_compute_noalloc(ctypes.c_void_p(table.ptr), table.n, int(layout),
-                                                            _stream_ptr(stream), _opts(err, max_ctas)),
+                                                            _stream_ptr(stream),
+                                                            _opts(err, max_ctas, wait_limit_ns=wait_limit_ns)),
            "qz_quantize_grouped_nvfp4_compute_noalloc")
 
 

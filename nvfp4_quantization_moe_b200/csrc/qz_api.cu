@@ -11,9 +11,10 @@
 #include "../../include/qz.h"
 
 namespace qz {
-cudaError_t launch_mxfp8(const qz_expert* table, int n, int layout, int grid, cudaStream_t s, unsigned* d_err);
+cudaError_t launch_mxfp8(const qz_expert* table, int n, int layout, int grid, cudaStream_t s, unsigned* d_err,
+                         bool independent);
 cudaError_t launch_nvfp4_tensor(const qz_expert* table, int n, int layout, bool compute_amax, int grid,
-                                cudaStream_t s, unsigned* d_err);
+                                cudaStream_t s, unsigned* d_err, bool independent);
 cudaError_t launch_nvfp4_rows(const qz_expert* table, int n, int layout, int grid, cudaStream_t s, unsigned* d_err);
 cudaError_t launch_swizzle(const qz_sf_pair* table, int n, int grid, cudaStream_t s, unsigned* d_err);
 cudaError_t launch_rmsnorm_quant(const uint16_t* x, const uint16_t* r, const uint16_t* g, float eps, int64_t T,
@@ -26,9 +27,9 @@ cudaError_t launch_allreduce_norm_quant(const uint16_t* const* xs, int n_x, cons
 int grouped_blocks_per_sm(int which, int n);
 size_t workspace_bytes(int n);
 cudaError_t launch_nvfp4_compute_l2(const qz_expert* table, int n, int layout, int grid, unsigned* ws,
-                                    cudaStream_t s, unsigned* d_err);
+                                    cudaStream_t s, unsigned* d_err, long long wait_ns, unsigned test_flags);
 cudaError_t launch_nvfp4_compute_l2_static(const qz_expert* table, int n, int layout, int grid, cudaStream_t s,
-                                           unsigned* d_err);
+                                           unsigned* d_err, long long wait_ns, unsigned test_flags);
 int rows_blocks_per_sm(int n);
 cudaError_t launch_dequant(const qz_dq_expert* table, int n, int fmt, bool per_row, int layout, int grid,
                            cudaStream_t s, unsigned* d_err);
@@ -101,6 +102,9 @@ int device_sms() {
 bool aligned(const void* p, uintptr_t a) { return ((uintptr_t)p & (a - 1)) == 0; }
 
 unsigned* err_word(const qz_launch_opts* opts) { return opts ? opts->d_err : nullptr; }
+long long wait_limit(const qz_launch_opts* opts) { return opts ? (long long)opts->wait_limit_ns : 0; }
+unsigned test_flags(const qz_launch_opts* opts) { return opts ? opts->test_flags : 0u; }
+bool independent(const qz_launch_opts* opts) { return opts && (opts->launch_flags & QZ_OPT_INDEPENDENT) != 0u; }
 
 qz_status check_table(const void* table, int n) {
     if (n < 0 || n > QZ_MAX_EXPERTS) return QZ_ERR_INVALID_ARG;
@@ -161,7 +165,7 @@ qz_status qz_quantize_grouped_mxfp8(const qz_expert* d_table, int n_experts, int
     if (!valid_layout(layout)) return QZ_ERR_INVALID_ARG;
     if (n_experts == 0) return QZ_OK;
     return from_cuda(qz::launch_mxfp8(d_table, n_experts, layout, sized_grid(0, opts), (cudaStream_t)stream,
-                                      err_word(opts)));
+                                      err_word(opts), independent(opts)));
 }
 
 qz_status qz_quantize_grouped_nvfp4(const qz_expert* d_table, int n_experts, int mode, int layout, void* stream,
@@ -171,6 +175,7 @@ qz_status qz_quantize_grouped_nvfp4(const qz_expert* d_table, int n_experts, int
     if (!valid_layout(layout)) return QZ_ERR_INVALID_ARG;
     if (mode != QZ_NVFP4_PER_TENSOR_GIVEN && mode != QZ_NVFP4_PER_TENSOR_COMPUTE && mode != QZ_NVFP4_PER_ROW)
         return QZ_ERR_INVALID_ARG;
+    if (opts && opts->wait_limit_ns < 0) return QZ_ERR_INVALID_ARG;
     if (mode == QZ_NVFP4_PER_TENSOR_COMPUTE && opts && opts->d_workspace) {
         if (n_experts > 0 && opts->workspace_bytes < qz::workspace_bytes(n_experts)) return QZ_ERR_INVALID_ARG;
         if (!aligned(opts->d_workspace, 4)) return QZ_ERR_ALIGNMENT;
@@ -179,11 +184,12 @@ qz_status qz_quantize_grouped_nvfp4(const qz_expert* d_table, int n_experts, int
     cudaStream_t s = (cudaStream_t)stream;
     if (mode == QZ_NVFP4_PER_TENSOR_COMPUTE && opts && opts->d_workspace)
         return from_cuda(qz::launch_nvfp4_compute_l2(d_table, n_experts, layout, wave_grid(5, opts),
-                                                     static_cast<unsigned*>(opts->d_workspace), s, err_word(opts)));
+                                                     static_cast<unsigned*>(opts->d_workspace), s, err_word(opts),
+                                                     wait_limit(opts), test_flags(opts)));
     if (mode == QZ_NVFP4_PER_ROW)
         return from_cuda(qz::launch_nvfp4_rows(d_table, n_experts, layout, wave_grid(4, opts), s, err_word(opts)));
     return from_cuda(qz::launch_nvfp4_tensor(d_table, n_experts, layout, mode == QZ_NVFP4_PER_TENSOR_COMPUTE,
-                                             wave_grid(1, opts), s, err_word(opts)));
+                                             wave_grid(1, opts), s, err_word(opts), independent(opts)));
 }
 
 qz_status qz_rmsnorm_quantize(const void* d_x, const void* d_residual, const void* d_gamma, float eps, int64_t T,
@@ -258,10 +264,12 @@ qz_status qz_quantize_grouped_nvfp4_compute_noalloc(const qz_expert* d_table, in
                                                     void* stream, const qz_launch_opts* opts) {
     if (n_experts < 0 || n_experts > QZ_STATIC_WS_MAX_EXPERTS) return QZ_ERR_INVALID_ARG;
     if (n_experts > 0 && d_table == nullptr) return QZ_ERR_INVALID_ARG;
+    if (opts && opts->wait_limit_ns < 0) return QZ_ERR_INVALID_ARG;
     if (!valid_layout(layout)) return QZ_ERR_INVALID_ARG;
     if (n_experts == 0) return QZ_OK;
     return from_cuda(qz::launch_nvfp4_compute_l2_static(d_table, n_experts, layout, wave_grid(5, opts),
-                                                        (cudaStream_t)stream, err_word(opts)));
+                                                        (cudaStream_t)stream, err_word(opts), wait_limit(opts),
+                                                        test_flags(opts)));
 }
 
 qz_status qz_dequantize_grouped(const qz_dq_expert* d_table, int n_experts, int fmt, int per_row, int layout,

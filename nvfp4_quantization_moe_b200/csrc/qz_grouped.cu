@@ -235,15 +235,26 @@ __device__ __forceinline__ void tile_flush_sf(const TileRef& t, int w, int lane,
     __syncwarp();
 }
 
+// Programmatic dependent launch (PTX griddepcontrol, sm_90+).  The tile
+// kernels are launched with programmatic stream serialization: each CTA
+// allows the next such launch on the stream to start as soon as it begins,
+// and -- unless the call was declared independent of the work before it --
+// waits for the preceding grid to complete (and its writes to be visible)
+// before it reads anything.  Without a preceding trigger both are no-ops.
+__device__ __forceinline__ void pdl_allow_next() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait_prior() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 template <int FMT, int LAYOUT>
 __global__ void __launch_bounds__(kThreads, 3) grouped_tile_kernel(const qz_expert* __restrict__ table, int n,
-                                                                   unsigned* d_err) {
+                                                                   unsigned* d_err, int wait_prior) {
     using G = TileGeo<FMT>;
     extern __shared__ int s_prefix[];
     __shared__ long long s_scan[33];
     __shared__ __align__(16) uint8_t s_sf[kThreads / 32][64 * G::kSfTiles];
     __shared__ float s_inv[16];
     constexpr bool kAmax = FMT == QZ_FMT_NVFP4;
+    pdl_allow_next();
+    if (wait_prior) pdl_wait_prior();
     if (kAmax) fill_inv_table(s_inv);  // published by the barriers in block_prefix
     const int total = block_prefix(n, s_prefix, s_scan, TableTiles<FMT, LAYOUT, kAmax>{table, d_err}, d_err);
     const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -296,245 +307,403 @@ __global__ void amax_clear_kernel(const qz_expert* __restrict__ table, int n, in
 }
 
 // Same tile walk and prefetch ring as the quantize kernel; each warp keeps a
-// running maximum while its tiles stay in one expert and publishes it with
-// one atomic max (non-negative floats order like their bit patterns).
+// running maximum while its tiles stay in one expert and folds it into the
+// CTA's per-expert maximum in shared memory; at the end the CTA publishes one
+// atomic max per expert it touched (non-negative floats order like their bit
+// patterns).  Folding in shared memory first keeps the global atomics to one
+// per CTA and expert: amax slots of many experts often share a few cache
+// lines, where atomics from every warp would serialize.
 template <int LAYOUT>
 __global__ void __launch_bounds__(kThreads, 3) amax_grouped_kernel(const qz_expert* __restrict__ table, int n,
                                                                    unsigned* d_err) {
     using G = TileGeo<QZ_FMT_NVFP4>;
     extern __shared__ int s_prefix[];
+    unsigned* s_amax = reinterpret_cast<unsigned*>(s_prefix + (n + 1));  // n words
     __shared__ long long s_scan[33];
+    for (int i = threadIdx.x; i < n; i += blockDim.x) s_amax[i] = 0u;  // published by block_prefix's barriers
     const int total = block_prefix(n, s_prefix, s_scan, TableTiles<QZ_FMT_NVFP4, LAYOUT, true>{table, d_err}, d_err);
     const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
     int tile = blockIdx.x;
-    if (tile >= total) return;
-    TileRef cur = tile_ref<QZ_FMT_NVFP4, LAYOUT>(table, s_prefix, n, tile, w, lane);
-    uint32_t v[G::kPasses][G::kWords];
+    if (tile < total) {
+        TileRef cur = tile_ref<QZ_FMT_NVFP4, LAYOUT>(table, s_prefix, n, tile, w, lane);
+        uint32_t v[G::kPasses][G::kWords];
 #pragma unroll
-    for (int p = 0; p < G::kPasses; ++p) tile_load<QZ_FMT_NVFP4>(cur, p, v[p]);
-    uint32_t run = 0;
-    for (;;) {
-        const int next = tile + gridDim.x;
-        const bool more = next < total;
-        const TileRef nxt = more ? tile_ref<QZ_FMT_NVFP4, LAYOUT>(table, s_prefix, n, next, w, lane, cur.expert) : cur;
+        for (int p = 0; p < G::kPasses; ++p) tile_load<QZ_FMT_NVFP4>(cur, p, v[p]);
+        uint32_t run = 0;
+        for (;;) {
+            const int next = tile + gridDim.x;
+            const bool more = next < total;
+            const TileRef nxt = more ? tile_ref<QZ_FMT_NVFP4, LAYOUT>(table, s_prefix, n, next, w, lane, cur.expert) : cur;
 #pragma unroll
-        for (int p = 0; p < G::kPasses; ++p) {
-            run = max(run, absmax_words<G::kWords>(v[p]));
-            if (more) tile_load<QZ_FMT_NVFP4>(nxt, p, v[p]);
+            for (int p = 0; p < G::kPasses; ++p) {
+                run = max(run, absmax_words<G::kWords>(v[p]));
+                if (more) tile_load<QZ_FMT_NVFP4>(nxt, p, v[p]);
+            }
+            if (!more || nxt.expert != cur.expert) {
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) run = max(run, __shfl_xor_sync(0xFFFFFFFFu, run, o));
+                if (lane == 0 && run != 0u) atomicMax(s_amax + cur.expert, run << 16);
+                run = 0;
+            }
+            if (!more) break;
+            cur = nxt;
+            tile = next;
         }
-        if (!more || nxt.expert != cur.expert) {
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) run = max(run, __shfl_xor_sync(0xFFFFFFFFu, run, o));
-            if (lane == 0) atomicMax(reinterpret_cast<unsigned int*>(const_cast<float*>(cur.amax)), run << 16);
-            run = 0;
-        }
-        if (!more) break;
-        cur = nxt;
-        tile = next;
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+        const unsigned m = s_amax[i];
+        if (m != 0u) atomicMax(reinterpret_cast<unsigned int*>(load_entry(table, i).amax), m);
     }
 }
 
 // ---------------------------------------------------------------------------
-// NVFP4 with a computed per-tensor amax in one launch (L2-chunked)
+// NVFP4 with a computed per-tensor amax in one launch: bulk copies feed the
+// amax side from HBM ahead of the quantize warps, which re-read from L2
 //
-// The experts are cut into chunks of consecutive experts holding about
-// kChunkTiles tiles (~16 MB of bf16).  Work items are runs of up to
-// kItemTiles tiles of one chunk, fetched from an atomic counter in segment
-// order: segment s holds A(s) then Q(s - kLag) (the last kLag segments hold
-// only Q items).  An A item folds its tiles' amax into their experts' slots
-// (atomic max) and adds its tile count to its chunk's done counter; a Q item
-// quantizes tiles of chunk s - kLag once that chunk's A tiles are all done,
-// re-reading the input from L2 where the A pass left it.  kLag chunks of A
-// items (more than the items in flight on the whole GPU) separate a chunk's
-// A and Q items, so Q items rarely wait, while the kLag + 1 live chunks stay
-// well inside L2.  Every item waits only on items fetched before it and A
-// items never wait, so all items finish whatever the number of resident CTAs;
-// the wait is still bounded (QZ_DERR_TIMEOUT).  A CTA consumes each fetched
-// item index one item later, so the atomic's latency is hidden.
+// A tensor's encode scale needs the amax of the whole tensor, so no element
+// of an expert can be quantized before all of it has been read.  Every CTA
+// (one per SM, all resident: a cooperative launch) runs
+//  - a producer warp that walks this CTA's amax units (units b, b + grid, ...
+//    of the call; a unit is up to 32 KB of one expert: a block of whole rows,
+//    or one 16384-column segment of a row) and copies each into a ring of
+//    kStages shared-memory stages with cp.async.bulk (the copy engine moves
+//    the bytes; no register holds them in flight), completion counted in
+//    bytes on each stage's mbarrier;
+//  - kStages consumer warps (consumer i takes stage i): the unit's largest
+//    magnitude from shared memory, folded into its expert's amax word (atomic
+//    max of bf16 magnitude bits), then -- after a fence -- one count on the
+//    expert's unit counter; a consumer holds no global load in flight, so its
+//    fence waits only for its own two atomics;
+//  - kQWarps quantize warps (the tile walk of the grouped kernel: 8 warps own
+//    the row groups of a 128 x 128 tile) that take tiles b, b + grid, ... and
+//    quantize each once its expert's unit counter is complete (a bounded
+//    acquire wait), re-reading the input from L2 with loads that release the
+//    lines.
+// The producer copies a unit only while its expert starts within kWindowTiles
+// tiles of this CTA's quantize front, so about kWindowTiles tiles plus one
+// expert stay live in L2 (an expert whose first tile is inside the window is
+// always admitted whole, so the quantize warps can never wait on a unit the
+// window holds back).  Every wait is bounded by a time limit; when one runs
+// out the kernel reports QZ_DERR_TIMEOUT, raises an abort word that ends the
+// other waits early, lets the copies it issued land, and returns.
 //
 // Workspace (caller's device memory, zeroed by the call):
-//   ws[0] next item, ws[8 + k] done A tiles of chunk k, then one amax word per
-//   expert (bf16 magnitude bits << 16).
+//   ws[0] abort word; ws[8 + e] units of expert e folded into its amax;
+//   ws[8 + kMaxChunks + e] expert e's amax (bf16 magnitude bits << 16).
 // ---------------------------------------------------------------------------
 
-constexpr int kChunkTiles = 512;       // ~16 MB of bf16 input per chunk
-constexpr int kItemTiles = 2;          // tiles per work item
-constexpr int kLag = 2;                // chunks between a chunk's A items and its Q items
-constexpr int kMaxChunks = 4096;
+constexpr int kQGroups = 1;            // quantize groups: each walks its own tiles
+constexpr int kQWarps = 8 * kQGroups;  // quantize warps: 8 per group (the 8 row groups of a tile)
+constexpr int kStages = 4;             // shared-memory stages of the amax ring (one consumer warp each)
+constexpr int kUnitBytes = 32768;      // bytes of one amax unit (one stage)
+constexpr int kWindowTiles = 1536;     // how far (in tiles, ~48 MB) the copies may run ahead
+constexpr int kPipeThreads = 32 * (kQWarps + 1 + kStages);
+constexpr int kMaxChunks = 4096;       // workspace words reserved for the per-expert unit counters
 constexpr int kWsHeader = 8;
-static_assert(kLag >= 1, "Q items of a chunk must follow all of its A items");
+constexpr long long kDefaultWaitNs = 20LL * 1000 * 1000;  // 20 ms: far above any legitimate wait
+static_assert(QZ_MAX_EXPERTS <= kMaxChunks, "one unit counter per expert");
 
 __host__ __device__ constexpr size_t workspace_words(int n) { return (size_t)kWsHeader + kMaxChunks + (size_t)n; }
 
-struct ItemRef {
-    int first_tile;  // first tile of the run
-    int ntiles;      // tiles in the run (1..kItemTiles)
-    int chunk;
-    bool is_a;
+__device__ __forceinline__ long long global_ns() {
+    long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// --- mbarrier and bulk-copy primitives (PTX ISA: mbarrier, cp.async.bulk) ---
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, unsigned count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, unsigned bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
+
+// true once the phase with the given parity has completed
+__device__ __forceinline__ bool mbar_test(uint64_t* bar, unsigned parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_addr(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// global -> shared bulk copy completing `bytes` on bar (16-byte aligned
+// addresses, bytes a multiple of 16; the CTA is its own cluster)
+__device__ __forceinline__ void bulk_copy_g2s(void* dst, const void* src, unsigned bytes, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_addr(dst)),
+        "l"(src), "r"(bytes), "r"(smem_addr(bar))
+        : "memory");
+}
+
+// --- amax units ---
+
+// How an expert is cut into units of at most kUnitBytes: row blocks of krows
+// whole rows, or (rows wider than a unit) row segments of seg columns.
+struct UnitGeo {
+    int seg;    // columns per segment (cols, or kUnitBytes / 2 for wider rows)
+    int nseg;   // segments per row
+    int krows;  // rows per unit
 };
 
+__device__ __forceinline__ UnitGeo unit_geo(const qz_expert& E) {
+    UnitGeo g;
+    const int64_t wide = kUnitBytes / 2;
+    g.seg = (int)(E.cols < wide ? E.cols : wide);
+    g.nseg = (int)((E.cols + g.seg - 1) / g.seg);
+    g.krows = max(1, kUnitBytes / (2 * g.seg));
+    return g;
+}
+
+__device__ __forceinline__ long long unit_count(const qz_expert& E) {
+    const UnitGeo g = unit_geo(E);
+    return ((E.rows + g.krows - 1) / g.krows) * g.nseg;
+}
+
 template <int LAYOUT>
-__global__ void __launch_bounds__(kThreads, 3) nvfp4_compute_l2_kernel(const qz_expert* __restrict__ table, int n,
-                                                                       unsigned* __restrict__ ws, unsigned* d_err) {
+struct TableUnits {
+    const qz_expert* table;
+    __device__ long long operator()(int i) const {
+        const qz_expert e = load_entry(table, i);
+        if (e.rows == 0 || entry_errors(e, QZ_FMT_NVFP4, LAYOUT, true)) return 0;
+        return unit_count(e);
+    }
+};
+
+// Warp-uniform bounded wait until every lane sees `ready()`; false when the
+// time limit ran out (QZ_DERR_TIMEOUT, abort raised) or the kernel aborted.
+template <typename Ready>
+__device__ __forceinline__ bool bounded_wait(Ready ready, volatile unsigned* abort_word, volatile int* s_abort,
+                                             long long limit, unsigned* d_err, int lane, unsigned sleep_ns) {
+    const long long t0 = global_ns();
+    for (;;) {
+        if (__all_sync(0xFFFFFFFFu, ready())) return true;
+        const bool aborted = *abort_word != 0u || *s_abort != 0;
+        const bool late = global_ns() - t0 > limit;
+        if (__any_sync(0xFFFFFFFFu, aborted || late)) {
+            if (!__any_sync(0xFFFFFFFFu, aborted) && lane == 0) {
+                if (d_err) atomicOr(d_err, QZ_DERR_TIMEOUT);
+                *abort_word = 1u;
+                *s_abort = 1;
+            }
+            return false;
+        }
+        if (sleep_ns) __nanosleep(sleep_ns);
+    }
+}
+
+template <int LAYOUT>
+__global__ void __launch_bounds__(kPipeThreads, 1) nvfp4_compute_pipe_kernel(
+    const qz_expert* __restrict__ table, int n, unsigned* __restrict__ ws, unsigned* d_err, long long wait_ns,
+    unsigned test_flags) {
     using G = TileGeo<QZ_FMT_NVFP4>;
-    extern __shared__ int s_dyn[];
-    int* s_prefix = s_dyn;                 // n + 1: first tile of each expert
-    int* s_cf = s_dyn + (n + 1);           // nchunks + 1: first tile of each chunk
-    int* s_seg = s_cf + (kMaxChunks + 1);  // nchunks + kLag + 1: first item of each segment
+    extern __shared__ __align__(128) unsigned char s_dyn[];
+    unsigned char* s_ring = s_dyn;                                           // kStages x kUnitBytes
+    int* s_prefix = reinterpret_cast<int*>(s_dyn + kStages * kUnitBytes);   // n + 1: first tile of each expert
+    int* s_uprefix = s_prefix + (n + 1);                                     // n + 1: first unit of each expert
+    unsigned* s_emax = reinterpret_cast<unsigned*>(s_uprefix + (n + 1));     // n: this CTA's maximum per expert
+    unsigned* s_ecnt = s_emax + n;                                           // n: this CTA's units folded per expert
     __shared__ long long s_scan[33];
-    __shared__ __align__(16) uint8_t s_sf[kThreads / 32][64 * G::kSfTiles];
+    __shared__ __align__(16) uint8_t s_sf[kQWarps][64 * G::kSfTiles];
     __shared__ float s_inv[16];
-    __shared__ int s_item[4];
-    __shared__ unsigned s_ok[2];
+    __shared__ __align__(8) uint64_t s_full[kStages], s_empty[kStages];
+    __shared__ int s_unit_expert[kStages];
+    __shared__ unsigned s_unit_bytes[kStages];
+    __shared__ volatile int s_qtile[kQWarps];  // quantize warp w has done this CTA's tiles below this
+    __shared__ volatile int s_abort;
     fill_inv_table(s_inv);
+    if (threadIdx.x < kQWarps) s_qtile[threadIdx.x] = 0;
+    for (int i = threadIdx.x; i < n; i += blockDim.x) s_emax[i] = s_ecnt[i] = 0u;  // published by block_prefix
+    if (threadIdx.x == 0) {
+        s_abort = 0;
+        for (int i = 0; i < kStages; ++i) {
+            mbar_init(&s_full[i], 1);
+            mbar_init(&s_empty[i], 1);
+        }
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
     const int total = block_prefix(n, s_prefix, s_scan, TableTiles<QZ_FMT_NVFP4, LAYOUT, true>{table, d_err}, d_err);
-    if (total == 0) return;
-    const int tpc = max(kChunkTiles, (total + kMaxChunks - 1) / kMaxChunks);  // tiles per chunk
-    const int nchunks = (total + tpc - 1) / tpc;
-    // chunk k starts at the first expert whose first tile is >= k * tpc
-    for (int k = threadIdx.x; k <= nchunks; k += blockDim.x) {
-        const int target = k * tpc;
-        int lo = 0, hi = n;  // first e in [0, n] with s_prefix[e] >= target (s_prefix[n] = total)
-        while (lo < hi) {
-            const int mid = (lo + hi) >> 1;
-            if (s_prefix[mid] >= target) hi = mid; else lo = mid + 1;
-        }
-        s_cf[k] = s_prefix[lo];
-    }
-    __syncthreads();
-    // items of chunk k: ceil(T(k) / kItemTiles); segment s = A(s) then Q(s - kLag)
-    auto chunk_items = [&](int k) {
-        return (k >= 0 && k < nchunks) ? (s_cf[k + 1] - s_cf[k] + kItemTiles - 1) / kItemTiles : 0;
-    };
-    const int nseg = nchunks + kLag;
-    if (threadIdx.x == 0) {
-        int run = 0;
-        for (int k = 0; k < nseg; ++k) {
-            s_seg[k] = run;
-            run += chunk_items(k) + chunk_items(k - kLag);
-        }
-        s_seg[nseg] = run;
-    }
-    unsigned* next_item = ws;
-    unsigned* done = ws + kWsHeader;
+    const int units = block_prefix(n, s_uprefix, s_scan, TableUnits<LAYOUT>{table}, d_err);
+    if (total == 0 || units == 0) return;
+
+    volatile unsigned* abort_word = ws;
+    unsigned* counted = ws + kWsHeader;
     unsigned* amax_ws = ws + kWsHeader + kMaxChunks;
-    unsigned pending = 0;  // thread 0: an item index fetched one iteration ahead
-    if (threadIdx.x == 0) {
-        s_item[0] = (int)atomicAdd(next_item, 1u);
-        pending = atomicAdd(next_item, 1u);
-    }
-    __syncthreads();
-    const int items = s_seg[nseg];
-    const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int wid = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int grid = gridDim.x, b = blockIdx.x;
+    const long long limit = wait_ns > 0 ? wait_ns : kDefaultWaitNs;
 
-    auto decode = [&](int j) {
-        int lo = 0, hi = nseg - 1;  // last s with s_seg[s] <= j
-        while (lo < hi) {
-            const int mid = (lo + hi + 1) >> 1;
-            if (s_seg[mid] <= j) lo = mid; else hi = mid - 1;
+    if (wid < kQWarps) {
+        // ---------------- quantize warps: group q takes tiles b + (q + kQGroups i) grid ----------------
+        const int w = wid & 7;              // row group within the tile
+        const int qg = wid >> 3;            // quantize group
+        const int stride = grid * kQGroups;
+        int t = b + qg * grid;
+        if (t >= total) {
+            s_qtile[wid] = total;
+            return;
         }
-        const int off = j - s_seg[lo];
-        const int a_items = chunk_items(lo);
-        ItemRef r;
-        r.is_a = off < a_items;
-        r.chunk = r.is_a ? lo : lo - kLag;
-        const int idx = r.is_a ? off : off - a_items;
-        r.first_tile = s_cf[r.chunk] + idx * kItemTiles;
-        r.ntiles = min(kItemTiles, s_cf[r.chunk + 1] - r.first_tile);
-        return r;
-    };
-
-    // A reads keep their lines in L2 for the Q re-read; Q reads release them
-    auto load_tile = [&](const TileRef& t, bool a_item, uint32_t (&v)[G::kPasses][G::kWords]) {
-        if (a_item) {
+        s_qtile[wid] = t;
+        TileRef cur = tile_ref<QZ_FMT_NVFP4, LAYOUT>(table, s_prefix, n, t, w, lane);
+        uint32_t v[G::kPasses][G::kWords];
 #pragma unroll
-            for (int p = 0; p < G::kPasses; ++p) tile_load<QZ_FMT_NVFP4, kL2Last>(t, p, v[p]);
-        } else {
+        for (int p = 0; p < G::kPasses; ++p) tile_load<QZ_FMT_NVFP4, kL2First>(cur, p, v[p]);
+        int ready = -1;  // the last expert whose amax is known complete
+        for (;;) {
+            const int t2 = t + stride;
+            const bool more = t2 < total;
+            const TileRef nxt = more ? tile_ref<QZ_FMT_NVFP4, LAYOUT>(table, s_prefix, n, t2, w, lane, cur.expert) : cur;
+            if (cur.expert != ready) {
+                const unsigned need = (unsigned)(s_uprefix[cur.expert + 1] - s_uprefix[cur.expert]);
+                const unsigned* cnt = counted + cur.expert;
+                if (!bounded_wait([&] { return ld_acquire_gpu(cnt) >= need; }, abort_word, &s_abort, limit, d_err,
+                                  lane, 32))
+                    return;
+                ready = cur.expert;
+            }
+            // ordered after this lane's acquire of the expert's unit count
+            const float A = __uint_as_float(ld_relaxed_gpu(amax_ws + cur.expert));
+            const float S = nvfp4_encode_scale(A);
+            const float qm = rcp_lane_quotient(S, s_inv, lane);
 #pragma unroll
-            for (int p = 0; p < G::kPasses; ++p) tile_load<QZ_FMT_NVFP4, kL2First>(t, p, v[p]);
-        }
-    };
-    int j = s_item[0];
-    if (j >= items) return;
-    ItemRef item = decode(j);
-    TileRef cur = tile_ref<QZ_FMT_NVFP4, LAYOUT>(table, s_prefix, n, item.first_tile, w, lane);
-    uint32_t v[G::kPasses][G::kWords];
-    load_tile(cur, item.is_a, v);
-    for (int it = 0;; ++it) {
-        // publish the index fetched during the previous item, fetch another
-        if (threadIdx.x == 0) {
-            s_item[(it + 1) & 3] = (int)pending;
-            pending = atomicAdd(next_item, 1u);
-            unsigned ok = 1;
-            if (!item.is_a) {
-                // wait until every A tile of this item's chunk is done
-                const unsigned need = (unsigned)(s_cf[item.chunk + 1] - s_cf[item.chunk]);
-                const long long t0 = clock64();
-                while (ld_acquire_gpu(done + item.chunk) < need) {
-                    if (clock64() - t0 > (1LL << 31)) {
-                        if (d_err) atomicOr(d_err, QZ_DERR_TIMEOUT);
-                        ok = 0;
-                        break;
-                    }
+            for (int p = 0; p < G::kPasses; p += 2) {
+                const uint32_t sc = tile_scales_nv(v[p], v[p + 1], S);
+#pragma unroll
+                for (int q = 0; q < 2; ++q) {
+                    const uint32_t scq = (sc >> (8 * q)) & 0xFFu;
+                    tile_pass_nv<LAYOUT>(cur, p + q, lane, v[p + q], scq, nvfp4_rcp_warp(qm, scq), s_sf[wid]);
+                    if (more) tile_load<QZ_FMT_NVFP4, kL2First>(nxt, p + q, v[p + q]);
                 }
             }
-            s_ok[it & 1] = ok;
-        }
-        __syncthreads();
-        const int jn = s_item[(it + 1) & 3];
-        const bool more_items = jn < items;
-        const ItemRef nitem = more_items ? decode(jn) : item;
-        uint32_t run = 0;  // A: running max of this warp over the item's tiles of one expert
-        for (int k = 0; k < item.ntiles; ++k) {
-            const bool last = k + 1 == item.ntiles;
-            const bool more = !last || more_items;
-            const int ntile = last ? nitem.first_tile : item.first_tile + k + 1;
-            const bool next_a = last ? nitem.is_a : item.is_a;
-            const TileRef nxt = more ? tile_ref<QZ_FMT_NVFP4, LAYOUT>(table, s_prefix, n, ntile, w, lane) : cur;
-            if (item.is_a) {
-#pragma unroll
-                for (int p = 0; p < G::kPasses; ++p) run = max(run, absmax_words<G::kWords>(v[p]));
-                if (more) load_tile(nxt, next_a, v);
-                if (last || nxt.expert != cur.expert) {
-#pragma unroll
-                    for (int o = 16; o > 0; o >>= 1) run = max(run, __shfl_xor_sync(0xFFFFFFFFu, run, o));
-                    if (lane == 0) atomicMax(amax_ws + cur.expert, run << 16);
-                    run = 0;
-                }
-            } else {
-                // ordered after thread 0's acquire of the chunk count by the barrier above
-                const float A = __uint_as_float(ld_relaxed_gpu(amax_ws + cur.expert));
-                const float S = nvfp4_encode_scale(A);
-                const float qm = rcp_lane_quotient(S, s_inv, lane);
-#pragma unroll
-                for (int p = 0; p < G::kPasses; p += 2) {
-                    const uint32_t sc = tile_scales_nv(v[p], v[p + 1], S);
-#pragma unroll
-                    for (int q = 0; q < 2; ++q) {
-                        const uint32_t scq = (sc >> (8 * q)) & 0xFFu;
-                        tile_pass_nv<LAYOUT>(cur, p + q, lane, v[p + q], scq, nvfp4_rcp_warp(qm, scq), s_sf[w]);
-                        if (more) {
-                            if (next_a) tile_load<QZ_FMT_NVFP4, kL2Last>(nxt, p + q, v[p + q]);
-                            else tile_load<QZ_FMT_NVFP4, kL2First>(nxt, p + q, v[p + q]);
-                        }
-                    }
-                }
-                if (LAYOUT == QZ_SF_SWIZZLED_128x4) tile_flush_sf<QZ_FMT_NVFP4>(cur, w, lane, s_sf[w]);
-                if (threadIdx.x == 0) *const_cast<float*>(cur.amax) = A;
-            }
+            if (LAYOUT == QZ_SF_SWIZZLED_128x4) tile_flush_sf<QZ_FMT_NVFP4>(cur, w, lane, s_sf[wid]);
+            if (w == 0 && lane == 0) *const_cast<float*>(cur.amax) = A;
+            s_qtile[wid] = more ? t2 : total;
+            if (!more) return;
             cur = nxt;
+            t = t2;
         }
-        if (item.is_a) {
-            // every warp's atomic max precedes the barrier; thread 0's fence
-            // then releases them all before the count (the grid-barrier idiom)
-            __syncthreads();
-            if (threadIdx.x == 0) {
-                __threadfence();
-                atomicAdd(done + item.chunk, (unsigned)item.ntiles);
+    }
+
+    if (wid == kQWarps) {
+        // ---------------- producer: units b, b + grid, ... into the ring ----------------
+        int k = 0;  // units of this CTA issued so far
+        bool ok = true;
+        for (int u = b; u < units && ok; u += grid, ++k) {
+            const int stage = k % kStages;
+            const int use = k / kStages;
+            if (use > 0) {
+                uint64_t* eb = &s_empty[stage];
+                const unsigned par = (unsigned)((use - 1) & 1);
+                ok = bounded_wait([&] { return mbar_test(eb, par); }, abort_word, &s_abort, limit, d_err, lane, 0);
+                if (!ok) break;
+            }
+            const int e = find_owner(s_uprefix, n, u);
+            const int first_tile = s_prefix[e];
+            ok = bounded_wait(
+                [&] {
+                    int lo = total;
+#pragma unroll
+                    for (int q = 0; q < kQWarps; ++q) lo = min(lo, s_qtile[q]);
+                    return first_tile - lo <= kWindowTiles;
+                },
+                abort_word, &s_abort, limit, d_err, lane, 64);
+            if (!ok) break;
+            const qz_expert E = load_entry(table, e);
+            const UnitGeo g = unit_geo(E);
+            const int j = u - s_uprefix[e];
+            const int64_t r0 = (int64_t)(j / g.nseg) * g.krows;
+            const int64_t c0 = (int64_t)(j % g.nseg) * g.seg;
+            const int nr = (int)min((int64_t)g.krows, E.rows - r0);
+            const int nc = (int)min((int64_t)g.seg, E.cols - c0);
+            const unsigned bytes = (unsigned)(nr * nc * 2);
+            const uint16_t* src = static_cast<const uint16_t*>(E.x) + r0 * E.ld + c0;
+            unsigned char* dst = s_ring + stage * kUnitBytes;
+            if (lane == 0) {
+                s_unit_expert[stage] = e;
+                s_unit_bytes[stage] = bytes;
+                mbar_arrive_expect_tx(&s_full[stage], bytes);  // releases the two words above
+            }
+            __syncwarp();
+            if (g.nseg == 1 && E.ld == E.cols) {
+                if (lane == 0) bulk_copy_g2s(dst, src, bytes, &s_full[stage]);  // whole rows, contiguous
+            } else {
+                for (int r = lane; r < nr; r += 32)
+                    bulk_copy_g2s(dst + r * nc * 2, src + (int64_t)r * E.ld, (unsigned)(nc * 2), &s_full[stage]);
             }
         }
-        if (!more_items) break;
-        item = nitem;
+        if (!ok) {
+            // let the copies already issued land before the CTA can retire
+            for (int i = max(0, k - kStages); i < k; ++i) {
+                uint64_t* fb = &s_full[i % kStages];
+                const unsigned par = (unsigned)((i / kStages) & 1);
+                const long long t0 = global_ns();
+                while (!__all_sync(0xFFFFFFFFu, mbar_test(fb, par)) && global_ns() - t0 < limit) {
+                }
+            }
+        }
+        return;
+    }
+
+    // ---------------- consumers: consumer i takes stage i (units k = i, i + kStages, ...) ----------------
+    const int ci = wid - kQWarps - 1;
+    const bool withhold = (test_flags & QZ_TEST_WITHHOLD_ARRIVALS) != 0u;
+    const int mine = (units - b + grid - 1) / grid;  // units of this CTA
+    for (int k = ci; k < mine; k += kStages) {
+        uint64_t* fb = &s_full[ci];
+        const unsigned par = (unsigned)((k / kStages) & 1);
+        if (!bounded_wait([&] { return mbar_test(fb, par); }, abort_word, &s_abort, limit, d_err, lane, 0)) return;
+        const int e = s_unit_expert[ci];
+        const unsigned bytes = s_unit_bytes[ci];
+        const uint4* src = reinterpret_cast<const uint4*>(s_ring + ci * kUnitBytes);
+        uint32_t m0 = 0u, m1 = 0u;
+        const unsigned chunks = bytes >> 4;  // 16-byte chunks (bytes is a multiple of 32)
+        unsigned i = lane;
+        for (; i + 32 < chunks; i += 64) {
+            const uint4 a = src[i], c = src[i + 32];
+            m0 = max_abs_bf16x2(max_abs_bf16x2(m0, a.x), max_abs_bf16x2(a.y, max_abs_bf16x2(a.z, a.w)));
+            m1 = max_abs_bf16x2(max_abs_bf16x2(m1, c.x), max_abs_bf16x2(c.y, max_abs_bf16x2(c.z, c.w)));
+        }
+        if (i < chunks) {
+            const uint4 a = src[i];
+            m0 = max_abs_bf16x2(max_abs_bf16x2(m0, a.x), max_abs_bf16x2(a.y, max_abs_bf16x2(a.z, a.w)));
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s_empty[ci]);  // the stage may be refilled
+        uint32_t r = larger_half(max_abs_bf16x2(m0, m1));
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) r = max(r, __shfl_xor_sync(0xFFFFFFFFu, r, o));
+        if (lane == 0) {
+            // fold into this CTA's maximum of expert e; the consumer that folds
+            // the CTA's last unit of e publishes the maximum and the CTA's
+            // unit count (one global max and one add per CTA and expert)
+            atomicMax(s_emax + e, r << 16);
+            __threadfence_block();
+            const int u0 = s_uprefix[e] - b, u1 = s_uprefix[e + 1] - b;
+            const unsigned mine_e = (unsigned)(max(0, (u1 + grid - 1) / grid) - max(0, (u0 + grid - 1) / grid));
+            if (atomicAdd(s_ecnt + e, 1u) + 1u == mine_e) {
+                __threadfence_block();
+                const unsigned m = atomicMax(s_emax + e, 0u);  // every fold of this CTA is in
+                if (m != 0u) atomicMax(amax_ws + e, m);
+                __threadfence();  // the maximum is visible before the count that releases it
+                if (!withhold) atomicAdd(counted + e, mine_e);
+            }
+        }
     }
 }
 
@@ -591,46 +760,75 @@ __global__ void __launch_bounds__(kThreads) swizzle_kernel(const qz_sf_pair* __r
 // ---------------------------------------------------------------------------
 
 size_t prefix_smem(int n) { return (size_t)(n + 1) * sizeof(int); }
+size_t amax_smem(int n) { return (size_t)(2 * n + 1) * sizeof(int); }
 
-cudaError_t launch_mxfp8(const qz_expert* table, int n, int layout, int grid, cudaStream_t s, unsigned* d_err) {
+// A tile-kernel launch with programmatic stream serialization (see
+// pdl_allow_next); wait_prior = 0 only for calls declared independent.
+template <int FMT, int LAYOUT>
+cudaError_t launch_tiles(const qz_expert* table, int n, int grid, cudaStream_t s, unsigned* d_err, int wait_prior) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = prefix_smem(n);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, grouped_tile_kernel<FMT, LAYOUT>, table, n, d_err, wait_prior);
+}
+
+cudaError_t launch_mxfp8(const qz_expert* table, int n, int layout, int grid, cudaStream_t s, unsigned* d_err,
+                         bool independent) {
+    const int wait = independent ? 0 : 1;
     if (layout == QZ_SF_SWIZZLED_128x4)
-        grouped_tile_kernel<QZ_FMT_MXFP8, QZ_SF_SWIZZLED_128x4><<<grid, kThreads, prefix_smem(n), s>>>(table, n, d_err);
-    else
-        grouped_tile_kernel<QZ_FMT_MXFP8, QZ_SF_LINEAR><<<grid, kThreads, prefix_smem(n), s>>>(table, n, d_err);
-    return cudaGetLastError();
+        return launch_tiles<QZ_FMT_MXFP8, QZ_SF_SWIZZLED_128x4>(table, n, grid, s, d_err, wait);
+    return launch_tiles<QZ_FMT_MXFP8, QZ_SF_LINEAR>(table, n, grid, s, d_err, wait);
 }
 
 cudaError_t launch_nvfp4_tensor(const qz_expert* table, int n, int layout, bool compute_amax, int grid,
-                                cudaStream_t s, unsigned* d_err) {
+                                cudaStream_t s, unsigned* d_err, bool independent) {
     if (compute_amax) {
         amax_clear_kernel<<<(n + kThreads - 1) / kThreads, kThreads, 0, s>>>(table, n, layout);
         if (layout == QZ_SF_SWIZZLED_128x4)
-            amax_grouped_kernel<QZ_SF_SWIZZLED_128x4><<<grid, kThreads, prefix_smem(n), s>>>(table, n, d_err);
+            amax_grouped_kernel<QZ_SF_SWIZZLED_128x4><<<grid, kThreads, amax_smem(n), s>>>(table, n, d_err);
         else
-            amax_grouped_kernel<QZ_SF_LINEAR><<<grid, kThreads, prefix_smem(n), s>>>(table, n, d_err);
+            amax_grouped_kernel<QZ_SF_LINEAR><<<grid, kThreads, amax_smem(n), s>>>(table, n, d_err);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
     }
+    // the quantize pass of a computed-amax call depends on the amax pass before it
+    const int wait = (independent && !compute_amax) ? 0 : 1;
     if (layout == QZ_SF_SWIZZLED_128x4)
-        grouped_tile_kernel<QZ_FMT_NVFP4, QZ_SF_SWIZZLED_128x4><<<grid, kThreads, prefix_smem(n), s>>>(table, n, d_err);
-    else
-        grouped_tile_kernel<QZ_FMT_NVFP4, QZ_SF_LINEAR><<<grid, kThreads, prefix_smem(n), s>>>(table, n, d_err);
-    return cudaGetLastError();
+        return launch_tiles<QZ_FMT_NVFP4, QZ_SF_SWIZZLED_128x4>(table, n, grid, s, d_err, wait);
+    return launch_tiles<QZ_FMT_NVFP4, QZ_SF_LINEAR>(table, n, grid, s, d_err, wait);
 }
 
 size_t workspace_bytes(int n) { return workspace_words(n) * sizeof(unsigned); }
 
-size_t compute_l2_smem(int n) { return (size_t)(n + 1 + kMaxChunks + 1 + kMaxChunks + kLag + 1) * sizeof(int); }
+size_t compute_pipe_smem(int n) { return (size_t)kStages * kUnitBytes + (size_t)(4 * n + 2) * sizeof(int); }
 
-// One launch of the L2-chunked computed-amax path on a zeroed workspace.
+// One cooperative launch of the computed-amax pipeline on a zeroed workspace
+// (every CTA resident: a quantize warp waits on amax warps of every CTA).
 cudaError_t launch_nvfp4_compute_l2(const qz_expert* table, int n, int layout, int grid, unsigned* ws,
-                                    cudaStream_t s, unsigned* d_err) {
+                                    cudaStream_t s, unsigned* d_err, long long wait_ns, unsigned test_flags) {
     cudaError_t e = cudaMemsetAsync(ws, 0, workspace_bytes(n), s);
     if (e != cudaSuccess) return e;
-    const size_t smem = compute_l2_smem(n);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(kPipeThreads);
+    cfg.dynamicSmemBytes = compute_pipe_smem(n);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
     if (layout == QZ_SF_SWIZZLED_128x4)
-        nvfp4_compute_l2_kernel<QZ_SF_SWIZZLED_128x4><<<grid, kThreads, smem, s>>>(table, n, ws, d_err);
-    else
-        nvfp4_compute_l2_kernel<QZ_SF_LINEAR><<<grid, kThreads, smem, s>>>(table, n, ws, d_err);
-    return cudaGetLastError();
+        return cudaLaunchKernelEx(&cfg, nvfp4_compute_pipe_kernel<QZ_SF_SWIZZLED_128x4>, table, n, ws, d_err, wait_ns,
+                                  test_flags);
+    return cudaLaunchKernelEx(&cfg, nvfp4_compute_pipe_kernel<QZ_SF_LINEAR>, table, n, ws, d_err, wait_ns, test_flags);
 }
 
 cudaError_t launch_swizzle(const qz_sf_pair* table, int n, int grid, cudaStream_t s, unsigned* d_err) {
@@ -646,12 +844,15 @@ int grouped_blocks_per_sm(int which, int n) {
         case 0: cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, grouped_tile_kernel<QZ_FMT_MXFP8, QZ_SF_SWIZZLED_128x4>, kThreads, smem); break;
         case 1: cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, grouped_tile_kernel<QZ_FMT_NVFP4, QZ_SF_SWIZZLED_128x4>, kThreads, smem); break;
         case 2: cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, swizzle_kernel, kThreads, smem); break;
-        case 3: cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, amax_grouped_kernel<QZ_SF_SWIZZLED_128x4>, kThreads, smem); break;
+        case 3: cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, amax_grouped_kernel<QZ_SF_SWIZZLED_128x4>, kThreads, amax_smem(n)); break;
         default: {
-            const size_t big = compute_l2_smem(n);
-            cudaFuncSetAttribute(nvfp4_compute_l2_kernel<QZ_SF_SWIZZLED_128x4>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)big);
-            cudaFuncSetAttribute(nvfp4_compute_l2_kernel<QZ_SF_LINEAR>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)big);
-            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, nvfp4_compute_l2_kernel<QZ_SF_SWIZZLED_128x4>, kThreads, big);
+            const size_t big = compute_pipe_smem(n);
+            cudaFuncSetAttribute(nvfp4_compute_pipe_kernel<QZ_SF_SWIZZLED_128x4>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)big);
+            cudaFuncSetAttribute(nvfp4_compute_pipe_kernel<QZ_SF_LINEAR>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)big);
+            int b2 = 1;
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, nvfp4_compute_pipe_kernel<QZ_SF_SWIZZLED_128x4>, kPipeThreads, big);
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b2, nvfp4_compute_pipe_kernel<QZ_SF_LINEAR>, kPipeThreads, big);
+            b = min(b, b2);  // a cooperative grid must fit resident for both instantiations
             break;
         }
     }
@@ -693,11 +894,11 @@ cudaError_t static_workspace(unsigned** out) {
 }
 
 cudaError_t launch_nvfp4_compute_l2_static(const qz_expert* table, int n, int layout, int grid, cudaStream_t s,
-                                           unsigned* d_err) {
+                                           unsigned* d_err, long long wait_ns, unsigned test_flags) {
     unsigned* ws = nullptr;
     cudaError_t e = static_workspace(&ws);
     if (e != cudaSuccess) return e;
-    return launch_nvfp4_compute_l2(table, n, layout, grid, ws, s, d_err);
+    return launch_nvfp4_compute_l2(table, n, layout, grid, ws, s, d_err, wait_ns, test_flags);
 }
 
 }  // namespace qz

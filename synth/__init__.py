@@ -20,6 +20,9 @@ shapes and a plausible value distribution):
   each N(0, 1/n) [T, 7168] (a row-parallel projection's partial outputs)
 * Qwen3-235B-A22B prequant: 128 experts/layer, gate_up [3072, 4096] and down
   [4096, 1536], N(0, 0.02), 94 layers, seed 5 + layer
+
+``moe_layer`` draws one projection of one layer of either MoE workload from
+its seed (``layer_seed``), so a sweep can regenerate every layer in place.
 """
 from __future__ import annotations
 
@@ -62,6 +65,25 @@ def tiny_group(seed: int = TINY["seed"], experts: int = TINY["experts"], shape=T
 def expert_stack(n: int, shape, std: float, seed: int, device="cpu") -> torch.Tensor:
     """n same-shape expert matrices stacked as one [n, rows, cols] bf16 tensor."""
     return normal_bf16((n, *shape), std=std, seed=seed, device=device)
+
+
+def layer_seed(cfg: dict, layer: int, proj: str, rank: int = 0) -> int:
+    """Seed of one projection of one MoE layer: the workload's seed + layer
+    (+500 for the down projection, +1000 per rank of a multi-GPU run)."""
+    return int(cfg["seed"]) + int(layer) + 1000 * int(rank) + (0 if proj == "gate_up" else 500)
+
+
+def moe_layer(cfg: dict, layer: int, proj: str, device="cuda", rank: int = 0, out=None) -> torch.Tensor:
+    """The experts of one projection ("gate_up" or "down") of layer ``layer``
+    as one [experts, rows, cols] bf16 tensor, N(0, std^2), regenerated from
+    its seed alone.  Drawn in place (each value rounded once to bf16), so a
+    layer of the largest workload needs no temporary beyond its own 3.2 GB."""
+    shape = (cfg["experts"], *cfg[proj])
+    if out is None:
+        out = torch.empty(shape, dtype=torch.bfloat16, device=device)
+    assert tuple(out.shape) == shape and out.dtype == torch.bfloat16
+    out.normal_(0.0, float(cfg["std"]), generator=_gen(layer_seed(cfg, layer, proj, rank), out.device))
+    return out
 
 
 def split_activation(tokens=SPLIT_ACT["tokens"], hidden=SPLIT_ACT["hidden"], seed=SPLIT_ACT["seed"],

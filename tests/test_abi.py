@@ -74,6 +74,10 @@ def test_host_errors_without_gpu(lib):
     assert lib.qz_quantize_grouped_nvfp4(P(0x1000), 4, 1, 1, None, ctypes.byref(small)) == qz.QZ_ERR_INVALID_ARG
     odd = qz.binding._Opts(None, 0, P(0x10002), ctypes.c_size_t(qz.workspace_bytes(4)))
     assert lib.qz_quantize_grouped_nvfp4(P(0x1000), 4, 1, 1, None, ctypes.byref(odd)) == qz.QZ_ERR_ALIGNMENT
+    neg = qz.binding._Opts(None, 0, P(0x10000), ctypes.c_size_t(qz.workspace_bytes(4)), 0, -1, 0)
+    assert lib.qz_quantize_grouped_nvfp4(P(0x1000), 4, 1, 1, None, ctypes.byref(neg)) == qz.QZ_ERR_INVALID_ARG
+    assert lib.qz_quantize_grouped_nvfp4_compute_noalloc(P(0x1000), 4, 1, None, ctypes.byref(neg)) == \
+        qz.QZ_ERR_INVALID_ARG
     assert qz.workspace_bytes(0) == 0 and qz.workspace_bytes(qz.MAX_EXPERTS + 1) == 0
     assert qz.workspace_bytes(128) >= 4 * (128 + 1)
     assert lib.qz_swizzle_scales(None, 0, None, None) == qz.QZ_OK
@@ -205,7 +209,7 @@ def test_element_hint_reaches_the_launch_options():
     assert qz.binding._opts(None, 0) is None
     raw = qz.ExpertTable.from_raw([(0, 0, 64, 64, 0, 0, 0)], torch.device("cpu"))
     assert raw.elems == 0
-    assert ctypes.sizeof(qz.binding._Opts) == 40
+    assert ctypes.sizeof(qz.binding._Opts) == 56
 
 
 

@@ -248,3 +248,70 @@ def _blocks_with_every_amax(block: int) -> torch.Tensor:
 def test_every_bf16_value_as_block_amax(layout):
     x = _blocks_with_every_amax(32).cuda()
     check_against_oracle([x], layout, run_mxfp8([x], layout))
+
+
+def test_back_to_back_calls_on_one_stream():
+    """Programmatic dependent launch between the tile kernels of consecutive
+    calls: a call that is not declared independent still sees stream order
+    (two calls writing the same outputs leave the second call's bytes; a
+    call after a torch kernel that writes its input sees the new input);
+    calls declared independent on disjoint experts give every call's bytes;
+    both also inside a captured CUDA graph."""
+    shape = (384, 1024)
+    a = synth.normal_bf16(shape, seed=1).cuda()
+    b = synth.blockwise_scaled(shape, 32, seed=2, lo=-20, hi=20).cuda()
+    (q, sf, _), = guarded_entries([a], qz.FMT_MXFP8, qz.SF_SWIZZLED)[1]
+    ta = qz.ExpertTable([qz.Entry(a, q.view.view(shape), sf.view)])
+    tb = qz.ExpertTable([qz.Entry(b, q.view.view(shape), sf.view)])
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        for _ in range(20):                        # write-after-write on the same outputs, in stream order
+            qz.quantize_grouped_mxfp8(ta, qz.SF_SWIZZLED, stream=s)
+            qz.quantize_grouped_mxfp8(tb, qz.SF_SWIZZLED, stream=s)
+    torch.cuda.synchronize()
+    check_against_oracle([b], qz.SF_SWIZZLED, [(q.host().reshape(shape), sf.host())])
+    c = torch.zeros(shape, dtype=torch.bfloat16, device="cuda")
+    tc = qz.ExpertTable([qz.Entry(c, q.view.view(shape), sf.view)])
+    with torch.cuda.stream(s):
+        qz.quantize_grouped_mxfp8(ta, qz.SF_SWIZZLED, stream=s)
+        c.copy_(b).mul_(3.0)                       # a torch kernel writes the next call's input
+        qz.quantize_grouped_mxfp8(tc, qz.SF_SWIZZLED, stream=s)
+    torch.cuda.synchronize()
+    check_against_oracle([c], qz.SF_SWIZZLED, [(q.host().reshape(shape), sf.host())])
+    # independent calls on disjoint experts, MXFP8 and NVFP4 given, and as a graph
+    xs = [synth.blockwise_scaled((200 + 17 * i, 512), 32, seed=30 + i, lo=-8, hi=8).cuda() for i in range(12)]
+    mx, mkeep = guarded_entries(xs, qz.FMT_MXFP8, qz.SF_SWIZZLED)
+    amax_in = [float(x.float().abs().max()) for x in xs]
+    nv, nkeep = guarded_entries(xs, qz.FMT_NVFP4, qz.SF_LINEAR, qz.NVFP4_PER_TENSOR_GIVEN, amax_in)
+    mtabs = [qz.ExpertTable([e]) for e in mx]
+    ntabs = [qz.ExpertTable([e]) for e in nv]
+
+    def burst():
+        for mt, nt in zip(mtabs, ntabs):
+            qz.quantize_grouped_mxfp8(mt, qz.SF_SWIZZLED, stream=s, independent=True)
+            qz.quantize_grouped_nvfp4(nt, qz.NVFP4_PER_TENSOR_GIVEN, qz.SF_LINEAR, stream=s, independent=True)
+
+    def verify():
+        got = [(qq.host().reshape(x.shape[0], -1), ss.host()) for (qq, ss, _), x in zip(mkeep, xs)]
+        check_against_oracle(xs, qz.SF_SWIZZLED, got)
+        ref = oracle.quantize_grouped([host_bits(x) for x in xs], oracle.NVFP4, oracle.LINEAR,
+                                      oracle.NVFP4_PER_TENSOR_GIVEN, amax_in, threads=oracle_threads())
+        for (qq, ss, aa), x, (rq, rs, _) in zip(nkeep, xs, ref):
+            assert qq.guards_intact() and ss.guards_intact()
+            assert_bytes_equal(qq.host(), rq.reshape(-1), "NVFP4 payload")
+            assert_bytes_equal(ss.host(), rs, "NVFP4 scales")
+
+    with torch.cuda.stream(s):
+        burst()
+    torch.cuda.synchronize()
+    verify()
+    for qq, ss, _ in mkeep + nkeep:
+        qq.view.fill_(0xA5)
+        ss.view.fill_(0xA5)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g, stream=s):
+            burst()
+    g.replay()
+    torch.cuda.synchronize()
+    verify()

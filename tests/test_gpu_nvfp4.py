@@ -295,6 +295,50 @@ def test_compute_l2_workspace_too_small_is_rejected():
     assert torch.all(keep[0][0].raw == 0xA5)
 
 
+@pytest.mark.parametrize("layout", LAYOUTS)
+def test_compute_l2_wait_runs_out(layout):
+    """The failure path of the single-launch pipeline, with no GPU fault: the
+    amax warps withhold the counts that release the quantize warps, so every
+    wait runs out after the 0.2 ms limit.  The launch must end on its own
+    with QZ_DERR_TIMEOUT in the error word and no output byte written; the
+    context stays usable and the next call on the same buffers is exact."""
+    xs = [synth.normal_bf16((300, 1024), std=0.02, seed=700 + i).cuda() for i in range(24)]
+    entries, keep = guarded_entries(xs, qz.FMT_NVFP4, layout, qz.NVFP4_PER_TENSOR_COMPUTE)
+    for (_, _, a) in keep:
+        a.view.fill_(0xA5)
+    table = qz.ExpertTable(entries)
+    ws = qz.alloc_workspace(len(xs))
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record()
+    qz.quantize_grouped_nvfp4(table, qz.NVFP4_PER_TENSOR_COMPUTE, layout, err=err, workspace=ws,
+                              wait_limit_ns=200_000, test_flags=qz.TEST_WITHHOLD_ARRIVALS)
+    ev1.record()
+    torch.cuda.synchronize()
+    assert int(err.item()) & qz.DERR_TIMEOUT
+    assert ev0.elapsed_time(ev1) < 1000.0, "the launch must end soon after its waits run out"
+    for q, sf, a in keep:
+        assert torch.all(q.raw == 0xA5) and torch.all(sf.raw == 0xA5) and torch.all(a.raw == 0xA5)
+    # the same buffers, a normal call: exact against the oracle
+    err.zero_()
+    qz.quantize_grouped_nvfp4(table, qz.NVFP4_PER_TENSOR_COMPUTE, layout, err=err, workspace=ws)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    got = [(q.host().reshape(x.shape[0], -1), sf.host(), a.view.view(torch.float32).cpu().numpy())
+           for (q, sf, a), x in zip(keep, xs)]
+    check(xs, layout, qz.NVFP4_PER_TENSOR_COMPUTE, got)
+
+
+def test_compute_l2_large_experts_one_per_chunk():
+    """Experts larger than a chunk's minimum (each its own chunk) next to
+    small ones that share a chunk, and a call smaller than one chunk."""
+    shapes = [(3072, 512), (16, 64), (5, 4096), (1100, 1024), (1, 16), (2048, 2048)]
+    xs = [synth.blockwise_scaled(s, 16, seed=800 + i, lo=-6, hi=6).cuda() for i, s in enumerate(shapes)]
+    for layout in LAYOUTS:
+        check(xs, layout, qz.NVFP4_PER_TENSOR_COMPUTE, run_compute_l2(xs, layout))
+        check(xs[1:3], layout, qz.NVFP4_PER_TENSOR_COMPUTE, run_compute_l2(xs[1:3], layout))
+
+
 def _order_cases():
     from golden_io import rows
     return rows("nvfp4_rounding_order.txt")
