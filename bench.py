@@ -1187,7 +1187,7 @@ def main():
     ap.add_argument("--layers", type=int, default=None,
                     help="layers per step (default: 94 for the Qwen3-235B-A22B sweep, 48 for the 30B refit)")
     ap.add_argument("--streams", type=int, default=2, help="streams the independent 30B refit calls are spread over")
-    ap.add_argument("--compute-path", choices=["single", "three"], default="three",
+    ap.add_argument("--compute-path", choices=["single", "three"], default="single",
                     help="NVFP4 computed amax: one cooperative launch with a workspace, or clear + amax + quantize")
     ap.add_argument("--no-extra", action="store_true", help="skip the other workloads")
     ap.add_argument("--no-e2e", action="store_true")

@@ -393,7 +393,7 @@ __global__ void __launch_bounds__(kThreads, 3) amax_grouped_kernel(const qz_expe
 //   ws[8 + kMaxChunks + e] expert e's amax (bf16 magnitude bits << 16).
 // ---------------------------------------------------------------------------
 
-constexpr int kQGroups = 1;            // quantize groups: each walks its own tiles
+constexpr int kQGroups = 2;            // quantize groups: each walks its own tiles
 constexpr int kQWarps = 8 * kQGroups;  // quantize warps: 8 per group (the 8 row groups of a tile)
 constexpr int kStages = 4;             // shared-memory stages of the amax ring (one consumer warp each)
 constexpr int kUnitBytes = 32768;      // bytes of one amax unit (one stage)
