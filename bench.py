@@ -1061,6 +1061,67 @@ def _extra_allreduce(qz, device, out, peak, tokens=None, ranks=8):
 # CPU oracle timing (the reference arm and the cpu_baseline key)
 # ---------------------------------------------------------------------------
 
+def allreduce_nvlink(qz, device, rank, world, tokens=(16, 512, 4096)):
+    """The AllReduce epilogue across the ranks' GPUs (only under torchrun,
+    N > 1): every rank's buffer is mapped into every process through CUDA IPC
+    (PeerBuffers), the rank inputs are read and the destinations written with
+    plain peer loads and stores over NVLink (no multicast), and each call sits
+    between two stream-ordered NCCL barriers.  CUDA events bracket the kernel
+    alone on each rank; the time is the max over ranks.  The NVLink bound of a
+    call is the bytes that must cross it (one-shot: (n - 1) T H 2 reads per
+    rank; slice form: (n - 1)/n of them plus (n - 1)/n of the outputs written
+    to peers) over the measured 770 GB/s peer copy per direction."""
+    from nvfp4_quantization_moe_b200 import allreduce as ar
+    H = synth.FUSED_NORM["hidden"]
+    fmt, layout = qz.FMT_MXFP8, qz.SF_SWIZZLED
+    Tmax = max(tokens)
+    L = ar.SymmetricLayout(Tmax, H, fmt, layout)
+    buf = torch.zeros(L.total, dtype=torch.uint8, device=device)
+    xs, r, g = synth.rank_partials(world, Tmax, device=device)
+    buf[L.x:L.x + Tmax * H * 2].view(torch.bfloat16).view(Tmax, H).copy_(xs[rank])
+    one = torch.ones(1, dtype=torch.int32, device=device)
+
+    def barrier():
+        torch.distributed.all_reduce(one, op=torch.distributed.ReduceOp.MAX)  # every rank's prior stream work is done
+
+    timed = []
+
+    def launch(*a, **kw):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        qz.allreduce_rmsnorm_quantize(*a, **kw)
+        e1.record()
+        timed.append((e0, e1))
+
+    out = {"ranks": world, "H": H, "format": "MXFP8 swizzled, residual_out written", "sweep": []}
+    with ar.PeerBuffers(buf.data_ptr()) as pb:
+        for slice_form in (False, True):
+            ep = ar.AllReduceEpilogue(rank, world, pb.bases, L, barrier, slice_form=slice_form, launch=launch)
+            for T in tokens:
+                for _ in range(3):
+                    ep(T, r[:T], g, 1e-6)
+                torch.cuda.synchronize()
+                timed.clear()
+                for _ in range(10):
+                    ep(T, r[:T], g, 1e-6)
+                torch.cuda.synchronize()
+                us = 1e3 * statistics.median(a.elapsed_time(b) for a, b in timed)
+                us = max_over_ranks([us], device)[0]
+                rows = T if not slice_form else ar.rank_rows(T, world, rank)[1] - ar.rank_rows(T, world, rank)[0]
+                bf = T * H * 2
+                remote_in = (world - 1) * bf if not slice_form else (world - 1) * rows * H * 2
+                outs = rows * H * (2 + 2 + 1) + qz.sf_bytes(rows, H, fmt, layout)
+                remote_out = 0 if not slice_form else (world - 1) * outs
+                nvl = remote_in + remote_out
+                out["sweep"].append({"form": "slice" if slice_form else "one-shot", "T": T, "us": round(us, 2),
+                                     "nvlink_bytes": int(nvl), "nvlink_GB/s": round(nvl / (us / 1e3) / GB, 1),
+                                     "frac_of_770": round(nvl / (us / 1e3) / GB / 770.0, 4)})
+        torch.cuda.synchronize()
+        torch.distributed.barrier()
+    del buf
+    return out
+
+
 def oracle_prequant_sample(threads: int, target_s: float = 10.0, min_pairs: int = 1, pairs: int = 0):
     """Time the CPU oracle on a bounded sample of the headline workload: whole
     Qwen3-235B-A22B experts (one gate_up [3072, 4096] and one down
@@ -1193,6 +1254,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     ap.add_argument("--no-refit", action="store_true", help="skip the Qwen3-30B-A3B refit step")
+    ap.add_argument("--no-allreduce", action="store_true",
+                    help="with N > 1: skip the AllReduce epilogue across the ranks' GPUs")
     ap.add_argument("--config", type=int, choices=[1, 2, 3, 4, 5], default=None,
                     help="one of the five workloads: 1 tiny MXFP8 group (latency), 2 the Qwen3-30B-A3B refit step, "
                          "3 the row-scaled NVFP4 split activation, 4 the fused residual + RMSNorm sweep, 5 the "
@@ -1292,6 +1355,11 @@ def main():
     del work
     torch.cuda.empty_cache()
 
+    if dist_ok and not args.no_allreduce:
+        try:
+            line["allreduce_nvlink"] = allreduce_nvlink(qz, device, rank, world)
+        except Exception as exc:  # reported, never allowed to void the measured line
+            line["allreduce_nvlink"] = {"error": f"{type(exc).__name__}: {exc}"[:300]}
     if rank == 0 and not args.no_e2e:
         line["e2e"] = e2e_prequant(qz, device, steps=2, warmup=1, compute_workspace=args.compute_path == "single")
     if rank == 0 and not args.no_extra and args.config is None:

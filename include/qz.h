@@ -351,6 +351,37 @@ qz_status qz_allreduce_rmsnorm_quantize(const void *const *rank_x, int n_ranks, 
                                         const qz_norm_dest *dests, int n_dests, int fmt, int layout,
                                         const float *d_global_amax, void *stream);
 
+/* Peer mappings for the AllReduce epilogue on a node: every rank exports a
+ * CUDA IPC handle of its own buffer, the handles are exchanged over the
+ * process group, and every rank imports its peers' buffers, so that one
+ * process holds device pointers to all ranks' inputs and destinations
+ * ([LSF] commits 1-2: the epilogue reads every rank's partial and writes the
+ * result to every rank).  Host-side calls; no stream work, no allocation. */
+typedef struct qz_ipc_handle {
+    unsigned char handle[64]; /* cudaIpcMemHandle_t of the device allocation holding the pointer */
+    uint64_t offset;          /* pointer - start of that allocation */
+    uint64_t alloc_bytes;     /* bytes of that allocation */
+    int device;               /* the exporting process's device ordinal */
+    int reserved;
+} qz_ipc_handle;
+
+/* Fill *out for the device pointer d_ptr of the calling process (an address
+ * inside a cudaMalloc allocation, on the current device).
+ * Errors: QZ_ERR_INVALID_ARG for NULL arguments; QZ_ERR_CUDA when the runtime
+ * or driver refuses (no device, not a device allocation, IPC unsupported). */
+qz_status qz_ipc_export(const void *d_ptr, qz_ipc_handle *out);
+
+/* Map a peer process's exported allocation into this process (current device;
+ * peer access is enabled as needed) and return the peer's pointer in
+ * *d_ptr_out (mapping base + offset).  A handle exported by the calling process
+ * itself cannot be imported (CUDA IPC): use the pointer directly.
+ * Errors: QZ_ERR_INVALID_ARG for NULL arguments; QZ_ERR_CUDA from the runtime. */
+qz_status qz_ipc_import(const qz_ipc_handle *h, void **d_ptr_out);
+
+/* Unmap a pointer returned by qz_ipc_import for the same handle.
+ * Errors: QZ_ERR_INVALID_ARG for NULL arguments; QZ_ERR_CUDA from the runtime. */
+qz_status qz_ipc_close(void *d_ptr, const qz_ipc_handle *h);
+
 /* Linear -> swizzled 128x4 conversion of n SF matrices in one launch, padding
  * written as 0x00 ([MX] Summary; [CAR] commit 5: swizzled and linear agree).
  * Errors: QZ_ERR_INVALID_ARG for n < 0, n > QZ_MAX_EXPERTS or a NULL table

@@ -12,9 +12,9 @@ from .binding import (  # noqa: F401
     FMT_FP8_BLOCK128, FMT_MXFP8, FMT_NVFP4, LIB_PATH, MAX_EXPERTS, MAX_HIDDEN, MAX_RANKS, NVFP4_PER_ROW,
     NVFP4_PER_TENSOR_COMPUTE, NVFP4_PER_TENSOR_GIVEN, QZ_ERR_ALIGNMENT, QZ_ERR_CUDA, QZ_ERR_INVALID_ARG,
     QZ_ERR_UNSUPPORTED, QZ_OK, SF_LINEAR, SF_SWIZZLED, STATIC_WS_MAX_EXPERTS, DqEntry, DqTable, Entry, ExpertTable,
-    NormDest, QzError, SfPairTable, SplitEntry, SplitTable, alloc_outputs, alloc_workspace,
+    IpcHandle, NormDest, QzError, SfPairTable, SplitEntry, SplitTable, alloc_outputs, alloc_workspace,
     allreduce_rmsnorm_quantize, attention_merge_quantize,
-    dequantize_grouped, load, quantize_experts, quantize_grouped_colwise, quantize_grouped_mxfp8,
+    dequantize_grouped, ipc_close, ipc_export, ipc_import, load, quantize_experts, quantize_grouped_colwise, quantize_grouped_mxfp8,
     quantize_grouped_nvfp4, quantize_grouped_nvfp4_compute_noalloc, rmsnorm_quantize, sf_bytes,
     split_fused_experts, status_string, swizzle_scales, workspace_bytes,
 )

@@ -15,10 +15,13 @@ another GPU.  This module owns what surrounds it:
   order, and a second barrier (no rank overwrites its input, or reads a
   destination that peers write, before all have finished).
 
-The addresses come from whatever maps the ranks' allocations into each
-process (CUDA IPC handles, or a symmetric-memory allocator's per-rank buffer
-pointers), and the barrier can be an NCCL all-reduce of one integer on the
-launching stream, whose waits the process group's timeout bounds on the host.
+The addresses come from ``PeerBuffers``: every rank exports a CUDA IPC handle
+of its own allocation (``qz_ipc_export``), the handles are all-gathered over
+the process group, and every rank maps its peers' allocations
+(``qz_ipc_import``); a symmetric-memory allocator's per-rank pointers serve as
+well.  The barrier can be an NCCL all-reduce of one integer on the launching
+stream, or a synchronize plus a process-group barrier; either way the process
+group's timeout bounds its waits on the host.
 
 The one-shot form computes all T rows on every rank into its own buffers;
 the slice form computes ``rank_rows(T, world, rank)`` and writes them to every
@@ -27,6 +30,8 @@ rank's buffers (reduce-scatter and all-gather in one kernel).
 from __future__ import annotations
 
 from typing import Callable, List, Optional, Sequence, Tuple
+
+import torch.distributed as dist
 
 from . import binding
 
@@ -111,3 +116,47 @@ class AllReduceEpilogue:
         self.launch(xs, residual, gamma, eps, dests, L.fmt, L.sf_layout, T, L.H, rows=rows,
                     global_amax=global_amax, stream=stream)
         self.barrier()
+
+
+class PeerBuffers:
+    """Every rank's allocation as mapped in this process, in rank order.
+
+    Each rank exports an IPC handle of ``local_ptr`` (its own buffer), the
+    handles are all-gathered over ``group`` (any backend), and every peer's
+    allocation is mapped; this rank's own pointer is used as is (CUDA IPC
+    does not map a handle into the process that exported it).  ``bases`` is
+    the list the epilogue takes; ``close()`` unmaps the peers (call it after
+    the last launch that reads or writes them has finished)."""
+
+    def __init__(self, local_ptr: int, group=None, export: Callable = binding.ipc_export,
+                 import_: Callable = binding.ipc_import, close: Callable = binding.ipc_close):
+        self.rank = dist.get_rank(group)
+        self.world = dist.get_world_size(group)
+        mine = export(int(local_ptr))
+        self.handles: List[bytes] = [b""] * self.world
+        dist.all_gather_object(self.handles, mine, group=group)
+        self._close = close
+        self.bases: List[int] = []
+        self._opened: List[Tuple[int, bytes]] = []
+        try:
+            for r, h in enumerate(self.handles):
+                if r == self.rank:
+                    self.bases.append(int(local_ptr))
+                else:
+                    p = import_(h)
+                    self._opened.append((p, h))
+                    self.bases.append(p)
+        except Exception:
+            self.close()
+            raise
+
+    def close(self):
+        while self._opened:
+            p, h = self._opened.pop()
+            self._close(p, h)
+
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *exc):
+        self.close()

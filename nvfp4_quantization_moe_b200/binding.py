@@ -49,6 +49,9 @@ EXPORTED = (
     "qz_quantize_grouped_colwise",
     "qz_split_fused_experts",
     "qz_allreduce_rmsnorm_quantize",
+    "qz_ipc_export",
+    "qz_ipc_import",
+    "qz_ipc_close",
 )
 STATIC_WS_MAX_EXPERTS = 1024
 
@@ -82,6 +85,13 @@ class _FusedSplit(ctypes.Structure):
                 ("q_out", ctypes.c_void_p * 2), ("sf_out", ctypes.c_void_p * 2), ("amax_out", ctypes.c_void_p * 2)]
 
 
+class IpcHandle(ctypes.Structure):
+    """struct qz_ipc_handle: a CUDA IPC handle of an allocation and the offset
+    of the exported pointer in it."""
+    _fields_ = [("handle", ctypes.c_ubyte * 64), ("offset", ctypes.c_uint64), ("alloc_bytes", ctypes.c_uint64),
+                ("device", ctypes.c_int), ("reserved", ctypes.c_int)]
+
+
 class _Opts(ctypes.Structure):
     _fields_ = [("d_err", ctypes.c_void_p), ("max_ctas", ctypes.c_int), ("d_workspace", ctypes.c_void_p),
                 ("workspace_bytes", ctypes.c_size_t), ("elems_hint", ctypes.c_int64),
@@ -89,7 +99,7 @@ class _Opts(ctypes.Structure):
 
 
 assert ctypes.sizeof(_Expert) == 56 and ctypes.sizeof(_SfPair) == 32 and ctypes.sizeof(_DqExpert) == 56
-assert ctypes.sizeof(_FusedSplit) == 96
+assert ctypes.sizeof(_FusedSplit) == 96 and ctypes.sizeof(IpcHandle) == 88
 
 _lock = threading.Lock()
 _lib = None
@@ -132,6 +142,12 @@ def load(path: str = LIB_PATH):
         lib.qz_attention_merge_quantize.argtypes = [P, P, I, i64, i64, P, P, P, I, P]
         lib.qz_split_fused_experts.restype = I
         lib.qz_split_fused_experts.argtypes = [P, I, I, I, I, I, P, P]
+        lib.qz_ipc_export.restype = I
+        lib.qz_ipc_export.argtypes = [P, P]
+        lib.qz_ipc_import.restype = I
+        lib.qz_ipc_import.argtypes = [P, P]
+        lib.qz_ipc_close.restype = I
+        lib.qz_ipc_close.argtypes = [P, P]
         lib.qz_allreduce_rmsnorm_quantize.restype = I
         lib.qz_allreduce_rmsnorm_quantize.argtypes = [P, I, P, P, ctypes.c_float, i64, i64, i64, i64, P, I, I, I,
                                                       P, P]
@@ -428,6 +444,28 @@ def allreduce_rmsnorm_quantize(rank_x, residual, gamma, eps: float, dests, fmt: 
         ctypes.cast(ds, ctypes.c_void_p), len(dests), int(fmt), int(layout), ctypes.c_void_p(_addr(global_amax)),
         _stream_ptr(stream)),
         "qz_allreduce_rmsnorm_quantize")
+
+
+def ipc_export(ptr: int) -> bytes:
+    """qz_ipc_export: the IPC handle (88 bytes) of the device allocation holding ``ptr``."""
+    h = IpcHandle()
+    _check(load().qz_ipc_export(ctypes.c_void_p(int(ptr)), ctypes.byref(h)), "qz_ipc_export")
+    return bytes(h)
+
+
+def ipc_import(handle: bytes) -> int:
+    """qz_ipc_import: map a peer process's exported allocation; returns the
+    peer's pointer as an address in this process."""
+    h = IpcHandle.from_buffer_copy(handle)
+    out = ctypes.c_void_p()
+    _check(load().qz_ipc_import(ctypes.byref(h), ctypes.byref(out)), "qz_ipc_import")
+    return int(out.value)
+
+
+def ipc_close(ptr: int, handle: bytes) -> None:
+    """qz_ipc_close: unmap a pointer returned by ipc_import for ``handle``."""
+    h = IpcHandle.from_buffer_copy(handle)
+    _check(load().qz_ipc_close(ctypes.c_void_p(int(ptr)), ctypes.byref(h)), "qz_ipc_close")
 
 
 def dequantize_grouped(table: DqTable, fmt: int, per_row: bool, layout: int, stream=None, err=None,

@@ -6,6 +6,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <cstring>
 #include <mutex>
 
 #include "../../include/qz.h"
@@ -323,6 +324,48 @@ qz_status qz_split_fused_experts(const qz_fused_split* d_table, int n, int fmt, 
     if (n == 0) return QZ_OK;
     return from_cuda(qz::launch_split_fused(d_table, n, fmt, amax_kind, src_layout, dst_layout, wave_grid(8, opts),
                                             (cudaStream_t)stream, err_word(opts)));
+}
+
+qz_status qz_ipc_export(const void* d_ptr, qz_ipc_handle* out) {
+    if (!d_ptr || !out) return QZ_ERR_INVALID_ARG;
+    static_assert(sizeof(cudaIpcMemHandle_t) == sizeof(out->handle), "IPC handle size");
+    // the allocation's start and size: the driver's address-range query,
+    // reached through the runtime so the library needs no link to the driver
+    typedef int (*AddressRange)(unsigned long long*, size_t*, unsigned long long);
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult found;
+    if (cudaGetDriverEntryPointByVersion("cuMemGetAddressRange", &fn, 12000, cudaEnableDefault, &found) !=
+            cudaSuccess ||
+        found != cudaDriverEntryPointSuccess || !fn)
+        return QZ_ERR_CUDA;
+    unsigned long long base = 0;
+    size_t size = 0;
+    if (reinterpret_cast<AddressRange>(fn)(&base, &size, (unsigned long long)(uintptr_t)d_ptr) != 0) return QZ_ERR_CUDA;
+    cudaIpcMemHandle_t h;
+    if (cudaIpcGetMemHandle(&h, reinterpret_cast<void*>(base)) != cudaSuccess) return QZ_ERR_CUDA;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return QZ_ERR_CUDA;
+    memcpy(out->handle, &h, sizeof(h));
+    out->offset = (uint64_t)((uintptr_t)d_ptr - base);
+    out->alloc_bytes = (uint64_t)size;
+    out->device = dev;
+    out->reserved = 0;
+    return QZ_OK;
+}
+
+qz_status qz_ipc_import(const qz_ipc_handle* h, void** d_ptr_out) {
+    if (!h || !d_ptr_out) return QZ_ERR_INVALID_ARG;
+    cudaIpcMemHandle_t ipc;
+    memcpy(&ipc, h->handle, sizeof(ipc));
+    void* base = nullptr;
+    if (cudaIpcOpenMemHandle(&base, ipc, cudaIpcMemLazyEnablePeerAccess) != cudaSuccess) return QZ_ERR_CUDA;
+    *d_ptr_out = static_cast<char*>(base) + h->offset;
+    return QZ_OK;
+}
+
+qz_status qz_ipc_close(void* d_ptr, const qz_ipc_handle* h) {
+    if (!d_ptr || !h) return QZ_ERR_INVALID_ARG;
+    return from_cuda(cudaIpcCloseMemHandle(static_cast<char*>(d_ptr) - h->offset));
 }
 
 size_t qz_workspace_bytes(int n_experts) {

@@ -78,6 +78,16 @@ def test_host_errors_without_gpu(lib):
     assert lib.qz_quantize_grouped_nvfp4(P(0x1000), 4, 1, 1, None, ctypes.byref(neg)) == qz.QZ_ERR_INVALID_ARG
     assert lib.qz_quantize_grouped_nvfp4_compute_noalloc(P(0x1000), 4, 1, None, ctypes.byref(neg)) == \
         qz.QZ_ERR_INVALID_ARG
+    h = qz.IpcHandle()
+    out = ctypes.c_void_p()
+    assert lib.qz_ipc_export(None, ctypes.byref(h)) == qz.QZ_ERR_INVALID_ARG
+    assert lib.qz_ipc_export(P(0x1000), None) == qz.QZ_ERR_INVALID_ARG
+    assert lib.qz_ipc_import(None, ctypes.byref(out)) == qz.QZ_ERR_INVALID_ARG
+    assert lib.qz_ipc_import(ctypes.byref(h), None) == qz.QZ_ERR_INVALID_ARG
+    assert lib.qz_ipc_close(None, ctypes.byref(h)) == qz.QZ_ERR_INVALID_ARG
+    if not torch.cuda.is_available():
+        # no device: the runtime refuses, the call reports it
+        assert lib.qz_ipc_export(P(0x1000), ctypes.byref(h)) == qz.QZ_ERR_CUDA
     assert qz.workspace_bytes(0) == 0 and qz.workspace_bytes(qz.MAX_EXPERTS + 1) == 0
     assert qz.workspace_bytes(128) >= 4 * (128 + 1)
     assert lib.qz_swizzle_scales(None, 0, None, None) == qz.QZ_OK
@@ -218,7 +228,8 @@ def test_binding_structs_match_the_header(tmp_path):
     field offsets (a probe compiled by gcc against include/qz.h prints them)."""
     b = qz.binding
     mirrors = {"qz_expert": b._Expert, "qz_dq_expert": b._DqExpert, "qz_sf_pair": b._SfPair,
-               "qz_fused_split": b._FusedSplit, "qz_launch_opts": b._Opts, "qz_norm_dest": b.NormDest}
+               "qz_fused_split": b._FusedSplit, "qz_launch_opts": b._Opts, "qz_norm_dest": b.NormDest,
+               "qz_ipc_handle": b.IpcHandle}
     lines = ["#include <stdio.h>", "#include <stddef.h>", '#include "qz.h"', "int main(void) {"]
     for cname, cls in mirrors.items():
         lines.append(f'  printf("{cname} size %zu\\n", sizeof({cname}));')

@@ -100,3 +100,50 @@ def test_two_gloo_ranks_call_sequence():
         # one-shot form: the same inputs, all rows, this rank's own buffers only
         assert one[1] == xs and one[2] == (0, 300) and one[3] == [dests[rank]]
     assert rows_seen == [(0, 150), (150, 300)]
+
+
+def _ipc_worker(rank, world, port, out):
+    import sys
+    sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    from nvfp4_quantization_moe_b200 import allreduce as ar_
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        local = (rank + 1) << 40
+        opened, closed = [], []
+
+        def export(ptr):                      # a handle that names its exporter
+            return f"h:{ptr}".encode()
+
+        def import_(h):
+            ptr = int(h.decode().split(":")[1])
+            opened.append(ptr)
+            return ptr + 0x10                 # the peer's pointer as mapped here
+
+        def close(p, h):
+            closed.append((p, h))
+
+        with ar_.PeerBuffers(local, export=export, import_=import_, close=close) as pb:
+            bases = list(pb.bases)
+        out[rank] = (bases, opened, closed)
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.timeout(120)
+def test_peer_buffers_exchange_over_gloo():
+    """Three gloo ranks: every rank's handle reaches every rank, peers are
+    mapped in rank order, a rank's own pointer is not mapped, and every
+    mapping is closed again."""
+    world = 3
+    port = _free_port()
+    manager = mp.get_context("spawn").Manager()
+    out = manager.dict()
+    mp.start_processes(_ipc_worker, args=(world, port, out), nprocs=world, join=True, start_method="spawn")
+    locals_ = [(r + 1) << 40 for r in range(world)]
+    for rank in range(world):
+        bases, opened, closed = out[rank]
+        assert bases == [p if r == rank else p + 0x10 for r, p in enumerate(locals_)]
+        assert opened == [p for r, p in enumerate(locals_) if r != rank]
+        assert sorted(p for p, _ in closed) == sorted(p + 0x10 for p in opened)
