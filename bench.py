@@ -101,9 +101,10 @@ def kernel_sources_sha(kernel: str) -> str:
     return h.hexdigest()[:16]
 
 
-def ncu_traffic(kernel: str):
+def ncu_traffic(kernel: str, workload: str = ""):
     """Per-launch DRAM bytes of `kernel` from the committed ncu summary, or
-    None when the summary was taken on other kernel sources."""
+    None when the summary was taken on other kernel sources (or, with
+    `workload`, for a workload whose tag does not start with it)."""
     path = os.path.join(ROOT, "profiles", "ncu_traffic.md")
     if not os.path.exists(path):
         return None
@@ -112,7 +113,7 @@ def ncu_traffic(kernel: str):
     with open(path) as f:
         for line in f:
             m = pat.match(line.strip())
-            if m and m.group(1) == kernel and m.group(4) == sha:
+            if m and m.group(1) == kernel and m.group(4) == sha and m.group(2).startswith(workload):
                 return int(m.group(3))
     return None
 
@@ -529,7 +530,8 @@ def sweep_roofline(per, peak, peak_kind, launches, kernels):
         achieved = d["bytes"] / (d["ms"] / 1e3) / GB
         k = kernels[mode]
         out[mode] = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                     "frac": round(achieved / peak, 4), "traffic": ncu_traffic(k) if k in KERNEL_SOURCES else None,
+                     "frac": round(achieved / peak, 4),
+                     "traffic": ncu_traffic(k, "qwen3-235b-sweep") if k in KERNEL_SOURCES else None,
                      "kernel": k,
                      "launches_per_call": launches.get(mode, 1),
                      "bytes_per_launch": int(d["bytes"] / max(1, d["calls"])),
@@ -826,7 +828,7 @@ def _extra_nvfp4_30b(qz, device, rec):
     stack = synth.expert_stack(cfg["experts"], (rows, cols), cfg["std"], seed=cfg["seed"], device=device)
     ws = qz.alloc_workspace(cfg["experts"], device)
     for mode, fname, w in ((qz.NVFP4_PER_TENSOR_GIVEN, "given amax", None),
-                           (qz.NVFP4_PER_TENSOR_COMPUTE, "computed amax (one L2-chunked launch)", ws),
+                           (qz.NVFP4_PER_TENSOR_COMPUTE, "computed amax (one cooperative launch)", ws),
                            (qz.NVFP4_PER_TENSOR_COMPUTE, "computed amax (amax pass + quantize pass)", None)):
         ents = qz.alloc_outputs(list(stack.unbind(0)), qz.FMT_NVFP4, qz.SF_SWIZZLED, mode)
         for e in ents:
@@ -1225,7 +1227,7 @@ def refit_30b(qz, device, args, rank, dist_ok, peak):
            "issue": f"calls round-robin on {args.streams} streams" if side else "calls in order on one stream",
            "bytes_per_launch": int(np.mean([b for _, b in work.calls])),
            "effective_launch_us": round(1e3 * total_ms / (work.launches * args.steps), 2),
-           "traffic": ncu_traffic(work.kernel),
+           "traffic": ncu_traffic(work.kernel, "qwen3-30b-refit"),
            "single_stream": {"value": round(aggregate_gbs(work.bytes, world, args.steps, single_ms), 1),
                              "frac": round(achieved_single / peak, 4),
                              "mean_launch_us": round(1e3 * float(np.mean(single_launch_ms)), 2)},

@@ -364,17 +364,22 @@ __global__ void __launch_bounds__(kThreads, 3) amax_grouped_kernel(const qz_expe
 // A tensor's encode scale needs the amax of the whole tensor, so no element
 // of an expert can be quantized before all of it has been read.  Every CTA
 // (one per SM, all resident: a cooperative launch) runs
-//  - a producer warp that walks this CTA's amax units (units b, b + grid, ...
-//    of the call; a unit is up to 32 KB of one expert: a block of whole rows,
-//    or one 16384-column segment of a row) and copies each into a ring of
-//    kStages shared-memory stages with cp.async.bulk (the copy engine moves
-//    the bytes; no register holds them in flight), completion counted in
-//    bytes on each stage's mbarrier;
+//  - a producer warp whose lane i feeds stage i of a ring of kStages
+//    shared-memory stages: it walks its share of this CTA's amax units (units
+//    b, b + grid, ... of the call; a unit is up to 32 KB of one expert: a
+//    block of whole rows, or one 16384-column segment of a row) and copies
+//    each into the stage with cp.async.bulk (the copy engine moves the bytes;
+//    no register holds them in flight), completion counted in bytes on the
+//    stage's mbarrier -- the lanes work independently, so no unit waits for
+//    another stage's bookkeeping;
 //  - kStages consumer warps (consumer i takes stage i): the unit's largest
-//    magnitude from shared memory, folded into its expert's amax word (atomic
-//    max of bf16 magnitude bits), then -- after a fence -- one count on the
-//    expert's unit counter; a consumer holds no global load in flight, so its
-//    fence waits only for its own two atomics;
+//    magnitude from shared memory, folded into the CTA's maximum of its
+//    expert (shared memory); the consumer that folds the CTA's last unit of
+//    an expert queues the expert for
+//  - a publisher warp, which takes the finished experts in batches of up to
+//    32: the CTA's maxima into the experts' amax words (atomic max of bf16
+//    magnitude bits), one fence, then the CTA's unit counts -- so no stage
+//    ever waits for a fence;
 //  - kQWarps quantize warps (the tile walk of the grouped kernel: 8 warps own
 //    the row groups of a 128 x 128 tile) that take tiles b, b + grid, ... and
 //    quantize each once its expert's unit counter is complete (a bounded
@@ -398,7 +403,7 @@ constexpr int kQWarps = 8 * kQGroups;  // quantize warps: 8 per group (the 8 row
 constexpr int kStages = 4;             // shared-memory stages of the amax ring (one consumer warp each)
 constexpr int kUnitBytes = 32768;      // bytes of one amax unit (one stage)
 constexpr int kWindowTiles = 1536;     // how far (in tiles, ~48 MB) the copies may run ahead
-constexpr int kPipeThreads = 32 * (kQWarps + 1 + kStages);
+constexpr int kPipeThreads = 32 * (kQWarps + 1 + kStages + 1);  // + producer, consumers, publisher
 constexpr int kMaxChunks = 4096;       // workspace words reserved for the per-expert unit counters
 constexpr int kWsHeader = 8;
 constexpr long long kDefaultWaitNs = 20LL * 1000 * 1000;  // 20 ms: far above any legitimate wait
@@ -488,14 +493,18 @@ struct TableUnits {
 
 // Warp-uniform bounded wait until every lane sees `ready()`; false when the
 // time limit ran out (QZ_DERR_TIMEOUT, abort raised) or the kernel aborted.
+// The CTA's abort flag (shared memory) is checked on every poll; the global
+// abort word and the timer only on every 64th, so that a poll costs no
+// L2 round trip of its own.
 template <typename Ready>
 __device__ __forceinline__ bool bounded_wait(Ready ready, volatile unsigned* abort_word, volatile int* s_abort,
                                              long long limit, unsigned* d_err, int lane, unsigned sleep_ns) {
     const long long t0 = global_ns();
-    for (;;) {
+    for (unsigned it = 1;; ++it) {
         if (__all_sync(0xFFFFFFFFu, ready())) return true;
-        const bool aborted = *abort_word != 0u || *s_abort != 0;
-        const bool late = global_ns() - t0 > limit;
+        const bool rare = (it & 63u) == 0u;
+        const bool aborted = *s_abort != 0 || (rare && *abort_word != 0u);
+        const bool late = rare && global_ns() - t0 > limit;
         if (__any_sync(0xFFFFFFFFu, aborted || late)) {
             if (!__any_sync(0xFFFFFFFFu, aborted) && lane == 0) {
                 if (d_err) atomicOr(d_err, QZ_DERR_TIMEOUT);
@@ -519,6 +528,7 @@ __global__ void __launch_bounds__(kPipeThreads, 1) nvfp4_compute_pipe_kernel(
     int* s_uprefix = s_prefix + (n + 1);                                     // n + 1: first unit of each expert
     unsigned* s_emax = reinterpret_cast<unsigned*>(s_uprefix + (n + 1));     // n: this CTA's maximum per expert
     unsigned* s_ecnt = s_emax + n;                                           // n: this CTA's units folded per expert
+    volatile int* s_pubq = reinterpret_cast<volatile int*>(s_ecnt + n);      // n: experts this CTA has finished, in order
     __shared__ long long s_scan[33];
     __shared__ __align__(16) uint8_t s_sf[kQWarps][64 * G::kSfTiles];
     __shared__ float s_inv[16];
@@ -527,9 +537,14 @@ __global__ void __launch_bounds__(kPipeThreads, 1) nvfp4_compute_pipe_kernel(
     __shared__ unsigned s_unit_bytes[kStages];
     __shared__ volatile int s_qtile[kQWarps];  // quantize warp w has done this CTA's tiles below this
     __shared__ volatile int s_abort;
+    __shared__ unsigned s_pubtail;  // entries pushed to s_pubq
     fill_inv_table(s_inv);
     if (threadIdx.x < kQWarps) s_qtile[threadIdx.x] = 0;
-    for (int i = threadIdx.x; i < n; i += blockDim.x) s_emax[i] = s_ecnt[i] = 0u;  // published by block_prefix
+    for (int i = threadIdx.x; i < n; i += blockDim.x) {  // published by block_prefix's barriers
+        s_emax[i] = s_ecnt[i] = 0u;
+        s_pubq[i] = -1;
+    }
+    if (threadIdx.x == 0) s_pubtail = 0u;
     if (threadIdx.x == 0) {
         s_abort = 0;
         for (int i = 0; i < kStages; ++i) {
@@ -601,68 +616,132 @@ __global__ void __launch_bounds__(kPipeThreads, 1) nvfp4_compute_pipe_kernel(
     }
 
     if (wid == kQWarps) {
-        // ---------------- producer: units b, b + grid, ... into the ring ----------------
-        int k = 0;  // units of this CTA issued so far
-        bool ok = true;
-        for (int u = b; u < units && ok; u += grid, ++k) {
-            const int stage = k % kStages;
-            const int use = k / kStages;
-            if (use > 0) {
-                uint64_t* eb = &s_empty[stage];
-                const unsigned par = (unsigned)((use - 1) & 1);
-                ok = bounded_wait([&] { return mbar_test(eb, par); }, abort_word, &s_abort, limit, d_err, lane, 0);
-                if (!ok) break;
-            }
-            const int e = find_owner(s_uprefix, n, u);
-            const int first_tile = s_prefix[e];
-            ok = bounded_wait(
-                [&] {
+        // ---------------- producer: lane i < kStages feeds stage i with this CTA's units
+        //                  k = i, i + kStages, ... (unit b + k grid of the call) ----------------
+        const bool feeds = lane < kStages;
+        int k = lane;  // this lane's next unit, counted among the CTA's units
+        long long t_last = global_ns();
+        bool stop = false;
+        for (unsigned it = 1;; ++it) {
+            const int u = b + k * grid;
+            const bool pending = feeds && u < units;
+            if (!__any_sync(0xFFFFFFFFu, pending)) break;
+            bool issued = false;
+            if (pending) {
+                const int use = k / kStages;
+                bool ready = use == 0 || mbar_test(&s_empty[lane], (unsigned)((use - 1) & 1));
+                int e = 0;
+                if (ready) {
+                    e = find_owner(s_uprefix, n, u);
                     int lo = total;
 #pragma unroll
                     for (int q = 0; q < kQWarps; ++q) lo = min(lo, s_qtile[q]);
-                    return first_tile - lo <= kWindowTiles;
-                },
-                abort_word, &s_abort, limit, d_err, lane, 64);
-            if (!ok) break;
-            const qz_expert E = load_entry(table, e);
-            const UnitGeo g = unit_geo(E);
-            const int j = u - s_uprefix[e];
-            const int64_t r0 = (int64_t)(j / g.nseg) * g.krows;
-            const int64_t c0 = (int64_t)(j % g.nseg) * g.seg;
-            const int nr = (int)min((int64_t)g.krows, E.rows - r0);
-            const int nc = (int)min((int64_t)g.seg, E.cols - c0);
-            const unsigned bytes = (unsigned)(nr * nc * 2);
-            const uint16_t* src = static_cast<const uint16_t*>(E.x) + r0 * E.ld + c0;
-            unsigned char* dst = s_ring + stage * kUnitBytes;
-            if (lane == 0) {
-                s_unit_expert[stage] = e;
-                s_unit_bytes[stage] = bytes;
-                mbar_arrive_expect_tx(&s_full[stage], bytes);  // releases the two words above
-            }
-            __syncwarp();
-            if (g.nseg == 1 && E.ld == E.cols) {
-                if (lane == 0) bulk_copy_g2s(dst, src, bytes, &s_full[stage]);  // whole rows, contiguous
-            } else {
-                for (int r = lane; r < nr; r += 32)
-                    bulk_copy_g2s(dst + r * nc * 2, src + (int64_t)r * E.ld, (unsigned)(nc * 2), &s_full[stage]);
-            }
-        }
-        if (!ok) {
-            // let the copies already issued land before the CTA can retire
-            for (int i = max(0, k - kStages); i < k; ++i) {
-                uint64_t* fb = &s_full[i % kStages];
-                const unsigned par = (unsigned)((i / kStages) & 1);
-                const long long t0 = global_ns();
-                while (!__all_sync(0xFFFFFFFFu, mbar_test(fb, par)) && global_ns() - t0 < limit) {
+                    ready = s_prefix[e] - lo <= kWindowTiles;  // the expert starts within the window
+                }
+                if (ready) {
+                    const qz_expert E = load_entry(table, e);
+                    const UnitGeo g = unit_geo(E);
+                    const int j = u - s_uprefix[e];
+                    const int rb = g.nseg == 1 ? j : j / g.nseg;
+                    const int64_t r0 = (int64_t)rb * g.krows;
+                    const int64_t c0 = (int64_t)(j - rb * g.nseg) * g.seg;
+                    const int nr = (int)min((int64_t)g.krows, E.rows - r0);
+                    const int nc = (int)min((int64_t)g.seg, E.cols - c0);
+                    const unsigned bytes = (unsigned)(nr * nc * 2);
+                    const uint16_t* src = static_cast<const uint16_t*>(E.x) + r0 * E.ld + c0;
+                    unsigned char* dst = s_ring + lane * kUnitBytes;
+                    s_unit_expert[lane] = e;
+                    s_unit_bytes[lane] = bytes;
+                    mbar_arrive_expect_tx(&s_full[lane], bytes);  // releases the two words above
+                    if (g.nseg == 1 && E.ld == E.cols) {
+                        bulk_copy_g2s(dst, src, bytes, &s_full[lane]);  // whole rows, contiguous
+                    } else {
+                        for (int r = 0; r < nr; ++r)
+                            bulk_copy_g2s(dst + r * nc * 2, src + (int64_t)r * E.ld, (unsigned)(nc * 2), &s_full[lane]);
+                    }
+                    k += kStages;
+                    issued = true;
                 }
             }
+            if (__any_sync(0xFFFFFFFFu, issued)) {
+                t_last = global_ns();  // the limit counts from the last progress
+            } else {
+                const bool rare = (it & 63u) == 0u;
+                const bool aborted = s_abort != 0 || (rare && *abort_word != 0u);
+                const bool late = rare && global_ns() - t_last > limit;
+                if (__any_sync(0xFFFFFFFFu, aborted || late)) {
+                    if (!__any_sync(0xFFFFFFFFu, aborted) && lane == 0) {
+                        if (d_err) atomicOr(d_err, QZ_DERR_TIMEOUT);
+                        *abort_word = 1u;
+                        s_abort = 1;
+                    }
+                    stop = true;
+                    break;
+                }
+                __nanosleep(32);
+            }
+        }
+        // the copies already issued must land before the CTA can retire
+        if (stop && feeds && k >= kStages) {
+            const int last = k - kStages;  // this lane's last issued unit
+            const long long t0 = global_ns();
+            while (!mbar_test(&s_full[lane], (unsigned)((last / kStages) & 1)) && global_ns() - t0 < limit) {
+            }
+        }
+        return;
+    }
+
+    // this CTA's units of expert e: units b + k grid inside [s_uprefix[e], s_uprefix[e + 1])
+    auto mine_of = [&](int e) {
+        const int u0 = s_uprefix[e] - b, u1 = s_uprefix[e + 1] - b;
+        return (unsigned)(max(0, (u1 + grid - 1) / grid) - max(0, (u0 + grid - 1) / grid));
+    };
+    const bool withhold = (test_flags & QZ_TEST_WITHHOLD_ARRIVALS) != 0u;
+
+    if (wid == kQWarps + 1 + kStages) {
+        // ---------------- publisher: the experts this CTA has finished, in batches of up
+        //                  to 32: every maximum, one fence, then every count ----------------
+        int expect = 0;  // experts with at least one unit of this CTA
+        for (int e = lane; e < n; e += 32) expect += mine_of(e) != 0u ? 1 : 0;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) expect += __shfl_xor_sync(0xFFFFFFFFu, expect, o);
+        int head = 0;
+        long long t_last = global_ns();
+        for (unsigned it = 1; head < expect; ++it) {
+            const int e = head + lane < expect ? s_pubq[head + lane] : -1;
+            const unsigned have = __ballot_sync(0xFFFFFFFFu, e >= 0);
+            const int nb = have == 0xFFFFFFFFu ? 32 : __ffs(~have) - 1;  // the leading run of finished experts
+            if (nb == 0) {
+                const bool rare = (it & 63u) == 0u;
+                const bool aborted = s_abort != 0 || (rare && *abort_word != 0u);
+                const bool late = rare && global_ns() - t_last > limit;
+                if (__any_sync(0xFFFFFFFFu, aborted || late)) {
+                    if (!__any_sync(0xFFFFFFFFu, aborted) && lane == 0) {
+                        if (d_err) atomicOr(d_err, QZ_DERR_TIMEOUT);
+                        *abort_word = 1u;
+                        s_abort = 1;
+                    }
+                    return;
+                }
+                __nanosleep(64);
+                continue;
+            }
+            __threadfence_block();  // the queue entries were written after the experts' last folds
+            if (lane < nb) {
+                const unsigned m = atomicMax(s_emax + e, 0u);  // every fold of this CTA is in
+                if (m != 0u) atomicMax(amax_ws + e, m);
+            }
+            __threadfence();  // the maxima are visible before the counts that release them
+            if (lane < nb && !withhold) atomicAdd(counted + e, mine_of(e));
+            __syncwarp();
+            head += nb;
+            t_last = global_ns();
         }
         return;
     }
 
     // ---------------- consumers: consumer i takes stage i (units k = i, i + kStages, ...) ----------------
     const int ci = wid - kQWarps - 1;
-    const bool withhold = (test_flags & QZ_TEST_WITHHOLD_ARRIVALS) != 0u;
     const int mine = (units - b + grid - 1) / grid;  // units of this CTA
     for (int k = ci; k < mine; k += kStages) {
         uint64_t* fb = &s_full[ci];
@@ -690,18 +769,12 @@ __global__ void __launch_bounds__(kPipeThreads, 1) nvfp4_compute_pipe_kernel(
         for (int o = 16; o > 0; o >>= 1) r = max(r, __shfl_xor_sync(0xFFFFFFFFu, r, o));
         if (lane == 0) {
             // fold into this CTA's maximum of expert e; the consumer that folds
-            // the CTA's last unit of e publishes the maximum and the CTA's
-            // unit count (one global max and one add per CTA and expert)
+            // the CTA's last unit of e hands the expert to the publisher
             atomicMax(s_emax + e, r << 16);
             __threadfence_block();
-            const int u0 = s_uprefix[e] - b, u1 = s_uprefix[e + 1] - b;
-            const unsigned mine_e = (unsigned)(max(0, (u1 + grid - 1) / grid) - max(0, (u0 + grid - 1) / grid));
-            if (atomicAdd(s_ecnt + e, 1u) + 1u == mine_e) {
+            if (atomicAdd(s_ecnt + e, 1u) + 1u == mine_of(e)) {
                 __threadfence_block();
-                const unsigned m = atomicMax(s_emax + e, 0u);  // every fold of this CTA is in
-                if (m != 0u) atomicMax(amax_ws + e, m);
-                __threadfence();  // the maximum is visible before the count that releases it
-                if (!withhold) atomicAdd(counted + e, mine_e);
+                s_pubq[atomicAdd(&s_pubtail, 1u)] = e;
             }
         }
     }
@@ -807,7 +880,7 @@ cudaError_t launch_nvfp4_tensor(const qz_expert* table, int n, int layout, bool 
 
 size_t workspace_bytes(int n) { return workspace_words(n) * sizeof(unsigned); }
 
-size_t compute_pipe_smem(int n) { return (size_t)kStages * kUnitBytes + (size_t)(4 * n + 2) * sizeof(int); }
+size_t compute_pipe_smem(int n) { return (size_t)kStages * kUnitBytes + (size_t)(5 * n + 2) * sizeof(int); }
 
 // One cooperative launch of the computed-amax pipeline on a zeroed workspace
 // (every CTA resident: a quantize warp waits on amax warps of every CTA).
