@@ -102,8 +102,8 @@ typedef enum qz_nvfp4_scale_mode {
                                   aligned (swizzled); amax not 4-byte aligned */
 #define QZ_DERR_TOO_LARGE 0x8u /* the call's total tile or row count exceeds 2^31 - 1 */
 #define QZ_DERR_TIMEOUT 0x10u  /* a bounded wait of the single-launch computed-amax path (quantize
-                                  warps waiting until every amax warp is done with a chunk, or
-                                  amax warps waiting for their CTA's quantize warps) exceeded
+                                  warps waiting for an expert's amax, or the copy, amax and
+                                  publishing warps waiting on one another) exceeded
                                   qz_launch_opts.wait_limit_ns; the launch stopped early and some
                                   outputs are unwritten (no such wait is expected to expire) */
 #define QZ_DERR_CUT 0x20u      /* qz_split_fused_experts: the cut falls inside a scale block
@@ -192,8 +192,9 @@ typedef struct qz_launch_opts {
                                The results do not depend on it. */
     void *d_workspace;      /* optional device scratch for QZ_NVFP4_PER_TENSOR_COMPUTE: with
                                at least qz_workspace_bytes(n_experts) bytes (4-byte aligned),
-                               the call runs one L2-chunked launch instead of an amax pass
-                               and a quantize pass over HBM.  The call zeroes it first (in
+                               the call runs one cooperative launch that reads the input from
+                               HBM once (the quantize side re-reads it from L2) instead of an
+                               amax pass and a quantize pass over HBM.  The call zeroes it first (in
                                stream order); calls sharing a workspace must not overlap. */
     size_t workspace_bytes; /* size of d_workspace in bytes */
     int64_t elems_hint;     /* qz_quantize_grouped_mxfp8 and the MXFP8 qz_dequantize_grouped: the call's
@@ -207,8 +208,9 @@ typedef struct qz_launch_opts {
                                GPU's global timer; 0 = the default of 20 ms.  A wait that runs out
                                sets QZ_DERR_TIMEOUT and ends the launch early. */
     unsigned int test_flags; /* 0 in normal use.  QZ_TEST_WITHHOLD_ARRIVALS makes the single-launch
-                               computed-amax path skip the counts that release its quantize warps, so
-                               every wait runs out: a test of the timeout path that needs no fault. */
+                               computed-amax path withhold the counts that release its quantize
+                               warps, so their waits run out: a test of the timeout path that
+                               needs no fault. */
     unsigned int launch_flags; /* QZ_OPT_INDEPENDENT: see below; 0 otherwise. */
 } qz_launch_opts;
 
@@ -262,9 +264,10 @@ qz_status qz_quantize_grouped_mxfp8(const qz_expert *d_table, int n_experts, int
  * PER_TENSOR_COMPUTE without a workspace runs a clear, an amax pass and the
  * quantize pass (three launches in stream order, the input read twice from
  * HBM); with opts->d_workspace it runs one cooperative launch (plus a memset
- * of the workspace) in which amax warps read each chunk of whole experts from
- * HBM one chunk ahead of quantize warps, which re-read it from L2 once every
- * amax warp of the grid is done with it (bounded waits: wait_limit_ns).
+ * of the workspace) in which bulk copies bring every expert from HBM into
+ * shared memory for its amax, ahead of quantize warps that re-read the expert
+ * from L2 once every CTA's share of its amax is in (bounded waits:
+ * wait_limit_ns).
  * PER_ROW reads each row once.
  * Entries may share one amax slot, so that the gate and up halves of a fused
  * expert ([FOLD]: one amax over the fused (2I, H) slice, one weight_scale_2)
@@ -482,9 +485,9 @@ qz_status qz_split_fused_experts(const qz_fused_split *d_table, int n, int fmt, 
 #define QZ_STATIC_WS_MAX_EXPERTS 1024
 
 /* Allocation-free NVFP4 quantization with a computed per-tensor amax: the
- * same single L2-chunked launch as qz_quantize_grouped_nvfp4 in
+ * same single cooperative launch as qz_quantize_grouped_nvfp4 in
  * QZ_NVFP4_PER_TENSOR_COMPUTE mode with opts->d_workspace, but its scratch
- * (a work counter, per-chunk counters and per-expert amax words, about 21 KB)
+ * (an abort word, per-expert unit counters and amax words, about 21 KB)
  * is a device array inside the library, so the caller passes only the table,
  * inputs and outputs.  The source pages have no counterpart of this entry
  * point; it exists for callers that cannot allocate device memory themselves,

@@ -935,7 +935,7 @@ int grouped_blocks_per_sm(int which, int n) {
 }  // namespace qz
 
 // ---------------------------------------------------------------------------
-// Allocation-free variant of the L2-chunked computed-amax launch: its scratch
+// Allocation-free variant of the single-launch computed-amax path: its scratch
 // is this file-scope device array instead of a caller workspace.  Every GPU
 // that loads the library holds it until the process exits.
 // ---------------------------------------------------------------------------

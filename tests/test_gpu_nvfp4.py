@@ -246,7 +246,7 @@ def test_strided_rows_all_modes(mode):
 
 
 def run_compute_l2(xs, layout, **kw):
-    """Computed per-tensor amax through the single-launch L2-chunked path."""
+    """Computed per-tensor amax through the single cooperative launch."""
     entries, keep = guarded_entries(xs, qz.FMT_NVFP4, layout, qz.NVFP4_PER_TENSOR_COMPUTE)
     ws = qz.alloc_workspace(len(xs))
     ws.fill_(0xFF)                       # the call zeroes what it needs
