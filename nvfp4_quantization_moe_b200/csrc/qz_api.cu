@@ -34,10 +34,10 @@ cudaError_t launch_nvfp4_compute_l2_static(const qz_expert* table, int n, int la
 int rows_blocks_per_sm(int n);
 cudaError_t launch_dequant(const qz_dq_expert* table, int n, int fmt, bool per_row, int layout, int grid,
                            cudaStream_t s, unsigned* d_err);
-int dequant_blocks_per_sm(int n);
+int dequant_blocks_per_sm(int n, int fmt);
 cudaError_t launch_colwise(const qz_expert* table, int n, int fmt, int layout, int grid, cudaStream_t s,
                            unsigned* d_err);
-int colwise_blocks_per_sm(int n);
+int colwise_blocks_per_sm(int n, int fmt);
 cudaError_t launch_split_fused(const qz_fused_split* table, int n, int fmt, int amax_kind, int src_layout,
                                int dst_layout, int grid, cudaStream_t s, unsigned* d_err);
 int split_blocks_per_sm(int n);
@@ -48,12 +48,12 @@ cudaError_t launch_attention_merge(const float* O, const float* lse, int S, int6
 namespace {
 
 constexpr int kMaxDevices = 64;
-constexpr int kKinds = 9;  // mxfp8, nvfp4 tile, swizzle, amax, rows, computed-amax L2 path, dequantize, colwise,
-                           // fused split
+constexpr int kKinds = 11;  // mxfp8, nvfp4 tile, swizzle, amax, rows, computed-amax L2 path, dequantize MXFP8,
+                            // colwise MXFP8, fused split, dequantize NVFP4, colwise NVFP4
 
 struct DeviceLimits {
     int sms = 0;
-    int per_sm[kKinds] = {0, 0, 0, 0, 0, 0, 0, 0, 0};
+    int per_sm[kKinds] = {0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0};
 };
 
 std::mutex g_mu;
@@ -76,8 +76,10 @@ int wave_grid(int kind, const qz_launch_opts* opts) {
         }
         if (d.per_sm[kind] == 0)
             d.per_sm[kind] = (kind == 4)   ? qz::rows_blocks_per_sm(QZ_MAX_EXPERTS)
-                             : (kind == 6) ? qz::dequant_blocks_per_sm(QZ_MAX_EXPERTS)
-                             : (kind == 7) ? qz::colwise_blocks_per_sm(QZ_MAX_EXPERTS)
+                             : (kind == 6) ? qz::dequant_blocks_per_sm(QZ_MAX_EXPERTS, QZ_FMT_MXFP8)
+                             : (kind == 9) ? qz::dequant_blocks_per_sm(QZ_MAX_EXPERTS, QZ_FMT_NVFP4)
+                             : (kind == 7) ? qz::colwise_blocks_per_sm(QZ_MAX_EXPERTS, QZ_FMT_MXFP8)
+                             : (kind == 10) ? qz::colwise_blocks_per_sm(QZ_MAX_EXPERTS, QZ_FMT_NVFP4)
                              : (kind == 8) ? qz::split_blocks_per_sm(QZ_MAX_EXPERTS)
                                            : qz::grouped_blocks_per_sm(kind, QZ_MAX_EXPERTS);
         grid = d.sms * d.per_sm[kind];
@@ -281,7 +283,7 @@ qz_status qz_dequantize_grouped(const qz_dq_expert* d_table, int n_experts, int 
     if (fmt != QZ_FMT_MXFP8 && fmt != QZ_FMT_NVFP4) return QZ_ERR_INVALID_ARG;
     if (n_experts == 0) return QZ_OK;
     return from_cuda(qz::launch_dequant(d_table, n_experts, fmt, per_row != 0, layout,
-                                        fmt == QZ_FMT_MXFP8 ? sized_grid(6, opts) : wave_grid(6, opts),
+                                        fmt == QZ_FMT_MXFP8 ? sized_grid(6, opts) : wave_grid(9, opts),
                                         (cudaStream_t)stream, err_word(opts)));
 }
 
@@ -292,7 +294,8 @@ qz_status qz_quantize_grouped_colwise(const qz_expert* d_table, int n_experts, i
     if (!valid_layout(layout)) return QZ_ERR_INVALID_ARG;
     if (fmt != QZ_FMT_MXFP8 && fmt != QZ_FMT_NVFP4) return QZ_ERR_INVALID_ARG;
     if (n_experts == 0) return QZ_OK;
-    return from_cuda(qz::launch_colwise(d_table, n_experts, fmt, layout, wave_grid(7, opts), (cudaStream_t)stream,
+    return from_cuda(qz::launch_colwise(d_table, n_experts, fmt, layout,
+                                        wave_grid(fmt == QZ_FMT_MXFP8 ? 7 : 10, opts), (cudaStream_t)stream,
                                         err_word(opts)));
 }
 

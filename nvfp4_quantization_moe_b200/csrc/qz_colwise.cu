@@ -10,23 +10,37 @@
 //
 // One persistent launch walks all experts' 128 x 128 tiles, each CTA a
 // contiguous run of them (so its expert -- the entry and the NVFP4 scale --
-// changes rarely).  Each CTA keeps three tiles in flight: asynchronous
-// 16-byte copies (cp.async, zero-filled past the matrix) bring a tile
-// row-major into one of three shared-memory stages while the tile before it
-// is quantized, so the loads never wait on the arithmetic and one CTA
-// barrier per tile suffices.  A thread reads one
-// 32-bit word per row -- two neighbouring columns -- for 32 rows, pairs
-// consecutive rows of each column into bf16x2 words, quantizes the two
-// 32-element column segments with the library's block quantizers
-// (include/qz_quant.cuh) and writes them to the transposed payload.  NVFP4
-// takes the tensor amax as given (the row-wise computed-amax call of the
-// same tensor produces it).
+// changes rarely).  Each CTA keeps
+// three tiles in flight: asynchronous 16-byte copies (cp.async, zero-filled
+// past the matrix) bring a tile row-major into one of three shared-memory
+// stages while the tile before it is quantized, so the loads never wait on
+// the arithmetic and one CTA barrier per tile suffices.
+//   MXFP8: a thread reads one 32-bit word per row -- two neighbouring
+//   columns -- for 32 rows, pairs consecutive rows of each column into bf16x2
+//   words and quantizes the two 32-element column segments with the
+//   library's block quantizers (include/qz_quant.cuh).
+//   NVFP4: the transpose is done by ldmatrix.trans from a swizzled stage,
+//   which hands each thread two whole 16-row column blocks in the same bf16x2
+//   word form, four instructions for 32 elements.
+// The quantized blocks go straight to the transposed payload.  NVFP4 takes
+// the tensor amax as given (the row-wise computed-amax call of the same
+// tensor produces it).
 #include "../../include/qz_quant.cuh"
 #include "qz_async.cuh"
 
 namespace qz {
 
 constexpr int kColThreads = 256;
+constexpr int kColStages = 3;  // tiles in flight per CTA
+
+// Per format: tile columns, CTAs per SM, and whether the stage is swizzled.
+template <int FMT>
+struct ColGeo {
+    static constexpr int kTC = 128;
+    static constexpr int kCtas = 2;
+    static constexpr int kStageBytes = kTileRows * kTC * 2;  // one bf16 tile, row-major (32 / 16 KB)
+    static constexpr int kBlock = FMT == QZ_FMT_MXFP8 ? 32 : 16;
+};
 
 // NVFP4 block scale codes of two 16-element blocks (8 bf16x2 words each).
 __device__ __forceinline__ uint32_t tile_scales_nv_words(const uint32_t* w0, const uint32_t* w1, float S) {
@@ -49,7 +63,14 @@ __device__ __forceinline__ unsigned colwise_entry_errors(const qz_expert& e, int
     return bad;
 }
 
-template <int FMT, int LAYOUT>
+// Column tiles of an expert with C columns: whole 128-column groups, so that
+// the tiles also cover the swizzled layout's padded scale rows up to the next
+// multiple of 128 (with 64-column tiles a group past the last column is a
+// tile of zeros that writes only padding).
+template <int TC>
+__device__ __forceinline__ int64_t col_tiles_c(int64_t C) { return (C + 127) / 128 * (128 / TC); }
+
+template <int FMT, int LAYOUT, int TC>
 struct ColTiles {
     const qz_expert* table;
     unsigned* d_err;
@@ -58,7 +79,7 @@ struct ColTiles {
         const unsigned bad = colwise_entry_errors(e, FMT, LAYOUT);
         if (bad && d_err && blockIdx.x == 0) atomicOr(d_err, bad);
         if (bad || e.rows == 0) return 0;
-        return ((e.rows + kTileRows - 1) / kTileRows) * ((e.cols + kTileCols - 1) / kTileCols);
+        return ((e.rows + kTileRows - 1) / kTileRows) * col_tiles_c<TC>(e.cols);
     }
 };
 
@@ -75,12 +96,13 @@ struct ColRef {
     int expert;
 };
 
+template <int TC>
 __device__ __forceinline__ ColRef col_ref(const qz_expert* table, const int* s_prefix, int tile, int e) {
     while (tile >= s_prefix[e + 1]) ++e;  // tiles increase; s_prefix[n] == total > tile
     const qz_expert E = load_entry(table, e);
     const int local = tile - s_prefix[e];
     ColRef r;
-    r.nct = (int)((E.cols + kTileCols - 1) / kTileCols);
+    r.nct = (int)col_tiles_c<TC>(E.cols);
     r.rt = local / r.nct;
     r.ct = local - r.rt * r.nct;
     r.x = static_cast<const uint16_t*>(E.x);
@@ -95,6 +117,7 @@ __device__ __forceinline__ ColRef col_ref(const qz_expert* table, const int* s_p
 }
 
 // r describes tile - 1; make it describe tile.
+template <int TC>
 __device__ __forceinline__ void col_next(ColRef& r, const qz_expert* table, const int* s_prefix, int tile) {
     if (tile < s_prefix[r.expert + 1]) {
         if (++r.ct == r.nct) {
@@ -102,40 +125,159 @@ __device__ __forceinline__ void col_next(ColRef& r, const qz_expert* table, cons
             ++r.rt;
         }
     } else {
-        r = col_ref(table, s_prefix, tile, r.expert + 1);
+        r = col_ref<TC>(table, s_prefix, tile, r.expert + 1);
     }
 }
 
-constexpr int kColStages = 3;                                     // tiles in flight per CTA
-constexpr int kColStageBytes = kTileRows * kTileCols * 2;         // one bf16 tile, row-major (32 KB)
+// NVFP4 stages hold a tile row-major with its 16-byte chunks permuted per
+// row: chunk cc of row r sits at chunk position cc ^ swz(r), swz(r) = bit 0
+// of r and bits 4-5 of r as bits 1-2.  The eight rows that one ldmatrix
+// reads (below) then fall into eight different bank groups.
+__device__ __forceinline__ int nv_stage_swz(int r) { return (r & 1) | (((r >> 4) & 3) << 1); }
 
-// Issue thread t's copies of a tile into a stage: chunk t % 16 (8 columns)
-// of rows t / 16 + 16 k.  Rows past the matrix and columns past its last one
-// are zero-filled without reading.
+// Issue thread t's copies of a tile into a stage: chunk t % (TC / 8) (8
+// columns) of rows t / (TC / 8) + (2048 / TC) k.  Rows past the matrix and
+// columns past its last one are zero-filled without reading.
+template <int TC, bool SWZ>
 __device__ __forceinline__ void col_issue(const ColRef& r, uint32_t stage, int t) {
-    const int cc = t & 15;
-    const int64_t c = (int64_t)r.ct * kTileCols + 8 * cc;
+    constexpr int kChunks = TC / 8;                  // 16-byte chunks per tile row
+    constexpr int kRowsPer = kColThreads / kChunks;  // rows per round of the CTA's threads
+    const int cc = t % kChunks;
+    const int64_t c = (int64_t)r.ct * TC + 8 * cc;
     const int64_t cols_left = r.C - c;
     const int cbytes = cols_left >= 8 ? 16 : (cols_left > 0 ? (int)cols_left * 2 : 0);
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
-        const int row = (t >> 4) + 16 * k;
+    for (int k = 0; k < kTileRows / kRowsPer; ++k) {
+        const int row = t / kChunks + kRowsPer * k;
         const int64_t rg = (int64_t)r.rt * kTileRows + row;
         const bool in = rg < r.R && cbytes > 0;
         const void* src = in ? static_cast<const void*>(r.x + rg * r.ld + c) : static_cast<const void*>(r.x);
-        cp_async_16(stage + (uint32_t)(row * (kTileCols * 2) + 16 * cc), src, in ? cbytes : 0);
+        const int pc = SWZ ? (cc ^ nv_stage_swz(row)) : cc;
+        cp_async_16(stage + (uint32_t)(row * (TC * 2) + 16 * pc), src, in ? cbytes : 0);
+    }
+}
+
+// Four 8x8 bf16 matrices from shared memory, transposed: lanes 8 m .. 8 m + 7
+// give the 16-byte source rows of matrix m; register m of lane l receives the
+// elements of source rows 2 (l % 4) and + 1 in column l / 4 (low half first).
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t& a, uint32_t& b, uint32_t& c, uint32_t& d) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(a), "=r"(b), "=r"(c), "=r"(d)
+                 : "r"(addr)
+                 : "memory");
+}
+
+// MXFP8: the tile in stage s_words (128 x 128, row-major); thread (warp w,
+// lane l) quantizes tile columns 64 (w % 2) + 2 l and + 1, rows 32 (w / 2) ..
+// + 31 of each: one word per row holds both columns.
+template <int LAYOUT>
+__device__ __forceinline__ void col_tile_mx(const ColRef& cur, const uint32_t* s_words, int w, int lane) {
+    constexpr int kTC = 128, kBlock = 32;
+    const int ch = w & 1, rs = w >> 1;
+    const int64_t R = cur.R, C = cur.C;
+    const uint32_t* tw = s_words + (32 * rs) * (kTC / 2) + 32 * ch + lane;
+    uint32_t xa[16], xb[16];  // column pairs (row 2i low, row 2i + 1 high) of the two columns
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const uint32_t r0 = tw[(2 * i) * (kTC / 2)], r1 = tw[(2 * i + 1) * (kTC / 2)];
+        xa[i] = __byte_perm(r0, r1, 0x5410);
+        xb[i] = __byte_perm(r0, r1, 0x7632);
+    }
+    const int64_t cg = (int64_t)cur.ct * kTC + 64 * ch + 2 * lane;  // x column = transposed row
+    const int64_t e0 = (int64_t)cur.rt * kTileRows + 32 * rs;       // first x row of the segment
+    const int64_t cpad = LAYOUT == QZ_SF_SWIZZLED_128x4 ? ((C + 127) & ~(int64_t)127) : C;
+    const int64_t kvT = R / kBlock;  // scale columns of the transposed matrix
+    const int64_t kvs = LAYOUT == QZ_SF_SWIZZLED_128x4 ? ((kvT + 3) & ~(int64_t)3) : kvT;
+    const int64_t k0 = e0 / kBlock;  // the segment's scale column
+    uint32_t qa[8], qb[8];
+    const uint32_t sa = qzq::mxfp8_block(xa, qa);
+    const uint32_t sb = qzq::mxfp8_block(xb, qb);
+    if (e0 < R) {
+        const bool q32 = ((reinterpret_cast<uintptr_t>(cur.q) & 31) == 0);
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            if (cg + j >= C) continue;
+            const uint32_t* qq = j ? qb : qa;
+            uint8_t* dst = cur.q + (cg + j) * R + e0;
+            const uint4 lo = make_uint4(qq[0], qq[1], qq[2], qq[3]), hi = make_uint4(qq[4], qq[5], qq[6], qq[7]);
+            if (q32) {
+                st_v8(dst, lo, hi);
+            } else {
+                st_v4(dst, lo);
+                st_v4(dst + 16, hi);
+            }
+        }
+    }
+    // scale bytes (a block past the last row holds zeros and gets scale 0;
+    // padded transposed rows C <= cg < cpad get 0x00)
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+        const int64_t row = cg + j;
+        if (row >= cpad || k0 >= kvs) continue;
+        cur.sf[qzq::sf_offset(row, k0, kvT, LAYOUT)] = row < C ? (uint8_t)(j ? sb : sa) : (uint8_t)0;
+    }
+}
+
+// NVFP4: the tile at stage address st (128 x TC, swizzled).  Lane 4 c + j of
+// warp w holds column 8 (w + 8 u) + c of the tile (u < TC / 64) and the
+// blocks of rows 16 j + 64 h .. + 15 (h = 0, 1) as 8 bf16x2 words each (word
+// m = rows 2m, 2m + 1 of the block, low half first).  Matrix m of half h
+// reads, in source row i (supplied by lane 8 (m % 4) + i of the x4 that
+// covers it), tile row 64 h + 16 (i / 2) + 2 m + i % 2, whose swizzle is i:
+// the 8 rows hit 8 bank groups.
+template <int LAYOUT, int TC>
+__device__ __forceinline__ void col_tile_nv(const ColRef& cur, uint32_t st, int w, int lane, float S, float qm) {
+    constexpr int kBlock = 16;
+    const int mi = lane & 7, mm = lane >> 3;
+    const uint32_t base = st + (uint32_t)((16 * (mi >> 1) + 2 * mm + (mi & 1)) * (TC * 2) + 16 * (w ^ mi));
+    const int64_t R = cur.R, C = cur.C;
+    const int64_t cpad = LAYOUT == QZ_SF_SWIZZLED_128x4 ? ((C + 127) & ~(int64_t)127) : C;
+    const int64_t kvT = R / kBlock;  // scale columns of the transposed matrix
+    const int64_t kvs = LAYOUT == QZ_SF_SWIZZLED_128x4 ? ((kvT + 3) & ~(int64_t)3) : kvT;
+#pragma unroll
+    for (int u = 0; u < TC / 64; ++u) {  // chunk w + 8 u: (w + 8 u) ^ mi == (w ^ mi) + 8 u
+        uint32_t v[2][8];
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int qd = 0; qd < 2; ++qd)
+                ldsm_x4_trans(base + (uint32_t)(128 * u + 64 * (TC * 2) * h + 8 * (TC * 2) * qd), v[h][4 * qd],
+                              v[h][4 * qd + 1], v[h][4 * qd + 2], v[h][4 * qd + 3]);
+        // the tile kernels' NVFP4 arithmetic (same bytes as qzq::nvfp4_block): both
+        // blocks' scales at once, element multipliers from 16 per-tile quotients
+        const uint32_t two = tile_scales_nv_words(v[0], v[1], S);
+        const uint32_t sc[2] = {two & 0xFFu, two >> 8};
+        uint32_t c[2][2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const float rcp = nvfp4_rcp_warp(qm, sc[h]);
+            c[h][0] = e2m1x8_words(v[h][0], v[h][1], v[h][2], v[h][3], rcp);
+            c[h][1] = e2m1x8_words(v[h][4], v[h][5], v[h][6], v[h][7], rcp);
+        }
+        const int64_t cg = (int64_t)cur.ct * TC + 8 * (w + 8 * u) + (lane >> 2);  // x column = transposed row
+        if (cg < cpad) {
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int64_t e0 = (int64_t)cur.rt * kTileRows + 64 * h + 16 * (lane & 3);  // the block's first x row
+                const int64_t k = e0 / kBlock;
+                if (cg < C && e0 < R) st_v2(cur.q + cg * (R >> 1) + (e0 >> 1), c[h][0], c[h][1]);
+                // scale byte (a block past the last row holds zeros and gets scale 0;
+                // padded transposed rows C <= cg < cpad get 0x00)
+                if (k < kvs) cur.sf[qzq::sf_offset(cg, k, kvT, LAYOUT)] = cg < C ? (uint8_t)sc[h] : (uint8_t)0;
+            }
+        }
     }
 }
 
 template <int FMT, int LAYOUT>
-__global__ void __launch_bounds__(kColThreads, 2) colwise_kernel(const qz_expert* __restrict__ table, int n,
-                                                                 unsigned* d_err) {
-    constexpr int kBlock = FMT == QZ_FMT_MXFP8 ? 32 : 16;
+__global__ void __launch_bounds__(kColThreads, ColGeo<FMT>::kCtas) colwise_kernel(const qz_expert* __restrict__ table,
+                                                                                 int n, unsigned* d_err) {
+    using G = ColGeo<FMT>;
     extern __shared__ __align__(16) int s_prefix[];  // [n + 1] prefix, then the stages (16-byte aligned)
     __shared__ long long s_scan[33];
     __shared__ float s_inv[16];
     if (FMT == QZ_FMT_NVFP4) fill_inv_table(s_inv);  // published by the barriers in block_prefix
-    const int total = block_prefix(n, s_prefix, s_scan, ColTiles<FMT, LAYOUT>{table, d_err}, d_err);
+    const int total = block_prefix(n, s_prefix, s_scan, ColTiles<FMT, LAYOUT, G::kTC>{table, d_err}, d_err);
     const int t = threadIdx.x;
     const uint32_t stages = (uint32_t)__cvta_generic_to_shared(s_prefix + ((n + 4) & ~3));
     const uint32_t* s_words = reinterpret_cast<const uint32_t*>(s_prefix + ((n + 4) & ~3));
@@ -145,19 +287,18 @@ __global__ void __launch_bounds__(kColThreads, 2) colwise_kernel(const qz_expert
     const int beg = (int)((int64_t)total * blockIdx.x / gridDim.x);
     const int end = (int)((int64_t)total * (blockIdx.x + 1) / gridDim.x);
     if (beg >= end) return;
-    ColRef iss = col_ref(table, s_prefix, beg, find_owner(s_prefix, n, beg));  // the walk issuing copies
-    ColRef cur = iss;                                                         // the walk quantizing
+    ColRef iss = col_ref<G::kTC>(table, s_prefix, beg, find_owner(s_prefix, n, beg));  // the walk issuing copies
+    ColRef cur = iss;                                                                 // the walk quantizing
     // prologue: the first kColStages - 1 tiles in flight
 #pragma unroll
     for (int s = 0; s < kColStages - 1; ++s) {
         if (beg + s < end) {
-            if (s > 0) col_next(iss, table, s_prefix, beg + s);
-            col_issue(iss, stages + s * kColStageBytes, t);
+            if (s > 0) col_next<G::kTC>(iss, table, s_prefix, beg + s);
+            col_issue<G::kTC, FMT == QZ_FMT_NVFP4>(iss, stages + s * G::kStageBytes, t);
         }
         cp_async_commit();
     }
     const int w = t >> 5, lane = t & 31;
-    const int ch = w & 1, rs = w >> 1;  // this warp's column half and 32-row segment of a tile
     // NVFP4: the expert's encode scale, and lanes 1..15 holding RN(S / m)
     int scale_expert = -1;
     float S = 0.0f, qm = 0.0f;
@@ -170,109 +311,42 @@ __global__ void __launch_bounds__(kColThreads, 2) colwise_kernel(const qz_expert
         {
             const int ahead = tile + kColStages - 1;
             if (ahead < end) {
-                col_next(iss, table, s_prefix, ahead);
-                col_issue(iss, stages + ((k + kColStages - 1) % kColStages) * kColStageBytes, t);
+                col_next<G::kTC>(iss, table, s_prefix, ahead);
+                col_issue<G::kTC, FMT == QZ_FMT_NVFP4>(iss, stages + ((k + kColStages - 1) % kColStages) * G::kStageBytes,
+                                                       t);
             }
             cp_async_commit();
         }
-        if (k > 0) col_next(cur, table, s_prefix, tile);
-        if (FMT == QZ_FMT_NVFP4 && cur.expert != scale_expert) {
-            scale_expert = cur.expert;
-            S = nvfp4_encode_scale(__ldg(cur.amax));
-            qm = rcp_lane_quotient(S, s_inv, lane);  // every lane: the shuffles below need all
-        }
-        const int64_t R = cur.R, C = cur.C;
-        // ---- thread (warp w, lane l) quantizes tile columns 64 ch + 2 l and + 1,
-        //      rows 32 rs .. 32 rs + 31 of each: one word per row holds both columns
-        const uint32_t* tw = s_words + cur_s * (kColStageBytes / 4) + (32 * rs) * (kTileCols / 2) + 32 * ch + lane;
-        uint32_t xa[16], xb[16];  // column pairs (row 2i low, row 2i + 1 high) of the two columns
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            const uint32_t r0 = tw[(2 * i) * (kTileCols / 2)], r1 = tw[(2 * i + 1) * (kTileCols / 2)];
-            xa[i] = __byte_perm(r0, r1, 0x5410);
-            xb[i] = __byte_perm(r0, r1, 0x7632);
-        }
-        const int64_t cg = (int64_t)cur.ct * kTileCols + 64 * ch + 2 * lane;  // x column = transposed row
-        const int64_t e0 = (int64_t)cur.rt * kTileRows + 32 * rs;             // first x row of the segment
-        const int64_t cpad = LAYOUT == QZ_SF_SWIZZLED_128x4 ? ((C + 127) & ~(int64_t)127) : C;
-        const int64_t kvT = R / kBlock;  // scale columns of the transposed matrix
-        const int64_t kvs = LAYOUT == QZ_SF_SWIZZLED_128x4 ? ((kvT + 3) & ~(int64_t)3) : kvT;
-        const int64_t k0 = e0 / kBlock;  // the segment's first scale column
-        constexpr int kSeg = 32 / kBlock;  // scale blocks per column segment: 1 / 2
-        uint32_t sc[2][kSeg];
-        if (FMT == QZ_FMT_MXFP8) {
-            uint32_t qa[8], qb[8];
-            sc[0][0] = qzq::mxfp8_block(xa, qa);
-            sc[1][0] = qzq::mxfp8_block(xb, qb);
-            if (e0 < R) {
-                const bool q32 = ((reinterpret_cast<uintptr_t>(cur.q) & 31) == 0);
-#pragma unroll
-                for (int j = 0; j < 2; ++j) {
-                    if (cg + j >= C) continue;
-                    const uint32_t* qq = j ? qb : qa;
-                    uint8_t* dst = cur.q + (cg + j) * R + e0;
-                    const uint4 lo = make_uint4(qq[0], qq[1], qq[2], qq[3]), hi = make_uint4(qq[4], qq[5], qq[6], qq[7]);
-                    if (q32) {
-                        st_v8(dst, lo, hi);
-                    } else {
-                        st_v4(dst, lo);
-                        st_v4(dst + 16, hi);
-                    }
-                }
-            }
+        if (k > 0) col_next<G::kTC>(cur, table, s_prefix, tile);
+        if constexpr (FMT == QZ_FMT_MXFP8) {
+            col_tile_mx<LAYOUT>(cur, s_words + cur_s * (G::kStageBytes / 4), w, lane);
         } else {
-            // the tile kernels' NVFP4 arithmetic (same bytes as qzq::nvfp4_block): block
-            // scales two at a time, element multipliers from 16 per-tile quotients
-            uint32_t c[2][4];
-#pragma unroll
-            for (int j = 0; j < 2; ++j) {
-                const uint32_t* xx = j ? xb : xa;
-                const uint32_t two = tile_scales_nv_words(xx, xx + 8, S);
-                sc[j][0] = two & 0xFFu;
-                sc[j][1] = two >> 8;
-#pragma unroll
-                for (int b = 0; b < 2; ++b) {
-                    const float rcp = nvfp4_rcp_warp(qm, sc[j][b]);
-                    c[j][2 * b] = e2m1x8_words(xx[8 * b], xx[8 * b + 1], xx[8 * b + 2], xx[8 * b + 3], rcp);
-                    c[j][2 * b + 1] = e2m1x8_words(xx[8 * b + 4], xx[8 * b + 5], xx[8 * b + 6], xx[8 * b + 7], rcp);
-                }
+            if (cur.expert != scale_expert) {
+                scale_expert = cur.expert;
+                S = nvfp4_encode_scale(__ldg(cur.amax));
+                qm = rcp_lane_quotient(S, s_inv, lane);  // every lane: the shuffles below need all
             }
-#pragma unroll
-            for (int j = 0; j < 2; ++j) {
-                if (cg + j >= C || e0 >= R) continue;
-                uint8_t* dst = cur.q + (cg + j) * (R >> 1) + (e0 >> 1);
-                if (e0 + 32 <= R && (reinterpret_cast<uintptr_t>(dst) & 15) == 0) {
-                    st_v4(dst, make_uint4(c[j][0], c[j][1], c[j][2], c[j][3]));
-                } else {
-                    st_v2(dst, c[j][0], c[j][1]);
-                    if (e0 + 32 <= R) st_v2(dst + 8, c[j][2], c[j][3]);
-                }
-            }
-        }
-        // scale bytes: kSeg consecutive ones per column (blocks past the last row
-        // hold zeros and get scale 0; padded transposed rows C <= cg < cpad get 0x00)
-#pragma unroll
-        for (int j = 0; j < 2; ++j) {
-            const int64_t row = cg + j;
-            if (row >= cpad) continue;
-            const bool live = row < C;
-#pragma unroll
-            for (int b = 0; b < kSeg; ++b)
-                if (k0 + b < kvs) cur.sf[qzq::sf_offset(row, k0 + b, kvT, LAYOUT)] = live ? (uint8_t)sc[j][b] : (uint8_t)0;
+            col_tile_nv<LAYOUT, G::kTC>(cur, stages + cur_s * G::kStageBytes, w, lane, S, qm);
         }
     }
     cp_async_wait<0>();  // nothing is left in flight at exit
 }
 
+template <int FMT>
+size_t colwise_smem(int n) {
+    return (size_t)((n + 4) & ~3) * sizeof(int) + (size_t)kColStages * ColGeo<FMT>::kStageBytes;
+}
+
 cudaError_t launch_colwise(const qz_expert* table, int n, int fmt, int layout, int grid, cudaStream_t s,
                            unsigned* d_err) {
-    const size_t smem = (size_t)((n + 4) & ~3) * sizeof(int) + (size_t)kColStages * kColStageBytes;
     if (fmt == QZ_FMT_MXFP8) {
+        const size_t smem = colwise_smem<QZ_FMT_MXFP8>(n);
         if (layout == QZ_SF_SWIZZLED_128x4)
             colwise_kernel<QZ_FMT_MXFP8, QZ_SF_SWIZZLED_128x4><<<grid, kColThreads, smem, s>>>(table, n, d_err);
         else
             colwise_kernel<QZ_FMT_MXFP8, QZ_SF_LINEAR><<<grid, kColThreads, smem, s>>>(table, n, d_err);
     } else {
+        const size_t smem = colwise_smem<QZ_FMT_NVFP4>(n);
         if (layout == QZ_SF_SWIZZLED_128x4)
             colwise_kernel<QZ_FMT_NVFP4, QZ_SF_SWIZZLED_128x4><<<grid, kColThreads, smem, s>>>(table, n, d_err);
         else
@@ -281,19 +355,25 @@ cudaError_t launch_colwise(const qz_expert* table, int n, int fmt, int layout, i
     return cudaGetLastError();
 }
 
-// Resident CTAs per SM (for a one-wave persistent grid).  The stages plus the
-// largest prefix table exceed 48 KB, so every instantiation is allowed more
-// dynamic shared memory on the current device first (this runs once per
-// device before its first launch).
-int colwise_blocks_per_sm(int n) {
-    const int bytes = (int)((size_t)((QZ_MAX_EXPERTS + 4) & ~3) * sizeof(int) + (size_t)kColStages * kColStageBytes);
-    cudaFuncSetAttribute(colwise_kernel<QZ_FMT_MXFP8, QZ_SF_SWIZZLED_128x4>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-    cudaFuncSetAttribute(colwise_kernel<QZ_FMT_MXFP8, QZ_SF_LINEAR>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-    cudaFuncSetAttribute(colwise_kernel<QZ_FMT_NVFP4, QZ_SF_SWIZZLED_128x4>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-    cudaFuncSetAttribute(colwise_kernel<QZ_FMT_NVFP4, QZ_SF_LINEAR>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+// Resident CTAs per SM of the format's kernel (for a one-wave persistent
+// grid).  The stages plus the largest prefix table exceed 48 KB, so both
+// layouts are allowed more dynamic shared memory on the current device first
+// (this runs once per device and format before the first launch).
+int colwise_blocks_per_sm(int n, int fmt) {
     int b = 1;
-    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, colwise_kernel<QZ_FMT_MXFP8, QZ_SF_SWIZZLED_128x4>, kColThreads,
-                                                  (size_t)((n + 4) & ~3) * sizeof(int) + (size_t)kColStages * kColStageBytes);
+    if (fmt == QZ_FMT_MXFP8) {
+        const int bytes = (int)colwise_smem<QZ_FMT_MXFP8>(QZ_MAX_EXPERTS);
+        cudaFuncSetAttribute(colwise_kernel<QZ_FMT_MXFP8, QZ_SF_SWIZZLED_128x4>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+        cudaFuncSetAttribute(colwise_kernel<QZ_FMT_MXFP8, QZ_SF_LINEAR>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, colwise_kernel<QZ_FMT_MXFP8, QZ_SF_SWIZZLED_128x4>, kColThreads,
+                                                      colwise_smem<QZ_FMT_MXFP8>(n));
+    } else {
+        const int bytes = (int)colwise_smem<QZ_FMT_NVFP4>(QZ_MAX_EXPERTS);
+        cudaFuncSetAttribute(colwise_kernel<QZ_FMT_NVFP4, QZ_SF_SWIZZLED_128x4>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+        cudaFuncSetAttribute(colwise_kernel<QZ_FMT_NVFP4, QZ_SF_LINEAR>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, colwise_kernel<QZ_FMT_NVFP4, QZ_SF_SWIZZLED_128x4>, kColThreads,
+                                                      colwise_smem<QZ_FMT_NVFP4>(n));
+    }
     return b > 0 ? b : 1;
 }
 

@@ -12,8 +12,12 @@
 // kernels: lane l of warp w owns one scale block per pass (MXFP8: 32
 // elements, NVFP4: 16) of rows w + 8 * (lane / LPR) + 64 p (MXFP8) or
 // + 32 p (NVFP4) of the tile.  The next tile's payload and scale loads are
-// issued before the current tile is decoded; the bf16 output leaves as
+// issued before the current tile is decoded (payload loads do not allocate
+// in L1, which keeps the expert table there); the bf16 output leaves as
 // 32-byte stores (16-byte ones when the rows are only 16-byte aligned).
+// NVFP4 decodes through a per-block table of its eight magnitudes (below),
+// which leaves it bound by load latency rather than by arithmetic, so it runs
+// four CTAs per SM where MXFP8 runs three.
 #include <cuda_fp16.h>
 
 #include "qz_device.cuh"
@@ -74,12 +78,6 @@ struct DqTiles {
     }
 };
 
-__device__ __forceinline__ uint32_t __hmul2_rn_bits(uint32_t a, uint32_t b) {
-    uint32_t r;
-    asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
-    return r;
-}
-
 // bf16 bits of the exact value hi + lo (hi = RN32 of it, lo the exact
 // remainder), rounded to nearest even: rounding hi again is right unless hi
 // lies exactly halfway between two bf16 numbers, where lo decides.
@@ -96,13 +94,6 @@ __device__ __forceinline__ uint32_t bf16_of_exact(float hi, float lo) {
 __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t pair) {
     uint32_t h;
     asm("{\n\t.reg .b16 c;\n\tcvt.u16.u32 c, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, c;\n\t}" : "=r"(h) : "r"(pair));
-    return h;
-}
-
-// Two e2m1 codes (bits 0-7, low nibble first) as an f16x2 pair, exactly.
-__device__ __forceinline__ uint32_t e2m1x2_to_f16x2(uint32_t pair) {
-    uint32_t h;
-    asm("{\n\t.reg .b8 c;\n\tcvt.u8.u32 c, %1;\n\tcvt.rn.f16x2.e2m1x2 %0, c;\n\t}" : "=r"(h) : "r"(pair));
     return h;
 }
 
@@ -190,9 +181,9 @@ __device__ __forceinline__ void dq_load(const DqRef& r, DqTile<FMT>& t) {
             t.qw[p][0] = a.x; t.qw[p][1] = a.y; t.qw[p][2] = a.z; t.qw[p][3] = a.w;
             t.qw[p][4] = b.x; t.qw[p][5] = b.y; t.qw[p][6] = b.z; t.qw[p][7] = b.w;
         } else {
-            const uint2 a = __ldg(reinterpret_cast<const uint2*>(src));
-            t.qw[p][0] = a.x;
-            t.qw[p][1] = a.y;
+            asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0,%1}, [%2];"
+                         : "=r"(t.qw[p][0]), "=r"(t.qw[p][1])
+                         : "l"(src));
         }
         t.sc[p] = __ldg(r.sf + dq_sf_index(LAYOUT, r.row0 + p * G::kRpp, r.k, r.kv));
     }
@@ -211,45 +202,92 @@ __device__ __forceinline__ uint4 dq_mx8(uint32_t w0, uint32_t w1, float s) {
     return o;
 }
 
-// NVFP4: 8 elements (one payload word) of one block: sv2 = value(s) as f16x2
-// (both halves), g the decode scale.  code value * value(s) is exact in f16
-// (at most 6 significant bits, at most 2688); RN32 of its product with g is
-// rounded to bf16, and the rare element whose RN32 product lies exactly
-// halfway between two bf16 numbers is rounded from the exact product.
-__device__ __forceinline__ uint4 dq_nv8(uint32_t word, uint32_t sv2, float g) {
-    uint4 o;
-    uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
-    float hv[8], pv[8];
+// NVFP4 decode table of one block: the bf16 bits of value(m) * value(s) * g
+// for the eight e2m1 magnitudes m = 0, 0.5, 1, 1.5, 2, 3, 4, 6 (codes 0-7),
+// as byte tables -- lo[k] / hi[k] the low / high byte of entry k, entries
+// 0-3 in the first word of each pair, 4-7 in the second -- so that a
+// prmt with the magnitude codes as selectors looks up four elements at once.
+// value(m) * value(s) is exact in binary32 (at most 6 significant bits); its
+// RN32 product with g is rounded to bf16, and an entry whose RN32 product
+// lies exactly halfway between two bf16 numbers is rounded from the exact
+// product (RN32 product + the remainder the fma gives exactly).
+struct NvTable {
+    uint32_t lo0, lo1, hi0, hi1;
+};
+
+__device__ __forceinline__ NvTable nv_table(float sv, float g) {
+    float a[8];
+    a[0] = 0.0f;
+    a[1] = 0.5f * sv;
+    a[2] = sv;
+    a[3] = 1.5f * sv;
+    a[4] = 2.0f * sv;
+    a[5] = 3.0f * sv;
+    a[6] = 4.0f * sv;
+    a[7] = 6.0f * sv;
+    float h[8];
+    uint32_t p[4];
     // the low 16 bits of every RN32 product, xor 0x8000: a zero half marks a
-    // bf16 midpoint; their running minimum (per 16-bit half) finds any
+    // bf16 midpoint; their minimum (per 16-bit half) finds any
     uint32_t mid = 0xFFFFFFFFu;
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-        const uint32_t ph = __hmul2_rn_bits(e2m1x2_to_f16x2((word >> (8 * j)) & 0xFFu), sv2);
-        const float2 p = __half22float2(*reinterpret_cast<const __half2*>(&ph));
-        const float2 h = f16x2_times(ph, g);
-        pv[2 * j] = p.x;
-        pv[2 * j + 1] = p.y;
-        hv[2 * j] = h.x;
-        hv[2 * j + 1] = h.y;
-        ow[j] = bf16x2_rn(h.x, h.y);
-        mid = __vminu2(mid, __byte_perm(__float_as_uint(h.x), __float_as_uint(h.y), 0x5410) ^ 0x80008000u);
+        asm("{\n\t.reg .b64 x, y;\n\tmov.b64 x, {%2, %3};\n\tmov.b64 y, {%4, %4};\n\t"
+            "mul.rn.f32x2 x, x, y;\n\tmov.b64 {%0, %1}, x;\n\t}"
+            : "=f"(h[2 * j]), "=f"(h[2 * j + 1])
+            : "f"(a[2 * j]), "f"(a[2 * j + 1]), "f"(g));
+        p[j] = bf16x2_rn(h[2 * j], h[2 * j + 1]);
+        mid = __vminu2(mid, __byte_perm(__float_as_uint(h[2 * j]), __float_as_uint(h[2 * j + 1]), 0x5410) ^ 0x80008000u);
     }
-    const bool tie = (mid & 0xFFFFu) == 0u || (mid >> 16) == 0u;
-    if (tie) {
+    if ((mid & 0xFFFFu) == 0u || (mid >> 16) == 0u) {
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-            const float l0 = __fmaf_rn(pv[2 * j], g, -hv[2 * j]);
-            const float l1 = __fmaf_rn(pv[2 * j + 1], g, -hv[2 * j + 1]);
-            ow[j] = bf16_of_exact(hv[2 * j], l0) | (bf16_of_exact(hv[2 * j + 1], l1) << 16);
+            const float l0 = __fmaf_rn(a[2 * j], g, -h[2 * j]);
+            const float l1 = __fmaf_rn(a[2 * j + 1], g, -h[2 * j + 1]);
+            p[j] = bf16_of_exact(h[2 * j], l0) | (bf16_of_exact(h[2 * j + 1], l1) << 16);
         }
     }
+    NvTable t;
+    t.lo0 = __byte_perm(p[0], p[1], 0x6420);
+    t.hi0 = __byte_perm(p[0], p[1], 0x7531);
+    t.lo1 = __byte_perm(p[2], p[3], 0x6420);
+    t.hi1 = __byte_perm(p[2], p[3], 0x7531);
+    return t;
+}
+
+// NVFP4: the 8 elements of one payload word (element i in nibble i) through
+// the block's table.  Four codes at a time: their magnitudes (the low three
+// bits of each nibble) select the low and the high bytes; the high byte takes
+// the sign bit of its code; the two byte words interleave into bf16 pairs.
+// bf16(-v) is bf16(v) with the sign bit set (round to nearest is symmetric),
+// so a negative code decodes to its magnitude's entry with the sign set.
+__device__ __forceinline__ uint32_t nv_hi_signed(uint32_t hi, uint32_t codes4) {
+    // prmt in sign-replicate mode: a nibble with bit 3 set (a negative code)
+    // gives the replicated top bit of 0x7F, 0x00; a positive one gives 0x7F.
+    // Adding one per byte (no carries) leaves the top bit set exactly for the
+    // positive codes.
+    uint32_t t;
+    asm("prmt.b32 %0, %1, %1, %2;" : "=r"(t) : "r"(0x7F7F7F7Fu), "r"(codes4));
+    t += 0x01010101u;
+    return hi | (~t & 0x80808080u);
+}
+
+__device__ __forceinline__ uint4 dq_nv8(uint32_t word, const NvTable& T) {
+    const uint32_t m = word & 0x77777777u;
+    const uint32_t lo_a = __byte_perm(T.lo0, T.lo1, m), lo_b = __byte_perm(T.lo0, T.lo1, m >> 16);
+    const uint32_t hi_a = nv_hi_signed(__byte_perm(T.hi0, T.hi1, m), word);
+    const uint32_t hi_b = nv_hi_signed(__byte_perm(T.hi0, T.hi1, m >> 16), word >> 16);
+    uint4 o;
+    o.x = __byte_perm(lo_a, hi_a, 0x5140);
+    o.y = __byte_perm(lo_a, hi_a, 0x7362);
+    o.z = __byte_perm(lo_b, hi_b, 0x5140);
+    o.w = __byte_perm(lo_b, hi_b, 0x7362);
     return o;
 }
 
 template <int FMT, int LAYOUT>
-__global__ void __launch_bounds__(kDqThreads, 3) dequant_kernel(const qz_dq_expert* __restrict__ table, int n,
-                                                                bool per_row, unsigned* d_err) {
+__global__ void __launch_bounds__(kDqThreads, FMT == QZ_FMT_NVFP4 ? 4 : 3)
+    dequant_kernel(const qz_dq_expert* __restrict__ table, int n, bool per_row, unsigned* d_err) {
     using G = DqGeo<FMT>;
     extern __shared__ int s_prefix[];
     __shared__ long long s_scan[33];
@@ -288,11 +326,9 @@ __global__ void __launch_bounds__(kDqThreads, 3) dequant_kernel(const qz_dq_expe
                 }
             } else {
                 if (per_row) g = __fdiv_rn(__ldg(cur.amax + (int64_t)p * G::kRpp), 2688.0f);
-                const __half sh = __float2half_rn(e4m3_value(t.sc[p]));  // exact: e4m3 values are f16 values
-                const __half2 sv = __halves2half2(sh, sh);
-                const uint32_t sv2 = *reinterpret_cast<const uint32_t*>(&sv);
-                const uint4 a = dq_nv8(t.qw[p][0], sv2, g);
-                const uint4 b = dq_nv8(t.qw[p][1], sv2, g);
+                const NvTable T = nv_table(e4m3_value(t.sc[p]), g);
+                const uint4 a = dq_nv8(t.qw[p][0], T);
+                const uint4 b = dq_nv8(t.qw[p][1], T);
                 if (cur.y32) {
                     st_v8(dst, a, b);
                 } else {
@@ -324,10 +360,14 @@ cudaError_t launch_dequant(const qz_dq_expert* table, int n, int fmt, bool per_r
     return cudaGetLastError();
 }
 
-int dequant_blocks_per_sm(int n) {
+int dequant_blocks_per_sm(int n, int fmt) {
     int b = 1;
-    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, dequant_kernel<QZ_FMT_NVFP4, QZ_SF_SWIZZLED_128x4>, kDqThreads,
-                                                  (size_t)(n + 1) * sizeof(int));
+    if (fmt == QZ_FMT_NVFP4)
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, dequant_kernel<QZ_FMT_NVFP4, QZ_SF_SWIZZLED_128x4>, kDqThreads,
+                                                      (size_t)(n + 1) * sizeof(int));
+    else
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, dequant_kernel<QZ_FMT_MXFP8, QZ_SF_SWIZZLED_128x4>, kDqThreads,
+                                                      (size_t)(n + 1) * sizeof(int));
     return b > 0 ? b : 1;
 }
 
