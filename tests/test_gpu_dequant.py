@@ -158,12 +158,11 @@ def test_qwen3_30b_gate_up_layer_sampled(fmt):
             assert_bytes_equal(got[r:r + 1, :cols], ref, f"expert {i} row {r}")
 
 
-@pytest.mark.parametrize("per_row", [False, True])
-def test_every_code_and_scale_including_midpoint_products(per_row):
-    """Every e2m1 code under every finite E4M3 scale code, for amax values
-    among which some binary32 products RN(value(q) * value(s) * g) land exactly
-    on a bf16 midpoint (those elements need the exact product to round): the
-    decoder must match the oracle there too."""
+def _every_code_and_scale(amaxes, per_row):
+    """Decode every e2m1 code under every finite E4M3 scale code for each amax
+    A in `amaxes` (per row: A spread over [A/2, 2A] down the rows) and compare
+    with the oracle's decoder; returns how many binary32 products landed on a
+    bf16 midpoint."""
     scales = np.arange(127, dtype=np.uint8)
     R = len(scales)
     codes = np.arange(16, dtype=np.uint8)
@@ -171,15 +170,37 @@ def test_every_code_and_scale_including_midpoint_products(per_row):
     e2m1 = np.array([0, 0.5, 1, 1.5, 2, 3, 4, 6, -0.0, -0.5, -1, -1.5, -2, -3, -4, -6], dtype=np.float32)
     e4m3 = torch.arange(256, dtype=torch.uint8).view(torch.float8_e4m3fn).float().numpy()
     midpoints = 0
-    for A in (3.0, 1.0 / 3.0, 5.0e4, 27.50284194946289, 36.21154022216797, 76.34375):
+    for A in amaxes:
         amax = np.full(R if per_row else 1, A, dtype=np.float32)
         if per_row:
             amax = (amax * np.linspace(0.5, 2.0, R)).astype(np.float32)
-        g = (amax / np.float32(2688.0)).astype(np.float32).reshape(-1, 1)
-        prod = ((e2m1[None, :] * e4m3[scales][:, None]).astype(np.float32) * g).astype(np.float32)
+        with np.errstate(over="ignore", under="ignore"):
+            g = (amax / np.float32(2688.0)).astype(np.float32).reshape(-1, 1)
+            prod = ((e2m1[None, :] * e4m3[scales][:, None]).astype(np.float32) * g).astype(np.float32)
         midpoints += int(np.count_nonzero((prod.view(np.uint32) & 0xFFFF) == 0x8000))
         out = run_dequant([(q, scales.copy(), amax, R, 16)], qz.FMT_NVFP4, qz.SF_LINEAR, per_row)[0]
         ref = oracle.dequantize_nvfp4(q, scales.copy(), amax, per_row, oracle.LINEAR)
         assert_bytes_equal(host_bits(out)[:, :16], ref, f"amax {A}")
+    return midpoints
+
+
+@pytest.mark.parametrize("per_row", [False, True])
+def test_every_code_and_scale_at_extreme_amax(per_row):
+    """Amax values whose decode scale is subnormal or whose products approach
+    the binary32 overflow: the decoder builds these tables entry by entry (its
+    two-product shortcut needs every entry normal and finite) and must still
+    round each exact product once."""
+    amaxes = (1e-36, 3e-37, 2e-38, 5e-39, 3e-40, 1e37, 8e37, 1.5e38)
+    _every_code_and_scale(amaxes if per_row else amaxes + (3.3e38,), per_row)  # per row: up to 2A, finite
+
+
+@pytest.mark.parametrize("per_row", [False, True])
+def test_every_code_and_scale_including_midpoint_products(per_row):
+    """Every e2m1 code under every finite E4M3 scale code, for amax values
+    among which some binary32 products RN(value(q) * value(s) * g) land exactly
+    on a bf16 midpoint (those elements need the exact product to round): the
+    decoder must match the oracle there too."""
+    midpoints = _every_code_and_scale((3.0, 1.0 / 3.0, 5.0e4, 27.50284194946289, 36.21154022216797, 76.34375),
+                                      per_row)
     assert midpoints > 0, "no product fell on a bf16 midpoint: the exact-rounding path went untested"
 
