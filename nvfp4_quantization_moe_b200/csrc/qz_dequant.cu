@@ -12,8 +12,7 @@
 // kernels: lane l of warp w owns one scale block per pass (MXFP8: 32
 // elements, NVFP4: 16) of rows w + 8 * (lane / LPR) + 64 p (MXFP8) or
 // + 32 p (NVFP4) of the tile.  The next tile's payload and scale loads are
-// issued before the current tile is decoded (payload loads do not allocate
-// in L1, which keeps the expert table there); the bf16 output leaves as
+// issued before the current tile is decoded; the bf16 output leaves as
 // 32-byte stores (16-byte ones when the rows are only 16-byte aligned).
 // NVFP4 decodes through a per-block table of its eight magnitudes (below),
 // which leaves it bound by load latency rather than by arithmetic, so it runs
@@ -181,9 +180,9 @@ __device__ __forceinline__ void dq_load(const DqRef& r, DqTile<FMT>& t) {
             t.qw[p][0] = a.x; t.qw[p][1] = a.y; t.qw[p][2] = a.z; t.qw[p][3] = a.w;
             t.qw[p][4] = b.x; t.qw[p][5] = b.y; t.qw[p][6] = b.z; t.qw[p][7] = b.w;
         } else {
-            asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0,%1}, [%2];"
-                         : "=r"(t.qw[p][0]), "=r"(t.qw[p][1])
-                         : "l"(src));
+            const uint2 a = __ldg(reinterpret_cast<const uint2*>(src));
+            t.qw[p][0] = a.x;
+            t.qw[p][1] = a.y;
         }
         t.sc[p] = __ldg(r.sf + dq_sf_index(LAYOUT, r.row0 + p * G::kRpp, r.k, r.kv));
     }
