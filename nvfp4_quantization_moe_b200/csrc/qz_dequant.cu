@@ -14,6 +14,9 @@
 // + 32 p (NVFP4) of the tile.  The next tile's payload and scale loads are
 // issued before the current tile is decoded; the bf16 output leaves as
 // 32-byte stores (16-byte ones when the rows are only 16-byte aligned).
+// NVFP4 decodes through a per-block table of the bf16 results of its eight
+// e2m1 magnitudes (below), four codes per byte permute, and runs four CTAs
+// per SM where MXFP8 runs three.
 // NVFP4 decodes through a per-block table of its eight magnitudes (below),
 // which leaves it bound by load latency rather than by arithmetic, so it runs
 // four CTAs per SM where MXFP8 runs three.
@@ -214,7 +217,7 @@ struct NvTable {
     uint32_t lo0, lo1, hi0, hi1;
 };
 
-__device__ __forceinline__ NvTable nv_table(float sv, float g) {
+__device__ __forceinline__ NvTable nv_table_exact(float sv, float g) {
     float a[8];
     a[0] = 0.0f;
     a[1] = 0.5f * sv;
@@ -251,6 +254,34 @@ __device__ __forceinline__ NvTable nv_table(float sv, float g) {
     t.hi0 = __byte_perm(p[0], p[1], 0x7531);
     t.lo1 = __byte_perm(p[2], p[3], 0x6420);
     t.hi1 = __byte_perm(p[2], p[3], 0x7531);
+    return t;
+}
+
+// The same table from two products.  The magnitudes are 2^k and 1.5 * 2^k, and
+// scaling by a power of two commutes with both roundings while every value
+// stays normal and finite: with b1 = bf16(value(s) * g) and b3 =
+// bf16(1.5 value(s) * g) (each from its RN32 product, midpoints rounded from
+// the exact one as above), entry 2^k (k = -1, 0, 1, 2) is b1 with k added to
+// its exponent field and entry 1.5 * 2^k (k = 0, 1, 2) is b3 with k added.
+// The exponent field e1 of b1 in [3, 251] keeps every entry and every RN32
+// product normal and finite (b3's field is e1 or e1 + 1); outside it the
+// entries are built one by one.
+__device__ __forceinline__ NvTable nv_table(float sv, float g) {
+    const float a3 = 1.5f * sv;  // exact
+    const float p1 = __fmul_rn(sv, g), p3 = __fmul_rn(a3, g);
+    uint32_t b = bf16x2_rn(p1, p3);  // b1 low, b3 high
+    if (((__float_as_uint(p1) & 0xFFFFu) == 0x8000u) || ((__float_as_uint(p3) & 0xFFFFu) == 0x8000u))
+        b = bf16_of_exact(p1, __fmaf_rn(sv, g, -p1)) | (bf16_of_exact(p3, __fmaf_rn(a3, g, -p3)) << 16);
+    const uint32_t e1 = (b >> 7) & 0xFFu;
+    if (e1 - 3u > 248u) return nv_table_exact(sv, g);
+    const uint32_t p0 = ((b & 0xFFFFu) - 0x80u) << 16;  // magnitudes 0 (zero) and 0.5
+    const uint32_t p2 = b + 0x00800080u;                 // magnitudes 2 and 3 (b: 1 and 1.5)
+    const uint32_t p4 = b + 0x01000100u;                 // magnitudes 4 and 6
+    NvTable t;
+    t.lo0 = __byte_perm(p0, b, 0x6420);
+    t.hi0 = __byte_perm(p0, b, 0x7531);
+    t.lo1 = __byte_perm(p2, p4, 0x6420);
+    t.hi1 = __byte_perm(p2, p4, 0x7531);
     return t;
 }
 
