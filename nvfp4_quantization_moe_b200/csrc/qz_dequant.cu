@@ -171,9 +171,14 @@ __device__ __forceinline__ bool dq_live(const DqRef& r, int p) {
     return r.col_ok && r.row0 + p * DqGeo<FMT>::kRpp < r.rows;
 }
 
+// The scale bytes of a lane's passes are affine in the pass: a tile's rows
+// lie in one 128-row group and the lane's first row is in its first
+// G::kRpp rows, so in the swizzled layout each pass moves kRpp / 32 4-byte
+// slices; in the linear one it moves kRpp rows.
 template <int FMT, int LAYOUT>
 __device__ __forceinline__ void dq_load(const DqRef& r, DqTile<FMT>& t) {
     using G = DqGeo<FMT>;
+    const uint8_t* sfp = r.sf + dq_sf_index(LAYOUT, r.row0, r.k, r.kv);
 #pragma unroll
     for (int p = 0; p < G::kPasses; ++p) {
         if (!dq_live<FMT>(r, p)) continue;
@@ -187,7 +192,7 @@ __device__ __forceinline__ void dq_load(const DqRef& r, DqTile<FMT>& t) {
             t.qw[p][0] = a.x;
             t.qw[p][1] = a.y;
         }
-        t.sc[p] = __ldg(r.sf + dq_sf_index(LAYOUT, r.row0 + p * G::kRpp, r.k, r.kv));
+        t.sc[p] = __ldg(sfp + (LAYOUT == QZ_SF_SWIZZLED_128x4 ? (G::kRpp / 32) * 4 * p : p * G::kRpp * r.kv));
     }
 }
 
@@ -202,6 +207,15 @@ __device__ __forceinline__ uint4 dq_mx8(uint32_t w0, uint32_t w1, float s) {
     v = f16x2_times(e4m3x2_to_f16x2(w1 & 0xFFFFu), s); o.z = bf16x2_rn(v.x, v.y);
     v = f16x2_times(e4m3x2_to_f16x2(w1 >> 16), s);     o.w = bf16x2_rn(v.x, v.y);
     return o;
+}
+
+// Value of a non-negative e4m3 code below 0x7F without a branch: the
+// subnormal m * 2^-9 is (1 + m/8) * 2^-6 - 2^-6 (both terms and the
+// difference exact).
+__device__ __forceinline__ float e4m3_value_nb(uint32_t s) {
+    const uint32_t ef = s >> 3, m = s & 7u;
+    const float v = __uint_as_float(((ef ? ef + 120u : 121u) << 23) | (m << 20));
+    return ef ? v : __fsub_rn(v, 0x1p-6f);
 }
 
 // NVFP4 decode table of one block: the bf16 bits of value(m) * value(s) * g
@@ -356,7 +370,7 @@ __global__ void __launch_bounds__(kDqThreads, FMT == QZ_FMT_NVFP4 ? 4 : 3)
                 }
             } else {
                 if (per_row) g = __fdiv_rn(__ldg(cur.amax + (int64_t)p * G::kRpp), 2688.0f);
-                const NvTable T = nv_table(e4m3_value(t.sc[p]), g);
+                const NvTable T = nv_table(e4m3_value_nb(t.sc[p]), g);
                 const uint4 a = dq_nv8(t.qw[p][0], T);
                 const uint4 b = dq_nv8(t.qw[p][1], T);
                 if (cur.y32) {
