@@ -10,7 +10,10 @@
 //
 // One persistent launch walks all experts' 128 x 128 tiles, each CTA a
 // contiguous run of them (so its expert -- the entry and the NVFP4 scale --
-// changes rarely).  Each CTA keeps
+// changes rarely), down the rows of x first: consecutive tiles of a CTA fill
+// consecutive pieces of the same 128 transposed output rows, so the output
+// leaves L2 in whole lines of few DRAM pages instead of 64- or 128-byte
+// pieces of 128 different rows per tile.  Each CTA keeps
 // three tiles in flight: asynchronous 16-byte copies (cp.async, zero-filled
 // past the matrix) bring a tile row-major into one of three shared-memory
 // stages while the tile before it is quantized, so the loads never wait on
@@ -84,15 +87,15 @@ struct ColTiles {
 };
 
 // A walk over consecutive tiles of the call: the tile's expert (its entry)
-// and its row / column tile.  Moving to the next tile reloads the entry only
-// when the expert changes.
+// and its row / column tile, row tiles fastest.  Moving to the next tile
+// reloads the entry only when the expert changes.
 struct ColRef {
     const uint16_t* x;
     int64_t R, C, ld;
     uint8_t* q;
     uint8_t* sf;
     const float* amax;
-    int rt, ct, nct;
+    int rt, ct, nrt;
     int expert;
 };
 
@@ -102,9 +105,9 @@ __device__ __forceinline__ ColRef col_ref(const qz_expert* table, const int* s_p
     const qz_expert E = load_entry(table, e);
     const int local = tile - s_prefix[e];
     ColRef r;
-    r.nct = (int)col_tiles_c<TC>(E.cols);
-    r.rt = local / r.nct;
-    r.ct = local - r.rt * r.nct;
+    r.nrt = (int)((E.rows + kTileRows - 1) / kTileRows);
+    r.ct = local / r.nrt;
+    r.rt = local - r.ct * r.nrt;
     r.x = static_cast<const uint16_t*>(E.x);
     r.R = E.rows;
     r.C = E.cols;
@@ -120,9 +123,9 @@ __device__ __forceinline__ ColRef col_ref(const qz_expert* table, const int* s_p
 template <int TC>
 __device__ __forceinline__ void col_next(ColRef& r, const qz_expert* table, const int* s_prefix, int tile) {
     if (tile < s_prefix[r.expert + 1]) {
-        if (++r.ct == r.nct) {
-            r.ct = 0;
-            ++r.rt;
+        if (++r.rt == r.nrt) {
+            r.rt = 0;
+            ++r.ct;
         }
     } else {
         r = col_ref<TC>(table, s_prefix, tile, r.expert + 1);
