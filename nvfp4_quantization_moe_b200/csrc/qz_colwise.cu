@@ -237,6 +237,28 @@ __device__ __forceinline__ void col_tile_nv(const ColRef& cur, uint32_t st, int 
     const int64_t cpad = LAYOUT == QZ_SF_SWIZZLED_128x4 ? ((C + 127) & ~(int64_t)127) : C;
     const int64_t kvT = R / kBlock;  // scale columns of the transposed matrix
     const int64_t kvs = LAYOUT == QZ_SF_SWIZZLED_128x4 ? ((kvT + 3) & ~(int64_t)3) : kvT;
+    // This thread's four blocks: transposed rows cg0 + 64 u (u = 0, 1), blocks
+    // starting at x row e00 + 64 h (h = 0, 1).  Their payload bytes and scale
+    // bytes are affine in (u, h): payload + 64 u rows of the transposed payload
+    // + 32 h bytes; scale + 8 u + 512 h (swizzled: cg0 % 128 < 64, so + 64 rows
+    // stays in the 128-row group and moves two 4-row slices; + 4 scale columns
+    // is the next 512-byte tile) or + 64 u kvT + 4 h (linear).
+    const int64_t cg0 = (int64_t)cur.ct * TC + 8 * w + (lane >> 2);
+    const int64_t e00 = (int64_t)cur.rt * kTileRows + 16 * (lane & 3);
+    const int64_t k00 = e00 / kBlock;
+    const int64_t qrow = R >> 1;  // payload bytes per transposed row
+    uint8_t* const q0 = cur.q + cg0 * qrow + (e00 >> 1);
+    int64_t s0, su, sh;
+    if (LAYOUT == QZ_SF_SWIZZLED_128x4) {
+        const int r = (int)(cg0 & 127);
+        s0 = (((cg0 >> 7) * ((kvT + 3) >> 2) + (k00 >> 2)) << 9) + ((((r & 31) << 2) + (r >> 5)) << 2) + (k00 & 3);
+        su = 8;
+        sh = 512;
+    } else {
+        s0 = cg0 * kvT + k00;
+        su = 64 * kvT;
+        sh = 4;
+    }
 #pragma unroll
     for (int u = 0; u < TC / 64; ++u) {  // chunk w + 8 u: (w + 8 u) ^ mi == (w ^ mi) + 8 u
         uint32_t v[2][8];
@@ -257,16 +279,15 @@ __device__ __forceinline__ void col_tile_nv(const ColRef& cur, uint32_t st, int 
             c[h][0] = e2m1x8_words(v[h][0], v[h][1], v[h][2], v[h][3], rcp);
             c[h][1] = e2m1x8_words(v[h][4], v[h][5], v[h][6], v[h][7], rcp);
         }
-        const int64_t cg = (int64_t)cur.ct * TC + 8 * (w + 8 * u) + (lane >> 2);  // x column = transposed row
+        const int64_t cg = cg0 + 64 * u;  // x column = transposed row
         if (cg < cpad) {
+            const bool live = cg < C;
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
-                const int64_t e0 = (int64_t)cur.rt * kTileRows + 64 * h + 16 * (lane & 3);  // the block's first x row
-                const int64_t k = e0 / kBlock;
-                if (cg < C && e0 < R) st_v2(cur.q + cg * (R >> 1) + (e0 >> 1), c[h][0], c[h][1]);
+                if (live && e00 + 64 * h < R) st_v2(q0 + u * (qrow << 6) + 32 * h, c[h][0], c[h][1]);
                 // scale byte (a block past the last row holds zeros and gets scale 0;
                 // padded transposed rows C <= cg < cpad get 0x00)
-                if (k < kvs) cur.sf[qzq::sf_offset(cg, k, kvT, LAYOUT)] = cg < C ? (uint8_t)sc[h] : (uint8_t)0;
+                if (k00 + 4 * h < kvs) cur.sf[s0 + u * su + h * sh] = live ? (uint8_t)sc[h] : (uint8_t)0;
             }
         }
     }
