@@ -8,16 +8,17 @@
 // factors those of a [cols, rows] matrix in the linear or swizzled 128x4
 // layout, padding written as 0x00 by the kernel.
 //
-// One persistent launch walks all experts' 128 x 128 tiles, each CTA a
-// contiguous run of them (so its expert -- the entry and the NVFP4 scale --
-// changes rarely), down the rows of x first: consecutive tiles of a CTA fill
-// consecutive pieces of the same 128 transposed output rows, so the output
-// leaves L2 in whole lines of few DRAM pages instead of 64- or 128-byte
-// pieces of 128 different rows per tile.  Each CTA keeps
-// three tiles in flight: asynchronous 16-byte copies (cp.async, zero-filled
-// past the matrix) bring a tile row-major into one of three shared-memory
-// stages while the tile before it is quantized, so the loads never wait on
-// the arithmetic and one CTA barrier per tile suffices.
+// One persistent launch walks all experts' 128 x 128 tiles, each CTA (MXFP8)
+// or each group of 8 warps (NVFP4) a contiguous run of them (so its expert --
+// the entry and the NVFP4 scale -- changes rarely), down the rows of x
+// first: consecutive tiles fill consecutive pieces of the same 128
+// transposed output rows, so the output leaves L2 in whole lines of few DRAM
+// pages instead of 64- or 128-byte pieces of 128 different rows per tile.
+// Asynchronous 16-byte copies (cp.async, zero-filled past the matrix) bring
+// a tile row-major into a shared-memory stage while the tile before it is
+// quantized: MXFP8 runs two CTAs per SM with three stages each and one CTA
+// barrier per tile; NVFP4 runs one CTA per SM of three independent 8-warp
+// groups (24 warps) with two stages each and a named barrier per group.
 //   MXFP8: a thread reads one 32-bit word per row -- two neighbouring
 //   columns -- for 32 rows, pairs consecutive rows of each column into bf16x2
 //   words and quantizes the two 32-element column segments with the
@@ -356,6 +357,69 @@ __global__ void __launch_bounds__(kColThreads, ColGeo<FMT>::kCtas) colwise_kerne
     cp_async_wait<0>();  // nothing is left in flight at exit
 }
 
+// NVFP4: one CTA per SM of three independent groups of 8 warps (24 warps per
+// SM) that share the prefix table.  Each group walks its own contiguous run
+// of tiles through two 32 KB stages of its own (one tile copied while the
+// previous one is quantized) and synchronizes on its own named barrier, so
+// the groups never wait for one another; a thread quantizes as in the
+// two-CTA form, one 64-column half at a time.
+constexpr int kNvGroups = 3;
+constexpr int kNvGroupStages = 2;
+constexpr int kNvStageBytes = kTileRows * 128 * 2;
+
+__device__ __forceinline__ void group_barrier(int g) {
+    asm volatile("bar.sync %0, %1;" ::"r"(1 + g), "r"(kColThreads) : "memory");
+}
+
+template <int LAYOUT>
+__global__ void __launch_bounds__(kColThreads * kNvGroups, 1) colwise_nv_kernel(const qz_expert* __restrict__ table,
+                                                                               int n, unsigned* d_err) {
+    constexpr int kTC = 128;
+    extern __shared__ __align__(16) int s_prefix[];  // [n + 1] prefix, then the groups' stages
+    __shared__ long long s_scan[33];
+    __shared__ float s_inv[16];
+    fill_inv_table(s_inv);  // published by the barriers in block_prefix
+    const int total = block_prefix(n, s_prefix, s_scan, ColTiles<QZ_FMT_NVFP4, LAYOUT, kTC>{table, d_err}, d_err);
+    const int g = threadIdx.x / kColThreads, t = threadIdx.x % kColThreads;
+    const uint32_t stages = (uint32_t)__cvta_generic_to_shared(s_prefix + ((n + 4) & ~3)) +
+                            (uint32_t)(g * kNvGroupStages * kNvStageBytes);
+    // this group's tiles: a contiguous run [beg, end) of the call's tiles
+    const int64_t groups = (int64_t)gridDim.x * kNvGroups, gi = (int64_t)blockIdx.x * kNvGroups + g;
+    const int beg = (int)((int64_t)total * gi / groups);
+    const int end = (int)((int64_t)total * (gi + 1) / groups);
+    if (beg >= end) return;  // only group barriers follow
+    ColRef iss = col_ref<kTC>(table, s_prefix, beg, find_owner(s_prefix, n, beg));  // the walk issuing copies
+    ColRef cur = iss;                                                             // the walk quantizing
+    col_issue<kTC, true>(iss, stages, t);
+    cp_async_commit();
+    const int w = t >> 5, lane = t & 31;
+    int scale_expert = -1;
+    float S = 0.0f, qm = 0.0f;
+    for (int k = 0;; ++k) {
+        const int tile = beg + k;
+        if (tile >= end) break;
+        cp_async_wait<0>();  // this thread's copies of tile k have landed
+        group_barrier(g);    // ... and the group's; tile k - 1's stage is free again
+        if (tile + 1 < end) {
+            col_next<kTC>(iss, table, s_prefix, tile + 1);
+            col_issue<kTC, true>(iss, stages + ((k + 1) & 1) * kNvStageBytes, t);
+        }
+        cp_async_commit();
+        if (k > 0) col_next<kTC>(cur, table, s_prefix, tile);
+        if (cur.expert != scale_expert) {
+            scale_expert = cur.expert;
+            S = nvfp4_encode_scale(__ldg(cur.amax));
+            qm = rcp_lane_quotient(S, s_inv, lane);  // every lane: the shuffles below need all
+        }
+        col_tile_nv<LAYOUT, kTC>(cur, stages + (k & 1) * kNvStageBytes, w, lane, S, qm);
+    }
+    cp_async_wait<0>();  // nothing is left in flight at exit
+}
+
+size_t colwise_nv_smem(int n) {
+    return (size_t)((n + 4) & ~3) * sizeof(int) + (size_t)kNvGroups * kNvGroupStages * kNvStageBytes;
+}
+
 template <int FMT>
 size_t colwise_smem(int n) {
     return (size_t)((n + 4) & ~3) * sizeof(int) + (size_t)kColStages * ColGeo<FMT>::kStageBytes;
@@ -370,11 +434,11 @@ cudaError_t launch_colwise(const qz_expert* table, int n, int fmt, int layout, i
         else
             colwise_kernel<QZ_FMT_MXFP8, QZ_SF_LINEAR><<<grid, kColThreads, smem, s>>>(table, n, d_err);
     } else {
-        const size_t smem = colwise_smem<QZ_FMT_NVFP4>(n);
+        const size_t smem = colwise_nv_smem(n);
         if (layout == QZ_SF_SWIZZLED_128x4)
-            colwise_kernel<QZ_FMT_NVFP4, QZ_SF_SWIZZLED_128x4><<<grid, kColThreads, smem, s>>>(table, n, d_err);
+            colwise_nv_kernel<QZ_SF_SWIZZLED_128x4><<<grid, kColThreads * kNvGroups, smem, s>>>(table, n, d_err);
         else
-            colwise_kernel<QZ_FMT_NVFP4, QZ_SF_LINEAR><<<grid, kColThreads, smem, s>>>(table, n, d_err);
+            colwise_nv_kernel<QZ_SF_LINEAR><<<grid, kColThreads * kNvGroups, smem, s>>>(table, n, d_err);
     }
     return cudaGetLastError();
 }
@@ -392,11 +456,11 @@ int colwise_blocks_per_sm(int n, int fmt) {
         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, colwise_kernel<QZ_FMT_MXFP8, QZ_SF_SWIZZLED_128x4>, kColThreads,
                                                       colwise_smem<QZ_FMT_MXFP8>(n));
     } else {
-        const int bytes = (int)colwise_smem<QZ_FMT_NVFP4>(QZ_MAX_EXPERTS);
-        cudaFuncSetAttribute(colwise_kernel<QZ_FMT_NVFP4, QZ_SF_SWIZZLED_128x4>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-        cudaFuncSetAttribute(colwise_kernel<QZ_FMT_NVFP4, QZ_SF_LINEAR>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, colwise_kernel<QZ_FMT_NVFP4, QZ_SF_SWIZZLED_128x4>, kColThreads,
-                                                      colwise_smem<QZ_FMT_NVFP4>(n));
+        const int bytes = (int)colwise_nv_smem(QZ_MAX_EXPERTS);
+        cudaFuncSetAttribute(colwise_nv_kernel<QZ_SF_SWIZZLED_128x4>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+        cudaFuncSetAttribute(colwise_nv_kernel<QZ_SF_LINEAR>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, colwise_nv_kernel<QZ_SF_SWIZZLED_128x4>, kColThreads * kNvGroups,
+                                                      colwise_nv_smem(n));
     }
     return b > 0 ? b : 1;
 }
